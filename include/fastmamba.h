@@ -1,0 +1,265 @@
+/*
+ * fastmamba.h -- C ABI of the quantised Mamba2 mixer library (libfastmamba.so).
+ *
+ * The method is FastMamba's quantisation scheme for a Mamba2 mixer layer
+ * (arXiv 2505.18975; cited below by web page and section):
+ *   - Hadamard-rotated 8-bit linear layers, Y = (XH)(H^T W^T) with H
+ *     orthonormal after 1/sqrt(n) (pith.science review, "What carries the
+ *     argument"; scales from the max of the rotated tensors: Referee Report,
+ *     major comment 1, on Algorithm 1 and Fig. 6);
+ *   - power-of-two (2^p, shift-only) fixed point for the causal conv1d and
+ *     the SSM recurrence (same section; original abstract);
+ *   - an 8-segment first-order linear approximation of 2^v, with
+ *     e^x = 2^(x log2 e) and SoftPlus(x) = x + SoftPlus(-x) (same section;
+ *     Referee minor comment 5 on Eq. (5): SoftPlus(x) ~ e^x for x <= 0).
+ * The Mamba2 block structure (in_proj -> conv1d + SiLU -> selective scan ->
+ * gate + RMSNorm -> out_proj; Figure 2 caption) is that of Mamba2, the
+ * paper's reference [2].
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the
+ *     library never allocates, frees or retains them.  Tensors are dense,
+ *     row-major (last index fastest).  Pointers must be 16-byte aligned.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the
+ *     legacy default stream).  Host-side validation happens before any
+ *     launch; on error nothing is launched and a status is returned.
+ *   - Kernels that wait (the GEMM's pipeline barriers) give up after a
+ *     bounded number of polls and set a device error word instead of
+ *     hanging; fm_sync_status() reports it.
+ *   - Shapes: K of every linear layer and d_model, d_inner are multiples of
+ *     256 (the Hadamard block); headdim = 64, d_state = 128, ngroups = 1,
+ *     d_conv = 4 (the Mamba2-130M / 2.7B configuration); conv_ch and
+ *     d_inner are multiples of 16.
+ *   - Fixed-point conventions (rshr, satb, Q.16, exponent table) are
+ *     described next to fm_exp_layout below.
+ *   - No exceptions cross the ABI; no global mutable state except a
+ *     per-device device error word and the per-process entry-point cache.
+ */
+#ifndef FASTMAMBA_H
+#define FASTMAMBA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum fm_status {
+    FM_OK = 0,
+    FM_ERR_INVALID_ARG = 1, /* null pointer, bad enum value */
+    FM_ERR_SHAPE = 2,       /* unsupported or inconsistent sizes */
+    FM_ERR_ALIGNMENT = 3,   /* pointer not 16-byte aligned */
+    FM_ERR_WORKSPACE = 4,   /* workspace missing or too small */
+    FM_ERR_NONFINITE = 5,   /* reserved: non-finite statistic seen on device */
+    FM_ERR_TIMEOUT = 6,     /* a bounded device-side wait gave up */
+    FM_ERR_CUDA = 7,        /* a CUDA runtime/driver call failed */
+    FM_ERR_UNSUPPORTED = 8  /* no sm_100 device, or driver entry point missing */
+} fm_status;
+
+enum { FM_DYNAMIC = 0, FM_STATIC = 1 };
+
+typedef void *fm_stream; /* cudaStream_t */
+
+/* Human-readable name of a status code (static string). */
+const char *fm_status_string(fm_status s);
+/* Detail of the last failed call on this host thread (static, thread-local). */
+const char *fm_last_error(void);
+/* Synchronises `stream`, then reads and clears the device error word of the
+ * current device: FM_OK, FM_ERR_TIMEOUT (a bounded wait gave up) or
+ * FM_ERR_CUDA (the synchronisation itself failed). */
+fm_status fm_sync_status(fm_stream stream);
+/* Library ABI version (major * 100 + minor). */
+int fm_version(void);
+
+/* ------------------------------------------------------------------ */
+/* shapes and the exponent table                                       */
+/* ------------------------------------------------------------------ */
+typedef struct fm_shape {
+    int d_model, d_inner, headdim, d_state, ngroups, d_conv;
+} fm_shape;
+
+/* Derived sizes: nheads = d_inner / headdim; conv_ch = d_inner + 2 d_state;
+ * n_in = 2 d_inner + 2 d_state + nheads (in_proj columns z | x | B | C | dt). */
+
+/* Power-of-two exponent table of one layer: one device int32 array.  A value
+ * e means "the integer code times 2^e".  Layout (offsets in int32 elements):
+ *   [0, cc)            e_u  conv input, per conv channel
+ *   [cc, 2cc)          e_w  conv weights, per conv channel
+ *   [2cc, 3cc)         e_o  conv output, per conv channel (x: its head's e_x; B: e_B; C: e_C)
+ *   [3cc, 3cc+nh)      e_x  per head
+ *   3cc+nh             e_B
+ *   3cc+nh+1           e_C
+ *   [3cc+nh+2, +nh)    e_h  state, per head
+ *   [3cc+2nh+2, +nh)   e_y  scan output, per head
+ *   [3cc+3nh+2, +nh)   e_D  skip parameter D, per head
+ *   3cc+4nh+2          e_g  gate output
+ * Size: 3cc + 4nh + 3. */
+typedef struct fm_exp_layout {
+    int e_u, e_w, e_o, e_x, e_B, e_C, e_h, e_y, e_D, e_g, size;
+} fm_exp_layout;
+fm_exp_layout fm_exp_table_layout(const fm_shape *shape);
+
+/* ------------------------------------------------------------------ */
+/* a0 + a1 / a10: (pre-RMSNorm) + Hadamard rotation + int8 quantisation */
+/* ------------------------------------------------------------------ */
+/* x [M, K] fp32 -> q [M, K] int8 codes and s_x [M] fp32 scales, so that
+ * dequant = q * s_x[row] approximates (RMSNorm(x) * prenorm_w) H_bd.
+ *   prenorm_w  [K] or NULL: apply RMSNorm (eps 1e-5, fixed summation order)
+ *              and this weight before rotating (stack layers).
+ *   rotate     1: block-diagonal Sylvester Hadamard (block 256) / 16; 0: identity.
+ *   mode       FM_DYNAMIC: per-row amax; FM_STATIC: *static_amax (device
+ *              scalar) for every row, values beyond it clip to +-127.
+ *   amax_row   [M] or NULL: receives each row's max |rotated value|.
+ * K % 256 == 0, K <= 8192. */
+fm_status fm_hadamard_quant(const float *x, int64_t M, int64_t K, const float *prenorm_w,
+                            int rotate, int mode, const float *static_amax, int8_t *q,
+                            float *s_x, float *amax_row, fm_stream stream);
+
+/* Offline: W [N, K] fp32 -> Wq [N, K] int8 and s_w [N] fp32 with
+ * W' = W H_bd (fp64), s_w = max|W'[n,:]| / 127, Wq = rint(W' / s_w). */
+fm_status fm_prepare_linear(const float *W, int64_t N, int64_t K, int rotate, int8_t *Wq,
+                            float *s_w, fm_stream stream);
+
+/* ------------------------------------------------------------------ */
+/* a2 + a3 / a11: W8A8 GEMM on the tensor cores + dequantisation        */
+/* ------------------------------------------------------------------ */
+/* Y[m,n] = fl(fl(float(acc[m,n]) * s_x[m]) * s_w[n]) (+ residual[m,n]),
+ * acc = sum_k A[m,k] Wq[n,k] (exact int32).
+ *   A [M, K] int8, Wq [N, K] int8 (both K-major), residual [M, N] or NULL
+ *   (may alias Y), acc_out [M, N] int32 or NULL (raw accumulators).
+ * K % 128 == 0. */
+fm_status fm_w8a8_gemm(const int8_t *A, const float *s_x, int64_t M, const int8_t *Wq,
+                       const float *s_w, int64_t N, int64_t K, const float *residual, float *Y,
+                       int32_t *acc_out, fm_stream stream);
+
+/* in_proj: the same GEMM (N = n_in, K = d_model) with the split epilogue:
+ *   z   [M, d_inner] fp32   (columns [0, di))
+ *   xbc [M, conv_ch] int8   (columns [di, di+cc)): satb(rint(y * 2^-e_u[c]), 8)
+ *   dt  [M, nheads] fp32    (columns [di+cc, n_in))
+ * e_u is the exponent table's first region (device). */
+fm_status fm_in_proj(const int8_t *A, const float *s_x, int64_t M, const int8_t *Wq,
+                     const float *s_w, const fm_shape *shape, const int32_t *exps, float *z,
+                     int8_t *xbc, float *dt, fm_stream stream);
+
+/* ------------------------------------------------------------------ */
+/* a4: power-of-two causal depthwise conv1d (kernel 4) + SiLU           */
+/* ------------------------------------------------------------------ */
+/* u [B, T, cc] int8 codes at e_u -> out [B, T, cc] int8 codes at e_o:
+ *   acc = bq[c] + sum_{k=0..3} wq[c,k] u[t-3+k, c]   (tap 3 = current token)
+ *   x16 = satb(rshr(acc, -(e_w+e_u+16)), 32); s = SiLU_pwl(x16)
+ *   out = satb(rshr(s, e_o + 16), 8)
+ *   wq [cc, 4] int8, bq [cc] int32 (at e_w + e_u), exps = exponent table.
+ *   conv_state [B, 3, cc] int8 or NULL: history (oldest first) read before
+ *   the first token and replaced by the last three inputs. */
+fm_status fm_conv1d_pot(const int8_t *u, int B, int T, const fm_shape *shape, const int8_t *wq,
+                        const int32_t *bq, const int32_t *exps, int8_t *conv_state, int8_t *out,
+                        fm_stream stream);
+
+/* ------------------------------------------------------------------ */
+/* a5 - a8: selective scan in power-of-two fixed point                  */
+/* ------------------------------------------------------------------ */
+/* xbc [B, T, cc] int8 conv output (x | B | C), dt_raw [B, T, nh] fp32.
+ * Per token and head (Q.16): dt_q = SoftPlus_pwl(to_q16(dt_raw + dt_bias)),
+ * dA_q = 2^(-rshr(dt_q * A_q, 12)).  Per (b, h, p, n), t in order:
+ *   u = satb(rshr(dt_q x[p], e_h - e_B - e_x + 16), 24)
+ *   h = clamp(rshr(dA_q h, 16) + u B[n], +-(2^30 - 1))
+ *   y[p] = satb(rshr(sum_n C[n] h, e_y - e_C - e_h) + rshr(D_q x[p], e_y - e_D - e_x), 32)
+ *   dt_bias [nh] fp32, A_q [nh] int32 (exp(A_log) log2(e) 2^12), D_q [nh] int32.
+ *   state [B, nh, hd, ds] int32 or NULL (zeros): initial state in, final out.
+ *   y [B, T, d_inner] int32 at e_y. */
+fm_status fm_ssm_scan_pot(const int8_t *xbc, const float *dt_raw, int B, int T,
+                          const fm_shape *shape, const float *dt_bias, const int32_t *A_q,
+                          const int32_t *D_q, const int32_t *exps, int32_t *state, int32_t *y,
+                          fm_stream stream);
+
+/* ------------------------------------------------------------------ */
+/* a9 + a10: gate, gated RMSNorm, rotation, int8 quantisation           */
+/* ------------------------------------------------------------------ */
+/* y [M, di] int32 (at e_y per head), z [M, di] fp32 -> q [M, di] int8, s_x [M]:
+ *   g = y SiLU_pwl(to_q16(z)); g_q = satb(rshr(g, e_g - e_y + 16), 16)
+ *   rstd = 1/sqrt(sum g_q^2 2^(2 e_g) / di + 1e-5) (exact integer sum)
+ *   o = g_q 2^e_g rstd norm_w, then as fm_hadamard_quant. */
+fm_status fm_gate_norm_quant(const int32_t *y, const float *z, int64_t M, const fm_shape *shape,
+                             const int32_t *exps, const float *norm_w, int rotate, int mode,
+                             const float *static_amax, int8_t *q, float *s_x, float *amax_row,
+                             fm_stream stream);
+
+/* ------------------------------------------------------------------ */
+/* the nonlinear approximation unit, element-wise (verification)        */
+/* ------------------------------------------------------------------ */
+/* The shared 8-segment first-order approximation of 2^v and the functions
+ * built on it (pith.science review of FastMamba, "What carries the
+ * argument"; Referee minor comment 5, Eq. (5)), evaluated element-wise over
+ * a device int64 array -- the same device functions the conv, scan and gate
+ * kernels use.  kind: 0 = 2^v (Q.16 in, v <= 0), 1 = e^x, 2 = SoftPlus,
+ * 3 = SiLU (in clamped to int32), 4 = to_q16 of the fp32 bit pattern held
+ * in the low 32 bits.  in, out: [n] int64. */
+fm_status fm_eval_pwl(int kind, const int64_t *in, int64_t n, int64_t *out, fm_stream stream);
+
+/* ------------------------------------------------------------------ */
+/* layers                                                               */
+/* ------------------------------------------------------------------ */
+/* A prepared layer: device pointers to quantised parameters (caller-owned). */
+typedef struct fm_layer {
+    fm_shape shape;
+    int rotate;                 /* 1: Hadamard rotation in both linear layers */
+    int mode;                   /* FM_DYNAMIC or FM_STATIC activation scales */
+    const int8_t *w_in_q;       /* [n_in, d_model] */
+    const float *w_in_s;        /* [n_in] */
+    const int8_t *w_out_q;      /* [d_model, d_inner] */
+    const float *w_out_s;       /* [d_model] */
+    const float *prenorm_w;     /* [d_model] or NULL: stack layer pre-RMSNorm */
+    const int8_t *conv_wq;      /* [conv_ch, 4] */
+    const int32_t *conv_bq;     /* [conv_ch] */
+    const float *dt_bias;       /* [nheads] */
+    const int32_t *A_q;         /* [nheads] */
+    const int32_t *D_q;         /* [nheads] */
+    const float *norm_w;        /* [d_inner] gated-norm weight */
+    const int32_t *exps;        /* exponent table (fm_exp_table_layout) */
+    const float *static_amax;   /* [2]: in_proj input, out_proj input (FM_STATIC) */
+} fm_layer;
+
+/* Workspace bytes fm_mixer_prefill / fm_decode_step need for B*T tokens. */
+size_t fm_workspace_bytes(const fm_shape *shape, int B, int T);
+
+/* One mixer layer on x [B, T, d_model] fp32 -> out [B, T, d_model] fp32.
+ *   residual 1: out = x + mixer(x) (stack layer; out may alias x).
+ *   conv_state [B, 3, conv_ch] int8 / ssm_state [B, nh, hd, ds] int32, or
+ *   NULL: carried state in/out (prefill in chunks is bit-identical to one pass).
+ *   ws: device workspace of at least fm_workspace_bytes(shape, B, T). */
+fm_status fm_mixer_prefill(const fm_layer *L, const float *x, int B, int T, int residual,
+                           int8_t *conv_state, int32_t *ssm_state, float *out, void *ws,
+                           size_t ws_bytes, fm_stream stream);
+
+/* Single-token decode step for B sequences: x [B, d_model] -> out [B, d_model],
+ * updating conv_state and ssm_state (both required). */
+fm_status fm_decode_step(const fm_layer *L, const float *x, int B, int residual,
+                         int8_t *conv_state, int32_t *ssm_state, float *out, void *ws,
+                         size_t ws_bytes, fm_stream stream);
+
+/* Offline, per layer: quantise conv taps (e_w, wq) and the SSM parameters
+ * (A_q, D_q, e_D) from fp32 device tensors: conv_w [cc, 4], a_log [nh], D [nh].
+ * Writes the e_w and e_D regions of `exps`. */
+fm_status fm_prepare_mixer_params(const fm_shape *shape, const float *conv_w, const float *a_log,
+                                  const float *D, int8_t *conv_wq, int32_t *A_q, int32_t *D_q,
+                                  int32_t *exps, fm_stream stream);
+
+/* Calibration workspace bytes for B*T calibration tokens. */
+size_t fm_calib_workspace_bytes(const fm_shape *shape, int B, int T);
+
+/* Stage-by-stage calibration of one prepared layer on xcal [B, T, d_model]:
+ * fills the remaining regions of exps (e_u, e_o, e_x, e_B, e_C, e_h, e_y,
+ * e_g), conv_bq (from conv_b [cc] fp32 at e_w + e_u) and static_amax[2],
+ * and writes the layer's output on xcal to out (next layer's calibration
+ * input).  L->exps / L->conv_bq / L->static_amax are written through the
+ * non-const pointers given here (they must be the same arrays). */
+fm_status fm_calibrate_layer(const fm_layer *L, const float *conv_b, int32_t *exps,
+                             int32_t *conv_bq, float *static_amax, const float *xcal, int B,
+                             int T, int residual, float *out, void *ws, size_t ws_bytes,
+                             fm_stream stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FASTMAMBA_H */

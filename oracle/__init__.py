@@ -426,8 +426,10 @@ def calibrate_layer(L: Layer, xcal, residual=False):
     y = ssm_scan_pot(xo, dt3, L.dt_bias, L.A_q, L.D_q, L.e_x, L.e_B, L.e_C, L.e_h, L.e_y, L.e_D,
                      hd, ds)
     # gate exponent (int16 g), then the out_proj input amax
-    _, _, gs = gate_norm_quant(y.reshape(M, di), z, hd, L.e_y, 0, L.norm_w, L.rotate, DYNAMIC,
-                               0.0, want_gstat=True)
+    # (the statistic does not depend on e_g; the pass uses its lower bound so
+    # that every gate shift is a right shift)
+    _, _, gs = gate_norm_quant(y.reshape(M, di), z, hd, L.e_y, int(L.e_y.max()) - 16, L.norm_w,
+                               L.rotate, DYNAMIC, 0.0, want_gstat=True)
     L.e_g = int(max(max(pot_exponent(float(gs[h]), 32767.0) + int(L.e_y[h]) - 16
                         for h in range(nh)), int(L.e_y.max()) - 16))
     q2, sx2, am2 = gate_norm_quant(y.reshape(M, di), z, hd, L.e_y, L.e_g, L.norm_w, L.rotate,

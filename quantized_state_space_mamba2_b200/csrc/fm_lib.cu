@@ -1,0 +1,851 @@
+// fm_lib.cu -- libfastmamba.so: the C ABI (include/fastmamba.h), host-side
+// validation, TMA descriptors, the mixer composition and the calibration.
+//
+// Every step of the hot path runs in the kernels included below; this file
+// only checks arguments, carves the caller's workspace and launches.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <type_traits>
+
+#include "../../include/fastmamba.h"
+
+#include "fm_common.cuh"
+#include "k_conv.cuh"
+#include "k_gemm.cuh"
+#include "k_rows.cuh"
+#include "k_scan.cuh"
+
+using namespace fm;
+
+// ------------------------------------------------------------------ errors
+static thread_local char tl_msg[512] = "";
+
+static fm_status fail(fm_status s, const char *fmt, ...) __attribute__((format(printf, 2, 3)));
+static fm_status fail(fm_status s, const char *fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(tl_msg, sizeof(tl_msg), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+#define FM_CHECK_CUDA(expr)                                                          \
+  do {                                                                               \
+    cudaError_t e_ = (expr);                                                         \
+    if (e_ != cudaSuccess)                                                           \
+      return fail(FM_ERR_CUDA, "%s: %s", #expr, cudaGetErrorString(e_));             \
+  } while (0)
+
+#define FM_TRY(expr)                   \
+  do {                                 \
+    fm_status s_ = (expr);             \
+    if (s_ != FM_OK) return s_;        \
+  } while (0)
+
+static fm_status launched(const char *what) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(FM_ERR_CUDA, "launch of %s: %s", what, cudaGetErrorString(e));
+  return FM_OK;
+}
+
+extern "C" const char *fm_status_string(fm_status s) {
+  switch (s) {
+    case FM_OK: return "FM_OK";
+    case FM_ERR_INVALID_ARG: return "FM_ERR_INVALID_ARG";
+    case FM_ERR_SHAPE: return "FM_ERR_SHAPE";
+    case FM_ERR_ALIGNMENT: return "FM_ERR_ALIGNMENT";
+    case FM_ERR_WORKSPACE: return "FM_ERR_WORKSPACE";
+    case FM_ERR_NONFINITE: return "FM_ERR_NONFINITE";
+    case FM_ERR_TIMEOUT: return "FM_ERR_TIMEOUT";
+    case FM_ERR_CUDA: return "FM_ERR_CUDA";
+    case FM_ERR_UNSUPPORTED: return "FM_ERR_UNSUPPORTED";
+  }
+  return "FM_ERR_UNKNOWN";
+}
+
+extern "C" const char *fm_last_error(void) { return tl_msg; }
+extern "C" int fm_version(void) { return 100; }
+
+extern "C" fm_status fm_sync_status(fm_stream stream) {
+  FM_CHECK_CUDA(cudaStreamSynchronize((cudaStream_t)stream));
+  unsigned int word = 0, zero = 0;
+  FM_CHECK_CUDA(cudaMemcpyFromSymbol(&word, g_error_word, sizeof(word)));
+  if (word) {
+    FM_CHECK_CUDA(cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)));
+    if (word & kErrTimeout) return fail(FM_ERR_TIMEOUT, "a bounded device wait gave up");
+  }
+  return FM_OK;
+}
+
+// ------------------------------------------------------------------ checks
+static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+#define NEED(p)                                                                   \
+  do {                                                                            \
+    if (!(p)) return fail(FM_ERR_INVALID_ARG, "%s: %s is null", __func__, #p);    \
+    if (!aligned16(p))                                                            \
+      return fail(FM_ERR_ALIGNMENT, "%s: %s is not 16-byte aligned", __func__, #p); \
+  } while (0)
+#define OPT(p)                                                                    \
+  do {                                                                            \
+    if ((p) && !aligned16(p))                                                     \
+      return fail(FM_ERR_ALIGNMENT, "%s: %s is not 16-byte aligned", __func__, #p); \
+  } while (0)
+
+struct Dims {
+  int dm, di, hd, ds, nh, cc, n_in;
+};
+
+static fm_status check_shape(const fm_shape *s, Dims *d, const char *fn) {
+  if (!s) return fail(FM_ERR_INVALID_ARG, "%s: shape is null", fn);
+  if (s->headdim != 64 || s->d_state != 128 || s->ngroups != 1 || s->d_conv != 4)
+    return fail(FM_ERR_SHAPE, "%s: need headdim 64, d_state 128, ngroups 1, d_conv 4", fn);
+  if (s->d_model <= 0 || s->d_model % 256 || s->d_model > 256 * kMaxBlocks || s->d_inner <= 0 ||
+      s->d_inner % 256 || s->d_inner > 256 * kMaxBlocks)
+    return fail(FM_ERR_SHAPE, "%s: d_model and d_inner must be positive multiples of 256, <= %d",
+                fn, 256 * kMaxBlocks);
+  d->dm = s->d_model;
+  d->di = s->d_inner;
+  d->hd = s->headdim;
+  d->ds = s->d_state;
+  d->nh = s->d_inner / s->headdim;
+  d->cc = s->d_inner + 2 * s->d_state;
+  d->n_in = 2 * s->d_inner + 2 * s->d_state + d->nh;
+  return FM_OK;
+}
+
+extern "C" fm_exp_layout fm_exp_table_layout(const fm_shape *shape) {
+  fm_exp_layout L;
+  std::memset(&L, 0, sizeof(L));
+  if (!shape || shape->headdim <= 0) return L;
+  const int nh = shape->d_inner / shape->headdim;
+  const int cc = shape->d_inner + 2 * shape->d_state;
+  L.e_u = 0;
+  L.e_w = cc;
+  L.e_o = 2 * cc;
+  L.e_x = 3 * cc;
+  L.e_B = 3 * cc + nh;
+  L.e_C = 3 * cc + nh + 1;
+  L.e_h = 3 * cc + nh + 2;
+  L.e_y = 3 * cc + 2 * nh + 2;
+  L.e_D = 3 * cc + 3 * nh + 2;
+  L.e_g = 3 * cc + 4 * nh + 2;
+  L.size = 3 * cc + 4 * nh + 3;
+  return L;
+}
+
+// ------------------------------------------------------------------ TMA descriptors
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// int8 K-major [rows, K] -> tiles of box_rows x 128 bytes, 128-byte swizzle;
+// rows beyond the tensor read as zero.
+static fm_status make_tmap(CUtensorMap *tm, const int8_t *ptr, long long rows, long long K,
+                           int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(FM_ERR_UNSUPPORTED, "cuTensorMapEncodeTiled entry point unavailable");
+  cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)K};
+  cuuint32_t box[2] = {(cuuint32_t)kGemmBK, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t *>(ptr), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(FM_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return FM_OK;
+}
+
+// ------------------------------------------------------------------ launches
+constexpr int kBN = 128;
+constexpr int kStages = 6;
+
+static fm_status launch_gemm(const int8_t *A, long long M, const int8_t *W, long long N,
+                             long long K, const GemmEpilogue &ep, cudaStream_t s) {
+  if (K % kGemmBK) return fail(FM_ERR_SHAPE, "gemm: K=%lld is not a multiple of 128", K);
+  if ((N + kBN - 1) / kBN > 2147483647LL || (M + kGemmBM - 1) / kGemmBM > 65535)
+    return fail(FM_ERR_SHAPE, "gemm: M=%lld or N=%lld too large", M, N);
+  CUtensorMap ta, tb;
+  FM_TRY(make_tmap(&ta, A, M, K, kGemmBM));
+  FM_TRY(make_tmap(&tb, W, N, K, kBN));
+  constexpr int smem = gemm_smem_bytes(kBN, kStages);
+  auto kern = k_gemm_i8_tc<kBN, kStages>;
+  FM_CHECK_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+  dim3 grid((unsigned)((N + kBN - 1) / kBN), (unsigned)((M + kGemmBM - 1) / kGemmBM));
+  kern<<<grid, kGemmThreads, smem, s>>>(ta, tb, (int)(K / kGemmBK), ep);
+  return launched("k_gemm_i8_tc");
+}
+
+static fm_status launch_hadamard_quant(const float *x, long long M, int K, const float *prenorm_w,
+                                       int rotate, int mode, const float *static_amax, int8_t *q,
+                                       float *s_x, float *amax_row, cudaStream_t s) {
+  if (M <= 0) return FM_OK;
+  k_hadamard_quant<<<(unsigned)M, 32 * (K / 256), 0, s>>>(x, K, prenorm_w, rotate, mode,
+                                                           static_amax, q, s_x, amax_row);
+  return launched("k_hadamard_quant");
+}
+
+static fm_status launch_conv(const int8_t *u, int B, int T, int cc, const int8_t *wq,
+                             const int32_t *bq, const int32_t *exps, int8_t *conv_state,
+                             int8_t *out, unsigned int *amax, cudaStream_t s) {
+  if ((long long)B * T == 0) return FM_OK;
+  const int groups = (cc / kConvCPT + kConvThreads - 1) / kConvThreads;
+  // token chunk: aim at >= ~4 CTAs per SM; one chunk when the sequence is short
+  int tch = 64;
+  const long long want = 4LL * 148;
+  while (tch > 8 && (long long)groups * ((T + tch - 1) / tch) * B < want) tch >>= 1;
+  if (T <= tch) tch = T;
+  const int chunks = (T + tch - 1) / tch;
+  if (chunks > 65535 || B > 65535) return fail(FM_ERR_SHAPE, "conv: T or B too large");
+  const int single = chunks == 1;
+  k_conv1d_pot<<<dim3(groups, chunks, B), kConvThreads, 0, s>>>(u, T, cc, tch, wq, bq, exps,
+                                                                 conv_state, single, out, amax);
+  FM_TRY(launched("k_conv1d_pot"));
+  if (conv_state && !single) {
+    const long long n = 3LL * B * cc;
+    k_conv_state_update<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(u, B, T, cc, conv_state);
+    FM_TRY(launched("k_conv_state_update"));
+  }
+  return FM_OK;
+}
+
+static ScanArgs scan_args(const Dims &d, const int8_t *xbc, const float *dt_raw, int T,
+                          const float *dt_bias, const int32_t *A_q, const int32_t *D_q,
+                          const int32_t *exps, const fm_exp_layout &X, int32_t *state, int32_t *y,
+                          unsigned long long *stat) {
+  ScanArgs a;
+  a.xbc = xbc;
+  a.dt_raw = dt_raw;
+  a.T = T;
+  a.nh = d.nh;
+  a.hd = d.hd;
+  a.cc = d.cc;
+  a.di = d.di;
+  a.dt_bias = dt_bias;
+  a.A_q = A_q;
+  a.D_q = D_q;
+  a.e_x = exps + X.e_x;
+  a.e_B = exps + X.e_B;
+  a.e_C = exps + X.e_C;
+  a.e_h = exps + X.e_h;
+  a.e_y = exps + X.e_y;
+  a.e_D = exps + X.e_D;
+  a.state = state;
+  a.y = y;
+  a.stat = stat;
+  return a;
+}
+
+template <int MODE>
+static fm_status launch_scan(const ScanArgs &a, int B, cudaStream_t s) {
+  if ((long long)B * a.T == 0) return FM_OK;
+  if (B > 65535) return fail(FM_ERR_SHAPE, "scan: B too large");
+  dim3 grid(a.hd / kScanPC, a.nh, B);
+  k_ssm_scan_pot<MODE><<<grid, kScanThreads, 0, s>>>(a);
+  return launched("k_ssm_scan_pot");
+}
+
+// ------------------------------------------------------------------ entry points
+extern "C" fm_status fm_hadamard_quant(const float *x, int64_t M, int64_t K, const float *prenorm_w,
+                                       int rotate, int mode, const float *static_amax, int8_t *q,
+                                       float *s_x, float *amax_row, fm_stream stream) {
+  if (M < 0) return fail(FM_ERR_SHAPE, "fm_hadamard_quant: M < 0");
+  if (K <= 0 || K % 256 || K > 256 * kMaxBlocks)
+    return fail(FM_ERR_SHAPE, "fm_hadamard_quant: K=%lld must be a multiple of 256 <= %d",
+                (long long)K, 256 * kMaxBlocks);
+  if (M > 2147483647LL) return fail(FM_ERR_SHAPE, "fm_hadamard_quant: M too large");
+  if (mode != FM_DYNAMIC && mode != FM_STATIC)
+    return fail(FM_ERR_INVALID_ARG, "fm_hadamard_quant: bad mode %d", mode);
+  if (M == 0) return FM_OK;
+  NEED(x);
+  NEED(q);
+  NEED(s_x);
+  OPT(prenorm_w);
+  OPT(amax_row);
+  if (mode == FM_STATIC && !static_amax)
+    return fail(FM_ERR_INVALID_ARG, "fm_hadamard_quant: static mode needs static_amax");
+  return launch_hadamard_quant(x, M, (int)K, prenorm_w, rotate ? 1 : 0, mode, static_amax, q, s_x,
+                               amax_row, (cudaStream_t)stream);
+}
+
+extern "C" fm_status fm_prepare_linear(const float *W, int64_t N, int64_t K, int rotate,
+                                       int8_t *Wq, float *s_w, fm_stream stream) {
+  if (N < 0 || N > 2147483647LL) return fail(FM_ERR_SHAPE, "fm_prepare_linear: bad N");
+  if (K <= 0 || K % 256 || K > 256 * kMaxBlocks)
+    return fail(FM_ERR_SHAPE, "fm_prepare_linear: K=%lld must be a multiple of 256", (long long)K);
+  if (N == 0) return FM_OK;
+  NEED(W);
+  NEED(Wq);
+  NEED(s_w);
+  k_prepare_linear<<<(unsigned)N, 32 * (int)(K / 256), 0, (cudaStream_t)stream>>>(
+      W, (int)K, rotate ? 1 : 0, Wq, s_w);
+  return launched("k_prepare_linear");
+}
+
+static GemmEpilogue plain_epilogue(long long M, long long N, const float *s_x, const float *s_w,
+                                   const float *residual, float *Y, int32_t *acc_out) {
+  GemmEpilogue ep;
+  std::memset(&ep, 0, sizeof(ep));
+  ep.mode = 0;
+  ep.M = M;
+  ep.N = N;
+  ep.s_x = s_x;
+  ep.s_w = s_w;
+  ep.residual = residual;
+  ep.Y = Y;
+  ep.acc_out = acc_out;
+  return ep;
+}
+
+extern "C" fm_status fm_w8a8_gemm(const int8_t *A, const float *s_x, int64_t M, const int8_t *Wq,
+                                  const float *s_w, int64_t N, int64_t K, const float *residual,
+                                  float *Y, int32_t *acc_out, fm_stream stream) {
+  if (M < 0 || N < 0 || K <= 0 || K % 128)
+    return fail(FM_ERR_SHAPE, "fm_w8a8_gemm: need M, N >= 0 and K a positive multiple of 128");
+  if (M == 0 || N == 0) return FM_OK;
+  NEED(A);
+  NEED(s_x);
+  NEED(Wq);
+  NEED(s_w);
+  NEED(Y);
+  OPT(residual);
+  OPT(acc_out);
+  return launch_gemm(A, M, Wq, N, K, plain_epilogue(M, N, s_x, s_w, residual, Y, acc_out),
+                     (cudaStream_t)stream);
+}
+
+static fm_status in_proj_impl(const int8_t *A, const float *s_x, long long M, const int8_t *Wq,
+                              const float *s_w, const Dims &d, const int32_t *e_u, float *z,
+                              int8_t *xbc, float *dt, cudaStream_t s) {
+  GemmEpilogue ep;
+  std::memset(&ep, 0, sizeof(ep));
+  ep.mode = 1;
+  ep.M = M;
+  ep.N = d.n_in;
+  ep.s_x = s_x;
+  ep.s_w = s_w;
+  ep.di = d.di;
+  ep.cc = d.cc;
+  ep.nh = d.nh;
+  ep.e_u = e_u;
+  ep.z = z;
+  ep.xbc = xbc;
+  ep.dt = dt;
+  return launch_gemm(A, M, Wq, d.n_in, d.dm, ep, s);
+}
+
+extern "C" fm_status fm_in_proj(const int8_t *A, const float *s_x, int64_t M, const int8_t *Wq,
+                                const float *s_w, const fm_shape *shape, const int32_t *exps,
+                                float *z, int8_t *xbc, float *dt, fm_stream stream) {
+  Dims d;
+  FM_TRY(check_shape(shape, &d, __func__));
+  if (M < 0) return fail(FM_ERR_SHAPE, "fm_in_proj: M < 0");
+  if (M == 0) return FM_OK;
+  NEED(A);
+  NEED(s_x);
+  NEED(Wq);
+  NEED(s_w);
+  NEED(exps);
+  NEED(z);
+  NEED(xbc);
+  NEED(dt);
+  return in_proj_impl(A, s_x, M, Wq, s_w, d, exps, z, xbc, dt, (cudaStream_t)stream);
+}
+
+extern "C" fm_status fm_conv1d_pot(const int8_t *u, int B, int T, const fm_shape *shape,
+                                   const int8_t *wq, const int32_t *bq, const int32_t *exps,
+                                   int8_t *conv_state, int8_t *out, fm_stream stream) {
+  Dims d;
+  FM_TRY(check_shape(shape, &d, __func__));
+  if (B < 0 || T < 0) return fail(FM_ERR_SHAPE, "fm_conv1d_pot: B, T must be >= 0");
+  if ((long long)B * T == 0) return FM_OK;
+  NEED(u);
+  NEED(wq);
+  NEED(bq);
+  NEED(exps);
+  NEED(out);
+  OPT(conv_state);
+  return launch_conv(u, B, T, d.cc, wq, bq, exps, conv_state, out, nullptr, (cudaStream_t)stream);
+}
+
+extern "C" fm_status fm_ssm_scan_pot(const int8_t *xbc, const float *dt_raw, int B, int T,
+                                     const fm_shape *shape, const float *dt_bias,
+                                     const int32_t *A_q, const int32_t *D_q, const int32_t *exps,
+                                     int32_t *state, int32_t *y, fm_stream stream) {
+  Dims d;
+  FM_TRY(check_shape(shape, &d, __func__));
+  if (B < 0 || T < 0) return fail(FM_ERR_SHAPE, "fm_ssm_scan_pot: B, T must be >= 0");
+  if ((long long)B * T == 0) return FM_OK;
+  NEED(xbc);
+  NEED(dt_raw);
+  NEED(dt_bias);
+  NEED(A_q);
+  NEED(D_q);
+  NEED(exps);
+  NEED(y);
+  OPT(state);
+  const fm_exp_layout X = fm_exp_table_layout(shape);
+  return launch_scan<0>(scan_args(d, xbc, dt_raw, T, dt_bias, A_q, D_q, exps, X, state, y, nullptr),
+                        B, (cudaStream_t)stream);
+}
+
+static fm_status gate_impl(const int32_t *y, const float *z, long long M, const Dims &d,
+                           const int32_t *exps, const fm_exp_layout &X, const float *norm_w,
+                           int rotate, int mode, const float *static_amax, int8_t *q, float *s_x,
+                           float *amax_row, unsigned long long *gstat, const int32_t *e_g_override,
+                           cudaStream_t s) {
+  if (M <= 0) return FM_OK;
+  k_gate_norm_quant<<<(unsigned)M, 32 * (d.di / 256), 0, s>>>(
+      y, z, d.di, d.hd, exps + X.e_y, e_g_override ? e_g_override : exps + X.e_g, norm_w, rotate,
+      mode, static_amax, q, s_x, amax_row, gstat);
+  return launched("k_gate_norm_quant");
+}
+
+extern "C" fm_status fm_gate_norm_quant(const int32_t *y, const float *z, int64_t M,
+                                        const fm_shape *shape, const int32_t *exps,
+                                        const float *norm_w, int rotate, int mode,
+                                        const float *static_amax, int8_t *q, float *s_x,
+                                        float *amax_row, fm_stream stream) {
+  Dims d;
+  FM_TRY(check_shape(shape, &d, __func__));
+  if (M < 0 || M > 2147483647LL) return fail(FM_ERR_SHAPE, "fm_gate_norm_quant: bad M");
+  if (mode != FM_DYNAMIC && mode != FM_STATIC)
+    return fail(FM_ERR_INVALID_ARG, "fm_gate_norm_quant: bad mode %d", mode);
+  if (M == 0) return FM_OK;
+  NEED(y);
+  NEED(z);
+  NEED(exps);
+  NEED(norm_w);
+  NEED(q);
+  NEED(s_x);
+  OPT(amax_row);
+  if (mode == FM_STATIC && !static_amax)
+    return fail(FM_ERR_INVALID_ARG, "fm_gate_norm_quant: static mode needs static_amax");
+  return gate_impl(y, z, M, d, exps, fm_exp_table_layout(shape), norm_w, rotate ? 1 : 0, mode,
+                   static_amax, q, s_x, amax_row, nullptr, nullptr, (cudaStream_t)stream);
+}
+
+__global__ void k_eval_pwl(int kind, const int64_t *in, long long n, int64_t *out) {
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  const long long v = in[i];
+  long long r = 0;
+  switch (kind) {
+    case 0: r = pow2_pwl(v); break;
+    case 1: r = exp_pwl(v); break;
+    case 2: r = softplus_pwl((int)satb64(v, 32)); break;
+    case 3: r = silu_pwl((int)satb64(v, 32)); break;
+    default: r = to_q16(__uint_as_float((unsigned int)(v & 0xFFFFFFFFLL))); break;
+  }
+  out[i] = r;
+}
+
+extern "C" fm_status fm_eval_pwl(int kind, const int64_t *in, int64_t n, int64_t *out,
+                                 fm_stream stream) {
+  if (kind < 0 || kind > 4) return fail(FM_ERR_INVALID_ARG, "fm_eval_pwl: bad kind %d", kind);
+  if (n < 0) return fail(FM_ERR_SHAPE, "fm_eval_pwl: n < 0");
+  if (n == 0) return FM_OK;
+  NEED(in);
+  NEED(out);
+  k_eval_pwl<<<(unsigned)((n + 255) / 256), 256, 0, (cudaStream_t)stream>>>(kind, in, n, out);
+  return launched("k_eval_pwl");
+}
+
+// ------------------------------------------------------------------ layers
+namespace {
+struct Carver {
+  uint8_t *base;
+  size_t off;
+  template <typename T>
+  T *take(size_t n) {
+    off = (off + 255) & ~size_t(255);
+    T *p = base ? reinterpret_cast<T *>(base + off) : nullptr;
+    off += n * sizeof(T);
+    return p;
+  }
+};
+
+struct MixerWs {
+  int8_t *q_in;
+  float *sx_in;
+  float *z;
+  int8_t *xbc;
+  float *dt;
+  int8_t *xo;
+  int32_t *y;
+  int8_t *q_out;
+  float *sx_out;
+};
+
+MixerWs carve_mixer(Carver &c, const Dims &d, long long M) {
+  MixerWs w;
+  w.q_in = c.take<int8_t>(M * d.dm);
+  w.sx_in = c.take<float>(M);
+  w.z = c.take<float>(M * d.di);
+  w.xbc = c.take<int8_t>(M * d.cc);
+  w.dt = c.take<float>(M * d.nh);
+  w.xo = c.take<int8_t>(M * d.cc);
+  w.y = c.take<int32_t>(M * d.di);
+  w.q_out = c.take<int8_t>(M * d.di);
+  w.sx_out = c.take<float>(M);
+  return w;
+}
+}  // namespace
+
+extern "C" size_t fm_workspace_bytes(const fm_shape *shape, int B, int T) {
+  Dims d;
+  if (check_shape(shape, &d, __func__) != FM_OK || B < 0 || T < 0) return 0;
+  Carver c{nullptr, 0};
+  carve_mixer(c, d, (long long)B * T);
+  return c.off + 256;
+}
+
+static fm_status check_layer(const fm_layer *L, Dims *d, const char *fn) {
+  if (!L) return fail(FM_ERR_INVALID_ARG, "%s: layer is null", fn);
+  FM_TRY(check_shape(&L->shape, d, fn));
+  if (L->mode != FM_DYNAMIC && L->mode != FM_STATIC)
+    return fail(FM_ERR_INVALID_ARG, "%s: bad mode %d", fn, L->mode);
+  const void *req[] = {L->w_in_q, L->w_in_s, L->w_out_q, L->w_out_s, L->conv_wq, L->conv_bq,
+                       L->dt_bias, L->A_q, L->D_q, L->norm_w, L->exps};
+  for (const void *p : req) {
+    if (!p) return fail(FM_ERR_INVALID_ARG, "%s: a required layer pointer is null", fn);
+    if (!aligned16(p)) return fail(FM_ERR_ALIGNMENT, "%s: a layer pointer is misaligned", fn);
+  }
+  if (L->mode == FM_STATIC && !L->static_amax)
+    return fail(FM_ERR_INVALID_ARG, "%s: static mode needs static_amax", fn);
+  if (L->prenorm_w && !aligned16(L->prenorm_w))
+    return fail(FM_ERR_ALIGNMENT, "%s: prenorm_w misaligned", fn);
+  return FM_OK;
+}
+
+static fm_status mixer_impl(const fm_layer *L, const Dims &d, const float *x, int B, int T,
+                            int residual, int8_t *conv_state, int32_t *ssm_state, float *out,
+                            const MixerWs &w, cudaStream_t s) {
+  const long long M = (long long)B * T;
+  const fm_exp_layout X = fm_exp_table_layout(&L->shape);
+  const float *amax_in = L->static_amax, *amax_out = L->static_amax ? L->static_amax + 1 : nullptr;
+  FM_TRY(launch_hadamard_quant(x, M, d.dm, L->prenorm_w, L->rotate, L->mode, amax_in, w.q_in,
+                               w.sx_in, nullptr, s));
+  FM_TRY(in_proj_impl(w.q_in, w.sx_in, M, L->w_in_q, L->w_in_s, d, L->exps + X.e_u, w.z, w.xbc,
+                      w.dt, s));
+  FM_TRY(launch_conv(w.xbc, B, T, d.cc, L->conv_wq, L->conv_bq, L->exps, conv_state, w.xo,
+                     nullptr, s));
+  FM_TRY(launch_scan<0>(scan_args(d, w.xo, w.dt, T, L->dt_bias, L->A_q, L->D_q, L->exps, X,
+                                  ssm_state, w.y, nullptr),
+                        B, s));
+  FM_TRY(gate_impl(w.y, w.z, M, d, L->exps, X, L->norm_w, L->rotate, L->mode, amax_out, w.q_out,
+                   w.sx_out, nullptr, nullptr, nullptr, s));
+  return launch_gemm(w.q_out, M, L->w_out_q, d.dm, d.di,
+                     plain_epilogue(M, d.dm, w.sx_out, L->w_out_s, residual ? x : nullptr, out,
+                                    nullptr),
+                     s);
+}
+
+extern "C" fm_status fm_mixer_prefill(const fm_layer *L, const float *x, int B, int T,
+                                      int residual, int8_t *conv_state, int32_t *ssm_state,
+                                      float *out, void *ws, size_t ws_bytes, fm_stream stream) {
+  Dims d;
+  FM_TRY(check_layer(L, &d, __func__));
+  if (B < 0 || T < 0) return fail(FM_ERR_SHAPE, "fm_mixer_prefill: B, T must be >= 0");
+  if ((long long)B * T == 0) return FM_OK;
+  NEED(x);
+  NEED(out);
+  OPT(conv_state);
+  OPT(ssm_state);
+  const size_t need = fm_workspace_bytes(&L->shape, B, T);
+  if (!ws || ws_bytes < need)
+    return fail(FM_ERR_WORKSPACE, "fm_mixer_prefill: workspace needs %zu bytes", need);
+  if (out != x) {
+    const char *xb = reinterpret_cast<const char *>(x), *ob = reinterpret_cast<const char *>(out);
+    const size_t bytes = (size_t)B * T * d.dm * sizeof(float);
+    if (ob < xb + bytes && xb < ob + bytes)
+      return fail(FM_ERR_INVALID_ARG, "fm_mixer_prefill: out partially overlaps x");
+  }
+  Carver c{reinterpret_cast<uint8_t *>(ws), 0};
+  if (!aligned16(ws)) return fail(FM_ERR_ALIGNMENT, "fm_mixer_prefill: ws misaligned");
+  const MixerWs w = carve_mixer(c, d, (long long)B * T);
+  return mixer_impl(L, d, x, B, T, residual, conv_state, ssm_state, out, w, (cudaStream_t)stream);
+}
+
+extern "C" fm_status fm_decode_step(const fm_layer *L, const float *x, int B, int residual,
+                                    int8_t *conv_state, int32_t *ssm_state, float *out, void *ws,
+                                    size_t ws_bytes, fm_stream stream) {
+  if (!conv_state || !ssm_state)
+    return fail(FM_ERR_INVALID_ARG, "fm_decode_step: conv_state and ssm_state are required");
+  return fm_mixer_prefill(L, x, B, 1, residual, conv_state, ssm_state, out, ws, ws_bytes, stream);
+}
+
+// ------------------------------------------------------------------ offline preparation
+__global__ void k_prepare_mixer_params(const float *conv_w, const float *a_log, const float *D,
+                                       int cc, int nh, int8_t *conv_wq, int32_t *A_q,
+                                       int32_t *D_q, int32_t *e_w, int32_t *e_D) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < cc) {
+    double amax = 0.0;
+    for (int k = 0; k < 4; ++k) amax = fmax(amax, fabs((double)conv_w[i * 4 + k]));
+    const int e = pot_exponent(amax, 127.0);
+    e_w[i] = e;
+    for (int k = 0; k < 4; ++k)
+      conv_wq[i * 4 + k] = (int8_t)round_clamp(__fmul_rn(conv_w[i * 4 + k], ldexpf(1.0f, -e)), 127.0f);
+  }
+  if (i < nh) {
+    // A_q = rint(exp(A_log) log2(e) 2^12): A = -exp(A_log) folded with log2(e)
+    A_q[i] = (int32_t)llrint(__dmul_rn(__ddiv_rn(exp((double)a_log[i]), 0.69314718055994530942), 4096.0));
+    const int e = pot_exponent(fabs((double)D[i]), 16384.0);
+    e_D[i] = e;
+    D_q[i] = (int32_t)satb64(llrint(ldexp((double)D[i], -e)), 16);
+  }
+}
+
+extern "C" fm_status fm_prepare_mixer_params(const fm_shape *shape, const float *conv_w,
+                                             const float *a_log, const float *D, int8_t *conv_wq,
+                                             int32_t *A_q, int32_t *D_q, int32_t *exps,
+                                             fm_stream stream) {
+  Dims d;
+  FM_TRY(check_shape(shape, &d, __func__));
+  NEED(conv_w);
+  NEED(a_log);
+  NEED(D);
+  NEED(conv_wq);
+  NEED(A_q);
+  NEED(D_q);
+  NEED(exps);
+  const fm_exp_layout X = fm_exp_table_layout(shape);
+  const int n = d.cc > d.nh ? d.cc : d.nh;
+  k_prepare_mixer_params<<<(n + 127) / 128, 128, 0, (cudaStream_t)stream>>>(
+      conv_w, a_log, D, d.cc, d.nh, conv_wq, A_q, D_q, exps + X.e_w, exps + X.e_D);
+  return launched("k_prepare_mixer_params");
+}
+
+// ------------------------------------------------------------------ calibration
+// Stage statistics -> exponents, all on the device (see fm_calibrate_layer).
+__global__ void k_calib_fill(int32_t *p, int n, int v) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) p[i] = v;
+}
+__global__ void k_max_f32(const float *v, long long n, float *out) {
+  __shared__ float red[32];
+  float m = 0.0f;
+  for (long long i = threadIdx.x; i < n; i += blockDim.x) m = fmaxf(m, v[i]);
+  m = warp_max(m);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float r = 0.0f;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) r = fmaxf(r, red[w]);
+    *out = r;
+  }
+}
+// per-column max |Y[:, c0 + c]| as float bits (non-negative floats order like uint)
+__global__ void k_col_amax(const float *Y, long long M, int N, int c0, int nc, unsigned int *out) {
+  const int c = blockIdx.x * blockDim.x + threadIdx.x;
+  if (c >= nc) return;
+  float m = 0.0f;
+  for (long long r = blockIdx.y; r < M; r += gridDim.y) m = fmaxf(m, fabsf(Y[r * N + c0 + c]));
+  atomicMax(out + c, __float_as_uint(m));
+}
+__global__ void k_exp_conv_in(const unsigned int *amax_bits, const float *conv_b,
+                              const int32_t *e_w, int cc, int32_t *e_u, int32_t *bq) {
+  const int c = blockIdx.x * blockDim.x + threadIdx.x;
+  if (c >= cc) return;
+  const int e = pot_exponent((double)__uint_as_float(amax_bits[c]), 127.0);
+  e_u[c] = e;
+  double v = rint(ldexp((double)conv_b[c], -(e_w[c] + e)));
+  v = fmin(fmax(v, -2147483647.0), 2147483647.0);
+  bq[c] = (int32_t)v;
+}
+// conv output exponents from max |SiLU| per channel (single CTA)
+__global__ void k_exp_conv_out(const unsigned int *amax, int di, int hd, int ds, int32_t *exps,
+                               fm_exp_layout X) {
+  const int nh = di / hd, cc = di + 2 * ds;
+  for (int h = threadIdx.x; h < nh + 2; h += blockDim.x) {
+    const int lo = h < nh ? h * hd : (h == nh ? di : di + ds);
+    const int n = h < nh ? hd : ds;
+    unsigned int m = 0;
+    for (int c = lo; c < lo + n; ++c) m = amax[c] > m ? amax[c] : m;
+    const int e = pot_exponent((double)m, 127.0) - 16;
+    if (h < nh) exps[X.e_x + h] = e;
+    else if (h == nh) exps[X.e_B] = e;
+    else exps[X.e_C] = e;
+  }
+  __syncthreads();
+  for (int c = threadIdx.x; c < cc; c += blockDim.x)
+    exps[X.e_o + c] = c < di ? exps[X.e_x + c / hd] : (c < di + ds ? exps[X.e_B] : exps[X.e_C]);
+}
+__global__ void k_exp_state(const unsigned long long *amax_h, int nh, int32_t *exps,
+                            fm_exp_layout X) {
+  const int h = threadIdx.x;
+  if (h >= nh) return;
+  const int ef = exps[X.e_x + h] + exps[X.e_B] - 15;
+  const int e = pot_exponent((double)amax_h[h], 536870912.0) + ef;
+  exps[X.e_h + h] = e > ef ? e : ef;
+}
+__global__ void k_exp_y(const unsigned long long *ystat, int nh, int32_t *exps, fm_exp_layout X) {
+  const int h = threadIdx.x;
+  if (h >= nh) return;
+  const int a = exps[X.e_C] + exps[X.e_h + h], b = exps[X.e_D + h] + exps[X.e_x + h];
+  const int ef = a < b ? a : b, hi = a > b ? a : b;
+  const int e = pot_exponent((double)ystat[h], 536870912.0) + ef;
+  exps[X.e_y + h] = e > hi - 16 ? e : hi - 16;
+}
+// e_g: before the statistics pass (gstat == null) the lower bound max e_y - 16
+// (every gate shift >= 0), after it the calibrated value.
+__global__ void k_exp_gate(const unsigned long long *gstat, int nh, int32_t *exps,
+                           fm_exp_layout X) {
+  if (threadIdx.x != 0) return;
+  int ymax = -1000000;
+  for (int h = 0; h < nh; ++h) ymax = exps[X.e_y + h] > ymax ? exps[X.e_y + h] : ymax;
+  int e = ymax - 16;
+  if (gstat)
+    for (int h = 0; h < nh; ++h) {
+      const int eh = pot_exponent((double)gstat[h], 32767.0) + exps[X.e_y + h] - 16;
+      e = eh > e ? eh : e;
+    }
+  exps[X.e_g] = e;
+}
+
+namespace {
+struct CalibWs {
+  MixerWs m;
+  float *Y;               // [M, n_in] in_proj output (fp32)
+  float *amax_row;        // [M]
+  unsigned int *col_amax; // [cc]
+  unsigned int *silu_amax;// [cc]
+  unsigned long long *stat;  // [nh]
+};
+CalibWs carve_calib(Carver &c, const Dims &d, long long M) {
+  CalibWs w;
+  w.m = carve_mixer(c, d, M);
+  w.Y = c.take<float>(M * d.n_in);
+  w.amax_row = c.take<float>(M);
+  w.col_amax = c.take<unsigned int>(d.cc);
+  w.silu_amax = c.take<unsigned int>(d.cc);
+  w.stat = c.take<unsigned long long>(d.nh);
+  return w;
+}
+}  // namespace
+
+extern "C" size_t fm_calib_workspace_bytes(const fm_shape *shape, int B, int T) {
+  Dims d;
+  if (check_shape(shape, &d, __func__) != FM_OK || B < 0 || T < 0) return 0;
+  Carver c{nullptr, 0};
+  carve_calib(c, d, (long long)B * T);
+  return c.off + 256;
+}
+
+extern "C" fm_status fm_calibrate_layer(const fm_layer *L, const float *conv_b, int32_t *exps,
+                                        int32_t *conv_bq, float *static_amax, const float *xcal,
+                                        int B, int T, int residual, float *out, void *ws,
+                                        size_t ws_bytes, fm_stream stream) {
+  Dims d;
+  FM_TRY(check_layer(L, &d, __func__));
+  NEED(conv_b);
+  NEED(exps);
+  NEED(conv_bq);
+  NEED(static_amax);
+  NEED(xcal);
+  NEED(out);
+  if (exps != L->exps || conv_bq != L->conv_bq || static_amax != L->static_amax)
+    return fail(FM_ERR_INVALID_ARG, "fm_calibrate_layer: table pointers must be the layer's own");
+  if (B <= 0 || T <= 0) return fail(FM_ERR_SHAPE, "fm_calibrate_layer: need B, T > 0");
+  const size_t need = fm_calib_workspace_bytes(&L->shape, B, T);
+  if (!ws || ws_bytes < need || !aligned16(ws))
+    return fail(FM_ERR_WORKSPACE, "fm_calibrate_layer: workspace needs %zu bytes", need);
+  cudaStream_t s = (cudaStream_t)stream;
+  const long long M = (long long)B * T;
+  const fm_exp_layout X = fm_exp_table_layout(&L->shape);
+  Carver c{reinterpret_cast<uint8_t *>(ws), 0};
+  const CalibWs w = carve_calib(c, d, M);
+  const MixerWs &m = w.m;
+
+  // 1. in_proj input: max |rotated (normed) input| -> static_amax[0]
+  FM_TRY(launch_hadamard_quant(xcal, M, d.dm, L->prenorm_w, L->rotate, FM_DYNAMIC, nullptr, m.q_in,
+                               m.sx_in, w.amax_row, s));
+  k_max_f32<<<1, 1024, 0, s>>>(w.amax_row, M, static_amax);
+  FM_TRY(launched("k_max_f32"));
+  if (L->mode == FM_STATIC)
+    FM_TRY(launch_hadamard_quant(xcal, M, d.dm, L->prenorm_w, L->rotate, FM_STATIC, static_amax,
+                                 m.q_in, m.sx_in, nullptr, s));
+  // 2. conv input exponents from the dequantised in_proj output; bias codes
+  FM_TRY(launch_gemm(m.q_in, M, L->w_in_q, d.n_in, d.dm,
+                     plain_epilogue(M, d.n_in, m.sx_in, L->w_in_s, nullptr, w.Y, nullptr), s));
+  FM_CHECK_CUDA(cudaMemsetAsync(w.col_amax, 0, sizeof(unsigned int) * d.cc, s));
+  {
+    const long long gy = M < 1024 ? M : 1024;
+    k_col_amax<<<dim3((d.cc + 127) / 128, (unsigned)gy), 128, 0, s>>>(w.Y, M, d.n_in, d.di, d.cc,
+                                                                       w.col_amax);
+    FM_TRY(launched("k_col_amax"));
+  }
+  k_exp_conv_in<<<(d.cc + 127) / 128, 128, 0, s>>>(w.col_amax, conv_b, exps + X.e_w, d.cc,
+                                                   exps + X.e_u, conv_bq);
+  FM_TRY(launched("k_exp_conv_in"));
+  FM_TRY(in_proj_impl(m.q_in, m.sx_in, M, L->w_in_q, L->w_in_s, d, exps + X.e_u, m.z, m.xbc, m.dt,
+                      s));
+  // 3. conv output exponents (statistics pass with e_o = 0, then the real pass)
+  k_calib_fill<<<(d.cc + 127) / 128, 128, 0, s>>>(exps + X.e_o, d.cc, 0);
+  FM_TRY(launched("k_calib_fill"));
+  FM_CHECK_CUDA(cudaMemsetAsync(w.silu_amax, 0, sizeof(unsigned int) * d.cc, s));
+  FM_TRY(launch_conv(m.xbc, B, T, d.cc, L->conv_wq, conv_bq, exps, nullptr, m.xo, w.silu_amax, s));
+  k_exp_conv_out<<<1, 256, 0, s>>>(w.silu_amax, d.di, d.hd, d.ds, exps, X);
+  FM_TRY(launched("k_exp_conv_out"));
+  FM_TRY(launch_conv(m.xbc, B, T, d.cc, L->conv_wq, conv_bq, exps, nullptr, m.xo, nullptr, s));
+  // 4. state exponent: 64-bit run at the finest exponent
+  FM_CHECK_CUDA(cudaMemsetAsync(w.stat, 0, sizeof(unsigned long long) * d.nh, s));
+  FM_TRY(launch_scan<2>(scan_args(d, m.xo, m.dt, T, L->dt_bias, L->A_q, L->D_q, exps, X, nullptr,
+                                  m.y, w.stat),
+                        B, s));
+  k_exp_state<<<1, 128, 0, s>>>(w.stat, d.nh, exps, X);
+  FM_TRY(launched("k_exp_state"));
+  // 5. output exponent: max |y| at the finer term exponent
+  FM_CHECK_CUDA(cudaMemsetAsync(w.stat, 0, sizeof(unsigned long long) * d.nh, s));
+  FM_TRY(launch_scan<1>(scan_args(d, m.xo, m.dt, T, L->dt_bias, L->A_q, L->D_q, exps, X, nullptr,
+                                  m.y, w.stat),
+                        B, s));
+  k_exp_y<<<1, 128, 0, s>>>(w.stat, d.nh, exps, X);
+  FM_TRY(launched("k_exp_y"));
+  FM_TRY(launch_scan<0>(scan_args(d, m.xo, m.dt, T, L->dt_bias, L->A_q, L->D_q, exps, X, nullptr,
+                                  m.y, nullptr),
+                        B, s));
+  // 6. gate exponent, then the out_proj input amax
+  k_exp_gate<<<1, 32, 0, s>>>(nullptr, d.nh, exps, X);
+  FM_TRY(launched("k_exp_gate"));
+  FM_CHECK_CUDA(cudaMemsetAsync(w.stat, 0, sizeof(unsigned long long) * d.nh, s));
+  FM_TRY(gate_impl(m.y, m.z, M, d, exps, X, L->norm_w, L->rotate, FM_DYNAMIC, nullptr, m.q_out,
+                   m.sx_out, nullptr, w.stat, nullptr, s));
+  k_exp_gate<<<1, 32, 0, s>>>(w.stat, d.nh, exps, X);
+  FM_TRY(launched("k_exp_gate"));
+  FM_TRY(gate_impl(m.y, m.z, M, d, exps, X, L->norm_w, L->rotate, FM_DYNAMIC, nullptr, m.q_out,
+                   m.sx_out, w.amax_row, nullptr, nullptr, s));
+  k_max_f32<<<1, 1024, 0, s>>>(w.amax_row, M, static_amax + 1);
+  FM_TRY(launched("k_max_f32"));
+  if (L->mode == FM_STATIC)
+    FM_TRY(gate_impl(m.y, m.z, M, d, exps, X, L->norm_w, L->rotate, FM_STATIC, static_amax + 1,
+                     m.q_out, m.sx_out, nullptr, nullptr, nullptr, s));
+  // 7. the layer's output on the calibration set
+  return launch_gemm(m.q_out, M, L->w_out_q, d.dm, d.di,
+                     plain_epilogue(M, d.dm, m.sx_out, L->w_out_s, residual ? xcal : nullptr, out,
+                                    nullptr),
+                     s);
+}

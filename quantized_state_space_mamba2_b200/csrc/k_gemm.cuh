@@ -1,0 +1,340 @@
+// k_gemm.cuh -- W8A8 GEMM on the 5th-generation tensor cores (tcgen05, kind::i8).
+//
+// acc[m, n] = sum_k A[m, k] W[n, k] in exact int32 (Hadamard-rotated int8
+// operands; FastMamba, arXiv 2505.18975, pith.science review "What carries
+// the argument": Y = (XH)(H^T W^T)), followed by the dequantisation
+// fl(fl(float(acc) * s_x[m]) * s_w[n]) and either a plain fp32 store (+ an
+// optional residual) or the in_proj split into z / xBC power-of-two codes /
+// dt (Mamba2 column order).
+//
+// Structure (one 128 x BN output tile per CTA, 6 warps):
+//   warp 0      TMA producer: 128-byte-swizzled A and W tiles (128 x 128 and
+//               BN x 128 int8) into a STAGES-deep shared-memory ring;
+//   warp 1      allocates TMEM (BN columns of int32) and one elected lane
+//               issues tcgen05.mma (M=128, N=BN, K=32 per instruction);
+//               tcgen05.commit frees each ring slot and finally signals the
+//               accumulator;
+//   warps 2..5  epilogue: tcgen05.ld 32 columns at a time from their TMEM
+//               lane quarter, dequantise and store.
+// Every mbarrier wait is bounded by a wall-clock limit; on expiry the thread
+// sets the device error word and the kernel runs to its end (TMEM is always
+// released), so a broken pipeline can never hang the GPU.
+#pragma once
+#include <cuda.h>
+#include "fm_common.cuh"
+
+namespace fm {
+
+constexpr int kGemmBM = 128;
+constexpr int kGemmBK = 128;  // int8 elements = bytes per row per stage (one swizzle atom)
+constexpr int kGemmThreads = 192;
+constexpr unsigned long long kWaitLimitNs = 4000000000ull;  // 4 s
+
+struct GemmEpilogue {
+  int mode;  // 0: plain (Y, residual), 1: in_proj split
+  long long M, N;
+  const float *s_x, *s_w;
+  const float *residual;
+  float *Y;
+  int32_t *acc_out;
+  // in_proj split
+  int di, cc, nh;
+  const int32_t *e_u;
+  float *z;
+  int8_t *xbc;
+  float *dt;
+};
+
+// ------------------------------------------------------------ PTX wrappers
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ unsigned long long globaltimer() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// bounded wait: false (and the error word set) if the phase never completes
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (globaltimer() - t0 > kWaitLimitNs) {
+      raise_error(kErrTimeout);
+      return false;
+    }
+  }
+}
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *tm, int c0, int c1,
+                                            uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+      "l"((unsigned long long)tm), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+// Shared-memory matrix descriptor (sm_100 format): K-major operand whose rows
+// are 128 bytes, 128-byte swizzle, 8-row groups 1024 bytes apart.
+//   bits  0-13 start address >> 4      bits 16-29 leading byte offset >> 4 (1, unused)
+//   bits 32-45 stride byte offset >> 4 (1024 >> 4)
+//   bits 46-47 descriptor version (1)  bits 61-63 layout (2 = 128-byte swizzle)
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)1u << 16;
+  d |= (uint64_t)(1024u >> 4) << 32;
+  d |= (uint64_t)1u << 46;
+  d |= (uint64_t)2u << 61;
+  return d;
+}
+// Instruction descriptor, kind::i8: D = s32 (bits 4-5 = 2), A and B signed
+// int8 (bits 7-9 = 1, 10-12 = 1), both K-major, N >> 3 at bits 17-22,
+// M >> 4 at bits 24-28.
+__host__ __device__ constexpr uint32_t i8_idesc(int M, int N) {
+  return (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
+         ((uint32_t)(M >> 4) << 24);
+}
+__device__ __forceinline__ void mma_i8(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                       uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mma_commit(uint64_t *bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+        "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+        "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__host__ __device__ constexpr int gemm_smem_bytes(int BN, int stages) {
+  return stages * (kGemmBM + BN) * kGemmBK + 1024 /*align slack*/ + 256 /*barriers*/;
+}
+
+// ------------------------------------------------------------ epilogue
+__device__ __forceinline__ float pow2f(int e) {  // exact 2^e for e in [-126, 127]
+  return __int_as_float((127 + e) << 23);
+}
+
+__device__ __forceinline__ void gemm_store_chunk(const GemmEpilogue &ep, long long row,
+                                                 long long col0, const uint32_t (&r)[32]) {
+  if (row >= ep.M) return;
+  const float sx = ep.s_x[row];
+  const bool full = col0 + 32 <= ep.N;
+  if (ep.acc_out) {
+    int32_t *dst = ep.acc_out + row * ep.N + col0;
+    for (int j = 0; j < 32; ++j)
+      if (col0 + j < ep.N) dst[j] = (int32_t)r[j];
+  }
+  float y[32];
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    const long long c = col0 + j;
+    const float sw = c < ep.N ? ep.s_w[c] : 0.0f;
+    y[j] = __fmul_rn(__fmul_rn(__int2float_rn((int)r[j]), sx), sw);
+  }
+  if (ep.mode == 0) {
+    float *dst = ep.Y + row * ep.N + col0;
+    const float *res = ep.residual ? ep.residual + row * ep.N + col0 : nullptr;
+    if (full && ((ep.N & 3) == 0)) {
+#pragma unroll
+      for (int j = 0; j < 32; j += 4) {
+        float4 o = make_float4(y[j], y[j + 1], y[j + 2], y[j + 3]);
+        if (res) {
+          const float4 rv = *reinterpret_cast<const float4 *>(res + j);
+          o.x = __fadd_rn(rv.x, o.x);
+          o.y = __fadd_rn(rv.y, o.y);
+          o.z = __fadd_rn(rv.z, o.z);
+          o.w = __fadd_rn(rv.w, o.w);
+        }
+        *reinterpret_cast<float4 *>(dst + j) = o;
+      }
+    } else {
+      for (int j = 0; j < 32; ++j) {
+        if (col0 + j >= ep.N) break;
+        dst[j] = res ? __fadd_rn(res[j], y[j]) : y[j];
+      }
+    }
+    return;
+  }
+  // in_proj split: [0, di) z | [di, di+cc) xBC codes | [di+cc, N) dt
+  const long long di = ep.di, cc = ep.cc;
+  if (full && col0 + 32 <= di && (di & 3) == 0) {
+    float *dst = ep.z + row * di + col0;
+#pragma unroll
+    for (int j = 0; j < 32; j += 4)
+      *reinterpret_cast<float4 *>(dst + j) = make_float4(y[j], y[j + 1], y[j + 2], y[j + 3]);
+    return;
+  }
+  if (full && col0 >= di && col0 + 32 <= di + cc && ((col0 - di) & 15) == 0 && (cc & 15) == 0) {
+    const long long c0 = col0 - di;
+    uint32_t packed[8];
+#pragma unroll
+    for (int j = 0; j < 32; j += 4) {
+      uint32_t w = 0;
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        const int code = round_clamp(__fmul_rn(y[j + b], pow2f(-ep.e_u[c0 + j + b])), 127.0f);
+        w |= ((uint32_t)(code & 0xFF)) << (8 * b);
+      }
+      packed[j / 4] = w;
+    }
+    uint4 *dst = reinterpret_cast<uint4 *>(ep.xbc + row * cc + c0);
+    dst[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+    dst[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+    return;
+  }
+  for (int j = 0; j < 32; ++j) {
+    const long long c = col0 + j;
+    if (c >= ep.N) break;
+    if (c < di) {
+      ep.z[row * di + c] = y[j];
+    } else if (c < di + cc) {
+      const long long cx = c - di;
+      ep.xbc[row * cc + cx] = (int8_t)round_clamp(__fmul_rn(y[j], pow2f(-ep.e_u[cx])), 127.0f);
+    } else {
+      ep.dt[row * ep.nh + (c - di - cc)] = y[j];
+    }
+  }
+}
+
+// ------------------------------------------------------------ the kernel
+template <int BN, int STAGES>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    k_gemm_i8_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                 int num_k_blocks, GemmEpilogue ep) {
+  static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN");
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~static_cast<uintptr_t>(1023));
+  uint8_t *sA = smem;
+  uint8_t *sB = smem + STAGES * kGemmBM * kGemmBK;
+  uint64_t *full_bar = reinterpret_cast<uint64_t *>(sB + STAGES * BN * kGemmBK);
+  uint64_t *empty_bar = full_bar + STAGES;
+  uint64_t *accum_bar = empty_bar + STAGES;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(accum_bar + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int m0 = blockIdx.y * kGemmBM;
+  const int n0 = blockIdx.x * BN;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    mbar_init(accum_bar, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"((unsigned long long)&tmA) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"((unsigned long long)&tmB) : "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"((uint32_t)BN)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      for (int kb = 0; kb < num_k_blocks; ++kb) {
+        const int s = kb % STAGES;
+        const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
+        if (!mbar_wait(&empty_bar[s], ph ^ 1u)) break;
+        mbar_arrive_expect_tx(&full_bar[s], (uint32_t)((kGemmBM + BN) * kGemmBK));
+        tma_load_2d(sA + s * kGemmBM * kGemmBK, &tmA, kb * kGemmBK, m0, &full_bar[s]);
+        tma_load_2d(sB + s * BN * kGemmBK, &tmB, kb * kGemmBK, n0, &full_bar[s]);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = i8_idesc(kGemmBM, BN);
+      for (int kb = 0; kb < num_k_blocks; ++kb) {
+        const int s = kb % STAGES;
+        const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
+        if (!mbar_wait(&full_bar[s], ph)) break;
+        tc_fence_after();
+        const uint64_t ad = sw128_desc(smem_u32(sA + s * kGemmBM * kGemmBK));
+        const uint64_t bd = sw128_desc(smem_u32(sB + s * BN * kGemmBK));
+#pragma unroll
+        for (int k = 0; k < kGemmBK / 32; ++k) {
+          // advance the start address by 32 bytes (2 x 16 B) per K=32 slice
+          mma_i8(tmem_base, ad + (uint64_t)(2 * k), bd + (uint64_t)(2 * k), idesc,
+                 (kb > 0 || k > 0) ? 1u : 0u);
+        }
+        mma_commit(&empty_bar[s]);
+      }
+      mma_commit(accum_bar);
+    }
+  } else {
+    const bool ok = mbar_wait(accum_bar, 0);
+    tc_fence_after();
+    const int quarter = warp & 3;  // TMEM lanes [32*quarter, 32*quarter + 32)
+    const long long row = (long long)m0 + quarter * 32 + lane;
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 32) {
+      uint32_t r[32];
+      tmem_ld32(tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)c, r);
+      if (ok && n0 + c < ep.N) gemm_store_chunk(ep, row, (long long)n0 + c, r);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"((uint32_t)BN)
+                 : "memory");
+  }
+}
+
+}  // namespace fm

@@ -1,0 +1,231 @@
+// k_rows.cuh -- row-wise kernels: Hadamard rotation + int8 quantisation of
+// the linear-layer inputs, the fused gate + gated RMSNorm in front of
+// out_proj, and the offline fp64 weight rotation.
+//
+// FastMamba (arXiv 2505.18975), pith.science review: "What carries the
+// argument" (Y = (XH)(H^T W^T), H orthonormal after 1/sqrt(n)); Referee
+// Report, major comment 1 (scales from the max of the rotated tensors, static
+// scales in the hardware of Fig. 6); minor comment 2 (H depends only on the
+// dimension).  Gate-then-normalise order and RMSNorm are those of Mamba2 (the
+// paper's references [2], [10]).
+//
+// Layout: one CTA per row, one warp per 256-column Hadamard block, each lane
+// holding 8 consecutive elements (two 16-byte loads), so the whole row's
+// rotation happens in registers and shuffles; HBM traffic is one read of the
+// row and one write of its codes.
+#pragma once
+#include "fm_common.cuh"
+
+namespace fm {
+
+constexpr int kMaxBlocks = 32;  // K <= 8192
+
+// Row max over all warps of the CTA (every thread returns the result).
+__device__ __forceinline__ float cta_max(float v, float *s_red, float *s_out) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  v = warp_max(v);
+  if (lane == 0) s_red[warp] = v;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float m = 0.0f;
+    for (int w = 0; w < nw; ++w) m = fmaxf(m, s_red[w]);
+    *s_out = m;
+  }
+  __syncthreads();
+  return *s_out;
+}
+
+// Rotation (optional) + per-row or static quantisation of v[8] (this lane's
+// 8 elements at column 256*warp + 8*lane); thread 0 writes s_x / amax_row.
+__device__ __forceinline__ void rotate_quant_store(float (&v)[8], int rotate, int mode,
+                                                   const float *static_amax, int8_t *qrow,
+                                                   float *sx_out, float *amax_out,
+                                                   float *s_red, float *s_bc) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (rotate) fwht256_lane8(v, lane);
+  float a = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) a = fmaxf(a, fabsf(v[i]));
+  const float amax = cta_max(a, s_red, s_bc);
+  const float use = (mode == 0) ? amax : *static_amax;
+  uint32_t lo = 0, hi = 0;
+  if (use > 0.0f) {
+    const float inv = __fdiv_rn(127.0f, use);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const uint32_t c = (uint32_t)(round_clamp(__fmul_rn(v[i], inv), 127.0f) & 0xFF);
+      if (i < 4) lo |= c << (8 * i);
+      else hi |= c << (8 * (i - 4));
+    }
+  }
+  *reinterpret_cast<uint2 *>(qrow + warp * 256 + lane * 8) = make_uint2(lo, hi);
+  if (threadIdx.x == 0) {
+    *sx_out = use > 0.0f ? __fdiv_rn(use, 127.0f) : 0.0f;
+    if (amax_out) *amax_out = amax;
+  }
+}
+
+// a0 + a1 (and a10's tail): blockDim = 32 * (K / 256), grid = M.
+__global__ void __launch_bounds__(1024) k_hadamard_quant(const float *__restrict__ x, int K,
+                                                         const float *__restrict__ prenorm_w,
+                                                         int rotate, int mode,
+                                                         const float *static_amax,
+                                                         int8_t *__restrict__ q, float *s_x,
+                                                         float *amax_row) {
+  __shared__ double s_blk[kMaxBlocks];
+  __shared__ float s_red[kMaxBlocks];
+  __shared__ float s_bc;
+  __shared__ float s_rstd;
+  const long long row = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nb = blockDim.x >> 5;
+  const float *src = x + row * K + warp * 256 + lane * 8;
+  float v[8];
+  {
+    const float4 a = *reinterpret_cast<const float4 *>(src);
+    const float4 b = *reinterpret_cast<const float4 *>(src + 4);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  }
+  if (prenorm_w) {
+    // RMSNorm (eps 1e-5): sum of squares in double in the fixed order
+    // (lane-sequential 8, xor tree over the warp, blocks in increasing order)
+    double P = 0.0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const double e = (double)v[i];
+      P = __dadd_rn(P, __dmul_rn(e, e));
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) P = __dadd_rn(P, __shfl_xor_sync(0xffffffffu, P, o));
+    if (lane == 0) s_blk[warp] = P;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      double tot = 0.0;
+      for (int b = 0; b < nb; ++b) tot = __dadd_rn(tot, s_blk[b]);
+      const double var = __ddiv_rn(tot, (double)K);
+      s_rstd = (float)__drcp_rn(__dsqrt_rn(__dadd_rn(var, 1e-5)));
+    }
+    __syncthreads();
+    const float rstd = s_rstd;
+    const float *w = prenorm_w + warp * 256 + lane * 8;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(__fmul_rn(v[i], rstd), w[i]);
+  }
+  rotate_quant_store(v, rotate, mode, static_amax, q + row * K, s_x + row,
+                     amax_row ? amax_row + row : nullptr, s_red, &s_bc);
+}
+
+// a9 + a10: gate y * SiLU(z), g_q int16 at e_g, exact-integer RMSNorm,
+// rotation, quantisation.  blockDim = 32 * (di / 256), grid = M.
+// gstat (nullable, [nh] u64): max |g| per head (calibration).
+__global__ void __launch_bounds__(1024) k_gate_norm_quant(
+    const int32_t *__restrict__ y, const float *__restrict__ z, int di, int hd,
+    const int32_t *__restrict__ e_y, const int32_t *__restrict__ e_g_ptr,
+    const float *__restrict__ norm_w, int rotate, int mode, const float *static_amax,
+    int8_t *__restrict__ q, float *s_x, float *amax_row, unsigned long long *gstat) {
+  __shared__ long long s_ss[kMaxBlocks];
+  __shared__ float s_red[kMaxBlocks];
+  __shared__ float s_bc;
+  __shared__ float s_rstd;
+  const long long row = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nb = blockDim.x >> 5;
+  const int col = warp * 256 + lane * 8;
+  const int head = col / hd;  // hd is a multiple of 8: the lane's 8 columns share a head
+  const int e_g = *e_g_ptr;
+  const int sg_shift = e_g - e_y[head] + 16;
+  int32_t yv[8];
+  float zv[8];
+  {
+    const int4 a = *reinterpret_cast<const int4 *>(y + row * di + col);
+    const int4 b = *reinterpret_cast<const int4 *>(y + row * di + col + 4);
+    yv[0] = a.x; yv[1] = a.y; yv[2] = a.z; yv[3] = a.w;
+    yv[4] = b.x; yv[5] = b.y; yv[6] = b.z; yv[7] = b.w;
+    const float4 c = *reinterpret_cast<const float4 *>(z + row * di + col);
+    const float4 d = *reinterpret_cast<const float4 *>(z + row * di + col + 4);
+    zv[0] = c.x; zv[1] = c.y; zv[2] = c.z; zv[3] = c.w;
+    zv[4] = d.x; zv[5] = d.y; zv[6] = d.z; zv[7] = d.w;
+  }
+  int gq[8];
+  long long ss = 0;
+  unsigned long long gmax = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const long long g = (long long)yv[i] * silu_pwl(to_q16(zv[i]));
+    const unsigned long long ag = (unsigned long long)(g < 0 ? -g : g);
+    gmax = ag > gmax ? ag : gmax;
+    gq[i] = (int)satb64(rshr64(g, sg_shift), 16);
+    ss += (long long)gq[i] * gq[i];
+  }
+  if (gstat) {
+    // the 8 lanes of a 64-column head combine, one atomic per head
+#pragma unroll
+    for (int o = 1; o < 8; o <<= 1) {
+      const unsigned long long other = __shfl_xor_sync(0xffffffffu, gmax, o);
+      gmax = other > gmax ? other : gmax;
+    }
+    if ((lane & 7) == 0) atomicMax(gstat + head, gmax);
+  }
+  ss = warp_sum_ll(ss);
+  if (lane == 0) s_ss[warp] = ss;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    long long tot = 0;
+    for (int b = 0; b < nb; ++b) tot += s_ss[b];
+    const double var = __ddiv_rn(ldexp((double)tot, 2 * e_g), (double)di);
+    s_rstd = (float)__drcp_rn(__dsqrt_rn(__dadd_rn(var, 1e-5)));
+  }
+  __syncthreads();
+  const float rstd = s_rstd;
+  const float scale = ldexpf(1.0f, e_g);
+  const float *w = norm_w + col;
+  float v[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(__fmul_rn(__fmul_rn((float)gq[i], scale), rstd), w[i]);
+  rotate_quant_store(v, rotate, mode, static_amax, q + row * di, s_x + row,
+                     amax_row ? amax_row + row : nullptr, s_red, &s_bc);
+}
+
+// Offline weight preparation: W' = W H (fp64, same butterfly order),
+// s_w = fl32(max|W'| / 127), Wq = satb(rint(W' / s_w), 8).  grid = N rows.
+__global__ void __launch_bounds__(1024) k_prepare_linear(const float *__restrict__ W, int K,
+                                                         int rotate, int8_t *__restrict__ Wq,
+                                                         float *__restrict__ s_w) {
+  __shared__ double s_red[kMaxBlocks];
+  __shared__ double s_amax;
+  const long long row = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nb = blockDim.x >> 5;
+  const int col = warp * 256 + lane * 8;
+  double v[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = (double)W[row * K + col + i];
+  if (rotate) fwht256_lane8(v, lane);
+  double a = 0.0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) a = fmax(a, fabs(v[i]));
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) a = fmax(a, __shfl_xor_sync(0xffffffffu, a, o));
+  if (lane == 0) s_red[warp] = a;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double m = 0.0;
+    for (int b = 0; b < nb; ++b) m = fmax(m, s_red[b]);
+    s_amax = m;
+  }
+  __syncthreads();
+  const float s = (float)__ddiv_rn(s_amax, 127.0);
+  if (threadIdx.x == 0) s_w[row] = s;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    int c = 0;
+    if (s > 0.0f) {
+      double r = rint(__ddiv_rn(v[i], (double)s));
+      r = fmin(fmax(r, -127.0), 127.0);
+      c = (int)r;
+    }
+    Wq[row * K + col + i] = (int8_t)c;
+  }
+}
+
+}  // namespace fm

@@ -1,0 +1,216 @@
+"""ctypes binding of libfastmamba.so (include/fastmamba.h), same names.
+
+Argument marshalling only: tensors are torch CUDA tensors (device memory
+owned by the caller), streams are torch streams; every computation happens
+in the library's kernels.  There is no CPU fallback: if the shared library
+is missing or no CUDA device is present the calls raise.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+SO_PATH = os.path.join(_HERE, "libfastmamba.so")
+
+FM_DYNAMIC, FM_STATIC = 0, 1
+STATUS = {0: "FM_OK", 1: "FM_ERR_INVALID_ARG", 2: "FM_ERR_SHAPE", 3: "FM_ERR_ALIGNMENT",
+          4: "FM_ERR_WORKSPACE", 5: "FM_ERR_NONFINITE", 6: "FM_ERR_TIMEOUT", 7: "FM_ERR_CUDA",
+          8: "FM_ERR_UNSUPPORTED"}
+
+# every entry point the header declares
+EXPORTS = (
+    "fm_status_string", "fm_last_error", "fm_sync_status", "fm_version", "fm_exp_table_layout",
+    "fm_hadamard_quant", "fm_prepare_linear", "fm_w8a8_gemm", "fm_in_proj", "fm_conv1d_pot",
+    "fm_ssm_scan_pot", "fm_gate_norm_quant", "fm_eval_pwl", "fm_workspace_bytes",
+    "fm_mixer_prefill", "fm_decode_step", "fm_prepare_mixer_params", "fm_calib_workspace_bytes",
+    "fm_calibrate_layer",
+)
+
+
+class FmError(RuntimeError):
+    def __init__(self, status: int, detail: str):
+        super().__init__(f"{STATUS.get(status, status)}: {detail}")
+        self.status = status
+
+
+class fm_shape(C.Structure):
+    _fields_ = [("d_model", C.c_int), ("d_inner", C.c_int), ("headdim", C.c_int),
+                ("d_state", C.c_int), ("ngroups", C.c_int), ("d_conv", C.c_int)]
+
+
+class fm_exp_layout(C.Structure):
+    _fields_ = [(n, C.c_int) for n in ("e_u", "e_w", "e_o", "e_x", "e_B", "e_C", "e_h", "e_y",
+                                       "e_D", "e_g", "size")]
+
+
+_P = C.c_void_p
+
+
+class fm_layer(C.Structure):
+    _fields_ = [("shape", fm_shape), ("rotate", C.c_int), ("mode", C.c_int),
+                ("w_in_q", _P), ("w_in_s", _P), ("w_out_q", _P), ("w_out_s", _P),
+                ("prenorm_w", _P), ("conv_wq", _P), ("conv_bq", _P), ("dt_bias", _P),
+                ("A_q", _P), ("D_q", _P), ("norm_w", _P), ("exps", _P), ("static_amax", _P)]
+
+
+_lib = None
+
+
+def load():
+    """Load the in-tree library (raises if it was not built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(SO_PATH):
+        raise ImportError(f"{SO_PATH} is missing: build it with "
+                          "`python -m quantized_state_space_mamba2_b200.build`")
+    L = C.CDLL(SO_PATH)
+    I, I64, SZ = C.c_int, C.c_int64, C.c_size_t
+    sp = C.POINTER(fm_shape)
+    lp = C.POINTER(fm_layer)
+    sig = {
+        "fm_status_string": (C.c_char_p, [I]),
+        "fm_last_error": (C.c_char_p, []),
+        "fm_sync_status": (I, [_P]),
+        "fm_version": (I, []),
+        "fm_exp_table_layout": (fm_exp_layout, [sp]),
+        "fm_hadamard_quant": (I, [_P, I64, I64, _P, I, I, _P, _P, _P, _P, _P]),
+        "fm_prepare_linear": (I, [_P, I64, I64, I, _P, _P, _P]),
+        "fm_w8a8_gemm": (I, [_P, _P, I64, _P, _P, I64, I64, _P, _P, _P, _P]),
+        "fm_in_proj": (I, [_P, _P, I64, _P, _P, sp, _P, _P, _P, _P, _P]),
+        "fm_conv1d_pot": (I, [_P, I, I, sp, _P, _P, _P, _P, _P, _P]),
+        "fm_ssm_scan_pot": (I, [_P, _P, I, I, sp, _P, _P, _P, _P, _P, _P, _P]),
+        "fm_gate_norm_quant": (I, [_P, _P, I64, sp, _P, _P, I, I, _P, _P, _P, _P, _P]),
+        "fm_eval_pwl": (I, [I, _P, I64, _P, _P]),
+        "fm_workspace_bytes": (SZ, [sp, I, I]),
+        "fm_mixer_prefill": (I, [lp, _P, I, I, I, _P, _P, _P, _P, SZ, _P]),
+        "fm_decode_step": (I, [lp, _P, I, I, _P, _P, _P, _P, SZ, _P]),
+        "fm_prepare_mixer_params": (I, [sp, _P, _P, _P, _P, _P, _P, _P, _P]),
+        "fm_calib_workspace_bytes": (SZ, [sp, I, I]),
+        "fm_calibrate_layer": (I, [lp, _P, _P, _P, _P, _P, I, I, I, _P, _P, SZ, _P]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(L, name)
+        f.restype = res
+        f.argtypes = args
+    _lib = L
+    return L
+
+
+def _p(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("libfastmamba takes CUDA tensors only")
+    if not t.is_contiguous():
+        raise ValueError("libfastmamba takes contiguous tensors only")
+    return C.c_void_p(t.data_ptr())
+
+
+def _s(stream):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return C.c_void_p(s.cuda_stream)
+
+
+def _check(status: int):
+    if status != 0:
+        raise FmError(status, load().fm_last_error().decode())
+
+
+def shape_struct(shape) -> fm_shape:
+    return fm_shape(shape.d_model, shape.d_inner, shape.headdim, shape.d_state, shape.ngroups,
+                    shape.d_conv)
+
+
+def exp_table_layout(shape) -> fm_exp_layout:
+    return load().fm_exp_table_layout(C.byref(shape_struct(shape)))
+
+
+def sync_status(stream=None):
+    _check(load().fm_sync_status(_s(stream)))
+
+
+def hadamard_quant(x, K, prenorm_w, rotate, mode, static_amax, q, s_x, amax_row=None, stream=None):
+    M = x.numel() // K
+    _check(load().fm_hadamard_quant(_p(x), M, K, _p(prenorm_w), rotate, mode, _p(static_amax),
+                                    _p(q), _p(s_x), _p(amax_row), _s(stream)))
+
+
+def prepare_linear(W, rotate, Wq, s_w, stream=None):
+    N, K = W.shape
+    _check(load().fm_prepare_linear(_p(W), N, K, rotate, _p(Wq), _p(s_w), _s(stream)))
+
+
+def w8a8_gemm(A, s_x, Wq, s_w, Y, residual=None, acc_out=None, stream=None):
+    M, K = A.shape
+    N = Wq.shape[0]
+    _check(load().fm_w8a8_gemm(_p(A), _p(s_x), M, _p(Wq), _p(s_w), N, K, _p(residual), _p(Y),
+                               _p(acc_out), _s(stream)))
+
+
+def in_proj(A, s_x, Wq, s_w, shape, exps, z, xbc, dt, stream=None):
+    sh = shape_struct(shape)
+    _check(load().fm_in_proj(_p(A), _p(s_x), A.shape[0], _p(Wq), _p(s_w), C.byref(sh), _p(exps),
+                             _p(z), _p(xbc), _p(dt), _s(stream)))
+
+
+def conv1d_pot(u, B, T, shape, wq, bq, exps, conv_state, out, stream=None):
+    sh = shape_struct(shape)
+    _check(load().fm_conv1d_pot(_p(u), B, T, C.byref(sh), _p(wq), _p(bq), _p(exps),
+                                _p(conv_state), _p(out), _s(stream)))
+
+
+def ssm_scan_pot(xbc, dt_raw, B, T, shape, dt_bias, A_q, D_q, exps, state, y, stream=None):
+    sh = shape_struct(shape)
+    _check(load().fm_ssm_scan_pot(_p(xbc), _p(dt_raw), B, T, C.byref(sh), _p(dt_bias), _p(A_q),
+                                  _p(D_q), _p(exps), _p(state), _p(y), _s(stream)))
+
+
+def gate_norm_quant(y, z, shape, exps, norm_w, rotate, mode, static_amax, q, s_x, amax_row=None,
+                    stream=None):
+    sh = shape_struct(shape)
+    M = y.numel() // shape.d_inner
+    _check(load().fm_gate_norm_quant(_p(y), _p(z), M, C.byref(sh), _p(exps), _p(norm_w), rotate,
+                                     mode, _p(static_amax), _p(q), _p(s_x), _p(amax_row),
+                                     _s(stream)))
+
+
+def eval_pwl(kind: int, inp, out, stream=None):
+    _check(load().fm_eval_pwl(kind, _p(inp), inp.numel(), _p(out), _s(stream)))
+
+
+def workspace_bytes(shape, B, T) -> int:
+    return load().fm_workspace_bytes(C.byref(shape_struct(shape)), B, T)
+
+
+def calib_workspace_bytes(shape, B, T) -> int:
+    return load().fm_calib_workspace_bytes(C.byref(shape_struct(shape)), B, T)
+
+
+def mixer_prefill(layer: fm_layer, x, B, T, residual, conv_state, ssm_state, out, ws,
+                  stream=None):
+    _check(load().fm_mixer_prefill(C.byref(layer), _p(x), B, T, residual, _p(conv_state),
+                                   _p(ssm_state), _p(out), _p(ws), ws.numel() * ws.element_size(),
+                                   _s(stream)))
+
+
+def decode_step(layer: fm_layer, x, B, residual, conv_state, ssm_state, out, ws, stream=None):
+    _check(load().fm_decode_step(C.byref(layer), _p(x), B, residual, _p(conv_state),
+                                 _p(ssm_state), _p(out), _p(ws), ws.numel() * ws.element_size(),
+                                 _s(stream)))
+
+
+def prepare_mixer_params(shape, conv_w, a_log, D, conv_wq, A_q, D_q, exps, stream=None):
+    sh = shape_struct(shape)
+    _check(load().fm_prepare_mixer_params(C.byref(sh), _p(conv_w), _p(a_log), _p(D),
+                                          _p(conv_wq), _p(A_q), _p(D_q), _p(exps), _s(stream)))
+
+
+def calibrate_layer(layer: fm_layer, conv_b, exps, conv_bq, static_amax, xcal, B, T, residual,
+                    out, ws, stream=None):
+    _check(load().fm_calibrate_layer(C.byref(layer), _p(conv_b), _p(exps), _p(conv_bq),
+                                     _p(static_amax), _p(xcal), B, T, residual, _p(out), _p(ws),
+                                     ws.numel() * ws.element_size(), _s(stream)))

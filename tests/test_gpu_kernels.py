@@ -1,0 +1,276 @@
+"""GPU parity of every kernel against the CPU oracle, through the C ABI.
+
+Integer codes, int32 accumulators and all fixed-point stages must be
+bit-exact; fp32 outputs computed from identical codes by the same IEEE
+operations in the same order must be bit-exact too.  Sizes span several
+tiles with ragged tails.
+"""
+import numpy as np
+import pytest
+
+import oracle as O
+from quantized_state_space_mamba2_b200 import synth as S
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+MAMBA130 = S.MAMBA2_130M
+
+
+@pytest.fixture(scope="module")
+def L():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from quantized_state_space_mamba2_b200 import build, lib
+    build.build()
+    lib.load()
+    return lib
+
+
+def dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def host(t):
+    torch.cuda.synchronize()
+    return t.cpu().numpy()
+
+
+# ------------------------------------------------------------------ nonlinear unit
+
+@pytest.mark.parametrize("kind,name,lo,hi", [(0, "pow2", -20 * 65536, 0), (1, "exp", -20 * 65536, 0),
+                                             (2, "softplus", -12 * 65536, 12 * 65536),
+                                             (3, "silu", -12 * 65536, 12 * 65536)])
+def test_pwl_exhaustive(L, kind, name, lo, hi):
+    x = np.arange(lo, hi + 1, dtype=np.int64)
+    out = torch.empty(x.size, dtype=torch.int64, device="cuda")
+    L.eval_pwl(kind, dev(x), out)
+    assert np.array_equal(host(out), O.eval_array(name, x))
+    L.sync_status()
+
+
+def test_pwl_extremes_and_to_q16(L):
+    x = np.array([-(2 ** 31) + 1, -(2 ** 31) + 1000, -1, 0, 1, 2 ** 31 - 1, 123456789, -98765432],
+                 np.int64)
+    out = torch.empty(x.size, dtype=torch.int64, device="cuda")
+    for kind, name in ((2, "softplus"), (3, "silu")):
+        L.eval_pwl(kind, dev(x), out)
+        assert np.array_equal(host(out), O.eval_array(name, x))
+    f = np.concatenate([S.normal(4096, 3.0, seed=1), S.normal(64, 1e5, seed=2),
+                        np.array([0.0, -0.0, 1e30, -1e30, np.inf, -np.inf, np.nan, 2.0 ** -20,
+                                  32767.99], np.float32)]).astype(np.float32)
+    bits = f.view(np.uint32).astype(np.int64)
+    out = torch.empty(bits.size, dtype=torch.int64, device="cuda")
+    L.eval_pwl(4, dev(bits), out)
+    assert np.array_equal(host(out), O.eval_array("to_q16", f))
+
+
+# ------------------------------------------------------------------ rotation + quantisation
+
+@pytest.mark.parametrize("M,K", [(1, 256), (7, 768), (300, 768), (33, 2560), (5, 5120)])
+@pytest.mark.parametrize("rotate", [1, 0])
+def test_hadamard_quant_dynamic(L, M, K, rotate):
+    x = S.activations(1, M, K, seed=M + K, n_outliers=8, outlier_scale=50.0)[0]
+    q = torch.empty((M, K), dtype=torch.int8, device="cuda")
+    sx = torch.empty(M, dtype=torch.float32, device="cuda")
+    am = torch.empty(M, dtype=torch.float32, device="cuda")
+    L.hadamard_quant(dev(x), K, None, rotate, 0, None, q, sx, am)
+    qr, sr, ar = O.hadamard_quant(x, None, rotate, O.DYNAMIC, want_amax=True)
+    assert np.array_equal(host(q), qr)
+    assert np.array_equal(host(sx), sr)
+    assert np.array_equal(host(am), ar)
+
+
+@pytest.mark.parametrize("K", [768, 2560])
+def test_hadamard_quant_prenorm_static(L, K):
+    M = 130
+    x = S.activations(1, M, K, seed=9, n_outliers=8, outlier_scale=50.0)[0]
+    w = (1.0 + S.normal(K, 0.1, seed=10)).astype(np.float32)
+    q = torch.empty((M, K), dtype=torch.int8, device="cuda")
+    sx = torch.empty(M, dtype=torch.float32, device="cuda")
+    L.hadamard_quant(dev(x), K, dev(w), 1, 0, None, q, sx)
+    qr, sr = O.hadamard_quant(x, w, 1, O.DYNAMIC)
+    assert np.array_equal(host(q), qr) and np.array_equal(host(sx), sr)
+    amax = np.float32(3.5)
+    L.hadamard_quant(dev(x), K, dev(w), 1, 1, dev(np.array([amax, 0, 0, 0], np.float32)), q, sx)
+    qr, sr = O.hadamard_quant(x, w, 1, O.STATIC, float(amax))
+    assert np.array_equal(host(q), qr) and np.array_equal(host(sx), sr)
+
+
+@pytest.mark.parametrize("N,K", [(3352, 768), (768, 1536), (40, 5120)])
+def test_prepare_linear(L, N, K):
+    W = S.normal((N, K), 0.02, seed=N)
+    wq = torch.empty((N, K), dtype=torch.int8, device="cuda")
+    sw = torch.empty(N, dtype=torch.float32, device="cuda")
+    for rot in (1, 0):
+        L.prepare_linear(dev(W), rot, wq, sw)
+        wr, sr = O.prepare_linear(W, rot)
+        assert np.array_equal(host(wq), wr) and np.array_equal(host(sw), sr)
+
+
+# ------------------------------------------------------------------ GEMM
+
+@pytest.mark.parametrize("M,N,K", [(1, 24, 128), (100, 136, 256), (256, 3352, 768),
+                                   (300, 768, 1536), (129, 257, 640), (2048, 768, 1536)])
+def test_w8a8_gemm(L, M, N, K):
+    A = S.uniform_ints((M, K), -127, 127, seed=M * 3 + K, dtype=np.int8)
+    W = S.uniform_ints((N, K), -127, 127, seed=N * 5 + K, dtype=np.int8)
+    sx = np.abs(S.normal(M, 0.01, seed=1)) + 1e-3
+    sw = np.abs(S.normal(N, 0.001, seed=2)) + 1e-4
+    res = S.normal((M, N), 1.0, seed=3)
+    Y = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    acc = torch.empty((M, N), dtype=torch.int32, device="cuda")
+    L.w8a8_gemm(dev(A), dev(sx), dev(W), dev(sw), Y, None, acc)
+    ref = A.astype(np.int64) @ W.astype(np.int64).T
+    assert np.array_equal(host(acc), ref)
+    assert np.array_equal(host(Y), O.dequant(ref.astype(np.int32), sx, sw))
+    Yr = dev(res)
+    L.w8a8_gemm(dev(A), dev(sx), dev(W), dev(sw), Yr, Yr, None)    # residual aliasing Y
+    assert np.array_equal(host(Yr), O.dequant(ref.astype(np.int32), sx, sw, residual=res))
+    L.sync_status()
+
+
+@pytest.mark.parametrize("M", [5, 256, 1000])
+def test_in_proj_split(L, M):
+    s = MAMBA130
+    A = S.uniform_ints((M, s.d_model), -127, 127, seed=M, dtype=np.int8)
+    W = S.uniform_ints((s.n_in, s.d_model), -127, 127, seed=M + 1, dtype=np.int8)
+    sx = np.abs(S.normal(M, 0.01, seed=4)) + 1e-3
+    sw = np.abs(S.normal(s.n_in, 1e-4, seed=5)) + 1e-5
+    e_u = S.uniform_ints(s.conv_ch, -5, -1, seed=6)
+    exps = np.zeros(L.exp_table_layout(s).size, np.int32)
+    exps[:s.conv_ch] = e_u
+    z = torch.empty((M, s.d_inner), dtype=torch.float32, device="cuda")
+    xbc = torch.empty((M, s.conv_ch), dtype=torch.int8, device="cuda")
+    dt = torch.empty((M, s.nheads), dtype=torch.float32, device="cuda")
+    L.in_proj(dev(A), dev(sx), dev(W), dev(sw), s, dev(exps), z, xbc, dt)
+    acc = (A.astype(np.int64) @ W.astype(np.int64).T).astype(np.int32)
+    zr, xr, dr = O.in_proj_epilogue(acc, sx, sw, s.d_inner, s.conv_ch, s.nheads, e_u)
+    assert np.array_equal(host(z), zr)
+    assert np.array_equal(host(xbc), xr)
+    assert np.array_equal(host(dt), dr)
+    assert np.abs(xr).max() == 127 and (xr == 0).mean() < 0.5   # codes exercise the range
+
+
+# ------------------------------------------------------------------ conv
+
+def _conv_case(s, seed):
+    cc = s.conv_ch
+    w = S.normal((cc, 4), 0.2, seed=seed)
+    b = S.normal(cc, 0.3, seed=seed + 1)
+    e_u = S.uniform_ints(cc, -5, -1, seed=seed + 2)
+    wq, bq, e_w = O.prepare_conv(w, b, e_u)
+    e_x = S.uniform_ints(s.nheads, -5, -3, seed=seed + 3)
+    e_B, e_C = -4, -3
+    e_o = np.concatenate([np.repeat(e_x, s.headdim), np.full(s.d_state, e_B),
+                          np.full(s.d_state, e_C)]).astype(np.int32)
+    return w, wq, bq, e_u, e_w, e_o
+
+
+@pytest.mark.parametrize("B,T", [(1, 1), (2, 5), (1, 37), (2, 300), (1, 2048)])
+@pytest.mark.parametrize("with_state", [False, True])
+def test_conv1d_pot(L, B, T, with_state):
+    s = MAMBA130
+    cc = s.conv_ch
+    _, wq, bq, e_u, e_w, e_o = _conv_case(s, 40)
+    exps = np.zeros(L.exp_table_layout(s).size, np.int32)
+    exps[:cc], exps[cc:2 * cc], exps[2 * cc:3 * cc] = e_u, e_w, e_o
+    u = S.uniform_ints((B, T, cc), -127, 127, seed=B * 1000 + T, dtype=np.int8)
+    st = S.uniform_ints((B, 3, cc), -127, 127, seed=7, dtype=np.int8) if with_state else None
+    out = torch.empty((B, T, cc), dtype=torch.int8, device="cuda")
+    st_d = dev(st) if with_state else None
+    L.conv1d_pot(dev(u), B, T, s, dev(wq), dev(bq), dev(exps), st_d, out)
+    st_r = st.copy() if with_state else None
+    ref = O.conv1d_pot(u, wq, bq, e_u, e_w, e_o, conv_state=st_r)
+    assert np.array_equal(host(out), ref)
+    if with_state:
+        assert np.array_equal(host(st_d), st_r)
+
+
+def test_prepare_mixer_params(L):
+    s = MAMBA130
+    P = S.layer_params(s, 11, conv_bias_std=0.1)
+    conv_wq = torch.empty((s.conv_ch, 4), dtype=torch.int8, device="cuda")
+    A_q = torch.empty(s.nheads, dtype=torch.int32, device="cuda")
+    D_q = torch.empty(s.nheads, dtype=torch.int32, device="cuda")
+    exps = torch.zeros(L.exp_table_layout(s).size, dtype=torch.int32, device="cuda")
+    D = (S.normal(s.nheads, 1.0, seed=12)).astype(np.float32)
+    L.prepare_mixer_params(s, dev(P["conv_w"]), dev(P["a_log"]), dev(D), conv_wq, A_q, D_q, exps)
+    wq, _, e_w = O.prepare_conv(P["conv_w"], P["conv_b"])
+    Aq, Dq, eD = O.prepare_ssm(P["a_log"], D)
+    X = L.exp_table_layout(s)
+    e = host(exps)
+    assert np.array_equal(host(conv_wq), wq)
+    assert np.array_equal(e[X.e_w:X.e_w + s.conv_ch], e_w)
+    assert np.array_equal(host(A_q), Aq) and np.array_equal(host(D_q), Dq)
+    assert np.array_equal(e[X.e_D:X.e_D + s.nheads], eD)
+
+
+# ------------------------------------------------------------------ scan
+
+def _scan_case(s, B, T, seed):
+    cc, nh = s.conv_ch, s.nheads
+    xbc = S.uniform_ints((B, T, cc), -127, 127, seed=seed, dtype=np.int8)
+    dt_raw = S.normal((B, T, nh), 2.0, seed=seed + 1)
+    P = S.layer_params(s, seed)
+    A_q, D_q, e_D = O.prepare_ssm(P["a_log"], P["D"])
+    e_x = S.uniform_ints(nh, -5, -3, seed=seed + 2)
+    e_B, e_C = -4, -3
+    e_h = (e_x + e_B - 15 + S.uniform_ints(nh, 2, 8, seed=seed + 3)).astype(np.int32)
+    e_y = (np.maximum(e_C + e_h, e_D + e_x) - S.uniform_ints(nh, 0, 6, seed=seed + 4)).astype(np.int32)
+    return xbc, dt_raw, P["dt_bias"], A_q, D_q, e_D, e_x, e_B, e_C, e_h, e_y
+
+
+def _exps_for_scan(L, s, e_x, e_B, e_C, e_h, e_y, e_D):
+    X = L.exp_table_layout(s)
+    nh = s.nheads
+    e = np.zeros(X.size, np.int32)
+    e[X.e_x:X.e_x + nh], e[X.e_B], e[X.e_C] = e_x, e_B, e_C
+    e[X.e_h:X.e_h + nh], e[X.e_y:X.e_y + nh], e[X.e_D:X.e_D + nh] = e_h, e_y, e_D
+    return e
+
+
+@pytest.mark.parametrize("B,T", [(1, 1), (2, 33), (1, 100), (1, 513)])
+@pytest.mark.parametrize("with_state", [False, True])
+def test_ssm_scan_pot(L, B, T, with_state):
+    s = MAMBA130
+    xbc, dt_raw, dt_bias, A_q, D_q, e_D, e_x, e_B, e_C, e_h, e_y = _scan_case(s, B, T, 60 + T)
+    exps = _exps_for_scan(L, s, e_x, e_B, e_C, e_h, e_y, e_D)
+    st = S.uniform_ints((B, s.nheads, s.headdim, s.d_state), -2 ** 26, 2 ** 26,
+                        seed=5) if with_state else None
+    y = torch.empty((B, T, s.d_inner), dtype=torch.int32, device="cuda")
+    st_d = dev(st) if with_state else None
+    L.ssm_scan_pot(dev(xbc), dev(dt_raw), B, T, s, dev(dt_bias), dev(A_q), dev(D_q), dev(exps),
+                   st_d, y)
+    st_r = st.copy() if with_state else None
+    yr = O.ssm_scan_pot(xbc, dt_raw, dt_bias, A_q, D_q, e_x, e_B, e_C, e_h, e_y, e_D,
+                        s.headdim, s.d_state, state=st_r)
+    assert np.array_equal(host(y), yr)
+    if with_state:
+        assert np.array_equal(host(st_d), st_r)
+
+
+# ------------------------------------------------------------------ gate + norm
+
+@pytest.mark.parametrize("M", [1, 77, 512])
+@pytest.mark.parametrize("mode", [0, 1])
+def test_gate_norm_quant(L, M, mode):
+    s = MAMBA130
+    y = S.uniform_ints((M, s.d_inner), -2 ** 29, 2 ** 29, seed=M, dtype=np.int32)
+    z = S.normal((M, s.d_inner), 3.0, seed=M + 1)
+    e_y = S.uniform_ints(s.nheads, -22, -18, seed=M + 2)
+    e_g = int(e_y.max()) - 16 + 14
+    w = (1.0 + S.normal(s.d_inner, 0.2, seed=9)).astype(np.float32)
+    X = L.exp_table_layout(s)
+    exps = np.zeros(X.size, np.int32)
+    exps[X.e_y:X.e_y + s.nheads] = e_y
+    exps[X.e_g] = e_g
+    amax = np.array([0.0, 2.5, 0, 0], np.float32)
+    q = torch.empty((M, s.d_inner), dtype=torch.int8, device="cuda")
+    sx = torch.empty(M, dtype=torch.float32, device="cuda")
+    am = torch.empty(M, dtype=torch.float32, device="cuda")
+    L.gate_norm_quant(dev(y), dev(z), s, dev(exps), dev(w), 1, mode, dev(amax)[1:], q, sx, am)
+    qr, sr, ar = O.gate_norm_quant(y, z, s.headdim, e_y, e_g, w, 1, mode, 2.5, want_amax=True)
+    assert np.array_equal(host(q), qr)
+    assert np.array_equal(host(sx), sr)
+    assert np.array_equal(host(am), ar)
