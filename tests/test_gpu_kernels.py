@@ -136,8 +136,8 @@ def test_in_proj_split(L, M):
     A = S.uniform_ints((M, s.d_model), -127, 127, seed=M, dtype=np.int8)
     W = S.uniform_ints((s.n_in, s.d_model), -127, 127, seed=M + 1, dtype=np.int8)
     sx = np.abs(S.normal(M, 0.01, seed=4)) + 1e-3
-    sw = np.abs(S.normal(s.n_in, 1e-4, seed=5)) + 1e-5
-    e_u = S.uniform_ints(s.conv_ch, -5, -1, seed=6)
+    sw = np.abs(S.normal(s.n_in, 5e-3, seed=5)) + 1e-4
+    e_u = S.uniform_ints(s.conv_ch, -6, -2, seed=6)
     exps = np.zeros(L.exp_table_layout(s).size, np.int32)
     exps[:s.conv_ch] = e_u
     z = torch.empty((M, s.d_inner), dtype=torch.float32, device="cuda")
