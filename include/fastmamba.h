@@ -238,6 +238,32 @@ fm_status fm_decode_step(const fm_layer *L, const float *x, int B, int residual,
                          int8_t *conv_state, int32_t *ssm_state, float *out, void *ws,
                          size_t ws_bytes, fm_stream stream);
 
+/* Decode step that allocates nothing and takes no workspace.
+ *
+ * The paper has no counterpart to this entry point: it exists for callers
+ * that cannot call cudaMalloc -- for example a plugin running inside a host
+ * framework that owns all device memory, or a serving loop whose memory
+ * budget is fixed at start-up and must never reach the allocator.  Its
+ * scratch (the intermediates fm_decode_step keeps in `ws`) lives in a
+ * file-scope device array of FM_NOALLOC_SCRATCH_BYTES that every GPU which
+ * loads the library holds until the process exits.
+ *   - Same arguments and results as fm_decode_step, minus ws/ws_bytes.
+ *   - Batches whose workspace (fm_workspace_bytes(shape, B, 1)) exceeds
+ *     FM_NOALLOC_SCRATCH_BYTES are rejected with FM_ERR_WORKSPACE before
+ *     any launch.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     before any stream capture.
+ *   - Every call on a device shares the one array and leaves the last
+ *     call's intermediates in it; nothing in it needs to start at zero (each
+ *     intermediate is written before it is read).  Calls that overlap on
+ *     the GPU (different streams, or different host threads) race on the
+ *     array: serialise them. */
+#define FM_NOALLOC_SCRATCH_BYTES (16u << 20)
+fm_status fm_decode_step_noalloc(const fm_layer *L, const float *x, int B, int residual,
+                                 int8_t *conv_state, int32_t *ssm_state, float *out,
+                                 fm_stream stream);
+
 /* Offline, per layer: quantise conv taps (e_w, wq) and the SSM parameters
  * (A_q, D_q, e_D) from fp32 device tensors: conv_w [cc, 4], a_log [nh], D [nh].
  * Writes the e_w and e_D regions of `exps`. */

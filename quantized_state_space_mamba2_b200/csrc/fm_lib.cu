@@ -597,6 +597,54 @@ extern "C" fm_status fm_decode_step(const fm_layer *L, const float *x, int B, in
   return fm_mixer_prefill(L, x, B, 1, residual, conv_state, ssm_state, out, ws, ws_bytes, stream);
 }
 
+// ------------------------------------------------------------------ allocation-free decode
+// Scratch for fm_decode_step_noalloc: a fixed device array instead of a
+// caller workspace, for callers that cannot allocate device memory.  Host
+// code only sees a stand-in for this symbol; its device address comes from
+// cudaGetSymbolAddress, once per device, with that device current.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[FM_NOALLOC_SCRATCH_BYTES];
+
+static fm_status noalloc_scratch_ptr(void **out) {
+  constexpr int kMaxDevices = 64;
+  static void *cache[kMaxDevices] = {nullptr};
+  static std::mutex mu;
+  int devid = 0;
+  FM_CHECK_CUDA(cudaGetDevice(&devid));
+  if (devid < 0 || devid >= kMaxDevices)
+    return fail(FM_ERR_UNSUPPORTED, "fm_decode_step_noalloc: device id %d out of range", devid);
+  std::lock_guard<std::mutex> lock(mu);
+  if (!cache[devid]) {
+    void *p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || !p)
+      return fail(FM_ERR_CUDA, "fm_decode_step_noalloc: cudaGetSymbolAddress: %s",
+                  cudaGetErrorString(e));
+    cache[devid] = p;
+  }
+  *out = cache[devid];
+  return FM_OK;
+}
+
+extern "C" fm_status fm_decode_step_noalloc(const fm_layer *L, const float *x, int B,
+                                            int residual, int8_t *conv_state, int32_t *ssm_state,
+                                            float *out, fm_stream stream) {
+  Dims d;
+  FM_TRY(check_layer(L, &d, __func__));
+  if (!conv_state || !ssm_state)
+    return fail(FM_ERR_INVALID_ARG, "fm_decode_step_noalloc: conv_state and ssm_state are required");
+  if (B < 0) return fail(FM_ERR_SHAPE, "fm_decode_step_noalloc: B must be >= 0");
+  if (B == 0) return FM_OK;
+  const size_t need = fm_workspace_bytes(&L->shape, B, 1);
+  if (need > (size_t)FM_NOALLOC_SCRATCH_BYTES)
+    return fail(FM_ERR_WORKSPACE,
+                "fm_decode_step_noalloc: batch %d needs %zu bytes of scratch, more than the "
+                "fixed %u-byte array (FM_NOALLOC_SCRATCH_BYTES); use fm_decode_step",
+                B, need, (unsigned)FM_NOALLOC_SCRATCH_BYTES);
+  void *ws = nullptr;
+  FM_TRY(noalloc_scratch_ptr(&ws));
+  return fm_decode_step(L, x, B, residual, conv_state, ssm_state, out, ws, need, stream);
+}
+
 // ------------------------------------------------------------------ offline preparation
 __global__ void k_prepare_mixer_params(const float *conv_w, const float *a_log, const float *D,
                                        int cc, int nh, int8_t *conv_wq, int32_t *A_q,

@@ -26,8 +26,9 @@ EXPORTS = (
     "fm_hadamard_quant", "fm_prepare_linear", "fm_w8a8_gemm", "fm_in_proj", "fm_conv1d_pot",
     "fm_ssm_scan_pot", "fm_gate_norm_quant", "fm_eval_pwl", "fm_workspace_bytes",
     "fm_mixer_prefill", "fm_decode_step", "fm_prepare_mixer_params", "fm_calib_workspace_bytes",
-    "fm_calibrate_layer",
+    "fm_calibrate_layer", "fm_decode_step_noalloc",
 )
+NOALLOC_SCRATCH_BYTES = 16 << 20  # FM_NOALLOC_SCRATCH_BYTES
 
 
 class FmError(RuntimeError):
@@ -88,6 +89,7 @@ def load():
         "fm_workspace_bytes": (SZ, [sp, I, I]),
         "fm_mixer_prefill": (I, [lp, _P, I, I, I, _P, _P, _P, _P, SZ, _P]),
         "fm_decode_step": (I, [lp, _P, I, I, _P, _P, _P, _P, SZ, _P]),
+        "fm_decode_step_noalloc": (I, [lp, _P, I, I, _P, _P, _P, _P]),
         "fm_prepare_mixer_params": (I, [sp, _P, _P, _P, _P, _P, _P, _P, _P]),
         "fm_calib_workspace_bytes": (SZ, [sp, I, I]),
         "fm_calibrate_layer": (I, [lp, _P, _P, _P, _P, _P, I, I, I, _P, _P, SZ, _P]),
@@ -201,6 +203,14 @@ def decode_step(layer: fm_layer, x, B, residual, conv_state, ssm_state, out, ws,
     _check(load().fm_decode_step(C.byref(layer), _p(x), B, residual, _p(conv_state),
                                  _p(ssm_state), _p(out), _p(ws), ws.numel() * ws.element_size(),
                                  _s(stream)))
+
+
+def decode_step_noalloc(layer: fm_layer, x, B, residual, conv_state, ssm_state, out,
+                        stream=None):
+    """fm_decode_step without a workspace: the library's fixed device scratch
+    array is used instead (for callers that cannot allocate device memory)."""
+    _check(load().fm_decode_step_noalloc(C.byref(layer), _p(x), B, residual, _p(conv_state),
+                                         _p(ssm_state), _p(out), _s(stream)))
 
 
 def prepare_mixer_params(shape, conv_w, a_log, D, conv_wq, A_q, D_q, exps, stream=None):
