@@ -47,6 +47,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--mode", default="dynamic", choices=["dynamic", "static"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--scan-tile", default=None,
+                    help="npt,pc,tch of the sequential scan kernel (a compiled variant)")
     return ap.parse_args()
 
 
@@ -179,7 +181,8 @@ def config_block(args, shape, n_layers, B, T):
             "d_model": shape.d_model, "d_inner": shape.d_inner, "nheads": shape.nheads,
             "d_state": shape.d_state, "act_quant": args.mode, "hadamard": True,
             "calibration": "16 seeded sequences x 512 tokens (GPU, stage by stage)",
-            "l2": "flushed between timed steps (512 MiB write)", "parallelism": f"replica x{args.gpus}"}
+            "l2": "flushed between timed steps (512 MiB write)", "parallelism": f"replica x{args.gpus}",
+            "scan_tile": args.scan_tile or "4,4,16"}
 
 
 # ---------------------------------------------------------------- the GPU arm
@@ -205,6 +208,8 @@ def main():
     if world > 1:
         dist.barrier()
     lib.load()
+    if args.scan_tile:
+        lib.set_scan_tile(*[int(v) for v in args.scan_tile.split(",")])
     dev = torch.device("cuda", local)
     shape, n_layers, B, T, n_out, scale = workload()
     mode = lib.FM_DYNAMIC if args.mode == "dynamic" else lib.FM_STATIC
@@ -233,7 +238,8 @@ def main():
     y = torch.empty((M, d.d_inner), dtype=torch.int32, device=dev)
     q_out = torch.empty((M, d.d_inner), dtype=torch.int8, device=dev)
     sx_out = torch.empty(M, dtype=torch.float32, device=dev)
-    launches_per_step = 6 * n_layers
+    sws = torch.empty(lib.scan_workspace_bytes(d, B, T), dtype=torch.uint8, device=dev)
+    launches_per_step = 7 * n_layers  # FWHT+quant, in_proj, conv, scan prep, scan, gate, out_proj
 
     def step(scan_events=None):
         src = x0
@@ -243,7 +249,7 @@ def main():
             lib.conv1d_pot(xbc, B, T, d, Ly.conv_wq, Ly.conv_bq, Ly.exps, None, xo)
             if scan_events is not None:
                 scan_events[i][0].record(stream)
-            lib.ssm_scan_pot(xo, dtr, B, T, d, Ly.dt_bias, Ly.A_q, Ly.D_q, Ly.exps, None, y)
+            lib.ssm_scan_pot(xo, dtr, B, T, d, Ly.dt_bias, Ly.A_q, Ly.D_q, Ly.exps, None, y, sws)
             if scan_events is not None:
                 scan_events[i][1].record(stream)
             lib.gate_norm_quant(y, z, d, Ly.exps, Ly.norm_w, 1, mode, Ly.static_amax[1:], q_out,
@@ -303,7 +309,8 @@ def main():
     achieved = cells * SCAN_OPS_PER_CELL / scan_avg_s / 1e12
     sm_mhz_peak = (peaks or {}).get("sm_max_mhz", 1965.0)
     alu_peak = 148 * 4 * 32 * sm_mhz_peak * 1e6 / 1e12
-    roofline = {"bound": "alu", "kernel": "k_ssm_scan_pot", "achieved": achieved,
+    roofline = {"bound": "alu", "kernel": "fm_ssm_scan_pot (k_scan_prep + k_scan_seq)",
+                "achieved": achieved,
                 "peak": alu_peak, "unit": "Tops/s (int32)", "frac": achieved / alu_peak,
                 "traffic": None,
                 "peak_basis": f"148 SMs x 4 SMSPs x 32 lanes x 1 int op/clk x {sm_mhz_peak:.0f} MHz",

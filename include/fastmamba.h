@@ -159,6 +159,18 @@ fm_status fm_conv1d_pot(const int8_t *u, int B, int T, const fm_shape *shape, co
 /* ------------------------------------------------------------------ */
 /* a5 - a8: selective scan in power-of-two fixed point                  */
 /* ------------------------------------------------------------------ */
+/* Tuning: selects the tile of the sequential scan kernel used by every later
+ * call in this process -- npt state columns per thread, pc channels per CTA,
+ * tch time steps per staged chunk.  Compiled variants: (4,4,16) (default),
+ * (4,2,16), (4,8,16), (8,4,16), (8,2,16), (8,8,16);
+ * anything else returns FM_ERR_INVALID_ARG.  All variants compute the same
+ * bits. */
+fm_status fm_set_scan_tile(int npt, int pc, int tch);
+
+/* Workspace bytes fm_ssm_scan_pot needs for B*T tokens (per-token dt/dA, the
+ * dt*x factor and the skip term, B and C widened). */
+size_t fm_scan_workspace_bytes(const fm_shape *shape, int B, int T);
+
 /* xbc [B, T, cc] int8 conv output (x | B | C), dt_raw [B, T, nh] fp32.
  * Per token and head (Q.16): dt_q = SoftPlus_pwl(to_q16(dt_raw + dt_bias)),
  * dA_q = 2^(-rshr(dt_q * A_q, 12)).  Per (b, h, p, n), t in order:
@@ -167,11 +179,12 @@ fm_status fm_conv1d_pot(const int8_t *u, int B, int T, const fm_shape *shape, co
  *   y[p] = satb(rshr(sum_n C[n] h, e_y - e_C - e_h) + rshr(D_q x[p], e_y - e_D - e_x), 32)
  *   dt_bias [nh] fp32, A_q [nh] int32 (exp(A_log) log2(e) 2^12), D_q [nh] int32.
  *   state [B, nh, hd, ds] int32 or NULL (zeros): initial state in, final out.
- *   y [B, T, d_inner] int32 at e_y. */
+ *   y [B, T, d_inner] int32 at e_y.
+ *   ws: device workspace of at least fm_scan_workspace_bytes(shape, B, T). */
 fm_status fm_ssm_scan_pot(const int8_t *xbc, const float *dt_raw, int B, int T,
                           const fm_shape *shape, const float *dt_bias, const int32_t *A_q,
                           const int32_t *D_q, const int32_t *exps, int32_t *state, int32_t *y,
-                          fm_stream stream);
+                          void *ws, size_t ws_bytes, fm_stream stream);
 
 /* ------------------------------------------------------------------ */
 /* a9 + a10: gate, gated RMSNorm, rotation, int8 quantisation           */

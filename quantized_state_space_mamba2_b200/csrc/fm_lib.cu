@@ -9,7 +9,9 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 #include <string>
 #include <type_traits>
@@ -21,6 +23,7 @@
 #include "k_gemm.cuh"
 #include "k_rows.cuh"
 #include "k_scan.cuh"
+#include "k_scan2.cuh"
 
 using namespace fm;
 
@@ -212,19 +215,12 @@ static fm_status launch_conv(const int8_t *u, int B, int T, int cc, const int8_t
                              int8_t *out, unsigned int *amax, cudaStream_t s) {
   if ((long long)B * T == 0) return FM_OK;
   const int groups = (cc / kConvCPT + kConvThreads - 1) / kConvThreads;
-  // token chunk: aim at >= ~4 CTAs per SM; one chunk when the sequence is short
-  int tch = 64;
-  const long long want = 4LL * 148;
-  while (tch > 8 && (long long)groups * ((T + tch - 1) / tch) * B < want) tch >>= 1;
-  if (T <= tch) tch = T;
-  const int chunks = (T + tch - 1) / tch;
-  if (chunks > 65535 || B > 65535) return fail(FM_ERR_SHAPE, "conv: T or B too large");
-  const int single = chunks == 1;
-  k_conv1d_pot<<<dim3(groups, chunks, B), kConvThreads, 0, s>>>(u, T, cc, tch, wq, bq, exps,
-                                                                 conv_state, single, out, amax);
+  if (T > 2147483647 || B > 65535) return fail(FM_ERR_SHAPE, "conv: T or B too large");
+  k_conv1d_pot<<<dim3(groups, (unsigned)T, B), kConvThreads, 0, s>>>(u, T, cc, wq, bq, exps,
+                                                                      conv_state, out, amax);
   FM_TRY(launched("k_conv1d_pot"));
-  if (conv_state && !single) {
-    const long long n = 3LL * B * cc;
+  if (conv_state) {
+    const long long n = (long long)B * cc;
     k_conv_state_update<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(u, B, T, cc, conv_state);
     FM_TRY(launched("k_conv_state_update"));
   }
@@ -265,6 +261,99 @@ static fm_status launch_scan(const ScanArgs &a, int B, cudaStream_t s) {
   dim3 grid(a.hd / kScanPC, a.nh, B);
   k_ssm_scan_pot<MODE><<<grid, kScanThreads, 0, s>>>(a);
   return launched("k_ssm_scan_pot");
+}
+
+// Sequential-scan tile (n per thread, p per CTA, steps per staged chunk);
+// process-wide, chosen with fm_set_scan_tile among the compiled variants.
+struct ScanTile {
+  int npt, pc, tch;
+};
+static const ScanTile kScanTiles[] = {{4, 4, 16}, {4, 2, 16}, {4, 8, 16},
+                                      {8, 4, 16}, {8, 2, 16}, {8, 8, 16}};
+static std::atomic<int> g_scan_tile{0};
+static ScanTile scan_tile() { return kScanTiles[g_scan_tile.load(std::memory_order_relaxed)]; }
+
+extern "C" fm_status fm_set_scan_tile(int npt, int pc, int tch) {
+  for (int i = 0; i < (int)(sizeof(kScanTiles) / sizeof(kScanTiles[0])); ++i)
+    if (kScanTiles[i].npt == npt && kScanTiles[i].pc == pc && kScanTiles[i].tch == tch) {
+      g_scan_tile.store(i, std::memory_order_relaxed);
+      return FM_OK;
+    }
+  return fail(FM_ERR_INVALID_ARG, "fm_set_scan_tile: (%d, %d, %d) is not a compiled variant", npt,
+              pc, tch);
+}
+
+template <int NPT, int PC, int TCH>
+static fm_status launch_seq(const ScanSeqArgs &a, int B, cudaStream_t s) {
+  using Sm = ScanSeqSmem<NPT, PC, TCH>;
+  constexpr int smem = (int)sizeof(Sm);
+  auto kern = k_scan_seq<NPT, PC, TCH>;
+  FM_CHECK_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+  dim3 grid(a.hd / PC, a.nh, B);
+  kern<<<grid, PC * (128 / NPT) + 32, smem, s>>>(a);
+  return launched("k_scan_seq");
+}
+
+struct ScanWs {
+  int32_t *dA;  // [B, nh, Tp]
+  int32_t *u;   // [B, nh, hd, Tp]
+  int32_t *dx;  // [B, nh, hd, Tp]
+  int32_t *bc;  // [B*T, 256]
+};
+
+// prep (parallel over token tiles and heads) + the sequential kernel
+static fm_status launch_scan_v2(const ScanArgs &a, int B, const ScanWs &w, cudaStream_t s) {
+  const long long M = (long long)B * a.T;
+  if (M == 0) return FM_OK;
+  if (B > 65535 || M > 2147483647LL) return fail(FM_ERR_SHAPE, "scan: B or B*T too large");
+  const long long Tp = scan_tpad(a.T);
+  ScanPrepArgs p;
+  p.xbc = a.xbc;
+  p.dt_raw = a.dt_raw;
+  p.T = a.T;
+  p.nh = a.nh;
+  p.hd = a.hd;
+  p.cc = a.cc;
+  p.di = a.di;
+  p.dt_bias = a.dt_bias;
+  p.A_q = a.A_q;
+  p.D_q = a.D_q;
+  p.e_x = a.e_x;
+  p.e_B = a.e_B;
+  p.e_h = a.e_h;
+  p.e_y = a.e_y;
+  p.e_D = a.e_D;
+  p.dA = w.dA;
+  p.u = w.u;
+  p.dx = w.dx;
+  p.bc = w.bc;
+  k_scan_prep<<<dim3((unsigned)(Tp / kPrepTT), a.nh, B), 256, 0, s>>>(p);
+  FM_TRY(launched("k_scan_prep"));
+  ScanSeqArgs q;
+  q.dA = w.dA;
+  q.u = w.u;
+  q.dx = w.dx;
+  q.bc = w.bc;
+  q.T = a.T;
+  q.nh = a.nh;
+  q.hd = a.hd;
+  q.di = a.di;
+  q.e_C = a.e_C;
+  q.e_h = a.e_h;
+  q.e_y = a.e_y;
+  q.state = a.state;
+  q.y = a.y;
+  const ScanTile t = scan_tile();
+#define FM_SEQ(N, P, C) \
+  if (t.npt == N && t.pc == P && t.tch == C) return launch_seq<N, P, C>(q, B, s);
+  FM_SEQ(4, 4, 16)
+  FM_SEQ(4, 2, 16)
+  FM_SEQ(4, 8, 16)
+  FM_SEQ(8, 4, 16)
+  FM_SEQ(8, 2, 16)
+  FM_SEQ(8, 8, 16)
+#undef FM_SEQ
+  return fail(FM_ERR_INVALID_ARG, "scan tile (%d, %d, %d) is not compiled", t.npt, t.pc, t.tch);
 }
 
 // ------------------------------------------------------------------ entry points
@@ -390,10 +479,43 @@ extern "C" fm_status fm_conv1d_pot(const int8_t *u, int B, int T, const fm_shape
   return launch_conv(u, B, T, d.cc, wq, bq, exps, conv_state, out, nullptr, (cudaStream_t)stream);
 }
 
+namespace {
+struct Carver {
+  uint8_t *base;
+  size_t off;
+  template <typename T>
+  T *take(size_t n) {
+    off = (off + 255) & ~size_t(255);
+    T *p = base ? reinterpret_cast<T *>(base + off) : nullptr;
+    off += n * sizeof(T);
+    return p;
+  }
+};
+
+ScanWs carve_scan(Carver &c, const Dims &d, int B, int T) {
+  const long long Tp = scan_tpad(T), M = (long long)B * T;
+  ScanWs w;
+  w.dA = c.take<int32_t>((long long)B * d.nh * Tp);
+  w.u = c.take<int32_t>((long long)B * d.di * Tp);
+  w.dx = c.take<int32_t>((long long)B * d.di * Tp);
+  w.bc = c.take<int32_t>(M * 256);
+  return w;
+}
+}  // namespace
+
+extern "C" size_t fm_scan_workspace_bytes(const fm_shape *shape, int B, int T) {
+  Dims d;
+  if (check_shape(shape, &d, __func__) != FM_OK || B < 0 || T < 0) return 0;
+  Carver c{nullptr, 0};
+  carve_scan(c, d, B, T);
+  return c.off + 256;
+}
+
 extern "C" fm_status fm_ssm_scan_pot(const int8_t *xbc, const float *dt_raw, int B, int T,
                                      const fm_shape *shape, const float *dt_bias,
                                      const int32_t *A_q, const int32_t *D_q, const int32_t *exps,
-                                     int32_t *state, int32_t *y, fm_stream stream) {
+                                     int32_t *state, int32_t *y, void *ws, size_t ws_bytes,
+                                     fm_stream stream) {
   Dims d;
   FM_TRY(check_shape(shape, &d, __func__));
   if (B < 0 || T < 0) return fail(FM_ERR_SHAPE, "fm_ssm_scan_pot: B, T must be >= 0");
@@ -406,9 +528,14 @@ extern "C" fm_status fm_ssm_scan_pot(const int8_t *xbc, const float *dt_raw, int
   NEED(exps);
   NEED(y);
   OPT(state);
+  const size_t need = fm_scan_workspace_bytes(shape, B, T);
+  if (!ws || ws_bytes < need || !aligned16(ws))
+    return fail(FM_ERR_WORKSPACE, "fm_ssm_scan_pot: workspace needs %zu bytes", need);
+  Carver c{reinterpret_cast<uint8_t *>(ws), 0};
+  const ScanWs w = carve_scan(c, d, B, T);
   const fm_exp_layout X = fm_exp_table_layout(shape);
-  return launch_scan<0>(scan_args(d, xbc, dt_raw, T, dt_bias, A_q, D_q, exps, X, state, y, nullptr),
-                        B, (cudaStream_t)stream);
+  return launch_scan_v2(scan_args(d, xbc, dt_raw, T, dt_bias, A_q, D_q, exps, X, state, y, nullptr),
+                        B, w, (cudaStream_t)stream);
 }
 
 static fm_status gate_impl(const int32_t *y, const float *z, long long M, const Dims &d,
@@ -475,18 +602,6 @@ extern "C" fm_status fm_eval_pwl(int kind, const int64_t *in, int64_t n, int64_t
 
 // ------------------------------------------------------------------ layers
 namespace {
-struct Carver {
-  uint8_t *base;
-  size_t off;
-  template <typename T>
-  T *take(size_t n) {
-    off = (off + 255) & ~size_t(255);
-    T *p = base ? reinterpret_cast<T *>(base + off) : nullptr;
-    off += n * sizeof(T);
-    return p;
-  }
-};
-
 struct MixerWs {
   int8_t *q_in;
   float *sx_in;
@@ -497,9 +612,11 @@ struct MixerWs {
   int32_t *y;
   int8_t *q_out;
   float *sx_out;
+  ScanWs scan;
 };
 
-MixerWs carve_mixer(Carver &c, const Dims &d, long long M) {
+MixerWs carve_mixer(Carver &c, const Dims &d, int B, int T) {
+  const long long M = (long long)B * T;
   MixerWs w;
   w.q_in = c.take<int8_t>(M * d.dm);
   w.sx_in = c.take<float>(M);
@@ -510,6 +627,7 @@ MixerWs carve_mixer(Carver &c, const Dims &d, long long M) {
   w.y = c.take<int32_t>(M * d.di);
   w.q_out = c.take<int8_t>(M * d.di);
   w.sx_out = c.take<float>(M);
+  w.scan = carve_scan(c, d, B, T);
   return w;
 }
 }  // namespace
@@ -518,7 +636,7 @@ extern "C" size_t fm_workspace_bytes(const fm_shape *shape, int B, int T) {
   Dims d;
   if (check_shape(shape, &d, __func__) != FM_OK || B < 0 || T < 0) return 0;
   Carver c{nullptr, 0};
-  carve_mixer(c, d, (long long)B * T);
+  carve_mixer(c, d, B, T);
   return c.off + 256;
 }
 
@@ -552,9 +670,9 @@ static fm_status mixer_impl(const fm_layer *L, const Dims &d, const float *x, in
                       w.dt, s));
   FM_TRY(launch_conv(w.xbc, B, T, d.cc, L->conv_wq, L->conv_bq, L->exps, conv_state, w.xo,
                      nullptr, s));
-  FM_TRY(launch_scan<0>(scan_args(d, w.xo, w.dt, T, L->dt_bias, L->A_q, L->D_q, L->exps, X,
+  FM_TRY(launch_scan_v2(scan_args(d, w.xo, w.dt, T, L->dt_bias, L->A_q, L->D_q, L->exps, X,
                                   ssm_state, w.y, nullptr),
-                        B, s));
+                        B, w.scan, s));
   FM_TRY(gate_impl(w.y, w.z, M, d, L->exps, X, L->norm_w, L->rotate, L->mode, amax_out, w.q_out,
                    w.sx_out, nullptr, nullptr, nullptr, s));
   return launch_gemm(w.q_out, M, L->w_out_q, d.dm, d.di,
@@ -585,7 +703,7 @@ extern "C" fm_status fm_mixer_prefill(const fm_layer *L, const float *x, int B, 
   }
   Carver c{reinterpret_cast<uint8_t *>(ws), 0};
   if (!aligned16(ws)) return fail(FM_ERR_ALIGNMENT, "fm_mixer_prefill: ws misaligned");
-  const MixerWs w = carve_mixer(c, d, (long long)B * T);
+  const MixerWs w = carve_mixer(c, d, B, T);
   return mixer_impl(L, d, x, B, T, residual, conv_state, ssm_state, out, w, (cudaStream_t)stream);
 }
 
@@ -783,9 +901,10 @@ struct CalibWs {
   unsigned int *silu_amax;// [cc]
   unsigned long long *stat;  // [nh]
 };
-CalibWs carve_calib(Carver &c, const Dims &d, long long M) {
+CalibWs carve_calib(Carver &c, const Dims &d, int B, int T) {
+  const long long M = (long long)B * T;
   CalibWs w;
-  w.m = carve_mixer(c, d, M);
+  w.m = carve_mixer(c, d, B, T);
   w.Y = c.take<float>(M * d.n_in);
   w.amax_row = c.take<float>(M);
   w.col_amax = c.take<unsigned int>(d.cc);
@@ -799,7 +918,7 @@ extern "C" size_t fm_calib_workspace_bytes(const fm_shape *shape, int B, int T) 
   Dims d;
   if (check_shape(shape, &d, __func__) != FM_OK || B < 0 || T < 0) return 0;
   Carver c{nullptr, 0};
-  carve_calib(c, d, (long long)B * T);
+  carve_calib(c, d, B, T);
   return c.off + 256;
 }
 
@@ -825,7 +944,7 @@ extern "C" fm_status fm_calibrate_layer(const fm_layer *L, const float *conv_b, 
   const long long M = (long long)B * T;
   const fm_exp_layout X = fm_exp_table_layout(&L->shape);
   Carver c{reinterpret_cast<uint8_t *>(ws), 0};
-  const CalibWs w = carve_calib(c, d, M);
+  const CalibWs w = carve_calib(c, d, B, T);
   const MixerWs &m = w.m;
 
   // 1. in_proj input: max |rotated (normed) input| -> static_amax[0]
@@ -873,9 +992,9 @@ extern "C" fm_status fm_calibrate_layer(const fm_layer *L, const float *conv_b, 
                         B, s));
   k_exp_y<<<1, 128, 0, s>>>(w.stat, d.nh, exps, X);
   FM_TRY(launched("k_exp_y"));
-  FM_TRY(launch_scan<0>(scan_args(d, m.xo, m.dt, T, L->dt_bias, L->A_q, L->D_q, exps, X, nullptr,
+  FM_TRY(launch_scan_v2(scan_args(d, m.xo, m.dt, T, L->dt_bias, L->A_q, L->D_q, exps, X, nullptr,
                                   m.y, nullptr),
-                        B, s));
+                        B, m.scan, s));
   // 6. gate exponent, then the out_proj input amax
   k_exp_gate<<<1, 32, 0, s>>>(nullptr, d.nh, exps, X);
   FM_TRY(launched("k_exp_gate"));

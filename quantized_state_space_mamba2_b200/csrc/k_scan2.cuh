@@ -1,0 +1,333 @@
+// k_scan2.cuh -- the selective scan in power-of-two fixed point, latency-hidden.
+//
+// Same arithmetic as k_scan.cuh (FastMamba, arXiv 2505.18975: power-of-two
+// fixed point for the SSM block, pith.science review "What carries the
+// argument"; shift-based e^Delta, verdict record citation [15]; SoftPlus via
+// Eq. (5) and the symmetry of citation [16]), split in two kernels:
+//
+//  k_scan_prep   parallel over (32-token tile, head, batch): per (token, head)
+//                the fixed-point dt_q and dA_q; per (token, channel p) the
+//                state input factor u = satb(rshr(dt_q x, s_h), 24) and the
+//                skip term rshr(D_q x, s_D); B and C widened to int32.  dA,
+//                u and the skip term are written head-major and time-
+//                contiguous ([B, nh, (hd,) Tp], Tp = T rounded up to 32) so a
+//                chunk of one head / channel is one contiguous run.
+//  k_scan_seq    the time-sequential part only.  One CTA per (batch, head,
+//                PC consecutive p); NPT consecutive n of one p per thread,
+//                state in registers.  One elected thread fetches each chunk
+//                of TCH steps with a handful of bulk copies (cp.async.bulk on
+//                an mbarrier) into a two-slot shared-memory ring one chunk
+//                ahead, so the other threads issue no load instructions and
+//                no global latency sits on the recurrence; the C.h partial
+//                sums of a chunk stay in registers and are added across the
+//                p's threads once per chunk through padded shared memory.
+// Per state cell and step the loop issues a 32x32->64 multiply-add and a
+// funnel shift (rounded decay), a multiply-add (+ u B), two min/max (clamp)
+// and a 32x32->64 multiply-accumulate (C h).
+#pragma once
+#include "fm_common.cuh"
+#include "k_gemm.cuh"  // mbarrier helpers (bounded waits)
+
+namespace fm {
+
+constexpr int kPrepTT = 32;  // tokens per prep tile; Tp is a multiple of it
+
+__host__ __device__ inline long long scan_tpad(long long T) {
+  return (T + kPrepTT - 1) / kPrepTT * kPrepTT;
+}
+
+struct ScanPrepArgs {
+  const int8_t *xbc;    // [B, T, cc] conv output: x | B | C
+  const float *dt_raw;  // [B, T, nh]
+  int T, nh, hd, cc, di;
+  const float *dt_bias;
+  const int32_t *A_q, *D_q;
+  const int32_t *e_x, *e_B, *e_h, *e_y, *e_D;
+  int32_t *dA;   // [B, nh, Tp]
+  int32_t *u;    // [B, nh, hd, Tp]
+  int32_t *dx;   // [B, nh, hd, Tp]
+  int32_t *bc;   // [B*T, 256]: B then C, int32
+};
+
+// grid = (Tp / 32, nh, B), block = 256; hd == 64
+__global__ void __launch_bounds__(256) k_scan_prep(ScanPrepArgs a) {
+  __shared__ int s_dtq[kPrepTT];
+  __shared__ __align__(16) int8_t sx[kPrepTT][64];
+  const int tid = threadIdx.x;
+  const int t0 = blockIdx.x * kPrepTT;
+  const int h = blockIdx.y;
+  const int b = blockIdx.z;
+  const int T = a.T, nh = a.nh, hd = a.hd;
+  const long long Tp = scan_tpad(T);
+  const int nt = min(kPrepTT, T - t0);
+  const long long rowbase = (long long)b * T;
+  if (tid < kPrepTT) {
+    int dtq = 0, dA = 0;
+    if (tid < nt) {
+      const float xf = __fadd_rn(a.dt_raw[(rowbase + t0 + tid) * nh + h], a.dt_bias[h]);
+      dtq = softplus_pwl(to_q16(xf));
+      dA = pow2_pwl(-rshr64((long long)dtq * a.A_q[h], 12));
+    }
+    s_dtq[tid] = dtq;
+    a.dA[((long long)b * nh + h) * Tp + t0 + tid] = dA;
+  }
+  {  // x tile: 32 tokens x 64 channels, 8 bytes per thread
+    const int tt = tid >> 3, k = tid & 7;
+    uint2 v = make_uint2(0u, 0u);
+    if (tt < nt)
+      v = *reinterpret_cast<const uint2 *>(a.xbc + (rowbase + t0 + tt) * a.cc + (long long)h * hd + k * 8);
+    *reinterpret_cast<uint2 *>(&sx[tt][k * 8]) = v;
+  }
+  __syncthreads();
+  {  // (u, skip) for channel p = tid / 4, tokens 8 * (tid % 4) .. + 8
+    const int p = tid >> 2, tb = (tid & 3) * 8;
+    const int s_h = a.e_h[h] - *a.e_B - a.e_x[h] + 16;
+    const int s_D = a.e_y[h] - a.e_D[h] - a.e_x[h];
+    const long long Dq = a.D_q[h];
+    int uv[8], dv[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const long long x = sx[tb + k][p];
+      uv[k] = (int)satb64(rshr64((long long)s_dtq[tb + k] * x, s_h), 24);
+      dv[k] = (int)satb64(rshr64(Dq * x, s_D), 32);
+    }
+    const long long off = (((long long)b * nh + h) * hd + p) * Tp + t0 + tb;
+    *reinterpret_cast<int4 *>(a.u + off) = make_int4(uv[0], uv[1], uv[2], uv[3]);
+    *reinterpret_cast<int4 *>(a.u + off + 4) = make_int4(uv[4], uv[5], uv[6], uv[7]);
+    *reinterpret_cast<int4 *>(a.dx + off) = make_int4(dv[0], dv[1], dv[2], dv[3]);
+    *reinterpret_cast<int4 *>(a.dx + off + 4) = make_int4(dv[4], dv[5], dv[6], dv[7]);
+  }
+  // widened B and C rows of these tokens: the CTAs of the tile share the work
+  for (int i = h * 256 + tid; i < nt * 64; i += nh * 256) {
+    const int tt = i >> 6, k = i & 63;  // 4 channels per item
+    const uint32_t w =
+        *reinterpret_cast<const uint32_t *>(a.xbc + (rowbase + t0 + tt) * a.cc + a.di + k * 4);
+    *reinterpret_cast<int4 *>(a.bc + (rowbase + t0 + tt) * 256 + k * 4) =
+        make_int4((int)(int8_t)(w & 0xFF), (int)(int8_t)((w >> 8) & 0xFF),
+                  (int)(int8_t)((w >> 16) & 0xFF), (int)(int8_t)(w >> 24));
+  }
+}
+
+struct ScanSeqArgs {
+  const int32_t *dA;  // [B, nh, Tp]
+  const int32_t *u;   // [B, nh, hd, Tp]
+  const int32_t *dx;  // [B, nh, hd, Tp]
+  const int32_t *bc;  // [B*T, 256]
+  int T, nh, hd, di;
+  const int32_t *e_C, *e_h, *e_y;
+  int32_t *state;     // [B, nh, hd, 128] or null
+  int32_t *y;         // [B*T, di]
+};
+
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes,
+                                         uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+constexpr int kScanSlots = 3;  // chunks in flight in the shared-memory ring
+
+template <int NPT, int PC, int TCH>
+struct ScanSeqSmem {
+  static constexpr int LPP = 128 / NPT;          // threads per p
+  static constexpr int NW = PC * LPP / 32;       // compute warps
+  // int64 per partial row: LPP + 1 (odd multiple of 16 B apart) keeps the
+  // per-row reads of a half-warp on distinct banks
+  static constexpr int PSTRIDE = LPP + 1;
+  struct Slot {
+    int32_t bc[TCH][256];
+    int32_t dA[TCH];
+    int32_t u[PC][TCH];
+    int32_t dx[PC][TCH];
+  };
+  Slot slot[kScanSlots];
+  long long part[NW][TCH * (32 / LPP)][PSTRIDE];
+  uint64_t full[kScanSlots];
+  uint64_t empty[kScanSlots];
+};
+
+template <int NPT>
+__device__ __forceinline__ void load_bc(const int32_t (*bc)[256], int tt, int n0, int (&Bv)[NPT],
+                                        int (&Cv)[NPT]) {
+  if constexpr (NPT >= 4) {
+#pragma unroll
+    for (int j = 0; j < NPT; j += 4) {
+      *reinterpret_cast<int4 *>(&Bv[j]) = *reinterpret_cast<const int4 *>(&bc[tt][n0 + j]);
+      *reinterpret_cast<int4 *>(&Cv[j]) = *reinterpret_cast<const int4 *>(&bc[tt][128 + n0 + j]);
+    }
+  } else {
+    *reinterpret_cast<int2 *>(&Bv[0]) = *reinterpret_cast<const int2 *>(&bc[tt][n0]);
+    *reinterpret_cast<int2 *>(&Cv[0]) = *reinterpret_cast<const int2 *>(&bc[tt][128 + n0]);
+  }
+}
+
+// TCH steps of the recurrence for this thread's NPT cells; the next step's
+// B / C are loaded while the current step computes.
+template <int NPT, int TCH, bool FULL>
+__device__ __forceinline__ void scan_chunk_steps(int (&hs)[NPT], long long (&part)[TCH],
+                                                 const int32_t (*bc)[256], const int32_t *dAv,
+                                                 const int32_t *uv, int n0, int nt) {
+  int Bn[NPT], Cn[NPT];
+  load_bc<NPT>(bc, 0, n0, Bn, Cn);
+#pragma unroll
+  for (int tg = 0; tg < TCH; tg += 4) {
+    const int4 dA4 = *reinterpret_cast<const int4 *>(dAv + tg);
+    const int4 u4 = *reinterpret_cast<const int4 *>(uv + tg);
+    const int dAs[4] = {dA4.x, dA4.y, dA4.z, dA4.w};
+    const int us[4] = {u4.x, u4.y, u4.z, u4.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int tt = tg + k;
+      if (!FULL && tt >= nt) {
+        part[tt] = 0;
+        continue;
+      }
+      int Bv[NPT], Cv[NPT];
+#pragma unroll
+      for (int j = 0; j < NPT; ++j) {
+        Bv[j] = Bn[j];
+        Cv[j] = Cn[j];
+      }
+      if (tt + 1 < TCH && (FULL || tt + 1 < nt)) load_bc<NPT>(bc, tt + 1, n0, Bn, Cn);
+      const long long dA = dAs[k];
+      const int u = us[k];
+      long long acc0 = 0, acc1 = 0;
+#pragma unroll
+      for (int j = 0; j < NPT; ++j) {
+        const int dec = (int)((dA * hs[j] + 32768LL) >> 16);
+        int hn = dec + u * Bv[j];
+        hn = min(max(hn, -(int)kHLim), (int)kHLim);
+        hs[j] = hn;
+        if (j & 1) acc1 += (long long)Cv[j] * hn;
+        else acc0 += (long long)Cv[j] * hn;
+      }
+      part[tt] = acc0 + acc1;
+    }
+  }
+}
+
+// Warps 0 .. NW-1 compute (each warp owns 32 / LPP channels p); warp NW is the
+// producer: one lane fetches chunk c into slot c % kScanSlots once every
+// compute warp has released the chunk that used the slot before (empty
+// barrier, one arrival per compute warp), and signals it through the slot's
+// transaction-count barrier.  Compute warps never wait for each other.
+template <int NPT, int PC, int TCH>
+__global__ void __launch_bounds__(PC *(128 / NPT) + 32) k_scan_seq(ScanSeqArgs a) {
+  constexpr int LPP = 128 / NPT;
+  constexpr int NW = PC * LPP / 32;
+  constexpr int PPW = 32 / LPP;  // channels per warp
+  static_assert(LPP <= 32 && 32 % LPP == 0, "a channel's threads stay inside one warp");
+  static_assert(TCH % 4 == 0 && kPrepTT % TCH == 0, "chunk must tile the padded time axis");
+  using Sm = ScanSeqSmem<NPT, PC, TCH>;
+  constexpr int PSTRIDE = Sm::PSTRIDE;
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  Sm &sm = *reinterpret_cast<Sm *>(smem_raw);
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane32 = tid & 31;
+  const int p0 = blockIdx.x * PC;
+  const int h = blockIdx.y;
+  const int b = blockIdx.z;
+  const int T = a.T, nh = a.nh, hd = a.hd, di = a.di;
+  const long long Tp = scan_tpad(T);
+  const long long rowbase = (long long)b * T;
+  const long long headrow = (long long)b * nh + h;
+  const int nchunks = (T + TCH - 1) / TCH;
+
+  if (tid == 0) {
+    for (int i = 0; i < kScanSlots; ++i) {
+      mbar_init(&sm.full[i], 1);
+      mbar_init(&sm.empty[i], NW);
+    }
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+
+  if (warp == NW) {  // ---------------- producer
+    if (lane32 == 0) {
+      for (int c = 0; c < nchunks; ++c) {
+        const int sl = c % kScanSlots;
+        if (c >= kScanSlots &&
+            !mbar_wait(&sm.empty[sl], (uint32_t)((c / kScanSlots) - 1) & 1u))
+          break;  // error word set; consumers time out on the full barrier
+        typename Sm::Slot &s = sm.slot[sl];
+        const int t0 = c * TCH;
+        const int nt = min(TCH, T - t0);
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        mbar_arrive_expect_tx(&sm.full[sl], (uint32_t)(nt * 1024 + TCH * 4 * (1 + 2 * PC)));
+        bulk_g2s(&s.bc[0][0], a.bc + (rowbase + t0) * 256, (uint32_t)(nt * 1024), &sm.full[sl]);
+        bulk_g2s(&s.dA[0], a.dA + headrow * Tp + t0, TCH * 4, &sm.full[sl]);
+#pragma unroll
+        for (int q = 0; q < PC; ++q) {
+          const long long off = (headrow * hd + p0 + q) * Tp + t0;
+          bulk_g2s(&s.u[q][0], a.u + off, TCH * 4, &sm.full[sl]);
+          bulk_g2s(&s.dx[q][0], a.dx + off, TCH * 4, &sm.full[sl]);
+        }
+      }
+    }
+    return;
+  }
+
+  // ---------------- compute warps
+  const int pp = tid / LPP;          // channel within the CTA
+  const int lane = tid % LPP;        // position within the channel
+  const int n0 = lane * NPT;
+  const int wp = pp % PPW;           // channel within the warp
+  const int s_y = a.e_y[h] - *a.e_C - a.e_h[h];
+  int hs[NPT];
+  int32_t *st = a.state ? a.state + (((headrow * hd) + p0 + pp) * 128 + n0) : nullptr;
+  if (st) {
+#pragma unroll
+    for (int j = 0; j < NPT; ++j) hs[j] = st[j];
+  } else {
+#pragma unroll
+    for (int j = 0; j < NPT; ++j) hs[j] = 0;
+  }
+  long long(*part)[PSTRIDE] = sm.part[warp];
+  for (int c = 0; c < nchunks; ++c) {
+    const int sl = c % kScanSlots;
+    if (!mbar_wait(&sm.full[sl], (uint32_t)(c / kScanSlots) & 1u)) return;  // error word set
+    const typename Sm::Slot &s = sm.slot[sl];
+    const int t0 = c * TCH;
+    const int nt = min(TCH, T - t0);
+    long long pr[TCH];
+    if (nt == TCH)
+      scan_chunk_steps<NPT, TCH, true>(hs, pr, s.bc, s.dA, s.u[pp], n0, nt);
+    else
+      scan_chunk_steps<NPT, TCH, false>(hs, pr, s.bc, s.dA, s.u[pp], n0, nt);
+    // partials of this warp: row (step, channel-in-warp), column = lane in channel
+#pragma unroll
+    for (int tt = 0; tt < TCH; ++tt) part[tt * PPW + wp][lane] = pr[tt];
+    __syncwarp();
+    // lane r sums row r (r < TCH * PPW) over the channel's LPP lanes, in two halves
+    constexpr int ROWS = TCH * PPW;
+    static_assert(ROWS <= 32 && 32 % ROWS == 0, "rows map onto the warp's lanes");
+    constexpr int SPLIT = 32 / ROWS;  // lanes sharing a row
+    constexpr int PER = LPP / SPLIT;
+    const int row = lane32 % ROWS, half = lane32 / ROWS;
+    long long sum0 = 0, sum1 = 0;
+#pragma unroll
+    for (int l = 0; l < PER; l += 2) {
+      sum0 += part[row][half * PER + l];
+      if (l + 1 < PER) sum1 += part[row][half * PER + l + 1];
+    }
+    long long sum = sum0 + sum1;
+#pragma unroll
+    for (int o = ROWS; o < 32; o <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    const int tt = row / PPW, q = warp * PPW + row % PPW;
+    if (half == 0 && tt < nt)
+      a.y[(rowbase + t0 + tt) * di + (long long)h * hd + p0 + q] =
+          (int)satb64(rshr64(sum, s_y) + s.dx[q][tt], 32);
+    __syncwarp();
+    if (lane32 == 0) mbar_arrive(&sm.empty[sl]);
+  }
+  if (st) {
+#pragma unroll
+    for (int j = 0; j < NPT; ++j) st[j] = hs[j];
+  }
+}
+
+}  // namespace fm

@@ -26,7 +26,8 @@ EXPORTS = (
     "fm_hadamard_quant", "fm_prepare_linear", "fm_w8a8_gemm", "fm_in_proj", "fm_conv1d_pot",
     "fm_ssm_scan_pot", "fm_gate_norm_quant", "fm_eval_pwl", "fm_workspace_bytes",
     "fm_mixer_prefill", "fm_decode_step", "fm_prepare_mixer_params", "fm_calib_workspace_bytes",
-    "fm_calibrate_layer", "fm_decode_step_noalloc",
+    "fm_calibrate_layer", "fm_decode_step_noalloc", "fm_scan_workspace_bytes",
+    "fm_set_scan_tile",
 )
 NOALLOC_SCRATCH_BYTES = 16 << 20  # FM_NOALLOC_SCRATCH_BYTES
 
@@ -83,7 +84,9 @@ def load():
         "fm_w8a8_gemm": (I, [_P, _P, I64, _P, _P, I64, I64, _P, _P, _P, _P]),
         "fm_in_proj": (I, [_P, _P, I64, _P, _P, sp, _P, _P, _P, _P, _P]),
         "fm_conv1d_pot": (I, [_P, I, I, sp, _P, _P, _P, _P, _P, _P]),
-        "fm_ssm_scan_pot": (I, [_P, _P, I, I, sp, _P, _P, _P, _P, _P, _P, _P]),
+        "fm_ssm_scan_pot": (I, [_P, _P, I, I, sp, _P, _P, _P, _P, _P, _P, _P, SZ, _P]),
+        "fm_scan_workspace_bytes": (SZ, [sp, I, I]),
+        "fm_set_scan_tile": (I, [I, I, I]),
         "fm_gate_norm_quant": (I, [_P, _P, I64, sp, _P, _P, I, I, _P, _P, _P, _P, _P]),
         "fm_eval_pwl": (I, [I, _P, I64, _P, _P]),
         "fm_workspace_bytes": (SZ, [sp, I, I]),
@@ -165,10 +168,22 @@ def conv1d_pot(u, B, T, shape, wq, bq, exps, conv_state, out, stream=None):
                                 _p(conv_state), _p(out), _s(stream)))
 
 
-def ssm_scan_pot(xbc, dt_raw, B, T, shape, dt_bias, A_q, D_q, exps, state, y, stream=None):
+SCAN_TILES = ((4, 4, 16), (4, 2, 16), (4, 8, 16), (8, 4, 16), (8, 2, 16), (8, 8, 16))
+
+
+def set_scan_tile(npt: int, pc: int, tch: int):
+    _check(load().fm_set_scan_tile(npt, pc, tch))
+
+
+def scan_workspace_bytes(shape, B, T) -> int:
+    return load().fm_scan_workspace_bytes(C.byref(shape_struct(shape)), B, T)
+
+
+def ssm_scan_pot(xbc, dt_raw, B, T, shape, dt_bias, A_q, D_q, exps, state, y, ws, stream=None):
     sh = shape_struct(shape)
     _check(load().fm_ssm_scan_pot(_p(xbc), _p(dt_raw), B, T, C.byref(sh), _p(dt_bias), _p(A_q),
-                                  _p(D_q), _p(exps), _p(state), _p(y), _s(stream)))
+                                  _p(D_q), _p(exps), _p(state), _p(y), _p(ws),
+                                  ws.numel() * ws.element_size(), _s(stream)))
 
 
 def gate_norm_quant(y, z, shape, exps, norm_w, rotate, mode, static_amax, q, s_x, amax_row=None,

@@ -49,8 +49,9 @@ def test_exp_layout_and_workspace(so):
     assert (L.e_u, L.e_w, L.e_o, L.e_x) == (0, cc, 2 * cc, 3 * cc)
     assert L.e_g == 3 * cc + 4 * nh + 2 and L.size == 3 * cc + 4 * nh + 3
     ws = lib.workspace_bytes(s, 1, 2048)
-    per_tok = s.d_model + 9 * s.d_inner + 2 * cc + 4 * nh + 8
-    assert per_tok * 2048 <= ws <= per_tok * 2048 + 256 * 12
+    # mixer intermediates + the scan's per-token dt/dA, (u, D x) and widened B, C
+    per_tok = s.d_model + 9 * s.d_inner + 2 * cc + 4 * nh + 8 + (4 * nh + 8 * s.d_inner + 1024)
+    assert per_tok * 2048 <= ws <= per_tok * 2048 + 256 * 16
     assert lib.calib_workspace_bytes(s, 16, 512) > lib.workspace_bytes(s, 16, 512)
     bad = S.MixerShape(d_model=300, d_inner=512, headdim=64, d_state=128)
     assert lib.workspace_bytes(bad, 1, 1) == 0

@@ -230,24 +230,43 @@ def _exps_for_scan(L, s, e_x, e_B, e_C, e_h, e_y, e_D):
     return e
 
 
-@pytest.mark.parametrize("B,T", [(1, 1), (2, 33), (1, 100), (1, 513)])
-@pytest.mark.parametrize("with_state", [False, True])
-def test_ssm_scan_pot(L, B, T, with_state):
-    s = MAMBA130
-    xbc, dt_raw, dt_bias, A_q, D_q, e_D, e_x, e_B, e_C, e_h, e_y = _scan_case(s, B, T, 60 + T)
+def _run_scan(L, s, B, T, with_state, seed):
+    xbc, dt_raw, dt_bias, A_q, D_q, e_D, e_x, e_B, e_C, e_h, e_y = _scan_case(s, B, T, seed)
     exps = _exps_for_scan(L, s, e_x, e_B, e_C, e_h, e_y, e_D)
     st = S.uniform_ints((B, s.nheads, s.headdim, s.d_state), -2 ** 26, 2 ** 26,
                         seed=5) if with_state else None
     y = torch.empty((B, T, s.d_inner), dtype=torch.int32, device="cuda")
     st_d = dev(st) if with_state else None
+    ws = torch.empty(L.scan_workspace_bytes(s, B, T), dtype=torch.uint8, device="cuda")
     L.ssm_scan_pot(dev(xbc), dev(dt_raw), B, T, s, dev(dt_bias), dev(A_q), dev(D_q), dev(exps),
-                   st_d, y)
+                   st_d, y, ws)
     st_r = st.copy() if with_state else None
     yr = O.ssm_scan_pot(xbc, dt_raw, dt_bias, A_q, D_q, e_x, e_B, e_C, e_h, e_y, e_D,
                         s.headdim, s.d_state, state=st_r)
     assert np.array_equal(host(y), yr)
     if with_state:
         assert np.array_equal(host(st_d), st_r)
+
+
+@pytest.mark.parametrize("B,T", [(1, 1), (2, 33), (1, 100), (1, 513)])
+@pytest.mark.parametrize("with_state", [False, True])
+def test_ssm_scan_pot(L, B, T, with_state):
+    _run_scan(L, MAMBA130, B, T, with_state, 60 + T)
+
+
+@pytest.mark.parametrize("tile", [(4, 2, 16), (4, 8, 16), (8, 4, 16), (8, 2, 16), (8, 8, 16)])
+def test_ssm_scan_tiles(L, tile):
+    """Every compiled tile of the sequential kernel computes the same bits
+    (ragged chunk tail, carried state, two heads' worth of CTAs per SM)."""
+    L.set_scan_tile(*tile)
+    try:
+        _run_scan(L, MAMBA130, 2, 45, True, 70)
+    finally:
+        L.set_scan_tile(4, 4, 16)
+
+
+def test_ssm_scan_2p7b_shape(L):
+    _run_scan(L, S.MAMBA2_2P7B, 1, 37, True, 80)
 
 
 # ------------------------------------------------------------------ gate + norm
