@@ -178,7 +178,8 @@ size_t fm_scan_workspace_bytes(const fm_shape *shape, int B, int T);
  *   h = clamp(rshr(dA_q h, 16) + u B[n], +-(2^30 - 1))
  *   y[p] = satb(rshr(sum_n C[n] h, e_y - e_C - e_h) + rshr(D_q x[p], e_y - e_D - e_x), 32)
  *   dt_bias [nh] fp32, A_q [nh] int32 (exp(A_log) log2(e) 2^12), D_q [nh] int32.
- *   state [B, nh, hd, ds] int32 or NULL (zeros): initial state in, final out.
+ *   state [B, nh, hd, ds] int32 or NULL (zeros): initial state in, final out;
+ *   values must lie within +-(2^30 - 1), the range the recurrence produces.
  *   y [B, T, d_inner] int32 at e_y.
  *   ws: device workspace of at least fm_scan_workspace_bytes(shape, B, T). */
 fm_status fm_ssm_scan_pot(const int8_t *xbc, const float *dt_raw, int B, int T,

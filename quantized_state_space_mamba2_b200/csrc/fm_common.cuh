@@ -76,25 +76,40 @@ __device__ __forceinline__ int pwl_S(int i) {
 }
 constexpr long long kLog2eQ15 = 47274;  // rint(2^15 * log2(e)) = rint(47274.23...)
 
-// 2^(w / 2^16) in Q.16 for w <= 0 (w > 0 is treated as 0); result in [0, 2^16]
-__device__ __forceinline__ int pow2_pwl(long long w) {
+// The unit below is written in 32-bit integer arithmetic only (32x32->64
+// multiplies are several times slower on this GPU); every split is exact.
+
+// 2^(w / 2^16) in Q.16 for w <= 0 (w > 0 is treated as 0); result in [0, 2^16].
+// With n = floor(w / 2^16) the integer part is a right shift by k = -n; k >= 32
+// (w < -31 * 2^16) gives 0.
+__device__ __forceinline__ int pow2_pwl32(int w) {
   if (w > 0) w = 0;
-  long long n = w >> 16;              // floor
-  int f = (int)(w - n * 65536);       // [0, 65535]
-  int i = f >> 13;
-  int r = f & 8191;
-  int m = pwl_P(i) + ((pwl_S(i) * r + 4096) >> 13);  // < 2^17
-  long long k = -n;
-  if (k >= 32) return 0;
+  if (w < -(31 << 16)) return 0;
+  const int n = w >> 16;               // floor, in [-31, 0]
+  const int f = w & 0xFFFF;
+  const int i = f >> 13;
+  const int r = f & 8191;
+  const int m = pwl_P(i) + ((pwl_S(i) * r + 4096) >> 13);  // < 2^17
+  const int k = -n;
   if (k == 0) return m;
-  int kk = (int)k;
-  return (int)(((long long)m + (1LL << (kk - 1))) >> kk);
+  return (m + (1 << (k - 1))) >> k;
 }
 
-// e^(x / 2^16) in Q.16 for x <= 0
+__device__ __forceinline__ int pow2_pwl(long long w) {
+  return w < -(31LL << 16) ? 0 : pow2_pwl32((int)(w > 0 ? 0 : w));
+}
+
+// e^(x / 2^16) in Q.16 for x <= 0 (x > 0 is treated as 0):
+// 2^rshr(x log2e_Q15, 15).  For |x| >= 2^21 the exponent is below -31 * 2^16
+// (result 0); otherwise |x| = ah 2^15 + al and
+// rshr(-|x| L, 15) = -ah L + ((2^14 - al L) >> 15), all within int32.
 __device__ __forceinline__ int exp_pwl(long long x) {
-  if (x > 0) x = 0;
-  return pow2_pwl(rshr64(x * kLog2eQ15, 15));
+  if (x >= 0) return 65536;
+  if (x <= -(1LL << 21)) return 0;
+  const int ax = (int)(-x);
+  const int ah = ax >> 15, al = ax & 0x7FFF;
+  const int w = -ah * (int)kLog2eQ15 + ((16384 - al * (int)kLog2eQ15) >> 15);
+  return pow2_pwl32(w);
 }
 
 // SoftPlus: x <= 0 -> e^x; x > 0 -> x + e^-x; clamped to 2^31 - 1
@@ -103,24 +118,94 @@ __device__ __forceinline__ int softplus_pwl(int v) {
   return r > 2147483647LL ? 2147483647 : (int)r;
 }
 
-// SiLU(x / 2^16) in Q.16: sigma from E = e^-|x|; x >= 0: floor(2^32 / (2^16 + E)),
-// x < 0: floor(E 2^16 / (2^16 + E)); result rshr(x * sigma, 16).
-__device__ __forceinline__ long long silu_pwl(int x) {
-  long long ax = x < 0 ? -(long long)x : (long long)x;
-  unsigned E = (unsigned)exp_pwl(-ax);
-  unsigned d = 65536u + E;  // [2^16, 2^17]
+// SiLU(x / 2^16) in Q.16 for x in +-(2^31 - 1): sigma from E = e^-|x|;
+// x >= 0: floor(2^32 / (2^16 + E)), x < 0: floor(E 2^16 / (2^16 + E));
+// result rshr(x sigma, 16) = xh sigma + ((xl sigma + 2^15) >> 16) with
+// x = xh 2^16 + xl, xl in [0, 2^16) (both products fit 32 bits).
+__device__ __forceinline__ int silu_pwl32(int x) {
+  const unsigned E = (unsigned)exp_pwl(x < 0 ? (long long)x : -(long long)x);
+  const unsigned d = 65536u + E;  // [2^16, 2^17]
   unsigned sig;
   if (x >= 0) {
-    sig = 0xFFFFFFFFu / d;           // floor((2^32 - 1) / d)
+    sig = 0xFFFFFFFFu / d;                // floor((2^32 - 1) / d)
     if ((d & (d - 1u)) == 0u) sig += 1u;  // d divides 2^32
   } else if (E >= 65536u) {
-    sig = 32768u;                    // 2^32 / 2^17
+    sig = 32768u;                         // 2^32 / 2^17
   } else {
     sig = (E << 16) / d;
   }
-  long long prod = (long long)x * (long long)sig;
-  return (prod + 32768LL) >> 16;
+  const int xh = x >> 16;
+  const unsigned xl = (unsigned)x & 0xFFFFu;
+  return xh * (int)sig + (int)((xl * sig + 32768u) >> 16);
 }
+
+__device__ __forceinline__ long long silu_pwl(int x) { return silu_pwl32(x); }
+
+// ---------------------------------------------------------------- fast forms
+// The same functions for element-wise kernels: the 8 (P_i, S_i) pairs are read
+// from a shared-memory table packed as P | S << 17 (per-lane indices would
+// serialise on the constant cache), and the SiLU division uses a reciprocal
+// estimate with an exact integer correction.  Bit-identical to the forms above.
+__device__ __forceinline__ void pwl_table_init(int *tab) {
+  if (threadIdx.x < 8 && threadIdx.y == 0) tab[threadIdx.x] = pwl_P(threadIdx.x) | (pwl_S(threadIdx.x) << 17);
+}
+
+__device__ __forceinline__ int pow2_pwl32_t(int w, const int *tab) {
+  if (w > 0) w = 0;
+  if (w < -(31 << 16)) return 0;
+  const int k = -(w >> 16);
+  const int f = w & 0xFFFF;
+  const int e = tab[f >> 13];
+  const int m = (e & 0x1FFFF) + ((((unsigned)e >> 17) * (f & 8191) + 4096) >> 13);
+  if (k == 0) return m;
+  return (m + (1 << (k - 1))) >> k;
+}
+
+__device__ __forceinline__ int exp_pwl_t(int x, const int *tab) {  // x <= 0 in int32
+  if (x >= 0) return 65536;
+  if (x <= -(1 << 21)) return 0;
+  const int ax = -x;
+  const int ah = ax >> 15, al = ax & 0x7FFF;
+  return pow2_pwl32_t(-ah * (int)kLog2eQ15 + ((16384 - al * (int)kLog2eQ15) >> 15), tab);
+}
+
+// floor(num / d) for d in [2^16, 2^17] and num in [0, 2^32]; numf = num as a
+// float (exact: num is 2^32 or a multiple of 2^16 below it), num_mod = num
+// mod 2^32.  The float estimate is within one of the quotient; the remainder,
+// exact modulo 2^32, lies in (-2d, 2d) and fixes it.
+__device__ __forceinline__ unsigned div_q16(float numf, unsigned num_mod, unsigned d) {
+  float rd;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(rd) : "f"((float)d));
+  unsigned q = (unsigned)__fmul_rz(numf, rd);
+  unsigned rem = num_mod - q * d;
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    if ((int)rem < 0) {
+      q -= 1u;
+      rem += d;
+    } else if (rem >= d) {
+      q += 1u;
+      rem -= d;
+    }
+  }
+  return q;
+}
+
+__device__ __forceinline__ int silu_pwl_t(int x, const int *tab) {
+  const unsigned E = (unsigned)exp_pwl_t(x < 0 ? x : -x, tab);
+  const unsigned d = 65536u + E;
+  // x >= 0: num = 2^32; x < 0: num = E 2^16 (= 2^32 when E = 2^16)
+  const float numf = x >= 0 ? 4294967296.0f : (float)E * 65536.0f;
+  const unsigned nmod = x >= 0 ? 0u : (E << 16);
+  const unsigned sig = div_q16(numf, nmod, d);
+  const int xh = x >> 16;
+  const unsigned xl = (unsigned)x & 0xFFFFu;
+  return xh * (int)sig + (int)((xl * sig + 32768u) >> 16);
+}
+
+// rshr(v, k) for int32 v and k in [1, 31] without overflow: floor(v / 2^k) +
+// the bit below (round half up)
+__device__ __forceinline__ int rshr32(int v, int k) { return (v >> k) + ((v >> (k - 1)) & 1); }
 
 // ---------------------------------------------------------------- PoT exponent
 // smallest integer e with a <= Q 2^e (exact), a <= 0 -> -30

@@ -182,29 +182,39 @@ static fm_status make_tmap(CUtensorMap *tm, const int8_t *ptr, long long rows, l
 }
 
 // ------------------------------------------------------------------ launches
-constexpr int kBN = 128;
-constexpr int kStages = 6;
+template <int BN, int STAGES>
+static fm_status launch_gemm_t(const CUtensorMap &ta, const CUtensorMap &tb, long long M,
+                               long long N, long long K, const GemmEpilogue &ep, cudaStream_t s) {
+  constexpr int smem = gemm_smem_bytes(BN, STAGES);
+  auto kern = k_gemm_i8_tc<BN, STAGES>;
+  FM_CHECK_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+  dim3 grid((unsigned)((N + BN - 1) / BN), (unsigned)((M + kGemmBM - 1) / kGemmBM));
+  kern<<<grid, kGemmThreads, smem, s>>>(ta, tb, (int)(K / kGemmBK), ep);
+  return launched("k_gemm_i8_tc");
+}
 
+// 128 x 128 tiles with a 3-stage ring (96 KB: two CTAs per SM, one's
+// epilogue overlapping the other's main loop); 128 x 64 tiles when the 128-wide
+// grid would leave SMs idle (small N, e.g. out_proj).
 static fm_status launch_gemm(const int8_t *A, long long M, const int8_t *W, long long N,
                              long long K, const GemmEpilogue &ep, cudaStream_t s) {
   if (K % kGemmBK) return fail(FM_ERR_SHAPE, "gemm: K=%lld is not a multiple of 128", K);
-  if ((N + kBN - 1) / kBN > 2147483647LL || (M + kGemmBM - 1) / kGemmBM > 65535)
+  if ((M + kGemmBM - 1) / kGemmBM > 65535 || (N + 63) / 64 > 2147483647LL)
     return fail(FM_ERR_SHAPE, "gemm: M=%lld or N=%lld too large", M, N);
+  const long long tiles128 = ((N + 127) / 128) * ((M + kGemmBM - 1) / kGemmBM);
+  const bool narrow = tiles128 < 2 * 148;
   CUtensorMap ta, tb;
   FM_TRY(make_tmap(&ta, A, M, K, kGemmBM));
-  FM_TRY(make_tmap(&tb, W, N, K, kBN));
-  constexpr int smem = gemm_smem_bytes(kBN, kStages);
-  auto kern = k_gemm_i8_tc<kBN, kStages>;
-  FM_CHECK_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
-  dim3 grid((unsigned)((N + kBN - 1) / kBN), (unsigned)((M + kGemmBM - 1) / kGemmBM));
-  kern<<<grid, kGemmThreads, smem, s>>>(ta, tb, (int)(K / kGemmBK), ep);
-  return launched("k_gemm_i8_tc");
+  FM_TRY(make_tmap(&tb, W, N, K, narrow ? 64 : 128));
+  if (narrow) return launch_gemm_t<64, 4>(ta, tb, M, N, K, ep, s);
+  return launch_gemm_t<128, 3>(ta, tb, M, N, K, ep, s);
 }
 
 static fm_status launch_hadamard_quant(const float *x, long long M, int K, const float *prenorm_w,
                                        int rotate, int mode, const float *static_amax, int8_t *q,
                                        float *s_x, float *amax_row, cudaStream_t s) {
   if (M <= 0) return FM_OK;
+
   k_hadamard_quant<<<(unsigned)M, 32 * (K / 256), 0, s>>>(x, K, prenorm_w, rotate, mode,
                                                            static_amax, q, s_x, amax_row);
   return launched("k_hadamard_quant");
@@ -299,6 +309,7 @@ struct ScanWs {
   int32_t *u;   // [B, nh, hd, Tp]
   int32_t *dx;  // [B, nh, hd, Tp]
   int32_t *bc;  // [B*T, 256]
+  long long *bound;  // [B, nh, Tp/16, hd]
 };
 
 // prep (parallel over token tiles and heads) + the sequential kernel
@@ -327,6 +338,7 @@ static fm_status launch_scan_v2(const ScanArgs &a, int B, const ScanWs &w, cudaS
   p.u = w.u;
   p.dx = w.dx;
   p.bc = w.bc;
+  p.bound = w.bound;
   k_scan_prep<<<dim3((unsigned)(Tp / kPrepTT), a.nh, B), 256, 0, s>>>(p);
   FM_TRY(launched("k_scan_prep"));
   ScanSeqArgs q;
@@ -334,6 +346,7 @@ static fm_status launch_scan_v2(const ScanArgs &a, int B, const ScanWs &w, cudaS
   q.u = w.u;
   q.dx = w.dx;
   q.bc = w.bc;
+  q.bound = w.bound;
   q.T = a.T;
   q.nh = a.nh;
   q.hd = a.hd;
@@ -499,6 +512,7 @@ ScanWs carve_scan(Carver &c, const Dims &d, int B, int T) {
   w.u = c.take<int32_t>((long long)B * d.di * Tp);
   w.dx = c.take<int32_t>((long long)B * d.di * Tp);
   w.bc = c.take<int32_t>(M * 256);
+  w.bound = c.take<long long>((long long)B * d.di * (Tp / 16));
   return w;
 }
 }  // namespace

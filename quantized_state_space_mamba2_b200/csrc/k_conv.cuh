@@ -34,6 +34,9 @@ __global__ void __launch_bounds__(kConvThreads) k_conv1d_pot(
     const int8_t *__restrict__ u, int T, int cc, const int8_t *__restrict__ wq,
     const int32_t *__restrict__ bq, const int32_t *__restrict__ exps,
     const int8_t *__restrict__ conv_state, int8_t *__restrict__ out, unsigned int *amax) {
+  __shared__ int tab[8];
+  pwl_table_init(tab);
+  __syncthreads();
   const int c0 = (blockIdx.x * kConvThreads + threadIdx.x) * kConvCPT;
   if (c0 >= cc) return;
   const int t = blockIdx.y;
@@ -65,12 +68,31 @@ __global__ void __launch_bounds__(kConvThreads) k_conv1d_pot(
   for (int j = 0; j < kConvCPT; ++j) {
     int w[4];
     unpack4(wr[j], w);
-    const long long acc = (long long)bs[j] + w[0] * win[0][j] + w[1] * win[1][j] +
-                          w[2] * win[2][j] + w[3] * win[3][j];
-    const int x16 = (int)satb64(rshr64(acc, s_in[j]), 32);
-    const long long sv = silu_pwl(x16);
+    const int dot = w[0] * win[0][j] + w[1] * win[1][j] + w[2] * win[2][j] + w[3] * win[3][j];
+    int x16;
+    const int si = s_in[j];
+    if (bs[j] >= -(1 << 29) && bs[j] <= (1 << 29) && si >= -30 && si <= 29) {
+      // 32-bit path: |acc| < 2^30 (the taps add at most 4 * 127^2)
+      const int acc = bs[j] + dot;
+      if (si > 0) {
+        x16 = rshr32(acc, si);
+      } else {
+        const int k = -si, lim = 0x7FFFFFFF >> k;
+        x16 = acc > lim ? 2147483647 : (acc < -lim ? -2147483647 : acc * (1 << k));
+      }
+    } else {
+      x16 = (int)satb64(rshr64((long long)bs[j] + dot, si), 32);
+    }
+    const int sv = silu_pwl_t(x16, tab);
     if (amax) atomicMax(amax + c0 + j, (unsigned int)(sv < 0 ? -sv : sv));
-    packed |= ((uint32_t)((int)satb64(rshr64(sv, s_out[j]), 8) & 0xFF)) << (8 * j);
+    const int so = s_out[j];
+    int code;
+    if (so >= 1 && so <= 31) {
+      code = min(max(rshr32(sv, so), -127), 127);
+    } else {
+      code = (int)satb64(rshr64(sv, so), 8);
+    }
+    packed |= ((uint32_t)(code & 0xFF)) << (8 * j);
   }
   *reinterpret_cast<uint32_t *>(out + ((long long)b * T + t) * cc + c0) = packed;
 }

@@ -154,7 +154,8 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
 }
 
 __host__ __device__ constexpr int gemm_smem_bytes(int BN, int stages) {
-  return stages * (kGemmBM + BN) * kGemmBK + 1024 /*align slack*/ + 256 /*barriers*/;
+  return stages * (kGemmBM + BN) * kGemmBK + 1024 /*align slack*/ + 256 /*barriers*/ +
+         2 * BN * 4 /*staged column scales*/;
 }
 
 // ------------------------------------------------------------ epilogue
@@ -162,36 +163,45 @@ __device__ __forceinline__ float pow2f(int e) {  // exact 2^e for e in [-126, 12
   return __int_as_float((127 + e) << 23);
 }
 
-__device__ __forceinline__ void gemm_store_chunk(const GemmEpilogue &ep, long long row,
-                                                 long long col0, const uint32_t (&r)[32]) {
+// One 32-column chunk of one output row.  colw / cole: this chunk's column
+// scales s_w and (split mode) the PoT factors 2^-e_u staged in shared memory.
+__device__ __forceinline__ void gemm_store_chunk(const GemmEpilogue &ep, long long row, float sx,
+                                                 long long col0, uint32_t (&r)[32],
+                                                 const float *colw, const float *cole) {
   if (row >= ep.M) return;
-  const float sx = ep.s_x[row];
   const bool full = col0 + 32 <= ep.N;
   if (ep.acc_out) {
     int32_t *dst = ep.acc_out + row * ep.N + col0;
     for (int j = 0; j < 32; ++j)
       if (col0 + j < ep.N) dst[j] = (int32_t)r[j];
   }
-  float y[32];
+  // dequantise in place (the accumulator registers become the fp32 values)
+  float(&y)[32] = reinterpret_cast<float(&)[32]>(r);
 #pragma unroll
-  for (int j = 0; j < 32; ++j) {
-    const long long c = col0 + j;
-    const float sw = c < ep.N ? ep.s_w[c] : 0.0f;
-    y[j] = __fmul_rn(__fmul_rn(__int2float_rn((int)r[j]), sx), sw);
+  for (int j = 0; j < 32; j += 4) {
+    const float4 sw = *reinterpret_cast<const float4 *>(colw + j);
+    y[j] = __fmul_rn(__fmul_rn(__int2float_rn((int)r[j]), sx), sw.x);
+    y[j + 1] = __fmul_rn(__fmul_rn(__int2float_rn((int)r[j + 1]), sx), sw.y);
+    y[j + 2] = __fmul_rn(__fmul_rn(__int2float_rn((int)r[j + 2]), sx), sw.z);
+    y[j + 3] = __fmul_rn(__fmul_rn(__int2float_rn((int)r[j + 3]), sx), sw.w);
   }
   if (ep.mode == 0) {
     float *dst = ep.Y + row * ep.N + col0;
     const float *res = ep.residual ? ep.residual + row * ep.N + col0 : nullptr;
     if (full && ((ep.N & 3) == 0)) {
+      float4 rv[8];
+      if (res) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) rv[j] = *reinterpret_cast<const float4 *>(res + 4 * j);
+      }
 #pragma unroll
       for (int j = 0; j < 32; j += 4) {
         float4 o = make_float4(y[j], y[j + 1], y[j + 2], y[j + 3]);
         if (res) {
-          const float4 rv = *reinterpret_cast<const float4 *>(res + j);
-          o.x = __fadd_rn(rv.x, o.x);
-          o.y = __fadd_rn(rv.y, o.y);
-          o.z = __fadd_rn(rv.z, o.z);
-          o.w = __fadd_rn(rv.w, o.w);
+          o.x = __fadd_rn(rv[j / 4].x, o.x);
+          o.y = __fadd_rn(rv[j / 4].y, o.y);
+          o.z = __fadd_rn(rv[j / 4].z, o.z);
+          o.w = __fadd_rn(rv[j / 4].w, o.w);
         }
         *reinterpret_cast<float4 *>(dst + j) = o;
       }
@@ -217,10 +227,12 @@ __device__ __forceinline__ void gemm_store_chunk(const GemmEpilogue &ep, long lo
     uint32_t packed[8];
 #pragma unroll
     for (int j = 0; j < 32; j += 4) {
+      const float4 es = *reinterpret_cast<const float4 *>(cole + j);
+      const float e4[4] = {es.x, es.y, es.z, es.w};
       uint32_t w = 0;
 #pragma unroll
       for (int b = 0; b < 4; ++b) {
-        const int code = round_clamp(__fmul_rn(y[j + b], pow2f(-ep.e_u[c0 + j + b])), 127.0f);
+        const int code = round_clamp(__fmul_rn(y[j + b], e4[b]), 127.0f);
         w |= ((uint32_t)(code & 0xFF)) << (8 * b);
       }
       packed[j / 4] = w;
@@ -236,8 +248,7 @@ __device__ __forceinline__ void gemm_store_chunk(const GemmEpilogue &ep, long lo
     if (c < di) {
       ep.z[row * di + c] = y[j];
     } else if (c < di + cc) {
-      const long long cx = c - di;
-      ep.xbc[row * cc + cx] = (int8_t)round_clamp(__fmul_rn(y[j], pow2f(-ep.e_u[cx])), 127.0f);
+      ep.xbc[row * cc + (c - di)] = (int8_t)round_clamp(__fmul_rn(y[j], cole[j]), 127.0f);
     } else {
       ep.dt[row * ep.nh + (c - di - cc)] = y[j];
     }
@@ -246,7 +257,7 @@ __device__ __forceinline__ void gemm_store_chunk(const GemmEpilogue &ep, long lo
 
 // ------------------------------------------------------------ the kernel
 template <int BN, int STAGES>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+__global__ void __launch_bounds__(kGemmThreads, 2)
     k_gemm_i8_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                  int num_k_blocks, GemmEpilogue ep) {
   static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN");
@@ -259,6 +270,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t *empty_bar = full_bar + STAGES;
   uint64_t *accum_bar = empty_bar + STAGES;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(accum_bar + 1);
+  // [BN] s_w of this tile, 16-byte aligned (read as float4)
+  float *col_w = reinterpret_cast<float *>((reinterpret_cast<uintptr_t>(tmem_slot + 1) + 15) &
+                                           ~static_cast<uintptr_t>(15));
+  float *col_e = col_w + BN;                                // [BN] 2^-e_u (split mode)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -319,15 +334,26 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mma_commit(accum_bar);
     }
   } else {
-    const bool ok = mbar_wait(accum_bar, 0);
-    tc_fence_after();
+    // while the main loop runs: stage this tile's column scales and the row scale
+    const int et = threadIdx.x - 64;  // 0 .. 127
+    for (int j = et; j < BN; j += 128) {
+      const long long c = (long long)n0 + j;
+      col_w[j] = c < ep.N ? ep.s_w[c] : 0.0f;
+      float e = 0.0f;
+      if (ep.mode == 1 && c >= ep.di && c < (long long)ep.di + ep.cc) e = pow2f(-ep.e_u[c - ep.di]);
+      col_e[j] = e;
+    }
     const int quarter = warp & 3;  // TMEM lanes [32*quarter, 32*quarter + 32)
     const long long row = (long long)m0 + quarter * 32 + lane;
+    const float sx = row < ep.M ? ep.s_x[row] : 0.0f;
+    asm volatile("bar.sync 1, 128;" ::: "memory");  // the 4 epilogue warps only
+    const bool ok = mbar_wait(accum_bar, 0);
+    tc_fence_after();
 #pragma unroll 1
     for (int c = 0; c < BN; c += 32) {
       uint32_t r[32];
       tmem_ld32(tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)c, r);
-      if (ok && n0 + c < ep.N) gemm_store_chunk(ep, row, (long long)n0 + c, r);
+      if (ok && n0 + c < ep.N) gemm_store_chunk(ep, row, sx, (long long)n0 + c, r, col_w + c, col_e + c);
     }
   }
   tc_fence_before();

@@ -128,6 +128,9 @@ __global__ void __launch_bounds__(1024) k_gate_norm_quant(
   __shared__ float s_red[kMaxBlocks];
   __shared__ float s_bc;
   __shared__ float s_rstd;
+  __shared__ int tab[8];
+  pwl_table_init(tab);
+  __syncthreads();
   const long long row = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nb = blockDim.x >> 5;
@@ -148,16 +151,24 @@ __global__ void __launch_bounds__(1024) k_gate_norm_quant(
     zv[4] = d.x; zv[5] = d.y; zv[6] = d.z; zv[7] = d.w;
   }
   int gq[8];
-  long long ss = 0;
+  unsigned ss0 = 0, ss1 = 0;  // g_q^2 < 2^30: four per partial fit 32 bits
   unsigned long long gmax = 0;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const long long g = (long long)yv[i] * silu_pwl(to_q16(zv[i]));
-    const unsigned long long ag = (unsigned long long)(g < 0 ? -g : g);
-    gmax = ag > gmax ? ag : gmax;
+    const int sg = silu_pwl_t(to_q16(zv[i]), tab);
+    // g = y sg as a 64-bit value from two 32-bit multiplies
+    const long long g = (long long)(((unsigned long long)(unsigned)__mulhi(yv[i], sg) << 32) |
+                                    (unsigned)(yv[i] * sg));
+    if (gstat) {
+      const unsigned long long ag = (unsigned long long)(g < 0 ? -g : g);
+      gmax = ag > gmax ? ag : gmax;
+    }
     gq[i] = (int)satb64(rshr64(g, sg_shift), 16);
-    ss += (long long)gq[i] * gq[i];
+    const unsigned sq = (unsigned)(gq[i] * gq[i]);
+    if (i < 4) ss0 += sq;
+    else ss1 += sq;
   }
+  long long ss = (long long)ss0 + ss1;
   if (gstat) {
     // the 8 lanes of a 64-column head combine, one atomic per head
 #pragma unroll

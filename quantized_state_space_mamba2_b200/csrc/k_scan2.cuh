@@ -47,6 +47,7 @@ struct ScanPrepArgs {
   int32_t *u;    // [B, nh, hd, Tp]
   int32_t *dx;   // [B, nh, hd, Tp]
   int32_t *bc;   // [B*T, 256]: B then C, int32
+  long long *bound;  // [B, nh, Tp/16, hd]: per 16-step chunk, sum of |u| max|B|
 };
 
 // grid = (Tp / 32, nh, B), block = 256; hd == 64
@@ -61,6 +62,22 @@ __global__ void __launch_bounds__(256) k_scan_prep(ScanPrepArgs a) {
   const long long Tp = scan_tpad(T);
   const int nt = min(kPrepTT, T - t0);
   const long long rowbase = (long long)b * T;
+  __shared__ int s_bmax[kPrepTT];
+  {  // max |B[n]| of each token (0 past the end): 8 threads x 16 bytes per token
+    const int tt = tid >> 3, k = tid & 7;
+    int m = 0;
+    if (tt < nt) {
+      const uint4 v = *reinterpret_cast<const uint4 *>(a.xbc + (rowbase + t0 + tt) * a.cc + a.di + k * 16);
+      const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) m = max(m, abs((int)(int8_t)((w4[q] >> (8 * i)) & 0xFF)));
+    }
+#pragma unroll
+    for (int o = 1; o < 8; o <<= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (k == 0) s_bmax[tt] = m;
+  }
   if (tid < kPrepTT) {
     int dtq = 0, dA = 0;
     if (tid < nt) {
@@ -91,6 +108,13 @@ __global__ void __launch_bounds__(256) k_scan_prep(ScanPrepArgs a) {
       uv[k] = (int)satb64(rshr64((long long)s_dtq[tb + k] * x, s_h), 24);
       dv[k] = (int)satb64(rshr64(Dq * x, s_D), 32);
     }
+    // growth bound of |h| over this thread's 8 steps; two threads make a 16-step chunk
+    long long gb = 0;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) gb += (long long)abs(uv[k]) * s_bmax[tb + k];
+    gb += __shfl_xor_sync(0xffffffffu, gb, 1);
+    if ((tid & 1) == 0)
+      a.bound[(((long long)b * nh + h) * (Tp / 16) + (t0 + tb) / 16) * hd + p] = gb;
     const long long off = (((long long)b * nh + h) * hd + p) * Tp + t0 + tb;
     *reinterpret_cast<int4 *>(a.u + off) = make_int4(uv[0], uv[1], uv[2], uv[3]);
     *reinterpret_cast<int4 *>(a.u + off + 4) = make_int4(uv[4], uv[5], uv[6], uv[7]);
@@ -113,6 +137,7 @@ struct ScanSeqArgs {
   const int32_t *u;   // [B, nh, hd, Tp]
   const int32_t *dx;  // [B, nh, hd, Tp]
   const int32_t *bc;  // [B*T, 256]
+  const long long *bound;  // [B, nh, Tp/16, hd]
   int T, nh, hd, di;
   const int32_t *e_C, *e_h, *e_y;
   int32_t *state;     // [B, nh, hd, 128] or null
@@ -134,17 +159,18 @@ template <int NPT, int PC, int TCH>
 struct ScanSeqSmem {
   static constexpr int LPP = 128 / NPT;          // threads per p
   static constexpr int NW = PC * LPP / 32;       // compute warps
-  // int64 per partial row: LPP + 1 (odd multiple of 16 B apart) keeps the
-  // per-row reads of a half-warp on distinct banks
+  // int2 per partial row: LPP + 1 (rows an odd number of 8-byte words apart)
+  // keeps the per-row reads of a half-warp on distinct banks
   static constexpr int PSTRIDE = LPP + 1;
   struct Slot {
     int32_t bc[TCH][256];
     int32_t dA[TCH];
     int32_t u[PC][TCH];
     int32_t dx[PC][TCH];
+    long long bound[PC];
   };
   Slot slot[kScanSlots];
-  long long part[NW][TCH * (32 / LPP)][PSTRIDE];
+  int2 part[NW][TCH * (32 / LPP)][PSTRIDE];
   uint64_t full[kScanSlots];
   uint64_t empty[kScanSlots];
 };
@@ -164,14 +190,43 @@ __device__ __forceinline__ void load_bc(const int32_t (*bc)[256], int tt, int n0
   }
 }
 
-// TCH steps of the recurrence for this thread's NPT cells; the next step's
-// B / C are loaded while the current step computes.
-template <int NPT, int TCH, bool FULL>
-__device__ __forceinline__ void scan_chunk_steps(int (&hs)[NPT], long long (&part)[TCH],
-                                                 const int32_t (*bc)[256], const int32_t *dAv,
-                                                 const int32_t *uv, int n0, int nt) {
-  int Bn[NPT], Cn[NPT];
-  load_bc<NPT>(bc, 0, n0, Bn, Cn);
+// TCH steps of the recurrence for this thread's NPT cells, in 32-bit integer
+// arithmetic only (32x32->64 multiplies are several times slower).  The state
+// is carried split as h = hh 2^16 + hl with hl in [0, 2^16), so that
+//   rshr(dA h, 16) = dA hh + ((dA hl + 2^15) >> 16)     (both products < 2^32)
+//   C h            = 2^16 (C hh) + C hl                 (partials per thread
+//                    and per channel stay within int32)
+// The next step's B / C are loaded while the current step computes.  CLAMP =
+// false is used only when the chunk provably never reaches the clamp (see
+// k_scan_seq), so both instantiations give the same bits.  part[tt] holds the
+// (C hh, C hl) partial sums of step tt.
+template <int NPT, bool CLAMP>
+__device__ __forceinline__ int2 scan_one_step(int (&hh)[NPT], unsigned (&hl)[NPT],
+                                              const int (&Bv)[NPT], const int (&Cv)[NPT], int dA,
+                                              int u) {
+  int ahi = 0, alo = 0;
+#pragma unroll
+  for (int j = 0; j < NPT; ++j) {
+    const unsigned t = (unsigned)dA * hl[j] + 0x8000u;
+    int hn = dA * hh[j] + (int)(t >> 16) + u * Bv[j];
+    if (CLAMP) hn = min(max(hn, -(int)kHLim), (int)kHLim);
+    hh[j] = hn >> 16;
+    hl[j] = (unsigned)hn & 0xFFFFu;
+    ahi += Cv[j] * hh[j];
+    alo += Cv[j] * (int)hl[j];
+  }
+  return make_int2(ahi, alo);
+}
+
+template <int NPT, int TCH, bool FULL, bool CLAMP>
+__device__ __forceinline__ void scan_chunk_steps(int (&hh)[NPT], unsigned (&hl)[NPT],
+                                                 int2 (&part)[TCH], const int32_t (*bc)[256],
+                                                 const int32_t *dAv, const int32_t *uv, int n0,
+                                                 int nt) {
+  // two register sets for B / C: the even step's set is refilled two steps
+  // ahead while the odd step computes, and vice versa (no copies)
+  int B0[NPT], C0[NPT], B1[NPT], C1[NPT];
+  load_bc<NPT>(bc, 0, n0, B0, C0);
 #pragma unroll
   for (int tg = 0; tg < TCH; tg += 4) {
     const int4 dA4 = *reinterpret_cast<const int4 *>(dAv + tg);
@@ -179,32 +234,15 @@ __device__ __forceinline__ void scan_chunk_steps(int (&hs)[NPT], long long (&par
     const int dAs[4] = {dA4.x, dA4.y, dA4.z, dA4.w};
     const int us[4] = {u4.x, u4.y, u4.z, u4.w};
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
+    for (int k = 0; k < 4; k += 2) {
       const int tt = tg + k;
-      if (!FULL && tt >= nt) {
-        part[tt] = 0;
-        continue;
-      }
-      int Bv[NPT], Cv[NPT];
-#pragma unroll
-      for (int j = 0; j < NPT; ++j) {
-        Bv[j] = Bn[j];
-        Cv[j] = Cn[j];
-      }
-      if (tt + 1 < TCH && (FULL || tt + 1 < nt)) load_bc<NPT>(bc, tt + 1, n0, Bn, Cn);
-      const long long dA = dAs[k];
-      const int u = us[k];
-      long long acc0 = 0, acc1 = 0;
-#pragma unroll
-      for (int j = 0; j < NPT; ++j) {
-        const int dec = (int)((dA * hs[j] + 32768LL) >> 16);
-        int hn = dec + u * Bv[j];
-        hn = min(max(hn, -(int)kHLim), (int)kHLim);
-        hs[j] = hn;
-        if (j & 1) acc1 += (long long)Cv[j] * hn;
-        else acc0 += (long long)Cv[j] * hn;
-      }
-      part[tt] = acc0 + acc1;
+      if (FULL || tt + 1 < nt) load_bc<NPT>(bc, tt + 1, n0, B1, C1);
+      if (FULL || tt < nt) part[tt] = scan_one_step<NPT, CLAMP>(hh, hl, B0, C0, dAs[k], us[k]);
+      else part[tt] = make_int2(0, 0);
+      if (tt + 2 < TCH && (FULL || tt + 2 < nt)) load_bc<NPT>(bc, tt + 2, n0, B0, C0);
+      if (FULL || tt + 1 < nt)
+        part[tt + 1] = scan_one_step<NPT, CLAMP>(hh, hl, B1, C1, dAs[k + 1], us[k + 1]);
+      else part[tt + 1] = make_int2(0, 0);
     }
   }
 }
@@ -220,7 +258,7 @@ __global__ void __launch_bounds__(PC *(128 / NPT) + 32) k_scan_seq(ScanSeqArgs a
   constexpr int NW = PC * LPP / 32;
   constexpr int PPW = 32 / LPP;  // channels per warp
   static_assert(LPP <= 32 && 32 % LPP == 0, "a channel's threads stay inside one warp");
-  static_assert(TCH % 4 == 0 && kPrepTT % TCH == 0, "chunk must tile the padded time axis");
+  static_assert(TCH == 16, "the growth bounds are per 16-step chunk");
   using Sm = ScanSeqSmem<NPT, PC, TCH>;
   constexpr int PSTRIDE = Sm::PSTRIDE;
   extern __shared__ __align__(16) uint8_t smem_raw[];
@@ -257,7 +295,10 @@ __global__ void __launch_bounds__(PC *(128 / NPT) + 32) k_scan_seq(ScanSeqArgs a
         const int t0 = c * TCH;
         const int nt = min(TCH, T - t0);
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        mbar_arrive_expect_tx(&sm.full[sl], (uint32_t)(nt * 1024 + TCH * 4 * (1 + 2 * PC)));
+        mbar_arrive_expect_tx(&sm.full[sl],
+                              (uint32_t)(nt * 1024 + TCH * 4 * (1 + 2 * PC) + PC * 8));
+        bulk_g2s(&s.bound[0], a.bound + ((headrow * (Tp / 16) + c) * hd + p0), PC * 8,
+                 &sm.full[sl]);
         bulk_g2s(&s.bc[0][0], a.bc + (rowbase + t0) * 256, (uint32_t)(nt * 1024), &sm.full[sl]);
         bulk_g2s(&s.dA[0], a.dA + headrow * Tp + t0, TCH * 4, &sm.full[sl]);
 #pragma unroll
@@ -277,56 +318,71 @@ __global__ void __launch_bounds__(PC *(128 / NPT) + 32) k_scan_seq(ScanSeqArgs a
   const int n0 = lane * NPT;
   const int wp = pp % PPW;           // channel within the warp
   const int s_y = a.e_y[h] - *a.e_C - a.e_h[h];
-  int hs[NPT];
+  int hh[NPT];
+  unsigned hl[NPT];
   int32_t *st = a.state ? a.state + (((headrow * hd) + p0 + pp) * 128 + n0) : nullptr;
-  if (st) {
 #pragma unroll
-    for (int j = 0; j < NPT; ++j) hs[j] = st[j];
-  } else {
-#pragma unroll
-    for (int j = 0; j < NPT; ++j) hs[j] = 0;
+  for (int j = 0; j < NPT; ++j) {
+    const int v = st ? st[j] : 0;
+    hh[j] = v >> 16;
+    hl[j] = (unsigned)v & 0xFFFFu;
   }
-  long long(*part)[PSTRIDE] = sm.part[warp];
+  int2(*part)[PSTRIDE] = sm.part[warp];
   for (int c = 0; c < nchunks; ++c) {
     const int sl = c % kScanSlots;
     if (!mbar_wait(&sm.full[sl], (uint32_t)(c / kScanSlots) & 1u)) return;  // error word set
     const typename Sm::Slot &s = sm.slot[sl];
     const int t0 = c * TCH;
     const int nt = min(TCH, T - t0);
-    long long pr[TCH];
-    if (nt == TCH)
-      scan_chunk_steps<NPT, TCH, true>(hs, pr, s.bc, s.dA, s.u[pp], n0, nt);
-    else
-      scan_chunk_steps<NPT, TCH, false>(hs, pr, s.bc, s.dA, s.u[pp], n0, nt);
+    // |rshr(dA h, 16)| <= |h| for dA <= 2^16, so over the chunk
+    // |h| <= max|h_start| + sum_t |u_t| max|B_t|: below the clamp, clamping
+    // is the identity at every step and the cheaper path is exact.
+    int hmax = 0;
+#pragma unroll
+    for (int j = 0; j < NPT; ++j) hmax = max(hmax, abs((int)(((unsigned)hh[j] << 16) | hl[j])));
+    const bool no_clamp = __all_sync(0xffffffffu, (long long)hmax + s.bound[pp] <= kHLim);
+    int2 pr[TCH];
+    if (nt == TCH) {
+      if (no_clamp) scan_chunk_steps<NPT, TCH, true, false>(hh, hl, pr, s.bc, s.dA, s.u[pp], n0, nt);
+      else scan_chunk_steps<NPT, TCH, true, true>(hh, hl, pr, s.bc, s.dA, s.u[pp], n0, nt);
+    } else {
+      scan_chunk_steps<NPT, TCH, false, true>(hh, hl, pr, s.bc, s.dA, s.u[pp], n0, nt);
+    }
     // partials of this warp: row (step, channel-in-warp), column = lane in channel
 #pragma unroll
     for (int tt = 0; tt < TCH; ++tt) part[tt * PPW + wp][lane] = pr[tt];
     __syncwarp();
-    // lane r sums row r (r < TCH * PPW) over the channel's LPP lanes, in two halves
+    // lane r sums row r over the channel's LPP lanes (int32: |sum C hh| < 2^28,
+    // |sum C hl| < 2^30), lanes sharing a row combine by shuffles
     constexpr int ROWS = TCH * PPW;
     static_assert(ROWS <= 32 && 32 % ROWS == 0, "rows map onto the warp's lanes");
     constexpr int SPLIT = 32 / ROWS;  // lanes sharing a row
     constexpr int PER = LPP / SPLIT;
     const int row = lane32 % ROWS, half = lane32 / ROWS;
-    long long sum0 = 0, sum1 = 0;
+    int shi = 0, slo = 0;
 #pragma unroll
-    for (int l = 0; l < PER; l += 2) {
-      sum0 += part[row][half * PER + l];
-      if (l + 1 < PER) sum1 += part[row][half * PER + l + 1];
+    for (int l = 0; l < PER; ++l) {
+      const int2 v = part[row][half * PER + l];
+      shi += v.x;
+      slo += v.y;
     }
-    long long sum = sum0 + sum1;
 #pragma unroll
-    for (int o = ROWS; o < 32; o <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    for (int o = ROWS; o < 32; o <<= 1) {
+      shi += __shfl_xor_sync(0xffffffffu, shi, o);
+      slo += __shfl_xor_sync(0xffffffffu, slo, o);
+    }
     const int tt = row / PPW, q = warp * PPW + row % PPW;
-    if (half == 0 && tt < nt)
+    if (half == 0 && tt < nt) {
+      const long long sum = (long long)shi * 65536 + slo;
       a.y[(rowbase + t0 + tt) * di + (long long)h * hd + p0 + q] =
           (int)satb64(rshr64(sum, s_y) + s.dx[q][tt], 32);
+    }
     __syncwarp();
     if (lane32 == 0) mbar_arrive(&sm.empty[sl]);
   }
   if (st) {
 #pragma unroll
-    for (int j = 0; j < NPT; ++j) st[j] = hs[j];
+    for (int j = 0; j < NPT; ++j) st[j] = (int)(((unsigned)hh[j] << 16) | hl[j]);
   }
 }
 

@@ -269,6 +269,40 @@ def test_ssm_scan_2p7b_shape(L):
     _run_scan(L, S.MAMBA2_2P7B, 1, 37, True, 80)
 
 
+@pytest.mark.parametrize("regime", ["saturating", "small"])
+def test_ssm_scan_clamp_regimes(L, regime):
+    """The sequential kernel skips the clamp for a chunk only when
+    max|h| + sum |u| max|B| stays below it; both regimes must match the oracle:
+    a state driven into the +-(2^30 - 1) clamp, and one that never nears it."""
+    s = MAMBA130
+    B, T = 1, 160
+    xbc, dt_raw, dt_bias, A_q, D_q, e_D, e_x, e_B, e_C, e_h, e_y = _scan_case(s, B, T, 90)
+    if regime == "saturating":
+        e_h = (e_x + e_B - 16 - 4).astype(np.int32)          # s_h = -4: u saturates at 2^23
+        dt_raw = np.zeros_like(dt_raw)                        # dt = softplus(bias), small
+        xbc[..., :s.d_inner] = 127
+        xbc[..., s.d_inner:s.d_inner + s.d_state] = 127       # B = 127 everywhere
+    else:
+        e_h = (e_x + e_B - 15 + 12).astype(np.int32)          # s_h = 13: small u
+    e_y = (np.maximum(e_C + e_h, e_D + e_x) - 2).astype(np.int32)
+    exps = _exps_for_scan(L, s, e_x, e_B, e_C, e_h, e_y, e_D)
+    st = np.zeros((B, s.nheads, s.headdim, s.d_state), np.int32)
+    y = torch.empty((B, T, s.d_inner), dtype=torch.int32, device="cuda")
+    st_d = dev(st)
+    ws = torch.empty(L.scan_workspace_bytes(s, B, T), dtype=torch.uint8, device="cuda")
+    L.ssm_scan_pot(dev(xbc), dev(dt_raw), B, T, s, dev(dt_bias), dev(A_q), dev(D_q), dev(exps),
+                   st_d, y, ws)
+    yr = O.ssm_scan_pot(xbc, dt_raw, dt_bias, A_q, D_q, e_x, e_B, e_C, e_h, e_y, e_D,
+                        s.headdim, s.d_state, state=st)
+    assert np.array_equal(host(y), yr)
+    assert np.array_equal(host(st_d), st)
+    lim = 2 ** 30 - 1
+    if regime == "saturating":
+        assert (np.abs(st) == lim).mean() > 0.5
+    else:
+        assert np.abs(st).max() < lim // 4 and np.abs(st).max() > 1000
+
+
 # ------------------------------------------------------------------ gate + norm
 
 @pytest.mark.parametrize("M", [1, 77, 512])
