@@ -317,6 +317,10 @@ static fm_status launch_scan_v2(const ScanArgs &a, int B, const ScanWs &w, cudaS
   const long long M = (long long)B * a.T;
   if (M == 0) return FM_OK;
   if (B > 65535 || M > 2147483647LL) return fail(FM_ERR_SHAPE, "scan: B or B*T too large");
+  if (a.T == 1) {  // decode: one step per sequence, no staging
+    k_scan_step<<<dim3(a.hd / 8, a.nh, B), 256, 0, s>>>(a);
+    return launched("k_scan_step");
+  }
   const long long Tp = scan_tpad(a.T);
   ScanPrepArgs p;
   p.xbc = a.xbc;
@@ -506,8 +510,14 @@ struct Carver {
 };
 
 ScanWs carve_scan(Carver &c, const Dims &d, int B, int T) {
-  const long long Tp = scan_tpad(T), M = (long long)B * T;
   ScanWs w;
+  if (T == 1) {  // single steps run k_scan_step, which stages nothing
+    w.dA = nullptr;
+    w.u = w.dx = w.bc = nullptr;
+    w.bound = nullptr;
+    return w;
+  }
+  const long long Tp = scan_tpad(T), M = (long long)B * T;
   w.dA = c.take<int32_t>((long long)B * d.nh * Tp);
   w.u = c.take<int32_t>((long long)B * d.di * Tp);
   w.dx = c.take<int32_t>((long long)B * d.di * Tp);

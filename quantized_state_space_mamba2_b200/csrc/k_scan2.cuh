@@ -16,14 +16,15 @@
 //                PC consecutive p); NPT consecutive n of one p per thread,
 //                state in registers.  One elected thread fetches each chunk
 //                of TCH steps with a handful of bulk copies (cp.async.bulk on
-//                an mbarrier) into a two-slot shared-memory ring one chunk
-//                ahead, so the other threads issue no load instructions and
+//                an mbarrier) into a three-slot shared-memory ring up to two
+//                chunks ahead, so the other threads issue no load instructions and
 //                no global latency sits on the recurrence; the C.h partial
 //                sums of a chunk stay in registers and are added across the
 //                p's threads once per chunk through padded shared memory.
-// Per state cell and step the loop issues a 32x32->64 multiply-add and a
-// funnel shift (rounded decay), a multiply-add (+ u B), two min/max (clamp)
-// and a 32x32->64 multiply-accumulate (C h).
+// Per state cell and step the loop issues, in 32-bit integer arithmetic on the
+// split state h = hh 2^16 + hl: the rounded decay (two multiplies, a shift),
+// the multiply-add of u B, the clamp (two min/max, skipped where a chunk
+// provably stays inside it) and the two C h multiply-accumulates.
 #pragma once
 #include "fm_common.cuh"
 #include "k_gemm.cuh"  // mbarrier helpers (bounded waits)
@@ -383,6 +384,63 @@ __global__ void __launch_bounds__(PC *(128 / NPT) + 32) k_scan_seq(ScanSeqArgs a
   if (st) {
 #pragma unroll
     for (int j = 0; j < NPT; ++j) st[j] = (int)(((unsigned)hh[j] << 16) | hl[j]);
+  }
+}
+
+// Decode (T == 1): one recurrence step per sequence (state null: zeros, not
+// written back).  The step reads and rewrites the whole state once, so HBM
+// bandwidth bounds it; one warp per channel p, each lane owning 4 consecutive
+// state columns (one 16-byte load and store), the C.h sum reduced by shuffles
+// in the split (hi, lo) 32-bit form.  Same arithmetic as one step of
+// k_scan_seq with the clamp.  Grid (hd / 8, nh, B), block 256.
+__global__ void __launch_bounds__(256) k_scan_step(ScanArgs a) {
+  __shared__ int tab[8];
+  pwl_table_init(tab);
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int p = blockIdx.x * 8 + warp;
+  const int n0 = lane * 4;
+  const int nh = a.nh, hd = a.hd, cc = a.cc, di = a.di;
+  const int8_t *row = a.xbc + (long long)b * cc;
+  const int e_x = a.e_x[h], e_B = *a.e_B, e_C = *a.e_C, e_h = a.e_h[h], e_y = a.e_y[h];
+  const int e_D = a.e_D[h];
+  const float xf = __fadd_rn(a.dt_raw[(long long)b * nh + h], a.dt_bias[h]);
+  const int dtq = softplus_pwl(to_q16(xf));
+  const int dA = pow2_pwl(-rshr64((long long)dtq * a.A_q[h], 12));
+  const long long xq = row[h * hd + p];
+  const int u = (int)satb64(rshr64((long long)dtq * xq, e_h - e_B - e_x + 16), 24);
+  const uint32_t bw = *reinterpret_cast<const uint32_t *>(row + di + n0);
+  const uint32_t cw = *reinterpret_cast<const uint32_t *>(row + di + 128 + n0);
+  int32_t *st = a.state ? a.state + ((((long long)b * nh + h) * hd + p) * 128 + n0) : nullptr;
+  const int4 hv = st ? *reinterpret_cast<const int4 *>(st) : make_int4(0, 0, 0, 0);
+  const int hs[4] = {hv.x, hv.y, hv.z, hv.w};
+  int hn[4];
+  int ahi = 0, alo = 0;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int Bj = (int)(int8_t)((bw >> (8 * j)) & 0xFF);
+    const int Cj = (int)(int8_t)((cw >> (8 * j)) & 0xFF);
+    const int hh = hs[j] >> 16;
+    const unsigned hl = (unsigned)hs[j] & 0xFFFFu;
+    const unsigned t = (unsigned)dA * hl + 0x8000u;
+    int v = dA * hh + (int)(t >> 16) + u * Bj;
+    v = min(max(v, -(int)kHLim), (int)kHLim);
+    hn[j] = v;
+    ahi += Cj * (v >> 16);
+    alo += Cj * (int)((unsigned)v & 0xFFFFu);
+  }
+  if (st) *reinterpret_cast<int4 *>(st) = make_int4(hn[0], hn[1], hn[2], hn[3]);
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) {
+    ahi += __shfl_xor_sync(0xffffffffu, ahi, o);
+    alo += __shfl_xor_sync(0xffffffffu, alo, o);
+  }
+  if (lane == 0) {
+    const long long sum = (long long)ahi * 65536 + alo;
+    const int dx = (int)satb64(rshr64((long long)a.D_q[h] * xq, e_y - e_D - e_x), 32);
+    a.y[(long long)b * di + (long long)h * hd + p] =
+        (int)satb64(rshr64(sum, e_y - e_C - e_h) + dx, 32);
   }
 }
 

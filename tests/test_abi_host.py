@@ -55,6 +55,8 @@ def test_exp_layout_and_workspace(so):
                + s.d_inner // 2)
     assert per_tok * 2048 <= ws <= per_tok * 2048 + 256 * 16
     assert lib.calib_workspace_bytes(s, 16, 512) > lib.workspace_bytes(s, 16, 512)
+    # a single decode step stages nothing for the scan
+    assert lib.scan_workspace_bytes(s, 64, 1) == 256
     bad = S.MixerShape(d_model=300, d_inner=512, headdim=64, d_state=128)
     assert lib.workspace_bytes(bad, 1, 1) == 0
 

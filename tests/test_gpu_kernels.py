@@ -269,6 +269,42 @@ def test_ssm_scan_2p7b_shape(L):
     _run_scan(L, S.MAMBA2_2P7B, 1, 37, True, 80)
 
 
+@pytest.mark.parametrize("shape,B", [("130m", 3), ("2p7b", 64)])
+def test_ssm_scan_decode_step(L, shape, B):
+    """T = 1 runs the single-step decode kernel (no staging): same bits as
+    the oracle's one recurrence step, state updated in place."""
+    s = MAMBA130 if shape == "130m" else S.MAMBA2_2P7B
+    _run_scan(L, s, B, 1, True, 85)
+
+
+def test_ssm_scan_decode_step_clamped(L):
+    """One decode step from a state at the clamp with saturated inputs: the
+    single-step kernel clamps exactly like the oracle."""
+    s = MAMBA130
+    B, T = 2, 1
+    xbc, dt_raw, dt_bias, A_q, D_q, e_D, e_x, e_B, e_C, e_h, e_y = _scan_case(s, B, T, 95)
+    e_h = (e_x + e_B - 16 - 4).astype(np.int32)
+    dt_raw = np.zeros_like(dt_raw)
+    xbc[..., :s.d_inner] = 127
+    xbc[..., s.d_inner:s.d_inner + s.d_state] = np.where(
+        S.uniform_ints((B, T, s.d_state), 0, 1, seed=96) > 0, 127, -127).astype(np.int8)
+    e_y = (np.maximum(e_C + e_h, e_D + e_x) - 2).astype(np.int32)
+    exps = _exps_for_scan(L, s, e_x, e_B, e_C, e_h, e_y, e_D)
+    lim = 2 ** 30 - 1
+    st = np.where(S.uniform_ints((B, s.nheads, s.headdim, s.d_state), 0, 1, seed=97) > 0,
+                  lim, -lim).astype(np.int32)
+    y = torch.empty((B, T, s.d_inner), dtype=torch.int32, device="cuda")
+    st_d = dev(st)
+    ws = torch.empty(L.scan_workspace_bytes(s, B, T), dtype=torch.uint8, device="cuda")
+    L.ssm_scan_pot(dev(xbc), dev(dt_raw), B, T, s, dev(dt_bias), dev(A_q), dev(D_q), dev(exps),
+                   st_d, y, ws)
+    yr = O.ssm_scan_pot(xbc, dt_raw, dt_bias, A_q, D_q, e_x, e_B, e_C, e_h, e_y, e_D,
+                        s.headdim, s.d_state, state=st)
+    assert np.array_equal(host(y), yr)
+    assert np.array_equal(host(st_d), st)
+    assert (np.abs(st) == lim).mean() > 0.2
+
+
 @pytest.mark.parametrize("regime", ["saturating", "small"])
 def test_ssm_scan_clamp_regimes(L, regime):
     """The sequential kernel skips the clamp for a chunk only when
