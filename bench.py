@@ -1,19 +1,30 @@
 #!/usr/bin/env python3
-"""Benchmark: W8A8 / power-of-two Mamba2 prefill tokens/s on one B200 per rank.
+"""Benchmark: W8A8 / power-of-two Mamba2 tokens/s on one B200 per rank.
 
-Workload (default): the Mamba2-130M-shaped stack -- 24 pre-normed residual
-mixer layers (d_model 768, d_inner 1536, 24 heads of 64, d_state 128),
-batch 1, 2048 tokens, outlier-injected N(0,1) inputs, random-init weights,
-activation scales dynamic per token, PoT exponents calibrated on the GPU
-from 16 seeded sequences of 512 tokens.  One step = one prefill of the whole
-stack over the batch.
+Default workload (the headline line), stack130m_24l_b1_t2048: the
+Mamba2-130M-shaped stack -- 24 pre-normed residual mixer layers (d_model 768,
+d_inner 1536, 24 heads of 64, d_state 128), batch 1, 2048 tokens,
+outlier-injected N(0,1) inputs, random-init weights, activation scales
+dynamic per token (--mode static: calibrated), power-of-two exponents
+calibrated on the GPU from 16 seeded sequences of 512 tokens.  One step = one
+prefill of the whole stack over the batch.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--mode dynamic|static]
+Other workloads (--workload):
+  mixer130m_b1_t256       one bare 130M mixer layer, batch 1, 256 tokens
+  gemm2p7b_inproj         FWHT + int8 quantisation + the in_proj W8A8 GEMM at
+                          the 2.7B shapes (K 2560, N 10576), M = --gemm-m
+                          (2048 | 8192 | 32768), fp32 dequantised output
+  stack2p7b_64l_b2_t4096  64 2.7B-shaped stack layers, batch 2, 4096 tokens
+  decode2p7b_64l_b64      one decode step of 64 sequences through the 64
+                          2.7B-shaped layers, states from a 512-token prefill
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload W] [--mode dynamic|static]
     python bench.py --impl reference ...   # the CPU oracle on the host cores
 
 Under torchrun each rank runs an independent replica on its own GPU (the
-prefill of independent sequences needs no collective): weak scaling; the
-step time is the max over ranks.  Prints one JSON line on rank 0.
+sequences of a batch are independent problems; no collective on the data
+path): weak scaling; the step time is the max over ranks.  Prints one JSON
+line on rank 0.
 """
 from __future__ import annotations
 
@@ -33,41 +44,68 @@ if ROOT not in sys.path:
 
 from quantized_state_space_mamba2_b200 import synth as S  # noqa: E402
 
-WORKLOAD = "stack130m_24l_b1_t2048"
+METRIC = "W8A8 Mamba2 prefill tokens/s (130M/2.7B shapes); int8 TOPS & HBM GB/s vs peak"
+DEFAULT_WORKLOAD = "stack130m_24l_b1_t2048"
+WORKLOAD_NAMES = ["mixer130m_b1_t256", "stack130m_24l_b1_t2048", "gemm2p7b_inproj",
+                  "stack2p7b_64l_b2_t4096", "decode2p7b_64l_b64"]
 OUTLIER_SEED = 4242
 L2_FLUSH_BYTES = 512 << 20
-SCAN_OPS_PER_CELL = 6  # decay multiply, rounding shift, dt*x*B multiply-add, clamp (2), C*h MAC
+# Algorithmic work of one state-cell update of the scan: decay multiply,
+# rounding shift, dt*x*B multiply-add, clamp (2), C*h multiply-accumulate.
+SCAN_OPS_PER_CELL = 6
+NOMINAL_INT8_OVER_BF16 = 2.0  # 4.5 / 2.25 PFLOP/s dense
+CPU_SAMPLE_MIN_S = 10.0
 
 
-def parse():
+def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=WORKLOAD_NAMES)
+    ap.add_argument("--gemm-m", type=int, default=32768, choices=[2048, 8192, 32768])
     ap.add_argument("--mode", default="dynamic", choices=["dynamic", "static"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--scan-tile", default=None,
                     help="npt,pc,tch of the sequential scan kernel (a compiled variant)")
-    return ap.parse_args()
-
-
-def workload():
-    w = S.WORKLOADS[WORKLOAD]
-    return w["shape"], w["layers"], w["batch"], w["seqlen"], w["n_outliers"], w["outlier_scale"]
-
-
-def layer_params(n_layers, shape):
-    return [S.layer_params(shape, 1000 + l) for l in range(n_layers)]
+    return ap.parse_args(argv)
 
 
 def measured_peaks():
-    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
-        with open(p) as f:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
             return json.load(f)
     except OSError:
         return None
+
+
+def workload_tokens(args) -> int:
+    """Tokens one step processes on one rank."""
+    w = S.WORKLOADS[args.workload]
+    if args.workload == "gemm2p7b_inproj":
+        return args.gemm_m
+    return w["batch"] * w["seqlen"]
+
+
+def config_block(args) -> dict:
+    w = S.WORKLOADS[args.workload]
+    d = w["shape"]
+    c = {"workload": args.workload, "d_model": d.d_model, "d_inner": d.d_inner,
+         "nheads": d.nheads, "headdim": d.headdim, "d_state": d.d_state, "act_quant": args.mode,
+         "hadamard": "block 256", "l2": "flushed between timed steps (512 MiB write)",
+         "parallelism": f"replica x{args.gpus}"}
+    if args.workload == "gemm2p7b_inproj":
+        c.update(M=args.gemm_m, N=d.n_in, K=d.d_model)
+    else:
+        c.update(layers=w.get("layers", 1), batch=w["batch"], seq_len=w["seqlen"],
+                 calibration=f"{S.CALIB_SEQS} seeded sequences x "
+                             f"{min(w.get('prefill_len', w['seqlen']), S.CALIB_MAX_LEN)} tokens "
+                             "(GPU, stage by stage)",
+                 scan_tile=args.scan_tile or "4,4,16")
+        if "prefill_len" in w:
+            c.update(prefill_len=w["prefill_len"], step="one decode token per sequence")
+    return c
 
 
 # ---------------------------------------------------------------- clocks
@@ -95,114 +133,443 @@ class ClockSampler:
         time.sleep(0.25)
         self.proc.terminate()
         out, _ = self.proc.communicate(timeout=10)
-        sm, smax, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in out.strip().splitlines():
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 7:
-                continue
-            try:
-                sm.append(float(parts[0]))
-                smax.append(float(parts[1]))
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[3:7]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
-                "reasons": sorted(reasons), "samples": len(sm)}
+        return parse_clock_samples(out)
 
 
-# ---------------------------------------------------------------- CPU oracle baseline
+def parse_clock_samples(text: str) -> dict:
+    sm, smax, reasons = [], [], set()
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    for line in text.strip().splitlines():
+        parts = [p.strip() for p in line.split(",")]
+        if len(parts) < 7:
+            continue
+        try:
+            sm.append(float(parts[0]))
+            smax.append(float(parts[1]))
+        except ValueError:
+            continue
+        for n, v in zip(names, parts[3:7]):
+            if v.lower().startswith("active"):
+                reasons.add(n)
+    if not sm:
+        return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+    return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+            "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- CPU oracle samples
 class OracleSample:
-    """The oracle as it stands (single-threaded C, composed by numpy) on a
-    bounded sample of the workload: one stack layer (pre-norm + mixer +
-    residual) over the full batch, scaled to the stack's token rate
-    (tokens / (layers x one layer's time))."""
+    """The oracle as it stands (single-threaded C composed by numpy) on a
+    bounded sample of a workload: one layer over a slice of its tokens (the
+    oracle's cost is linear in tokens and in layers), or a slice of the GEMM's
+    rows.  value = sample tokens / (sample seconds x the workload's layers)."""
 
-    def __init__(self, shape, n_layers, mode: str):
+    def __init__(self, workload: str, mode: str, gemm_m: int = 32768):
         import oracle as O
-        _, _, B, T, n_out, scale = workload()
-        self.O, self.B, self.T, self.n_layers = O, B, T, n_layers
-        P = S.layer_params(shape, 1000)
-        self.L = O.prepare_layer(P, shape, rotate=1,
-                                 mode=O.DYNAMIC if mode == "dynamic" else O.STATIC, prenorm=True)
+        self.O, self.workload = O, workload
+        w = S.WORKLOADS[workload]
+        shape = w["shape"]
+        omode = O.DYNAMIC if mode == "dynamic" else O.STATIC
+        n_out, scale = w["n_outliers"], w["outlier_scale"]
+        self.layers = w.get("layers", 1)
+        if workload == "gemm2p7b_inproj":
+            rows = 128
+            self.x = S.activations(1, rows, shape.d_model, seed=11, n_outliers=n_out,
+                                   outlier_scale=scale, outlier_seed=OUTLIER_SEED)[0]
+            self.wq, self.sw = O.prepare_linear(S.layer_params(shape, 1000)["w_in"])
+            self.tokens = rows
+            self.desc = f"{rows} of the {gemm_m} rows (FWHT + quantisation + in_proj GEMM)"
+            self.run_fn = self._gemm
+            return
+        prenorm = self.layers > 1
+        L = O.prepare_layer(S.layer_params(shape, 1000), shape, rotate=1, mode=omode,
+                            prenorm=prenorm)
         xcal = S.calibration_batch(shape.d_model, 64, n_out, scale, OUTLIER_SEED, n_seqs=1)
-        O.calibrate_layer(self.L, xcal, residual=True)
-        self.x = S.activations(B, T, shape.d_model, seed=1, n_outliers=n_out, outlier_scale=scale,
-                               outlier_seed=OUTLIER_SEED)
+        O.calibrate_layer(L, xcal, residual=prenorm)
+        self.L, self.prenorm = L, prenorm
+        if workload == "decode2p7b_64l_b64":
+            Bs = w["batch"]
+            self.x = S.activations(Bs, 1, shape.d_model, seed=5, n_outliers=n_out,
+                                   outlier_scale=scale, outlier_seed=OUTLIER_SEED)
+            self.cs = np.zeros((Bs, 3, shape.conv_ch), np.int8)
+            self.ss = np.zeros((Bs, shape.nheads, shape.headdim, shape.d_state), np.int32)
+            self.tokens = Bs
+            self.desc = f"one decode step of 1 of {self.layers} layers for all {Bs} sequences"
+            self.run_fn = self._decode
+            return
+        B, T = w["batch"], w["seqlen"]
+        Ts = min(B * T, 2048 if shape.d_model <= 1024 else 256)  # ~5-10 s a run
+        self.x = S.activations(1, Ts, shape.d_model, seed=1, n_outliers=n_out,
+                               outlier_scale=scale, outlier_seed=OUTLIER_SEED)
+        self.tokens = Ts
+        self.desc = f"1 of {self.layers} layers over {Ts} of the {B}x{T} tokens"
+        self.run_fn = self._prefill
+
+    def _gemm(self):
+        q, sx = self.O.hadamard_quant(self.x)
+        self.O.dequant(self.O.gemm_i8(q, self.wq), sx, self.sw)
+
+    def _prefill(self):
+        self.O.mixer_prefill(self.L, self.x, residual=self.prenorm)
+
+    def _decode(self):
+        self.O.mixer_prefill(self.L, self.x, residual=True, conv_state=self.cs,
+                             ssm_state=self.ss)
 
     def run(self) -> float:
         t0 = time.perf_counter()
-        self.O.mixer_prefill(self.L, self.x, residual=True)
+        self.run_fn()
         return time.perf_counter() - t0
 
-    def describe(self, seconds: float) -> dict:
-        return {"value": self.B * self.T / (seconds * self.n_layers), "unit": "tokens/s",
-                "cores": 1, "kind": "oracle",
-                "sample": f"1 of {self.n_layers} stack layers over {self.B}x{self.T} tokens "
-                          f"({seconds:.2f} s), scaled to {self.n_layers} layers"}
+    def value(self, seconds: float) -> float:
+        return self.tokens / (seconds * self.layers)
 
+    def measure(self, min_seconds: float = CPU_SAMPLE_MIN_S, max_runs: int = 16) -> dict:
+        secs = []
+        while sum(secs) < min_seconds and len(secs) < max_runs:
+            secs.append(self.run())
+        return self.describe(statistics.mean(secs), len(secs))
 
-def cpu_oracle_sample(shape, n_layers, mode: str) -> dict:
-    o = OracleSample(shape, n_layers, mode)
-    return o.describe(o.run())
+    def describe(self, seconds: float, runs: int) -> dict:
+        scaled = "" if self.layers == 1 else f", scaled to {self.layers} layers"
+        return {"value": self.value(seconds), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                "sample": f"{self.desc}{scaled}; {runs} run(s), {seconds:.2f} s each"}
 
 
 def run_reference(args):
     """--impl reference: the CPU oracle on this host's cores (rank 0 only);
-    each step is the bounded sample above."""
-    rank = int(os.environ.get("RANK", "0"))
-    if rank != 0:
+    each step is the bounded sample of the chosen workload."""
+    if int(os.environ.get("RANK", "0")) != 0:
         return
-    shape, n_layers, B, T, _, _ = workload()
-    o = OracleSample(shape, n_layers, args.mode)
+    o = OracleSample(args.workload, args.mode, args.gemm_m)
     for _ in range(args.warmup):
         o.run()
     secs = [o.run() for _ in range(max(1, args.steps))]
-    per_step = statistics.mean(secs) * n_layers      # one stack prefill
-    value = B * T / per_step
-    cb = o.describe(statistics.mean(secs))
-    line = {"impl": "reference", "metric": "W8A8 Mamba2 prefill tokens/s", "value": value,
-            "unit": "tokens/s", "n_gpus": args.gpus, "steps": len(secs), "warmup": args.warmup,
-            "ms_per_step": 1000.0 * per_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "int8+int32 fixed point (CPU oracle)",
-            "data": "synthetic", "config": config_block(args, shape, n_layers, B, T),
-            "cpu_baseline": dict(cb, value=value),
+    mean_s = statistics.mean(secs)
+    value = o.value(mean_s)
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": args.gpus, "steps": len(secs), "warmup": args.warmup,
+            "ms_per_step": 1000.0 * workload_tokens(args) / value, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "int8/int32 fixed point (CPU oracle)",
+            "data": "synthetic", "config": config_block(args),
+            "cpu_baseline": o.describe(mean_s, len(secs)),
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
-def config_block(args, shape, n_layers, B, T):
-    return {"workload": WORKLOAD, "layers": n_layers, "batch": B, "seq_len": T,
-            "d_model": shape.d_model, "d_inner": shape.d_inner, "nheads": shape.nheads,
-            "d_state": shape.d_state, "act_quant": args.mode, "hadamard": True,
-            "calibration": "16 seeded sequences x 512 tokens (GPU, stage by stage)",
-            "l2": "flushed between timed steps (512 MiB write)", "parallelism": f"replica x{args.gpus}",
-            "scan_tile": args.scan_tile or "4,4,16"}
+# ---------------------------------------------------------------- GPU workloads
+def _stage_buffers(torch, d, M, dev):
+    e = lambda *sh, dt: torch.empty(sh, dtype=dt, device=dev)
+    return dict(q_in=e(M, d.d_model, dt=torch.int8), sx_in=e(M, dt=torch.float32),
+                z=e(M, d.d_inner, dt=torch.float32), xbc=e(M, d.conv_ch, dt=torch.int8),
+                dtr=e(M, d.nheads, dt=torch.float32), xo=e(M, d.conv_ch, dt=torch.int8),
+                y=e(M, d.d_inner, dt=torch.int32), q_out=e(M, d.d_inner, dt=torch.int8),
+                sx_out=e(M, dt=torch.float32))
+
+
+class StackWorkload:
+    """Prefill of a stack (or of one bare mixer layer).  The timed step calls
+    the stage entry points in the order fm_mixer_prefill composes them (checked
+    bit for bit against it), with events around each layer's scan."""
+
+    launches_per_layer = 7  # FWHT+quant, in_proj, conv, scan prep, scan, gate, out_proj
+
+    def __init__(self, args, torch, lib, dev, rank):
+        from quantized_state_space_mamba2_b200.model import DeviceLayer, DeviceStack
+        self.torch, self.lib, self.dev = torch, lib, dev
+        w = S.WORKLOADS[args.workload]
+        self.shape = d = w["shape"]
+        self.n_layers = w.get("layers", 1)
+        self.B, self.T = w["batch"], w["seqlen"]
+        self.stack_mode = self.n_layers > 1
+        self.mode = lib.FM_DYNAMIC if args.mode == "dynamic" else lib.FM_STATIC
+        params = (S.layer_params(d, 1000 + l) for l in range(self.n_layers))
+        xcal = torch.from_numpy(S.calibration_batch(d.d_model, self.T, w["n_outliers"],
+                                                    w["outlier_scale"], OUTLIER_SEED)).to(dev)
+        if self.stack_mode:
+            self.stack = DeviceStack(list(params), d, rotate=1, mode=self.mode, device=dev)
+            self.layers = self.stack.layers
+            self.stack.calibrate(xcal)
+        else:
+            self.layers = [DeviceLayer(next(params), d, rotate=1, mode=self.mode, device=dev)]
+            self.layers[0].calibrate(xcal)
+        del xcal
+        self.x_host = S.activations(self.B, self.T, d.d_model, seed=1 + rank,
+                                    n_outliers=w["n_outliers"], outlier_scale=w["outlier_scale"],
+                                    outlier_seed=OUTLIER_SEED)
+        self.x0 = torch.from_numpy(self.x_host).to(dev)
+        self.r = torch.empty_like(self.x0)
+        M = self.B * self.T
+        self.ws = self.layers[0].workspace(self.B, self.T)
+        self.sws = torch.empty(lib.scan_workspace_bytes(d, self.B, self.T), dtype=torch.uint8,
+                               device=dev)
+        self.buf = _stage_buffers(torch, d, M, dev)
+        self.tokens = M
+        self.launches = self.launches_per_layer * self.n_layers
+
+    def states(self, i):
+        return None, None
+
+    def step(self, ev=None):
+        lib, d, B, T, b = self.lib, self.shape, self.B, self.T, self.buf
+        stream = self.torch.cuda.current_stream(self.dev)
+        src = self.x0
+        for i, Ly in enumerate(self.layers):
+            cs, ss = self.states(i)
+            lib.hadamard_quant(src, d.d_model, Ly.prenorm_w, 1, self.mode, Ly.static_amax,
+                               b["q_in"], b["sx_in"])
+            lib.in_proj(b["q_in"], b["sx_in"], Ly.w_in_q, Ly.w_in_s, d, Ly.exps, b["z"], b["xbc"],
+                        b["dtr"])
+            lib.conv1d_pot(b["xbc"], B, T, d, Ly.conv_wq, Ly.conv_bq, Ly.exps, cs, b["xo"])
+            if ev is not None:
+                ev[i][0].record(stream)
+            lib.ssm_scan_pot(b["xo"], b["dtr"], B, T, d, Ly.dt_bias, Ly.A_q, Ly.D_q, Ly.exps, ss,
+                             b["y"], self.sws)
+            if ev is not None:
+                ev[i][1].record(stream)
+            lib.gate_norm_quant(b["y"], b["z"], d, Ly.exps, Ly.norm_w, 1, self.mode,
+                                Ly.static_amax[1:], b["q_out"], b["sx_out"])
+            lib.w8a8_gemm(b["q_out"], b["sx_out"], Ly.w_out_q, Ly.w_out_s, self.r,
+                          residual=src if self.stack_mode else None)
+            src = self.r
+
+    def output(self):
+        return self.r
+
+    def public_output(self):
+        """The same input through the public per-layer entry point."""
+        if self.stack_mode:
+            out = self.x0.clone()
+            self.stack.prefill_(out, ws=self.ws)
+            return out
+        return self.layers[0].prefill(self.x0, ws=self.ws)
+
+    def e2e_setup(self):
+        torch = self.torch
+        self.xh = torch.from_numpy(self.x_host).pin_memory()
+        self.oh = torch.empty_like(self.xh).pin_memory()
+        self.xd = torch.empty_like(self.x0)
+        self.od = torch.empty_like(self.x0)
+        self.h2d_bytes = self.d2h_bytes = self.x_host.nbytes
+
+    def e2e_step(self):
+        self.xd.copy_(self.xh, non_blocking=True)
+        if self.stack_mode:
+            self.stack.prefill_(self.xd, ws=self.ws)
+            self.oh.copy_(self.xd, non_blocking=True)
+        else:
+            self.layers[0].prefill(self.xd, out=self.od, ws=self.ws)
+            self.oh.copy_(self.od, non_blocking=True)
+
+    def e2e_matches(self, ref) -> bool:
+        return self.torch.equal(self.oh, ref.cpu())
+
+    def roofline(self, dom_ms, peaks):
+        d = self.shape
+        cells = self.B * d.nheads * d.headdim * d.d_state * self.T
+        achieved = cells * SCAN_OPS_PER_CELL / (dom_ms / 1e3) / 1e12
+        mhz = (peaks or {}).get("sm_max_mhz", 1965.0)
+        peak = 148 * 4 * 32 * mhz * 1e6 / 1e12
+        return {"bound": "alu", "kernel": "fm_ssm_scan_pot (k_scan_prep + k_scan_seq)",
+                "achieved": achieved, "peak": peak, "unit": "Tops/s (int32)",
+                "frac": achieved / peak, "traffic": None,
+                "peak_basis": f"derived: 148 SMs x 4 SMSPs x 32 lanes x 1 int op/clk x "
+                              f"{mhz:.0f} MHz (measured max SM clock)",
+                "algorithmic": f"{SCAN_OPS_PER_CELL} int ops per state-cell update x {cells} "
+                               "updates per launch"}
+
+
+class DecodeWorkload(StackWorkload):
+    """One decode step of B sequences through the whole stack; conv and SSM
+    states come from a seeded prefill and advance by one token per step."""
+
+    launches_per_layer = 7  # FWHT+quant, in_proj, conv, conv-state update, scan step, gate, out_proj
+
+    def __init__(self, args, torch, lib, dev, rank):
+        from quantized_state_space_mamba2_b200.model import DeviceStack
+        self.torch, self.lib, self.dev = torch, lib, dev
+        w = S.WORKLOADS[args.workload]
+        self.shape = d = w["shape"]
+        self.n_layers, self.B, self.T = w["layers"], w["batch"], 1
+        self.stack_mode = True
+        self.mode = lib.FM_DYNAMIC if args.mode == "dynamic" else lib.FM_STATIC
+        P = w["prefill_len"]
+        self.stack = DeviceStack([S.layer_params(d, 1000 + l) for l in range(self.n_layers)], d,
+                                 rotate=1, mode=self.mode, device=dev)
+        self.layers = self.stack.layers
+        xcal = torch.from_numpy(S.calibration_batch(d.d_model, P, w["n_outliers"],
+                                                    w["outlier_scale"], OUTLIER_SEED)).to(dev)
+        self.stack.calibrate(xcal)
+        del xcal
+        self.st = [L.new_states(self.B) for L in self.layers]
+        pre = torch.from_numpy(S.activations(self.B, P, d.d_model, seed=77 + rank,
+                                             n_outliers=w["n_outliers"],
+                                             outlier_scale=w["outlier_scale"],
+                                             outlier_seed=OUTLIER_SEED)).to(dev)
+        self.stack.prefill_(pre, states=self.st)
+        del pre
+        torch.cuda.synchronize()
+        self.st0 = [(c.clone(), s.clone()) for c, s in self.st]
+        self.x_host = S.activations(self.B, 1, d.d_model, seed=5 + rank,
+                                    n_outliers=w["n_outliers"], outlier_scale=w["outlier_scale"],
+                                    outlier_seed=OUTLIER_SEED)
+        self.x0 = torch.from_numpy(self.x_host).to(dev)
+        self.r = torch.empty_like(self.x0)
+        self.ws = self.layers[0].workspace(self.B, 1)
+        self.sws = torch.empty(lib.scan_workspace_bytes(d, self.B, 1), dtype=torch.uint8,
+                               device=dev)
+        self.buf = _stage_buffers(torch, d, self.B, dev)
+        self.tokens = self.B
+        self.launches = self.launches_per_layer * self.n_layers
+
+    def states(self, i):
+        return self.st[i]
+
+    def restore(self):
+        for (c, s), (c0, s0) in zip(self.st, self.st0):
+            c.copy_(c0)
+            s.copy_(s0)
+
+    def public_output(self):
+        self.restore()
+        out = self.x0.clone()
+        for (cs, ss), Ly in zip(self.st, self.layers):
+            Ly.decode(out, cs, ss, residual=True, out=out, ws=self.ws)
+        self.torch.cuda.synchronize()
+        self.restore()
+        return out
+
+    def e2e_step(self):
+        self.xd.copy_(self.xh, non_blocking=True)
+        for (cs, ss), Ly in zip(self.st, self.layers):
+            Ly.decode(self.xd, cs, ss, residual=True, out=self.xd, ws=self.ws)
+        self.oh.copy_(self.xd, non_blocking=True)
+
+    def e2e_matches(self, ref) -> bool:
+        return True  # the states have advanced; the public path was checked before timing
+
+    def roofline(self, dom_ms, peaks):
+        d = self.shape
+        state = self.B * d.nheads * d.headdim * d.d_state * 4
+        io = self.B * (d.conv_ch + 4 * d.nheads + 4 * d.d_inner)
+        achieved = (2 * state + io) / (dom_ms / 1e3) / 1e9
+        peak = (peaks or {}).get("hbm_gbs", 6548.0)
+        return {"bound": "hbm", "kernel": "fm_ssm_scan_pot, T = 1 (k_scan_step)",
+                "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                "traffic": None, "peak_basis": "measured copy bandwidth (hbm_gbs)",
+                "algorithmic": f"state read + write {2 * state} B + x, B, C, dt, y {io} B "
+                               "per launch"}
+
+
+class GemmWorkload:
+    """FWHT + quantisation of X [M, 2560] and the in_proj W8A8 GEMM
+    (N = 10576) with an fp32 dequantised output, at the 2.7B shapes; events
+    around the GEMM."""
+
+    n_layers = 1
+
+    def __init__(self, args, torch, lib, dev, rank):
+        self.torch, self.lib, self.dev = torch, lib, dev
+        w = S.WORKLOADS["gemm2p7b_inproj"]
+        d = w["shape"]
+        self.M, self.N, self.K = args.gemm_m, d.n_in, d.d_model
+        self.x_host = S.activations(1, self.M, self.K, seed=11 + rank, n_outliers=w["n_outliers"],
+                                    outlier_scale=w["outlier_scale"],
+                                    outlier_seed=OUTLIER_SEED)[0]
+        self.x0 = torch.from_numpy(self.x_host).to(dev)
+        W = torch.from_numpy(S.layer_params(d, 1000)["w_in"]).to(dev)
+        self.wq = torch.empty((self.N, self.K), dtype=torch.int8, device=dev)
+        self.sw = torch.empty(self.N, dtype=torch.float32, device=dev)
+        lib.prepare_linear(W, 1, self.wq, self.sw)
+        del W
+        self.q = torch.empty((self.M, self.K), dtype=torch.int8, device=dev)
+        self.sx = torch.empty(self.M, dtype=torch.float32, device=dev)
+        self.Y = torch.empty((self.M, self.N), dtype=torch.float32, device=dev)
+        self.tokens = self.M
+        self.launches = 2
+
+    def _run(self, x, ev=None):
+        lib = self.lib
+        stream = self.torch.cuda.current_stream(self.dev)
+        lib.hadamard_quant(x, self.K, None, 1, lib.FM_DYNAMIC, None, self.q, self.sx)
+        if ev is not None:
+            ev[0][0].record(stream)
+        lib.w8a8_gemm(self.q, self.sx, self.wq, self.sw, self.Y)
+        if ev is not None:
+            ev[0][1].record(stream)
+
+    def step(self, ev=None):
+        self._run(self.x0, ev)
+
+    def output(self):
+        return self.Y
+
+    def public_output(self):
+        return None
+
+    def e2e_setup(self):
+        torch = self.torch
+        self.xh = torch.from_numpy(self.x_host).pin_memory()
+        self.oh = torch.empty((self.M, self.N), dtype=torch.float32).pin_memory()
+        self.xd = torch.empty_like(self.x0)
+        self.h2d_bytes = self.x_host.nbytes
+        self.d2h_bytes = self.M * self.N * 4
+
+    def e2e_step(self):
+        self.xd.copy_(self.xh, non_blocking=True)
+        self._run(self.xd)
+        self.oh.copy_(self.Y, non_blocking=True)
+
+    def e2e_matches(self, ref) -> bool:
+        return True
+
+    def roofline(self, dom_ms, peaks):
+        ops = 2.0 * self.M * self.N * self.K
+        achieved = ops / (dom_ms / 1e3) / 1e12
+        bf16 = (peaks or {}).get("bf16_tflops", 1590.0)
+        peak = bf16 * NOMINAL_INT8_OVER_BF16
+        return {"bound": "tensor", "kernel": "fm_w8a8_gemm (k_gemm_i8_tc, tcgen05 kind::i8)",
+                "achieved": achieved, "peak": peak, "unit": "TOPS (int8)",
+                "frac": achieved / peak, "traffic": None,
+                "peak_basis": "measured bf16 burst (bf16_tflops) x nominal int8/bf16 ratio 2",
+                "algorithmic": f"2 M N K = {ops:.4g} int8 ops per launch"}
+
+
+def make_workload(args, torch, lib, dev, rank):
+    if args.workload == "gemm2p7b_inproj":
+        return GemmWorkload(args, torch, lib, dev, rank)
+    if args.workload == "decode2p7b_64l_b64":
+        return DecodeWorkload(args, torch, lib, dev, rank)
+    return StackWorkload(args, torch, lib, dev, rank)
 
 
 # ---------------------------------------------------------------- the GPU arm
+def max_over_ranks(torch, dist, world, value, dev) -> float:
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
         return
+    import datetime
+
     import torch
     import torch.distributed as dist
 
     from quantized_state_space_mamba2_b200 import build, lib
-    from quantized_state_space_mamba2_b200.model import DeviceStack
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
         torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     if rank == 0:
         build.build()
     if world > 1:
@@ -211,69 +578,27 @@ def main():
     if args.scan_tile:
         lib.set_scan_tile(*[int(v) for v in args.scan_tile.split(",")])
     dev = torch.device("cuda", local)
-    shape, n_layers, B, T, n_out, scale = workload()
-    mode = lib.FM_DYNAMIC if args.mode == "dynamic" else lib.FM_STATIC
-
-    stack = DeviceStack(layer_params(n_layers, shape), shape, rotate=1, mode=mode, device=dev)
-    xcal = S.calibration_batch(shape.d_model, T, n_out, scale, OUTLIER_SEED)
-    stack.calibrate(torch.from_numpy(xcal).to(dev))
-    del xcal
-    x_host = S.activations(B, T, shape.d_model, seed=1 + rank, n_outliers=n_out,
-                           outlier_scale=scale, outlier_seed=OUTLIER_SEED)
-    x0 = torch.from_numpy(x_host).to(dev)
-    r = torch.empty_like(x0)
-    M = B * T
-    ws = stack.layers[0].workspace(B, T)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream(dev)
+    wl = make_workload(args, torch, lib, dev, rank)
 
-    # stage buffers inside the workspace-equivalent set (same composition as fm_mixer_prefill)
-    d = shape
-    q_in = torch.empty((M, d.d_model), dtype=torch.int8, device=dev)
-    sx_in = torch.empty(M, dtype=torch.float32, device=dev)
-    z = torch.empty((M, d.d_inner), dtype=torch.float32, device=dev)
-    xbc = torch.empty((M, d.conv_ch), dtype=torch.int8, device=dev)
-    dtr = torch.empty((M, d.nheads), dtype=torch.float32, device=dev)
-    xo = torch.empty((M, d.conv_ch), dtype=torch.int8, device=dev)
-    y = torch.empty((M, d.d_inner), dtype=torch.int32, device=dev)
-    q_out = torch.empty((M, d.d_inner), dtype=torch.int8, device=dev)
-    sx_out = torch.empty(M, dtype=torch.float32, device=dev)
-    sws = torch.empty(lib.scan_workspace_bytes(d, B, T), dtype=torch.uint8, device=dev)
-    launches_per_step = 7 * n_layers  # FWHT+quant, in_proj, conv, scan prep, scan, gate, out_proj
-
-    def step(scan_events=None):
-        src = x0
-        for i, Ly in enumerate(stack.layers):
-            lib.hadamard_quant(src, d.d_model, Ly.prenorm_w, 1, mode, Ly.static_amax, q_in, sx_in)
-            lib.in_proj(q_in, sx_in, Ly.w_in_q, Ly.w_in_s, d, Ly.exps, z, xbc, dtr)
-            lib.conv1d_pot(xbc, B, T, d, Ly.conv_wq, Ly.conv_bq, Ly.exps, None, xo)
-            if scan_events is not None:
-                scan_events[i][0].record(stream)
-            lib.ssm_scan_pot(xo, dtr, B, T, d, Ly.dt_bias, Ly.A_q, Ly.D_q, Ly.exps, None, y, sws)
-            if scan_events is not None:
-                scan_events[i][1].record(stream)
-            lib.gate_norm_quant(y, z, d, Ly.exps, Ly.norm_w, 1, mode, Ly.static_amax[1:], q_out,
-                                sx_out)
-            lib.w8a8_gemm(q_out, sx_out, Ly.w_out_q, Ly.w_out_s, r, residual=src)
-            src = r
-
-    # the stage-by-stage step must equal the public fm_mixer_prefill path
-    step()
-    ref = x0.clone()
-    stack.prefill_(ref, ws=ws)
+    # the stage-by-stage step must equal the public entry points bit for bit
+    ref = wl.public_output()
+    wl.step()
     torch.cuda.synchronize()
     lib.sync_status()
-    if not torch.equal(ref, r):
-        raise SystemExit("bench: stage-by-stage step differs from fm_mixer_prefill")
+    if ref is not None and not torch.equal(ref, wl.output()):
+        raise SystemExit("bench: stage-by-stage step differs from the public entry points")
 
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     for _ in range(args.warmup):
-        step()
+        wl.step()
     torch.cuda.synchronize()
 
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(args.steps)]
-    sev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-            for _ in range(n_layers)] for _ in range(args.steps)]
+    dev_ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(wl.n_layers)] for _ in range(args.steps)]
     clocks = ClockSampler(local)
     if world > 1:
         dist.barrier()
@@ -284,7 +609,7 @@ def main():
         flush.zero_()
         torch.cuda.nvtx.range_push("bench_step")
         ev[k][0].record(stream)
-        step(sev[k])
+        wl.step(dev_ev[k])
         ev[k][1].record(stream)
         torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize()
@@ -293,77 +618,48 @@ def main():
         dist.barrier()
     lib.sync_status()
     step_ms = [a.elapsed_time(b) for a, b in ev]
-    scan_ms = [a.elapsed_time(b) for row in sev for a, b in row]
-    total_ms = sum(step_ms)
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms = float(t.item())
-    ms_per_step = total_ms / args.steps
-    value = world * B * T * args.steps / (total_ms / 1000.0)
+    dom_ms = [a.elapsed_time(b) for row in dev_ev for a, b in row]
+    total_ms = max_over_ranks(torch, dist, world, sum(step_ms), dev)
+    value = world * wl.tokens * args.steps / (total_ms / 1000.0)
+    roofline = wl.roofline(statistics.mean(dom_ms), measured_peaks())
+    roofline["avg_launch_us"] = 1000.0 * statistics.mean(dom_ms)
+    roofline["share_of_step"] = sum(dom_ms) / sum(step_ms)
 
-    # roofline of the dominant kernel (the sequential fixed-point scan, integer-ALU bound)
-    peaks = measured_peaks()
-    cells = B * d.nheads * d.headdim * d.d_state * T
-    scan_avg_s = statistics.mean(scan_ms) / 1000.0
-    achieved = cells * SCAN_OPS_PER_CELL / scan_avg_s / 1e12
-    sm_mhz_peak = (peaks or {}).get("sm_max_mhz", 1965.0)
-    alu_peak = 148 * 4 * 32 * sm_mhz_peak * 1e6 / 1e12
-    roofline = {"bound": "alu", "kernel": "fm_ssm_scan_pot (k_scan_prep + k_scan_seq)",
-                "achieved": achieved,
-                "peak": alu_peak, "unit": "Tops/s (int32)", "frac": achieved / alu_peak,
-                "traffic": None,
-                "peak_basis": f"148 SMs x 4 SMSPs x 32 lanes x 1 int op/clk x {sm_mhz_peak:.0f} MHz",
-                "avg_launch_us": 1e6 * scan_avg_s,
-                "share_of_step": sum(scan_ms) / sum(step_ms)}
-
-    # end to end through the public API: pinned host input -> device, 24 x
-    # fm_mixer_prefill, device -> pinned host output, every step
-    xh = torch.from_numpy(x_host).pin_memory()
-    oh = torch.empty_like(xh).pin_memory()
-    xd = torch.empty_like(x0)
-
-    def e2e_step():
-        xd.copy_(xh, non_blocking=True)
-        stack.prefill_(xd, ws=ws)
-        oh.copy_(xd, non_blocking=True)
-
+    # end to end through the public API: pinned host input -> device, the
+    # computation, device -> pinned host output, every step
+    wl.e2e_setup()
     for _ in range(2):
-        e2e_step()
+        wl.e2e_step()
     torch.cuda.synchronize()
     e2e_ms = []
     for _ in range(args.steps):
         flush.zero_()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
-        e2e_step()
+        wl.e2e_step()
         b.record(stream)
         torch.cuda.synchronize()
         e2e_ms.append(a.elapsed_time(b))
     lib.sync_status()
-    if not torch.equal(oh, ref.cpu()):
+    if ref is not None and not wl.e2e_matches(ref):
         raise SystemExit("bench: end-to-end output differs from the device-resident step")
-    e2e_t = torch.tensor([sum(e2e_ms)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
-    e2e_value = world * B * T * args.steps / (float(e2e_t.item()) / 1000.0)
-    nbytes = x_host.nbytes
+    e2e_total = max_over_ranks(torch, dist, world, sum(e2e_ms), dev)
+    e2e_value = world * wl.tokens * args.steps / (e2e_total / 1000.0)
 
     if rank == 0:
         cpu = None
         if not args.no_cpu_baseline and world == 1:
-            cpu = cpu_oracle_sample(shape, n_layers, args.mode)
-        line = {"metric": "W8A8 Mamba2 prefill tokens/s", "value": value, "unit": "tokens/s",
-                "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-                "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-                "vs_baseline": None, "dtype": "int8 GEMM (int32 acc) + int32 fixed point",
+            cpu = OracleSample(args.workload, args.mode, args.gemm_m).measure()
+        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "int8 x int8 -> int32 GEMM + int32 fixed point",
                 "data": "synthetic (seeded outlier-injected N(0,1), random-init weights)",
-                "config": config_block(args, shape, n_layers, B, T),
-                "roofline": roofline, "cpu_baseline": cpu, "clocks": clk,
-                "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": nbytes,
-                        "d2h_bytes_per_step": nbytes},
-                "gpu_launches": launches_per_step * args.steps,
-                "scan_ms_per_layer": statistics.mean(scan_ms)}
+                "config": config_block(args), "roofline": roofline, "cpu_baseline": cpu,
+                "clocks": clk,
+                "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": wl.h2d_bytes,
+                        "d2h_bytes_per_step": wl.d2h_bytes},
+                "gpu_launches": wl.launches * args.steps}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
