@@ -193,21 +193,59 @@ static fm_status launch_gemm_t(const CUtensorMap &ta, const CUtensorMap &tb, lon
   return launched("k_gemm_i8_tc");
 }
 
-// 128 x 128 tiles with a 3-stage ring (96 KB: two CTAs per SM, one's
-// epilogue overlapping the other's main loop); 128 x 64 tiles when the 128-wide
-// grid would leave SMs idle (small N, e.g. out_proj).
+template <int BN, int STAGES, int EW>
+static fm_status launch_gemm_persist(const CUtensorMap &ta, const CUtensorMap &tb, long long M,
+                                     long long N, long long K, int sms, const GemmEpilogue &ep,
+                                     cudaStream_t s) {
+  constexpr int smem = PersistSmem<BN, STAGES, EW>::kBytes;
+  static_assert(smem <= 227 * 1024, "shared memory per CTA");
+  auto kern = k_gemm_i8_persist<BN, STAGES, EW>;
+  FM_CHECK_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+  const int m_tiles = (int)((M + kGemmBM - 1) / kGemmBM), n_tiles = (int)((N + BN - 1) / BN);
+  const long long tiles = (long long)m_tiles * n_tiles;
+  const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);
+  kern<<<grid, 64 + 32 * EW, smem, s>>>(ta, tb, (int)(K / kGemmBK), m_tiles, n_tiles, ep);
+  return launched("k_gemm_i8_persist");
+}
+
+static int sm_count() {
+  constexpr int kMaxDevices = 64;
+  static int cache[kMaxDevices] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+  if (!cache[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+// Large problems: the persistent kernel, 128 x 256 tiles when there are at
+// least two per SM (fewer L2 bytes per MMA), else 128 x 128.  Small grids
+// (fewer 128-wide tiles than SMs, e.g. out_proj at 130M shapes or a decode
+// batch): one 128 x 64 tile per CTA, two CTAs per SM.
 static fm_status launch_gemm(const int8_t *A, long long M, const int8_t *W, long long N,
                              long long K, const GemmEpilogue &ep, cudaStream_t s) {
   if (K % kGemmBK) return fail(FM_ERR_SHAPE, "gemm: K=%lld is not a multiple of 128", K);
-  if ((M + kGemmBM - 1) / kGemmBM > 65535 || (N + 63) / 64 > 2147483647LL)
+  if ((M + kGemmBM - 1) / kGemmBM > 65535 || (N + 63) / 64 > 65535)
     return fail(FM_ERR_SHAPE, "gemm: M=%lld or N=%lld too large", M, N);
-  const long long tiles128 = ((N + 127) / 128) * ((M + kGemmBM - 1) / kGemmBM);
-  const bool narrow = tiles128 < 2 * 148;
+  const long long mt = (M + kGemmBM - 1) / kGemmBM;
+  const long long tiles256 = mt * ((N + 255) / 256), tiles128 = mt * ((N + 127) / 128);
+  const int sms = sm_count();
   CUtensorMap ta, tb;
   FM_TRY(make_tmap(&ta, A, M, K, kGemmBM));
-  FM_TRY(make_tmap(&tb, W, N, K, narrow ? 64 : 128));
-  if (narrow) return launch_gemm_t<64, 4>(ta, tb, M, N, K, ep, s);
-  return launch_gemm_t<128, 3>(ta, tb, M, N, K, ep, s);
+  if (tiles256 >= 2LL * sms) {
+    FM_TRY(make_tmap(&tb, W, N, K, 256));
+    return launch_gemm_persist<256, 4, 8>(ta, tb, M, N, K, sms, ep, s);
+  }
+  if (tiles128 >= sms) {
+    FM_TRY(make_tmap(&tb, W, N, K, 128));
+    return launch_gemm_persist<128, 6, 8>(ta, tb, M, N, K, sms, ep, s);
+  }
+  FM_TRY(make_tmap(&tb, W, N, K, 64));
+  return launch_gemm_t<64, 4>(ta, tb, M, N, K, ep, s);
 }
 
 static fm_status launch_hadamard_quant(const float *x, long long M, int K, const float *prenorm_w,
@@ -318,7 +356,7 @@ static fm_status launch_scan_v2(const ScanArgs &a, int B, const ScanWs &w, cudaS
   if (M == 0) return FM_OK;
   if (B > 65535 || M > 2147483647LL) return fail(FM_ERR_SHAPE, "scan: B or B*T too large");
   if (a.T == 1) {  // decode: one step per sequence, no staging
-    k_scan_step<<<dim3(a.hd / 8, a.nh, B), 256, 0, s>>>(a);
+    k_scan_step<<<dim3(a.nh, B), 256, 0, s>>>(a);
     return launched("k_scan_step");
   }
   const long long Tp = scan_tpad(a.T);

@@ -366,4 +366,200 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
   }
 }
 
+// ------------------------------------------------------------ the persistent kernel
+// One CTA per SM walks the output tiles (tile t = m_blk * n_tiles + n_blk,
+// strided by the grid), so the set/teardown cost is paid once and the
+// epilogue of tile i overlaps the main loop of tile i + 1: the accumulator is
+// double-buffered in TMEM (2 x BN int32 columns).
+//   warp 0          TMA producer (the smem ring runs across tile boundaries)
+//   warp 1          TMEM allocation; one lane issues tcgen05.mma, commits each
+//                   ring slot back to the producer and each finished
+//                   accumulator to the epilogue
+//   warps 2..2+EW   epilogue: EW / 4 warps per TMEM lane quarter, each taking
+//                   BN / (EW / 4) columns; the accumulator is handed back to
+//                   the MMA warp as soon as its last tcgen05.ld has completed
+// Barriers: full[s] / empty[s] for the ring, tfull[a] / tempty[a] for the two
+// accumulators.  Every wait is bounded; after a failed wait a thread stops
+// waiting (it still meets its named barriers), the MMA lane drains its
+// outstanding MMAs and the producer its outstanding copies before TMEM is
+// released, so the kernel always ends.
+template <int BN, int STAGES, int EW>
+struct PersistSmem {
+  static constexpr int kA = kGemmBM * kGemmBK;  // bytes per A stage
+  static constexpr int kB = BN * kGemmBK;       // bytes per B stage
+  static constexpr int kBytes = 1024 /*align slack*/ + STAGES * (kA + kB) +
+                                (2 * STAGES + 5) * 8 /*barriers*/ + 16 /*tmem slot*/ +
+                                4 * BN * 4 /*column scales, double-buffered*/;
+};
+
+template <int BN, int STAGES, int EW>
+__global__ void __launch_bounds__(64 + 32 * EW, 1)
+    k_gemm_i8_persist(const __grid_constant__ CUtensorMap tmA,
+                      const __grid_constant__ CUtensorMap tmB, int num_k_blocks, int m_tiles,
+                      int n_tiles, GemmEpilogue ep) {
+  static_assert(BN % 32 == 0 && BN >= 64 && BN <= 256, "BN");
+  static_assert(EW % 4 == 0 && (BN / (EW / 4)) % 32 == 0, "epilogue split");
+  using Sm = PersistSmem<BN, STAGES, EW>;
+  constexpr int kEpiThreads = 32 * EW;
+  constexpr int kColsPerWarp = BN / (EW / 4);
+  constexpr uint32_t kTmemCols = 2 * BN;  // a power of two >= 32 for BN in {64, 128, 256}
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~static_cast<uintptr_t>(1023));
+  uint8_t *sA = smem;
+  uint8_t *sB = smem + STAGES * Sm::kA;
+  uint64_t *full_bar = reinterpret_cast<uint64_t *>(sB + STAGES * Sm::kB);
+  uint64_t *empty_bar = full_bar + STAGES;
+  uint64_t *tfull = empty_bar + STAGES;   // [2]
+  uint64_t *tempty = tfull + 2;           // [2]
+  uint64_t *drain_bar = tempty + 2;       // [1]
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain_bar + 1);
+  float *col_w = reinterpret_cast<float *>((reinterpret_cast<uintptr_t>(tmem_slot + 1) + 15) &
+                                           ~static_cast<uintptr_t>(15));  // [2][BN]
+  float *col_e = col_w + 2 * BN;                                          // [2][BN]
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int num_tiles = m_tiles * n_tiles;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < STAGES; ++i) {
+      mbar_init(&full_bar[i], 1);
+      mbar_init(&empty_bar[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tfull[i], 1);
+      mbar_init(&tempty[i], EW);
+    }
+    mbar_init(drain_bar, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"((unsigned long long)&tmA) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"((unsigned long long)&tmB) : "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      long long it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        const int m0 = (t / n_tiles) * kGemmBM, n0 = (t % n_tiles) * BN;
+        for (int kb = 0; kb < num_k_blocks; ++kb, ++it) {
+          const int s = (int)(it % STAGES);
+          const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+          if (!mbar_wait(&empty_bar[s], ph ^ 1u)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full_bar[s], (uint32_t)(Sm::kA + Sm::kB));
+          tma_load_2d(sA + s * Sm::kA, &tmA, kb * kGemmBK, m0, &full_bar[s]);
+          tma_load_2d(sB + s * Sm::kB, &tmB, kb * kGemmBK, n0, &full_bar[s]);
+        }
+      }
+      // every copy issued must have landed before the CTA may exit (on the
+      // normal path the MMA lane has consumed them all and these return at once)
+      const long long first = it > STAGES ? it - STAGES : 0;
+      for (long long j = first; j < it; ++j)
+        if (!mbar_wait(&full_bar[j % STAGES], (uint32_t)(j / STAGES) & 1u)) break;
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = i8_idesc(kGemmBM, BN);
+      long long it = 0;
+      int tl = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x, ++tl) {
+        const int acc = tl & 1;
+        const uint32_t use = (uint32_t)(tl >> 1);
+        if (!mbar_wait(&tempty[acc], (use & 1u) ^ 1u)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d = tmem_base + (uint32_t)(acc * BN);
+        for (int kb = 0; kb < num_k_blocks; ++kb, ++it) {
+          const int s = (int)(it % STAGES);
+          const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+          if (!mbar_wait(&full_bar[s], ph)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t ad = sw128_desc(smem_u32(sA + s * Sm::kA));
+          const uint64_t bd = sw128_desc(smem_u32(sB + s * Sm::kB));
+#pragma unroll
+          for (int k = 0; k < kGemmBK / 32; ++k)
+            mma_i8(d, ad + (uint64_t)(2 * k), bd + (uint64_t)(2 * k), idesc,
+                   (kb > 0 || k > 0) ? 1u : 0u);
+          mma_commit(&empty_bar[s]);
+        }
+        if (ok) mma_commit(&tfull[acc]);
+      }
+      // wait for every MMA issued so far before TMEM can be released
+      mma_commit(drain_bar);
+      mbar_wait(drain_bar, 0);
+    }
+  } else {
+    const int e = warp - 2;                 // 0 .. EW-1
+    const int quarter = warp & 3;           // TMEM lanes [32 quarter, 32 quarter + 32)
+    const int part = e / 4;                 // which column slice of the tile
+    const int et = threadIdx.x - 64;        // 0 .. kEpiThreads-1
+    int tl = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++tl) {
+      const int acc = tl & 1;
+      const uint32_t use = (uint32_t)(tl >> 1);
+      const int m0 = (t / n_tiles) * kGemmBM, n0 = (t % n_tiles) * BN;
+      float *cw = col_w + acc * BN, *ce = col_e + acc * BN;
+      // this tile's column scales (buffer acc was last read two tiles ago,
+      // before every epilogue warp passed the previous tile's barrier)
+      for (int j = et; j < BN; j += kEpiThreads) {
+        const long long c = (long long)n0 + j;
+        cw[j] = c < ep.N ? ep.s_w[c] : 0.0f;
+        float ev = 0.0f;
+        if (ep.mode == 1 && c >= ep.di && c < (long long)ep.di + ep.cc) ev = pow2f(-ep.e_u[c - ep.di]);
+        ce[j] = ev;
+      }
+      const long long row = (long long)m0 + quarter * 32 + lane;
+      const float sx = row < ep.M ? ep.s_x[row] : 0.0f;
+      asm volatile("bar.sync 1, %0;" ::"r"(kEpiThreads) : "memory");
+      if (ok) ok = mbar_wait(&tfull[acc], use & 1u);
+      ok = __all_sync(0xffffffffu, ok);  // tcgen05.ld below is warp-collective
+      tc_fence_after();
+      const int c_begin = part * kColsPerWarp;
+#pragma unroll 1
+      for (int c = c_begin; c < c_begin + kColsPerWarp; c += 32) {
+        uint32_t r[32];
+        if (ok) {
+          tmem_ld32(tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN + c), r);
+          if (c + 32 >= c_begin + kColsPerWarp) {  // last load of this warp: hand the buffer back
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tempty[acc]);
+          }
+          if (n0 + c < ep.N) gemm_store_chunk(ep, row, sx, (long long)n0 + c, r, cw + c, ce + c);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"(kTmemCols)
+                 : "memory");
+  }
+}
+
 }  // namespace fm

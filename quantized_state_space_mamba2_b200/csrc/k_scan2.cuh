@@ -389,59 +389,75 @@ __global__ void __launch_bounds__(PC *(128 / NPT) + 32) k_scan_seq(ScanSeqArgs a
 
 // Decode (T == 1): one recurrence step per sequence (state null: zeros, not
 // written back).  The step reads and rewrites the whole state once, so HBM
-// bandwidth bounds it; one warp per channel p, each lane owning 4 consecutive
-// state columns (one 16-byte load and store), the C.h sum reduced by shuffles
-// in the split (hi, lo) 32-bit form.  Same arithmetic as one step of
-// k_scan_seq with the clamp.  Grid (hd / 8, nh, B), block 256.
+// bandwidth bounds it.  One CTA per (head, sequence) covers all hd = 64
+// channels: warp w owns channels w, w + 8, ..., w + 56 and lane l the state
+// columns 4l .. 4l + 3, so each thread has eight 16-byte state loads in flight
+// (32 KB per CTA, read and written once with streaming cache hints).  The
+// C.h sums are reduced by shuffles in the split (hi, lo) 32-bit form.  Same
+// arithmetic as one step of k_scan_seq with the clamp.  Grid (nh, B), block 256.
+constexpr int kStepPPW = 8;  // channels per warp (hd / 8 warps)
+
 __global__ void __launch_bounds__(256) k_scan_step(ScanArgs a) {
-  __shared__ int tab[8];
-  pwl_table_init(tab);
-  __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int h = blockIdx.y, b = blockIdx.z;
-  const int p = blockIdx.x * 8 + warp;
-  const int n0 = lane * 4;
+  const int h = blockIdx.x, b = blockIdx.y;
   const int nh = a.nh, hd = a.hd, cc = a.cc, di = a.di;
+  const int n0 = lane * 4;
+  const long long headrow = (long long)b * nh + h;
+  int4 *st = a.state ? reinterpret_cast<int4 *>(a.state + headrow * hd * 128) : nullptr;
+  int4 hv[kStepPPW];
+#pragma unroll
+  for (int k = 0; k < kStepPPW; ++k)
+    hv[k] = st ? __ldcs(st + (warp + 8 * k) * 32 + lane) : make_int4(0, 0, 0, 0);
   const int8_t *row = a.xbc + (long long)b * cc;
-  const int e_x = a.e_x[h], e_B = *a.e_B, e_C = *a.e_C, e_h = a.e_h[h], e_y = a.e_y[h];
-  const int e_D = a.e_D[h];
-  const float xf = __fadd_rn(a.dt_raw[(long long)b * nh + h], a.dt_bias[h]);
-  const int dtq = softplus_pwl(to_q16(xf));
-  const int dA = pow2_pwl(-rshr64((long long)dtq * a.A_q[h], 12));
-  const long long xq = row[h * hd + p];
-  const int u = (int)satb64(rshr64((long long)dtq * xq, e_h - e_B - e_x + 16), 24);
   const uint32_t bw = *reinterpret_cast<const uint32_t *>(row + di + n0);
   const uint32_t cw = *reinterpret_cast<const uint32_t *>(row + di + 128 + n0);
-  int32_t *st = a.state ? a.state + ((((long long)b * nh + h) * hd + p) * 128 + n0) : nullptr;
-  const int4 hv = st ? *reinterpret_cast<const int4 *>(st) : make_int4(0, 0, 0, 0);
-  const int hs[4] = {hv.x, hv.y, hv.z, hv.w};
-  int hn[4];
-  int ahi = 0, alo = 0;
+  int8_t xs[kStepPPW];
+#pragma unroll
+  for (int k = 0; k < kStepPPW; ++k) xs[k] = row[h * hd + warp + 8 * k];
+  const int e_x = a.e_x[h], e_B = *a.e_B, e_C = *a.e_C, e_h = a.e_h[h], e_y = a.e_y[h];
+  const int e_D = a.e_D[h];
+  const long long Dq = a.D_q[h];
+  const float xf = __fadd_rn(a.dt_raw[headrow], a.dt_bias[h]);
+  const int dtq = softplus_pwl(to_q16(xf));
+  const int dA = pow2_pwl(-rshr64((long long)dtq * a.A_q[h], 12));
+  const int s_h = e_h - e_B - e_x + 16, s_y = e_y - e_C - e_h, s_D = e_y - e_D - e_x;
+  int Bv[4], Cv[4];
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
-    const int Bj = (int)(int8_t)((bw >> (8 * j)) & 0xFF);
-    const int Cj = (int)(int8_t)((cw >> (8 * j)) & 0xFF);
-    const int hh = hs[j] >> 16;
-    const unsigned hl = (unsigned)hs[j] & 0xFFFFu;
-    const unsigned t = (unsigned)dA * hl + 0x8000u;
-    int v = dA * hh + (int)(t >> 16) + u * Bj;
-    v = min(max(v, -(int)kHLim), (int)kHLim);
-    hn[j] = v;
-    ahi += Cj * (v >> 16);
-    alo += Cj * (int)((unsigned)v & 0xFFFFu);
+    Bv[j] = (int)(int8_t)((bw >> (8 * j)) & 0xFF);
+    Cv[j] = (int)(int8_t)((cw >> (8 * j)) & 0xFF);
   }
-  if (st) *reinterpret_cast<int4 *>(st) = make_int4(hn[0], hn[1], hn[2], hn[3]);
+  int yv = 0;  // lane k (< 8) ends up holding channel warp + 8k's output
 #pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) {
-    ahi += __shfl_xor_sync(0xffffffffu, ahi, o);
-    alo += __shfl_xor_sync(0xffffffffu, alo, o);
-  }
-  if (lane == 0) {
+  for (int k = 0; k < kStepPPW; ++k) {
+    const long long xq = xs[k];
+    const int u = (int)satb64(rshr64((long long)dtq * xq, s_h), 24);
+    const int hs[4] = {hv[k].x, hv[k].y, hv[k].z, hv[k].w};
+    int hn[4];
+    int ahi = 0, alo = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int hh = hs[j] >> 16;
+      const unsigned hl = (unsigned)hs[j] & 0xFFFFu;
+      const unsigned t = (unsigned)dA * hl + 0x8000u;
+      int v = dA * hh + (int)(t >> 16) + u * Bv[j];
+      v = min(max(v, -(int)kHLim), (int)kHLim);
+      hn[j] = v;
+      ahi += Cv[j] * (v >> 16);
+      alo += Cv[j] * (int)((unsigned)v & 0xFFFFu);
+    }
+    if (st) __stcs(st + (warp + 8 * k) * 32 + lane, make_int4(hn[0], hn[1], hn[2], hn[3]));
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+      ahi += __shfl_xor_sync(0xffffffffu, ahi, o);
+      alo += __shfl_xor_sync(0xffffffffu, alo, o);
+    }
     const long long sum = (long long)ahi * 65536 + alo;
-    const int dx = (int)satb64(rshr64((long long)a.D_q[h] * xq, e_y - e_D - e_x), 32);
-    a.y[(long long)b * di + (long long)h * hd + p] =
-        (int)satb64(rshr64(sum, e_y - e_C - e_h) + dx, 32);
+    const int dx = (int)satb64(rshr64(Dq * xq, s_D), 32);
+    const int yk = (int)satb64(rshr64(sum, s_y) + dx, 32);
+    if (lane == k) yv = yk;
   }
+  if (lane < kStepPPW) a.y[(long long)b * di + (long long)h * hd + warp + 8 * lane] = yv;
 }
 
 }  // namespace fm

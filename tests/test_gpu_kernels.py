@@ -130,6 +130,59 @@ def test_w8a8_gemm(L, M, N, K):
     L.sync_status()
 
 
+def _sample_rows(M, step=7, tail=130):
+    return np.unique(np.concatenate([np.arange(0, M, step), np.arange(max(0, M - tail), M)]))
+
+
+@pytest.mark.parametrize("M,N,K", [(2093, 3352, 768), (4173, 10576, 2560), (8192, 2560, 5120)])
+def test_w8a8_gemm_persistent(L, M, N, K):
+    """Grids with at least one 128-wide tile per SM run the persistent kernel
+    (128 x 128 tiles; 128 x 256 from two tiles per SM on; accumulators
+    double-buffered in TMEM, ring and tiles carried across the CTA's tiles).
+    Ragged M and N; every 7th row and the last 130 rows (the partial tile)
+    compared bit for bit."""
+    A = S.uniform_ints((M, K), -127, 127, seed=M + K, dtype=np.int8)
+    W = S.uniform_ints((N, K), -127, 127, seed=N + K, dtype=np.int8)
+    sx = np.abs(S.normal(M, 0.01, seed=7)) + 1e-3
+    sw = np.abs(S.normal(N, 0.001, seed=8)) + 1e-4
+    res = S.normal((M, N), 1.0, seed=9)
+    rows = _sample_rows(M)
+    ref = (A[rows].astype(np.float64) @ W.astype(np.float64).T).astype(np.int64)  # exact: |acc| < 2^53
+    Y = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    acc = torch.empty((M, N), dtype=torch.int32, device="cuda")
+    L.w8a8_gemm(dev(A), dev(sx), dev(W), dev(sw), Y, None, acc)
+    assert np.array_equal(host(acc)[rows], ref)
+    assert np.array_equal(host(Y)[rows], O.dequant(ref.astype(np.int32), sx[rows], sw))
+    Yr = dev(res)
+    L.w8a8_gemm(dev(A), dev(sx), dev(W), dev(sw), Yr, Yr, None)
+    assert np.array_equal(host(Yr)[rows],
+                          O.dequant(ref.astype(np.int32), sx[rows], sw, residual=res[rows]))
+    L.sync_status()
+
+
+def test_in_proj_split_2p7b_full_size(L):
+    """The in_proj split epilogue at the 2.7B shapes and 8192 tokens (the
+    persistent 128 x 256 kernel), sampled rows bit for bit."""
+    s, M = S.MAMBA2_2P7B, 8192
+    A = S.uniform_ints((M, s.d_model), -127, 127, seed=21, dtype=np.int8)
+    W = S.uniform_ints((s.n_in, s.d_model), -127, 127, seed=22, dtype=np.int8)
+    sx = np.abs(S.normal(M, 0.01, seed=23)) + 1e-3
+    sw = np.abs(S.normal(s.n_in, 3e-3, seed=24)) + 1e-4
+    e_u = S.uniform_ints(s.conv_ch, -6, -2, seed=25)
+    exps = np.zeros(L.exp_table_layout(s).size, np.int32)
+    exps[:s.conv_ch] = e_u
+    z = torch.empty((M, s.d_inner), dtype=torch.float32, device="cuda")
+    xbc = torch.empty((M, s.conv_ch), dtype=torch.int8, device="cuda")
+    dt = torch.empty((M, s.nheads), dtype=torch.float32, device="cuda")
+    L.in_proj(dev(A), dev(sx), dev(W), dev(sw), s, dev(exps), z, xbc, dt)
+    rows = _sample_rows(M, step=13)
+    acc = (A[rows].astype(np.float64) @ W.astype(np.float64).T).astype(np.int32)
+    zr, xr, dr = O.in_proj_epilogue(acc, sx[rows], sw, s.d_inner, s.conv_ch, s.nheads, e_u)
+    assert np.array_equal(host(z)[rows], zr)
+    assert np.array_equal(host(xbc)[rows], xr)
+    assert np.array_equal(host(dt)[rows], dr)
+
+
 @pytest.mark.parametrize("M", [5, 256, 1000])
 def test_in_proj_split(L, M):
     s = MAMBA130
