@@ -16,11 +16,14 @@
 //                PC consecutive p); NPT consecutive n of one p per thread,
 //                state in registers.  One elected thread fetches each chunk
 //                of TCH steps with a handful of bulk copies (cp.async.bulk on
-//                an mbarrier) into a three-slot shared-memory ring up to two
-//                chunks ahead, so the other threads issue no load instructions and
-//                no global latency sits on the recurrence; the C.h partial
-//                sums of a chunk stay in registers and are added across the
-//                p's threads once per chunk through padded shared memory.
+//                an mbarrier) into a two-slot shared-memory ring one chunk
+//                ahead, so the other threads issue no load instructions and
+//                no global latency sits on the recurrence.  The C.h sums:
+//                with one channel per warp (NPT = 4) each step's per-thread
+//                partials are added over the warp by redux.sync; otherwise a
+//                chunk's partials stay in registers and are added across the
+//                channel's threads once per chunk through padded shared
+//                memory.
 // Per state cell and step the loop issues, in 32-bit integer arithmetic on the
 // split state h = hh 2^16 + hl: the rounded decay (two multiplies, a shift),
 // the multiply-add of u B, the clamp (two min/max, skipped where a chunk
@@ -154,7 +157,7 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
       : "memory");
 }
 
-constexpr int kScanSlots = 3;  // chunks in flight in the shared-memory ring
+constexpr int kScanSlots = 2;  // chunks in flight in the shared-memory ring
 
 template <int NPT, int PC, int TCH>
 struct ScanSeqSmem {
@@ -162,7 +165,9 @@ struct ScanSeqSmem {
   static constexpr int NW = PC * LPP / 32;       // compute warps
   // int2 per partial row: LPP + 1 (rows an odd number of 8-byte words apart)
   // keeps the per-row reads of a half-warp on distinct banks
-  static constexpr int PSTRIDE = LPP + 1;
+  // (with one channel per warp the per-step sums come from redux.sync and
+  // only 16 int2 per warp are staged)
+  static constexpr int PSTRIDE = LPP == 32 ? 1 : LPP + 1;
   struct Slot {
     int32_t bc[TCH][256];
     int32_t dA[TCH];
@@ -219,14 +224,34 @@ __device__ __forceinline__ int2 scan_one_step(int (&hh)[NPT], unsigned (&hl)[NPT
   return make_int2(ahi, alo);
 }
 
-template <int NPT, int TCH, bool FULL, bool CLAMP>
+// The (C hh, C hl) partial sums of step tt go to part[tt] (REDUX = false), or
+// -- when one warp is one channel (32 threads per channel) -- are summed over
+// the warp at once (redux.sync) and lane 0 stores the step's sums to
+// wsum[tt] (REDUX = true): no per-step partials are kept in registers.
+template <int NPT, int TCH, bool FULL, bool CLAMP, bool REDUX>
 __device__ __forceinline__ void scan_chunk_steps(int (&hh)[NPT], unsigned (&hl)[NPT],
-                                                 int2 (&part)[TCH], const int32_t (*bc)[256],
-                                                 const int32_t *dAv, const int32_t *uv, int n0,
-                                                 int nt) {
+                                                 int2 (&part)[TCH], int2 *wsum,
+                                                 const int32_t (*bc)[256], const int32_t *dAv,
+                                                 const int32_t *uv, int n0, int nt) {
   // two register sets for B / C: the even step's set is refilled two steps
   // ahead while the odd step computes, and vice versa (no copies)
   int B0[NPT], C0[NPT], B1[NPT], C1[NPT];
+  const bool lead = (threadIdx.x & 31) == 0;
+  // a step's sums are stored one step later, so the warp never waits on the
+  // reduction's latency
+  int2 pend = make_int2(0, 0);
+  int pend_tt = -1;
+  auto emit = [&](int tt, int2 v) {
+    if constexpr (REDUX) {
+      const int shi = __reduce_add_sync(0xffffffffu, v.x);
+      const int slo = __reduce_add_sync(0xffffffffu, v.y);
+      if (lead && pend_tt >= 0) wsum[pend_tt] = pend;
+      pend = make_int2(shi, slo);
+      pend_tt = tt;
+    } else {
+      part[tt] = v;
+    }
+  };
   load_bc<NPT>(bc, 0, n0, B0, C0);
 #pragma unroll
   for (int tg = 0; tg < TCH; tg += 4) {
@@ -238,13 +263,16 @@ __device__ __forceinline__ void scan_chunk_steps(int (&hh)[NPT], unsigned (&hl)[
     for (int k = 0; k < 4; k += 2) {
       const int tt = tg + k;
       if (FULL || tt + 1 < nt) load_bc<NPT>(bc, tt + 1, n0, B1, C1);
-      if (FULL || tt < nt) part[tt] = scan_one_step<NPT, CLAMP>(hh, hl, B0, C0, dAs[k], us[k]);
-      else part[tt] = make_int2(0, 0);
+      if (FULL || tt < nt) emit(tt, scan_one_step<NPT, CLAMP>(hh, hl, B0, C0, dAs[k], us[k]));
+      else if constexpr (!REDUX) part[tt] = make_int2(0, 0);
       if (tt + 2 < TCH && (FULL || tt + 2 < nt)) load_bc<NPT>(bc, tt + 2, n0, B0, C0);
       if (FULL || tt + 1 < nt)
-        part[tt + 1] = scan_one_step<NPT, CLAMP>(hh, hl, B1, C1, dAs[k + 1], us[k + 1]);
-      else part[tt + 1] = make_int2(0, 0);
+        emit(tt + 1, scan_one_step<NPT, CLAMP>(hh, hl, B1, C1, dAs[k + 1], us[k + 1]));
+      else if constexpr (!REDUX) part[tt + 1] = make_int2(0, 0);
     }
+  }
+  if constexpr (REDUX) {
+    if (lead && pend_tt >= 0) wsum[pend_tt] = pend;
   }
 }
 
@@ -260,6 +288,7 @@ __global__ void __launch_bounds__(PC *(128 / NPT) + 32) k_scan_seq(ScanSeqArgs a
   constexpr int PPW = 32 / LPP;  // channels per warp
   static_assert(LPP <= 32 && 32 % LPP == 0, "a channel's threads stay inside one warp");
   static_assert(TCH == 16, "the growth bounds are per 16-step chunk");
+  constexpr bool REDUX = (LPP == 32);
   using Sm = ScanSeqSmem<NPT, PC, TCH>;
   constexpr int PSTRIDE = Sm::PSTRIDE;
   extern __shared__ __align__(16) uint8_t smem_raw[];
@@ -343,11 +372,26 @@ __global__ void __launch_bounds__(PC *(128 / NPT) + 32) k_scan_seq(ScanSeqArgs a
     for (int j = 0; j < NPT; ++j) hmax = max(hmax, abs((int)(((unsigned)hh[j] << 16) | hl[j])));
     const bool no_clamp = __all_sync(0xffffffffu, (long long)hmax + s.bound[pp] <= kHLim);
     int2 pr[TCH];
+    int2 *wsum = reinterpret_cast<int2 *>(&part[0][0]);
     if (nt == TCH) {
-      if (no_clamp) scan_chunk_steps<NPT, TCH, true, false>(hh, hl, pr, s.bc, s.dA, s.u[pp], n0, nt);
-      else scan_chunk_steps<NPT, TCH, true, true>(hh, hl, pr, s.bc, s.dA, s.u[pp], n0, nt);
+      if (no_clamp)
+        scan_chunk_steps<NPT, TCH, true, false, REDUX>(hh, hl, pr, wsum, s.bc, s.dA, s.u[pp], n0, nt);
+      else
+        scan_chunk_steps<NPT, TCH, true, true, REDUX>(hh, hl, pr, wsum, s.bc, s.dA, s.u[pp], n0, nt);
     } else {
-      scan_chunk_steps<NPT, TCH, false, true>(hh, hl, pr, s.bc, s.dA, s.u[pp], n0, nt);
+      scan_chunk_steps<NPT, TCH, false, true, REDUX>(hh, hl, pr, wsum, s.bc, s.dA, s.u[pp], n0, nt);
+    }
+    if constexpr (REDUX) {  // one channel per warp: lane tt finishes step tt
+      __syncwarp();
+      if (lane32 < nt) {
+        const int2 v = wsum[lane32];
+        const long long sum = (long long)v.x * 65536 + v.y;
+        a.y[(rowbase + t0 + lane32) * di + (long long)h * hd + p0 + pp] =
+            (int)satb64(rshr64(sum, s_y) + s.dx[pp][lane32], 32);
+      }
+      __syncwarp();
+      if (lane32 == 0) mbar_arrive(&sm.empty[sl]);
+      continue;
     }
     // partials of this warp: row (step, channel-in-warp), column = lane in channel
 #pragma unroll
