@@ -345,7 +345,7 @@ static fm_status launch_seq(const ScanSeqArgs &a, int B, cudaStream_t s) {
 struct ScanWs {
   int32_t *dA;  // [B, nh, Tp]
   int32_t *u;   // [B, nh, hd, Tp]
-  int32_t *dx;  // [B, nh, hd, Tp]
+  int32_t *xs;  // [B, nh, hd, Tp]: x codes, widened
   int32_t *bc;  // [B*T, 256]
   long long *bound;  // [B, nh, Tp/16, hd]
 };
@@ -378,7 +378,7 @@ static fm_status launch_scan_v2(const ScanArgs &a, int B, const ScanWs &w, cudaS
   p.e_D = a.e_D;
   p.dA = w.dA;
   p.u = w.u;
-  p.dx = w.dx;
+  p.xs = w.xs;
   p.bc = w.bc;
   p.bound = w.bound;
   k_scan_prep<<<dim3((unsigned)(Tp / kPrepTT), a.nh, B), 256, 0, s>>>(p);
@@ -386,7 +386,10 @@ static fm_status launch_scan_v2(const ScanArgs &a, int B, const ScanWs &w, cudaS
   ScanSeqArgs q;
   q.dA = w.dA;
   q.u = w.u;
-  q.dx = w.dx;
+  q.xs = w.xs;
+  q.D_q = a.D_q;
+  q.e_x = a.e_x;
+  q.e_D = a.e_D;
   q.bc = w.bc;
   q.bound = w.bound;
   q.T = a.T;
@@ -551,14 +554,14 @@ ScanWs carve_scan(Carver &c, const Dims &d, int B, int T) {
   ScanWs w;
   if (T == 1) {  // single steps run k_scan_step, which stages nothing
     w.dA = nullptr;
-    w.u = w.dx = w.bc = nullptr;
+    w.u = w.xs = w.bc = nullptr;
     w.bound = nullptr;
     return w;
   }
   const long long Tp = scan_tpad(T), M = (long long)B * T;
   w.dA = c.take<int32_t>((long long)B * d.nh * Tp);
   w.u = c.take<int32_t>((long long)B * d.di * Tp);
-  w.dx = c.take<int32_t>((long long)B * d.di * Tp);
+  w.xs = c.take<int32_t>((long long)B * d.di * Tp);
   w.bc = c.take<int32_t>(M * 256);
   w.bound = c.take<long long>((long long)B * d.di * (Tp / 16));
   return w;

@@ -8,8 +8,8 @@
 //  k_scan_prep   parallel over (32-token tile, head, batch): per (token, head)
 //                the fixed-point dt_q and dA_q; per (token, channel p) the
 //                state input factor u = satb(rshr(dt_q x, s_h), 24) and the
-//                skip term rshr(D_q x, s_D); B and C widened to int32.  dA,
-//                u and the skip term are written head-major and time-
+//                x code itself (for the skip term); B and C widened to
+//                int32.  dA, u and x are written head-major and time-
 //                contiguous ([B, nh, (hd,) Tp], Tp = T rounded up to 32) so a
 //                chunk of one head / channel is one contiguous run.
 //  k_scan_seq    the time-sequential part only.  One CTA per (batch, head,
@@ -49,7 +49,7 @@ struct ScanPrepArgs {
   const int32_t *e_x, *e_B, *e_h, *e_y, *e_D;
   int32_t *dA;   // [B, nh, Tp]
   int32_t *u;    // [B, nh, hd, Tp]
-  int32_t *dx;   // [B, nh, hd, Tp]
+  int32_t *xs;   // [B, nh, hd, Tp]: the x code, widened
   int32_t *bc;   // [B*T, 256]: B then C, int32
   long long *bound;  // [B, nh, Tp/16, hd]: per 16-step chunk, sum of |u| max|B|
 };
@@ -100,17 +100,15 @@ __global__ void __launch_bounds__(256) k_scan_prep(ScanPrepArgs a) {
     *reinterpret_cast<uint2 *>(&sx[tt][k * 8]) = v;
   }
   __syncthreads();
-  {  // (u, skip) for channel p = tid / 4, tokens 8 * (tid % 4) .. + 8
+  {  // (u, x) for channel p = tid / 4, tokens 8 * (tid % 4) .. + 8
     const int p = tid >> 2, tb = (tid & 3) * 8;
     const int s_h = a.e_h[h] - *a.e_B - a.e_x[h] + 16;
-    const int s_D = a.e_y[h] - a.e_D[h] - a.e_x[h];
-    const long long Dq = a.D_q[h];
     int uv[8], dv[8];
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
       const long long x = sx[tb + k][p];
       uv[k] = (int)satb64(rshr64((long long)s_dtq[tb + k] * x, s_h), 24);
-      dv[k] = (int)satb64(rshr64(Dq * x, s_D), 32);
+      dv[k] = (int)x;
     }
     // growth bound of |h| over this thread's 8 steps; two threads make a 16-step chunk
     long long gb = 0;
@@ -122,8 +120,8 @@ __global__ void __launch_bounds__(256) k_scan_prep(ScanPrepArgs a) {
     const long long off = (((long long)b * nh + h) * hd + p) * Tp + t0 + tb;
     *reinterpret_cast<int4 *>(a.u + off) = make_int4(uv[0], uv[1], uv[2], uv[3]);
     *reinterpret_cast<int4 *>(a.u + off + 4) = make_int4(uv[4], uv[5], uv[6], uv[7]);
-    *reinterpret_cast<int4 *>(a.dx + off) = make_int4(dv[0], dv[1], dv[2], dv[3]);
-    *reinterpret_cast<int4 *>(a.dx + off + 4) = make_int4(dv[4], dv[5], dv[6], dv[7]);
+    *reinterpret_cast<int4 *>(a.xs + off) = make_int4(dv[0], dv[1], dv[2], dv[3]);
+    *reinterpret_cast<int4 *>(a.xs + off + 4) = make_int4(dv[4], dv[5], dv[6], dv[7]);
   }
   // widened B and C rows of these tokens: the CTAs of the tile share the work
   for (int i = h * 256 + tid; i < nt * 64; i += nh * 256) {
@@ -139,11 +137,12 @@ __global__ void __launch_bounds__(256) k_scan_prep(ScanPrepArgs a) {
 struct ScanSeqArgs {
   const int32_t *dA;  // [B, nh, Tp]
   const int32_t *u;   // [B, nh, hd, Tp]
-  const int32_t *dx;  // [B, nh, hd, Tp]
+  const int32_t *xs;  // [B, nh, hd, Tp]
   const int32_t *bc;  // [B*T, 256]
   const long long *bound;  // [B, nh, Tp/16, hd]
   int T, nh, hd, di;
-  const int32_t *e_C, *e_h, *e_y;
+  const int32_t *D_q;
+  const int32_t *e_x, *e_C, *e_h, *e_y, *e_D;
   int32_t *state;     // [B, nh, hd, 128] or null
   int32_t *y;         // [B*T, di]
 };
@@ -172,7 +171,7 @@ struct ScanSeqSmem {
     int32_t bc[TCH][256];
     int32_t dA[TCH];
     int32_t u[PC][TCH];
-    int32_t dx[PC][TCH];
+    int32_t xs[PC][TCH];
     long long bound[PC];
   };
   Slot slot[kScanSlots];
@@ -335,7 +334,7 @@ __global__ void __launch_bounds__(PC *(128 / NPT) + 32) k_scan_seq(ScanSeqArgs a
         for (int q = 0; q < PC; ++q) {
           const long long off = (headrow * hd + p0 + q) * Tp + t0;
           bulk_g2s(&s.u[q][0], a.u + off, TCH * 4, &sm.full[sl]);
-          bulk_g2s(&s.dx[q][0], a.dx + off, TCH * 4, &sm.full[sl]);
+          bulk_g2s(&s.xs[q][0], a.xs + off, TCH * 4, &sm.full[sl]);
         }
       }
     }
@@ -348,6 +347,8 @@ __global__ void __launch_bounds__(PC *(128 / NPT) + 32) k_scan_seq(ScanSeqArgs a
   const int n0 = lane * NPT;
   const int wp = pp % PPW;           // channel within the warp
   const int s_y = a.e_y[h] - *a.e_C - a.e_h[h];
+  const int s_D = a.e_y[h] - a.e_D[h] - a.e_x[h];
+  const long long Dq = a.D_q[h];
   int hh[NPT];
   unsigned hl[NPT];
   int32_t *st = a.state ? a.state + (((headrow * hd) + p0 + pp) * 128 + n0) : nullptr;
@@ -387,40 +388,38 @@ __global__ void __launch_bounds__(PC *(128 / NPT) + 32) k_scan_seq(ScanSeqArgs a
         const int2 v = wsum[lane32];
         const long long sum = (long long)v.x * 65536 + v.y;
         a.y[(rowbase + t0 + lane32) * di + (long long)h * hd + p0 + pp] =
-            (int)satb64(rshr64(sum, s_y) + s.dx[pp][lane32], 32);
+            (int)satb64(rshr64(sum, s_y) + rshr64(Dq * s.xs[pp][lane32], s_D), 32);
       }
+    } else {
+      // partials of this warp: row (step, channel-in-warp), column = lane in channel
+#pragma unroll
+      for (int tt = 0; tt < TCH; ++tt) part[tt * PPW + wp][lane] = pr[tt];
       __syncwarp();
-      if (lane32 == 0) mbar_arrive(&sm.empty[sl]);
-      continue;
-    }
-    // partials of this warp: row (step, channel-in-warp), column = lane in channel
+      // lane r sums row r over the channel's LPP lanes (int32: |sum C hh| < 2^28,
+      // |sum C hl| < 2^30), lanes sharing a row combine by shuffles
+      constexpr int ROWS = TCH * PPW;
+      static_assert(ROWS <= 32 && 32 % ROWS == 0, "rows map onto the warp's lanes");
+      constexpr int SPLIT = 32 / ROWS;  // lanes sharing a row
+      constexpr int PER = LPP / SPLIT;
+      const int row = lane32 % ROWS, half = lane32 / ROWS;
+      int shi = 0, slo = 0;
 #pragma unroll
-    for (int tt = 0; tt < TCH; ++tt) part[tt * PPW + wp][lane] = pr[tt];
-    __syncwarp();
-    // lane r sums row r over the channel's LPP lanes (int32: |sum C hh| < 2^28,
-    // |sum C hl| < 2^30), lanes sharing a row combine by shuffles
-    constexpr int ROWS = TCH * PPW;
-    static_assert(ROWS <= 32 && 32 % ROWS == 0, "rows map onto the warp's lanes");
-    constexpr int SPLIT = 32 / ROWS;  // lanes sharing a row
-    constexpr int PER = LPP / SPLIT;
-    const int row = lane32 % ROWS, half = lane32 / ROWS;
-    int shi = 0, slo = 0;
+      for (int l = 0; l < PER; ++l) {
+        const int2 v = part[row][half * PER + l];
+        shi += v.x;
+        slo += v.y;
+      }
 #pragma unroll
-    for (int l = 0; l < PER; ++l) {
-      const int2 v = part[row][half * PER + l];
-      shi += v.x;
-      slo += v.y;
-    }
-#pragma unroll
-    for (int o = ROWS; o < 32; o <<= 1) {
-      shi += __shfl_xor_sync(0xffffffffu, shi, o);
-      slo += __shfl_xor_sync(0xffffffffu, slo, o);
-    }
-    const int tt = row / PPW, q = warp * PPW + row % PPW;
-    if (half == 0 && tt < nt) {
-      const long long sum = (long long)shi * 65536 + slo;
-      a.y[(rowbase + t0 + tt) * di + (long long)h * hd + p0 + q] =
-          (int)satb64(rshr64(sum, s_y) + s.dx[q][tt], 32);
+      for (int o = ROWS; o < 32; o <<= 1) {
+        shi += __shfl_xor_sync(0xffffffffu, shi, o);
+        slo += __shfl_xor_sync(0xffffffffu, slo, o);
+      }
+      const int tt = row / PPW, q = warp * PPW + row % PPW;
+      if (half == 0 && tt < nt) {
+        const long long sum = (long long)shi * 65536 + slo;
+        a.y[(rowbase + t0 + tt) * di + (long long)h * hd + p0 + q] =
+            (int)satb64(rshr64(sum, s_y) + rshr64(Dq * s.xs[q][tt], s_D), 32);
+      }
     }
     __syncwarp();
     if (lane32 == 0) mbar_arrive(&sm.empty[sl]);
@@ -497,8 +496,7 @@ __global__ void __launch_bounds__(256) k_scan_step(ScanArgs a) {
       alo += __shfl_xor_sync(0xffffffffu, alo, o);
     }
     const long long sum = (long long)ahi * 65536 + alo;
-    const int dx = (int)satb64(rshr64(Dq * xq, s_D), 32);
-    const int yk = (int)satb64(rshr64(sum, s_y) + dx, 32);
+    const int yk = (int)satb64(rshr64(sum, s_y) + rshr64(Dq * xq, s_D), 32);
     if (lane == k) yv = yk;
   }
   if (lane < kStepPPW) a.y[(long long)b * di + (long long)h * hd + warp + 8 * lane] = yv;

@@ -358,6 +358,36 @@ def test_ssm_scan_decode_step_clamped(L):
     assert (np.abs(st) == lim).mean() > 0.2
 
 
+@pytest.mark.parametrize("T", [1, 40])
+def test_ssm_scan_skip_term_beyond_int32(L, T):
+    """Exponents where both output terms exceed int32 before they are added
+    (s_D = -12, s_y = s_D - 15): the skip term rshr(D_q x, s_D) is formed in
+    64 bits and the sum saturates once, as the oracle does -- outputs whose two
+    terms cancel back into range must match exactly (sequential and
+    single-step kernels)."""
+    s = MAMBA130
+    B = 2
+    xbc, dt_raw, dt_bias, A_q, D_q, e_D, e_x, e_B, e_C, e_h, e_y = _scan_case(s, B, T, 111)
+    e_h = (e_D + e_x - e_C - 15).astype(np.int32)
+    e_y = (e_D + e_x - 12).astype(np.int32)
+    exps = _exps_for_scan(L, s, e_x, e_B, e_C, e_h, e_y, e_D)
+    st = S.uniform_ints((B, s.nheads, s.headdim, s.d_state), -2 ** 26, 2 ** 26, seed=112)
+    y = torch.empty((B, T, s.d_inner), dtype=torch.int32, device="cuda")
+    st_d = dev(st)
+    ws = torch.empty(L.scan_workspace_bytes(s, B, T), dtype=torch.uint8, device="cuda")
+    L.ssm_scan_pot(dev(xbc), dev(dt_raw), B, T, s, dev(dt_bias), dev(A_q), dev(D_q), dev(exps),
+                   st_d, y, ws)
+    yr = O.ssm_scan_pot(xbc, dt_raw, dt_bias, A_q, D_q, e_x, e_B, e_C, e_h, e_y, e_D,
+                        s.headdim, s.d_state, state=st)
+    assert np.array_equal(host(y), yr)
+    assert np.array_equal(host(st_d), st)
+    # the case is exercised: skip terms beyond int32 with an unsaturated output
+    x = xbc[..., :s.d_inner].astype(np.int64).reshape(B, T, s.nheads, s.headdim)
+    skip = (D_q.astype(np.int64)[None, None, :, None] * x) << 12
+    big = np.abs(skip.reshape(B, T, s.d_inner)) > 2 ** 31 - 1
+    assert (big & (np.abs(yr.astype(np.int64)) < 2 ** 31 - 1)).sum() > 0
+
+
 @pytest.mark.parametrize("regime", ["saturating", "small"])
 def test_ssm_scan_clamp_regimes(L, regime):
     """The sequential kernel skips the clamp for a chunk only when

@@ -420,3 +420,27 @@ def test_layer_chunked_and_decode_bit_exact(oracle, small_layers):
         parts.append(oracle.mixer_prefill(L, x[:, t:t + 1].copy(), conv_state=cs2, ssm_state=ss2))
     assert np.array_equal(np.concatenate(parts, 1), full)
     assert np.array_equal(cs2, cs) and np.array_equal(ss2, ss)
+
+
+def test_calibrated_exponents_fit_their_codes(oracle):
+    """Each calibrated power-of-two exponent is the smallest e with
+    amax <= Q 2^e, so on the calibration set itself the largest code of every
+    group lands in [64, 127]: conv input codes per channel, conv output codes
+    per head (x) and for B and C; in static mode the largest in_proj input
+    code is 127 and the static scale is the calibration set's amax."""
+    s = SMALL
+    P = S.layer_params(s, 4)
+    xc = S.calibration_batch(256, 64, 4, 50.0, outlier_seed=99, n_seqs=2)
+    L = oracle.prepare_layer(P, s, rotate=1, mode=oracle.STATIC)
+    oracle.calibrate_layer(L, xc)
+    tr = {}
+    oracle.mixer_prefill(L, xc, trace=tr)
+    u = np.abs(tr["xbc"].reshape(-1, s.conv_ch).astype(np.int32)).max(0)
+    assert u.min() >= 64 and u.max() <= 127
+    co = np.abs(tr["conv_out"].reshape(-1, s.conv_ch).astype(np.int32))
+    per_head = co[:, :s.d_inner].reshape(-1, s.nheads, s.headdim).max(axis=(0, 2))
+    assert per_head.min() >= 64 and per_head.max() <= 127
+    for part in (co[:, s.d_inner:s.d_inner + s.d_state], co[:, s.d_inner + s.d_state:]):
+        assert 64 <= part.max() <= 127
+    assert np.abs(tr["q_in"].astype(np.int32)).max() == 127
+    assert np.abs(tr["q_out"].astype(np.int32)).max() == 127
