@@ -69,7 +69,14 @@ def parse(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--scan-tile", default=None,
                     help="npt,pc,tch of the sequential scan kernel (a compiled variant)")
+    ap.add_argument("--layers", type=int, default=None,
+                    help="profiling only: run the first N layers of a stack workload")
     return ap.parse_args(argv)
+
+
+def n_layers(args) -> int:
+    w = S.WORKLOADS[args.workload]
+    return args.layers if args.layers else w.get("layers", 1)
 
 
 def measured_peaks():
@@ -98,7 +105,7 @@ def config_block(args) -> dict:
     if args.workload == "gemm2p7b_inproj":
         c.update(M=args.gemm_m, N=d.n_in, K=d.d_model)
     else:
-        c.update(layers=w.get("layers", 1), batch=w["batch"], seq_len=w["seqlen"],
+        c.update(layers=n_layers(args), batch=w["batch"], seq_len=w["seqlen"],
                  calibration=f"{S.CALIB_SEQS} seeded sequences x "
                              f"{min(w.get('prefill_len', w['seqlen']), S.CALIB_MAX_LEN)} tokens "
                              "(GPU, stage by stage)",
@@ -280,9 +287,9 @@ class StackWorkload:
         self.torch, self.lib, self.dev = torch, lib, dev
         w = S.WORKLOADS[args.workload]
         self.shape = d = w["shape"]
-        self.n_layers = w.get("layers", 1)
+        self.n_layers = n_layers(args)
         self.B, self.T = w["batch"], w["seqlen"]
-        self.stack_mode = self.n_layers > 1
+        self.stack_mode = w.get("layers", 1) > 1
         self.mode = lib.FM_DYNAMIC if args.mode == "dynamic" else lib.FM_STATIC
         params = (S.layer_params(d, 1000 + l) for l in range(self.n_layers))
         xcal = torch.from_numpy(S.calibration_batch(d.d_model, self.T, w["n_outliers"],
@@ -391,7 +398,7 @@ class DecodeWorkload(StackWorkload):
         self.torch, self.lib, self.dev = torch, lib, dev
         w = S.WORKLOADS[args.workload]
         self.shape = d = w["shape"]
-        self.n_layers, self.B, self.T = w["layers"], w["batch"], 1
+        self.n_layers, self.B, self.T = n_layers(args), w["batch"], 1
         self.stack_mode = True
         self.mode = lib.FM_DYNAMIC if args.mode == "dynamic" else lib.FM_STATIC
         P = w["prefill_len"]

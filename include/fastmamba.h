@@ -206,7 +206,9 @@ fm_status fm_gate_norm_quant(const int32_t *y, const float *z, int64_t M, const 
  * built on it (pith.science review of FastMamba, "What carries the
  * argument"; Referee minor comment 5, Eq. (5)), evaluated element-wise over
  * a device int64 array -- the same device functions the conv, scan and gate
- * kernels use.  kind: 0 = 2^v (Q.16 in, v <= 0), 1 = e^x, 2 = SoftPlus,
+ * kernels use (SiLU in the form the conv and gate kernels evaluate: table in
+ * shared memory, reciprocal-estimate division).  kind: 0 = 2^v (Q.16 in,
+ * v <= 0), 1 = e^x, 2 = SoftPlus,
  * 3 = SiLU (in clamped to int32), 4 = to_q16 of the fp32 bit pattern held
  * in the low 32 bits.  in, out: [n] int64. */
 fm_status fm_eval_pwl(int kind, const int64_t *in, int64_t n, int64_t *out, fm_stream stream);

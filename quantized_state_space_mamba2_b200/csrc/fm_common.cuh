@@ -51,13 +51,25 @@ __device__ __forceinline__ int round_clamp(float v, float lim) {
   return (int)r;
 }
 
-// fp32 -> Q.16 int32: clamp(rint(x * 2^16), +-(2^31-1)), NaN -> 0
+// fp32 -> Q.16 int32: clamp(rint(x * 2^16), +-(2^31-1)), NaN -> 0.  One
+// round-to-nearest-even conversion (it saturates to [-2^31, 2^31-1] and maps
+// NaN to 0), then the symmetric lower bound.
 __device__ __forceinline__ int to_q16(float x) {
-  if (x != x) return 0;
-  float r = rintf(__fmul_rn(x, 65536.0f));
-  if (r >= 2147483648.0f) return 2147483647;
-  if (r <= -2147483648.0f) return -2147483647;
-  return (int)r;
+  return max(__float2int_rn(__fmul_rn(x, 65536.0f)), -2147483647);
+}
+
+// The exact float of an integer |v| < 2^22 without the conversion unit:
+// 1.5 * 2^23 + v is exact in fp32, and so is the subtraction.
+__device__ __forceinline__ float small_i2f(int v) {
+  return __fsub_rn(__int_as_float(0x4B400000 + v), 12582912.0f);
+}
+
+// The int8 quantiser's rounding: rint(v) clamped to +-127 (NaN -> -127).  The
+// clamp commutes with rint for an integer bound; adding 1.5 * 2^23 then
+// rounds to the nearest integer (ties to even) in the fp32 add itself.
+__device__ __forceinline__ int quant127(float v) {
+  const float c = fminf(fmaxf(v, -127.0f), 127.0f);
+  return __float_as_int(__fadd_rn(c, 12582912.0f)) - 0x4B400000;
 }
 
 // ---------------------------------------------------------------- 2^v unit
@@ -118,29 +130,6 @@ __device__ __forceinline__ int softplus_pwl(int v) {
   return r > 2147483647LL ? 2147483647 : (int)r;
 }
 
-// SiLU(x / 2^16) in Q.16 for x in +-(2^31 - 1): sigma from E = e^-|x|;
-// x >= 0: floor(2^32 / (2^16 + E)), x < 0: floor(E 2^16 / (2^16 + E));
-// result rshr(x sigma, 16) = xh sigma + ((xl sigma + 2^15) >> 16) with
-// x = xh 2^16 + xl, xl in [0, 2^16) (both products fit 32 bits).
-__device__ __forceinline__ int silu_pwl32(int x) {
-  const unsigned E = (unsigned)exp_pwl(x < 0 ? (long long)x : -(long long)x);
-  const unsigned d = 65536u + E;  // [2^16, 2^17]
-  unsigned sig;
-  if (x >= 0) {
-    sig = 0xFFFFFFFFu / d;                // floor((2^32 - 1) / d)
-    if ((d & (d - 1u)) == 0u) sig += 1u;  // d divides 2^32
-  } else if (E >= 65536u) {
-    sig = 32768u;                         // 2^32 / 2^17
-  } else {
-    sig = (E << 16) / d;
-  }
-  const int xh = x >> 16;
-  const unsigned xl = (unsigned)x & 0xFFFFu;
-  return xh * (int)sig + (int)((xl * sig + 32768u) >> 16);
-}
-
-__device__ __forceinline__ long long silu_pwl(int x) { return silu_pwl32(x); }
-
 // ---------------------------------------------------------------- fast forms
 // The same functions for element-wise kernels: the 8 (P_i, S_i) pairs are read
 // from a shared-memory table packed as P | S << 17 (per-lane indices would
@@ -150,57 +139,46 @@ __device__ __forceinline__ void pwl_table_init(int *tab) {
   if (threadIdx.x < 8 && threadIdx.y == 0) tab[threadIdx.x] = pwl_P(threadIdx.x) | (pwl_S(threadIdx.x) << 17);
 }
 
-__device__ __forceinline__ int pow2_pwl32_t(int w, const int *tab) {
-  if (w > 0) w = 0;
-  if (w < -(31 << 16)) return 0;
-  const int k = -(w >> 16);
+// e^-|x| in Q.16 (|x| in Q.16): w = rshr(-|x| log2e_Q15, 15) as in exp_pwl,
+// then 2^(w / 2^16) from the table.  |x| is capped at 2^21 (w is then below
+// -31 * 2^16), and the rounding shift by k = -floor(w / 2^16) is capped at
+// 31, where m + 2^30 < 2^31 already rounds to 0 -- no branches.
+__device__ __forceinline__ unsigned exp_neg_abs_t(int x, const int *tab) {
+  const unsigned ux = x < 0 ? 0u - (unsigned)x : (unsigned)x;
+  const int ax = (int)min(ux, 1u << 21);
+  const int ah = ax >> 15, al = ax & 0x7FFF;
+  const int w = -ah * (int)kLog2eQ15 + ((16384 - al * (int)kLog2eQ15) >> 15);  // <= 0
+  const int k = min(-(w >> 16), 31);
   const int f = w & 0xFFFF;
   const int e = tab[f >> 13];
   const int m = (e & 0x1FFFF) + ((((unsigned)e >> 17) * (f & 8191) + 4096) >> 13);
-  if (k == 0) return m;
-  return (m + (1 << (k - 1))) >> k;
+  return ((unsigned)m + ((1u << k) >> 1)) >> k;
 }
 
-__device__ __forceinline__ int exp_pwl_t(int x, const int *tab) {  // x <= 0 in int32
-  if (x >= 0) return 65536;
-  if (x <= -(1 << 21)) return 0;
-  const int ax = -x;
-  const int ah = ax >> 15, al = ax & 0x7FFF;
-  return pow2_pwl32_t(-ah * (int)kLog2eQ15 + ((16384 - al * (int)kLog2eQ15) >> 15), tab);
-}
-
-// floor(num / d) for d in [2^16, 2^17] and num in [0, 2^32]; numf = num as a
-// float (exact: num is 2^32 or a multiple of 2^16 below it), num_mod = num
-// mod 2^32.  The float estimate is within one of the quotient; the remainder,
-// exact modulo 2^32, lies in (-2d, 2d) and fixes it.
-__device__ __forceinline__ unsigned div_q16(float numf, unsigned num_mod, unsigned d) {
-  float rd;
-  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(rd) : "f"((float)d));
-  unsigned q = (unsigned)__fmul_rz(numf, rd);
-  unsigned rem = num_mod - q * d;
-#pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    if ((int)rem < 0) {
-      q -= 1u;
-      rem += d;
-    } else if (rem >= d) {
-      q += 1u;
-      rem -= d;
-    }
-  }
-  return q;
-}
-
+// SiLU(x / 2^16) in Q.16 for x in +-(2^31 - 1): sigma from E = e^-|x|;
+// x >= 0: floor(2^32 / (2^16 + E)), x < 0: floor(E 2^16 / (2^16 + E));
+// result rshr(x sigma, 16) = xh sigma + ((xl sigma + 2^15) >> 16) with
+// x = xh 2^16 + xl, xl in [0, 2^16) (both products fit 32 bits).
+// The floor division: d = 2^16 + E in [2^16, 2^17] and the numerator (2^32,
+// or E 2^16) are exact floats; num * rcp(d), truncated, is within 2^-5 of the
+// quotient (a few ulp of relative error on a quotient below 2^17), so one
+// correction from the exact remainder (mod 2^32) gives the floor.  The float
+// conversions avoid the conversion unit (small_i2f and a round-to-zero add of
+// 2^23).
 __device__ __forceinline__ int silu_pwl_t(int x, const int *tab) {
-  const unsigned E = (unsigned)exp_pwl_t(x < 0 ? x : -x, tab);
+  const unsigned E = exp_neg_abs_t(x, tab);
   const unsigned d = 65536u + E;
-  // x >= 0: num = 2^32; x < 0: num = E 2^16 (= 2^32 when E = 2^16)
-  const float numf = x >= 0 ? 4294967296.0f : (float)E * 65536.0f;
-  const unsigned nmod = x >= 0 ? 0u : (E << 16);
-  const unsigned sig = div_q16(numf, nmod, d);
+  float rd;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(rd) : "f"(small_i2f((int)d)));
+  const float numf = x >= 0 ? 4294967296.0f : __fmul_rn(small_i2f((int)E), 65536.0f);
+  const unsigned nmod = x >= 0 ? 0u : (E << 16);  // numerator mod 2^32
+  unsigned q = __float_as_uint(__fadd_rz(__fmul_rz(numf, rd), 8388608.0f)) - 0x4B000000u;
+  const unsigned rem = nmod - q * d;
+  if ((int)rem < 0) q -= 1u;
+  else if (rem >= d) q += 1u;
   const int xh = x >> 16;
   const unsigned xl = (unsigned)x & 0xFFFFu;
-  return xh * (int)sig + (int)((xl * sig + 32768u) >> 16);
+  return xh * (int)q + (int)((xl * q + 32768u) >> 16);
 }
 
 // rshr(v, k) for int32 v and k in [1, 31] without overflow: floor(v / 2^k) +

@@ -262,10 +262,11 @@ static fm_status launch_conv(const int8_t *u, int B, int T, int cc, const int8_t
                              const int32_t *bq, const int32_t *exps, int8_t *conv_state,
                              int8_t *out, unsigned int *amax, cudaStream_t s) {
   if ((long long)B * T == 0) return FM_OK;
-  const int groups = (cc / kConvCPT + kConvThreads - 1) / kConvThreads;
-  if (T > 2147483647 || B > 65535) return fail(FM_ERR_SHAPE, "conv: T or B too large");
-  k_conv1d_pot<<<dim3(groups, (unsigned)T, B), kConvThreads, 0, s>>>(u, T, cc, wq, bq, exps,
-                                                                      conv_state, out, amax);
+  const int groups = (cc / kConvCPT + kConvQuads - 1) / kConvQuads;
+  if (B > 65535) return fail(FM_ERR_SHAPE, "conv: B too large");
+  const unsigned tiles = (unsigned)((T + kConvTokens - 1) / kConvTokens);
+  k_conv1d_pot<<<dim3(tiles, groups, B), kConvThreads, 0, s>>>(u, T, cc, wq, bq, exps,
+                                                                conv_state, out, amax);
   FM_TRY(launched("k_conv1d_pot"));
   if (conv_state) {
     const long long n = (long long)B * cc;
@@ -640,6 +641,9 @@ extern "C" fm_status fm_gate_norm_quant(const int32_t *y, const float *z, int64_
 }
 
 __global__ void k_eval_pwl(int kind, const int64_t *in, long long n, int64_t *out) {
+  __shared__ int tab[8];
+  pwl_table_init(tab);
+  __syncthreads();
   const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= n) return;
   const long long v = in[i];
@@ -648,7 +652,7 @@ __global__ void k_eval_pwl(int kind, const int64_t *in, long long n, int64_t *ou
     case 0: r = pow2_pwl(v); break;
     case 1: r = exp_pwl(v); break;
     case 2: r = softplus_pwl((int)satb64(v, 32)); break;
-    case 3: r = silu_pwl((int)satb64(v, 32)); break;
+    case 3: r = silu_pwl_t((int)satb64(v, 32), tab); break;
     default: r = to_q16(__uint_as_float((unsigned int)(v & 0xFFFFFFFFLL))); break;
   }
   out[i] = r;

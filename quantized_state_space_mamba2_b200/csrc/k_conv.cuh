@@ -8,25 +8,38 @@
 //   x16 = satb(rshr(acc, -(e_w + e_u + 16)), 32)             (to Q.16)
 //   out = satb(rshr(SiLU_pwl(x16), e_o + 16), 8)
 //
-// Layout: each thread owns 4 consecutive channels of one token (4-byte loads
-// of the 4-row window t-3 .. t and one 4-byte store); a warp covers 128
-// contiguous bytes of each row and the window rows shared by neighbouring
-// tokens come from L1/L2.  Every (token, channel) output is independent, so
-// the grid is (channel groups / 64, T, batch) of 64-thread blocks with few
-// registers per thread (high occupancy hides the PWL SiLU's latency).  The
-// conv state (the 3 inputs before the first token) is read here and replaced
-// afterwards by k_conv_state_update, in stream order.
+// Layout: each thread owns 4 consecutive channels and kConvTT consecutive
+// tokens.  It loads the kConvTT + 3 input rows of its channels once (4-byte
+// words: byte j = channel j), transposes the first window so that each
+// channel's 4 taps sit in one word (tap k = byte k), and slides it one token
+// at a time with one byte permute per channel; each 4-tap dot product is one
+// dp4a against the channel's packed weights.  A block is 64 channel quads
+// (256 channels) x 2 token groups; grid (token tiles of 16, channel groups,
+// batch).  Every (token, channel) output is
+// independent.  The conv state (the 3 inputs before the first token) is read
+// here and replaced afterwards by k_conv_state_update, in stream order.
 #pragma once
 #include "fm_common.cuh"
 
 namespace fm {
 
-constexpr int kConvCPT = 4;       // channels per thread
-constexpr int kConvThreads = 64;  // threads per block
+constexpr int kConvCPT = 4;        // channels per thread
+constexpr int kConvTT = 8;         // tokens per thread
+constexpr int kConvQuads = 64;     // channel quads per block (256 channels)
+constexpr int kConvTG = 2;         // token groups per block
+constexpr int kConvThreads = kConvQuads * kConvTG;
+constexpr int kConvTokens = kConvTT * kConvTG;  // tokens per block
 
-__device__ __forceinline__ void unpack4(uint32_t w, int (&v)[4]) {
-#pragma unroll
-  for (int i = 0; i < 4; ++i) v[i] = (int)(int8_t)((w >> (8 * i)) & 0xFF);
+// tap k of channel j -> byte k of column j, from the rows (byte j = channel j)
+// of tokens t-3 .. t
+__device__ __forceinline__ void conv_transpose4(uint32_t r0, uint32_t r1, uint32_t r2, uint32_t r3,
+                                                uint32_t (&col)[4]) {
+  const uint32_t a = __byte_perm(r0, r1, 0x5140), b = __byte_perm(r2, r3, 0x5140);
+  const uint32_t c = __byte_perm(r0, r1, 0x7362), d = __byte_perm(r2, r3, 0x7362);
+  col[0] = __byte_perm(a, b, 0x5410);
+  col[1] = __byte_perm(a, b, 0x7632);
+  col[2] = __byte_perm(c, d, 0x5410);
+  col[3] = __byte_perm(c, d, 0x7632);
 }
 
 // amax (nullable, [cc] u32): max |SiLU output| per channel (calibration).
@@ -37,64 +50,82 @@ __global__ void __launch_bounds__(kConvThreads) k_conv1d_pot(
   __shared__ int tab[8];
   pwl_table_init(tab);
   __syncthreads();
-  const int c0 = (blockIdx.x * kConvThreads + threadIdx.x) * kConvCPT;
+  const int quad = threadIdx.x % kConvQuads, tg = threadIdx.x / kConvQuads;
+  const int c0 = (blockIdx.y * kConvQuads + quad) * kConvCPT;
   if (c0 >= cc) return;
-  const int t = blockIdx.y;
+  const int t0 = (blockIdx.x * kConvTG + tg) * kConvTT;
+  if (t0 >= T) return;
   const int b = blockIdx.z;
   const int8_t *ub = u + (long long)b * T * cc;
-  int win[4][kConvCPT];
+  // input rows t0-3 .. t0+kConvTT-1 (rows past the end are never used)
+  uint32_t row[kConvTT + 3];
 #pragma unroll
-  for (int r = 0; r < 4; ++r) {
-    const int tt = t - 3 + r;
+  for (int r = 0; r < kConvTT + 3; ++r) {
+    const int tt = t0 - 3 + r;
     uint32_t raw = 0u;
-    if (tt >= 0)
-      raw = *reinterpret_cast<const uint32_t *>(ub + (long long)tt * cc + c0);
-    else if (conv_state)
+    if (tt >= 0) {
+      if (tt < T) raw = *reinterpret_cast<const uint32_t *>(ub + (long long)tt * cc + c0);
+    } else if (conv_state) {
       raw = *reinterpret_cast<const uint32_t *>(conv_state + ((long long)b * 3 + (3 + tt)) * cc + c0);
-    unpack4(raw, win[r]);
+    }
+    row[r] = raw;
   }
   const uint4 wp = *reinterpret_cast<const uint4 *>(wq + (long long)c0 * 4);  // 4 taps x 4 channels
   const int4 bias = *reinterpret_cast<const int4 *>(bq + c0);
   const int4 eu = *reinterpret_cast<const int4 *>(exps + c0);
   const int4 ew = *reinterpret_cast<const int4 *>(exps + cc + c0);
   const int4 eo = *reinterpret_cast<const int4 *>(exps + 2 * cc + c0);
-  const uint32_t wr[4] = {wp.x, wp.y, wp.z, wp.w};
+  const int wr[4] = {(int)wp.x, (int)wp.y, (int)wp.z, (int)wp.w};
   const int bs[4] = {bias.x, bias.y, bias.z, bias.w};
   const int s_in[4] = {-(ew.x + eu.x + 16), -(ew.y + eu.y + 16), -(ew.z + eu.z + 16),
                        -(ew.w + eu.w + 16)};
   const int s_out[4] = {eo.x + 16, eo.y + 16, eo.z + 16, eo.w + 16};
-  uint32_t packed = 0;
+  bool fast[4];  // |acc| < 2^30 (the taps add at most 4 * 127^2) and a 32-bit shift
 #pragma unroll
-  for (int j = 0; j < kConvCPT; ++j) {
-    int w[4];
-    unpack4(wr[j], w);
-    const int dot = w[0] * win[0][j] + w[1] * win[1][j] + w[2] * win[2][j] + w[3] * win[3][j];
-    int x16;
-    const int si = s_in[j];
-    if (bs[j] >= -(1 << 29) && bs[j] <= (1 << 29) && si >= -30 && si <= 29) {
-      // 32-bit path: |acc| < 2^30 (the taps add at most 4 * 127^2)
-      const int acc = bs[j] + dot;
-      if (si > 0) {
-        x16 = rshr32(acc, si);
+  for (int j = 0; j < 4; ++j)
+    fast[j] = bs[j] >= -(1 << 29) && bs[j] <= (1 << 29) && s_in[j] >= -30 && s_in[j] <= 29 &&
+              s_out[j] >= 1 && s_out[j] <= 31;
+  uint32_t col[4];
+  conv_transpose4(row[0], row[1], row[2], row[3], col);
+  const int nt = min(kConvTT, T - t0);
+#pragma unroll
+  for (int k = 0; k < kConvTT; ++k) {
+    if (k > 0) {  // slide: drop the oldest tap, append byte j of the new row
+      const uint32_t nr = row[k + 3];
+      col[0] = __byte_perm(col[0], nr, 0x4321);
+      col[1] = __byte_perm(col[1], nr, 0x5321);
+      col[2] = __byte_perm(col[2], nr, 0x6321);
+      col[3] = __byte_perm(col[3], nr, 0x7321);
+    }
+    if (k >= nt) break;
+    uint32_t packed = 0;
+#pragma unroll
+    for (int j = 0; j < kConvCPT; ++j) {
+      int code;
+      if (fast[j]) {
+        const int acc = __dp4a((int)col[j], wr[j], bs[j]);
+        const int si = s_in[j];
+        int x16;
+        if (si > 0) {
+          x16 = rshr32(acc, si);
+        } else {
+          const int sh = -si, lim = 0x7FFFFFFF >> sh;
+          x16 = acc > lim ? 2147483647 : (acc < -lim ? -2147483647 : acc * (1 << sh));
+        }
+        const int sv = silu_pwl_t(x16, tab);
+        if (amax) atomicMax(amax + c0 + j, (unsigned int)(sv < 0 ? -sv : sv));
+        code = min(max(rshr32(sv, s_out[j]), -127), 127);
       } else {
-        const int k = -si, lim = 0x7FFFFFFF >> k;
-        x16 = acc > lim ? 2147483647 : (acc < -lim ? -2147483647 : acc * (1 << k));
+        const long long acc = (long long)bs[j] + __dp4a((int)col[j], wr[j], 0);
+        const int x16 = (int)satb64(rshr64(acc, s_in[j]), 32);
+        const int sv = silu_pwl_t(x16, tab);
+        if (amax) atomicMax(amax + c0 + j, (unsigned int)(sv < 0 ? -sv : sv));
+        code = (int)satb64(rshr64(sv, s_out[j]), 8);
       }
-    } else {
-      x16 = (int)satb64(rshr64((long long)bs[j] + dot, si), 32);
+      packed |= ((uint32_t)(code & 0xFF)) << (8 * j);
     }
-    const int sv = silu_pwl_t(x16, tab);
-    if (amax) atomicMax(amax + c0 + j, (unsigned int)(sv < 0 ? -sv : sv));
-    const int so = s_out[j];
-    int code;
-    if (so >= 1 && so <= 31) {
-      code = min(max(rshr32(sv, so), -127), 127);
-    } else {
-      code = (int)satb64(rshr64(sv, so), 8);
-    }
-    packed |= ((uint32_t)(code & 0xFF)) << (8 * j);
+    *reinterpret_cast<uint32_t *>(out + ((long long)b * T + t0 + k) * cc + c0) = packed;
   }
-  *reinterpret_cast<uint32_t *>(out + ((long long)b * T + t) * cc + c0) = packed;
 }
 
 // After the conv: the state becomes the last 3 inputs (oldest first).  One

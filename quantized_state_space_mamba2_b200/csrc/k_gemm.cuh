@@ -232,7 +232,7 @@ __device__ __forceinline__ void gemm_store_chunk(const GemmEpilogue &ep, long lo
       uint32_t w = 0;
 #pragma unroll
       for (int b = 0; b < 4; ++b) {
-        const int code = round_clamp(__fmul_rn(y[j + b], e4[b]), 127.0f);
+        const int code = quant127(__fmul_rn(y[j + b], e4[b]));
         w |= ((uint32_t)(code & 0xFF)) << (8 * b);
       }
       packed[j / 4] = w;
@@ -248,7 +248,7 @@ __device__ __forceinline__ void gemm_store_chunk(const GemmEpilogue &ep, long lo
     if (c < di) {
       ep.z[row * di + c] = y[j];
     } else if (c < di + cc) {
-      ep.xbc[row * cc + (c - di)] = (int8_t)round_clamp(__fmul_rn(y[j], cole[j]), 127.0f);
+      ep.xbc[row * cc + (c - di)] = (int8_t)quant127(__fmul_rn(y[j], cole[j]));
     } else {
       ep.dt[row * ep.nh + (c - di - cc)] = y[j];
     }

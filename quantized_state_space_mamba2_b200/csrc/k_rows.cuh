@@ -53,7 +53,7 @@ __device__ __forceinline__ void rotate_quant_store(float (&v)[8], int rotate, in
     const float inv = __fdiv_rn(127.0f, use);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      const uint32_t c = (uint32_t)(round_clamp(__fmul_rn(v[i], inv), 127.0f) & 0xFF);
+      const uint32_t c = (uint32_t)(quant127(__fmul_rn(v[i], inv)) & 0xFF);
       if (i < 4) lo |= c << (8 * i);
       else hi |= c << (8 * (i - 4));
     }
@@ -193,7 +193,7 @@ __global__ void __launch_bounds__(1024) k_gate_norm_quant(
   const float *w = norm_w + col;
   float v[8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(__fmul_rn(__fmul_rn((float)gq[i], scale), rstd), w[i]);
+  for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(__fmul_rn(__fmul_rn(small_i2f(gq[i]), scale), rstd), w[i]);
   rotate_quant_store(v, rotate, mode, static_amax, q + row * di, s_x + row,
                      amax_row ? amax_row + row : nullptr, s_red, &s_bc);
 }
