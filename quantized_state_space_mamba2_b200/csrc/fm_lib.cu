@@ -231,10 +231,10 @@ static fm_status launch_gemm(const int8_t *A, long long M, const int8_t *W, long
   if (K % kGemmBK) return fail(FM_ERR_SHAPE, "gemm: K=%lld is not a multiple of 128", K);
   if ((M + kGemmBM - 1) / kGemmBM > 65535 || (N + 63) / 64 > 65535)
     return fail(FM_ERR_SHAPE, "gemm: M=%lld or N=%lld too large", M, N);
+  CUtensorMap ta, tb;
   const long long mt = (M + kGemmBM - 1) / kGemmBM;
   const long long tiles256 = mt * ((N + 255) / 256), tiles128 = mt * ((N + 127) / 128);
   const int sms = sm_count();
-  CUtensorMap ta, tb;
   FM_TRY(make_tmap(&ta, A, M, K, kGemmBM));
   if (tiles256 >= 2LL * sms) {
     FM_TRY(make_tmap(&tb, W, N, K, 256));
@@ -264,9 +264,14 @@ static fm_status launch_conv(const int8_t *u, int B, int T, int cc, const int8_t
   if ((long long)B * T == 0) return FM_OK;
   const int groups = (cc / kConvCPT + kConvQuads - 1) / kConvQuads;
   if (B > 65535) return fail(FM_ERR_SHAPE, "conv: B too large");
-  const unsigned tiles = (unsigned)((T + kConvTokens - 1) / kConvTokens);
-  k_conv1d_pot<<<dim3(tiles, groups, B), kConvThreads, 0, s>>>(u, T, cc, wq, bq, exps,
-                                                                conv_state, out, amax);
+  if (T >= kConvTT) {
+    const unsigned tiles = (unsigned)((T + kConvTokens - 1) / kConvTokens);
+    k_conv1d_pot<kConvTT, kConvTG><<<dim3(tiles, groups, B), kConvQuads * kConvTG, 0, s>>>(
+        u, T, cc, wq, bq, exps, conv_state, out, amax);
+  } else {  // decode steps and short chunks: one token per thread
+    k_conv1d_pot<1, 1><<<dim3((unsigned)T, groups, B), kConvQuads, 0, s>>>(
+        u, T, cc, wq, bq, exps, conv_state, out, amax);
+  }
   FM_TRY(launched("k_conv1d_pot"));
   if (conv_state) {
     const long long n = (long long)B * cc;

@@ -8,14 +8,13 @@
 //   x16 = satb(rshr(acc, -(e_w + e_u + 16)), 32)             (to Q.16)
 //   out = satb(rshr(SiLU_pwl(x16), e_o + 16), 8)
 //
-// Layout: each thread owns 4 consecutive channels and kConvTT consecutive
-// tokens.  It loads the kConvTT + 3 input rows of its channels once (4-byte
+// Layout: each thread owns 4 consecutive channels and TT consecutive tokens
+// (4 for prefill, 1 for decode steps).  It loads the TT + 3 input rows of its channels once (4-byte
 // words: byte j = channel j), transposes the first window so that each
 // channel's 4 taps sit in one word (tap k = byte k), and slides it one token
 // at a time with one byte permute per channel; each 4-tap dot product is one
 // dp4a against the channel's packed weights.  A block is 64 channel quads
-// (256 channels) x 2 token groups; grid (token tiles of 16, channel groups,
-// batch).  Every (token, channel) output is
+// (256 channels) x TG token groups; grid (token tiles, channel groups, batch).  Every (token, channel) output is
 // independent.  The conv state (the 3 inputs before the first token) is read
 // here and replaced afterwards by k_conv_state_update, in stream order.
 #pragma once
@@ -24,11 +23,10 @@
 namespace fm {
 
 constexpr int kConvCPT = 4;        // channels per thread
-constexpr int kConvTT = 8;         // tokens per thread
+constexpr int kConvTT = 4;         // tokens per thread (prefill)
 constexpr int kConvQuads = 64;     // channel quads per block (256 channels)
-constexpr int kConvTG = 2;         // token groups per block
-constexpr int kConvThreads = kConvQuads * kConvTG;
-constexpr int kConvTokens = kConvTT * kConvTG;  // tokens per block
+constexpr int kConvTG = 2;         // token groups per block (prefill)
+constexpr int kConvTokens = kConvTT * kConvTG;  // tokens per block (prefill)
 
 // tap k of channel j -> byte k of column j, from the rows (byte j = channel j)
 // of tokens t-3 .. t
@@ -43,7 +41,8 @@ __device__ __forceinline__ void conv_transpose4(uint32_t r0, uint32_t r1, uint32
 }
 
 // amax (nullable, [cc] u32): max |SiLU output| per channel (calibration).
-__global__ void __launch_bounds__(kConvThreads) k_conv1d_pot(
+template <int TT, int TG>
+__global__ void __launch_bounds__(kConvQuads *TG) k_conv1d_pot(
     const int8_t *__restrict__ u, int T, int cc, const int8_t *__restrict__ wq,
     const int32_t *__restrict__ bq, const int32_t *__restrict__ exps,
     const int8_t *__restrict__ conv_state, int8_t *__restrict__ out, unsigned int *amax) {
@@ -53,14 +52,14 @@ __global__ void __launch_bounds__(kConvThreads) k_conv1d_pot(
   const int quad = threadIdx.x % kConvQuads, tg = threadIdx.x / kConvQuads;
   const int c0 = (blockIdx.y * kConvQuads + quad) * kConvCPT;
   if (c0 >= cc) return;
-  const int t0 = (blockIdx.x * kConvTG + tg) * kConvTT;
+  const int t0 = (blockIdx.x * TG + tg) * TT;
   if (t0 >= T) return;
   const int b = blockIdx.z;
   const int8_t *ub = u + (long long)b * T * cc;
-  // input rows t0-3 .. t0+kConvTT-1 (rows past the end are never used)
-  uint32_t row[kConvTT + 3];
+  // input rows t0-3 .. t0+TT-1 (rows past the end are never used)
+  uint32_t row[TT + 3];
 #pragma unroll
-  for (int r = 0; r < kConvTT + 3; ++r) {
+  for (int r = 0; r < TT + 3; ++r) {
     const int tt = t0 - 3 + r;
     uint32_t raw = 0u;
     if (tt >= 0) {
@@ -87,9 +86,9 @@ __global__ void __launch_bounds__(kConvThreads) k_conv1d_pot(
               s_out[j] >= 1 && s_out[j] <= 31;
   uint32_t col[4];
   conv_transpose4(row[0], row[1], row[2], row[3], col);
-  const int nt = min(kConvTT, T - t0);
+  const int nt = min(TT, T - t0);
 #pragma unroll
-  for (int k = 0; k < kConvTT; ++k) {
+  for (int k = 0; k < TT; ++k) {
     if (k > 0) {  // slide: drop the oldest tap, append byte j of the new row
       const uint32_t nr = row[k + 3];
       col[0] = __byte_perm(col[0], nr, 0x4321);
