@@ -253,8 +253,13 @@ static fm_status launch_hadamard_quant(const float *x, long long M, int K, const
                                        float *s_x, float *amax_row, cudaStream_t s) {
   if (M <= 0) return FM_OK;
 
-  k_hadamard_quant<<<(unsigned)M, 32 * (K / 256), 0, s>>>(x, K, prenorm_w, rotate, mode,
-                                                           static_amax, q, s_x, amax_row);
+  const int nb = K / 256;  // two 256-blocks per warp when they pair up
+  if (nb % 2 == 0)
+    k_hadamard_quant<2><<<(unsigned)M, 32 * (nb / 2), 0, s>>>(x, K, prenorm_w, rotate, mode,
+                                                              static_amax, q, s_x, amax_row);
+  else
+    k_hadamard_quant<1><<<(unsigned)M, 32 * nb, 0, s>>>(x, K, prenorm_w, rotate, mode,
+                                                        static_amax, q, s_x, amax_row);
   return launched("k_hadamard_quant");
 }
 
@@ -615,7 +620,13 @@ static fm_status gate_impl(const int32_t *y, const float *z, long long M, const 
                            float *amax_row, unsigned long long *gstat, const int32_t *e_g_override,
                            cudaStream_t s) {
   if (M <= 0) return FM_OK;
-  k_gate_norm_quant<<<(unsigned)M, 32 * (d.di / 256), 0, s>>>(
+  const int nb = d.di / 256;
+  if (nb % 2 == 0)
+    k_gate_norm_quant<2><<<(unsigned)M, 32 * (nb / 2), 0, s>>>(
+      y, z, d.di, d.hd, exps + X.e_y, e_g_override ? e_g_override : exps + X.e_g, norm_w, rotate,
+      mode, static_amax, q, s_x, amax_row, gstat);
+  else
+    k_gate_norm_quant<1><<<(unsigned)M, 32 * nb, 0, s>>>(
       y, z, d.di, d.hd, exps + X.e_y, e_g_override ? e_g_override : exps + X.e_g, norm_w, rotate,
       mode, static_amax, q, s_x, amax_row, gstat);
   return launched("k_gate_norm_quant");

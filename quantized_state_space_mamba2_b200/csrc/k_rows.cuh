@@ -9,10 +9,11 @@
 // dimension).  Gate-then-normalise order and RMSNorm are those of Mamba2 (the
 // paper's references [2], [10]).
 //
-// Layout: one CTA per row, one warp per 256-column Hadamard block, each lane
-// holding 8 consecutive elements (two 16-byte loads), so the whole row's
-// rotation happens in registers and shuffles; HBM traffic is one read of the
-// row and one write of its codes.
+// Layout: one CTA per row, one warp per one or two 256-column Hadamard
+// blocks (two when the row has an even number of blocks), each lane holding 8
+// consecutive elements of each block (two 16-byte loads per block), so the
+// whole row's rotation happens in registers and shuffles; HBM traffic is one
+// read of the row and one write of its codes.
 #pragma once
 #include "fm_common.cuh"
 
@@ -35,37 +36,49 @@ __device__ __forceinline__ float cta_max(float v, float *s_red, float *s_out) {
   return *s_out;
 }
 
-// Rotation (optional) + per-row or static quantisation of v[8] (this lane's
-// 8 elements at column 256*warp + 8*lane); thread 0 writes s_x / amax_row.
-__device__ __forceinline__ void rotate_quant_store(float (&v)[8], int rotate, int mode,
+// Rotation (optional) + per-row or static quantisation of this lane's BPW
+// groups of 8 elements, group b at column 256 * (BPW * warp + b) + 8 * lane;
+// thread 0 writes s_x / amax_row.  The BPW blocks' transforms are independent
+// (more work in flight per warp, half the warps per row for BPW = 2).
+template <int BPW>
+__device__ __forceinline__ void rotate_quant_store(float (&v)[BPW][8], int rotate, int mode,
                                                    const float *static_amax, int8_t *qrow,
                                                    float *sx_out, float *amax_out,
                                                    float *s_red, float *s_bc) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  if (rotate) fwht256_lane8(v, lane);
+  if (rotate) {
+#pragma unroll
+    for (int b = 0; b < BPW; ++b) fwht256_lane8(v[b], lane);
+  }
   float a = 0.0f;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) a = fmaxf(a, fabsf(v[i]));
+  for (int b = 0; b < BPW; ++b)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) a = fmaxf(a, fabsf(v[b][i]));
   const float amax = cta_max(a, s_red, s_bc);
   const float use = (mode == 0) ? amax : *static_amax;
-  uint32_t lo = 0, hi = 0;
-  if (use > 0.0f) {
-    const float inv = __fdiv_rn(127.0f, use);
+  const float inv = use > 0.0f ? __fdiv_rn(127.0f, use) : 0.0f;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const uint32_t c = (uint32_t)(quant127(__fmul_rn(v[i], inv)) & 0xFF);
-      if (i < 4) lo |= c << (8 * i);
-      else hi |= c << (8 * (i - 4));
+  for (int b = 0; b < BPW; ++b) {
+    uint32_t lo = 0, hi = 0;
+    if (use > 0.0f) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const uint32_t c = (uint32_t)(quant127(__fmul_rn(v[b][i], inv)) & 0xFF);
+        if (i < 4) lo |= c << (8 * i);
+        else hi |= c << (8 * (i - 4));
+      }
     }
+    *reinterpret_cast<uint2 *>(qrow + (warp * BPW + b) * 256 + lane * 8) = make_uint2(lo, hi);
   }
-  *reinterpret_cast<uint2 *>(qrow + warp * 256 + lane * 8) = make_uint2(lo, hi);
   if (threadIdx.x == 0) {
     *sx_out = use > 0.0f ? __fdiv_rn(use, 127.0f) : 0.0f;
     if (amax_out) *amax_out = amax;
   }
 }
 
-// a0 + a1 (and a10's tail): blockDim = 32 * (K / 256), grid = M.
+// a0 + a1 (and a10's tail): blockDim = 32 * (K / 256 / BPW), grid = M.
+template <int BPW>
 __global__ void __launch_bounds__(1024) k_hadamard_quant(const float *__restrict__ x, int K,
                                                          const float *__restrict__ prenorm_w,
                                                          int rotate, int mode,
@@ -78,27 +91,31 @@ __global__ void __launch_bounds__(1024) k_hadamard_quant(const float *__restrict
   __shared__ float s_rstd;
   const long long row = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nb = blockDim.x >> 5;
-  const float *src = x + row * K + warp * 256 + lane * 8;
-  float v[8];
-  {
-    const float4 a = *reinterpret_cast<const float4 *>(src);
-    const float4 b = *reinterpret_cast<const float4 *>(src + 4);
-    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  const int nb = (blockDim.x >> 5) * BPW;  // 256-blocks in the row
+  float v[BPW][8];
+#pragma unroll
+  for (int b = 0; b < BPW; ++b) {
+    const float *src = x + row * K + (warp * BPW + b) * 256 + lane * 8;
+    const float4 p = *reinterpret_cast<const float4 *>(src);
+    const float4 r = *reinterpret_cast<const float4 *>(src + 4);
+    v[b][0] = p.x; v[b][1] = p.y; v[b][2] = p.z; v[b][3] = p.w;
+    v[b][4] = r.x; v[b][5] = r.y; v[b][6] = r.z; v[b][7] = r.w;
   }
   if (prenorm_w) {
     // RMSNorm (eps 1e-5): sum of squares in double in the fixed order
     // (lane-sequential 8, xor tree over the warp, blocks in increasing order)
-    double P = 0.0;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const double e = (double)v[i];
-      P = __dadd_rn(P, __dmul_rn(e, e));
+    for (int b = 0; b < BPW; ++b) {
+      double P = 0.0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const double e = (double)v[b][i];
+        P = __dadd_rn(P, __dmul_rn(e, e));
+      }
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) P = __dadd_rn(P, __shfl_xor_sync(0xffffffffu, P, o));
+      if (lane == 0) s_blk[warp * BPW + b] = P;
     }
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) P = __dadd_rn(P, __shfl_xor_sync(0xffffffffu, P, o));
-    if (lane == 0) s_blk[warp] = P;
     __syncthreads();
     if (threadIdx.x == 0) {
       double tot = 0.0;
@@ -108,17 +125,21 @@ __global__ void __launch_bounds__(1024) k_hadamard_quant(const float *__restrict
     }
     __syncthreads();
     const float rstd = s_rstd;
-    const float *w = prenorm_w + warp * 256 + lane * 8;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(__fmul_rn(v[i], rstd), w[i]);
+    for (int b = 0; b < BPW; ++b) {
+      const float *w = prenorm_w + (warp * BPW + b) * 256 + lane * 8;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[b][i] = __fmul_rn(__fmul_rn(v[b][i], rstd), w[i]);
+    }
   }
-  rotate_quant_store(v, rotate, mode, static_amax, q + row * K, s_x + row,
-                     amax_row ? amax_row + row : nullptr, s_red, &s_bc);
+  rotate_quant_store<BPW>(v, rotate, mode, static_amax, q + row * K, s_x + row,
+                          amax_row ? amax_row + row : nullptr, s_red, &s_bc);
 }
 
 // a9 + a10: gate y * SiLU(z), g_q int16 at e_g, exact-integer RMSNorm,
-// rotation, quantisation.  blockDim = 32 * (di / 256), grid = M.
+// rotation, quantisation.  blockDim = 32 * (di / 256 / BPW), grid = M.
 // gstat (nullable, [nh] u64): max |g| per head (calibration).
+template <int BPW>
 __global__ void __launch_bounds__(1024) k_gate_norm_quant(
     const int32_t *__restrict__ y, const float *__restrict__ z, int di, int hd,
     const int32_t *__restrict__ e_y, const int32_t *__restrict__ e_g_ptr,
@@ -133,69 +154,77 @@ __global__ void __launch_bounds__(1024) k_gate_norm_quant(
   __syncthreads();
   const long long row = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nb = blockDim.x >> 5;
-  const int col = warp * 256 + lane * 8;
-  const int head = col / hd;  // hd is a multiple of 8: the lane's 8 columns share a head
+  const int nw = blockDim.x >> 5;
   const int e_g = *e_g_ptr;
-  const int sg_shift = e_g - e_y[head] + 16;
-  int32_t yv[8];
-  float zv[8];
-  {
-    const int4 a = *reinterpret_cast<const int4 *>(y + row * di + col);
-    const int4 b = *reinterpret_cast<const int4 *>(y + row * di + col + 4);
-    yv[0] = a.x; yv[1] = a.y; yv[2] = a.z; yv[3] = a.w;
-    yv[4] = b.x; yv[5] = b.y; yv[6] = b.z; yv[7] = b.w;
-    const float4 c = *reinterpret_cast<const float4 *>(z + row * di + col);
-    const float4 d = *reinterpret_cast<const float4 *>(z + row * di + col + 4);
-    zv[0] = c.x; zv[1] = c.y; zv[2] = c.z; zv[3] = c.w;
-    zv[4] = d.x; zv[5] = d.y; zv[6] = d.z; zv[7] = d.w;
-  }
-  int gq[8];
-  unsigned ss0 = 0, ss1 = 0;  // g_q^2 < 2^30: four per partial fit 32 bits
-  unsigned long long gmax = 0;
+  int gq[BPW][8];
+  long long ss = 0;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int sg = silu_pwl_t(to_q16(zv[i]), tab);
-    // g = y sg as a 64-bit value from two 32-bit multiplies
-    const long long g = (long long)(((unsigned long long)(unsigned)__mulhi(yv[i], sg) << 32) |
-                                    (unsigned)(yv[i] * sg));
+  for (int b = 0; b < BPW; ++b) {
+    const int col = (warp * BPW + b) * 256 + lane * 8;
+    const int head = col / hd;  // hd is a multiple of 8: the lane's 8 columns share a head
+    const int sg_shift = e_g - e_y[head] + 16;
+    int32_t yv[8];
+    float zv[8];
+    {
+      const int4 p = *reinterpret_cast<const int4 *>(y + row * di + col);
+      const int4 r = *reinterpret_cast<const int4 *>(y + row * di + col + 4);
+      yv[0] = p.x; yv[1] = p.y; yv[2] = p.z; yv[3] = p.w;
+      yv[4] = r.x; yv[5] = r.y; yv[6] = r.z; yv[7] = r.w;
+      const float4 c = *reinterpret_cast<const float4 *>(z + row * di + col);
+      const float4 d = *reinterpret_cast<const float4 *>(z + row * di + col + 4);
+      zv[0] = c.x; zv[1] = c.y; zv[2] = c.z; zv[3] = c.w;
+      zv[4] = d.x; zv[5] = d.y; zv[6] = d.z; zv[7] = d.w;
+    }
+    unsigned ss0 = 0, ss1 = 0;  // g_q^2 < 2^30: four per partial fit 32 bits
+    unsigned long long gmax = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int sg = silu_pwl_t(to_q16(zv[i]), tab);
+      // g = y sg as a 64-bit value from two 32-bit multiplies
+      const long long g = (long long)(((unsigned long long)(unsigned)__mulhi(yv[i], sg) << 32) |
+                                      (unsigned)(yv[i] * sg));
+      if (gstat) {
+        const unsigned long long ag = (unsigned long long)(g < 0 ? -g : g);
+        gmax = ag > gmax ? ag : gmax;
+      }
+      gq[b][i] = (int)satb64(rshr64(g, sg_shift), 16);
+      const unsigned sq = (unsigned)(gq[b][i] * gq[b][i]);
+      if (i < 4) ss0 += sq;
+      else ss1 += sq;
+    }
+    ss += (long long)ss0 + ss1;
     if (gstat) {
-      const unsigned long long ag = (unsigned long long)(g < 0 ? -g : g);
-      gmax = ag > gmax ? ag : gmax;
-    }
-    gq[i] = (int)satb64(rshr64(g, sg_shift), 16);
-    const unsigned sq = (unsigned)(gq[i] * gq[i]);
-    if (i < 4) ss0 += sq;
-    else ss1 += sq;
-  }
-  long long ss = (long long)ss0 + ss1;
-  if (gstat) {
-    // the 8 lanes of a 64-column head combine, one atomic per head
+      // the 8 lanes of a 64-column head combine, one atomic per head
 #pragma unroll
-    for (int o = 1; o < 8; o <<= 1) {
-      const unsigned long long other = __shfl_xor_sync(0xffffffffu, gmax, o);
-      gmax = other > gmax ? other : gmax;
+      for (int o = 1; o < 8; o <<= 1) {
+        const unsigned long long other = __shfl_xor_sync(0xffffffffu, gmax, o);
+        gmax = other > gmax ? other : gmax;
+      }
+      if ((lane & 7) == 0) atomicMax(gstat + head, gmax);
     }
-    if ((lane & 7) == 0) atomicMax(gstat + head, gmax);
   }
   ss = warp_sum_ll(ss);
   if (lane == 0) s_ss[warp] = ss;
   __syncthreads();
   if (threadIdx.x == 0) {
     long long tot = 0;
-    for (int b = 0; b < nb; ++b) tot += s_ss[b];
+    for (int w = 0; w < nw; ++w) tot += s_ss[w];
     const double var = __ddiv_rn(ldexp((double)tot, 2 * e_g), (double)di);
     s_rstd = (float)__drcp_rn(__dsqrt_rn(__dadd_rn(var, 1e-5)));
   }
   __syncthreads();
   const float rstd = s_rstd;
   const float scale = ldexpf(1.0f, e_g);
-  const float *w = norm_w + col;
-  float v[8];
+  float v[BPW][8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(__fmul_rn(__fmul_rn(small_i2f(gq[i]), scale), rstd), w[i]);
-  rotate_quant_store(v, rotate, mode, static_amax, q + row * di, s_x + row,
-                     amax_row ? amax_row + row : nullptr, s_red, &s_bc);
+  for (int b = 0; b < BPW; ++b) {
+    const float *w = norm_w + (warp * BPW + b) * 256 + lane * 8;
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      v[b][i] = __fmul_rn(__fmul_rn(__fmul_rn(small_i2f(gq[b][i]), scale), rstd), w[i]);
+  }
+  rotate_quant_store<BPW>(v, rotate, mode, static_amax, q + row * di, s_x + row,
+                          amax_row ? amax_row + row : nullptr, s_red, &s_bc);
 }
 
 // Offline weight preparation: W' = W H (fp64, same butterfly order),

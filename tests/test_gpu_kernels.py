@@ -426,8 +426,11 @@ def test_ssm_scan_clamp_regimes(L, regime):
 
 @pytest.mark.parametrize("M", [1, 77, 512])
 @pytest.mark.parametrize("mode", [0, 1])
-def test_gate_norm_quant(L, M, mode):
-    s = MAMBA130
+@pytest.mark.parametrize("di", [1536, 768, 5120])
+def test_gate_norm_quant(L, M, mode, di):
+    """d_inner with an even number of 256-blocks (two per warp) and an odd one
+    (one per warp)."""
+    s = S.MixerShape(d_model=768, d_inner=di, headdim=64, d_state=128)
     y = S.uniform_ints((M, s.d_inner), -2 ** 29, 2 ** 29, seed=M, dtype=np.int32)
     z = S.normal((M, s.d_inner), 3.0, seed=M + 1)
     e_y = S.uniform_ints(s.nheads, -22, -18, seed=M + 2)
