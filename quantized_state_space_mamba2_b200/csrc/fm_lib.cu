@@ -225,7 +225,8 @@ static int sm_count() {
 // Large problems: the persistent kernel, 128 x 256 tiles when there are at
 // least two per SM (fewer L2 bytes per MMA), else 128 x 128.  Small grids
 // (fewer 128-wide tiles than SMs, e.g. out_proj at 130M shapes or a decode
-// batch): one 128 x 64 tile per CTA, two CTAs per SM.
+// batch): one 128 x 64 tile per CTA (128 x 32 when even those are fewer than
+// the SMs), two CTAs per SM.
 static fm_status launch_gemm(const int8_t *A, long long M, const int8_t *W, long long N,
                              long long K, const GemmEpilogue &ep, cudaStream_t s) {
   if (K % kGemmBK) return fail(FM_ERR_SHAPE, "gemm: K=%lld is not a multiple of 128", K);
@@ -243,6 +244,10 @@ static fm_status launch_gemm(const int8_t *A, long long M, const int8_t *W, long
   if (tiles128 >= sms) {
     FM_TRY(make_tmap(&tb, W, N, K, 128));
     return launch_gemm_persist<128, 6, 8>(ta, tb, M, N, K, sms, ep, s);
+  }
+  if (mt * ((N + 63) / 64) < sms) {  // fewer 64-wide tiles than SMs: halve the tile width
+    FM_TRY(make_tmap(&tb, W, N, K, 32));
+    return launch_gemm_t<32, 6>(ta, tb, M, N, K, ep, s);
   }
   FM_TRY(make_tmap(&tb, W, N, K, 64));
   return launch_gemm_t<64, 4>(ta, tb, M, N, K, ep, s);

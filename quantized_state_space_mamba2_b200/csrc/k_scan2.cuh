@@ -436,7 +436,8 @@ __global__ void __launch_bounds__(PC *(128 / NPT) + 32) k_scan_seq(ScanSeqArgs a
 // channels: warp w owns channels w, w + 8, ..., w + 56 and lane l the state
 // columns 4l .. 4l + 3, so each thread has eight 16-byte state loads in flight
 // (32 KB per CTA, read and written once with streaming cache hints).  The
-// C.h sums are reduced by shuffles in the split (hi, lo) 32-bit form.  Same
+// C.h sums are added over the warp by redux.sync in the split (hi, lo) 32-bit
+// form, and lane k forms channel warp + 8k's output.  Same
 // arithmetic as one step of k_scan_seq with the clamp.  Grid (nh, B), block 256.
 constexpr int kStepPPW = 8;  // channels per warp (hd / 8 warps)
 
@@ -470,7 +471,7 @@ __global__ void __launch_bounds__(256) k_scan_step(ScanArgs a) {
     Bv[j] = (int)(int8_t)((bw >> (8 * j)) & 0xFF);
     Cv[j] = (int)(int8_t)((cw >> (8 * j)) & 0xFF);
   }
-  int yv = 0;  // lane k (< 8) ends up holding channel warp + 8k's output
+  int shi = 0, slo = 0;  // lane k (< 8) ends up holding channel warp + 8k's C.h sums
 #pragma unroll
   for (int k = 0; k < kStepPPW; ++k) {
     const long long xq = xs[k];
@@ -490,16 +491,20 @@ __global__ void __launch_bounds__(256) k_scan_step(ScanArgs a) {
       alo += Cv[j] * (int)((unsigned)v & 0xFFFFu);
     }
     if (st) __stcs(st + (warp + 8 * k) * 32 + lane, make_int4(hn[0], hn[1], hn[2], hn[3]));
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) {
-      ahi += __shfl_xor_sync(0xffffffffu, ahi, o);
-      alo += __shfl_xor_sync(0xffffffffu, alo, o);
+    ahi = __reduce_add_sync(0xffffffffu, ahi);
+    alo = __reduce_add_sync(0xffffffffu, alo);
+    if (lane == k) {
+      shi = ahi;
+      slo = alo;
     }
-    const long long sum = (long long)ahi * 65536 + alo;
-    const int yk = (int)satb64(rshr64(sum, s_y) + rshr64(Dq * xq, s_D), 32);
-    if (lane == k) yv = yk;
   }
-  if (lane < kStepPPW) a.y[(long long)b * di + (long long)h * hd + warp + 8 * lane] = yv;
+  if (lane < kStepPPW) {  // one output per lane: channel warp + 8 lane
+    const int p = warp + 8 * lane;
+    const long long xq = row[h * hd + p];
+    const long long sum = (long long)shi * 65536 + slo;
+    a.y[(long long)b * di + (long long)h * hd + p] =
+        (int)satb64(rshr64(sum, s_y) + rshr64(Dq * xq, s_D), 32);
+  }
 }
 
 }  // namespace fm
