@@ -391,7 +391,7 @@ class DecodeWorkload(StackWorkload):
     """One decode step of B sequences through the whole stack; conv and SSM
     states come from a seeded prefill and advance by one token per step."""
 
-    launches_per_layer = 7  # FWHT+quant, in_proj, conv, conv-state update, scan step, gate, out_proj
+    launches_per_layer = 6  # FWHT+quant, in_proj, conv (+ conv-state update), scan step, gate, out_proj
 
     def __init__(self, args, torch, lib, dev, rank):
         from quantized_state_space_mamba2_b200.model import DeviceStack

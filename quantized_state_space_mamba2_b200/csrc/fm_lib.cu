@@ -277,13 +277,13 @@ static fm_status launch_conv(const int8_t *u, int B, int T, int cc, const int8_t
   if (T >= kConvTT) {
     const unsigned tiles = (unsigned)((T + kConvTokens - 1) / kConvTokens);
     k_conv1d_pot<kConvTT, kConvTG><<<dim3(tiles, groups, B), kConvQuads * kConvTG, 0, s>>>(
-        u, T, cc, wq, bq, exps, conv_state, out, amax);
+        u, T, cc, wq, bq, exps, conv_state, out, amax, nullptr);
   } else {  // decode steps and short chunks: one token per thread
     k_conv1d_pot<1, 1><<<dim3((unsigned)T, groups, B), kConvQuads, 0, s>>>(
-        u, T, cc, wq, bq, exps, conv_state, out, amax);
+        u, T, cc, wq, bq, exps, conv_state, out, amax, T == 1 ? conv_state : nullptr);
   }
   FM_TRY(launched("k_conv1d_pot"));
-  if (conv_state) {
+  if (conv_state && T > 1) {  // a single step updates its state in the conv kernel
     const long long n = (long long)B * cc;
     k_conv_state_update<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(u, B, T, cc, conv_state);
     FM_TRY(launched("k_conv_state_update"));

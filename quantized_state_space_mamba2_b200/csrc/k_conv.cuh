@@ -16,7 +16,9 @@
 // dp4a against the channel's packed weights.  A block is 64 channel quads
 // (256 channels) x TG token groups; grid (token tiles, channel groups, batch).  Every (token, channel) output is
 // independent.  The conv state (the 3 inputs before the first token) is read
-// here and replaced afterwards by k_conv_state_update, in stream order.
+// here and replaced afterwards by k_conv_state_update, in stream order -- or,
+// for a single token (a decode step), by the same thread that read it
+// (state_out).
 #pragma once
 #include "fm_common.cuh"
 
@@ -45,7 +47,8 @@ template <int TT, int TG>
 __global__ void __launch_bounds__(kConvQuads *TG) k_conv1d_pot(
     const int8_t *__restrict__ u, int T, int cc, const int8_t *__restrict__ wq,
     const int32_t *__restrict__ bq, const int32_t *__restrict__ exps,
-    const int8_t *__restrict__ conv_state, int8_t *__restrict__ out, unsigned int *amax) {
+    const int8_t *conv_state, int8_t *__restrict__ out, unsigned int *amax,
+    int8_t *state_out) {
   __shared__ int tab[8];
   pwl_table_init(tab);
   __syncthreads();
@@ -68,6 +71,11 @@ __global__ void __launch_bounds__(kConvQuads *TG) k_conv1d_pot(
       raw = *reinterpret_cast<const uint32_t *>(conv_state + ((long long)b * 3 + (3 + tt)) * cc + c0);
     }
     row[r] = raw;
+  }
+  if (state_out) {  // T == 1 (one token per thread): the new state is rows t-2 .. t
+#pragma unroll
+    for (int r = 0; r < 3; ++r)
+      *reinterpret_cast<uint32_t *>(state_out + ((long long)b * 3 + r) * cc + c0) = row[r + 1];
   }
   const uint4 wp = *reinterpret_cast<const uint4 *>(wq + (long long)c0 * 4);  // 4 taps x 4 channels
   const int4 bias = *reinterpret_cast<const int4 *>(bq + c0);
