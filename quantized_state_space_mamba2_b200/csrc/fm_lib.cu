@@ -181,6 +181,50 @@ static fm_status make_tmap(CUtensorMap *tm, const int8_t *ptr, long long rows, l
   return FM_OK;
 }
 
+// 2-D output map for the GEMM epilogue's TMA stores: rows of `cols` elements
+// `row_bytes` apart, boxes of 32 x 32 elements.  fp32 boxes are 128 bytes wide
+// and use the 128B swizzle (matching the epilogue's staging layout); int8 boxes
+// are 32 bytes wide, unswizzled.
+static fm_status make_tmap_out(CUtensorMap *tm, void *ptr, bool f32, long long cols, long long rows,
+                               long long row_bytes) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(FM_ERR_UNSUPPORTED, "cuTensorMapEncodeTiled entry point unavailable");
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+  cuuint32_t box[2] = {32, 32};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(tm, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, ptr,
+                  dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(FM_ERR_CUDA, "cuTensorMapEncodeTiled (output) failed (%d)", (int)r);
+  return FM_OK;
+}
+
+static bool aligned16p(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Output maps for the persistent kernel's TMA-store epilogue; ep.tma_store
+// stays 0 (per-thread stores) where a map cannot describe the output (raw
+// accumulators requested, or a row stride that is not a multiple of 16 bytes).
+static fm_status gemm_output_maps(GemmEpilogue &ep, CUtensorMap (&tm)[3], const CUtensorMap &dummy) {
+  ep.tma_store = 0;
+  for (auto &t : tm) t = dummy;
+  if (ep.acc_out) return FM_OK;
+  if (ep.mode == 0) {
+    if ((ep.N * 4) % 16 || !aligned16p(ep.Y)) return FM_OK;
+    FM_TRY(make_tmap_out(&tm[0], ep.Y, true, ep.N, ep.M, ep.N * 4));
+  } else {
+    if ((ep.di * 4) % 16 || ep.cc % 16 || (ep.nh * 4) % 16 || ep.di % 32 || ep.cc % 32 ||
+        !aligned16p(ep.z) || !aligned16p(ep.xbc) || !aligned16p(ep.dt))
+      return FM_OK;
+    FM_TRY(make_tmap_out(&tm[0], ep.z, true, ep.di, ep.M, (long long)ep.di * 4));
+    FM_TRY(make_tmap_out(&tm[1], ep.xbc, false, ep.cc, ep.M, ep.cc));
+    FM_TRY(make_tmap_out(&tm[2], ep.dt, true, ep.nh, ep.M, (long long)ep.nh * 4));
+  }
+  ep.tma_store = 1;
+  return FM_OK;
+}
+
 // ------------------------------------------------------------------ launches
 template <int BN, int STAGES>
 static fm_status launch_gemm_t(const CUtensorMap &ta, const CUtensorMap &tb, long long M,
@@ -195,8 +239,10 @@ static fm_status launch_gemm_t(const CUtensorMap &ta, const CUtensorMap &tb, lon
 
 template <int BN, int STAGES, int EW>
 static fm_status launch_gemm_persist(const CUtensorMap &ta, const CUtensorMap &tb, long long M,
-                                     long long N, long long K, int sms, const GemmEpilogue &ep,
+                                     long long N, long long K, int sms, GemmEpilogue ep,
                                      cudaStream_t s) {
+  CUtensorMap to[3];
+  FM_TRY(gemm_output_maps(ep, to, ta));
   constexpr int smem = PersistSmem<BN, STAGES, EW>::kBytes;
   static_assert(smem <= 227 * 1024, "shared memory per CTA");
   auto kern = k_gemm_i8_persist<BN, STAGES, EW>;
@@ -204,7 +250,8 @@ static fm_status launch_gemm_persist(const CUtensorMap &ta, const CUtensorMap &t
   const int m_tiles = (int)((M + kGemmBM - 1) / kGemmBM), n_tiles = (int)((N + BN - 1) / BN);
   const long long tiles = (long long)m_tiles * n_tiles;
   const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);
-  kern<<<grid, 64 + 32 * EW, smem, s>>>(ta, tb, (int)(K / kGemmBK), m_tiles, n_tiles, ep);
+  kern<<<grid, 64 + 32 * EW, smem, s>>>(ta, tb, to[0], to[1], to[2], (int)(K / kGemmBK), m_tiles,
+                                        n_tiles, ep);
   return launched("k_gemm_i8_persist");
 }
 
@@ -239,11 +286,11 @@ static fm_status launch_gemm(const int8_t *A, long long M, const int8_t *W, long
   FM_TRY(make_tmap(&ta, A, M, K, kGemmBM));
   if (tiles256 >= 2LL * sms) {
     FM_TRY(make_tmap(&tb, W, N, K, 256));
-    return launch_gemm_persist<256, 4, 8>(ta, tb, M, N, K, sms, ep, s);
+    return launch_gemm_persist<256, 3, 8>(ta, tb, M, N, K, sms, ep, s);
   }
   if (tiles128 >= sms) {
     FM_TRY(make_tmap(&tb, W, N, K, 128));
-    return launch_gemm_persist<128, 6, 8>(ta, tb, M, N, K, sms, ep, s);
+    return launch_gemm_persist<128, 5, 8>(ta, tb, M, N, K, sms, ep, s);
   }
   if (mt * ((N + 63) / 64) < sms) {  // fewer 64-wide tiles than SMs: halve the tile width
     FM_TRY(make_tmap(&tb, W, N, K, 32));

@@ -43,6 +43,9 @@ struct GemmEpilogue {
   float *z;
   int8_t *xbc;
   float *dt;
+  // persistent kernel only: write the outputs through TMA stores (the tensor
+  // maps passed beside this struct); 0 falls back to per-thread stores
+  int tma_store;
 };
 
 // ------------------------------------------------------------ PTX wrappers
@@ -96,6 +99,30 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *tm, in
       "l"((unsigned long long)tm), "r"(c0), "r"(c1), "r"(smem_u32(bar))
       : "memory");
 }
+// TMA store of a 2-D box from shared memory (bulk-group completion)
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *tm, int c0, int c1,
+                                             const void *src) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+          (unsigned long long)tm),
+      "r"(c0), "r"(c1), "r"(smem_u32(src))
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// the shared-memory sources of every committed store have been read
+__device__ __forceinline__ void bulk_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// every committed store has completed
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 __device__ __forceinline__ void tc_fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
@@ -387,15 +414,116 @@ template <int BN, int STAGES, int EW>
 struct PersistSmem {
   static constexpr int kA = kGemmBM * kGemmBK;  // bytes per A stage
   static constexpr int kB = BN * kGemmBK;       // bytes per B stage
-  static constexpr int kBytes = 1024 /*align slack*/ + STAGES * (kA + kB) +
+  static constexpr int kStage = 4096;           // per epilogue warp: 32 rows x 128 bytes
+  static constexpr int kBytes = 1024 /*align slack*/ + STAGES * (kA + kB) + EW * kStage +
                                 (2 * STAGES + 5) * 8 /*barriers*/ + 16 /*tmem slot*/ +
                                 4 * BN * 4 /*column scales, double-buffered*/;
 };
 
+// One 32 x 32 chunk of the tile (rows: this warp's TMEM lane quarter, lane =
+// row; 32 columns from col0) written by TMA: the lanes put their rows into
+// the warp's staging buffer (128-byte rows, 16-byte pieces swizzled by row so
+// the writes avoid bank conflicts; the store's tensor map uses the same 128B
+// swizzle), then lane 0 issues the store.  The buffer is reused only after the
+// warp's previous store has read it.  Rows past M and columns past N are
+// clipped by the TMA unit.
+__device__ __forceinline__ void tma_chunk_f32(const CUtensorMap *tm, int x, int y0,
+                                              const float (&v)[32], uint8_t *stage, int lane) {
+  if (lane == 0) bulk_wait_read_all();
+  __syncwarp();
+  float4 *row = reinterpret_cast<float4 *>(stage + lane * 128);
+#pragma unroll
+  for (int q = 0; q < 8; ++q)
+    row[q ^ (lane & 7)] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_2d(tm, x, y0, stage);
+    bulk_commit();
+  }
+}
+__device__ __forceinline__ void tma_chunk_i8(const CUtensorMap *tm, int x, int y0,
+                                             const uint32_t (&codes)[8], uint8_t *stage, int lane) {
+  if (lane == 0) bulk_wait_read_all();
+  __syncwarp();
+  uint4 *row = reinterpret_cast<uint4 *>(stage + lane * 32);  // 32-byte rows, no swizzle
+  row[0] = make_uint4(codes[0], codes[1], codes[2], codes[3]);
+  row[1] = make_uint4(codes[4], codes[5], codes[6], codes[7]);
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_2d(tm, x, y0, stage);
+    bulk_commit();
+  }
+}
+
+// The epilogue of one 32-column chunk through TMA stores: dequantise (same
+// operations and order as gemm_store_chunk), add the residual (plain mode),
+// and store the fp32 values -- or, in the in_proj split, the z / xBC-code / dt
+// piece the chunk falls in (the split points are multiples of 32).
+__device__ __forceinline__ void gemm_tma_chunk(const GemmEpilogue &ep, const CUtensorMap *tm0,
+                                               const CUtensorMap *tm1, const CUtensorMap *tm2,
+                                               long long row, int row0, float sx, int col0,
+                                               uint32_t (&r)[32], const float *colw,
+                                               const float *cole, uint8_t *stage, int lane) {
+  float(&y)[32] = reinterpret_cast<float(&)[32]>(r);
+#pragma unroll
+  for (int j = 0; j < 32; j += 4) {
+    const float4 sw = *reinterpret_cast<const float4 *>(colw + j);
+    y[j] = __fmul_rn(__fmul_rn(__int2float_rn((int)r[j]), sx), sw.x);
+    y[j + 1] = __fmul_rn(__fmul_rn(__int2float_rn((int)r[j + 1]), sx), sw.y);
+    y[j + 2] = __fmul_rn(__fmul_rn(__int2float_rn((int)r[j + 2]), sx), sw.z);
+    y[j + 3] = __fmul_rn(__fmul_rn(__int2float_rn((int)r[j + 3]), sx), sw.w);
+  }
+  if (ep.mode == 0) {
+    if (ep.residual && row < ep.M) {
+      const float *res = ep.residual + row * ep.N + col0;
+      if (col0 + 32 <= ep.N) {
+#pragma unroll
+        for (int j = 0; j < 32; j += 4) {
+          const float4 rv = *reinterpret_cast<const float4 *>(res + j);
+          y[j] = __fadd_rn(rv.x, y[j]);
+          y[j + 1] = __fadd_rn(rv.y, y[j + 1]);
+          y[j + 2] = __fadd_rn(rv.z, y[j + 2]);
+          y[j + 3] = __fadd_rn(rv.w, y[j + 3]);
+        }
+      } else {
+        for (int j = 0; j < 32 && col0 + j < ep.N; ++j) y[j] = __fadd_rn(res[j], y[j]);
+      }
+    }
+    tma_chunk_f32(tm0, col0, row0, y, stage, lane);
+    return;
+  }
+  const int di = ep.di, cc = ep.cc;
+  if (col0 < di) {
+    tma_chunk_f32(tm0, col0, row0, y, stage, lane);
+  } else if (col0 < di + cc) {
+    uint32_t packed[8];
+#pragma unroll
+    for (int j = 0; j < 32; j += 4) {
+      const float4 es = *reinterpret_cast<const float4 *>(cole + j);
+      const float e4[4] = {es.x, es.y, es.z, es.w};
+      uint32_t w = 0;
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        const int code = quant127(__fmul_rn(y[j + b], e4[b]));
+        w |= ((uint32_t)(code & 0xFF)) << (8 * b);
+      }
+      packed[j / 4] = w;
+    }
+    tma_chunk_i8(tm1, col0 - di, row0, packed, stage, lane);
+  } else {
+    tma_chunk_f32(tm2, col0 - di - cc, row0, y, stage, lane);
+  }
+}
+
 template <int BN, int STAGES, int EW>
 __global__ void __launch_bounds__(64 + 32 * EW, 1)
     k_gemm_i8_persist(const __grid_constant__ CUtensorMap tmA,
-                      const __grid_constant__ CUtensorMap tmB, int num_k_blocks, int m_tiles,
+                      const __grid_constant__ CUtensorMap tmB,
+                      const __grid_constant__ CUtensorMap tmO0,
+                      const __grid_constant__ CUtensorMap tmO1,
+                      const __grid_constant__ CUtensorMap tmO2, int num_k_blocks, int m_tiles,
                       int n_tiles, GemmEpilogue ep) {
   static_assert(BN % 32 == 0 && BN >= 64 && BN <= 256, "BN");
   static_assert(EW % 4 == 0 && (BN / (EW / 4)) % 32 == 0, "epilogue split");
@@ -408,7 +536,8 @@ __global__ void __launch_bounds__(64 + 32 * EW, 1)
                                               ~static_cast<uintptr_t>(1023));
   uint8_t *sA = smem;
   uint8_t *sB = smem + STAGES * Sm::kA;
-  uint64_t *full_bar = reinterpret_cast<uint64_t *>(sB + STAGES * Sm::kB);
+  uint8_t *sOut = sB + STAGES * Sm::kB;  // [EW][4096], 1024-aligned
+  uint64_t *full_bar = reinterpret_cast<uint64_t *>(sOut + EW * Sm::kStage);
   uint64_t *empty_bar = full_bar + STAGES;
   uint64_t *tfull = empty_bar + STAGES;   // [2]
   uint64_t *tempty = tfull + 2;           // [2]
@@ -435,6 +564,13 @@ __global__ void __launch_bounds__(64 + 32 * EW, 1)
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"((unsigned long long)&tmA) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"((unsigned long long)&tmB) : "memory");
+    if (ep.tma_store) {
+      asm volatile("prefetch.tensormap [%0];" ::"l"((unsigned long long)&tmO0) : "memory");
+      if (ep.mode == 1) {
+        asm volatile("prefetch.tensormap [%0];" ::"l"((unsigned long long)&tmO1) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"((unsigned long long)&tmO2) : "memory");
+      }
+    }
   }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -514,6 +650,21 @@ __global__ void __launch_bounds__(64 + 32 * EW, 1)
     const int quarter = warp & 3;           // TMEM lanes [32 quarter, 32 quarter + 32)
     const int part = e / 4;                 // which column slice of the tile
     const int et = threadIdx.x - 64;        // 0 .. kEpiThreads-1
+    static_assert(BN <= kEpiThreads, "one staged column per epilogue thread");
+    // the scales of a tile (column s_w and PoT factor, row s_x) are loaded one
+    // tile ahead into registers, so no global latency sits between tiles
+    auto load_scales = [&](int t, float &w, float &ev, float &sxv) {
+      const int m0 = (t / n_tiles) * kGemmBM, n0 = (t % n_tiles) * BN;
+      const long long c = (long long)n0 + et;
+      w = (et < BN && c < ep.N) ? ep.s_w[c] : 0.0f;
+      ev = 0.0f;
+      if (et < BN && ep.mode == 1 && c >= ep.di && c < (long long)ep.di + ep.cc)
+        ev = pow2f(-ep.e_u[c - ep.di]);
+      const long long row = (long long)m0 + quarter * 32 + lane;
+      sxv = row < ep.M ? ep.s_x[row] : 0.0f;
+    };
+    float nw = 0.0f, ne = 0.0f, nsx = 0.0f;
+    if ((int)blockIdx.x < num_tiles) load_scales(blockIdx.x, nw, ne, nsx);
     int tl = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++tl) {
@@ -521,17 +672,15 @@ __global__ void __launch_bounds__(64 + 32 * EW, 1)
       const uint32_t use = (uint32_t)(tl >> 1);
       const int m0 = (t / n_tiles) * kGemmBM, n0 = (t % n_tiles) * BN;
       float *cw = col_w + acc * BN, *ce = col_e + acc * BN;
-      // this tile's column scales (buffer acc was last read two tiles ago,
-      // before every epilogue warp passed the previous tile's barrier)
-      for (int j = et; j < BN; j += kEpiThreads) {
-        const long long c = (long long)n0 + j;
-        cw[j] = c < ep.N ? ep.s_w[c] : 0.0f;
-        float ev = 0.0f;
-        if (ep.mode == 1 && c >= ep.di && c < (long long)ep.di + ep.cc) ev = pow2f(-ep.e_u[c - ep.di]);
-        ce[j] = ev;
+      // stage this tile's column scales (buffer acc was last read two tiles
+      // ago, before every epilogue warp passed the previous tile's barrier)
+      if (et < BN) {
+        cw[et] = nw;
+        ce[et] = ne;
       }
+      const float sx = nsx;
+      if (t + (int)gridDim.x < num_tiles) load_scales(t + gridDim.x, nw, ne, nsx);
       const long long row = (long long)m0 + quarter * 32 + lane;
-      const float sx = row < ep.M ? ep.s_x[row] : 0.0f;
       asm volatile("bar.sync 1, %0;" ::"r"(kEpiThreads) : "memory");
       if (ok) ok = mbar_wait(&tfull[acc], use & 1u);
       ok = __all_sync(0xffffffffu, ok);  // tcgen05.ld below is warp-collective
@@ -547,10 +696,17 @@ __global__ void __launch_bounds__(64 + 32 * EW, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&tempty[acc]);
           }
-          if (n0 + c < ep.N) gemm_store_chunk(ep, row, sx, (long long)n0 + c, r, cw + c, ce + c);
+          if (n0 + c < ep.N) {
+            if (ep.tma_store)
+              gemm_tma_chunk(ep, &tmO0, &tmO1, &tmO2, row, m0 + quarter * 32, sx, n0 + c, r,
+                             cw + c, ce + c, sOut + e * Sm::kStage, lane);
+            else
+              gemm_store_chunk(ep, row, sx, (long long)n0 + c, r, cw + c, ce + c);
+          }
         }
       }
     }
+    if (ep.tma_store && lane == 0) bulk_wait_all();  // stores done before the CTA exits
   }
   tc_fence_before();
   __syncthreads();
