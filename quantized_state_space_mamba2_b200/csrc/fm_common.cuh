@@ -226,11 +226,13 @@ __device__ __forceinline__ void fwht256_lane8(T (&v)[8], int lane) {
 #pragma unroll
   for (int s = 0; s < 5; ++s) {
     const int m = 1 << s;
-    const bool upper = (lane & m) != 0;
+    // lower lane: v + other, upper lane: other - v; both are other + sg v with
+    // sg = +-1 (sg v is exact, so the fused form rounds the same single sum)
+    const T sg = (lane & m) ? T(-1) : T(1);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      T other = __shfl_xor_sync(0xffffffffu, v[i], m);
-      v[i] = upper ? (other - v[i]) : (v[i] + other);
+      const T other = __shfl_xor_sync(0xffffffffu, v[i], m);
+      v[i] = fma(sg, v[i], other);
     }
   }
 #pragma unroll
