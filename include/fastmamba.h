@@ -23,9 +23,10 @@
  *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the
  *     legacy default stream).  Host-side validation happens before any
  *     launch; on error nothing is launched and a status is returned.
- *   - Kernels that wait (the GEMM's pipeline barriers) give up after a
- *     bounded number of polls and set a device error word instead of
- *     hanging; fm_sync_status() reports it.
+ *   - Kernels that wait (the GEMM's and the sequential scan's pipeline
+ *     barriers) give up after a bounded time and set a device error word
+ *     instead of hanging; fm_sync_status() reports it (FM_ERR_TIMEOUT), and
+ *     the outputs of that call are then undefined.
  *   - Shapes: K of every linear layer and d_model, d_inner are multiples of
  *     256 (the Hadamard block); headdim = 64, d_state = 128, ngroups = 1,
  *     d_conv = 4 (the Mamba2-130M / 2.7B configuration); conv_ch and
