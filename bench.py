@@ -536,7 +536,7 @@ class GemmWorkload:
         achieved = ops / (dom_ms / 1e3) / 1e12
         bf16 = (peaks or {}).get("bf16_tflops", 1590.0)
         peak = bf16 * NOMINAL_INT8_OVER_BF16
-        return {"bound": "tensor", "kernel": "fm_w8a8_gemm (k_gemm_i8_tc, tcgen05 kind::i8)",
+        return {"bound": "tensor", "kernel": "fm_w8a8_gemm (k_gemm_i8_persist, tcgen05 kind::i8)",
                 "achieved": achieved, "peak": peak, "unit": "TOPS (int8)",
                 "frac": achieved / peak, "traffic": None,
                 "peak_basis": "measured bf16 burst (bf16_tflops) x nominal int8/bf16 ratio 2",
