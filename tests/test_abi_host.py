@@ -82,3 +82,63 @@ def test_validation_rejects_before_launch(so):
     assert b"shape" in so.fm_last_error() or so.fm_last_error() != b""
     # decode requires both states
     assert so.fm_decode_step(None, None, 1, 0, None, None, None, None, 0, None) == 1
+
+
+def _fake_layer(lib, S, mode=0, static_amax=None):
+    """A layer struct whose device pointers are distinct 16-byte-aligned
+    addresses that validation never dereferences."""
+    p = [C.c_void_p(0x100000 * (i + 1)) for i in range(12)]
+    return lib.fm_layer(lib.shape_struct(S.MAMBA2_130M), 1, mode, p[0], p[1], p[2], p[3], None,
+                        p[4], p[5], p[6], p[7], p[8], p[9], p[10], static_amax)
+
+
+def test_layer_validation_before_launch(so):
+    from quantized_state_space_mamba2_b200 import lib
+    from quantized_state_space_mamba2_b200 import synth as S
+    big = 1 << 40
+    x, ws = C.c_void_p(0x7000000), C.c_void_p(0x9000000)
+    L = _fake_layer(lib, S)
+    # out overlapping x partially (a whole-tensor alias is allowed)
+    assert so.fm_mixer_prefill(C.byref(L), x, 1, 4, 0, None, None, C.c_void_p(0x7000010), ws, big,
+                               None) == 1
+    assert b"overlap" in so.fm_last_error()
+    # workspace too small
+    assert so.fm_mixer_prefill(C.byref(L), x, 1, 4, 0, None, None, x, ws, 16, None) == 4
+    # static mode without its scales
+    Ls = _fake_layer(lib, S, mode=1)
+    assert so.fm_mixer_prefill(C.byref(Ls), x, 1, 4, 0, None, None, x, ws, big, None) == 1
+    # bad activation mode
+    Lb = _fake_layer(lib, S, mode=7)
+    assert so.fm_mixer_prefill(C.byref(Lb), x, 1, 4, 0, None, None, x, ws, big, None) == 1
+    # a misaligned required layer pointer
+    Lm = _fake_layer(lib, S)
+    Lm.w_in_s = C.c_void_p(0x100004)
+    assert so.fm_mixer_prefill(C.byref(Lm), x, 1, 4, 0, None, None, x, ws, big, None) == 3
+    # misaligned optional state
+    assert so.fm_mixer_prefill(C.byref(L), x, 1, 4, 0, C.c_void_p(0x3001), None, x, ws, big,
+                               None) == 3
+    # negative sizes
+    assert so.fm_mixer_prefill(C.byref(L), x, -1, 4, 0, None, None, x, ws, big, None) == 2
+
+
+def test_scan_and_tuning_validation(so):
+    from quantized_state_space_mamba2_b200 import lib
+    from quantized_state_space_mamba2_b200 import synth as S
+    sh = lib.shape_struct(S.MAMBA2_130M)
+    f = [C.c_void_p(0x200000 * (i + 1)) for i in range(9)]
+    # workspace below fm_scan_workspace_bytes
+    need = so.fm_scan_workspace_bytes(C.byref(sh), 1, 64)
+    assert need > 256
+    assert so.fm_ssm_scan_pot(f[0], f[1], 1, 64, C.byref(sh), f[2], f[3], f[4], f[5], None, f[6],
+                              f[7], need - 16, None) == 4
+    # tile variants: compiled ones accepted, others rejected
+    for t in lib.SCAN_TILES:
+        assert so.fm_set_scan_tile(*t) == 0
+    assert so.fm_set_scan_tile(4, 4, 16) == 0
+    assert so.fm_set_scan_tile(4, 3, 16) == 1 and so.fm_set_scan_tile(16, 4, 16) == 1
+    # the PWL evaluator: unknown kind, negative count
+    assert so.fm_eval_pwl(9, f[0], 4, f[1], None) == 1
+    assert so.fm_eval_pwl(0, f[0], -1, f[1], None) == 2
+    # gate: bad mode
+    assert so.fm_gate_norm_quant(f[0], f[1], 4, C.byref(sh), f[2], f[3], 1, 5, None, f[4], f[5],
+                                 None, None) == 1
