@@ -444,3 +444,73 @@ def test_calibrated_exponents_fit_their_codes(oracle):
         assert 64 <= part.max() <= 127
     assert np.abs(tr["q_in"].astype(np.int32)).max() == 127
     assert np.abs(tr["q_out"].astype(np.int32)).max() == 127
+
+
+def test_scan_state_amax_no_decay_closed_form(oracle):
+    """The calibration statistic of the state (64-bit state at the finest
+    exponent, u = rshr(dt_q x, 1), no clamp) against a closed form: with A = 0
+    the decay is exactly 2^0 (65536 in Q.16), so the state is the running sum
+    of u_t B_t[n]; with B one-hot (code 1 at one n) and positive x codes it
+    grows monotonically, and its maximum over the head is
+    max_p sum_t rshr(dt_q[t] x[t, p], 1), dt_q taken from the scan's own
+    dt output."""
+    nh, hd, ds, T = 2, 64, 128, 24
+    di = nh * hd
+    xbc = np.zeros((1, T, di + 2 * ds), np.int8)
+    xbc[0, :, :di] = S.uniform_ints((T, di), 1, 127, seed=31, dtype=np.int8)
+    xbc[0, :, di + 5] = 1                                    # B = e_5
+    xbc[0, :, di + ds:] = S.uniform_ints((T, ds), -127, 127, seed=32, dtype=np.int8)  # C
+    dt_raw = S.normal((1, T, nh), 1.0, seed=33)
+    dt_bias = np.array([0.5, -1.0], np.float32)
+    A_q = np.zeros(nh, np.int32)
+    am = oracle.scan_state_amax(xbc, dt_raw, dt_bias, A_q, hd, ds)
+    z = np.zeros(nh, np.int32)
+    _, dtq, dA = oracle.ssm_scan_pot(xbc, dt_raw, dt_bias, A_q, z + 16384, z - 4, -4, -4, z - 12,
+                                     z - 12, z - 14, hd, ds, want_dt=True)
+    assert (dA == 65536).all()
+    x = xbc[0, :, :di].astype(np.int64).reshape(T, nh, hd)
+    u = (dtq[0].astype(np.int64)[:, :, None] * x + 1) >> 1   # rshr(., 1) = floor((v + 1) / 2)
+    expect = u.sum(axis=0).max(axis=1)
+    assert np.array_equal(am, expect)
+    assert (expect > 0).all()
+
+
+def test_output_statistic_skip_term_closed_form(oracle):
+    """The calibration statistic of the scan output (max |y| at the finer of
+    the two term exponents) against a closed form: with B = 0 the state stays
+    0, so only the skip term D x remains; with e_D + e_x the finer exponent it
+    enters unshifted and the statistic is max_{t,p} |D_q x[t, p]| per head."""
+    nh, hd, ds, T = 2, 64, 128, 12
+    di = nh * hd
+    xbc = np.zeros((1, T, di + 2 * ds), np.int8)
+    xbc[0, :, :di] = S.uniform_ints((T, di), -127, 127, seed=41, dtype=np.int8)
+    xbc[0, :, di + ds:] = S.uniform_ints((T, ds), -127, 127, seed=42, dtype=np.int8)  # C, B = 0
+    dt_raw = S.normal((1, T, nh), 1.0, seed=43)
+    dt_bias = np.zeros(nh, np.float32)
+    A_q = np.array([4000, 9000], np.int32)
+    D_q = np.array([16384, -9000], np.int32)
+    e_x, e_D = np.array([-4, -5], np.int32), np.array([-14, -13], np.int32)
+    e_B, e_C = -4, -3
+    e_h = np.array([-2, -3], np.int32)            # e_C + e_h = -5 / -6 > e_D + e_x = -18
+    e_y = np.array([-10, -10], np.int32)
+    _, ys = oracle.ssm_scan_pot(xbc, dt_raw, dt_bias, A_q, D_q, e_x, e_B, e_C, e_h, e_y, e_D,
+                                hd, ds, want_ystat=True)
+    x = xbc[0, :, :di].astype(np.int64).reshape(T, nh, hd)
+    expect = np.abs(D_q.astype(np.int64)[None, :, None] * x).max(axis=(0, 2))
+    assert np.array_equal(ys, expect)
+
+
+def test_gate_statistic_closed_form(oracle):
+    """The calibration statistic of the gate (max |g| per head, g = y
+    SiLU(z) in Q.16) against a closed form: for z >= 40, e^-z is below the
+    2^v unit's smallest step, sigma is exactly 1 (2^16 in Q.16) and the PWL
+    SiLU returns its input, so g = y rint(z 2^16)."""
+    M, nh, hd = 5, 3, 64
+    di = nh * hd
+    y = S.uniform_ints((M, di), -2 ** 20, 2 ** 20, seed=51)
+    z = (40.0 + 3.0 * np.abs(S.normal((M, di), 1.0, seed=52))).astype(np.float32)
+    e_y = np.array([-20, -21, -19], np.int32)
+    *_, gs = oracle.gate_norm_quant(y, z, hd, e_y, -20, np.ones(di, np.float32), want_gstat=True)
+    z16 = np.rint(z.astype(np.float64) * 65536.0).astype(np.int64)
+    g = np.abs(y.astype(np.int64) * z16).reshape(M, nh, hd)
+    assert np.array_equal(gs, g.max(axis=(0, 2)))
