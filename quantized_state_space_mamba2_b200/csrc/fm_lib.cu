@@ -305,8 +305,10 @@ static fm_status launch_hadamard_quant(const float *x, long long M, int K, const
                                        float *s_x, float *amax_row, cudaStream_t s) {
   if (M <= 0) return FM_OK;
 
-  const int nb = K / 256;  // two 256-blocks per warp when they pair up
-  if (nb % 2 == 0)
+  // two 256-blocks per warp when they pair up and there are rows enough to
+  // fill the GPU; a handful of rows (a decode batch) keeps one per warp
+  const int nb = K / 256;
+  if (nb % 2 == 0 && M >= 2LL * sm_count())
     k_hadamard_quant<2><<<(unsigned)M, 32 * (nb / 2), 0, s>>>(x, K, prenorm_w, rotate, mode,
                                                               static_amax, q, s_x, amax_row);
   else
@@ -673,7 +675,7 @@ static fm_status gate_impl(const int32_t *y, const float *z, long long M, const 
                            cudaStream_t s) {
   if (M <= 0) return FM_OK;
   const int nb = d.di / 256;
-  if (nb % 2 == 0)
+  if (nb % 2 == 0 && M >= 2LL * sm_count())
     k_gate_norm_quant<2><<<(unsigned)M, 32 * (nb / 2), 0, s>>>(
       y, z, d.di, d.hd, exps + X.e_y, e_g_override ? e_g_override : exps + X.e_g, norm_w, rotate,
       mode, static_amax, q, s_x, amax_row, gstat);
