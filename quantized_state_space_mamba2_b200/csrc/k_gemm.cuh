@@ -7,7 +7,8 @@
 // optional residual) or the in_proj split into z / xBC power-of-two codes /
 // dt (Mamba2 column order).
 //
-// Structure (one 128 x BN output tile per CTA, 6 warps):
+// Two kernels share the pieces below.  k_gemm_i8_tc (small grids: one
+// 128 x BN output tile per CTA, 6 warps, two CTAs per SM):
 //   warp 0      TMA producer: 128-byte-swizzled A and W tiles (128 x 128 and
 //               BN x 128 int8) into a STAGES-deep shared-memory ring;
 //   warp 1      allocates TMEM (BN columns of int32) and one elected lane
@@ -16,6 +17,9 @@
 //               accumulator;
 //   warps 2..5  epilogue: tcgen05.ld 32 columns at a time from their TMEM
 //               lane quarter, dequantise and store.
+// k_gemm_i8_persist (large grids, further below): one CTA per SM walking the
+// tiles, the accumulator double-buffered in TMEM, 8 epilogue warps writing
+// through TMA stores.
 // Every mbarrier wait is bounded by a wall-clock limit; on expiry the thread
 // sets the device error word and the kernel runs to its end (TMEM is always
 // released), so a broken pipeline can never hang the GPU.
