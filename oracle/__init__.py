@@ -12,6 +12,8 @@ Two parts:
   * ``ref_mixer_f64`` -- the unquantised Mamba2 mixer in numpy fp64 with
     exact exp / softplus / SiLU, the reference for SQNR and for the
     "naive double recurrence" check.
+  * ``stages`` -- a mixer whose stages are each quantised or exact, for the
+    per-stage error attribution and the linears-only FastMamba-LQ variant.
 
 Sources are the web pages about FastMamba (arXiv 2505.18975); citations
 use the page's section (see fm_oracle.c for the full list).

@@ -8,7 +8,12 @@ outlier channels).
 The GPU library reproduces the oracle bit for bit, so these numbers are also
 the GPU path's.  Runs on the CPU in about a quarter of an hour:
 
-    python -m oracle.sqnr_report
+    python -m oracle.sqnr_report            # rotation tables
+    python -m oracle.sqnr_report --stages   # per-stage attribution only
+
+The attribution (``oracle.stages``) quantises the stages of one layer alone
+and cumulatively, in pipeline order; its first row is FastMamba-LQ, the
+linears-only variant.
 """
 from __future__ import annotations
 
@@ -22,6 +27,7 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 import oracle as O  # noqa: E402
+from oracle import stages as ST  # noqa: E402
 from quantized_state_space_mamba2_b200 import synth as S  # noqa: E402
 
 OUTLIER_SEED = 4242
@@ -64,7 +70,40 @@ def stack_case(rotate: int, mode: int, layers: int = 4, T: int = 256):
     return out
 
 
+def stage_rows(mode: int, T: int = 256):
+    """SQNR (dB) of one rotated 130M-shaped layer with the named stages
+    quantised, calibrated as in ``layer_case`` (8 outlier channels x50)."""
+    shape = S.MAMBA2_130M
+    P = S.layer_params(shape, 1000)
+    L = O.prepare_layer(P, shape, rotate=1, mode=mode)
+    O.calibrate_layer(L, S.calibration_batch(shape.d_model, T, 8, 50.0, OUTLIER_SEED))
+    x = S.activations(1, T, shape.d_model, seed=1, n_outliers=8, outlier_scale=50.0,
+                      outlier_seed=OUTLIER_SEED)
+    ref = O.ref_mixer_f64(P, shape, x)
+    rows = [("linears only (FastMamba-LQ)", ("lin",)),
+            ("conv only (PoT codes, PWL SiLU)", ("conv",)),
+            ("SoftPlus as Eq. (5), exact arithmetic", ("eq5",)),
+            ("dt, dA through the fixed-point 2^v unit", ("pwl",)),
+            ("fixed-point scan (with its dt, dA)", ("scan",)),
+            ("linears + conv", ("lin", "conv")),
+            ("linears + conv + dt, dA", ("lin", "conv", "pwl")),
+            ("linears + conv + scan", ("lin", "conv", "scan")),
+            ("all stages (the full method)", ST.STAGES)]
+    return [(name, O.sqnr_db(ref, ST.staged_mixer(L, P, x, q))) for name, q in rows]
+
+
+def print_stage_table():
+    dyn, sta = stage_rows(O.DYNAMIC), stage_rows(O.STATIC)
+    print("| stages quantised (rest exact fp64) | SQNR, dynamic (dB) | SQNR, static (dB) |")
+    print("|---|---|---|")
+    for (name, a), (_, b) in zip(dyn, sta):
+        print(f"| {name} | {a:.2f} | {b:.2f} |")
+
+
 def main():
+    if "--stages" in sys.argv[1:]:
+        print_stage_table()
+        return
     modes = [("dynamic", O.DYNAMIC), ("static", O.STATIC)]
     print("| input | act. scales | SQNR, rotated (dB) | SQNR, not rotated (dB) |")
     print("|---|---|---|---|")
@@ -81,6 +120,8 @@ def main():
         p = stack_case(0, m)
         print(f"| 8 outlier channels x50 | {mname} | {' / '.join(f'{v:.1f}' for v in r)} | "
               f"{' / '.join(f'{v:.1f}' for v in p)} |")
+    print()
+    print_stage_table()
 
 
 if __name__ == "__main__":
