@@ -478,11 +478,14 @@ def ref_scan_f64(xs, Bm, Cm, dt, A, D, h0=None):
     return y, h
 
 
-def ref_mixer_f64(params: dict, shape, x, prenorm=False, residual=False, return_state=False):
+def ref_mixer_f64(params: dict, shape, x, prenorm=False, residual=False, return_state=False,
+                  stats=None):
     """Unquantised Mamba2 mixer (the paper's reference [2]; flow of Fig. 2) in
     fp64 with exact nonlinearities: in_proj -> causal depthwise conv + SiLU ->
     selective scan (dt = softplus(dt_raw + dt_bias), dA = exp(dt A),
-    h = dA h + dt x B, y = C.h + D x) -> y * SiLU(z) -> RMSNorm -> out_proj."""
+    h = dA h + dt x B, y = C.h + D x) -> y * SiLU(z) -> RMSNorm -> out_proj.
+    ``stats`` (a dict, optional) receives the per-channel max |.| of the two
+    linears' inputs over all tokens ("in_absmax", "out_absmax")."""
     s = shape
     di, ds, nh, hd, cc = s.d_inner, s.d_state, s.nheads, s.headdim, s.conv_ch
     x = np.asarray(x, np.float64)
@@ -491,6 +494,8 @@ def ref_mixer_f64(params: dict, shape, x, prenorm=False, residual=False, return_
     if prenorm:
         u = u / np.sqrt((u * u).mean(-1, keepdims=True) + 1e-5) * params["prenorm_w"]
     Y = u @ params["w_in"].astype(np.float64).T
+    if stats is not None:
+        stats["in_absmax"] = np.abs(u).reshape(-1, dm).max(axis=0)
     z, xBC, dt_raw = Y[..., :di], Y[..., di:di + cc], Y[..., di + cc:]
     xc = _silu(ref_conv_f64(xBC, params["conv_w"].astype(np.float64),
                              params["conv_b"].astype(np.float64)))
@@ -500,6 +505,8 @@ def ref_mixer_f64(params: dict, shape, x, prenorm=False, residual=False, return_
     y, h = ref_scan_f64(xs, Bm, Cm, dt, A, params["D"].astype(np.float64))
     g = y.reshape(Bsz, T, di) * _silu(z)
     g = g / np.sqrt((g * g).mean(-1, keepdims=True) + 1e-5) * params["norm_w"]
+    if stats is not None:
+        stats["out_absmax"] = np.abs(g).reshape(-1, di).max(axis=0)
     out = g @ params["w_out"].astype(np.float64).T
     if residual:
         out = out + x

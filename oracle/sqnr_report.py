@@ -10,6 +10,7 @@ the GPU path's.  Runs on the CPU in about a quarter of an hour:
 
     python -m oracle.sqnr_report            # rotation tables
     python -m oracle.sqnr_report --stages   # per-stage attribution only
+    python -m oracle.sqnr_report --baselines  # plain W8A8 / SmoothQuant / rotated
 
 The attribution (``oracle.stages``) quantises the stages of one layer alone
 and cumulatively, in pipeline order; its first row is FastMamba-LQ, the
@@ -27,6 +28,7 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 import oracle as O  # noqa: E402
+from oracle import baselines as BL  # noqa: E402
 from oracle import stages as ST  # noqa: E402
 from quantized_state_space_mamba2_b200 import synth as S  # noqa: E402
 
@@ -100,9 +102,45 @@ def print_stage_table():
         print(f"| {name} | {a:.2f} | {b:.2f} |")
 
 
+def baseline_rows(T: int = 256):
+    """One 130M-shaped pre-norm layer (stack form, residual), 8 outlier
+    channels x50: SQNR of the mixer's contribution with plain W8A8,
+    SmoothQuant (alpha 0.5) and the Hadamard rotation, linears only (LQ) and
+    the full method, in both activation-scale modes."""
+    shape = S.MAMBA2_130M
+    P = S.layer_params(shape, 1000)
+    xc = S.calibration_batch(shape.d_model, T, 8, 50.0, OUTLIER_SEED)
+    x = S.activations(1, T, shape.d_model, seed=1, n_outliers=8, outlier_scale=50.0,
+                      outlier_seed=OUTLIER_SEED)
+    xr = x.astype(np.float64)
+    ref = O.ref_mixer_f64(P, shape, x, prenorm=True, residual=True) - xr
+    Q = BL.smooth_params(P, shape, xc)
+    rows = []
+    for name, prm, rot in (("plain W8A8", P, 0), ("SmoothQuant, alpha 0.5", Q, 0),
+                           ("Hadamard rotation (the method)", P, 1)):
+        vals = []
+        for mode in (O.DYNAMIC, O.STATIC):
+            L = O.prepare_layer(prm, shape, rotate=rot, mode=mode, prenorm=True)
+            O.calibrate_layer(L, xc, residual=True)
+            vals.append(O.sqnr_db(ref, ST.lq_mixer(L, prm, x, residual=True) - xr))
+            vals.append(O.sqnr_db(ref, O.mixer_prefill(L, x, residual=True) - xr))
+        rows.append((name, vals))
+    return rows
+
+
+def print_baseline_table():
+    print("| linears | LQ, dynamic (dB) | full, dynamic (dB) | LQ, static (dB) | full, static (dB) |")
+    print("|---|---|---|---|---|")
+    for name, v in baseline_rows():
+        print(f"| {name} | " + " | ".join(f"{a:.2f}" for a in v) + " |")
+
+
 def main():
     if "--stages" in sys.argv[1:]:
         print_stage_table()
+        return
+    if "--baselines" in sys.argv[1:]:
+        print_baseline_table()
         return
     modes = [("dynamic", O.DYNAMIC), ("static", O.STATIC)]
     print("| input | act. scales | SQNR, rotated (dB) | SQNR, not rotated (dB) |")
@@ -122,6 +160,8 @@ def main():
               f"{' / '.join(f'{v:.1f}' for v in p)} |")
     print()
     print_stage_table()
+    print()
+    print_baseline_table()
 
 
 if __name__ == "__main__":
