@@ -86,7 +86,12 @@ def _declare(L):
         "fmo_prepare_ssm": (None, [_P, _P, _I, _P, _P, _P]),
         "fmo_ssm_scan_pot": (None, [_P, _P, _P, _P, _P, _P, _I, _I, _P, _P, _P,
                                     _I, _I, _I, _I, _I, _P, _P, _P, _P, _P]),
+        "fmo_ssm_scan_pot_x": (None, [_P, _P, _P, _P, _P, _P, _I, _I, _P, _P, _P,
+                                      _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _I, _P]),
         "fmo_scan_state_amax": (None, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
+        "fmo_scan_state_amax_x": (None, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _I]),
+        "fmo_conv1d_pot_x": (None, [_P, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
+        "fmo_requant_per_token": (None, [_P, _I64, _I, _I, _I, _P, _P, _P]),
         "fmo_gate_norm_quant": (None, [_P, _P, _I64, _I, _I, _P, _I, _P, _I, _I, _F,
                                        _P, _P, _P, _P]),
         "fmo_eval_array": (None, [_I, _P, _I64, _I, _P]),
@@ -210,19 +215,34 @@ def prepare_conv(w, b, e_u=None):
     return wq, bq, e_w
 
 
-def conv1d_pot(u, wq, bq, e_u, e_w, e_o, conv_state=None, want_amax=False):
-    """u: int8 [B, T, cc]; conv_state (int8 [B,3,cc]) is updated in place."""
+def conv1d_pot(u, wq, bq, e_u, e_w, e_o, conv_state=None, want_amax=False, want_s16=False):
+    """u: int8 [B, T, cc]; conv_state (int8 [B,3,cc]) is updated in place.
+    want_s16 adds the Q.16 SiLU values before requantisation (int32 [B,T,cc])."""
     u = _c(u, np.int8)
     Bsz, T, cc = u.shape
     out = np.empty_like(u)
     am = np.zeros(cc, np.int64) if want_amax else None
+    s16 = np.empty((Bsz, T, cc), np.int32) if want_s16 else None
     if conv_state is not None:
         assert conv_state.dtype == np.int8 and conv_state.flags.c_contiguous
-    lib().fmo_conv1d_pot(_p(u), Bsz, T, cc, _p(_c(wq, np.int8)),
-                         _p(None if bq is None else _c(bq, np.int32)), _p(_c(e_u, np.int32)),
-                         _p(_c(e_w, np.int32)), _p(_c(e_o, np.int32)), _p(conv_state), _p(out),
-                         _p(am))
-    return (out, am) if want_amax else out
+    lib().fmo_conv1d_pot_x(_p(u), Bsz, T, cc, _p(_c(wq, np.int8)),
+                           _p(None if bq is None else _c(bq, np.int32)), _p(_c(e_u, np.int32)),
+                           _p(_c(e_w, np.int32)), _p(_c(e_o, np.int32)), _p(conv_state), _p(out),
+                           _p(am), _p(s16))
+    res = [out] + ([am] if want_amax else []) + ([s16] if want_s16 else [])
+    return res[0] if len(res) == 1 else tuple(res)
+
+
+def requant_per_token(s16, nh, hd, ds, e_o):
+    """Per-token PoT requantisation of the conv's Q.16 SiLU values [B,T,cc]:
+    returns (int8 codes [B,T,cc], exponents int32 [B,T,nh+2])."""
+    s16 = _c(s16, np.int32)
+    Bsz, T, cc = s16.shape
+    codes = np.empty((Bsz, T, cc), np.int8)
+    e_tok = np.empty((Bsz, T, nh + 2), np.int32)
+    lib().fmo_requant_per_token(_p(s16), Bsz * T, nh, hd, ds, _p(_c(e_o, np.int32)), _p(e_tok),
+                                _p(codes))
+    return codes, e_tok
 
 
 def prepare_ssm(a_log, D):
@@ -236,9 +256,11 @@ def prepare_ssm(a_log, D):
 
 
 def ssm_scan_pot(xbc, dt_raw, dt_bias, A_q, D_q, e_x, e_B, e_C, e_h, e_y, e_D, hd, ds,
-                 state=None, want_dt=False, want_ystat=False):
+                 state=None, want_dt=False, want_ystat=False, state_bits=31, e_tok=None):
     """xbc int8 [B,T,cc] (conv output), dt_raw fp32 [B,T,nh]; state int32 [B,nh,hd,ds]
-    is updated in place.  Returns y int32 [B,T,nh*hd] (+ extras)."""
+    is updated in place.  Returns y int32 [B,T,nh*hd] (+ extras).  state_bits
+    is the state word's width reading (31: the method as built; 16: int16);
+    e_tok (int32 [B,T,nh+2]) gives per-token exponents of x, B, C."""
     xbc = _c(xbc, np.int8)
     Bsz, T, cc = xbc.shape
     nh = len(A_q)
@@ -248,11 +270,16 @@ def ssm_scan_pot(xbc, dt_raw, dt_bias, A_q, D_q, e_x, e_B, e_C, e_h, e_y, e_D, h
     ys = np.zeros(nh, np.int64) if want_ystat else None
     if state is not None:
         assert state.dtype == np.int32 and state.flags.c_contiguous
-    lib().fmo_ssm_scan_pot(_p(xbc), _p(_c(dt_raw, np.float32)), _p(_c(dt_bias, np.float32)),
-                           _p(_c(A_q, np.int32)), _p(_c(D_q, np.int32)), _p(_c(e_x, np.int32)),
-                           int(e_B), int(e_C), _p(_c(e_h, np.int32)), _p(_c(e_y, np.int32)),
-                           _p(_c(e_D, np.int32)), Bsz, T, nh, hd, ds, _p(state), _p(y), _p(dtq),
-                           _p(dA), _p(ys))
+    if not 8 <= state_bits <= 31:
+        raise ValueError("state_bits must be in [8, 31]")
+    et = None if e_tok is None else _c(e_tok, np.int32)
+    if et is not None:
+        assert et.shape == (Bsz, T, nh + 2)
+    lib().fmo_ssm_scan_pot_x(_p(xbc), _p(_c(dt_raw, np.float32)), _p(_c(dt_bias, np.float32)),
+                             _p(_c(A_q, np.int32)), _p(_c(D_q, np.int32)), _p(_c(e_x, np.int32)),
+                             int(e_B), int(e_C), _p(_c(e_h, np.int32)), _p(_c(e_y, np.int32)),
+                             _p(_c(e_D, np.int32)), Bsz, T, nh, hd, ds, _p(state), _p(y), _p(dtq),
+                             _p(dA), _p(ys), int(state_bits), _p(et))
     out = [y]
     if want_dt:
         out += [dtq, dA]
@@ -261,13 +288,17 @@ def ssm_scan_pot(xbc, dt_raw, dt_bias, A_q, D_q, e_x, e_B, e_C, e_h, e_y, e_D, h
     return out[0] if len(out) == 1 else tuple(out)
 
 
-def scan_state_amax(xbc, dt_raw, dt_bias, A_q, hd, ds):
+def scan_state_amax(xbc, dt_raw, dt_bias, A_q, hd, ds, e_tok=None, e_x=None, e_B=0):
+    """Max |h| per head at the finest exponent e_x + e_B - 15; with per-token
+    exponents e_tok, at that of the static e_x, e_B given."""
     xbc = _c(xbc, np.int8)
     Bsz, T, cc = xbc.shape
     nh = len(A_q)
     am = np.zeros(nh, np.int64)
-    lib().fmo_scan_state_amax(_p(xbc), _p(_c(dt_raw, np.float32)), _p(_c(dt_bias, np.float32)),
-                              _p(_c(A_q, np.int32)), Bsz, T, nh, hd, ds, _p(am))
+    et = None if e_tok is None else _c(e_tok, np.int32)
+    lib().fmo_scan_state_amax_x(_p(xbc), _p(_c(dt_raw, np.float32)), _p(_c(dt_bias, np.float32)),
+                                _p(_c(A_q, np.int32)), Bsz, T, nh, hd, ds, _p(am), _p(et),
+                                _p(None if e_x is None else _c(e_x, np.int32)), int(e_B))
     return am
 
 
@@ -325,6 +356,8 @@ class Layer:
     e_g: int = 0
     amax_in: float = 0.0
     amax_out: float = 0.0
+    state_bits: int = 31    # state word width reading (31 as built; 16 the int16 reading)
+    xbc_exponents: str = "static"   # conv output exponents: "static" per head, or "token"
     extra: dict = field(default_factory=dict)
 
     def e_o(self) -> np.ndarray:
@@ -340,7 +373,10 @@ class Layer:
                     amax_in=self.amax_in, amax_out=self.amax_out)
 
 
-def prepare_layer(params: dict, shape, rotate=1, mode=DYNAMIC, prenorm=False) -> Layer:
+def prepare_layer(params: dict, shape, rotate=1, mode=DYNAMIC, prenorm=False,
+                  state_bits=31, xbc_exponents="static") -> Layer:
+    if xbc_exponents not in ("static", "token"):
+        raise ValueError("xbc_exponents is 'static' or 'token'")
     wq_in, sw_in = prepare_linear(params["w_in"], rotate)
     wq_out, sw_out = prepare_linear(params["w_out"], rotate)
     wq, _, e_w = prepare_conv(params["conv_w"], params["conv_b"])
@@ -349,13 +385,25 @@ def prepare_layer(params: dict, shape, rotate=1, mode=DYNAMIC, prenorm=False) ->
                  wq_out=wq_out, sw_out=sw_out, conv_wq=wq, conv_e_w=e_w,
                  conv_w=_c(params["conv_w"], np.float32), conv_b=_c(params["conv_b"], np.float32), A_q=A_q, D_q=D_q, e_D=e_D,
                  dt_bias=_c(params["dt_bias"], np.float32), norm_w=_c(params["norm_w"], np.float32),
-                 prenorm_w=_c(params["prenorm_w"], np.float32) if prenorm else None)
+                 prenorm_w=_c(params["prenorm_w"], np.float32) if prenorm else None,
+                 state_bits=int(state_bits), xbc_exponents=xbc_exponents)
 
 
 def set_conv_input_exponents(L: Layer, e_u):
     """Fix the conv input exponents and quantise the conv bias at e_w + e_u."""
     L.e_u = _c(e_u, np.int32)
     _, L.conv_bq, _ = prepare_conv(L.conv_w, L.conv_b, L.e_u)
+
+
+def conv_out(L: Layer, xbc, conv_state=None):
+    """The conv stage's int8 output for the layer's exponent reading:
+    (codes [B,T,cc], per-token exponents [B,T,nh+2] or None when static)."""
+    s = L.shape
+    if L.xbc_exponents == "static":
+        return conv1d_pot(xbc, L.conv_wq, L.conv_bq, L.e_u, L.conv_e_w, L.e_o(), conv_state), None
+    _, s16 = conv1d_pot(xbc, L.conv_wq, L.conv_bq, L.e_u, L.conv_e_w, L.e_o(), conv_state,
+                        want_s16=True)
+    return requant_per_token(s16, s.nheads, s.headdim, s.d_state, L.e_o())
 
 
 def mixer_prefill(L: Layer, x, residual=False, conv_state=None, ssm_state=None, trace=None):
@@ -368,10 +416,10 @@ def mixer_prefill(L: Layer, x, residual=False, conv_state=None, ssm_state=None, 
     q, sx = hadamard_quant(x.reshape(M, dm), L.prenorm_w, L.rotate, L.mode, L.amax_in)
     acc = gemm_i8(q, L.wq_in)
     z, xbc, dt = in_proj_epilogue(acc, sx, L.sw_in, di, cc, nh, L.e_u)
-    xo = conv1d_pot(xbc.reshape(Bsz, T, cc), L.conv_wq, L.conv_bq, L.e_u, L.conv_e_w, L.e_o(),
-                    conv_state)
+    xo, e_tok = conv_out(L, xbc.reshape(Bsz, T, cc), conv_state)
     y = ssm_scan_pot(xo, dt.reshape(Bsz, T, nh), L.dt_bias, L.A_q, L.D_q, L.e_x, L.e_B, L.e_C,
-                     L.e_h, L.e_y, L.e_D, hd, ds, ssm_state)
+                     L.e_h, L.e_y, L.e_D, hd, ds, ssm_state, state_bits=L.state_bits,
+                     e_tok=e_tok)
     q2, sx2 = gate_norm_quant(y.reshape(M, di), z, hd, L.e_y, L.e_g, L.norm_w, L.rotate, L.mode,
                               L.amax_out)
     acc2 = gemm_i8(q2, L.wq_out)
@@ -411,22 +459,25 @@ def calibrate_layer(L: Layer, xcal, residual=False):
                       for h in range(nh)], np.int32)
     L.e_B = pot_exponent(am_s[di:di + ds].max(), 127.0) - 16
     L.e_C = pot_exponent(am_s[di + ds:].max(), 127.0) - 16
-    xo = conv1d_pot(xbc, L.conv_wq, L.conv_bq, L.e_u, L.conv_e_w, L.e_o())
+    xo, e_tok = conv_out(L, xbc)
     dt3 = dt.reshape(Bsz, T, nh)
-    # state exponent: 64-bit run at the finest exponent, headroom 2^29 of 2^30
-    am_h = scan_state_amax(xo, dt3, L.dt_bias, L.A_q, hd, ds)
+    # state exponent: 64-bit run at the finest exponent, headroom 2^29 of the
+    # 2^30 clamp (2^(bits-2) of 2^(bits-1) for a narrower state word)
+    am_h = scan_state_amax(xo, dt3, L.dt_bias, L.A_q, hd, ds, e_tok, L.e_x, L.e_B)
     e_f = L.e_x + L.e_B - 15
-    L.e_h = np.array([max(pot_exponent(float(am_h[h]), 2.0 ** 29) + int(e_f[h]), int(e_f[h]))
+    head = 2.0 ** (L.state_bits - 2)
+    L.e_h = np.array([max(pot_exponent(float(am_h[h]), head) + int(e_f[h]), int(e_f[h]))
                       for h in range(nh)], np.int32)
     # output exponent from max |y| at the finer term exponent
     _, ys = ssm_scan_pot(xo, dt3, L.dt_bias, L.A_q, L.D_q, L.e_x, L.e_B, L.e_C, L.e_h,
-                         np.zeros(nh, np.int32), L.e_D, hd, ds, want_ystat=True)
+                         np.zeros(nh, np.int32), L.e_D, hd, ds, want_ystat=True,
+                         state_bits=L.state_bits, e_tok=e_tok)
     e_f = np.minimum(L.e_C + L.e_h, L.e_D + L.e_x)
     lo = np.maximum(L.e_C + L.e_h, L.e_D + L.e_x) - 16
     L.e_y = np.array([max(pot_exponent(float(ys[h]), 2.0 ** 29) + int(e_f[h]), int(lo[h]))
                       for h in range(nh)], np.int32)
     y = ssm_scan_pot(xo, dt3, L.dt_bias, L.A_q, L.D_q, L.e_x, L.e_B, L.e_C, L.e_h, L.e_y, L.e_D,
-                     hd, ds)
+                     hd, ds, state_bits=L.state_bits, e_tok=e_tok)
     # gate exponent (int16 g), then the out_proj input amax
     # (the statistic does not depend on e_g; the pass uses its lower bound so
     # that every gate shift is a right shift)

@@ -70,6 +70,7 @@ static int64_t floor_div_pow2(int64_t a, int s) /* floor(a / 2^s), s in [0,62] *
 
 int64_t fmo_rshr(int64_t a, int s)
 {
+    if (s >= 63) return 0; /* floor((a + 2^(s-1)) / 2^s) = 0 for every |a| < 2^62 */
     if (s > 0) return floor_div_pow2(a + ((int64_t)1 << (s - 1)), s);
     if (s == 0) return a;
     return a * ((int64_t)1 << (-s));
@@ -88,6 +89,12 @@ static int64_t shl_sat61(int64_t a, int k)
     int64_t m = a < 0 ? -a : a;
     if (k >= 61 || m > (LIM >> k)) return a < 0 ? -LIM : LIM;
     return a * ((int64_t)1 << k);
+}
+
+/* a * 2^k for any k: a left shift saturated to +-2^61, or rshr for k < 0. */
+static int64_t pow2_sat61(int64_t a, int k)
+{
+    return k >= 0 ? shl_sat61(a, k) : fmo_rshr(a, -k);
 }
 
 /* fp32 value -> nearest integer (half to even), clamped to +-lim; computed
@@ -405,9 +412,10 @@ void fmo_prepare_conv(const float *w, const float *b, int cc, const int32_t *e_u
  * s = SiLU_pwl(xq16),  out = satb(rshr(s, e_o[c] + 16), 8).
  * conv_state (nullable) is read as history and replaced by the last 3 inputs.
  * amax_silu (nullable, per channel) accumulates max |s| (calibration). */
-void fmo_conv1d_pot(const int8_t *u, int B, int T, int cc, const int8_t *wq, const int32_t *bq,
-                    const int32_t *e_u, const int32_t *e_w, const int32_t *e_o,
-                    int8_t *conv_state, int8_t *out, int64_t *amax_silu)
+void fmo_conv1d_pot_x(const int8_t *u, int B, int T, int cc, const int8_t *wq,
+                      const int32_t *bq, const int32_t *e_u, const int32_t *e_w,
+                      const int32_t *e_o, int8_t *conv_state, int8_t *out, int64_t *amax_silu,
+                      int32_t *s16_out)
 {
     for (int b = 0; b < B; ++b)
         for (int c = 0; c < cc; ++c) {
@@ -424,6 +432,7 @@ void fmo_conv1d_pot(const int8_t *u, int B, int T, int cc, const int8_t *wq, con
                 }
                 int64_t x16 = fmo_sat(fmo_rshr(acc, -(ea + 16)), 32);
                 int64_t s = fmo_silu_pwl(x16);
+                if (s16_out) s16_out[((int64_t)b * T + t) * cc + c] = (int32_t)s;
                 if (amax_silu) {
                     int64_t a = s < 0 ? -s : s;
                     if (a > amax_silu[c]) amax_silu[c] = a;
@@ -438,6 +447,42 @@ void fmo_conv1d_pot(const int8_t *u, int B, int T, int cc, const int8_t *wq, con
                 }
                 for (int k = 0; k < 3; ++k) conv_state[((int64_t)b * 3 + k) * cc + c] = (int8_t)all[k];
             }
+        }
+}
+
+/* s16_out (nullable, [B,T,cc]): the Q.16 SiLU values before requantisation. */
+void fmo_conv1d_pot(const int8_t *u, int B, int T, int cc, const int8_t *wq, const int32_t *bq,
+                    const int32_t *e_u, const int32_t *e_w, const int32_t *e_o,
+                    int8_t *conv_state, int8_t *out, int64_t *amax_silu)
+{
+    fmo_conv1d_pot_x(u, B, T, cc, wq, bq, e_u, e_w, e_o, conv_state, out, amax_silu, NULL);
+}
+
+/* Per-token power-of-two exponents for the conv output (the "fine-grained"
+ * granularity read per token instead of per calibrated head; [carry] leaves
+ * the granularity open).  For token m and group g (head h's x channels, then
+ * B, then C) the exponent is E(max_g |s| / 2^16, 127), floored 16 below the
+ * group's calibrated static exponent (e_o of its first channel), and the
+ * codes are satb(rshr(s, e + 16), 8).  e_tok is [M, nh + 2]. */
+void fmo_requant_per_token(const int32_t *s16, int64_t M, int nh, int hd, int ds,
+                           const int32_t *e_o, int32_t *e_tok, int8_t *codes)
+{
+    int cc = nh * hd + 2 * ds;
+    for (int64_t m = 0; m < M; ++m)
+        for (int g = 0; g < nh + 2; ++g) {
+            int c0 = g < nh ? g * hd : nh * hd + (g - nh) * ds;
+            int n = g < nh ? hd : ds;
+            int64_t amax = 0;
+            for (int c = c0; c < c0 + n; ++c) {
+                int64_t v = s16[m * cc + c];
+                v = v < 0 ? -v : v;
+                if (v > amax) amax = v;
+            }
+            int e = fmo_pot_exponent((double)amax, 127.0) - 16;
+            if (e < e_o[c0] - 16) e = e_o[c0] - 16;
+            e_tok[m * (nh + 2) + g] = e;
+            for (int c = c0; c < c0 + n; ++c)
+                codes[m * cc + c] = (int8_t)fmo_sat(fmo_rshr(s16[m * cc + c], e + 16), 8);
         }
 }
 
@@ -468,7 +513,7 @@ static void dt_dA(float dt_raw, float dt_bias, int32_t A_q, int64_t *dt_q, int64
     *dA_q = fmo_pow2_pwl(-fmo_rshr(d * (int64_t)A_q, 12));
 }
 
-#define H_LIM ((int64_t)(1 << 30) - 1) /* state saturates at +-(2^30 - 1) */
+#define H_BITS 31                      /* state saturates at +-(2^30 - 1) */
 #define U_BITS 24                      /* dt*x factor saturates at +-(2^23 - 1) */
 
 /* The recurrence, per (b, head h, p, n), over t in order (Mamba2 SSM, [fig2]):
@@ -481,25 +526,35 @@ static void dt_dA(float dt_raw, float dt_bias, int32_t A_q, int64_t *dt_q, int64
  * dtq_out / dA_out (nullable, [B,T,nh]) expose the per-head fixed-point dt and dA.
  * ystat (nullable, per head): max |y| measured at the finer of the two term
  * exponents ef (calibration): y_f = acc * 2^(e_C+e_h-ef) + D_q x_q 2^(e_D+e_x-ef),
- * each term saturated at +-2^61. */
-void fmo_ssm_scan_pot(const int8_t *xbc, const float *dt_raw, const float *dt_bias,
-                      const int32_t *A_q, const int32_t *D_q, const int32_t *e_x, int e_B,
-                      int e_C, const int32_t *e_h, const int32_t *e_y, const int32_t *e_D,
-                      int B, int T, int nh, int hd, int ds, int32_t *state, int32_t *y,
-                      int32_t *dtq_out, int32_t *dA_out, int64_t *ystat)
+ * each term saturated at +-2^61.
+ * hbits: the state word's width reading; the state clamps at +-(2^(hbits-1) - 1).
+ * 31 is the method as built (an int32 word with one bit of headroom); 16 is
+ * the narrower int16 reading (the pages fix no width).
+ * e_tok (nullable, [B*T, nh+2]): per-token exponents of x (per head), B and C
+ * replacing e_x, e_B, e_C in s_h, s_y, s_D; ystat then still measures at the
+ * finer of e_C + e_h and e_D + e_x with the static e_x, e_C given. */
+void fmo_ssm_scan_pot_x(const int8_t *xbc, const float *dt_raw, const float *dt_bias,
+                        const int32_t *A_q, const int32_t *D_q, const int32_t *e_x, int e_B,
+                        int e_C, const int32_t *e_h, const int32_t *e_y, const int32_t *e_D,
+                        int B, int T, int nh, int hd, int ds, int32_t *state, int32_t *y,
+                        int32_t *dtq_out, int32_t *dA_out, int64_t *ystat, int hbits,
+                        const int32_t *e_tok)
 {
+    const int64_t H_LIM = ((int64_t)1 << (hbits - 1)) - 1;
     int cc = nh * hd + 2 * ds;
     int64_t *S = (int64_t *)malloc(sizeof(int64_t) * (size_t)hd * ds);
     for (int b = 0; b < B; ++b)
         for (int h = 0; h < nh; ++h) {
             for (int i = 0; i < hd * ds; ++i)
                 S[i] = state ? state[(((int64_t)b * nh + h) * hd) * ds + i] : 0;
-            int s_h = e_h[h] - e_B - e_x[h] + 16;
-            int s_y = e_y[h] - e_C - e_h[h];
-            int s_D = e_y[h] - e_D[h] - e_x[h];
             int ef = e_C + e_h[h] < e_D[h] + e_x[h] ? e_C + e_h[h] : e_D[h] + e_x[h];
             for (int t = 0; t < T; ++t) {
                 int64_t bt = (int64_t)b * T + t;
+                const int32_t *et = e_tok ? e_tok + bt * (nh + 2) : NULL;
+                int ex = et ? et[h] : e_x[h], eb = et ? et[nh] : e_B, ec = et ? et[nh + 1] : e_C;
+                int s_h = e_h[h] - eb - ex + 16;
+                int s_y = e_y[h] - ec - e_h[h];
+                int s_D = e_y[h] - e_D[h] - ex;
                 int64_t dtq, dA;
                 dt_dA(dt_raw[bt * nh + h], dt_bias[h], A_q[h], &dtq, &dA);
                 if (dtq_out) dtq_out[bt * nh + h] = (int32_t)dtq;
@@ -521,8 +576,8 @@ void fmo_ssm_scan_pot(const int8_t *xbc, const float *dt_raw, const float *dt_bi
                     y[bt * (nh * hd) + h * hd + p] =
                         (int32_t)fmo_sat(fmo_rshr(acc, s_y) + fmo_rshr(dx, s_D), 32);
                     if (ystat) {
-                        int64_t yf = shl_sat61(acc, e_C + e_h[h] - ef) +
-                                     shl_sat61(dx, e_D[h] + e_x[h] - ef);
+                        int64_t yf = pow2_sat61(acc, ec + e_h[h] - ef) +
+                                     pow2_sat61(dx, e_D[h] + ex - ef);
                         yf = yf < 0 ? -yf : yf;
                         if (yf > ystat[h]) ystat[h] = yf;
                     }
@@ -535,12 +590,25 @@ void fmo_ssm_scan_pot(const int8_t *xbc, const float *dt_raw, const float *dt_bi
     free(S);
 }
 
+void fmo_ssm_scan_pot(const int8_t *xbc, const float *dt_raw, const float *dt_bias,
+                      const int32_t *A_q, const int32_t *D_q, const int32_t *e_x, int e_B,
+                      int e_C, const int32_t *e_h, const int32_t *e_y, const int32_t *e_D,
+                      int B, int T, int nh, int hd, int ds, int32_t *state, int32_t *y,
+                      int32_t *dtq_out, int32_t *dA_out, int64_t *ystat)
+{
+    fmo_ssm_scan_pot_x(xbc, dt_raw, dt_bias, A_q, D_q, e_x, e_B, e_C, e_h, e_y, e_D, B, T, nh, hd,
+                       ds, state, y, dtq_out, dA_out, ystat, H_BITS, NULL);
+}
+
 /* Calibration statistic of the state: the same recurrence at the finest
  * useful exponent e_f = e_x + e_B - 15 (s_h = 1), with a 64-bit state
- * (saturating at +-2^46) and no clamp on u; returns max |h| per head. */
-void fmo_scan_state_amax(const int8_t *xbc, const float *dt_raw, const float *dt_bias,
-                         const int32_t *A_q, int B, int T, int nh, int hd, int ds,
-                         int64_t *amax_h)
+ * (saturating at +-2^46) and no clamp on u; returns max |h| per head.
+ * With per-token exponents (e_tok, [B*T, nh+2], nullable) the state stays at
+ * the static e_f of e_x, e_B (given) and u takes the token's own shift
+ * 1 + (e_x + e_B) - (ex_t + eB_t). */
+void fmo_scan_state_amax_x(const int8_t *xbc, const float *dt_raw, const float *dt_bias,
+                           const int32_t *A_q, int B, int T, int nh, int hd, int ds,
+                           int64_t *amax_h, const int32_t *e_tok, const int32_t *e_x, int e_B)
 {
     const int64_t LIM = (int64_t)1 << 46;
     int cc = nh * hd + 2 * ds;
@@ -554,8 +622,11 @@ void fmo_scan_state_amax(const int8_t *xbc, const float *dt_raw, const float *dt
                 int64_t dtq, dA;
                 dt_dA(dt_raw[bt * nh + h], dt_bias[h], A_q[h], &dtq, &dA);
                 const int8_t *row = xbc + bt * cc;
+                int sh = 1;
+                if (e_tok)
+                    sh += e_x[h] + e_B - e_tok[bt * (nh + 2) + h] - e_tok[bt * (nh + 2) + nh];
                 for (int p = 0; p < hd; ++p) {
-                    int64_t u = fmo_rshr(dtq * (int64_t)row[h * hd + p], 1);
+                    int64_t u = pow2_sat61(dtq * (int64_t)row[h * hd + p], -sh);
                     for (int n = 0; n < ds; ++n) {
                         int64_t hn = fmo_rshr(dA * S[p * ds + n], 16) + u * (int64_t)row[nh * hd + n];
                         hn = hn > LIM ? LIM : (hn < -LIM ? -LIM : hn);
@@ -567,6 +638,13 @@ void fmo_scan_state_amax(const int8_t *xbc, const float *dt_raw, const float *dt
             }
         }
     free(S);
+}
+
+void fmo_scan_state_amax(const int8_t *xbc, const float *dt_raw, const float *dt_bias,
+                         const int32_t *A_q, int B, int T, int nh, int hd, int ds,
+                         int64_t *amax_h)
+{
+    fmo_scan_state_amax_x(xbc, dt_raw, dt_bias, A_q, B, T, nh, hd, ds, amax_h, NULL, NULL, 0);
 }
 
 /* ------------------------------------------------------------------ */

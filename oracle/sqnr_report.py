@@ -11,6 +11,8 @@ the GPU path's.  Runs on the CPU in about a quarter of an hour:
     python -m oracle.sqnr_report            # rotation tables
     python -m oracle.sqnr_report --stages   # per-stage attribution only
     python -m oracle.sqnr_report --baselines  # plain W8A8 / SmoothQuant / rotated
+    python -m oracle.sqnr_report --state-bits # width of the SSM state word
+    python -m oracle.sqnr_report --readings   # conv-output exponents x state width
 
 The attribution (``oracle.stages``) quantises the stages of one layer alone
 and cumulatively, in pipeline order; its first row is FastMamba-LQ, the
@@ -135,7 +137,74 @@ def print_baseline_table():
         print(f"| {name} | " + " | ".join(f"{a:.2f}" for a in v) + " |")
 
 
+def state_bits_rows(bits=(31, 24, 20, 16), T_cal: int = 512, T: int = 1024):
+    """One rotated 130M-shaped layer calibrated on 16 x 512 tokens and run
+    over 1024: SQNR of the whole output and of its last 256 tokens for
+    each width of the state word (both activation-scale modes)."""
+    shape = S.MAMBA2_130M
+    P = S.layer_params(shape, 1000)
+    xc = S.calibration_batch(shape.d_model, T_cal, 8, 50.0, OUTLIER_SEED)
+    x = S.activations(1, T, shape.d_model, seed=1, n_outliers=8, outlier_scale=50.0,
+                      outlier_seed=OUTLIER_SEED)
+    ref = O.ref_mixer_f64(P, shape, x)
+    rows = []
+    for b in bits:
+        vals = []
+        for mode in (O.DYNAMIC, O.STATIC):
+            L = O.prepare_layer(P, shape, mode=mode, state_bits=b)
+            O.calibrate_layer(L, xc)
+            out = O.mixer_prefill(L, x)
+            vals += [O.sqnr_db(ref, out), O.sqnr_db(ref[:, -256:], out[:, -256:])]
+        rows.append((b, vals))
+    return rows
+
+
+def print_state_bits_table():
+    print("| state word | dynamic, all (dB) | dynamic, last 256 (dB) | static, all (dB) | "
+          "static, last 256 (dB) |")
+    print("|---|---|---|---|---|")
+    for b, v in state_bits_rows():
+        name = f"{b} bits" + (" (as built)" if b == 31 else "")
+        print(f"| {name} | " + " | ".join(f"{a:.2f}" for a in v) + " |")
+
+
+def readings_rows(T: int = 256):
+    """One rotated 130M-shaped layer as in ``layer_case`` (8 outlier channels
+    x50): conv-output exponents static per head or per token, with the 31-bit
+    and the 16-bit state word."""
+    shape = S.MAMBA2_130M
+    P = S.layer_params(shape, 1000)
+    xc = S.calibration_batch(shape.d_model, T, 8, 50.0, OUTLIER_SEED)
+    x = S.activations(1, T, shape.d_model, seed=1, n_outliers=8, outlier_scale=50.0,
+                      outlier_seed=OUTLIER_SEED)
+    ref = O.ref_mixer_f64(P, shape, x)
+    rows = []
+    for xe, bits in (("static", 31), ("token", 31), ("static", 16), ("token", 16)):
+        vals = []
+        for mode in (O.DYNAMIC, O.STATIC):
+            L = O.prepare_layer(P, shape, mode=mode, state_bits=bits, xbc_exponents=xe)
+            O.calibrate_layer(L, xc)
+            vals.append(O.sqnr_db(ref, O.mixer_prefill(L, x)))
+        rows.append((xe, bits, vals))
+    return rows
+
+
+def print_readings_table():
+    print("| conv-output exponents | state word | SQNR, dynamic (dB) | SQNR, static (dB) |")
+    print("|---|---|---|---|")
+    for xe, bits, v in readings_rows():
+        name = "static per head" if xe == "static" else "per token"
+        tag = " (as built)" if (xe, bits) == ("static", 31) else ""
+        print(f"| {name}{tag} | {bits} bits | {v[0]:.2f} | {v[1]:.2f} |")
+
+
 def main():
+    if "--readings" in sys.argv[1:]:
+        print_readings_table()
+        return
+    if "--state-bits" in sys.argv[1:]:
+        print_state_bits_table()
+        return
     if "--stages" in sys.argv[1:]:
         print_stage_table()
         return
@@ -162,6 +231,10 @@ def main():
     print_stage_table()
     print()
     print_baseline_table()
+    print()
+    print_state_bits_table()
+    print()
+    print_readings_table()
 
 
 if __name__ == "__main__":

@@ -71,6 +71,8 @@ def staged_mixer(L, params: dict, x, quant=(), residual=False):
     """One layer on x [B,T,dm] with the stages named in ``quant`` quantised
     (L a calibrated oracle layer, params its fp32 weights).  Returns fp64
     [B,T,dm] (the fp32 output of the quantised steps, widened)."""
+    if L.xbc_exponents != "static":
+        raise ValueError("the staged mixer follows the static conv-output exponents")
     quant = set(quant)
     bad = quant - set(STAGES) - {"eq5"}
     if bad:
@@ -125,7 +127,7 @@ def staged_mixer(L, params: dict, x, quant=(), residual=False):
     # ---- dt, dA and the scan: y as int32 codes at e_y or as fp64
     if "scan" in quant:
         y_q = ssm_scan_pot(xo_q, dt3, L.dt_bias, L.A_q, L.D_q, L.e_x, L.e_B, L.e_C, L.e_h, L.e_y,
-                           L.e_D, hd, ds).reshape(M, di)
+                           L.e_D, hd, ds, state_bits=L.state_bits).reshape(M, di)
         y_f = y_q.astype(np.float64) * np.exp2(e_y.astype(np.float64))
     else:
         if "pwl" in quant:

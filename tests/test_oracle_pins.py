@@ -514,3 +514,180 @@ def test_gate_statistic_closed_form(oracle):
     z16 = np.rint(z.astype(np.float64) * 65536.0).astype(np.int64)
     g = np.abs(y.astype(np.int64) * z16).reshape(M, nh, hd)
     assert np.array_equal(gs, g.max(axis=(0, 2)))
+
+
+# ------------------------------------------------------------------ state word width
+
+def test_narrow_state_clamps_at_its_width(oracle):
+    """A 16-bit state word: with no decay (A = 0, dA exactly 1) and a one-hot
+    B the state is the running sum of u * B clamped at 2^15 - 1, closed form
+    min(sum_t u_t * 127, 32767) in the hot column and 0 elsewhere; the 31-bit
+    word does not clamp on the same input."""
+    nh, hd, ds, T = 1, 8, 16, 40
+    di = nh * hd
+    xbc = np.zeros((1, T, di + 2 * ds), np.int8)
+    xbc[0, :, :di] = S.uniform_ints((T, di), 20, 127, seed=71, dtype=np.int8)
+    xbc[0, :, di + 3] = 127                                  # B = 127 e_3
+    dt_raw = S.normal((1, T, nh), 1.0, seed=72)
+    z = np.zeros(nh, np.int32)
+    args = (np.array([0.5], np.float32), z, z + 16384, z - 4, -4, -4, z - 9, z - 12, z - 14, hd,
+            ds)
+    sums = {}
+    for bits in (16, 31):
+        st = np.zeros((1, nh, hd, ds), np.int32)
+        _, dtq, dA = oracle.ssm_scan_pot(xbc, dt_raw, *args, state=st, want_dt=True,
+                                         state_bits=bits)
+        assert (dA == 65536).all()
+        s_h = -9 - (-4) - (-4) + 16                          # e_h - e_B - e_x + 16
+        x = xbc[0, :, :di].astype(np.int64)
+        u = (dtq[0].astype(np.int64) * x + (1 << (s_h - 1))) >> s_h     # rshr(dt_q x, s_h)
+        total = (u * 127).sum(axis=0)
+        lim = (1 << (bits - 1)) - 1
+        assert np.array_equal(st[0, 0, :, 3], np.minimum(total, lim))
+        assert not np.delete(st, 3, axis=-1).any()
+        sums[bits] = total
+    assert (sums[16] > 32767).all()                          # the narrow word really clamps
+
+
+def test_narrow_state_against_double_recurrence(oracle):
+    """A 16-bit state at a coarser exponent stays within the same per-step
+    rounding budget of the naive fp64 recurrence, when the exponent leaves
+    room for the running maximum plus the budget (so nothing clamps)."""
+    Bsz, T, nh, hd, ds = 1, 48, 2, 8, 16
+    xbc, dt_raw, dt_bias, A_q, D_q, e_D, e_x = _scan_inputs(Bsz, T, nh, hd, ds, seed=50)
+    e_B = e_C = -5
+    e_h = np.full(nh, -10, np.int32)
+    st = np.zeros((Bsz, nh, hd, ds), np.int32)
+    _, dtq, dA = oracle.ssm_scan_pot(xbc, dt_raw, dt_bias, A_q, D_q, e_x, e_B, e_C, e_h,
+                                     np.full(nh, -6, np.int32), e_D, hd, ds, state=st,
+                                     want_dt=True, state_bits=16)
+    x = xbc[..., :nh * hd].reshape(Bsz, T, nh, hd) * 2.0 ** -5
+    Bm = xbc[..., nh * hd:nh * hd + ds] * 2.0 ** e_B
+    h = np.zeros((Bsz, nh, hd, ds))
+    peak = 0.0
+    for t in range(T):
+        h = (dA[:, t] / 65536.0)[:, :, None, None] * h + \
+            (dtq[:, t, :, None] / 65536.0 * x[:, t])[..., None] * Bm[:, t, None, None, :]
+        peak = max(peak, float(np.abs(h).max()))
+    lsb = 2.0 ** e_h[0]
+    budget = T * (0.5 + 0.5 * 127 + 1) * lsb
+    assert (peak + budget) / lsb < 2 ** 15 - 1               # the word never clamps
+    assert np.max(np.abs(st * lsb - h)) <= budget
+    assert peak > 5 * budget                                 # the check is not vacuous
+
+
+# ------------------------------------------------------------------ per-token conv-output exponents
+
+def _token_case(oracle, seed=81, Bsz=2, T=30, nh=2, hd=8, ds=16):
+    """Random Q.16 SiLU values with per-token magnitudes spread over 2^10."""
+    cc = nh * hd + 2 * ds
+    mag = np.exp2(S.uniform_ints((Bsz, T, 1), 0, 10, seed=seed)).astype(np.int64)
+    s16 = (S.uniform_ints((Bsz, T, cc), -2 ** 14, 2 ** 14, seed=seed + 1).astype(np.int64)
+           * mag // 4).astype(np.int32)
+    e_o = np.concatenate([np.repeat(np.array([-2, -3], np.int32), hd),
+                          np.full(ds, -1, np.int32), np.full(ds, -2, np.int32)])
+    return s16, e_o
+
+
+def test_per_token_exponents_fit_their_codes(oracle):
+    """E(amax, 127) is the smallest exponent that holds the token's group
+    maximum: the largest code of each (token, group) is in [64, 127] unless
+    the floor (16 below the static exponent) applies; zero groups give 0."""
+    nh, hd, ds = 2, 8, 16
+    s16, e_o = _token_case(oracle)
+    s16[0, 3, :hd] = 0                                       # an all-zero head group
+    codes, e_tok = oracle.requant_per_token(s16, nh, hd, ds, e_o)
+    groups = [slice(h * hd, (h + 1) * hd) for h in range(nh)] + \
+        [slice(nh * hd, nh * hd + ds), slice(nh * hd + ds, nh * hd + 2 * ds)]
+    floors = [e_o[g.start] - 16 for g in groups]
+    for b in range(s16.shape[0]):
+        for t in range(s16.shape[1]):
+            for g, (sl, fl) in enumerate(zip(groups, floors)):
+                top = np.abs(codes[b, t, sl].astype(np.int64)).max()
+                e = e_tok[b, t, g]
+                assert e >= fl
+                if np.abs(s16[b, t, sl]).max() == 0:
+                    assert top == 0
+                elif e > fl:
+                    assert 64 <= top <= 127, (b, t, g, top)
+                # dequantised codes within half a step of the value
+                err = np.abs(codes[b, t, sl] * 2.0 ** e - s16[b, t, sl] / 65536.0)
+                assert err.max() <= 2.0 ** e / 2 + 1e-12
+
+
+def test_scan_with_static_exponents_per_token_is_the_static_scan(oracle):
+    Bsz, T, nh, hd, ds = 2, 20, 2, 8, 16
+    xbc, dt_raw, dt_bias, A_q, D_q, e_D, e_x = _scan_inputs(Bsz, T, nh, hd, ds, seed=90)
+    e_h, e_y = np.full(nh, -13, np.int32), np.full(nh, -6, np.int32)
+    e_tok = np.empty((Bsz, T, nh + 2), np.int32)
+    e_tok[..., :nh], e_tok[..., nh], e_tok[..., nh + 1] = e_x, -5, -4
+    args = (dt_bias, A_q, D_q, e_x, -5, -4, e_h, e_y, e_D, hd, ds)
+    s1, s2 = (np.zeros((Bsz, nh, hd, ds), np.int32) for _ in range(2))
+    y1, ys1 = oracle.ssm_scan_pot(xbc, dt_raw, *args, state=s1, want_ystat=True)
+    y2, ys2 = oracle.ssm_scan_pot(xbc, dt_raw, *args, state=s2, want_ystat=True, e_tok=e_tok)
+    assert np.array_equal(y1, y2) and np.array_equal(s1, s2) and np.array_equal(ys1, ys2)
+    a1 = oracle.scan_state_amax(xbc, dt_raw, dt_bias, A_q, hd, ds)
+    a2 = oracle.scan_state_amax(xbc, dt_raw, dt_bias, A_q, hd, ds, e_tok, e_x, -5)
+    assert np.array_equal(a1, a2)
+
+
+def test_per_token_scan_against_double_recurrence(oracle):
+    """Per-token exponents for x, B, C: the fixed-point state and output
+    against the naive fp64 recurrence on the values the codes stand for,
+    within the per-step rounding budget (a sign or offset slip in any
+    per-token shift moves the result by powers of two)."""
+    Bsz, T, nh, hd, ds = 1, 40, 2, 8, 16
+    xbc, dt_raw, dt_bias, A_q, D_q, e_D, _ = _scan_inputs(Bsz, T, nh, hd, ds, seed=95)
+    e_tok = S.uniform_ints((Bsz, T, nh + 2), -9, -5, seed=96)
+    e_x, e_B, e_C = np.full(nh, -5, np.int32), -5, -5        # the static references
+    e_h, e_y = np.full(nh, -22, np.int32), np.full(nh, -14, np.int32)
+    st = np.zeros((Bsz, nh, hd, ds), np.int32)
+    y, dtq, dA = oracle.ssm_scan_pot(xbc, dt_raw, dt_bias, A_q, D_q, e_x, e_B, e_C, e_h, e_y,
+                                     e_D, hd, ds, state=st, want_dt=True, e_tok=e_tok)
+    x = xbc[..., :nh * hd].reshape(Bsz, T, nh, hd) * np.exp2(e_tok[..., :nh, None])
+    Bm = xbc[..., nh * hd:nh * hd + ds] * np.exp2(e_tok[..., nh, None])
+    Cm = xbc[..., nh * hd + ds:] * np.exp2(e_tok[..., nh + 1, None])
+    D = D_q * 2.0 ** e_D
+    h = np.zeros((Bsz, nh, hd, ds))
+    yr = np.empty((Bsz, T, nh, hd))
+    for t in range(T):
+        h = (dA[:, t] / 65536.0)[:, :, None, None] * h + \
+            (dtq[:, t, :, None] / 65536.0 * x[:, t])[..., None] * Bm[:, t, None, None, :]
+        yr[:, t] = np.einsum("bhpn,bn->bhp", h, Cm[:, t]) + D[None, :, None] * x[:, t]
+    lsb = 2.0 ** -22
+    budget = T * (0.5 + 0.5 * 127 + 1) * lsb
+    assert np.max(np.abs(st * lsb - h)) <= budget
+    assert np.max(np.abs(h)) > 100 * budget
+    # output: the state error times sum |C|, plus the two output roundings
+    ybud = budget * np.abs(Cm).sum(-1).max() + 2 ** -14
+    assert np.max(np.abs(y.reshape(Bsz, T, nh, hd) * 2.0 ** -14 - yr)) <= ybud
+    assert np.max(np.abs(yr)) > 50 * ybud
+
+
+def test_per_token_layer_chunking_and_gain(oracle):
+    """A layer with per-token conv-output exponents: chunked prefill plus
+    decode steps equal one prefill bit for bit (the exponents depend on the
+    token alone), and on outlier inputs it is closer to fp64 than the
+    static-exponent layer."""
+    P = S.layer_params(SMALL, 3)
+    xc = S.calibration_batch(256, 64, 4, 50.0, outlier_seed=99, n_seqs=2)
+    Ls = {}
+    for xe in ("static", "token"):
+        Ls[xe] = oracle.prepare_layer(P, SMALL, xbc_exponents=xe)
+        oracle.calibrate_layer(Ls[xe], xc)
+    L, s = Ls["token"], SMALL
+    x = S.activations(2, 10, 256, seed=6, n_outliers=4, outlier_scale=50.0, outlier_seed=99)
+    cs0, ss0 = np.zeros((2, 3, s.conv_ch), np.int8), np.zeros((2, s.nheads, s.headdim, s.d_state),
+                                                              np.int32)
+    full = oracle.mixer_prefill(L, x, conv_state=cs0, ssm_state=ss0)
+    cs, ss = np.zeros_like(cs0), np.zeros_like(ss0)
+    parts = [oracle.mixer_prefill(L, x[:, :7].copy(), conv_state=cs, ssm_state=ss)]
+    for t in range(7, 10):
+        parts.append(oracle.mixer_prefill(L, x[:, t:t + 1].copy(), conv_state=cs, ssm_state=ss))
+    assert np.array_equal(np.concatenate(parts, 1), full)
+    assert np.array_equal(cs, cs0) and np.array_equal(ss, ss0)
+    xt = S.activations(1, 64, 256, seed=5, n_outliers=4, outlier_scale=50.0, outlier_seed=99)
+    ref = oracle.ref_mixer_f64(P, SMALL, xt)
+    gain = oracle.sqnr_db(ref, oracle.mixer_prefill(Ls["token"], xt)) - \
+        oracle.sqnr_db(ref, oracle.mixer_prefill(Ls["static"], xt))
+    assert gain > 0.5, gain
