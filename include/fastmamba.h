@@ -244,7 +244,9 @@ size_t fm_workspace_bytes(const fm_shape *shape, int B, int T);
  *   residual 1: out = x + mixer(x) (stack layer; out may alias x).
  *   conv_state [B, 3, conv_ch] int8 / ssm_state [B, nh, hd, ds] int32, or
  *   NULL: carried state in/out (prefill in chunks is bit-identical to one pass).
- *   ws: device workspace of at least fm_workspace_bytes(shape, B, T). */
+ *   ws: device workspace of at least fm_workspace_bytes(shape, B, T).
+ *   Launch limits, checked before any kernel: B <= 65535 and
+ *   B * T <= 65535 * 128 rows, else FM_ERR_SHAPE (fm_calibrate_layer too). */
 fm_status fm_mixer_prefill(const fm_layer *L, const float *x, int B, int T, int residual,
                            int8_t *conv_state, int32_t *ssm_state, float *out, void *ws,
                            size_t ws_bytes, fm_stream stream);

@@ -257,16 +257,16 @@ static fm_status launch_gemm_persist(const CUtensorMap &ta, const CUtensorMap &t
 
 static int sm_count() {
   constexpr int kMaxDevices = 64;
-  static int cache[kMaxDevices] = {0};
+  static std::atomic<int> cache[kMaxDevices];  // zero-initialised (static storage)
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
-  if (!cache[dev]) {
-    int n = 0;
+  int n = cache[dev].load(std::memory_order_relaxed);
+  if (!n) {
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
       n = 148;
-    cache[dev] = n;
+    cache[dev].store(n, std::memory_order_relaxed);
   }
-  return cache[dev];
+  return n;
 }
 
 // Large problems: the persistent kernel, 128 x 256 tiles when there are at
@@ -797,6 +797,17 @@ static fm_status check_layer(const fm_layer *L, Dims *d, const char *fn) {
   return FM_OK;
 }
 
+// Launch limits of the whole layer, checked before its first kernel: B is a
+// grid dimension of the conv and the scan (<= 65535); B * T rows feed the
+// GEMMs, whose row-tile count is bounded by 65535.
+static fm_status check_batch(int B, int T, const char *fn) {
+  if (B > 65535) return fail(FM_ERR_SHAPE, "%s: B=%d exceeds 65535", fn, B);
+  if ((long long)B * T > 65535LL * kGemmBM)
+    return fail(FM_ERR_SHAPE, "%s: B*T=%lld exceeds %lld rows", fn, (long long)B * T,
+                65535LL * kGemmBM);
+  return FM_OK;
+}
+
 static fm_status mixer_impl(const fm_layer *L, const Dims &d, const float *x, int B, int T,
                             int residual, int8_t *conv_state, int32_t *ssm_state, float *out,
                             const MixerWs &w, cudaStream_t s) {
@@ -827,6 +838,7 @@ extern "C" fm_status fm_mixer_prefill(const fm_layer *L, const float *x, int B, 
   FM_TRY(check_layer(L, &d, __func__));
   if (B < 0 || T < 0) return fail(FM_ERR_SHAPE, "fm_mixer_prefill: B, T must be >= 0");
   if ((long long)B * T == 0) return FM_OK;
+  FM_TRY(check_batch(B, T, __func__));
   NEED(x);
   NEED(out);
   OPT(conv_state);
@@ -1076,6 +1088,7 @@ extern "C" fm_status fm_calibrate_layer(const fm_layer *L, const float *conv_b, 
   if (exps != L->exps || conv_bq != L->conv_bq || static_amax != L->static_amax)
     return fail(FM_ERR_INVALID_ARG, "fm_calibrate_layer: table pointers must be the layer's own");
   if (B <= 0 || T <= 0) return fail(FM_ERR_SHAPE, "fm_calibrate_layer: need B, T > 0");
+  FM_TRY(check_batch(B, T, __func__));
   const size_t need = fm_calib_workspace_bytes(&L->shape, B, T);
   if (!ws || ws_bytes < need || !aligned16(ws))
     return fail(FM_ERR_WORKSPACE, "fm_calibrate_layer: workspace needs %zu bytes", need);

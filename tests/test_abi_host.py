@@ -119,6 +119,14 @@ def test_layer_validation_before_launch(so):
                                None) == 3
     # negative sizes
     assert so.fm_mixer_prefill(C.byref(L), x, -1, 4, 0, None, None, x, ws, big, None) == 2
+    # launch limits, checked before the first kernel: B is a grid dimension
+    # (<= 65535), B * T the GEMMs' rows (<= 65535 tiles of 128)
+    assert so.fm_mixer_prefill(C.byref(L), x, 70000, 1, 0, None, None, x, ws, big, None) == 2
+    assert b"65535" in so.fm_last_error()
+    assert so.fm_mixer_prefill(C.byref(L), x, 1, 65535 * 128 + 1, 0, None, None, x, ws, big,
+                               None) == 2
+    assert so.fm_decode_step_noalloc(C.byref(L), x, 70000, 0, C.c_void_p(0x3000),
+                                     C.c_void_p(0x5000), x, None) in (2, 4)
 
 
 def test_scan_and_tuning_validation(so):
