@@ -358,6 +358,8 @@ class Layer:
     amax_out: float = 0.0
     state_bits: int = 31    # state word width reading (31 as built; 16 the int16 reading)
     xbc_exponents: str = "static"   # conv output exponents: "static" per head, or "token"
+    scan_mode: str = "seq"  # "seq": the sequential fixed-point scan; "ssd": the chunked form
+    ssd_chunk: int = 64
     extra: dict = field(default_factory=dict)
 
     def e_o(self) -> np.ndarray:
@@ -417,9 +419,16 @@ def mixer_prefill(L: Layer, x, residual=False, conv_state=None, ssm_state=None, 
     acc = gemm_i8(q, L.wq_in)
     z, xbc, dt = in_proj_epilogue(acc, sx, L.sw_in, di, cc, nh, L.e_u)
     xo, e_tok = conv_out(L, xbc.reshape(Bsz, T, cc), conv_state)
-    y = ssm_scan_pot(xo, dt.reshape(Bsz, T, nh), L.dt_bias, L.A_q, L.D_q, L.e_x, L.e_B, L.e_C,
-                     L.e_h, L.e_y, L.e_D, hd, ds, ssm_state, state_bits=L.state_bits,
-                     e_tok=e_tok)
+    if L.scan_mode == "ssd":
+        from .ssd import ssd_scan
+        if e_tok is not None or L.state_bits != 31:
+            raise ValueError("the chunked scan follows static exponents and the 31-bit state")
+        y = ssd_scan(xo, dt.reshape(Bsz, T, nh), L.dt_bias, L.A_q, L.D_q, L.e_x, L.e_B, L.e_C,
+                     L.e_h, L.e_y, L.e_D, hd, ds, Q=L.ssd_chunk, state=ssm_state)
+    else:
+        y = ssm_scan_pot(xo, dt.reshape(Bsz, T, nh), L.dt_bias, L.A_q, L.D_q, L.e_x, L.e_B,
+                         L.e_C, L.e_h, L.e_y, L.e_D, hd, ds, ssm_state,
+                         state_bits=L.state_bits, e_tok=e_tok)
     q2, sx2 = gate_norm_quant(y.reshape(M, di), z, hd, L.e_y, L.e_g, L.norm_w, L.rotate, L.mode,
                               L.amax_out)
     acc2 = gemm_i8(q2, L.wq_out)

@@ -13,6 +13,7 @@ the GPU path's.  Runs on the CPU in about a quarter of an hour:
     python -m oracle.sqnr_report --baselines  # plain W8A8 / SmoothQuant / rotated
     python -m oracle.sqnr_report --state-bits # width of the SSM state word
     python -m oracle.sqnr_report --readings   # conv-output exponents x state width
+    python -m oracle.sqnr_report --ssd        # the chunked (tensor-core form) scan mode
 
 The attribution (``oracle.stages``) quantises the stages of one layer alone
 and cumulatively, in pipeline order; its first row is FastMamba-LQ, the
@@ -198,7 +199,39 @@ def print_readings_table():
         print(f"| {name}{tag} | {bits} bits | {v[0]:.2f} | {v[1]:.2f} |")
 
 
+def ssd_rows(T: int = 256):
+    """One rotated 130M-shaped layer as in ``layer_case``: the sequential
+    fixed-point scan against the chunked scan mode (bf16 operands, chunks of
+    64 and 128 tokens), calibrated the same way."""
+    shape = S.MAMBA2_130M
+    P = S.layer_params(shape, 1000)
+    xc = S.calibration_batch(shape.d_model, T, 8, 50.0, OUTLIER_SEED)
+    x = S.activations(1, T, shape.d_model, seed=1, n_outliers=8, outlier_scale=50.0,
+                      outlier_seed=OUTLIER_SEED)
+    ref = O.ref_mixer_f64(P, shape, x)
+    rows = {("seq", 0): [], ("ssd", 64): [], ("ssd", 128): []}
+    for mode in (O.DYNAMIC, O.STATIC):
+        L = O.prepare_layer(P, shape, mode=mode)
+        O.calibrate_layer(L, xc)
+        for (sm, q), v in rows.items():
+            L.scan_mode, L.ssd_chunk = sm, q or 64
+            v.append(O.sqnr_db(ref, O.mixer_prefill(L, x)))
+    return rows
+
+
+def print_ssd_table():
+    print("| scan | SQNR, dynamic (dB) | SQNR, static (dB) |")
+    print("|---|---|---|")
+    for (sm, q), v in ssd_rows().items():
+        name = "sequential fixed point (as built)" if sm == "seq" else \
+            f"chunked, {q}-token chunks, bf16 operands"
+        print(f"| {name} | {v[0]:.2f} | {v[1]:.2f} |")
+
+
 def main():
+    if "--ssd" in sys.argv[1:]:
+        print_ssd_table()
+        return
     if "--readings" in sys.argv[1:]:
         print_readings_table()
         return
@@ -235,6 +268,8 @@ def main():
     print_state_bits_table()
     print()
     print_readings_table()
+    print()
+    print_ssd_table()
 
 
 if __name__ == "__main__":
