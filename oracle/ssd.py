@@ -22,11 +22,12 @@ chunks of Q tokens from the first token of the call; inside chunk c
   dtf[s]   = dt_q[s] 2^-16                          (exact in fp32)
   intra:  G = Cq Bq^T (exact integer), for s <= t
           M[t, s] = op(fl32(G[t, s] * fl32(a(s, t) dtf[s])))
-          Yi[t, p] = fl32(sum_s M[t, s] X[s, p])
-  inter:  Yo[t, p] = fl32(a0(t) * fl32(sum_n Cq[t, n] op(H[p, n])))
+  inter:  Ca[t, n] = op(fl32(a0(t) Cq[t, n]))
+  both in one sum (one accumulator on the tensor cores):
+          Y[t, p] = fl32(sum_s M[t, s] X[s, p] + sum_n Ca[t, n] op(H[p, n]))
   state:  K[s] = fl32(a(s, end) dtf[s]);  U[s, n] = op(fl32(K[s] Bq[s, n]))
           H <- fl32(fl32(a0(end) H) + fl32(sum_s X[s, p] U[s, n]))
-  output: y[t, p] = sat32(rint(fl32(Yi + Yo) 2^(e_C+e_x+e_B-e_y)) + rshr(D_q X[t, p], s_D))
+  output: y[t, p] = sat32(rint(Y[t, p] 2^(e_C+e_x+e_B-e_y)) + rshr(D_q X[t, p], s_D))
 H is the state in code units (2^(e_x+e_B)); it enters from and leaves to the
 sequential scan's int32 word at e_h: H = h 2^(e_h-e_x-e_B), h =
 sat31(rint(H 2^(e_x+e_B-e_h))), so a chunked prefill hands over to the
@@ -114,12 +115,12 @@ def ssd_scan(xbc, dt_raw, dt_bias, A_q, D_q, e_x, e_B, e_C, e_h, e_y, e_D, hd, d
                 a = np.where(low, _pow2(np.where(low, diff, 0)), F32(0))
                 ad = (a * dtf[None, t0:t1]).astype(F32)           # fl32(a(s,t) dtf[s])
                 M = _op((G.astype(F32) * ad).astype(F32), operand)
-                Yi = (M.astype(np.float64) @ X[t0:t1]).astype(F32)
-                # inter-chunk, from the state entering the chunk
+                # inter-chunk, from the state entering the chunk: the decay
+                # from the chunk's start scales C before the operand rounding
                 a0 = _pow2(W)
-                Z = (Cq[t0:t1] @ _op(H, operand).astype(np.float64).T).astype(F32)
-                Yo = (a0[:, None] * Z).astype(F32)
-                yf = (Yi + Yo).astype(F32)
+                Ca = _op((a0[:, None] * Cq[t0:t1].astype(F32)).astype(F32), operand)
+                yf = (M.astype(np.float64) @ X[t0:t1] +
+                      Ca.astype(np.float64) @ _op(H, operand).astype(np.float64).T).astype(F32)
                 # state leaving the chunk
                 K = (_pow2(W[-1] - W) * dtf[t0:t1]).astype(F32)
                 U = _op((K[:, None] * Bq[t0:t1].astype(F32)).astype(F32), operand)

@@ -70,9 +70,10 @@ def test_exact_operands_equal_the_recurrence(oracle, SSD, Q):
 
 
 def test_bf16_operands_within_budget(oracle, SSD):
-    """bf16 rounding of M, U and the carried state: each rounded operand is
-    off by at most 2^-9 of itself, so the output error stays below
-    3 * 2^-9 of the sum of |terms| (three rounded operand kinds)."""
+    """bf16 rounding of M, U, the decayed C and the carried state: each
+    rounded operand is off by at most 2^-9 of itself, so the output error
+    stays below 3 * 2^-9 of the sum of |terms| (a product of two rounded
+    operands is off by at most 2 * 2^-9 + 2^-18; the state adds its own)."""
     xbc, dt_raw, dt_bias, A_q = _inputs(T=48)
     hd, ds = 8, 16
     _, yb = SSD.ssd_scan(xbc, dt_raw, dt_bias, A_q, hd=hd, ds=ds, Q=16, operand="bf16",
