@@ -419,7 +419,7 @@ def mixer_prefill(L: Layer, x, residual=False, conv_state=None, ssm_state=None, 
     acc = gemm_i8(q, L.wq_in)
     z, xbc, dt = in_proj_epilogue(acc, sx, L.sw_in, di, cc, nh, L.e_u)
     xo, e_tok = conv_out(L, xbc.reshape(Bsz, T, cc), conv_state)
-    if L.scan_mode == "ssd":
+    if L.scan_mode == "ssd" and T > 1:   # single steps stay sequential
         from .ssd import ssd_scan
         if e_tok is not None or L.state_bits != 31:
             raise ValueError("the chunked scan follows static exponents and the 31-bit state")

@@ -28,6 +28,8 @@ chunks of Q tokens from the first token of the call; inside chunk c
   state:  K[s] = fl32(a(s, end) dtf[s]);  U[s, n] = op(fl32(K[s] Bq[s, n]))
           H <- fl32(fl32(a0(end) H) + fl32(sum_s X[s, p] U[s, n]))
   output: y[t, p] = sat32(rint(Y[t, p] 2^(e_C+e_x+e_B-e_y)) + rshr(D_q X[t, p], s_D))
+A layer in this mode (``scan_mode = "ssd"``) runs it for calls of more than
+one token; single decode steps stay sequential.
 H is the state in code units (2^(e_x+e_B)); it enters from and leaves to the
 sequential scan's int32 word at e_h: H = h 2^(e_h-e_x-e_B), h =
 sat31(rint(H 2^(e_x+e_B-e_h))), so a chunked prefill hands over to the
