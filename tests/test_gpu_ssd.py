@@ -79,9 +79,17 @@ def _check_codes(got, ref, mag):
 def test_ssd_scan_matches_its_oracle(L, SSD, shape, B, T, with_state):
     s = MAMBA130 if shape == "130m" else S.MAMBA2_2P7B
     xbc, dt_raw, dt_bias, A_q, D_q, e_D, e_x, e_B, e_C, e_h, e_y = _case(s, B, T, 200 + T)
-    exps = _exps(L, s, e_x, e_B, e_C, e_h, e_y, e_D)
     st = S.uniform_ints((B, s.nheads, s.headdim, s.d_state), -2 ** 26, 2 ** 26,
                         seed=7) if with_state else None
+    # output exponents that keep the y codes below 2^29 (random codes would
+    # otherwise saturate them and make the comparison vacuous)
+    _, yf0 = SSD.ssd_scan(xbc, dt_raw, dt_bias, A_q, D_q, e_x, e_B, e_C, e_h, e_y, e_D,
+                          s.headdim, s.d_state, Q=128,
+                          state=None if st is None else st.copy(), want_f32=True)
+    top = np.abs(yf0.astype(np.float64)).reshape(-1, s.nheads, s.headdim).max(axis=(0, 2))
+    e_y = (e_C + e_x + e_B + np.ceil(np.log2(np.maximum(top, 1.0))) - 29).astype(np.int32)
+    e_y = np.maximum(e_y, e_D + e_x - 16).astype(np.int32)      # skip term stays in range
+    exps = _exps(L, s, e_x, e_B, e_C, e_h, e_y, e_D)
     y = torch.empty((B, T, s.d_inner), dtype=torch.int32, device="cuda")
     st_d = dev(st) if with_state else None
     ws = torch.empty(L.ssd_workspace_bytes(s, B, T), dtype=torch.uint8, device="cuda")
@@ -97,6 +105,7 @@ def test_ssd_scan_matches_its_oracle(L, SSD, shape, B, T, with_state):
                           state=st_a, operand="fp32", want_f32=True)
     s_y = (e_C + np.repeat(e_x, s.headdim) + e_B - np.repeat(e_y, s.headdim)).astype(np.float64)
     mag = np.abs(mag.astype(np.float64)) * np.exp2(s_y)
+    assert np.abs(yr).max() < 2 ** 30                             # not saturated
     _check_codes(host(y), yr, mag)
     if with_state:
         # the state word: same bar, |terms| the absolute-code state
