@@ -272,11 +272,14 @@ __global__ void __launch_bounds__(256) k_ssd_pass(SsdArgs a) {
 }
 
 // ------------------------------------------------------------ chunk output
+// M reuses the int8 C / B tiles: it is written only after the MMA that reads
+// them has completed (the wait on bar[0]), which keeps the CTA at 109 KB (two
+// per SM).
 struct SsdOutSmem {
   static constexpr int kC8 = 0;                        // [128 t x 128 B] int8 (A of G)
   static constexpr int kB8 = kC8 + kSsdQ * 128;        // [128 s x 128 B] int8 (B of G)
-  static constexpr int kM = kB8 + kSsdQ * 128;         // [128 t x 256 B] bf16
-  static constexpr int kCa = kM + kSsdQ * 256;         // [128 t x 256 B] bf16
+  static constexpr int kM = kC8;                       // [128 t x 256 B] bf16, over C8 + B8
+  static constexpr int kCa = kB8 + kSsdQ * 128;        // [128 t x 256 B] bf16
   static constexpr int kX = kCa + kSsdQ * 256;         // [64 p x 256 B] bf16
   static constexpr int kH = kX + kSsdHd * 256;         // [64 p x 256 B] bf16
   static constexpr int kXt = kH + kSsdHd * 256;        // [128 s][64 p] int8
@@ -287,6 +290,7 @@ struct SsdOutSmem {
   static constexpr int kSlot = kBar + 16;
   static constexpr int kBytes = kSlot + 16 + 1024;
 };
+static_assert(SsdOutSmem::kBytes <= 113 * 1024, "two k_ssd_out CTAs per SM");
 
 // grid (nch, nh, B), 128 threads
 __global__ void __launch_bounds__(kSsdThreads) k_ssd_out(SsdArgs a) {
