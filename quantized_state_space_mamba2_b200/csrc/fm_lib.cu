@@ -769,7 +769,7 @@ static fm_status launch_ssd(const Dims &d, const int8_t *xbc, const float *dt_ra
                                      SsdOutSmem::kBytes));
   k_ssd_state<<<grid, kSsdThreads, SsdStateSmem::kBytes, s>>>(a);
   FM_TRY(launched("k_ssd_state"));
-  k_ssd_pass<<<dim3((unsigned)d.nh, (unsigned)B), 256, 0, s>>>(a);
+  k_ssd_pass<<<dim3(kSsdHd * kSsdDs / 256, (unsigned)d.nh, (unsigned)B), 256, 0, s>>>(a);
   FM_TRY(launched("k_ssd_pass"));
   k_ssd_out<<<grid, kSsdThreads, SsdOutSmem::kBytes, s>>>(a);
   return launched("k_ssd_out");

@@ -13,8 +13,8 @@
 //   state   dH[p, n] = sum_s X[s, p] bf16(2^(W[end] - W[s]) dt[s] Bq[s, n])
 //           H_next = 2^W[end] H + dH
 // Three kernels: k_ssd_state (per chunk: dH and the chunk's decay),
-// k_ssd_pass (per head, sequential over chunks: the state entering each
-// chunk), k_ssd_out (per chunk: Y and the int32 y codes).  Operand tiles are
+// k_ssd_pass (one thread per state cell, sequential over chunks: the state
+// entering each chunk), k_ssd_out (per chunk: Y and the int32 y codes).  Operand tiles are
 // written by the threads into 128-byte-swizzled K-major shared memory (rows
 // of 128 bytes, 8-row groups 1024 bytes apart, 16-byte pieces XOR-ed with
 // the row's index within its group), the layout sw128_desc() describes; one
@@ -237,37 +237,42 @@ __global__ void __launch_bounds__(kSsdThreads) k_ssd_state(SsdArgs a) {
 }
 
 // ------------------------------------------------------------ state passing
-// grid (nh, B), 256 threads; 32 state cells per thread, sequential over chunks
+// grid (64 * 128 / 256, nh, B), 256 threads: one state cell per thread,
+// sequential over the chunks; each group of 8 chunks' decays and dH are loaded
+// before the recurrence consumes them, so the loads overlap.
+constexpr int kSsdPassGroup = 8;
 __global__ void __launch_bounds__(256) k_ssd_pass(SsdArgs a) {
-  const int h = blockIdx.x, b = blockIdx.y;
+  constexpr int kCells = kSsdHd * kSsdDs;
+  const int e = blockIdx.x * 256 + threadIdx.x;  // cell p * 128 + n
+  const int h = blockIdx.y, b = blockIdx.z;
   const long long bh = (long long)b * a.nh + h;
   const int u_sh = a.e_h[h] - a.e_x[h] - *a.e_B;  // state word -> code units
-  constexpr int kCells = kSsdHd * kSsdDs;
-  float H[32];
-#pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    const int e = threadIdx.x + 256 * i;
-    H[i] = a.state ? __fmul_rn(__int2float_rn(a.state[bh * kCells + e]), pow2f(u_sh)) : 0.0f;
-  }
+  float H = a.state ? __fmul_rn(__int2float_rn(a.state[bh * kCells + e]), pow2f(u_sh)) : 0.0f;
+  const float *__restrict__ dH = a.dH + bh * a.nch * kCells + e;
+  const float *__restrict__ ach = a.achunk + bh * a.nch;
+  uint16_t *__restrict__ Hin = a.Hin + bh * a.nch * kCells + e;
 #pragma unroll 1
-  for (int c = 0; c < a.nch; ++c) {
-    const float ac = a.achunk[bh * a.nch + c];
-    const long long base = (bh * a.nch + c) * kCells;
+  for (int c0 = 0; c0 < a.nch; c0 += kSsdPassGroup) {
+    float d[kSsdPassGroup], ac[kSsdPassGroup];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      const int e = threadIdx.x + 256 * i;
-      a.Hin[base + e] = (uint16_t)bf16_bits(H[i]);
-      H[i] = __fadd_rn(__fmul_rn(ac, H[i]), a.dH[base + e]);
+    for (int k = 0; k < kSsdPassGroup; ++k) {
+      const int c = c0 + k;
+      d[k] = c < a.nch ? dH[(long long)c * kCells] : 0.0f;
+      ac[k] = c < a.nch ? ach[c] : 1.0f;
+    }
+#pragma unroll
+    for (int k = 0; k < kSsdPassGroup; ++k) {
+      const int c = c0 + k;
+      if (c < a.nch) {
+        Hin[(long long)c * kCells] = (uint16_t)bf16_bits(H);
+        H = __fadd_rn(__fmul_rn(ac[k], H), d[k]);
+      }
     }
   }
   if (a.state) {
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      const int e = threadIdx.x + 256 * i;
-      float v = rintf(__fmul_rn(H[i], pow2f(-u_sh)));
-      v = fminf(fmaxf(v, -1073741823.0f), 1073741823.0f);
-      a.state[bh * kCells + e] = (int32_t)v;
-    }
+    float v = rintf(__fmul_rn(H, pow2f(-u_sh)));
+    v = fminf(fmaxf(v, -1073741823.0f), 1073741823.0f);
+    a.state[bh * kCells + e] = (int32_t)v;
   }
 }
 
