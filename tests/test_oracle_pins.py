@@ -240,6 +240,14 @@ def test_conv_matches_library_convolution(oracle):
     assert np.all(np.abs(got - np.clip(ref, -127 / 16, 127 / 16)) <= 2.0 ** -5 + 2e-3 * np.abs(ref) + 1e-3)
     assert np.array_equal(st, u[:, -3:])                 # new state = last three inputs
     assert np.all(am > 0)
+    # the Q.16 SiLU values before requantisation (per-token exponent reading):
+    # the SiLU of the real-valued accumulation within the PWL SiLU's bound
+    _, s16 = oracle.conv1d_pot(u, wq, bq, e_u, e_w, e_o, conv_state=state.copy(), want_s16=True)
+    sv = s16 / 65536.0
+    rel = _chord_rel_bound() + 1.2e-4 * (np.abs(real) + 1.0)
+    bound = np.abs(real) * (rel * np.exp(-np.abs(real)) + 2.0 / 65536) + 2.0 / 65536
+    assert np.all(np.abs(sv - ref) <= bound)
+    assert np.abs(ref).max() > 4.0                       # spans the nonlinear range
 
 
 def test_conv_state_chunking_bit_exact(oracle):
