@@ -53,6 +53,7 @@ L2_FLUSH_BYTES = 512 << 20
 # Algorithmic work of one state-cell update of the scan: decay multiply,
 # rounding shift, dt*x*B multiply-add, clamp (2), C*h multiply-accumulate.
 SCAN_OPS_PER_CELL = 6
+SSD_CHUNK = 128  # tokens per chunk of the chunked scan mode
 NOMINAL_INT8_OVER_BF16 = 2.0  # 4.5 / 2.25 PFLOP/s dense
 CPU_SAMPLE_MIN_S = 10.0
 
@@ -69,6 +70,9 @@ def parse(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--scan-tile", default=None,
                     help="npt,pc,tch of the sequential scan kernel (a compiled variant)")
+    ap.add_argument("--scan-mode", default="seq", choices=["seq", "ssd"],
+                    help="seq: the sequential fixed-point scan (the method); ssd: the chunked "
+                         "tensor-core scan mode (its own error budget)")
     ap.add_argument("--layers", type=int, default=None,
                     help="profiling only: run the first N layers of a stack workload")
     return ap.parse_args(argv)
@@ -109,7 +113,7 @@ def config_block(args) -> dict:
                  calibration=f"{S.CALIB_SEQS} seeded sequences x "
                              f"{min(w.get('prefill_len', w['seqlen']), S.CALIB_MAX_LEN)} tokens "
                              "(GPU, stage by stage)",
-                 scan_tile=args.scan_tile or "4,4,16")
+                 scan_tile=args.scan_tile or "4,4,16", scan_mode=args.scan_mode)
         if "prefill_len" in w:
             c.update(prefill_len=w["prefill_len"], step="one decode token per sequence")
     return c
@@ -309,11 +313,13 @@ class StackWorkload:
         self.r = torch.empty_like(self.x0)
         M = self.B * self.T
         self.ws = self.layers[0].workspace(self.B, self.T)
-        self.sws = torch.empty(lib.scan_workspace_bytes(d, self.B, self.T), dtype=torch.uint8,
-                               device=dev)
+        self.ssd = getattr(args, "scan_mode", "seq") == "ssd" and self.T > 1
+        nb = (lib.ssd_workspace_bytes if self.ssd else lib.scan_workspace_bytes)(d, self.B, self.T)
+        self.sws = torch.empty(nb, dtype=torch.uint8, device=dev)
         self.buf = _stage_buffers(torch, d, M, dev)
         self.tokens = M
-        self.launches = self.launches_per_layer * self.n_layers
+        # the chunked scan is three kernels where the sequential one is two
+        self.launches = (self.launches_per_layer + (1 if self.ssd else 0)) * self.n_layers
 
     def states(self, i):
         return None, None
@@ -331,8 +337,9 @@ class StackWorkload:
             lib.conv1d_pot(b["xbc"], B, T, d, Ly.conv_wq, Ly.conv_bq, Ly.exps, cs, b["xo"])
             if ev is not None:
                 ev[i][0].record(stream)
-            lib.ssm_scan_pot(b["xo"], b["dtr"], B, T, d, Ly.dt_bias, Ly.A_q, Ly.D_q, Ly.exps, ss,
-                             b["y"], self.sws)
+            scan = lib.ssd_scan if self.ssd else lib.ssm_scan_pot
+            scan(b["xo"], b["dtr"], B, T, d, Ly.dt_bias, Ly.A_q, Ly.D_q, Ly.exps, ss, b["y"],
+                 self.sws)
             if ev is not None:
                 ev[i][1].record(stream)
             lib.gate_norm_quant(b["y"], b["z"], d, Ly.exps, Ly.norm_w, 1, self.mode,
@@ -374,6 +381,17 @@ class StackWorkload:
 
     def roofline(self, dom_ms, peaks):
         d = self.shape
+        if self.ssd:
+            # per token and head: C.B^T Q ds, M.X Q hd, state hd ds, inter ds hd MACs
+            macs = self.B * self.T * d.nheads * (SSD_CHUNK * d.d_state + SSD_CHUNK * d.headdim +
+                                                 2 * d.headdim * d.d_state)
+            achieved = 2 * macs / (dom_ms / 1e3) / 1e12
+            peak = (peaks or {}).get("bf16_tflops", 1590.0)
+            return {"bound": "tensor", "kernel": "fm_ssd_scan (k_ssd_state + k_ssd_pass + k_ssd_out)",
+                    "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                    "traffic": None,
+                    "peak_basis": "measured bf16 dense (burst); the C.B^T quarter runs as int8",
+                    "algorithmic": f"2 x {macs} MACs per launch"}
         cells = self.B * d.nheads * d.headdim * d.d_state * self.T
         achieved = cells * SCAN_OPS_PER_CELL / (dom_ms / 1e3) / 1e12
         mhz = (peaks or {}).get("sm_max_mhz", 1965.0)
@@ -584,6 +602,7 @@ def main():
     lib.load()
     if args.scan_tile:
         lib.set_scan_tile(*[int(v) for v in args.scan_tile.split(",")])
+    lib.set_scan_mode(args.scan_mode)
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream(dev)

@@ -237,6 +237,26 @@ typedef struct fm_layer {
     const float *static_amax;   /* [2]: in_proj input, out_proj input (FM_STATIC) */
 } fm_layer;
 
+/* Chunked (state-space-dual) scan mode: the same inputs and outputs as
+ * fm_ssm_scan_pot, computed chunk by chunk (128 tokens) on the tensor cores as
+ * in Mamba2's own algorithm (reference [2] of the FastMamba paper): exact
+ * int8 C.B^T, bf16 operands elsewhere, fp32 sums, decays 2^(running sum of the
+ * step's log2 decay) per chunk.  Not bit-identical to the sequential scan; its
+ * error budget is that of bf16 operands (relative 2^-9 per rounded operand).
+ * state (nullable): int32 at e_h in and out, interchangeable with the
+ * sequential scan's.  ws: device workspace of fm_ssd_workspace_bytes. */
+size_t fm_ssd_workspace_bytes(const fm_shape *shape, int B, int T);
+/* Process-wide scan mode of the layer entry points (fm_mixer_prefill and
+ * what calls it): 0 = the sequential fixed-point scan (default, the method),
+ * 1 = the chunked mode above for calls of more than one token.  The mode in
+ * force when fm_workspace_bytes is asked must also be in force for the call.
+ * FM_ERR_INVALID_ARG for any other value. */
+fm_status fm_set_scan_mode(int mode);
+fm_status fm_ssd_scan(const int8_t *xbc, const float *dt_raw, int B, int T,
+                      const fm_shape *shape, const float *dt_bias, const int32_t *A_q,
+                      const int32_t *D_q, const int32_t *exps, int32_t *state, int32_t *y,
+                      void *ws, size_t ws_bytes, fm_stream stream);
+
 /* Workspace bytes fm_mixer_prefill / fm_decode_step need for B*T tokens. */
 size_t fm_workspace_bytes(const fm_shape *shape, int B, int T);
 

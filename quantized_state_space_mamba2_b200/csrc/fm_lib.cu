@@ -24,6 +24,7 @@
 #include "k_rows.cuh"
 #include "k_scan.cuh"
 #include "k_scan2.cuh"
+#include "k_ssd.cuh"
 
 using namespace fm;
 
@@ -384,6 +385,16 @@ struct ScanTile {
 static const ScanTile kScanTiles[] = {{4, 4, 16}, {4, 2, 16}, {4, 8, 16},
                                       {8, 4, 16}, {8, 2, 16}, {8, 8, 16}};
 static std::atomic<int> g_scan_tile{0};
+// 0: the sequential fixed-point scan (the method); 1: the chunked scan mode for
+// prefills of more than one token (single steps stay sequential)
+static std::atomic<int> g_scan_mode{0};
+
+extern "C" fm_status fm_set_scan_mode(int mode) {
+  if (mode != 0 && mode != 1) return fail(FM_ERR_INVALID_ARG, "fm_set_scan_mode: bad mode %d", mode);
+  g_scan_mode.store(mode, std::memory_order_relaxed);
+  return FM_OK;
+}
+static bool use_ssd(int T) { return T > 1 && g_scan_mode.load(std::memory_order_relaxed) == 1; }
 static ScanTile scan_tile() { return kScanTiles[g_scan_tile.load(std::memory_order_relaxed)]; }
 
 extern "C" fm_status fm_set_scan_tile(int npt, int pc, int tch) {
@@ -668,6 +679,102 @@ extern "C" fm_status fm_ssm_scan_pot(const int8_t *xbc, const float *dt_raw, int
                         B, w, (cudaStream_t)stream);
 }
 
+// ------------------------------------------------------------------ chunked scan mode
+namespace {
+struct SsdWs {
+  float *dH;
+  float *achunk;
+  uint16_t *Hin;
+};
+SsdWs carve_ssd(Carver &c, const Dims &d, int B, int T) {
+  const long long nch = (T + kSsdQ - 1) / kSsdQ, units = (long long)B * d.nh * nch;
+  SsdWs w;
+  w.dH = c.take<float>(units * kSsdHd * kSsdDs);
+  w.achunk = c.take<float>(units);
+  w.Hin = c.take<uint16_t>(units * kSsdHd * kSsdDs);
+  return w;
+}
+}  // namespace
+
+extern "C" size_t fm_ssd_workspace_bytes(const fm_shape *shape, int B, int T) {
+  Dims d;
+  if (check_shape(shape, &d, __func__) != FM_OK || B < 0 || T < 0) return 0;
+  Carver c{nullptr, 0};
+  carve_ssd(c, d, B, T);
+  return c.off + 256;
+}
+
+static fm_status launch_ssd(const Dims &d, const int8_t *xbc, const float *dt_raw, int B, int T,
+                            const float *dt_bias, const int32_t *A_q, const int32_t *D_q,
+                            const int32_t *exps, const fm_exp_layout &X, int32_t *state,
+                            int32_t *y, const SsdWs &w, cudaStream_t s);
+
+extern "C" fm_status fm_ssd_scan(const int8_t *xbc, const float *dt_raw, int B, int T,
+                                 const fm_shape *shape, const float *dt_bias, const int32_t *A_q,
+                                 const int32_t *D_q, const int32_t *exps, int32_t *state,
+                                 int32_t *y, void *ws, size_t ws_bytes, fm_stream stream) {
+  Dims d;
+  FM_TRY(check_shape(shape, &d, __func__));
+  if (B < 0 || T < 0) return fail(FM_ERR_SHAPE, "fm_ssd_scan: B, T must be >= 0");
+  if ((long long)B * T == 0) return FM_OK;
+  if (B > 65535) return fail(FM_ERR_SHAPE, "fm_ssd_scan: B=%d exceeds 65535", B);
+  NEED(xbc);
+  NEED(dt_raw);
+  NEED(dt_bias);
+  NEED(A_q);
+  NEED(D_q);
+  NEED(exps);
+  NEED(y);
+  OPT(state);
+  if (d.cc % 16) return fail(FM_ERR_ALIGNMENT, "fm_ssd_scan: conv channels must be a multiple of 16");
+  const size_t need = fm_ssd_workspace_bytes(shape, B, T);
+  if (!ws || ws_bytes < need || !aligned16(ws))
+    return fail(FM_ERR_WORKSPACE, "fm_ssd_scan: workspace needs %zu bytes", need);
+  Carver c{reinterpret_cast<uint8_t *>(ws), 0};
+  const SsdWs w = carve_ssd(c, d, B, T);
+  return launch_ssd(d, xbc, dt_raw, B, T, dt_bias, A_q, D_q, exps, fm_exp_table_layout(shape),
+                    state, y, w, (cudaStream_t)stream);
+}
+
+static fm_status launch_ssd(const Dims &d, const int8_t *xbc, const float *dt_raw, int B, int T,
+                            const float *dt_bias, const int32_t *A_q, const int32_t *D_q,
+                            const int32_t *exps, const fm_exp_layout &X, int32_t *state,
+                            int32_t *y, const SsdWs &w, cudaStream_t s) {
+  SsdArgs a;
+  a.xbc = xbc;
+  a.dt_raw = dt_raw;
+  a.T = T;
+  a.nh = d.nh;
+  a.cc = d.cc;
+  a.di = d.di;
+  a.nch = (T + kSsdQ - 1) / kSsdQ;
+  a.dt_bias = dt_bias;
+  a.A_q = A_q;
+  a.D_q = D_q;
+  a.e_x = exps + X.e_x;
+  a.e_B = exps + X.e_B;
+  a.e_C = exps + X.e_C;
+  a.e_h = exps + X.e_h;
+  a.e_y = exps + X.e_y;
+  a.e_D = exps + X.e_D;
+  a.state = state;
+  a.y = y;
+  a.dH = w.dH;
+  a.achunk = w.achunk;
+  a.Hin = w.Hin;
+  const dim3 grid((unsigned)a.nch, (unsigned)d.nh, (unsigned)B);
+  FM_CHECK_CUDA(cudaFuncSetAttribute(k_ssd_state, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     SsdStateSmem::kBytes));
+  FM_CHECK_CUDA(cudaFuncSetAttribute(k_ssd_out, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     SsdOutSmem::kBytes));
+  k_ssd_state<<<grid, kSsdThreads, SsdStateSmem::kBytes, s>>>(a);
+  FM_TRY(launched("k_ssd_state"));
+  k_ssd_pass<<<dim3(kSsdHd * kSsdDs / 256, (unsigned)d.nh, (unsigned)B), 256, 0, s>>>(a);
+  FM_TRY(launched("k_ssd_pass"));
+  k_ssd_out<<<grid, kSsdThreads, SsdOutSmem::kBytes, s>>>(a);
+  return launched("k_ssd_out");
+}
+
 static fm_status gate_impl(const int32_t *y, const float *z, long long M, const Dims &d,
                            const int32_t *exps, const fm_exp_layout &X, const float *norm_w,
                            int rotate, int mode, const float *static_amax, int8_t *q, float *s_x,
@@ -752,6 +859,7 @@ struct MixerWs {
   int8_t *q_out;
   float *sx_out;
   ScanWs scan;
+  SsdWs ssd;  // chunked scan mode only (null otherwise)
 };
 
 MixerWs carve_mixer(Carver &c, const Dims &d, int B, int T) {
@@ -767,6 +875,12 @@ MixerWs carve_mixer(Carver &c, const Dims &d, int B, int T) {
   w.q_out = c.take<int8_t>(M * d.di);
   w.sx_out = c.take<float>(M);
   w.scan = carve_scan(c, d, B, T);
+  if (use_ssd(T)) {
+    w.ssd = carve_ssd(c, d, B, T);
+  } else {
+    w.ssd.dH = w.ssd.achunk = nullptr;
+    w.ssd.Hin = nullptr;
+  }
   return w;
 }
 }  // namespace
@@ -820,9 +934,13 @@ static fm_status mixer_impl(const fm_layer *L, const Dims &d, const float *x, in
                       w.dt, s));
   FM_TRY(launch_conv(w.xbc, B, T, d.cc, L->conv_wq, L->conv_bq, L->exps, conv_state, w.xo,
                      nullptr, s));
-  FM_TRY(launch_scan_v2(scan_args(d, w.xo, w.dt, T, L->dt_bias, L->A_q, L->D_q, L->exps, X,
-                                  ssm_state, w.y, nullptr),
-                        B, w.scan, s));
+  if (w.ssd.dH)
+    FM_TRY(launch_ssd(d, w.xo, w.dt, B, T, L->dt_bias, L->A_q, L->D_q, L->exps, X, ssm_state, w.y,
+                      w.ssd, s));
+  else
+    FM_TRY(launch_scan_v2(scan_args(d, w.xo, w.dt, T, L->dt_bias, L->A_q, L->D_q, L->exps, X,
+                                    ssm_state, w.y, nullptr),
+                          B, w.scan, s));
   FM_TRY(gate_impl(w.y, w.z, M, d, L->exps, X, L->norm_w, L->rotate, L->mode, amax_out, w.q_out,
                    w.sx_out, nullptr, nullptr, nullptr, s));
   return launch_gemm(w.q_out, M, L->w_out_q, d.dm, d.di,

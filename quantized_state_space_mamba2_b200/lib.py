@@ -27,7 +27,7 @@ EXPORTS = (
     "fm_ssm_scan_pot", "fm_gate_norm_quant", "fm_eval_pwl", "fm_workspace_bytes",
     "fm_mixer_prefill", "fm_decode_step", "fm_prepare_mixer_params", "fm_calib_workspace_bytes",
     "fm_calibrate_layer", "fm_decode_step_noalloc", "fm_scan_workspace_bytes",
-    "fm_set_scan_tile",
+    "fm_set_scan_tile", "fm_ssd_workspace_bytes", "fm_ssd_scan", "fm_set_scan_mode",
 )
 NOALLOC_SCRATCH_BYTES = 16 << 20  # FM_NOALLOC_SCRATCH_BYTES
 
@@ -86,6 +86,9 @@ def load():
         "fm_conv1d_pot": (I, [_P, I, I, sp, _P, _P, _P, _P, _P, _P]),
         "fm_ssm_scan_pot": (I, [_P, _P, I, I, sp, _P, _P, _P, _P, _P, _P, _P, SZ, _P]),
         "fm_scan_workspace_bytes": (SZ, [sp, I, I]),
+        "fm_ssd_scan": (I, [_P, _P, I, I, sp, _P, _P, _P, _P, _P, _P, _P, SZ, _P]),
+        "fm_ssd_workspace_bytes": (SZ, [sp, I, I]),
+        "fm_set_scan_mode": (I, [I]),
         "fm_set_scan_tile": (I, [I, I, I]),
         "fm_gate_norm_quant": (I, [_P, _P, I64, sp, _P, _P, I, I, _P, _P, _P, _P, _P]),
         "fm_eval_pwl": (I, [I, _P, I64, _P, _P]),
@@ -184,6 +187,26 @@ def ssm_scan_pot(xbc, dt_raw, B, T, shape, dt_bias, A_q, D_q, exps, state, y, ws
     _check(load().fm_ssm_scan_pot(_p(xbc), _p(dt_raw), B, T, C.byref(sh), _p(dt_bias), _p(A_q),
                                   _p(D_q), _p(exps), _p(state), _p(y), _p(ws),
                                   ws.numel() * ws.element_size(), _s(stream)))
+
+
+SCAN_MODES = {"seq": 0, "ssd": 1}
+
+
+def set_scan_mode(mode: str):
+    """'seq' (the sequential fixed-point scan, default) or 'ssd' (the chunked
+    tensor-core mode for prefills of more than one token)."""
+    _check(load().fm_set_scan_mode(SCAN_MODES[mode]))
+
+
+def ssd_workspace_bytes(shape, B, T) -> int:
+    return load().fm_ssd_workspace_bytes(C.byref(shape_struct(shape)), B, T)
+
+
+def ssd_scan(xbc, dt_raw, B, T, shape, dt_bias, A_q, D_q, exps, state, y, ws, stream=None):
+    sh = shape_struct(shape)
+    _check(load().fm_ssd_scan(_p(xbc), _p(dt_raw), B, T, C.byref(sh), _p(dt_bias), _p(A_q),
+                              _p(D_q), _p(exps), _p(state), _p(y), _p(ws),
+                              ws.numel() * ws.element_size(), _s(stream)))
 
 
 def gate_norm_quant(y, z, shape, exps, norm_w, rotate, mode, static_amax, q, s_x, amax_row=None,

@@ -150,3 +150,30 @@ def test_scan_and_tuning_validation(so):
     # gate: bad mode
     assert so.fm_gate_norm_quant(f[0], f[1], 4, C.byref(sh), f[2], f[3], 1, 5, None, f[4], f[5],
                                  None, None) == 1
+
+
+def test_chunked_scan_validation(so):
+    """The chunked scan mode's entry points reject bad arguments before any
+    launch; its workspace covers the chunk states (fp32 + bf16) and decays."""
+    from quantized_state_space_mamba2_b200 import lib
+    from quantized_state_space_mamba2_b200 import synth as S
+    sh = lib.shape_struct(S.MAMBA2_130M)
+    s = S.MAMBA2_130M
+    nch = (300 + 127) // 128
+    need = lib.ssd_workspace_bytes(s, 2, 300)
+    units = 2 * s.nheads * nch
+    assert need >= units * 64 * 128 * (4 + 2) + units * 4
+    assert lib.ssd_workspace_bytes(s, 0, 0) <= 1024
+    p = C.c_void_p(0x7000000)
+    # empty problem: nothing to do
+    assert so.fm_ssd_scan(None, None, 0, 7, C.byref(sh), None, None, None, None, None, None, None,
+                          0, None) == 0
+    # null / misaligned / workspace
+    assert so.fm_ssd_scan(None, p, 1, 7, C.byref(sh), p, p, p, p, None, p, p, 1 << 40, None) == 1
+    assert so.fm_ssd_scan(p, p, 1, 7, C.byref(sh), p, p, p, p, C.c_void_p(0x3001), p, p, 1 << 40,
+                          None) == 3
+    assert so.fm_ssd_scan(p, p, 1, 7, C.byref(sh), p, p, p, p, None, p, p, 16, None) == 4
+    assert so.fm_ssd_scan(p, p, 70000, 7, C.byref(sh), p, p, p, p, None, p, p, 1 << 40, None) == 2
+    # scan mode switch
+    assert so.fm_set_scan_mode(2) == 1
+    assert so.fm_set_scan_mode(0) == 0
