@@ -27,7 +27,7 @@ EXPORTS = (
     "fm_ssm_scan_pot", "fm_gate_norm_quant", "fm_eval_pwl", "fm_workspace_bytes",
     "fm_mixer_prefill", "fm_decode_step", "fm_prepare_mixer_params", "fm_calib_workspace_bytes",
     "fm_calibrate_layer", "fm_decode_step_noalloc", "fm_scan_workspace_bytes",
-    "fm_set_scan_tile",
+    "fm_set_scan_tile", "fm_set_state_spec",
 )
 NOALLOC_SCRATCH_BYTES = 16 << 20  # FM_NOALLOC_SCRATCH_BYTES
 
@@ -86,6 +86,7 @@ def load():
         "fm_conv1d_pot": (I, [_P, I, I, sp, _P, _P, _P, _P, _P, _P]),
         "fm_ssm_scan_pot": (I, [_P, _P, I, I, sp, _P, _P, _P, _P, _P, _P, _P, SZ, _P]),
         "fm_scan_workspace_bytes": (SZ, [sp, I, I]),
+        "fm_set_state_spec": (I, [I, I]),
         "fm_set_scan_tile": (I, [I, I, I]),
         "fm_gate_norm_quant": (I, [_P, _P, I64, sp, _P, _P, I, I, _P, _P, _P, _P, _P]),
         "fm_eval_pwl": (I, [I, _P, I64, _P, _P]),
@@ -173,6 +174,12 @@ SCAN_TILES = ((4, 4, 16), (4, 2, 16), (4, 8, 16), (8, 4, 16), (8, 2, 16), (8, 8,
 
 def set_scan_tile(npt: int, pc: int, tch: int):
     _check(load().fm_set_scan_tile(npt, pc, tch))
+
+
+def set_state_spec(bits: int, guard: int):
+    """(31, 0): the int32 state as built (default); (16, 7): the narrow state
+    with the guard-bit increment.  Process-wide; set it before calibrating."""
+    _check(load().fm_set_state_spec(bits, guard))
 
 
 def scan_workspace_bytes(shape, B, T) -> int:

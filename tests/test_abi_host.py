@@ -150,3 +150,11 @@ def test_scan_and_tuning_validation(so):
     # gate: bad mode
     assert so.fm_gate_norm_quant(f[0], f[1], 4, C.byref(sh), f[2], f[3], 1, 5, None, f[4], f[5],
                                  None, None) == 1
+
+
+def test_state_spec_validation(so):
+    """Only the two state specs with kernels behind them are accepted."""
+    assert so.fm_set_state_spec(16, 0) == 1
+    assert so.fm_set_state_spec(24, 7) == 1
+    assert so.fm_set_state_spec(16, 7) == 0
+    assert so.fm_set_state_spec(31, 0) == 0
