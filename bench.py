@@ -69,6 +69,9 @@ def parse(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--scan-tile", default=None,
                     help="npt,pc,tch of the sequential scan kernel (a compiled variant)")
+    ap.add_argument("--state-spec", default="31,0", choices=["31,0", "16,7"],
+                    help="scan state word and increment guard bits: 31,0 the method as built, "
+                         "16,7 the narrow state with the guard-bit increment")
     ap.add_argument("--layers", type=int, default=None,
                     help="profiling only: run the first N layers of a stack workload")
     return ap.parse_args(argv)
@@ -109,7 +112,7 @@ def config_block(args) -> dict:
                  calibration=f"{S.CALIB_SEQS} seeded sequences x "
                              f"{min(w.get('prefill_len', w['seqlen']), S.CALIB_MAX_LEN)} tokens "
                              "(GPU, stage by stage)",
-                 scan_tile=args.scan_tile or "4,4,16")
+                 scan_tile=args.scan_tile or "4,4,16", state_spec=args.state_spec)
         if "prefill_len" in w:
             c.update(prefill_len=w["prefill_len"], step="one decode token per sequence")
     return c
@@ -584,6 +587,7 @@ def main():
     lib.load()
     if args.scan_tile:
         lib.set_scan_tile(*[int(v) for v in args.scan_tile.split(",")])
+    lib.set_state_spec(*[int(v) for v in args.state_spec.split(",")])
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream(dev)
