@@ -461,7 +461,8 @@ class DecodeWorkload(StackWorkload):
 
     def roofline(self, dom_ms, peaks):
         d = self.shape
-        state = self.B * d.nheads * d.headdim * d.d_state * 4
+        esz = 2 if self.lib.STATE_BITS == 16 else 4      # int16 state under the narrow spec
+        state = self.B * d.nheads * d.headdim * d.d_state * esz
         io = self.B * (d.conv_ch + 4 * d.nheads + 4 * d.d_inner)
         achieved = (2 * state + io) / (dom_ms / 1e3) / 1e9
         peak = (peaks or {}).get("hbm_gbs", 6548.0)

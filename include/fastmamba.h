@@ -240,10 +240,12 @@ typedef struct fm_layer {
 /* Process-wide state spec of every scan entry point and of the calibration:
  * (31, 0), the default, is the method as built -- an int32 state clamped at
  * +-(2^30 - 1), the increment u B with u rounded first.  (16, 7) is the narrow
- * reading: the state clamps at +-32767 (still stored as int32) and the
- * increment is rshr(ug B, 7) with ug = satb(rshr(dt_q x, s_h - 7), 24); the
- * calibration leaves 2^14 of headroom.  Switch it before calibrating and keep
- * it for the layer's life.  Anything else: FM_ERR_INVALID_ARG. */
+ * reading: the state clamps at +-32767 and is stored as int16 -- every
+ * int32_t *state / ssm_state argument then points at an int16 [B, nh, hd, ds]
+ * buffer -- and the increment is rshr(ug B, 7) with
+ * ug = satb(rshr(dt_q x, s_h - 7), 24); the calibration leaves 2^14 of
+ * headroom.  Switch it before calibrating and allocating states, and keep it
+ * for the layer's life.  Anything else: FM_ERR_INVALID_ARG. */
 fm_status fm_set_state_spec(int bits, int guard);
 
 /* Workspace bytes fm_mixer_prefill / fm_decode_step need for B*T tokens. */

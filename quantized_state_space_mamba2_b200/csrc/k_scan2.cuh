@@ -373,10 +373,13 @@ __global__ void __launch_bounds__(PC *(128 / NPT) + 32) k_scan_seq(ScanSeqArgs a
   const long long Dq = a.D_q[h];
   int hh[NPT];
   unsigned hl[NPT];
-  int32_t *st = a.state ? a.state + (((headrow * hd) + p0 + pp) * 128 + n0) : nullptr;
+  // S16: the state buffer holds int16 (the narrow spec's storage)
+  const long long st_off = ((headrow * hd) + p0 + pp) * 128 + n0;
+  int32_t *st = a.state ? a.state + st_off : nullptr;
+  int16_t *st16 = a.state ? reinterpret_cast<int16_t *>(a.state) + st_off : nullptr;
 #pragma unroll
   for (int j = 0; j < NPT; ++j) {
-    const int v = st ? st[j] : 0;
+    const int v = a.state ? (S16 ? (int)st16[j] : st[j]) : 0;
     hh[j] = S16 ? v : v >> 16;
     hl[j] = S16 ? 0u : (unsigned)v & 0xFFFFu;
   }
@@ -448,9 +451,12 @@ __global__ void __launch_bounds__(PC *(128 / NPT) + 32) k_scan_seq(ScanSeqArgs a
     __syncwarp();
     if (lane32 == 0) mbar_arrive(&sm.empty[sl]);
   }
-  if (st) {
+  if (a.state) {
 #pragma unroll
-    for (int j = 0; j < NPT; ++j) st[j] = S16 ? hh[j] : (int)(((unsigned)hh[j] << 16) | hl[j]);
+    for (int j = 0; j < NPT; ++j) {
+      if constexpr (S16) st16[j] = (int16_t)hh[j];
+      else st[j] = (int)(((unsigned)hh[j] << 16) | hl[j]);
+    }
   }
 }
 
@@ -471,11 +477,25 @@ __global__ void __launch_bounds__(256) k_scan_step(ScanArgs a) {
   const int nh = a.nh, hd = a.hd, cc = a.cc, di = a.di;
   const int n0 = lane * 4;
   const long long headrow = (long long)b * nh + h;
+  // the narrow spec stores the state as int16: 4 columns = 8 bytes per load
+  const bool narrow = a.hlim <= kH16Lim;
   int4 *st = a.state ? reinterpret_cast<int4 *>(a.state + headrow * hd * 128) : nullptr;
+  int2 *st16 = a.state ? reinterpret_cast<int2 *>(reinterpret_cast<int16_t *>(a.state) +
+                                                  headrow * hd * 128)
+                       : nullptr;
   int4 hv[kStepPPW];
 #pragma unroll
-  for (int k = 0; k < kStepPPW; ++k)
-    hv[k] = st ? __ldcs(st + (warp + 8 * k) * 32 + lane) : make_int4(0, 0, 0, 0);
+  for (int k = 0; k < kStepPPW; ++k) {
+    if (!a.state) {
+      hv[k] = make_int4(0, 0, 0, 0);
+    } else if (narrow) {
+      const int2 w = __ldcs(st16 + (warp + 8 * k) * 32 + lane);
+      hv[k] = make_int4((int)(int16_t)(w.x & 0xFFFF), w.x >> 16, (int)(int16_t)(w.y & 0xFFFF),
+                        w.y >> 16);
+    } else {
+      hv[k] = __ldcs(st + (warp + 8 * k) * 32 + lane);
+    }
+  }
   const int8_t *row = a.xbc + (long long)b * cc;
   const uint32_t bw = *reinterpret_cast<const uint32_t *>(row + di + n0);
   const uint32_t cw = *reinterpret_cast<const uint32_t *>(row + di + 128 + n0);
@@ -496,7 +516,6 @@ __global__ void __launch_bounds__(256) k_scan_step(ScanArgs a) {
     Cv[j] = (int)(int8_t)((cw >> (8 * j)) & 0xFF);
   }
   // the state spec: a word of at most 16 bits needs no (hi, lo) split
-  const bool narrow = a.hlim <= kH16Lim;
   const int g = a.guard;
   int shi = 0, slo = 0;  // lane k (< 8) ends up holding channel warp + 8k's C.h sums
 #pragma unroll
@@ -528,7 +547,14 @@ __global__ void __launch_bounds__(256) k_scan_step(ScanArgs a) {
         alo += Cv[j] * (int)((unsigned)v & 0xFFFFu);
       }
     }
-    if (st) __stcs(st + (warp + 8 * k) * 32 + lane, make_int4(hn[0], hn[1], hn[2], hn[3]));
+    if (a.state) {
+      if (narrow)
+        __stcs(st16 + (warp + 8 * k) * 32 + lane,
+               make_int2((int)(((unsigned)hn[0] & 0xFFFFu) | ((unsigned)hn[1] << 16)),
+                         (int)(((unsigned)hn[2] & 0xFFFFu) | ((unsigned)hn[3] << 16))));
+      else
+        __stcs(st + (warp + 8 * k) * 32 + lane, make_int4(hn[0], hn[1], hn[2], hn[3]));
+    }
     ahi = __reduce_add_sync(0xffffffffu, ahi);
     alo = narrow ? 0 : __reduce_add_sync(0xffffffffu, alo);
     if (lane == k) {

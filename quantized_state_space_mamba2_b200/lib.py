@@ -176,10 +176,16 @@ def set_scan_tile(npt: int, pc: int, tch: int):
     _check(load().fm_set_scan_tile(npt, pc, tch))
 
 
+STATE_BITS = 31  # the state spec in force (set_state_spec)
+
+
 def set_state_spec(bits: int, guard: int):
     """(31, 0): the int32 state as built (default); (16, 7): the narrow state
-    with the guard-bit increment.  Process-wide; set it before calibrating."""
+    with the guard-bit increment, its state buffers int16.  Process-wide; set
+    it before calibrating and allocating states."""
+    global STATE_BITS
     _check(load().fm_set_state_spec(bits, guard))
+    STATE_BITS = bits
 
 
 def scan_workspace_bytes(shape, B, T) -> int:

@@ -1,7 +1,8 @@
 """The narrow state spec on the GPU (fm_set_state_spec(16, 7)): every scan
 kernel (sequential prefill, decode step, calibration statistics) against the
-oracle's 16-bit state with the guard-bit increment, bit for bit; a calibrated
-layer's tables, prefill output, decode steps and carried states likewise.
+oracle's 16-bit state with the guard-bit increment, bit for bit, the state
+stored as int16; a calibrated layer's tables, prefill output, decode steps
+and carried states likewise.
 The spec is process-wide, so each test restores the default."""
 import numpy as np
 import pytest
@@ -71,7 +72,7 @@ def test_scan_state16_matches_oracle(L, spec16, B, T):
     exps = _exps(L, s, e_x, e_B, e_C, e_h, e_y, e_D)
     st = S.uniform_ints((B, s.nheads, s.headdim, s.d_state), -20000, 20000, seed=9)
     y = torch.empty((B, T, s.d_inner), dtype=torch.int32, device="cuda")
-    st_d = dev(st)
+    st_d = dev(st.astype(np.int16))                          # the narrow spec's storage
     ws = torch.empty(L.scan_workspace_bytes(s, B, T), dtype=torch.uint8, device="cuda")
     L.ssm_scan_pot(dev(xbc), dev(dt_raw), B, T, s, dev(dt_bias), dev(A_q), dev(D_q), dev(exps),
                    st_d, y, ws)
@@ -81,7 +82,7 @@ def test_scan_state16_matches_oracle(L, spec16, B, T):
                         s.d_state, state=st_r, state_bits=16, ub_guard=7)
     assert np.abs(st_r).max() <= 32767
     assert np.array_equal(host(y), yr)
-    assert np.array_equal(host(st_d), st_r)
+    assert np.array_equal(host(st_d).astype(np.int32), st_r)
 
 
 def test_layer_state16_matches_oracle(L, spec16):
@@ -111,4 +112,5 @@ def test_layer_state16_matches_oracle(L, spec16):
     ss_r = np.zeros((2, s.nheads, s.headdim, s.d_state), np.int32)
     ref = O.mixer_prefill(ol, x, conv_state=cs_r, ssm_state=ss_r)
     assert np.array_equal(np.concatenate(outs, 1), ref)
-    assert np.array_equal(host(cs), cs_r) and np.array_equal(host(ss), ss_r)
+    assert ss.dtype == torch.int16
+    assert np.array_equal(host(cs), cs_r) and np.array_equal(host(ss).astype(np.int32), ss_r)
