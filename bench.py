@@ -73,6 +73,9 @@ def parse(argv=None):
     ap.add_argument("--scan-mode", default="seq", choices=["seq", "ssd"],
                     help="seq: the sequential fixed-point scan (the method); ssd: the chunked "
                          "tensor-core scan mode (its own error budget)")
+    ap.add_argument("--state-spec", default="31,0", choices=["31,0", "16,7"],
+                    help="scan state word and increment guard bits: 31,0 the method as built, "
+                         "16,7 the narrow state with the guard-bit increment")
     ap.add_argument("--layers", type=int, default=None,
                     help="profiling only: run the first N layers of a stack workload")
     return ap.parse_args(argv)
@@ -113,7 +116,8 @@ def config_block(args) -> dict:
                  calibration=f"{S.CALIB_SEQS} seeded sequences x "
                              f"{min(w.get('prefill_len', w['seqlen']), S.CALIB_MAX_LEN)} tokens "
                              "(GPU, stage by stage)",
-                 scan_tile=args.scan_tile or "4,4,16", scan_mode=args.scan_mode)
+                 scan_tile=args.scan_tile or "4,4,16", scan_mode=args.scan_mode,
+                 state_spec=args.state_spec)
         if "prefill_len" in w:
             c.update(prefill_len=w["prefill_len"], step="one decode token per sequence")
     return c
@@ -476,7 +480,8 @@ class DecodeWorkload(StackWorkload):
 
     def roofline(self, dom_ms, peaks):
         d = self.shape
-        state = self.B * d.nheads * d.headdim * d.d_state * 4
+        esz = 2 if self.lib.STATE_BITS == 16 else 4      # int16 state under the narrow spec
+        state = self.B * d.nheads * d.headdim * d.d_state * esz
         io = self.B * (d.conv_ch + 4 * d.nheads + 4 * d.d_inner)
         achieved = (2 * state + io) / (dom_ms / 1e3) / 1e9
         peak = (peaks or {}).get("hbm_gbs", 6548.0)
@@ -603,6 +608,7 @@ def main():
     if args.scan_tile:
         lib.set_scan_tile(*[int(v) for v in args.scan_tile.split(",")])
     lib.set_scan_mode(args.scan_mode)
+    lib.set_state_spec(*[int(v) for v in args.state_spec.split(",")])
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream(dev)

@@ -256,6 +256,16 @@ fm_status fm_ssd_scan(const int8_t *xbc, const float *dt_raw, int B, int T,
                       const fm_shape *shape, const float *dt_bias, const int32_t *A_q,
                       const int32_t *D_q, const int32_t *exps, int32_t *state, int32_t *y,
                       void *ws, size_t ws_bytes, fm_stream stream);
+/* Process-wide state spec of every scan entry point and of the calibration:
+ * (31, 0), the default, is the method as built -- an int32 state clamped at
+ * +-(2^30 - 1), the increment u B with u rounded first.  (16, 7) is the narrow
+ * reading: the state clamps at +-32767 and is stored as int16 -- every
+ * int32_t *state / ssm_state argument then points at an int16 [B, nh, hd, ds]
+ * buffer -- and the increment is rshr(ug B, 7) with
+ * ug = satb(rshr(dt_q x, s_h - 7), 24); the calibration leaves 2^14 of
+ * headroom.  Switch it before calibrating and allocating states, and keep it
+ * for the layer's life.  Anything else: FM_ERR_INVALID_ARG. */
+fm_status fm_set_state_spec(int bits, int guard);
 
 /* Workspace bytes fm_mixer_prefill / fm_decode_step need for B*T tokens. */
 size_t fm_workspace_bytes(const fm_shape *shape, int B, int T);

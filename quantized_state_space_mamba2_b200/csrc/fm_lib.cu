@@ -341,6 +341,22 @@ static fm_status launch_conv(const int8_t *u, int B, int T, int cc, const int8_t
   return FM_OK;
 }
 
+// The state spec, process-wide: the word width and the increment's guard
+// bits.  (31, 0) is the method as built; (16, 7) the narrow state whose
+// increment is rounded after the u B product (u with 7 guard bits).
+static std::atomic<int> g_state_bits{31};
+static std::atomic<int> g_state_guard{0};
+
+extern "C" fm_status fm_set_state_spec(int bits, int guard) {
+  if (!((bits == 31 && guard == 0) || (bits == 16 && guard == 7)))
+    return fail(FM_ERR_INVALID_ARG, "fm_set_state_spec: (%d, %d) is not a supported spec "
+                "(31, 0) or (16, 7)", bits, guard);
+  g_state_bits.store(bits, std::memory_order_relaxed);
+  g_state_guard.store(guard, std::memory_order_relaxed);
+  return FM_OK;
+}
+static bool state16() { return g_state_bits.load(std::memory_order_relaxed) == 16; }
+
 static ScanArgs scan_args(const Dims &d, const int8_t *xbc, const float *dt_raw, int T,
                           const float *dt_bias, const int32_t *A_q, const int32_t *D_q,
                           const int32_t *exps, const fm_exp_layout &X, int32_t *state, int32_t *y,
@@ -365,6 +381,8 @@ static ScanArgs scan_args(const Dims &d, const int8_t *xbc, const float *dt_raw,
   a.state = state;
   a.y = y;
   a.stat = stat;
+  a.hlim = state16() ? kH16Lim : (int)kHLim;
+  a.guard = g_state_guard.load(std::memory_order_relaxed);
   return a;
 }
 
@@ -407,11 +425,11 @@ extern "C" fm_status fm_set_scan_tile(int npt, int pc, int tch) {
               pc, tch);
 }
 
-template <int NPT, int PC, int TCH>
+template <int NPT, int PC, int TCH, bool S16>
 static fm_status launch_seq(const ScanSeqArgs &a, int B, cudaStream_t s) {
   using Sm = ScanSeqSmem<NPT, PC, TCH>;
   constexpr int smem = (int)sizeof(Sm);
-  auto kern = k_scan_seq<NPT, PC, TCH>;
+  auto kern = k_scan_seq<NPT, PC, TCH, S16>;
   FM_CHECK_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
   dim3 grid(a.hd / PC, a.nh, B);
   kern<<<grid, PC * (128 / NPT) + 32, smem, s>>>(a);
@@ -457,6 +475,7 @@ static fm_status launch_scan_v2(const ScanArgs &a, int B, const ScanWs &w, cudaS
   p.xs = w.xs;
   p.bc = w.bc;
   p.bound = w.bound;
+  p.guard = a.guard;
   k_scan_prep<<<dim3((unsigned)(Tp / kPrepTT), a.nh, B), 256, 0, s>>>(p);
   FM_TRY(launched("k_scan_prep"));
   ScanSeqArgs q;
@@ -478,8 +497,10 @@ static fm_status launch_scan_v2(const ScanArgs &a, int B, const ScanWs &w, cudaS
   q.state = a.state;
   q.y = a.y;
   const ScanTile t = scan_tile();
-#define FM_SEQ(N, P, C) \
-  if (t.npt == N && t.pc == P && t.tch == C) return launch_seq<N, P, C>(q, B, s);
+#define FM_SEQ(N, P, C)                                      \
+  if (t.npt == N && t.pc == P && t.tch == C)                 \
+    return state16() ? launch_seq<N, P, C, true>(q, B, s)    \
+                     : launch_seq<N, P, C, false>(q, B, s);
   FM_SEQ(4, 4, 16)
   FM_SEQ(4, 2, 16)
   FM_SEQ(4, 8, 16)
@@ -1129,12 +1150,13 @@ __global__ void k_exp_conv_out(const unsigned int *amax, int di, int hd, int ds,
   for (int c = threadIdx.x; c < cc; c += blockDim.x)
     exps[X.e_o + c] = c < di ? exps[X.e_x + c / hd] : (c < di + ds ? exps[X.e_B] : exps[X.e_C]);
 }
+// headroom: 2^29 of the 31-bit state's 2^30 clamp, 2^14 of the 16-bit one's 2^15
 __global__ void k_exp_state(const unsigned long long *amax_h, int nh, int32_t *exps,
-                            fm_exp_layout X) {
+                            fm_exp_layout X, double headroom) {
   const int h = threadIdx.x;
   if (h >= nh) return;
   const int ef = exps[X.e_x + h] + exps[X.e_B] - 15;
-  const int e = pot_exponent((double)amax_h[h], 536870912.0) + ef;
+  const int e = pot_exponent((double)amax_h[h], headroom) + ef;
   exps[X.e_h + h] = e > ef ? e : ef;
 }
 __global__ void k_exp_y(const unsigned long long *ystat, int nh, int32_t *exps, fm_exp_layout X) {
@@ -1253,7 +1275,7 @@ extern "C" fm_status fm_calibrate_layer(const fm_layer *L, const float *conv_b, 
   FM_TRY(launch_scan<2>(scan_args(d, m.xo, m.dt, T, L->dt_bias, L->A_q, L->D_q, exps, X, nullptr,
                                   m.y, w.stat),
                         B, s));
-  k_exp_state<<<1, 128, 0, s>>>(w.stat, d.nh, exps, X);
+  k_exp_state<<<1, 128, 0, s>>>(w.stat, d.nh, exps, X, state16() ? 16384.0 : 536870912.0);
   FM_TRY(launched("k_exp_state"));
   // 5. output exponent: max |y| at the finer term exponent
   FM_CHECK_CUDA(cudaMemsetAsync(w.stat, 0, sizeof(unsigned long long) * d.nh, s));

@@ -42,7 +42,16 @@ struct ScanArgs {
   int32_t *state;         // [B, nh, hd, ds] or null
   int32_t *y;             // [B, T, di]
   unsigned long long *stat;  // [nh]: MODE 1 max|y_f|, MODE 2 max|h64|
+  // state spec: the clamp +-hlim and the increment's guard bits g (the
+  // increment is rshr(ug B, g) with ug = satb(rshr(dt_q x, s_h - g), 24));
+  // the method as built is hlim = 2^30 - 1, g = 0
+  int hlim, guard;
 };
+
+// rshr(v, g) for g in [0, 7] (g = 0: v)
+__device__ __forceinline__ int rshr_guard(int v, int g) {
+  return g ? (v + (1 << (g - 1))) >> g : v;
+}
 
 // MODE 0: the scan.  MODE 1: the scan + max |y| at the finer term exponent
 // (calibration of e_y).  MODE 2: calibration of e_h -- 64-bit state at the
@@ -129,7 +138,7 @@ __global__ void __launch_bounds__(kScanThreads) k_ssm_scan_pot(ScanArgs a) {
     for (int i = tid; i < nt * kScanPC; i += kScanThreads) {
       const int tt = i / kScanPC, q = i % kScanPC;
       const long long prod = (long long)sdt[tt] * sx[tt][q];
-      su[tt][q] = MODE == 2 ? rshr64(prod, 1) : satb64(rshr64(prod, s_h), 24);
+      su[tt][q] = MODE == 2 ? rshr64(prod, 1) : satb64(rshr64(prod, s_h - a.guard), 24);
     }
     __syncthreads();
 
@@ -159,8 +168,8 @@ __global__ void __launch_bounds__(kScanThreads) k_ssm_scan_pot(ScanArgs a) {
 #pragma unroll
       for (int j = 0; j < kScanNPT; ++j) {
         const int dec = (int)((dA * (long long)hs[j] + 32768LL) >> 16);
-        int hn = dec + u32 * Bv[j];
-        hn = min(max(hn, -(int)kHLim), (int)kHLim);
+        int hn = dec + rshr_guard(u32 * Bv[j], a.guard);
+        hn = min(max(hn, -a.hlim), a.hlim);
         hs[j] = (StateT)hn;
         acc += (long long)Cv[j] * hn;
       }

@@ -51,7 +51,8 @@ struct ScanPrepArgs {
   int32_t *u;    // [B, nh, hd, Tp]
   int32_t *xs;   // [B, nh, hd, Tp]: the x code, widened
   int32_t *bc;   // [B*T, 256]: B then C, int32
-  long long *bound;  // [B, nh, Tp/16, hd]: per 16-step chunk, sum of |u| max|B|
+  long long *bound;  // [B, nh, Tp/16, hd]: per 16-step chunk, bound of the increments
+  int guard;         // the increment's guard bits (0: the method as built)
 };
 
 // grid = (Tp / 32, nh, B), block = 256; hd == 64
@@ -103,17 +104,21 @@ __global__ void __launch_bounds__(256) k_scan_prep(ScanPrepArgs a) {
   {  // (u, x) for channel p = tid / 4, tokens 8 * (tid % 4) .. + 8
     const int p = tid >> 2, tb = (tid & 3) * 8;
     const int s_h = a.e_h[h] - *a.e_B - a.e_x[h] + 16;
+    const int g = a.guard;
     int uv[8], dv[8];
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
       const long long x = sx[tb + k][p];
-      uv[k] = (int)satb64(rshr64((long long)s_dtq[tb + k] * x, s_h), 24);
+      uv[k] = (int)satb64(rshr64((long long)s_dtq[tb + k] * x, s_h - g), 24);
       dv[k] = (int)x;
     }
-    // growth bound of |h| over this thread's 8 steps; two threads make a 16-step chunk
+    // growth bound of |h| over this thread's 8 steps (an increment
+    // rshr(u B, g) is at most ceil(|u| max|B| / 2^g)); two threads make a
+    // 16-step chunk
     long long gb = 0;
 #pragma unroll
-    for (int k = 0; k < 8; ++k) gb += (long long)abs(uv[k]) * s_bmax[tb + k];
+    for (int k = 0; k < 8; ++k)
+      gb += ((long long)abs(uv[k]) * s_bmax[tb + k] + ((1LL << g) - 1)) >> g;
     gb += __shfl_xor_sync(0xffffffffu, gb, 1);
     if ((tid & 1) == 0)
       a.bound[(((long long)b * nh + h) * (Tp / 16) + (t0 + tb) / 16) * hd + p] = gb;
@@ -205,11 +210,28 @@ __device__ __forceinline__ void load_bc(const int32_t (*bc)[256], int tt, int n0
 // false is used only when the chunk provably never reaches the clamp (see
 // k_scan_seq), so both instantiations give the same bits.  part[tt] holds the
 // (C hh, C hl) partial sums of step tt.
-template <int NPT, bool CLAMP>
+// S16: the 16-bit state spec (|h| <= 2^15 - 1, so dA h fits int32 and no
+// split is needed; the increment is rshr(u B, 7) with u carrying 7 guard
+// bits): h lives in hh, hl is unused, and the C h sum is the single .x.
+constexpr int kH16Lim = 32767;
+constexpr int kH16Guard = 7;
+
+template <int NPT, bool CLAMP, bool S16 = false>
 __device__ __forceinline__ int2 scan_one_step(int (&hh)[NPT], unsigned (&hl)[NPT],
                                               const int (&Bv)[NPT], const int (&Cv)[NPT], int dA,
                                               int u) {
   int ahi = 0, alo = 0;
+  if constexpr (S16) {
+#pragma unroll
+    for (int j = 0; j < NPT; ++j) {
+      const int t = dA * hh[j] + 0x8000;
+      int hn = (t >> 16) + ((u * Bv[j] + (1 << (kH16Guard - 1))) >> kH16Guard);
+      if (CLAMP) hn = min(max(hn, -kH16Lim), kH16Lim);
+      hh[j] = hn;
+      ahi += Cv[j] * hn;
+    }
+    return make_int2(ahi, 0);
+  }
 #pragma unroll
   for (int j = 0; j < NPT; ++j) {
     const unsigned t = (unsigned)dA * hl[j] + 0x8000u;
@@ -227,7 +249,7 @@ __device__ __forceinline__ int2 scan_one_step(int (&hh)[NPT], unsigned (&hl)[NPT
 // -- when one warp is one channel (32 threads per channel) -- are summed over
 // the warp at once (redux.sync) and lane 0 stores the step's sums to
 // wsum[tt] (REDUX = true): no per-step partials are kept in registers.
-template <int NPT, int TCH, bool FULL, bool CLAMP, bool REDUX>
+template <int NPT, int TCH, bool FULL, bool CLAMP, bool REDUX, bool S16 = false>
 __device__ __forceinline__ void scan_chunk_steps(int (&hh)[NPT], unsigned (&hl)[NPT],
                                                  int2 (&part)[TCH], int2 *wsum,
                                                  const int32_t (*bc)[256], const int32_t *dAv,
@@ -243,7 +265,7 @@ __device__ __forceinline__ void scan_chunk_steps(int (&hh)[NPT], unsigned (&hl)[
   auto emit = [&](int tt, int2 v) {
     if constexpr (REDUX) {
       const int shi = __reduce_add_sync(0xffffffffu, v.x);
-      const int slo = __reduce_add_sync(0xffffffffu, v.y);
+      const int slo = S16 ? 0 : __reduce_add_sync(0xffffffffu, v.y);
       if (lead && pend_tt >= 0) wsum[pend_tt] = pend;
       pend = make_int2(shi, slo);
       pend_tt = tt;
@@ -262,11 +284,11 @@ __device__ __forceinline__ void scan_chunk_steps(int (&hh)[NPT], unsigned (&hl)[
     for (int k = 0; k < 4; k += 2) {
       const int tt = tg + k;
       if (FULL || tt + 1 < nt) load_bc<NPT>(bc, tt + 1, n0, B1, C1);
-      if (FULL || tt < nt) emit(tt, scan_one_step<NPT, CLAMP>(hh, hl, B0, C0, dAs[k], us[k]));
+      if (FULL || tt < nt) emit(tt, scan_one_step<NPT, CLAMP, S16>(hh, hl, B0, C0, dAs[k], us[k]));
       else if constexpr (!REDUX) part[tt] = make_int2(0, 0);
       if (tt + 2 < TCH && (FULL || tt + 2 < nt)) load_bc<NPT>(bc, tt + 2, n0, B0, C0);
       if (FULL || tt + 1 < nt)
-        emit(tt + 1, scan_one_step<NPT, CLAMP>(hh, hl, B1, C1, dAs[k + 1], us[k + 1]));
+        emit(tt + 1, scan_one_step<NPT, CLAMP, S16>(hh, hl, B1, C1, dAs[k + 1], us[k + 1]));
       else if constexpr (!REDUX) part[tt + 1] = make_int2(0, 0);
     }
   }
@@ -280,7 +302,7 @@ __device__ __forceinline__ void scan_chunk_steps(int (&hh)[NPT], unsigned (&hl)[
 // compute warp has released the chunk that used the slot before (empty
 // barrier, one arrival per compute warp), and signals it through the slot's
 // transaction-count barrier.  Compute warps never wait for each other.
-template <int NPT, int PC, int TCH>
+template <int NPT, int PC, int TCH, bool S16 = false>
 __global__ void __launch_bounds__(PC *(128 / NPT) + 32) k_scan_seq(ScanSeqArgs a) {
   constexpr int LPP = 128 / NPT;
   constexpr int NW = PC * LPP / 32;
@@ -351,12 +373,15 @@ __global__ void __launch_bounds__(PC *(128 / NPT) + 32) k_scan_seq(ScanSeqArgs a
   const long long Dq = a.D_q[h];
   int hh[NPT];
   unsigned hl[NPT];
-  int32_t *st = a.state ? a.state + (((headrow * hd) + p0 + pp) * 128 + n0) : nullptr;
+  // S16: the state buffer holds int16 (the narrow spec's storage)
+  const long long st_off = ((headrow * hd) + p0 + pp) * 128 + n0;
+  int32_t *st = a.state ? a.state + st_off : nullptr;
+  int16_t *st16 = a.state ? reinterpret_cast<int16_t *>(a.state) + st_off : nullptr;
 #pragma unroll
   for (int j = 0; j < NPT; ++j) {
-    const int v = st ? st[j] : 0;
-    hh[j] = v >> 16;
-    hl[j] = (unsigned)v & 0xFFFFu;
+    const int v = a.state ? (S16 ? (int)st16[j] : st[j]) : 0;
+    hh[j] = S16 ? v : v >> 16;
+    hl[j] = S16 ? 0u : (unsigned)v & 0xFFFFu;
   }
   int2(*part)[PSTRIDE] = sm.part[warp];
   for (int c = 0; c < nchunks; ++c) {
@@ -370,23 +395,25 @@ __global__ void __launch_bounds__(PC *(128 / NPT) + 32) k_scan_seq(ScanSeqArgs a
     // is the identity at every step and the cheaper path is exact.
     int hmax = 0;
 #pragma unroll
-    for (int j = 0; j < NPT; ++j) hmax = max(hmax, abs((int)(((unsigned)hh[j] << 16) | hl[j])));
-    const bool no_clamp = __all_sync(0xffffffffu, (long long)hmax + s.bound[pp] <= kHLim);
+    for (int j = 0; j < NPT; ++j)
+      hmax = max(hmax, abs(S16 ? hh[j] : (int)(((unsigned)hh[j] << 16) | hl[j])));
+    const bool no_clamp = __all_sync(0xffffffffu, (long long)hmax + s.bound[pp] <=
+                                                      (S16 ? (long long)kH16Lim : kHLim));
     int2 pr[TCH];
     int2 *wsum = reinterpret_cast<int2 *>(&part[0][0]);
     if (nt == TCH) {
       if (no_clamp)
-        scan_chunk_steps<NPT, TCH, true, false, REDUX>(hh, hl, pr, wsum, s.bc, s.dA, s.u[pp], n0, nt);
+        scan_chunk_steps<NPT, TCH, true, false, REDUX, S16>(hh, hl, pr, wsum, s.bc, s.dA, s.u[pp], n0, nt);
       else
-        scan_chunk_steps<NPT, TCH, true, true, REDUX>(hh, hl, pr, wsum, s.bc, s.dA, s.u[pp], n0, nt);
+        scan_chunk_steps<NPT, TCH, true, true, REDUX, S16>(hh, hl, pr, wsum, s.bc, s.dA, s.u[pp], n0, nt);
     } else {
-      scan_chunk_steps<NPT, TCH, false, true, REDUX>(hh, hl, pr, wsum, s.bc, s.dA, s.u[pp], n0, nt);
+      scan_chunk_steps<NPT, TCH, false, true, REDUX, S16>(hh, hl, pr, wsum, s.bc, s.dA, s.u[pp], n0, nt);
     }
     if constexpr (REDUX) {  // one channel per warp: lane tt finishes step tt
       __syncwarp();
       if (lane32 < nt) {
         const int2 v = wsum[lane32];
-        const long long sum = (long long)v.x * 65536 + v.y;
+        const long long sum = S16 ? (long long)v.x : (long long)v.x * 65536 + v.y;
         a.y[(rowbase + t0 + lane32) * di + (long long)h * hd + p0 + pp] =
             (int)satb64(rshr64(sum, s_y) + rshr64(Dq * s.xs[pp][lane32], s_D), 32);
       }
@@ -416,7 +443,7 @@ __global__ void __launch_bounds__(PC *(128 / NPT) + 32) k_scan_seq(ScanSeqArgs a
       }
       const int tt = row / PPW, q = warp * PPW + row % PPW;
       if (half == 0 && tt < nt) {
-        const long long sum = (long long)shi * 65536 + slo;
+        const long long sum = S16 ? (long long)shi : (long long)shi * 65536 + slo;
         a.y[(rowbase + t0 + tt) * di + (long long)h * hd + p0 + q] =
             (int)satb64(rshr64(sum, s_y) + rshr64(Dq * s.xs[q][tt], s_D), 32);
       }
@@ -424,9 +451,12 @@ __global__ void __launch_bounds__(PC *(128 / NPT) + 32) k_scan_seq(ScanSeqArgs a
     __syncwarp();
     if (lane32 == 0) mbar_arrive(&sm.empty[sl]);
   }
-  if (st) {
+  if (a.state) {
 #pragma unroll
-    for (int j = 0; j < NPT; ++j) st[j] = (int)(((unsigned)hh[j] << 16) | hl[j]);
+    for (int j = 0; j < NPT; ++j) {
+      if constexpr (S16) st16[j] = (int16_t)hh[j];
+      else st[j] = (int)(((unsigned)hh[j] << 16) | hl[j]);
+    }
   }
 }
 
@@ -447,11 +477,25 @@ __global__ void __launch_bounds__(256) k_scan_step(ScanArgs a) {
   const int nh = a.nh, hd = a.hd, cc = a.cc, di = a.di;
   const int n0 = lane * 4;
   const long long headrow = (long long)b * nh + h;
+  // the narrow spec stores the state as int16: 4 columns = 8 bytes per load
+  const bool narrow = a.hlim <= kH16Lim;
   int4 *st = a.state ? reinterpret_cast<int4 *>(a.state + headrow * hd * 128) : nullptr;
+  int2 *st16 = a.state ? reinterpret_cast<int2 *>(reinterpret_cast<int16_t *>(a.state) +
+                                                  headrow * hd * 128)
+                       : nullptr;
   int4 hv[kStepPPW];
 #pragma unroll
-  for (int k = 0; k < kStepPPW; ++k)
-    hv[k] = st ? __ldcs(st + (warp + 8 * k) * 32 + lane) : make_int4(0, 0, 0, 0);
+  for (int k = 0; k < kStepPPW; ++k) {
+    if (!a.state) {
+      hv[k] = make_int4(0, 0, 0, 0);
+    } else if (narrow) {
+      const int2 w = __ldcs(st16 + (warp + 8 * k) * 32 + lane);
+      hv[k] = make_int4((int)(int16_t)(w.x & 0xFFFF), w.x >> 16, (int)(int16_t)(w.y & 0xFFFF),
+                        w.y >> 16);
+    } else {
+      hv[k] = __ldcs(st + (warp + 8 * k) * 32 + lane);
+    }
+  }
   const int8_t *row = a.xbc + (long long)b * cc;
   const uint32_t bw = *reinterpret_cast<const uint32_t *>(row + di + n0);
   const uint32_t cw = *reinterpret_cast<const uint32_t *>(row + di + 128 + n0);
@@ -471,28 +515,48 @@ __global__ void __launch_bounds__(256) k_scan_step(ScanArgs a) {
     Bv[j] = (int)(int8_t)((bw >> (8 * j)) & 0xFF);
     Cv[j] = (int)(int8_t)((cw >> (8 * j)) & 0xFF);
   }
+  // the state spec: a word of at most 16 bits needs no (hi, lo) split
+  const int g = a.guard;
   int shi = 0, slo = 0;  // lane k (< 8) ends up holding channel warp + 8k's C.h sums
 #pragma unroll
   for (int k = 0; k < kStepPPW; ++k) {
     const long long xq = xs[k];
-    const int u = (int)satb64(rshr64((long long)dtq * xq, s_h), 24);
+    const int u = (int)satb64(rshr64((long long)dtq * xq, s_h - g), 24);
     const int hs[4] = {hv[k].x, hv[k].y, hv[k].z, hv[k].w};
     int hn[4];
     int ahi = 0, alo = 0;
+    if (narrow) {
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int hh = hs[j] >> 16;
-      const unsigned hl = (unsigned)hs[j] & 0xFFFFu;
-      const unsigned t = (unsigned)dA * hl + 0x8000u;
-      int v = dA * hh + (int)(t >> 16) + u * Bv[j];
-      v = min(max(v, -(int)kHLim), (int)kHLim);
-      hn[j] = v;
-      ahi += Cv[j] * (v >> 16);
-      alo += Cv[j] * (int)((unsigned)v & 0xFFFFu);
+      for (int j = 0; j < 4; ++j) {
+        const int t = dA * hs[j] + 0x8000;
+        int v = (t >> 16) + rshr_guard(u * Bv[j], g);
+        v = min(max(v, -a.hlim), a.hlim);
+        hn[j] = v;
+        ahi += Cv[j] * v;
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int hh = hs[j] >> 16;
+        const unsigned hl = (unsigned)hs[j] & 0xFFFFu;
+        const unsigned t = (unsigned)dA * hl + 0x8000u;
+        int v = dA * hh + (int)(t >> 16) + rshr_guard(u * Bv[j], g);
+        v = min(max(v, -a.hlim), a.hlim);
+        hn[j] = v;
+        ahi += Cv[j] * (v >> 16);
+        alo += Cv[j] * (int)((unsigned)v & 0xFFFFu);
+      }
     }
-    if (st) __stcs(st + (warp + 8 * k) * 32 + lane, make_int4(hn[0], hn[1], hn[2], hn[3]));
+    if (a.state) {
+      if (narrow)
+        __stcs(st16 + (warp + 8 * k) * 32 + lane,
+               make_int2((int)(((unsigned)hn[0] & 0xFFFFu) | ((unsigned)hn[1] << 16)),
+                         (int)(((unsigned)hn[2] & 0xFFFFu) | ((unsigned)hn[3] << 16))));
+      else
+        __stcs(st + (warp + 8 * k) * 32 + lane, make_int4(hn[0], hn[1], hn[2], hn[3]));
+    }
     ahi = __reduce_add_sync(0xffffffffu, ahi);
-    alo = __reduce_add_sync(0xffffffffu, alo);
+    alo = narrow ? 0 : __reduce_add_sync(0xffffffffu, alo);
     if (lane == k) {
       shi = ahi;
       slo = alo;
@@ -501,7 +565,7 @@ __global__ void __launch_bounds__(256) k_scan_step(ScanArgs a) {
   if (lane < kStepPPW) {  // one output per lane: channel warp + 8 lane
     const int p = warp + 8 * lane;
     const long long xq = row[h * hd + p];
-    const long long sum = (long long)shi * 65536 + slo;
+    const long long sum = narrow ? (long long)shi : (long long)shi * 65536 + slo;
     a.y[(long long)b * di + (long long)h * hd + p] =
         (int)satb64(rshr64(sum, s_y) + rshr64(Dq * xq, s_D), 32);
   }

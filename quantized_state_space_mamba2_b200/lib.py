@@ -28,6 +28,7 @@ EXPORTS = (
     "fm_mixer_prefill", "fm_decode_step", "fm_prepare_mixer_params", "fm_calib_workspace_bytes",
     "fm_calibrate_layer", "fm_decode_step_noalloc", "fm_scan_workspace_bytes",
     "fm_set_scan_tile", "fm_ssd_workspace_bytes", "fm_ssd_scan", "fm_set_scan_mode",
+    "fm_set_scan_tile", "fm_set_state_spec",
 )
 NOALLOC_SCRATCH_BYTES = 16 << 20  # FM_NOALLOC_SCRATCH_BYTES
 
@@ -89,6 +90,7 @@ def load():
         "fm_ssd_scan": (I, [_P, _P, I, I, sp, _P, _P, _P, _P, _P, _P, _P, SZ, _P]),
         "fm_ssd_workspace_bytes": (SZ, [sp, I, I]),
         "fm_set_scan_mode": (I, [I]),
+        "fm_set_state_spec": (I, [I, I]),
         "fm_set_scan_tile": (I, [I, I, I]),
         "fm_gate_norm_quant": (I, [_P, _P, I64, sp, _P, _P, I, I, _P, _P, _P, _P, _P]),
         "fm_eval_pwl": (I, [I, _P, I64, _P, _P]),
@@ -176,6 +178,18 @@ SCAN_TILES = ((4, 4, 16), (4, 2, 16), (4, 8, 16), (8, 4, 16), (8, 2, 16), (8, 8,
 
 def set_scan_tile(npt: int, pc: int, tch: int):
     _check(load().fm_set_scan_tile(npt, pc, tch))
+
+
+STATE_BITS = 31  # the state spec in force (set_state_spec)
+
+
+def set_state_spec(bits: int, guard: int):
+    """(31, 0): the int32 state as built (default); (16, 7): the narrow state
+    with the guard-bit increment, its state buffers int16.  Process-wide; set
+    it before calibrating and allocating states."""
+    global STATE_BITS
+    _check(load().fm_set_state_spec(bits, guard))
+    STATE_BITS = bits
 
 
 def scan_workspace_bytes(shape, B, T) -> int:

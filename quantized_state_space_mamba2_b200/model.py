@@ -127,9 +127,9 @@ class DeviceLayer:
 
     def new_states(self, B: int):
         s = self.shape
+        sdt = torch.int16 if lib.STATE_BITS == 16 else torch.int32  # the state spec's storage
         return (torch.zeros((B, 3, s.conv_ch), dtype=torch.int8, device=self.device),
-                torch.zeros((B, s.nheads, s.headdim, s.d_state), dtype=torch.int32,
-                            device=self.device))
+                torch.zeros((B, s.nheads, s.headdim, s.d_state), dtype=sdt, device=self.device))
 
 
 class DeviceStack:

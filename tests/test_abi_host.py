@@ -177,3 +177,9 @@ def test_chunked_scan_validation(so):
     # scan mode switch
     assert so.fm_set_scan_mode(2) == 1
     assert so.fm_set_scan_mode(0) == 0
+def test_state_spec_validation(so):
+    """Only the two state specs with kernels behind them are accepted."""
+    assert so.fm_set_state_spec(16, 0) == 1
+    assert so.fm_set_state_spec(24, 7) == 1
+    assert so.fm_set_state_spec(16, 7) == 0
+    assert so.fm_set_state_spec(31, 0) == 0
