@@ -283,6 +283,16 @@ def _stage_buffers(torch, d, M, dev):
                 sx_out=e(M, dt=torch.float32))
 
 
+def _gemm_workspace(torch, lib, d, M, dev):
+    """The split-K workspace of a layer's two GEMMs at M rows (None when neither
+    splits) and the extra launches (one epilogue kernel per split GEMM)."""
+    n_in = lib.gemm_workspace_bytes(M, d.n_in, d.d_model)
+    n_out = lib.gemm_workspace_bytes(M, d.d_model, d.d_inner)
+    n = max(n_in, n_out)
+    ws = torch.empty(n, dtype=torch.uint8, device=dev) if n else None
+    return ws, int(n_in > 0) + int(n_out > 0)
+
+
 class StackWorkload:
     """Prefill of a stack (or of one bare mixer layer).  The timed step calls
     the stage entry points in the order fm_mixer_prefill composes them (checked
@@ -322,8 +332,9 @@ class StackWorkload:
         self.sws = torch.empty(nb, dtype=torch.uint8, device=dev)
         self.buf = _stage_buffers(torch, d, M, dev)
         self.tokens = M
+        self.gws, extra = _gemm_workspace(torch, lib, d, M, dev)
         # the chunked scan is three kernels where the sequential one is two
-        self.launches = (self.launches_per_layer + (1 if self.ssd else 0)) * self.n_layers
+        self.launches = (self.launches_per_layer + extra + (1 if self.ssd else 0)) * self.n_layers
 
     def states(self, i):
         return None, None
@@ -337,7 +348,7 @@ class StackWorkload:
             lib.hadamard_quant(src, d.d_model, Ly.prenorm_w, 1, self.mode, Ly.static_amax,
                                b["q_in"], b["sx_in"])
             lib.in_proj(b["q_in"], b["sx_in"], Ly.w_in_q, Ly.w_in_s, d, Ly.exps, b["z"], b["xbc"],
-                        b["dtr"])
+                        b["dtr"], ws=self.gws)
             lib.conv1d_pot(b["xbc"], B, T, d, Ly.conv_wq, Ly.conv_bq, Ly.exps, cs, b["xo"])
             if ev is not None:
                 ev[i][0].record(stream)
@@ -349,7 +360,7 @@ class StackWorkload:
             lib.gate_norm_quant(b["y"], b["z"], d, Ly.exps, Ly.norm_w, 1, self.mode,
                                 Ly.static_amax[1:], b["q_out"], b["sx_out"])
             lib.w8a8_gemm(b["q_out"], b["sx_out"], Ly.w_out_q, Ly.w_out_s, self.r,
-                          residual=src if self.stack_mode else None)
+                          residual=src if self.stack_mode else None, ws=self.gws)
             src = self.r
 
     def output(self):
@@ -450,7 +461,8 @@ class DecodeWorkload(StackWorkload):
                                device=dev)
         self.buf = _stage_buffers(torch, d, self.B, dev)
         self.tokens = self.B
-        self.launches = self.launches_per_layer * self.n_layers
+        self.gws, extra = _gemm_workspace(torch, lib, d, self.B, dev)
+        self.launches = (self.launches_per_layer + extra) * self.n_layers
 
     def states(self, i):
         return self.st[i]

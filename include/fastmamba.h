@@ -143,6 +143,22 @@ fm_status fm_in_proj(const int8_t *A, const float *s_x, int64_t M, const int8_t 
                      const float *s_w, const fm_shape *shape, const int32_t *exps, float *z,
                      int8_t *xbc, float *dt, fm_stream stream);
 
+/* Workspace variants: the same results, bit for bit.  Given a device
+ * workspace of fm_gemm_workspace_bytes(M, N, K) bytes (0 when the problem
+ * would not split), a grid with fewer output tiles than the GPU has SMs
+ * splits K across CTAs: each slice adds its exact int32 partial sums into the
+ * workspace, and one epilogue pass dequantises the totals.  The layer entry
+ * points (fm_mixer_prefill, fm_decode_step) do this from their own workspace.
+ * ws may be NULL (no split) when fm_gemm_workspace_bytes returns 0. */
+size_t fm_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
+fm_status fm_w8a8_gemm_ws(const int8_t *A, const float *s_x, int64_t M, const int8_t *Wq,
+                          const float *s_w, int64_t N, int64_t K, const float *residual,
+                          float *Y, int32_t *acc_out, void *ws, size_t ws_bytes,
+                          fm_stream stream);
+fm_status fm_in_proj_ws(const int8_t *A, const float *s_x, int64_t M, const int8_t *Wq,
+                        const float *s_w, const fm_shape *shape, const int32_t *exps, float *z,
+                        int8_t *xbc, float *dt, void *ws, size_t ws_bytes, fm_stream stream);
+
 /* ------------------------------------------------------------------ */
 /* a4: power-of-two causal depthwise conv1d (kernel 4) + SiLU           */
 /* ------------------------------------------------------------------ */

@@ -227,15 +227,54 @@ static fm_status gemm_output_maps(GemmEpilogue &ep, CUtensorMap (&tm)[3], const 
 }
 
 // ------------------------------------------------------------------ launches
+static int sm_count();
+
+// Split-K for the small-grid kernel: enough K slices that the grid reaches
+// about two CTAs per SM, every slice at least one 128-deep block.  Returns the
+// number of slices (1: no split) and the blocks per slice.
+static int gemm_splits(long long M, long long N, long long K, int BN, int sms, int *kbs) {
+  const long long base = ((M + kGemmBM - 1) / kGemmBM) * ((N + BN - 1) / BN);
+  const int nkb = (int)(K / kGemmBK);
+  long long S = (2LL * sms + base - 1) / base;
+  if (S > nkb) S = nkb;
+  if (S < 1) S = 1;
+  *kbs = (int)((nkb + S - 1) / S);
+  return (nkb + *kbs - 1) / *kbs;
+}
+// the small-grid path would split this GEMM (the workspace must hold M x N int32)
+static bool gemm_would_split(long long M, long long N, long long K) {
+  const int sms = sm_count();
+  const long long mt = (M + kGemmBM - 1) / kGemmBM;
+  if (K % kGemmBK || mt * ((N + 127) / 128) >= sms) return false;
+  const int BN = mt * ((N + 63) / 64) < sms ? 32 : 64;
+  int kbs = 0;
+  return gemm_splits(M, N, K, BN, sms, &kbs) > 1;
+}
+
 template <int BN, int STAGES>
 static fm_status launch_gemm_t(const CUtensorMap &ta, const CUtensorMap &tb, long long M,
-                               long long N, long long K, const GemmEpilogue &ep, cudaStream_t s) {
+                               long long N, long long K, GemmEpilogue ep, int32_t *split_ws,
+                               cudaStream_t s) {
   constexpr int smem = gemm_smem_bytes(BN, STAGES);
-  auto kern = k_gemm_i8_tc<BN, STAGES>;
+  const int nkb = (int)(K / kGemmBK);
+  int kbs = nkb, splits = 1;
+  if (split_ws) splits = gemm_splits(M, N, K, BN, sm_count(), &kbs);
+  auto kern = splits > 1 ? k_gemm_i8_tc<BN, STAGES, true> : k_gemm_i8_tc<BN, STAGES, false>;
   FM_CHECK_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
-  dim3 grid((unsigned)((N + BN - 1) / BN), (unsigned)((M + kGemmBM - 1) / kGemmBM));
-  kern<<<grid, kGemmThreads, smem, s>>>(ta, tb, (int)(K / kGemmBK), ep);
-  return launched("k_gemm_i8_tc");
+  if (splits > 1) {
+    ep.split_acc = split_ws;
+    FM_CHECK_CUDA(cudaMemsetAsync(split_ws, 0, sizeof(int32_t) * (size_t)(M * N), s));
+  }
+  dim3 grid((unsigned)((N + BN - 1) / BN), (unsigned)((M + kGemmBM - 1) / kGemmBM),
+            (unsigned)splits);
+  kern<<<grid, kGemmThreads, smem, s>>>(ta, tb, nkb, kbs, ep);
+  FM_TRY(launched("k_gemm_i8_tc"));
+  if (splits > 1) {
+    const long long n = M * ((N + 31) / 32);
+    k_gemm_splitk_epilogue<<<(unsigned)((n + 127) / 128), 128, 0, s>>>(ep);
+    FM_TRY(launched("k_gemm_splitk_epilogue"));
+  }
+  return FM_OK;
 }
 
 template <int BN, int STAGES, int EW>
@@ -275,8 +314,10 @@ static int sm_count() {
 // (fewer 128-wide tiles than SMs, e.g. out_proj at 130M shapes or a decode
 // batch): one 128 x 64 tile per CTA (128 x 32 when even those are fewer than
 // the SMs), two CTAs per SM.
+// split_ws (nullable, M x N int32): lets the small-grid path split K.
 static fm_status launch_gemm(const int8_t *A, long long M, const int8_t *W, long long N,
-                             long long K, const GemmEpilogue &ep, cudaStream_t s) {
+                             long long K, const GemmEpilogue &ep, cudaStream_t s,
+                             int32_t *split_ws = nullptr) {
   if (K % kGemmBK) return fail(FM_ERR_SHAPE, "gemm: K=%lld is not a multiple of 128", K);
   if ((M + kGemmBM - 1) / kGemmBM > 65535 || (N + 63) / 64 > 65535)
     return fail(FM_ERR_SHAPE, "gemm: M=%lld or N=%lld too large", M, N);
@@ -295,10 +336,10 @@ static fm_status launch_gemm(const int8_t *A, long long M, const int8_t *W, long
   }
   if (mt * ((N + 63) / 64) < sms) {  // fewer 64-wide tiles than SMs: halve the tile width
     FM_TRY(make_tmap(&tb, W, N, K, 32));
-    return launch_gemm_t<32, 6>(ta, tb, M, N, K, ep, s);
+    return launch_gemm_t<32, 6>(ta, tb, M, N, K, ep, split_ws, s);
   }
   FM_TRY(make_tmap(&tb, W, N, K, 64));
-  return launch_gemm_t<64, 4>(ta, tb, M, N, K, ep, s);
+  return launch_gemm_t<64, 4>(ta, tb, M, N, K, ep, split_ws, s);
 }
 
 static fm_status launch_hadamard_quant(const float *x, long long M, int K, const float *prenorm_w,
@@ -582,7 +623,8 @@ extern "C" fm_status fm_w8a8_gemm(const int8_t *A, const float *s_x, int64_t M, 
 
 static fm_status in_proj_impl(const int8_t *A, const float *s_x, long long M, const int8_t *Wq,
                               const float *s_w, const Dims &d, const int32_t *e_u, float *z,
-                              int8_t *xbc, float *dt, cudaStream_t s) {
+                              int8_t *xbc, float *dt, cudaStream_t s,
+                              int32_t *split_ws = nullptr) {
   GemmEpilogue ep;
   std::memset(&ep, 0, sizeof(ep));
   ep.mode = 1;
@@ -597,7 +639,7 @@ static fm_status in_proj_impl(const int8_t *A, const float *s_x, long long M, co
   ep.z = z;
   ep.xbc = xbc;
   ep.dt = dt;
-  return launch_gemm(A, M, Wq, d.n_in, d.dm, ep, s);
+  return launch_gemm(A, M, Wq, d.n_in, d.dm, ep, s, split_ws);
 }
 
 extern "C" fm_status fm_in_proj(const int8_t *A, const float *s_x, int64_t M, const int8_t *Wq,
@@ -616,6 +658,63 @@ extern "C" fm_status fm_in_proj(const int8_t *A, const float *s_x, int64_t M, co
   NEED(xbc);
   NEED(dt);
   return in_proj_impl(A, s_x, M, Wq, s_w, d, exps, z, xbc, dt, (cudaStream_t)stream);
+}
+
+extern "C" size_t fm_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  if (M <= 0 || N <= 0 || K <= 0) return 0;
+  return gemm_would_split(M, N, K) ? sizeof(int32_t) * (size_t)(M * N) : 0;
+}
+
+static fm_status gemm_ws(void *ws, size_t ws_bytes, long long M, long long N, long long K,
+                         int32_t **split, const char *fn) {
+  const size_t need = fm_gemm_workspace_bytes(M, N, K);
+  *split = nullptr;
+  if (!need) return FM_OK;
+  if (!ws || ws_bytes < need || !aligned16(ws))
+    return fail(FM_ERR_WORKSPACE, "%s: workspace needs %zu bytes", fn, need);
+  *split = reinterpret_cast<int32_t *>(ws);
+  return FM_OK;
+}
+
+extern "C" fm_status fm_w8a8_gemm_ws(const int8_t *A, const float *s_x, int64_t M,
+                                     const int8_t *Wq, const float *s_w, int64_t N, int64_t K,
+                                     const float *residual, float *Y, int32_t *acc_out, void *ws,
+                                     size_t ws_bytes, fm_stream stream) {
+  if (M < 0 || N < 0 || K <= 0 || K % 128)
+    return fail(FM_ERR_SHAPE, "fm_w8a8_gemm_ws: need M, N >= 0 and K a positive multiple of 128");
+  if (M == 0 || N == 0) return FM_OK;
+  NEED(A);
+  NEED(s_x);
+  NEED(Wq);
+  NEED(s_w);
+  NEED(Y);
+  OPT(residual);
+  OPT(acc_out);
+  int32_t *split = nullptr;
+  FM_TRY(gemm_ws(ws, ws_bytes, M, N, K, &split, __func__));
+  return launch_gemm(A, M, Wq, N, K, plain_epilogue(M, N, s_x, s_w, residual, Y, acc_out),
+                     (cudaStream_t)stream, split);
+}
+
+extern "C" fm_status fm_in_proj_ws(const int8_t *A, const float *s_x, int64_t M,
+                                   const int8_t *Wq, const float *s_w, const fm_shape *shape,
+                                   const int32_t *exps, float *z, int8_t *xbc, float *dt,
+                                   void *ws, size_t ws_bytes, fm_stream stream) {
+  Dims d;
+  FM_TRY(check_shape(shape, &d, __func__));
+  if (M < 0) return fail(FM_ERR_SHAPE, "fm_in_proj_ws: M < 0");
+  if (M == 0) return FM_OK;
+  NEED(A);
+  NEED(s_x);
+  NEED(Wq);
+  NEED(s_w);
+  NEED(exps);
+  NEED(z);
+  NEED(xbc);
+  NEED(dt);
+  int32_t *split = nullptr;
+  FM_TRY(gemm_ws(ws, ws_bytes, M, d.n_in, d.dm, &split, __func__));
+  return in_proj_impl(A, s_x, M, Wq, s_w, d, exps, z, xbc, dt, (cudaStream_t)stream, split);
 }
 
 extern "C" fm_status fm_conv1d_pot(const int8_t *u, int B, int T, const fm_shape *shape,
@@ -881,6 +980,7 @@ struct MixerWs {
   float *sx_out;
   ScanWs scan;
   SsdWs ssd;  // chunked scan mode only (null otherwise)
+  int32_t *split;  // split-K partial sums of the small-grid GEMMs (null when none split)
 };
 
 MixerWs carve_mixer(Carver &c, const Dims &d, int B, int T) {
@@ -902,6 +1002,11 @@ MixerWs carve_mixer(Carver &c, const Dims &d, int B, int T) {
     w.ssd.dH = w.ssd.achunk = nullptr;
     w.ssd.Hin = nullptr;
   }
+  const bool in_split = gemm_would_split(M, d.n_in, d.dm);
+  const bool out_split = gemm_would_split(M, d.dm, d.di);
+  const long long n = in_split ? (out_split ? (d.n_in > d.dm ? d.n_in : d.dm) : d.n_in)
+                               : (out_split ? d.dm : 0);
+  w.split = n ? c.take<int32_t>(M * n) : nullptr;
   return w;
 }
 }  // namespace
@@ -952,7 +1057,7 @@ static fm_status mixer_impl(const fm_layer *L, const Dims &d, const float *x, in
   FM_TRY(launch_hadamard_quant(x, M, d.dm, L->prenorm_w, L->rotate, L->mode, amax_in, w.q_in,
                                w.sx_in, nullptr, s));
   FM_TRY(in_proj_impl(w.q_in, w.sx_in, M, L->w_in_q, L->w_in_s, d, L->exps + X.e_u, w.z, w.xbc,
-                      w.dt, s));
+                      w.dt, s, w.split));
   FM_TRY(launch_conv(w.xbc, B, T, d.cc, L->conv_wq, L->conv_bq, L->exps, conv_state, w.xo,
                      nullptr, s));
   if (w.ssd.dH)
@@ -967,7 +1072,7 @@ static fm_status mixer_impl(const fm_layer *L, const Dims &d, const float *x, in
   return launch_gemm(w.q_out, M, L->w_out_q, d.dm, d.di,
                      plain_epilogue(M, d.dm, w.sx_out, L->w_out_s, residual ? x : nullptr, out,
                                     nullptr),
-                     s);
+                     s, w.split);
 }
 
 extern "C" fm_status fm_mixer_prefill(const fm_layer *L, const float *x, int B, int T,

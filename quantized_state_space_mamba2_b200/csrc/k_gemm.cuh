@@ -50,6 +50,10 @@ struct GemmEpilogue {
   // persistent kernel only: write the outputs through TMA stores (the tensor
   // maps passed beside this struct); 0 falls back to per-thread stores
   int tma_store;
+  // split-K (small-grid kernel, gridDim.z > 1): each K slice adds its int32
+  // partial sums into split_acc [M, N] (zeroed by the host); the dequantising
+  // epilogue then runs once on the exact total (k_gemm_splitk_epilogue)
+  int32_t *split_acc;
 };
 
 // ------------------------------------------------------------ PTX wrappers
@@ -287,10 +291,10 @@ __device__ __forceinline__ void gemm_store_chunk(const GemmEpilogue &ep, long lo
 }
 
 // ------------------------------------------------------------ the kernel
-template <int BN, int STAGES>
+template <int BN, int STAGES, bool SPLIT = false>
 __global__ void __launch_bounds__(kGemmThreads, 2)
     k_gemm_i8_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                 int num_k_blocks, GemmEpilogue ep) {
+                 int num_k_blocks, int kb_per_split, GemmEpilogue ep) {
   static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN");
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -310,6 +314,10 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
   const int lane = threadIdx.x & 31;
   const int m0 = blockIdx.y * kGemmBM;
   const int n0 = blockIdx.x * BN;
+  // this CTA's K slice (SPLIT: the host launches only non-empty slices, so
+  // kb_n >= 1; otherwise the whole K)
+  const int kb0 = SPLIT ? (int)blockIdx.z * kb_per_split : 0;
+  const int kb_n = SPLIT ? min(kb_per_split, num_k_blocks - kb0) : num_k_blocks;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -335,19 +343,19 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
 
   if (warp == 0) {
     if (lane == 0) {
-      for (int kb = 0; kb < num_k_blocks; ++kb) {
+      for (int kb = 0; kb < kb_n; ++kb) {
         const int s = kb % STAGES;
         const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
         if (!mbar_wait(&empty_bar[s], ph ^ 1u)) break;
         mbar_arrive_expect_tx(&full_bar[s], (uint32_t)((kGemmBM + BN) * kGemmBK));
-        tma_load_2d(sA + s * kGemmBM * kGemmBK, &tmA, kb * kGemmBK, m0, &full_bar[s]);
-        tma_load_2d(sB + s * BN * kGemmBK, &tmB, kb * kGemmBK, n0, &full_bar[s]);
+        tma_load_2d(sA + s * kGemmBM * kGemmBK, &tmA, (kb0 + kb) * kGemmBK, m0, &full_bar[s]);
+        tma_load_2d(sB + s * BN * kGemmBK, &tmB, (kb0 + kb) * kGemmBK, n0, &full_bar[s]);
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t idesc = i8_idesc(kGemmBM, BN);
-      for (int kb = 0; kb < num_k_blocks; ++kb) {
+      for (int kb = 0; kb < kb_n; ++kb) {
         const int s = kb % STAGES;
         const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
         if (!mbar_wait(&full_bar[s], ph)) break;
@@ -384,7 +392,15 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
     for (int c = 0; c < BN; c += 32) {
       uint32_t r[32];
       tmem_ld32(tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)c, r);
-      if (ok && n0 + c < ep.N) gemm_store_chunk(ep, row, sx, (long long)n0 + c, r, col_w + c, col_e + c);
+      if (!ok || n0 + c >= ep.N) continue;
+      if constexpr (SPLIT) {  // add this slice's exact partial sums
+        if (row < ep.M) {
+          int32_t *dst = ep.split_acc + row * ep.N + n0 + c;
+          for (int j = 0; j < 32 && n0 + c + j < ep.N; ++j) atomicAdd(dst + j, (int)r[j]);
+        }
+      } else {
+        gemm_store_chunk(ep, row, sx, (long long)n0 + c, r, col_w + c, col_e + c);
+      }
     }
   }
   tc_fence_before();
@@ -395,6 +411,30 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
                  "r"((uint32_t)BN)
                  : "memory");
   }
+}
+
+// The dequantising epilogue of a split-K GEMM: one thread per (row, 32-column
+// chunk) reads the exact int32 totals and runs the same gemm_store_chunk as
+// the unsplit kernels, so the outputs are bit-identical to theirs.
+__global__ void __launch_bounds__(128) k_gemm_splitk_epilogue(GemmEpilogue ep) {
+  const long long nchunk = (ep.N + 31) / 32;
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= ep.M * nchunk) return;
+  const long long row = i / nchunk, col0 = (i % nchunk) * 32;
+  uint32_t r[32];
+  __align__(16) float colw[32];
+  __align__(16) float cole[32];
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    const long long c = col0 + j;
+    const bool in = c < ep.N;
+    r[j] = in ? (uint32_t)ep.split_acc[row * ep.N + c] : 0u;
+    colw[j] = in ? ep.s_w[c] : 0.0f;
+    float e = 0.0f;
+    if (in && ep.mode == 1 && c >= ep.di && c < (long long)ep.di + ep.cc) e = pow2f(-ep.e_u[c - ep.di]);
+    cole[j] = e;
+  }
+  gemm_store_chunk(ep, row, ep.s_x[row], col0, r, colw, cole);
 }
 
 // ------------------------------------------------------------ the persistent kernel

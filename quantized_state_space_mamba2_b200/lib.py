@@ -24,6 +24,7 @@ STATUS = {0: "FM_OK", 1: "FM_ERR_INVALID_ARG", 2: "FM_ERR_SHAPE", 3: "FM_ERR_ALI
 EXPORTS = (
     "fm_status_string", "fm_last_error", "fm_sync_status", "fm_version", "fm_exp_table_layout",
     "fm_hadamard_quant", "fm_prepare_linear", "fm_w8a8_gemm", "fm_in_proj", "fm_conv1d_pot",
+    "fm_gemm_workspace_bytes", "fm_w8a8_gemm_ws", "fm_in_proj_ws",
     "fm_ssm_scan_pot", "fm_gate_norm_quant", "fm_eval_pwl", "fm_workspace_bytes",
     "fm_mixer_prefill", "fm_decode_step", "fm_prepare_mixer_params", "fm_calib_workspace_bytes",
     "fm_calibrate_layer", "fm_decode_step_noalloc", "fm_scan_workspace_bytes",
@@ -84,6 +85,9 @@ def load():
         "fm_prepare_linear": (I, [_P, I64, I64, I, _P, _P, _P]),
         "fm_w8a8_gemm": (I, [_P, _P, I64, _P, _P, I64, I64, _P, _P, _P, _P]),
         "fm_in_proj": (I, [_P, _P, I64, _P, _P, sp, _P, _P, _P, _P, _P]),
+        "fm_gemm_workspace_bytes": (SZ, [I64, I64, I64]),
+        "fm_w8a8_gemm_ws": (I, [_P, _P, I64, _P, _P, I64, I64, _P, _P, _P, _P, SZ, _P]),
+        "fm_in_proj_ws": (I, [_P, _P, I64, _P, _P, sp, _P, _P, _P, _P, _P, SZ, _P]),
         "fm_conv1d_pot": (I, [_P, I, I, sp, _P, _P, _P, _P, _P, _P]),
         "fm_ssm_scan_pot": (I, [_P, _P, I, I, sp, _P, _P, _P, _P, _P, _P, _P, SZ, _P]),
         "fm_scan_workspace_bytes": (SZ, [sp, I, I]),
@@ -154,17 +158,35 @@ def prepare_linear(W, rotate, Wq, s_w, stream=None):
     _check(load().fm_prepare_linear(_p(W), N, K, rotate, _p(Wq), _p(s_w), _s(stream)))
 
 
-def w8a8_gemm(A, s_x, Wq, s_w, Y, residual=None, acc_out=None, stream=None):
+def gemm_workspace_bytes(M, N, K) -> int:
+    """Bytes of workspace that let a small-grid GEMM split K (0: it would not)."""
+    return load().fm_gemm_workspace_bytes(M, N, K)
+
+
+def _nbytes(t):
+    return 0 if t is None else t.numel() * t.element_size()
+
+
+def w8a8_gemm(A, s_x, Wq, s_w, Y, residual=None, acc_out=None, stream=None, ws=None):
     M, K = A.shape
     N = Wq.shape[0]
-    _check(load().fm_w8a8_gemm(_p(A), _p(s_x), M, _p(Wq), _p(s_w), N, K, _p(residual), _p(Y),
-                               _p(acc_out), _s(stream)))
+    if ws is None:
+        _check(load().fm_w8a8_gemm(_p(A), _p(s_x), M, _p(Wq), _p(s_w), N, K, _p(residual), _p(Y),
+                                   _p(acc_out), _s(stream)))
+    else:
+        _check(load().fm_w8a8_gemm_ws(_p(A), _p(s_x), M, _p(Wq), _p(s_w), N, K, _p(residual),
+                                      _p(Y), _p(acc_out), _p(ws), _nbytes(ws), _s(stream)))
 
 
-def in_proj(A, s_x, Wq, s_w, shape, exps, z, xbc, dt, stream=None):
+def in_proj(A, s_x, Wq, s_w, shape, exps, z, xbc, dt, stream=None, ws=None):
     sh = shape_struct(shape)
-    _check(load().fm_in_proj(_p(A), _p(s_x), A.shape[0], _p(Wq), _p(s_w), C.byref(sh), _p(exps),
-                             _p(z), _p(xbc), _p(dt), _s(stream)))
+    if ws is None:
+        _check(load().fm_in_proj(_p(A), _p(s_x), A.shape[0], _p(Wq), _p(s_w), C.byref(sh),
+                                 _p(exps), _p(z), _p(xbc), _p(dt), _s(stream)))
+    else:
+        _check(load().fm_in_proj_ws(_p(A), _p(s_x), A.shape[0], _p(Wq), _p(s_w), C.byref(sh),
+                                    _p(exps), _p(z), _p(xbc), _p(dt), _p(ws), _nbytes(ws),
+                                    _s(stream)))
 
 
 def conv1d_pot(u, B, T, shape, wq, bq, exps, conv_state, out, stream=None):
