@@ -466,6 +466,7 @@ static fm_status launch_scan_v2(const ScanArgs &a, int B, const ScanWs &w, cudaS
   q.e_y = a.e_y;
   q.state = a.state;
   q.y = a.y;
+  q.k16 = 65536;
   const ScanTile t = scan_tile();
 #define FM_SEQ(N, P, C) \
   if (t.npt == N && t.pc == P && t.tch == C) return launch_seq<N, P, C>(q, B, s);
