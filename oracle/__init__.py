@@ -87,7 +87,7 @@ def _declare(L):
         "fmo_ssm_scan_pot": (None, [_P, _P, _P, _P, _P, _P, _I, _I, _P, _P, _P,
                                     _I, _I, _I, _I, _I, _P, _P, _P, _P, _P]),
         "fmo_ssm_scan_pot_x": (None, [_P, _P, _P, _P, _P, _P, _I, _I, _P, _P, _P,
-                                      _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _I, _P]),
+                                      _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _I, _P, _I]),
         "fmo_scan_state_amax": (None, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
         "fmo_scan_state_amax_x": (None, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _I]),
         "fmo_conv1d_pot_x": (None, [_P, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
@@ -256,11 +256,13 @@ def prepare_ssm(a_log, D):
 
 
 def ssm_scan_pot(xbc, dt_raw, dt_bias, A_q, D_q, e_x, e_B, e_C, e_h, e_y, e_D, hd, ds,
-                 state=None, want_dt=False, want_ystat=False, state_bits=31, e_tok=None):
+                 state=None, want_dt=False, want_ystat=False, state_bits=31, e_tok=None,
+                 ub_guard=0):
     """xbc int8 [B,T,cc] (conv output), dt_raw fp32 [B,T,nh]; state int32 [B,nh,hd,ds]
     is updated in place.  Returns y int32 [B,T,nh*hd] (+ extras).  state_bits
     is the state word's width reading (31: the method as built; 16: int16);
-    e_tok (int32 [B,T,nh+2]) gives per-token exponents of x, B, C."""
+    e_tok (int32 [B,T,nh+2]) gives per-token exponents of x, B, C; ub_guard
+    (0 as built, else guard bits) rounds the increment after the u B product."""
     xbc = _c(xbc, np.int8)
     Bsz, T, cc = xbc.shape
     nh = len(A_q)
@@ -272,6 +274,13 @@ def ssm_scan_pot(xbc, dt_raw, dt_bias, A_q, D_q, e_x, e_B, e_C, e_h, e_y, e_D, h
         assert state.dtype == np.int32 and state.flags.c_contiguous
     if not 8 <= state_bits <= 31:
         raise ValueError("state_bits must be in [8, 31]")
+    if not 0 <= ub_guard <= 7:
+        raise ValueError("ub_guard must be in [0, 7]")
+    if ub_guard and state_bits + ub_guard > 24:
+        # u keeps its 24-bit saturation (u B inside 32 bits), so with g guard
+        # bits an increment saturates at 2^(23-g) state LSBs per unit of B
+        # code: harmless only when the state word itself is no wider
+        raise ValueError("ub_guard needs state_bits + ub_guard <= 24")
     et = None if e_tok is None else _c(e_tok, np.int32)
     if et is not None:
         assert et.shape == (Bsz, T, nh + 2)
@@ -279,7 +288,7 @@ def ssm_scan_pot(xbc, dt_raw, dt_bias, A_q, D_q, e_x, e_B, e_C, e_h, e_y, e_D, h
                              _p(_c(A_q, np.int32)), _p(_c(D_q, np.int32)), _p(_c(e_x, np.int32)),
                              int(e_B), int(e_C), _p(_c(e_h, np.int32)), _p(_c(e_y, np.int32)),
                              _p(_c(e_D, np.int32)), Bsz, T, nh, hd, ds, _p(state), _p(y), _p(dtq),
-                             _p(dA), _p(ys), int(state_bits), _p(et))
+                             _p(dA), _p(ys), int(state_bits), _p(et), int(ub_guard))
     out = [y]
     if want_dt:
         out += [dtq, dA]
@@ -358,6 +367,7 @@ class Layer:
     amax_out: float = 0.0
     state_bits: int = 31    # state word width reading (31 as built; 16 the int16 reading)
     xbc_exponents: str = "static"   # conv output exponents: "static" per head, or "token"
+    ub_guard: int = 0       # 0 as built; g: the increment rounded after u B, u with g more bits
     scan_mode: str = "seq"  # "seq": the sequential fixed-point scan; "ssd": the chunked form
     ssd_chunk: int = 64
     extra: dict = field(default_factory=dict)
@@ -376,9 +386,11 @@ class Layer:
 
 
 def prepare_layer(params: dict, shape, rotate=1, mode=DYNAMIC, prenorm=False,
-                  state_bits=31, xbc_exponents="static") -> Layer:
+                  state_bits=31, xbc_exponents="static", ub_guard=0) -> Layer:
     if xbc_exponents not in ("static", "token"):
         raise ValueError("xbc_exponents is 'static' or 'token'")
+    if ub_guard and state_bits + ub_guard > 24:
+        raise ValueError("ub_guard needs state_bits + ub_guard <= 24")
     wq_in, sw_in = prepare_linear(params["w_in"], rotate)
     wq_out, sw_out = prepare_linear(params["w_out"], rotate)
     wq, _, e_w = prepare_conv(params["conv_w"], params["conv_b"])
@@ -388,7 +400,8 @@ def prepare_layer(params: dict, shape, rotate=1, mode=DYNAMIC, prenorm=False,
                  conv_w=_c(params["conv_w"], np.float32), conv_b=_c(params["conv_b"], np.float32), A_q=A_q, D_q=D_q, e_D=e_D,
                  dt_bias=_c(params["dt_bias"], np.float32), norm_w=_c(params["norm_w"], np.float32),
                  prenorm_w=_c(params["prenorm_w"], np.float32) if prenorm else None,
-                 state_bits=int(state_bits), xbc_exponents=xbc_exponents)
+                 state_bits=int(state_bits), xbc_exponents=xbc_exponents,
+                 ub_guard=int(ub_guard))
 
 
 def set_conv_input_exponents(L: Layer, e_u):
@@ -428,7 +441,7 @@ def mixer_prefill(L: Layer, x, residual=False, conv_state=None, ssm_state=None, 
     else:
         y = ssm_scan_pot(xo, dt.reshape(Bsz, T, nh), L.dt_bias, L.A_q, L.D_q, L.e_x, L.e_B,
                          L.e_C, L.e_h, L.e_y, L.e_D, hd, ds, ssm_state,
-                         state_bits=L.state_bits, e_tok=e_tok)
+                         state_bits=L.state_bits, e_tok=e_tok, ub_guard=L.ub_guard)
     q2, sx2 = gate_norm_quant(y.reshape(M, di), z, hd, L.e_y, L.e_g, L.norm_w, L.rotate, L.mode,
                               L.amax_out)
     acc2 = gemm_i8(q2, L.wq_out)
@@ -480,13 +493,13 @@ def calibrate_layer(L: Layer, xcal, residual=False):
     # output exponent from max |y| at the finer term exponent
     _, ys = ssm_scan_pot(xo, dt3, L.dt_bias, L.A_q, L.D_q, L.e_x, L.e_B, L.e_C, L.e_h,
                          np.zeros(nh, np.int32), L.e_D, hd, ds, want_ystat=True,
-                         state_bits=L.state_bits, e_tok=e_tok)
+                         state_bits=L.state_bits, e_tok=e_tok, ub_guard=L.ub_guard)
     e_f = np.minimum(L.e_C + L.e_h, L.e_D + L.e_x)
     lo = np.maximum(L.e_C + L.e_h, L.e_D + L.e_x) - 16
     L.e_y = np.array([max(pot_exponent(float(ys[h]), 2.0 ** 29) + int(e_f[h]), int(lo[h]))
                       for h in range(nh)], np.int32)
     y = ssm_scan_pot(xo, dt3, L.dt_bias, L.A_q, L.D_q, L.e_x, L.e_B, L.e_C, L.e_h, L.e_y, L.e_D,
-                     hd, ds, state_bits=L.state_bits, e_tok=e_tok)
+                     hd, ds, state_bits=L.state_bits, e_tok=e_tok, ub_guard=L.ub_guard)
     # gate exponent (int16 g), then the out_proj input amax
     # (the statistic does not depend on e_g; the pass uses its lower bound so
     # that every gate shift is a right shift)

@@ -532,13 +532,18 @@ static void dt_dA(float dt_raw, float dt_bias, int32_t A_q, int64_t *dt_q, int64
  * the narrower int16 reading (the pages fix no width).
  * e_tok (nullable, [B*T, nh+2]): per-token exponents of x (per head), B and C
  * replacing e_x, e_B, e_C in s_h, s_y, s_D; ystat then still measures at the
- * finer of e_C + e_h and e_D + e_x with the static e_x, e_C given. */
+ * finer of e_C + e_h and e_D + e_x with the static e_x, e_C given.
+ * ub_guard: where the state increment is rounded.  0 (as built): u is rounded
+ * to the state's grid per unit of B code, then multiplied, u B.  g > 0: u
+ * keeps g more bits, ug = satb(rshr(dt_q x, s_h - g), 24), and the product is
+ * rounded once more, rshr(ug B, g) -- within about one state LSB of rounding
+ * dt x B exactly, however large B's codes, and inside 32 bits for g <= 7. */
 void fmo_ssm_scan_pot_x(const int8_t *xbc, const float *dt_raw, const float *dt_bias,
                         const int32_t *A_q, const int32_t *D_q, const int32_t *e_x, int e_B,
                         int e_C, const int32_t *e_h, const int32_t *e_y, const int32_t *e_D,
                         int B, int T, int nh, int hd, int ds, int32_t *state, int32_t *y,
                         int32_t *dtq_out, int32_t *dA_out, int64_t *ystat, int hbits,
-                        const int32_t *e_tok)
+                        const int32_t *e_tok, int ub_guard)
 {
     const int64_t H_LIM = ((int64_t)1 << (hbits - 1)) - 1;
     int cc = nh * hd + 2 * ds;
@@ -562,12 +567,12 @@ void fmo_ssm_scan_pot_x(const int8_t *xbc, const float *dt_raw, const float *dt_
                 const int8_t *row = xbc + bt * cc;
                 for (int p = 0; p < hd; ++p) {
                     int64_t xq = row[h * hd + p];
-                    int64_t u = fmo_sat(fmo_rshr(dtq * xq, s_h), U_BITS);
+                    int64_t u = fmo_sat(fmo_rshr(dtq * xq, s_h - ub_guard), U_BITS);
                     int64_t acc = 0;
                     for (int n = 0; n < ds; ++n) {
                         int64_t Bn = row[nh * hd + n];
                         int64_t Cn = row[nh * hd + ds + n];
-                        int64_t hn = fmo_rshr(dA * S[p * ds + n], 16) + u * Bn;
+                        int64_t hn = fmo_rshr(dA * S[p * ds + n], 16) + fmo_rshr(u * Bn, ub_guard);
                         hn = hn > H_LIM ? H_LIM : (hn < -H_LIM ? -H_LIM : hn);
                         S[p * ds + n] = hn;
                         acc += Cn * hn;
@@ -597,7 +602,7 @@ void fmo_ssm_scan_pot(const int8_t *xbc, const float *dt_raw, const float *dt_bi
                       int32_t *dtq_out, int32_t *dA_out, int64_t *ystat)
 {
     fmo_ssm_scan_pot_x(xbc, dt_raw, dt_bias, A_q, D_q, e_x, e_B, e_C, e_h, e_y, e_D, B, T, nh, hd,
-                       ds, state, y, dtq_out, dA_out, ystat, H_BITS, NULL);
+                       ds, state, y, dtq_out, dA_out, ystat, H_BITS, NULL, 0);
 }
 
 /* Calibration statistic of the state: the same recurrence at the finest

@@ -180,23 +180,27 @@ def readings_rows(T: int = 256):
                       outlier_seed=OUTLIER_SEED)
     ref = O.ref_mixer_f64(P, shape, x)
     rows = []
-    for xe, bits in (("static", 31), ("token", 31), ("static", 16), ("token", 16)):
+    for xe, bits, g in (("static", 31, 0), ("token", 31, 0), ("static", 16, 0), ("token", 16, 0),
+                        ("static", 16, 7), ("token", 16, 7)):
         vals = []
         for mode in (O.DYNAMIC, O.STATIC):
-            L = O.prepare_layer(P, shape, mode=mode, state_bits=bits, xbc_exponents=xe)
+            L = O.prepare_layer(P, shape, mode=mode, state_bits=bits, xbc_exponents=xe,
+                                ub_guard=g)
             O.calibrate_layer(L, xc)
             vals.append(O.sqnr_db(ref, O.mixer_prefill(L, x)))
-        rows.append((xe, bits, vals))
+        rows.append((xe, bits, g, vals))
     return rows
 
 
 def print_readings_table():
-    print("| conv-output exponents | state word | SQNR, dynamic (dB) | SQNR, static (dB) |")
-    print("|---|---|---|---|")
-    for xe, bits, v in readings_rows():
+    print("| conv-output exponents | state word | increment rounded | SQNR, dynamic (dB) | "
+          "SQNR, static (dB) |")
+    print("|---|---|---|---|---|")
+    for xe, bits, g, v in readings_rows():
         name = "static per head" if xe == "static" else "per token"
-        tag = " (as built)" if (xe, bits) == ("static", 31) else ""
-        print(f"| {name}{tag} | {bits} bits | {v[0]:.2f} | {v[1]:.2f} |")
+        tag = " (as built)" if (xe, bits, g) == ("static", 31, 0) else ""
+        rnd = "u, then u B" if g == 0 else f"after u B ({g} guard bits)"
+        print(f"| {name}{tag} | {bits} bits | {rnd} | {v[0]:.2f} | {v[1]:.2f} |")
 
 
 def ssd_rows(T: int = 256):

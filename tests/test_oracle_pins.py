@@ -699,3 +699,34 @@ def test_per_token_layer_chunking_and_gain(oracle):
     gain = oracle.sqnr_db(ref, oracle.mixer_prefill(Ls["token"], xt)) - \
         oracle.sqnr_db(ref, oracle.mixer_prefill(Ls["static"], xt))
     assert gain > 0.5, gain
+
+
+def test_guard_bit_rounding_tightens_the_narrow_state_budget(oracle):
+    """Rounding the state increment after the u B product (7 guard bits on u)
+    bounds each step's rounding by about one state LSB (decay 1/2, u 2^-8 per
+    unit of |B| <= 127, product 1/2), against |B|/2 LSBs when u is rounded
+    first: a 16-bit state then tracks the fp64 recurrence within 1.6 LSB per
+    step, which the as-built rounding exceeds on the same input."""
+    Bsz, T, nh, hd, ds = 1, 48, 2, 8, 16
+    xbc, dt_raw, dt_bias, A_q, D_q, e_D, e_x = _scan_inputs(Bsz, T, nh, hd, ds, seed=50)
+    e_B = e_C = -5
+    e_h = np.full(nh, -10, np.int32)
+    X = xbc[..., :nh * hd].reshape(Bsz, T, nh, hd) * 2.0 ** -5
+    Bm = xbc[..., nh * hd:nh * hd + ds] * 2.0 ** e_B
+    lsb = 2.0 ** e_h[0]
+    err = {}
+    for g in (0, 7):
+        st = np.zeros((Bsz, nh, hd, ds), np.int32)
+        _, dtq, dA = oracle.ssm_scan_pot(xbc, dt_raw, dt_bias, A_q, D_q, e_x, e_B, e_C, e_h,
+                                         np.full(nh, -6, np.int32), e_D, hd, ds, state=st,
+                                         want_dt=True, state_bits=16, ub_guard=g)
+        h = np.zeros((Bsz, nh, hd, ds))
+        for t in range(T):
+            h = (dA[:, t] / 65536.0)[:, :, None, None] * h + \
+                (dtq[:, t, :, None] / 65536.0 * X[:, t])[..., None] * Bm[:, t, None, None, :]
+        err[g] = np.max(np.abs(st * lsb - h)) / lsb
+    assert err[7] <= T * 1.6
+    assert err[0] > T * 1.6                      # the pin tells the two roundings apart
+    with pytest.raises(ValueError):
+        oracle.ssm_scan_pot(xbc, dt_raw, dt_bias, A_q, D_q, e_x, e_B, e_C, e_h,
+                            np.full(nh, -6, np.int32), e_D, hd, ds, state_bits=31, ub_guard=7)
