@@ -14,6 +14,7 @@ the GPU path's.  Runs on the CPU in about a quarter of an hour:
     python -m oracle.sqnr_report --state-bits # width of the SSM state word
     python -m oracle.sqnr_report --readings   # conv-output exponents x state width
     python -m oracle.sqnr_report --ssd        # the chunked (tensor-core form) scan mode
+    python -m oracle.sqnr_report --2p7b       # one 2.7B-shaped layer (about half an hour)
 
 The attribution (``oracle.stages``) quantises the stages of one layer alone
 and cumulatively, in pipeline order; its first row is FastMamba-LQ, the
@@ -232,7 +233,40 @@ def print_ssd_table():
         print(f"| {name} | {v[0]:.2f} | {v[1]:.2f} |")
 
 
+def rows_2p7b(T: int = 256, n_cal: int = 4):
+    """One 2.7B-shaped layer (d_model 2560, 80 heads), 8 outlier channels x50,
+    dynamic scales, calibrated on n_cal seeded sequences of T tokens (fewer
+    than the 16 of the 130M tables: the oracle's 2.7B calibration takes
+    minutes per sequence): the method with and without the rotation, and the
+    candidate spec (per-token exponents, 16-bit state, guard-bit increment)."""
+    shape = S.MAMBA2_2P7B
+    P = S.layer_params(shape, 1000)
+    xc = S.calibration_batch(shape.d_model, T, 8, 50.0, OUTLIER_SEED, n_seqs=n_cal)
+    x = S.activations(1, T, shape.d_model, seed=1, n_outliers=8, outlier_scale=50.0,
+                      outlier_seed=OUTLIER_SEED)
+    ref = O.ref_mixer_f64(P, shape, x)
+    rows = []
+    for name, kw in (("the method, rotated (as built)", dict(rotate=1)),
+                     ("the method, not rotated", dict(rotate=0)),
+                     ("rotated, per-token exponents, 16-bit state, guard bits",
+                      dict(rotate=1, state_bits=16, xbc_exponents="token", ub_guard=7))):
+        L = O.prepare_layer(P, shape, **kw)
+        O.calibrate_layer(L, xc)
+        rows.append((name, O.sqnr_db(ref, O.mixer_prefill(L, x))))
+    return rows
+
+
+def print_2p7b_table():
+    print("| 2.7B-shaped layer, dynamic scales | SQNR (dB) |")
+    print("|---|---|")
+    for name, v in rows_2p7b():
+        print(f"| {name} | {v:.2f} |", flush=True)
+
+
 def main():
+    if "--2p7b" in sys.argv[1:]:
+        print_2p7b_table()
+        return
     if "--ssd" in sys.argv[1:]:
         print_ssd_table()
         return

@@ -730,3 +730,32 @@ def test_guard_bit_rounding_tightens_the_narrow_state_budget(oracle):
     with pytest.raises(ValueError):
         oracle.ssm_scan_pot(xbc, dt_raw, dt_bias, A_q, D_q, e_x, e_B, e_C, e_h,
                             np.full(nh, -6, np.int32), e_D, hd, ds, state_bits=31, ub_guard=7)
+
+
+def test_candidate_spec_layer_chunking_and_gain(oracle):
+    """Per-token conv-output exponents, a 16-bit state and the guard-bit
+    increment together: chunked prefill plus decode steps equal one prefill
+    bit for bit, the carried state stays inside 16 bits, and on outlier
+    inputs the layer is closer to fp64 than the method as built."""
+    P = S.layer_params(SMALL, 3)
+    xc = S.calibration_batch(256, 64, 4, 50.0, outlier_seed=99, n_seqs=2)
+    built = oracle.prepare_layer(P, SMALL)
+    oracle.calibrate_layer(built, xc)
+    L = oracle.prepare_layer(P, SMALL, state_bits=16, xbc_exponents="token", ub_guard=7)
+    oracle.calibrate_layer(L, xc)
+    s = SMALL
+    x = S.activations(2, 12, 256, seed=16, n_outliers=4, outlier_scale=50.0, outlier_seed=99)
+    cs0 = np.zeros((2, 3, s.conv_ch), np.int8)
+    ss0 = np.zeros((2, s.nheads, s.headdim, s.d_state), np.int32)
+    full = oracle.mixer_prefill(L, x, conv_state=cs0, ssm_state=ss0)
+    cs, ss = np.zeros_like(cs0), np.zeros_like(ss0)
+    parts = [oracle.mixer_prefill(L, x[:, :9].copy(), conv_state=cs, ssm_state=ss)]
+    for t in range(9, 12):
+        parts.append(oracle.mixer_prefill(L, x[:, t:t + 1].copy(), conv_state=cs, ssm_state=ss))
+    assert np.array_equal(np.concatenate(parts, 1), full)
+    assert np.array_equal(ss, ss0) and np.abs(ss0).max() <= 2 ** 15 - 1
+    xt = S.activations(1, 64, 256, seed=5, n_outliers=4, outlier_scale=50.0, outlier_seed=99)
+    ref = oracle.ref_mixer_f64(P, SMALL, xt)
+    gain = oracle.sqnr_db(ref, oracle.mixer_prefill(L, xt)) - \
+        oracle.sqnr_db(ref, oracle.mixer_prefill(built, xt))
+    assert gain > 0.5, gain
