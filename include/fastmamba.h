@@ -316,14 +316,17 @@ fm_status fm_decode_step(const fm_layer *L, const float *x, int B, int residual,
  *   - Batches whose workspace (fm_workspace_bytes(shape, B, 1)) exceeds
  *     FM_NOALLOC_SCRATCH_BYTES are rejected with FM_ERR_WORKSPACE before
  *     any launch.
- *   - The first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress, with that device current); make that first call
- *     before any stream capture.
+ *   - The first call in a CUDA context looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current) and caches it under
+ *     the context's unique id; make that first call before any stream
+ *     capture.  After cudaDeviceReset the next call runs in a new context,
+ *     so it looks the address up again (and is again a first call).
  *   - Every call on a device shares the one array and leaves the last
- *     call's intermediates in it; nothing in it needs to start at zero (each
- *     intermediate is written before it is read).  Calls that overlap on
- *     the GPU (different streams, or different host threads) race on the
- *     array: serialise them. */
+ *     call's intermediates in it.  What must start at zero (the split-K
+ *     partial sums of a small-batch GEMM) is cleared by the call itself on
+ *     its stream; everything else is written before it is read.  Calls that
+ *     overlap on the GPU (different streams, or different host threads)
+ *     race on the array: serialise them. */
 #define FM_NOALLOC_SCRATCH_BYTES (16u << 20)
 fm_status fm_decode_step_noalloc(const fm_layer *L, const float *x, int B, int residual,
                                  int8_t *conv_state, int32_t *ssm_state, float *out,

@@ -537,6 +537,7 @@ static fm_status launch_scan_v2(const ScanArgs &a, int B, const ScanWs &w, cudaS
   q.e_y = a.e_y;
   q.state = a.state;
   q.y = a.y;
+  q.k16 = 65536;
   const ScanTile t = scan_tile();
 #define FM_SEQ(N, P, C)                                      \
   if (t.npt == N && t.pc == P && t.tch == C)                 \
@@ -847,6 +848,9 @@ extern "C" fm_status fm_ssd_scan(const int8_t *xbc, const float *dt_raw, int B, 
   NEED(y);
   OPT(state);
   if (d.cc % 16) return fail(FM_ERR_ALIGNMENT, "fm_ssd_scan: conv channels must be a multiple of 16");
+  if (state16())
+    return fail(FM_ERR_UNSUPPORTED, "fm_ssd_scan: the chunked scan carries the int32 state word; "
+                "the 16-bit state spec is not supported in this mode");
   const size_t need = fm_ssd_workspace_bytes(shape, B, T);
   if (!ws || ws_bytes < need || !aligned16(ws))
     return fail(FM_ERR_WORKSPACE, "fm_ssd_scan: workspace needs %zu bytes", need);
@@ -1060,6 +1064,8 @@ static fm_status mixer_impl(const fm_layer *L, const Dims &d, const float *x, in
                       w.dt, s, w.split));
   FM_TRY(launch_conv(w.xbc, B, T, d.cc, L->conv_wq, L->conv_bq, L->exps, conv_state, w.xo,
                      nullptr, s));
+  if (w.ssd.dH && state16())
+    return fail(FM_ERR_UNSUPPORTED, "chunked scan mode with the 16-bit state spec is not supported");
   if (w.ssd.dH)
     FM_TRY(launch_ssd(d, w.xo, w.dt, B, T, L->dt_bias, L->A_q, L->D_q, L->exps, X, ssm_state, w.y,
                       w.ssd, s));
@@ -1114,27 +1120,67 @@ extern "C" fm_status fm_decode_step(const fm_layer *L, const float *x, int B, in
 // Scratch for fm_decode_step_noalloc: a fixed device array instead of a
 // caller workspace, for callers that cannot allocate device memory.  Host
 // code only sees a stand-in for this symbol; its device address comes from
-// cudaGetSymbolAddress, once per device, with that device current.
+// cudaGetSymbolAddress, with the device current.
 static __device__ __align__(256) uint8_t g_noalloc_scratch[FM_NOALLOC_SCRATCH_BYTES];
 
+// The address is looked up once per CUDA context and cached under the
+// context's unique id (cuCtxGetId).  A context torn down and created again
+// (cudaDeviceReset, then the next call) has a new id, so the module's new
+// address is looked up again instead of reusing a stale one.  Without the
+// driver's context ids the address is looked up on every call.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long *);
+
+static bool current_context_id(unsigned long long *id) {
+  static CtxGetCurrentFn get_cur = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_cur = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  CUcontext ctx = nullptr;
+  if (!get_cur || !get_id || get_cur(&ctx) != CUDA_SUCCESS || !ctx) return false;
+  return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
 static fm_status noalloc_scratch_ptr(void **out) {
-  constexpr int kMaxDevices = 64;
-  static void *cache[kMaxDevices] = {nullptr};
+  constexpr int kSlots = 64;
+  static unsigned long long ids[kSlots] = {0};
+  static void *addrs[kSlots] = {nullptr};
+  static int next = 0;
   static std::mutex mu;
   int devid = 0;
   FM_CHECK_CUDA(cudaGetDevice(&devid));
-  if (devid < 0 || devid >= kMaxDevices)
-    return fail(FM_ERR_UNSUPPORTED, "fm_decode_step_noalloc: device id %d out of range", devid);
+  // no current context yet (nothing has touched the device): no id, so the
+  // lookup below runs, and it makes the primary context current
+  unsigned long long id = 0;
+  const bool have_id = current_context_id(&id) && id != 0;
   std::lock_guard<std::mutex> lock(mu);
-  if (!cache[devid]) {
-    void *p = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess || !p)
-      return fail(FM_ERR_CUDA, "fm_decode_step_noalloc: cudaGetSymbolAddress: %s",
-                  cudaGetErrorString(e));
-    cache[devid] = p;
+  if (have_id)
+    for (int i = 0; i < kSlots; ++i)
+      if (ids[i] == id && addrs[i]) {
+        *out = addrs[i];
+        return FM_OK;
+      }
+  void *p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+  if (e != cudaSuccess || !p)
+    return fail(FM_ERR_CUDA, "fm_decode_step_noalloc: cudaGetSymbolAddress on device %d: %s",
+                devid, cudaGetErrorString(e));
+  if (have_id) {
+    ids[next] = id;
+    addrs[next] = p;
+    next = (next + 1) % kSlots;
   }
-  *out = cache[devid];
+  *out = p;
   return FM_OK;
 }
 
