@@ -410,7 +410,8 @@ def test_layer_sqnr_and_rotation(oracle, small_layers):
     ref = oracle.ref_mixer_f64(P, SMALL, x)
     s_rot = oracle.sqnr_db(ref, oracle.mixer_prefill(Ls[1], x))
     s_plain = oracle.sqnr_db(ref, oracle.mixer_prefill(Ls[0], x))
-    assert s_rot > 12.0
+    # measured 20.6 dB rotated, 18.6 dB not: the floor sits 1.6 dB below
+    assert s_rot > 19.0
     assert s_rot > s_plain
 
 
@@ -522,6 +523,75 @@ def test_gate_statistic_closed_form(oracle):
     z16 = np.rint(z.astype(np.float64) * 65536.0).astype(np.int64)
     g = np.abs(y.astype(np.int64) * z16).reshape(M, nh, hd)
     assert np.array_equal(gs, g.max(axis=(0, 2)))
+
+
+def _gated_norm_case(M=6, nh=3, hd=64, seed=53):
+    """Inputs on which the gate and the int16 gated code are exact: z = 64
+    exactly, so z16 = 2^22, e^-z is below the 2^v unit's smallest step and
+    the PWL SiLU returns z16 unchanged; with e_g = e_y + 6 the gated code is
+    rshr(y 2^22, 22) = y.  The gated value is then y 2^e_y times z, exactly.
+    Rows 0-2 are large (the norm is a plain RMS); rows 3-5 are scaled so that
+    mean(g^2) is near or below eps = 1e-5 (eps then sets the scale)."""
+    di = nh * hd
+    y = S.uniform_ints((M, di), -30000, 30000, seed=seed)
+    y[3:5] //= 256                                 # mean(g^2) near eps in rows 3, 4
+    y[5] //= 2048                                  # and well below it in row 5
+    z = np.full((M, di), 64.0, np.float32)
+    e_y = np.full(nh, -20, np.int32)
+    e_g = -14
+    w = (0.5 + 1.5 * S.uniform_ints(di, 0, 1000, seed=seed + 1) / 1000.0).astype(np.float32)
+    g = y.astype(np.float64) * 2.0 ** -20 * 64.0   # the gated value, exact
+    return y, z, hd, e_y, e_g, w, g
+
+
+def _gated_norm_f64(g, w, eps=1e-5):
+    """Mamba2's gated RMSNorm (gate first, then normalise over all of d_inner
+    with one group), the paper's reference [10] (RMSNorm) and its Figure 2
+    block flow, in fp64."""
+    return g / np.sqrt((g * g).mean(axis=1, keepdims=True) + eps) * w.astype(np.float64)
+
+
+def test_gated_rmsnorm_closed_form(oracle):
+    """The gate + gated RMSNorm against its fp64 definition, on inputs where
+    the gate is exact (_gated_norm_case): the norm uses eps = 1e-5, the
+    per-channel weight, and the mean over d_inner.  Without rotation the
+    dequantised output is within half a quantisation step of the fp64 value
+    (plus fp32 rounding); the rows where eps dominates pin eps itself."""
+    y, z, hd, e_y, e_g, w, g = _gated_norm_case()
+    o = _gated_norm_f64(g, w)
+    ms = (g * g).mean(axis=1)
+    assert ms[0] > 1e3 * 1e-5 and ms[5] < 1e-5 < 1e3 * ms[5]
+    for mode, amax in ((oracle.DYNAMIC, 0.0), (oracle.STATIC, 1.25 * np.abs(o).max())):
+        q, sx = oracle.gate_norm_quant(y, z, hd, e_y, e_g, w, rotate=0, mode=mode,
+                                       static_amax=amax)
+        deq = q.astype(np.float64) * sx.astype(np.float64)[:, None] if mode == oracle.DYNAMIC \
+            else q.astype(np.float64) * float(sx[0])
+        step = sx.astype(np.float64)[:, None] if mode == oracle.DYNAMIC else float(sx[0])
+        err = np.abs(deq - o)
+        assert (err <= 0.5 * step + 1e-6 * np.abs(o) + 1e-30).all()
+        if mode == oracle.DYNAMIC:              # the row maximum maps to 127
+            assert (np.abs(q).max(axis=1) == 127).all()
+    # other eps, dropped weights, a mean over a part of d_inner: each is off
+    q, sx = oracle.gate_norm_quant(y, z, hd, e_y, e_g, w, rotate=0)
+    deq = q.astype(np.float64) * sx.astype(np.float64)[:, None]
+    for wrong in (_gated_norm_f64(g, w, eps=1e-3), _gated_norm_f64(g, np.ones_like(w)),
+                  g / np.sqrt((g[:, :hd] ** 2).mean(axis=1, keepdims=True) + 1e-5) * w):
+        assert not (np.abs(deq - wrong) <= 0.5 * sx[:, None] + 1e-6 * np.abs(wrong)).all()
+
+
+def test_gated_rmsnorm_rotated_closed_form(oracle):
+    """With the rotation on, the codes dequantise to the rotated fp64 output
+    o H (block 256) within half a step, so inverting the (orthonormal)
+    rotation gives o back within the step's L2 bound."""
+    y, z, hd, e_y, e_g, w, g = _gated_norm_case(nh=4)
+    o = _gated_norm_f64(g, w)
+    di = o.shape[1]
+    H = hadamard_bd(di)
+    q, sx = oracle.gate_norm_quant(y, z, hd, e_y, e_g, w, rotate=1)
+    deq = q.astype(np.float64) * sx.astype(np.float64)[:, None]
+    assert (np.abs(deq - o @ H) <= 0.5 * sx[:, None] + 1e-6 * np.abs(o @ H).max()).all()
+    back = deq @ H.T
+    assert (np.linalg.norm(back - o, axis=1) <= 0.5 * sx * np.sqrt(di) * (1 + 1e-6)).all()
 
 
 # ------------------------------------------------------------------ state word width
