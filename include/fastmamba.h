@@ -332,6 +332,59 @@ fm_status fm_decode_step_noalloc(const fm_layer *L, const float *x, int B, int r
                                  int8_t *conv_state, int32_t *ssm_state, float *out,
                                  fm_stream stream);
 
+/* ------------------------------------------------------------------ */
+/* FastMamba-LQ: W8A8 linears, exact fp32 conv, scan and gate            */
+/* ------------------------------------------------------------------ */
+/* The variant that quantises only the linear layers, which FastMamba's
+ * Table II reports beside the full method (pith.science review of
+ * arXiv 2505.18975, Desk Editor's Note: "FastMamba-LQ").  The two linears
+ * are the method's (rotation, int8, the same GEMM kernels and scales); the
+ * conv1d + SiLU, SoftPlus, exp, the selective scan and the gate are Mamba2's
+ * own fp32 arithmetic (the paper's reference [2]; Figure 2 caption), with
+ * CUDA's expf / log1pf and no power-of-two codes or PWL unit.
+ * The fp32 parameters it needs beyond an fm_layer: */
+typedef struct fm_lq_params {
+    const float *conv_w;  /* [conv_ch, 4], tap 3 multiplies the current token */
+    const float *conv_b;  /* [conv_ch] */
+    const float *a_log;   /* [nheads]: A = -exp(a_log) */
+    const float *D;       /* [nheads] */
+} fm_lq_params;
+
+/* Causal depthwise conv + SiLU in fp32:
+ *   out[b,t,c] = SiLU(conv_b[c] + sum_k conv_w[c,k] u[b,t-3+k,c]).
+ *   u: rows of stride ldu floats (>= conv_ch; the in_proj output's xBC
+ *   columns can be read in place, u = Y + d_inner, ldu = n_in), no alignment
+ *   requirement.  out [B, T, conv_ch].  conv_state [B, 3, conv_ch] fp32 or
+ *   NULL: the 3 inputs before token 0 (oldest first), replaced by the last 3. */
+fm_status fm_lq_conv1d(const float *u, int64_t ldu, int B, int T, const fm_shape *shape,
+                       const float *conv_w, const float *conv_b, float *conv_state, float *out,
+                       fm_stream stream);
+
+/* Selective scan in fp32 (Mamba2's recurrence, one group):
+ *   dt = SoftPlus(dt_raw[b,t,h] + dt_bias[h]), dA = exp(-dt exp(a_log[h]))
+ *   h[p,n] = dA h[p,n] + (dt x[p]) B[n];  y[p] = sum_n C[n] h[p,n] + D[h] x[p]
+ *   out = y SiLU(z) when z is given (the gate), else y.
+ *   xo [B, T, conv_ch] fp32 conv output (x | B | C); dt_raw rows of stride
+ *   ld_dt (column h), z rows of stride ld_z (NULL: no gate); out [B, T, d_inner].
+ *   state [B, nheads, 64, 128] fp32 or NULL (zeros): initial in, final out. */
+fm_status fm_lq_scan(const float *xo, const float *dt_raw, int64_t ld_dt, const float *z,
+                     int64_t ld_z, int B, int T, const fm_shape *shape, const float *dt_bias,
+                     const float *a_log, const float *D, float *state, float *out,
+                     fm_stream stream);
+
+/* One LQ layer: fm_hadamard_quant (with L->prenorm_w) -> in_proj GEMM (fp32
+ * output) -> fm_lq_conv1d -> fm_lq_scan with the gate -> gated RMSNorm
+ * (eps 1e-5, L->norm_w) + rotation + int8 (fm_hadamard_quant with norm_w as
+ * its pre-norm weight) -> out_proj GEMM (+ x when residual).  L supplies the
+ * linears, dt_bias, norm weights, mode and static scales; its fixed-point
+ * fields are not used.  conv_state [B, 3, conv_ch] fp32 and ssm_state
+ * [B, nheads, 64, 128] fp32 may be NULL (zero history, not kept).  ws: device
+ * workspace of fm_lq_workspace_bytes(shape, B, T). */
+size_t fm_lq_workspace_bytes(const fm_shape *shape, int B, int T);
+fm_status fm_lq_mixer_prefill(const fm_layer *L, const fm_lq_params *P, const float *x, int B,
+                              int T, int residual, float *conv_state, float *ssm_state,
+                              float *out, void *ws, size_t ws_bytes, fm_stream stream);
+
 /* Offline, per layer: quantise conv taps (e_w, wq) and the SSM parameters
  * (A_q, D_q, e_D) from fp32 device tensors: conv_w [cc, 4], a_log [nh], D [nh].
  * Writes the e_w and e_D regions of `exps`. */

@@ -25,6 +25,7 @@
 #include "k_scan.cuh"
 #include "k_scan2.cuh"
 #include "k_ssd.cuh"
+#include "k_lq.cuh"
 
 using namespace fm;
 
@@ -1202,6 +1203,177 @@ extern "C" fm_status fm_decode_step_noalloc(const fm_layer *L, const float *x, i
   void *ws = nullptr;
   FM_TRY(noalloc_scratch_ptr(&ws));
   return fm_decode_step(L, x, B, residual, conv_state, ssm_state, out, ws, need, stream);
+}
+
+// ------------------------------------------------------------------ FastMamba-LQ
+static fm_status lq_check_params(const fm_lq_params *P, const char *fn) {
+  if (!P) return fail(FM_ERR_INVALID_ARG, "%s: params is null", fn);
+  const void *req[] = {P->conv_w, P->conv_b, P->a_log, P->D};
+  for (const void *p : req) {
+    if (!p) return fail(FM_ERR_INVALID_ARG, "%s: a required LQ parameter pointer is null", fn);
+    if (!aligned16(p)) return fail(FM_ERR_ALIGNMENT, "%s: an LQ parameter pointer is misaligned", fn);
+  }
+  return FM_OK;
+}
+
+static fm_status launch_lq_conv(const float *u, long long ldu, int B, int T, int cc,
+                                const float *w, const float *bias, float *conv_state, float *out,
+                                cudaStream_t s) {
+  const dim3 grid((unsigned)((T + kLqConvTT - 1) / kLqConvTT), (unsigned)((cc + 255) / 256),
+                  (unsigned)B);
+  k_lq_conv<<<grid, 256, 0, s>>>(u, ldu, T, cc, w, bias, conv_state, out);
+  FM_TRY(launched("k_lq_conv"));
+  if (conv_state) {
+    const long long n = (long long)B * cc;
+    k_lq_conv_state_update<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(u, ldu, B, T, cc,
+                                                                        conv_state);
+    FM_TRY(launched("k_lq_conv_state_update"));
+  }
+  return FM_OK;
+}
+
+static fm_status launch_lq_scan(const Dims &d, const float *xo, const float *dt_raw,
+                                long long ld_dt, const float *z, long long ld_z, int B, int T,
+                                const float *dt_bias, const float *a_log, const float *D,
+                                float *state, float *out, cudaStream_t s) {
+  // 4 channels per warp once there are enough CTAs to fill the GPU, else 2
+  if ((long long)B * d.nh * (d.hd / 16) >= 2LL * 148) {
+    k_lq_scan<4><<<dim3((unsigned)(d.hd / 16), (unsigned)d.nh, (unsigned)B), 128, 0, s>>>(
+        xo, dt_raw, ld_dt, z, ld_z, T, d.nh, d.cc, d.di, dt_bias, a_log, D, state, out);
+  } else {
+    k_lq_scan<2><<<dim3((unsigned)(d.hd / 8), (unsigned)d.nh, (unsigned)B), 128, 0, s>>>(
+        xo, dt_raw, ld_dt, z, ld_z, T, d.nh, d.cc, d.di, dt_bias, a_log, D, state, out);
+  }
+  return launched("k_lq_scan");
+}
+
+extern "C" fm_status fm_lq_conv1d(const float *u, int64_t ldu, int B, int T,
+                                  const fm_shape *shape, const float *conv_w,
+                                  const float *conv_b, float *conv_state, float *out,
+                                  fm_stream stream) {
+  Dims d;
+  FM_TRY(check_shape(shape, &d, __func__));
+  if (B < 0 || T < 0) return fail(FM_ERR_SHAPE, "fm_lq_conv1d: B, T must be >= 0");
+  if ((long long)B * T == 0) return FM_OK;
+  if (B > 65535) return fail(FM_ERR_SHAPE, "fm_lq_conv1d: B=%d exceeds 65535", B);
+  if (ldu < d.cc) return fail(FM_ERR_SHAPE, "fm_lq_conv1d: ldu %lld < conv channels %d",
+                              (long long)ldu, d.cc);
+  if (!u) return fail(FM_ERR_INVALID_ARG, "fm_lq_conv1d: u is null");
+  NEED(conv_w);
+  NEED(conv_b);
+  NEED(out);
+  OPT(conv_state);
+  return launch_lq_conv(u, ldu, B, T, d.cc, conv_w, conv_b, conv_state, out,
+                        (cudaStream_t)stream);
+}
+
+extern "C" fm_status fm_lq_scan(const float *xo, const float *dt_raw, int64_t ld_dt,
+                                const float *z, int64_t ld_z, int B, int T,
+                                const fm_shape *shape, const float *dt_bias, const float *a_log,
+                                const float *D, float *state, float *out, fm_stream stream) {
+  Dims d;
+  FM_TRY(check_shape(shape, &d, __func__));
+  if (B < 0 || T < 0) return fail(FM_ERR_SHAPE, "fm_lq_scan: B, T must be >= 0");
+  if ((long long)B * T == 0) return FM_OK;
+  if (B > 65535) return fail(FM_ERR_SHAPE, "fm_lq_scan: B=%d exceeds 65535", B);
+  if (ld_dt < d.nh || (z && ld_z < d.di))
+    return fail(FM_ERR_SHAPE, "fm_lq_scan: row strides too small (ld_dt %lld, ld_z %lld)",
+                (long long)ld_dt, (long long)ld_z);
+  NEED(xo);
+  if (!dt_raw) return fail(FM_ERR_INVALID_ARG, "fm_lq_scan: dt_raw is null");
+  NEED(dt_bias);
+  NEED(a_log);
+  NEED(D);
+  NEED(out);
+  OPT(state);
+  return launch_lq_scan(d, xo, dt_raw, ld_dt, z, ld_z, B, T, dt_bias, a_log, D, state, out,
+                        (cudaStream_t)stream);
+}
+
+namespace {
+struct LqWs {
+  int8_t *q_in;
+  float *sx_in;
+  float *Y;  // [M, n_in] in_proj output: z | xBC | dt_raw
+  float *xo;
+  float *g;
+  int8_t *q_out;
+  float *sx_out;
+  int32_t *split;
+};
+LqWs carve_lq(Carver &c, const Dims &d, int B, int T) {
+  const long long M = (long long)B * T;
+  LqWs w;
+  w.q_in = c.take<int8_t>(M * d.dm);
+  w.sx_in = c.take<float>(M);
+  w.Y = c.take<float>(M * d.n_in);
+  w.xo = c.take<float>(M * d.cc);
+  w.g = c.take<float>(M * d.di);
+  w.q_out = c.take<int8_t>(M * d.di);
+  w.sx_out = c.take<float>(M);
+  const bool in_split = gemm_would_split(M, d.n_in, d.dm);
+  const bool out_split = gemm_would_split(M, d.dm, d.di);
+  const long long n = in_split ? (out_split ? (d.n_in > d.dm ? d.n_in : d.dm) : d.n_in)
+                               : (out_split ? d.dm : 0);
+  w.split = n ? c.take<int32_t>(M * n) : nullptr;
+  return w;
+}
+}  // namespace
+
+extern "C" size_t fm_lq_workspace_bytes(const fm_shape *shape, int B, int T) {
+  Dims d;
+  if (check_shape(shape, &d, __func__) != FM_OK || B < 0 || T < 0) return 0;
+  Carver c{nullptr, 0};
+  carve_lq(c, d, B, T);
+  return c.off + 256;
+}
+
+extern "C" fm_status fm_lq_mixer_prefill(const fm_layer *L, const fm_lq_params *P,
+                                         const float *x, int B, int T, int residual,
+                                         float *conv_state, float *ssm_state, float *out,
+                                         void *ws, size_t ws_bytes, fm_stream stream) {
+  Dims d;
+  FM_TRY(check_layer(L, &d, __func__));
+  FM_TRY(lq_check_params(P, __func__));
+  if (B < 0 || T < 0) return fail(FM_ERR_SHAPE, "fm_lq_mixer_prefill: B, T must be >= 0");
+  if ((long long)B * T == 0) return FM_OK;
+  FM_TRY(check_batch(B, T, __func__));
+  NEED(x);
+  NEED(out);
+  OPT(conv_state);
+  OPT(ssm_state);
+  const size_t need = fm_lq_workspace_bytes(&L->shape, B, T);
+  if (!ws || ws_bytes < need || !aligned16(ws))
+    return fail(FM_ERR_WORKSPACE, "fm_lq_mixer_prefill: workspace needs %zu bytes", need);
+  if (out != x) {
+    const char *xb = reinterpret_cast<const char *>(x), *ob = reinterpret_cast<const char *>(out);
+    const size_t bytes = (size_t)B * T * d.dm * sizeof(float);
+    if (ob < xb + bytes && xb < ob + bytes)
+      return fail(FM_ERR_INVALID_ARG, "fm_lq_mixer_prefill: out partially overlaps x");
+  }
+  Carver c{reinterpret_cast<uint8_t *>(ws), 0};
+  const LqWs w = carve_lq(c, d, B, T);
+  const cudaStream_t s = (cudaStream_t)stream;
+  const long long M = (long long)B * T;
+  const float *amax_in = L->static_amax, *amax_out = L->static_amax ? L->static_amax + 1 : nullptr;
+  // rotated W8A8 in_proj with a plain fp32 output
+  FM_TRY(launch_hadamard_quant(x, M, d.dm, L->prenorm_w, L->rotate, L->mode, amax_in, w.q_in,
+                               w.sx_in, nullptr, s));
+  FM_TRY(launch_gemm(w.q_in, M, L->w_in_q, d.n_in, d.dm,
+                     plain_epilogue(M, d.n_in, w.sx_in, L->w_in_s, nullptr, w.Y, nullptr), s,
+                     w.split));
+  // exact fp32 conv, scan and gate
+  FM_TRY(launch_lq_conv(w.Y + d.di, d.n_in, B, T, d.cc, P->conv_w, P->conv_b, conv_state, w.xo,
+                        s));
+  FM_TRY(launch_lq_scan(d, w.xo, w.Y + d.di + d.cc, d.n_in, w.Y, d.n_in, B, T, L->dt_bias,
+                        P->a_log, P->D, ssm_state, w.g, s));
+  // gated RMSNorm (the norm weight as the pre-norm weight), rotation, int8
+  FM_TRY(launch_hadamard_quant(w.g, M, d.di, L->norm_w, L->rotate, L->mode, amax_out, w.q_out,
+                               w.sx_out, nullptr, s));
+  return launch_gemm(w.q_out, M, L->w_out_q, d.dm, d.di,
+                     plain_epilogue(M, d.dm, w.sx_out, L->w_out_s, residual ? x : nullptr, out,
+                                    nullptr),
+                     s, w.split);
 }
 
 // ------------------------------------------------------------------ offline preparation

@@ -29,7 +29,8 @@ EXPORTS = (
     "fm_mixer_prefill", "fm_decode_step", "fm_prepare_mixer_params", "fm_calib_workspace_bytes",
     "fm_calibrate_layer", "fm_decode_step_noalloc", "fm_scan_workspace_bytes",
     "fm_set_scan_tile", "fm_ssd_workspace_bytes", "fm_ssd_scan", "fm_set_scan_mode",
-    "fm_set_scan_tile", "fm_set_state_spec",
+    "fm_set_state_spec", "fm_lq_conv1d", "fm_lq_scan", "fm_lq_workspace_bytes",
+    "fm_lq_mixer_prefill",
 )
 NOALLOC_SCRATCH_BYTES = 16 << 20  # FM_NOALLOC_SCRATCH_BYTES
 
@@ -58,6 +59,10 @@ class fm_layer(C.Structure):
                 ("w_in_q", _P), ("w_in_s", _P), ("w_out_q", _P), ("w_out_s", _P),
                 ("prenorm_w", _P), ("conv_wq", _P), ("conv_bq", _P), ("dt_bias", _P),
                 ("A_q", _P), ("D_q", _P), ("norm_w", _P), ("exps", _P), ("static_amax", _P)]
+
+
+class fm_lq_params(C.Structure):
+    _fields_ = [("conv_w", _P), ("conv_b", _P), ("a_log", _P), ("D", _P)]
 
 
 _lib = None
@@ -105,6 +110,11 @@ def load():
         "fm_prepare_mixer_params": (I, [sp, _P, _P, _P, _P, _P, _P, _P, _P]),
         "fm_calib_workspace_bytes": (SZ, [sp, I, I]),
         "fm_calibrate_layer": (I, [lp, _P, _P, _P, _P, _P, I, I, I, _P, _P, SZ, _P]),
+        "fm_lq_conv1d": (I, [_P, I64, I, I, sp, _P, _P, _P, _P, _P]),
+        "fm_lq_scan": (I, [_P, _P, I64, _P, I64, I, I, sp, _P, _P, _P, _P, _P, _P]),
+        "fm_lq_workspace_bytes": (SZ, [sp, I, I]),
+        "fm_lq_mixer_prefill": (I, [lp, C.POINTER(fm_lq_params), _P, I, I, I, _P, _P, _P, _P,
+                                    SZ, _P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(L, name)
@@ -298,3 +308,48 @@ def calibrate_layer(layer: fm_layer, conv_b, exps, conv_bq, static_amax, xcal, B
     _check(load().fm_calibrate_layer(C.byref(layer), _p(conv_b), _p(exps), _p(conv_bq),
                                      _p(static_amax), _p(xcal), B, T, residual, _p(out), _p(ws),
                                      ws.numel() * ws.element_size(), _s(stream)))
+
+
+# ------------------------------------------------------------------ FastMamba-LQ
+def _p_any(t):
+    """A CUDA tensor's address without the contiguity check (strided row views)."""
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("libfastmamba takes CUDA tensors only")
+    return C.c_void_p(t.data_ptr())
+
+
+def _row_view(t, width):
+    """(pointer, row stride) of a 2-D view whose rows are unit-stride."""
+    if t.dim() != 2 or t.stride(1) != 1 or t.shape[1] != width:
+        raise ValueError("expected a [rows, width] view with unit column stride")
+    return _p_any(t), t.stride(0)
+
+
+def lq_conv1d(u, B, T, shape, conv_w, conv_b, conv_state, out, stream=None):
+    """u: [B*T, conv_ch] rows (may be a column slice of a wider buffer)."""
+    sh = shape_struct(shape)
+    pu, ldu = _row_view(u, shape.conv_ch)
+    _check(load().fm_lq_conv1d(pu, ldu, B, T, C.byref(sh), _p(conv_w), _p(conv_b),
+                               _p(conv_state), _p(out), _s(stream)))
+
+
+def lq_scan(xo, dt_raw, z, B, T, shape, dt_bias, a_log, D, state, out, stream=None):
+    """dt_raw: [B*T, nheads] rows, z: [B*T, d_inner] rows or None (slices allowed)."""
+    sh = shape_struct(shape)
+    pdt, lddt = _row_view(dt_raw, shape.nheads)
+    pz, ldz = _row_view(z, shape.d_inner) if z is not None else (None, 0)
+    _check(load().fm_lq_scan(_p(xo), pdt, lddt, pz, ldz, B, T, C.byref(sh), _p(dt_bias),
+                             _p(a_log), _p(D), _p(state), _p(out), _s(stream)))
+
+
+def lq_workspace_bytes(shape, B, T) -> int:
+    return load().fm_lq_workspace_bytes(C.byref(shape_struct(shape)), B, T)
+
+
+def lq_mixer_prefill(layer: fm_layer, params: fm_lq_params, x, B, T, residual, conv_state,
+                     ssm_state, out, ws, stream=None):
+    _check(load().fm_lq_mixer_prefill(C.byref(layer), C.byref(params), _p(x), B, T, residual,
+                                      _p(conv_state), _p(ssm_state), _p(out), _p(ws),
+                                      ws.numel() * ws.element_size(), _s(stream)))

@@ -51,6 +51,8 @@ class DeviceLayer:
                                  self.D_q, self.exps, stream)
         del w_in, w_out
         self.struct = self._make_struct()
+        p = lambda t: t.data_ptr()
+        self.lq_struct = lib.fm_lq_params(p(self.conv_w), p(self.conv_b), p(self.a_log), p(self.D))
 
     def _make_struct(self) -> lib.fm_layer:
         p = lambda t: None if t is None else t.data_ptr()
@@ -83,26 +85,6 @@ class DeviceLayer:
                     e_g=int(e[X.e_g]), amax_in=float(amax[0]), amax_out=float(amax[1]),
                     conv_bq=self.conv_bq.cpu().numpy())
 
-    def set_exponents(self, ex: dict):
-        """Install an externally calibrated table (e_u, e_x, e_B, e_C, e_h, e_y, e_g,
-        amax_in, amax_out, conv_bq); e_w and e_D stay those of the preparation."""
-        e = self.exps.cpu().numpy().copy()
-        X, s = self.layout, self.shape
-        cc, nh, hd, ds, di = s.conv_ch, s.nheads, s.headdim, s.d_state, s.d_inner
-        e[X.e_u:X.e_u + cc] = ex["e_u"]
-        e[X.e_x:X.e_x + nh] = ex["e_x"]
-        e[X.e_B] = ex["e_B"]
-        e[X.e_C] = ex["e_C"]
-        e[X.e_o:X.e_o + cc] = np.concatenate([np.repeat(ex["e_x"], hd), np.full(ds, ex["e_B"]),
-                                              np.full(ds, ex["e_C"])])
-        e[X.e_h:X.e_h + nh] = ex["e_h"]
-        e[X.e_y:X.e_y + nh] = ex["e_y"]
-        e[X.e_g] = ex["e_g"]
-        self.exps.copy_(torch.from_numpy(e))
-        self.conv_bq.copy_(torch.from_numpy(np.ascontiguousarray(ex["conv_bq"], np.int32)))
-        self.static_amax.copy_(torch.tensor([ex["amax_in"], ex["amax_out"], 0.0, 0.0],
-                                            dtype=torch.float32))
-
     # ------------------------------------------------------------ running
     def workspace(self, B: int, T: int) -> torch.Tensor:
         return torch.empty(lib.workspace_bytes(self.shape, B, T), dtype=torch.uint8,
@@ -124,6 +106,28 @@ class DeviceLayer:
         ws = self.workspace(B, 1) if ws is None else ws
         lib.decode_step(self.struct, x, B, int(residual), conv_state, ssm_state, out, ws, stream)
         return out
+
+    # ------------------------------------------------------------ FastMamba-LQ
+    def lq_workspace(self, B: int, T: int) -> torch.Tensor:
+        return torch.empty(lib.lq_workspace_bytes(self.shape, B, T), dtype=torch.uint8,
+                           device=self.device)
+
+    def lq_prefill(self, x: torch.Tensor, residual: bool = False, conv_state=None,
+                   ssm_state=None, out=None, ws=None, stream=None) -> torch.Tensor:
+        """The LQ variant of this layer: the same W8A8 linears and scales, the
+        conv, scan and gate in fp32 (fp32 states from lq_new_states)."""
+        B, T, _ = x.shape
+        out = torch.empty_like(x) if out is None else out
+        ws = self.lq_workspace(B, T) if ws is None else ws
+        lib.lq_mixer_prefill(self.struct, self.lq_struct, x, B, T, int(residual), conv_state,
+                             ssm_state, out, ws, stream)
+        return out
+
+    def lq_new_states(self, B: int):
+        s = self.shape
+        return (torch.zeros((B, 3, s.conv_ch), dtype=torch.float32, device=self.device),
+                torch.zeros((B, s.nheads, s.headdim, s.d_state), dtype=torch.float32,
+                            device=self.device))
 
     def new_states(self, B: int):
         s = self.shape

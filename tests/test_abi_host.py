@@ -187,3 +187,41 @@ def test_state_spec_validation(so):
     assert so.fm_set_state_spec(24, 7) == 1
     assert so.fm_set_state_spec(16, 7) == 0
     assert so.fm_set_state_spec(31, 0) == 0
+
+
+def test_lq_entry_points_validate(so):
+    """The FastMamba-LQ entry points reject bad arguments before any launch,
+    and the layer workspace covers its fp32 intermediates."""
+    from quantized_state_space_mamba2_b200 import lib
+    from quantized_state_space_mamba2_b200 import synth as S
+    s = S.MAMBA2_130M
+    sh = lib.shape_struct(s)
+    p = C.c_void_p(0x7000000)
+    # empty problems: nothing to do
+    assert so.fm_lq_conv1d(None, 0, 0, 5, C.byref(sh), None, None, None, None, None) == 0
+    assert so.fm_lq_scan(None, None, 0, None, 0, 3, 0, C.byref(sh), None, None, None, None, None,
+                         None) == 0
+    # conv: a row stride below conv_ch, a null weight, a misaligned output
+    assert so.fm_lq_conv1d(p, s.conv_ch - 1, 1, 5, C.byref(sh), p, p, None, p, None) == 2
+    assert so.fm_lq_conv1d(p, s.conv_ch, 1, 5, C.byref(sh), None, p, None, p, None) == 1
+    assert so.fm_lq_conv1d(p, s.conv_ch, 1, 5, C.byref(sh), p, p, None, C.c_void_p(0x7000004),
+                           None) == 3
+    # scan: dt stride below nheads, z stride below d_inner, a null dt_bias
+    assert so.fm_lq_scan(p, p, s.nheads - 1, None, 0, 1, 5, C.byref(sh), p, p, p, None, p,
+                         None) == 2
+    assert so.fm_lq_scan(p, p, s.nheads, p, s.d_inner - 1, 1, 5, C.byref(sh), p, p, p, None, p,
+                         None) == 2
+    assert so.fm_lq_scan(p, p, s.nheads, None, 0, 1, 5, C.byref(sh), None, p, p, None, p,
+                         None) == 1
+    # the layer: workspace = int8 input + scale, fp32 in_proj output, conv
+    # output, gated value, int8 out_proj input + scale (+ split-K sums)
+    M = 300
+    need = lib.lq_workspace_bytes(s, 1, M)
+    base = M * (s.d_model + 4 + 4 * s.n_in + 4 * s.conv_ch + 4 * s.d_inner + s.d_inner + 4)
+    split = max(lib.gemm_workspace_bytes(M, s.n_in, s.d_model),
+                lib.gemm_workspace_bytes(M, s.d_model, s.d_inner))
+    assert base + split <= need <= base + split + 256 * 10
+    L = lib.fm_layer()
+    P = lib.fm_lq_params()
+    assert so.fm_lq_mixer_prefill(C.byref(L), C.byref(P), p, 1, 5, 0, None, None, p, p, 1 << 30,
+                                  None) in (1, 2)

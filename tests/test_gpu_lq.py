@@ -1,0 +1,199 @@
+"""GPU parity of the FastMamba-LQ path (fm_lq_conv1d, fm_lq_scan,
+fm_lq_mixer_prefill) against fp64 definitions and the oracle's LQ mixer.
+
+LQ keeps the method's rotated W8A8 linears and runs the conv, the scan and
+the gate in exact fp32 arithmetic (pith.science review of FastMamba, Desk
+Editor's Note: Table II's "FastMamba-LQ").  fp32 is not bit-exact against
+fp64, so each stage is held to a bound derived from fp32 rounding, scaled by
+the magnitude of its terms (the same computation on absolute values):
+  * conv + SiLU: 1e-6 |terms| per element (a handful of fp32 roundings);
+  * scan: 1e-4 |terms| per output, where |terms| is the scan on |x|, |B|,
+    |C| with the same decays (fp32 roundings of dt, dA and the state,
+    accumulated over the decay's memory of up to ~1000 steps);
+  * the layer: max abs error <= 1e-3 x RMS of the output (the fp32 rule of
+    the parity spec), against the oracle's LQ mixer on the same calibration.
+"""
+import numpy as np
+import pytest
+
+import oracle as O
+from oracle import stages
+from quantized_state_space_mamba2_b200 import synth as S
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+MAMBA130 = S.MAMBA2_130M
+
+
+@pytest.fixture(scope="module")
+def L():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from quantized_state_space_mamba2_b200 import build, lib
+    build.build()
+    lib.load()
+    return lib
+
+
+def dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def host(t):
+    torch.cuda.synchronize()
+    return t.cpu().numpy()
+
+
+def _silu(v):
+    return v / (1.0 + np.exp(-v))
+
+
+@pytest.mark.parametrize("B,T,with_state", [(1, 1, False), (2, 37, True), (1, 300, False),
+                                            (3, 1, True)])
+def test_lq_conv_matches_f64(L, B, T, with_state):
+    s = MAMBA130
+    cc, n_in = s.conv_ch, s.n_in
+    Y = S.normal((B * T, n_in), 1.5, seed=10 + T)            # an in_proj output, xBC in place
+    w = S.normal((cc, 4), 0.2, seed=11)
+    b = S.normal(cc, 0.1, seed=12)
+    st = S.normal((B, 3, cc), 1.0, seed=13) if with_state else None
+    out = torch.empty((B, T, cc), dtype=torch.float32, device="cuda")
+    Yd = dev(Y)
+    std = dev(st) if with_state else None
+    L.lq_conv1d(Yd[:, s.d_inner:s.d_inner + cc], B, T, s, dev(w), dev(b), std, out)
+    u = Y[:, s.d_inner:s.d_inner + cc].reshape(B, T, cc).astype(np.float64)
+    hist = st.astype(np.float64) if with_state else np.zeros((B, 3, cc))
+    up = np.concatenate([hist, u], axis=1)
+    acc = b.astype(np.float64) + sum(w[:, k].astype(np.float64) * up[:, k:k + T] for k in range(4))
+    mag = np.abs(b) + sum(np.abs(w[:, k]) * np.abs(up[:, k:k + T]) for k in range(4))
+    ref = _silu(acc)
+    got = host(out)
+    assert (np.abs(got - ref) <= 1e-6 * mag + 1e-30).all()
+    if with_state:
+        assert np.array_equal(host(std), up[:, T:T + 3].astype(np.float32))
+
+
+def _scan_f64(xo, dt_raw, dt_bias, a_log, D, di, ds, hd, h0=None, absval=False):
+    """Mamba2's recurrence in fp64 (one group); absval: the same decays on
+    |x|, |B|, |C| and |h0| (the magnitude of the terms)."""
+    Bsz, T, _ = xo.shape
+    nh = di // hd
+    x = xo[..., :di].reshape(Bsz, T, nh, hd).astype(np.float64)
+    Bm = xo[..., di:di + ds].astype(np.float64)
+    Cm = xo[..., di + ds:].astype(np.float64)
+    if absval:
+        x, Bm, Cm = np.abs(x), np.abs(Bm), np.abs(Cm)
+    dt = np.logaddexp(0.0, dt_raw.astype(np.float64) + dt_bias.astype(np.float64))
+    dA = np.exp(dt * -np.exp(a_log.astype(np.float64)))
+    h = np.zeros((Bsz, nh, hd, ds)) if h0 is None else h0.astype(np.float64)
+    if absval:
+        h = np.abs(h)
+    y = np.empty((Bsz, T, nh, hd))
+    Dv = np.abs(D) if absval else D
+    for t in range(T):
+        h = dA[:, t, :, None, None] * h + (dt[:, t, :, None] * x[:, t])[..., None] \
+            * Bm[:, t, None, None, :]
+        y[:, t] = np.einsum("bhpn,bn->bhp", h, Cm[:, t]) + Dv[None, :, None] * x[:, t]
+    return y.reshape(Bsz, T, di), h
+
+
+@pytest.mark.parametrize("shape,B,T,with_state,gate", [("130m", 1, 1, False, False),
+                                                      ("130m", 2, 77, True, True),
+                                                      ("130m", 1, 700, False, True),
+                                                      ("2p7b", 2, 40, True, False),
+                                                      ("2p7b", 5, 1, True, True)])
+def test_lq_scan_matches_f64(L, shape, B, T, with_state, gate):
+    s = MAMBA130 if shape == "130m" else S.MAMBA2_2P7B
+    di, ds, hd, nh, cc = s.d_inner, s.d_state, s.headdim, s.nheads, s.conv_ch
+    P = S.layer_params(s, 300 + T)
+    xo = S.normal((B, T, cc), 1.0, seed=20 + T)
+    Y = S.normal((B * T, s.n_in), 1.0, seed=21 + T)           # z and dt_raw read in place
+    Y[:, di + cc:] = S.normal((B * T, nh), 2.0, seed=22 + T)
+    st = S.normal((B, nh, hd, ds), 3.0, seed=23) if with_state else None
+    Yd = dev(Y)
+    std = dev(st) if with_state else None
+    out = torch.empty((B, T, di), dtype=torch.float32, device="cuda")
+    z = Yd[:, :di] if gate else None
+    L.lq_scan(dev(xo), Yd[:, di + cc:], z, B, T, s, dev(P["dt_bias"]), dev(P["a_log"]),
+              dev(P["D"]), std, out)
+    dt_raw = Y[:, di + cc:].reshape(B, T, nh)
+    y, hT = _scan_f64(xo, dt_raw, P["dt_bias"], P["a_log"], P["D"], di, ds, hd, st)
+    mag, hmag = _scan_f64(xo, dt_raw, P["dt_bias"], P["a_log"], P["D"], di, ds, hd, st,
+                          absval=True)
+    if gate:
+        sg = _silu(Y[:, :di].astype(np.float64)).reshape(B, T, di)
+        y, mag = y * sg, mag * np.abs(sg)
+    got = host(out)
+    err = np.abs(got - y)
+    assert (err <= 1e-4 * mag + 1e-30).all(), float((err / (mag + 1e-30)).max())
+    if with_state:
+        assert (np.abs(host(std) - hT) <= 1e-4 * hmag + 1e-30).all()
+
+
+def _lq_layers(s, seed, prenorm=False, mode=O.DYNAMIC):
+    from quantized_state_space_mamba2_b200.model import DeviceLayer
+    P = S.layer_params(s, seed, conv_bias_std=0.05)
+    xcal = S.calibration_batch(s.d_model, 64, 8, 50.0, 4242, n_seqs=2)
+    ol = O.prepare_layer(P, s, mode=mode, prenorm=prenorm)
+    O.calibrate_layer(ol, xcal, residual=prenorm)
+    dl = DeviceLayer(P, s, mode=mode, prenorm=prenorm)
+    dl.calibrate(dev(xcal), residual=prenorm)
+    return P, ol, dl
+
+
+@pytest.mark.parametrize("mode", [O.DYNAMIC, O.STATIC])
+def test_lq_layer_matches_oracle(L, mode):
+    """A calibrated 130M layer in LQ form against the oracle's lq_mixer (the
+    same calibration, computed on each side), within 1e-3 x RMS."""
+    s = MAMBA130
+    P, ol, dl = _lq_layers(s, 1000, mode=mode)
+    x = S.activations(1, 256, s.d_model, seed=3, n_outliers=8, outlier_scale=50.0,
+                      outlier_seed=4242)
+    got = host(dl.lq_prefill(dev(x)))
+    ref = stages.lq_mixer(ol, P, x)
+    rms = np.sqrt(np.mean(ref ** 2))
+    assert np.abs(got - ref).max() <= 1e-3 * rms
+    # the LQ variant is more accurate than the full method against fp64
+    f64 = O.ref_mixer_f64(P, s, x)
+    full = host(dl.prefill(dev(x)))
+    assert O.sqnr_db(f64, got) > O.sqnr_db(f64, full) + 5.0
+
+
+def test_lq_stack_layer_chunked_and_decode(L):
+    """A pre-normed residual layer: a 100-token prefill, a 60-token prefill
+    and 3 decode steps carrying the fp32 conv and SSM states equal one
+    163-token prefill -- states bit for bit (each is a per-element recurrence
+    in the same order), outputs within fp32 reduction-order rounding -- and
+    the whole agrees with the oracle's LQ mixer."""
+    s = MAMBA130
+    P, ol, dl = _lq_layers(s, 1001, prenorm=True)
+    x = S.activations(2, 163, s.d_model, seed=4, n_outliers=8, outlier_scale=50.0,
+                      outlier_seed=4242)
+    xd = dev(x)
+    cs, ss = dl.lq_new_states(2)
+    full = host(dl.lq_prefill(xd, residual=True, conv_state=cs, ssm_state=ss))
+    cs2, ss2 = dl.lq_new_states(2)
+    parts = [dl.lq_prefill(xd[:, :100].contiguous(), residual=True, conv_state=cs2, ssm_state=ss2),
+             dl.lq_prefill(xd[:, 100:160].contiguous(), residual=True, conv_state=cs2,
+                           ssm_state=ss2)]
+    for t in range(160, 163):
+        parts.append(dl.lq_prefill(xd[:, t:t + 1].contiguous(), residual=True, conv_state=cs2,
+                                   ssm_state=ss2))
+    chunked = host(torch.cat(parts, 1))
+    assert torch.equal(cs, cs2) and torch.equal(ss, ss2)
+    # compare the mixer's contribution (output minus the residual input)
+    mix = full - x
+    rms = np.sqrt(np.mean(mix ** 2))
+    assert np.abs(chunked - full).max() <= 1e-3 * rms
+    ref = stages.lq_mixer(ol, P, x, residual=True) - x
+    assert np.abs(mix - ref).max() <= 1e-3 * np.sqrt(np.mean(ref ** 2))
+
+
+def test_lq_validation(L):
+    s = MAMBA130
+    t = torch.zeros(64, dtype=torch.float32, device="cuda")
+    with pytest.raises(L.FmError) as e:             # dt_bias is null
+        L.lq_scan(t, t.view(2, 32)[:, :24], None, 1, 5, s, None, t, t, None, t)
+    assert e.value.status == 1
+    assert L.lq_workspace_bytes(s, 0, 0) <= 4096
