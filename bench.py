@@ -433,6 +433,7 @@ class DecodeWorkload(StackWorkload):
         self.shape = d = w["shape"]
         self.n_layers, self.B, self.T = n_layers(args), w["batch"], 1
         self.stack_mode = True
+        self.ssd = False  # a single-token step always runs the sequential scan step
         self.mode = lib.FM_DYNAMIC if args.mode == "dynamic" else lib.FM_STATIC
         P = w["prefill_len"]
         self.stack = DeviceStack([S.layer_params(d, 1000 + l) for l in range(self.n_layers)], d,

@@ -52,7 +52,7 @@ typedef enum fm_status {
     FM_ERR_SHAPE = 2,       /* unsupported or inconsistent sizes */
     FM_ERR_ALIGNMENT = 3,   /* pointer not 16-byte aligned */
     FM_ERR_WORKSPACE = 4,   /* workspace missing or too small */
-    FM_ERR_NONFINITE = 5,   /* reserved: non-finite statistic seen on device */
+    FM_ERR_NONFINITE = 5,   /* a NaN or Inf reached an int8 activation quantiser */
     FM_ERR_TIMEOUT = 6,     /* a bounded device-side wait gave up */
     FM_ERR_CUDA = 7,        /* a CUDA runtime/driver call failed */
     FM_ERR_UNSUPPORTED = 8  /* no sm_100 device, or driver entry point missing */
@@ -67,8 +67,12 @@ const char *fm_status_string(fm_status s);
 /* Detail of the last failed call on this host thread (static, thread-local). */
 const char *fm_last_error(void);
 /* Synchronises `stream`, then reads and clears the device error word of the
- * current device: FM_OK, FM_ERR_TIMEOUT (a bounded wait gave up) or
- * FM_ERR_CUDA (the synchronisation itself failed). */
+ * current device: FM_OK, FM_ERR_TIMEOUT (a bounded wait gave up; it takes
+ * precedence), FM_ERR_NONFINITE (an activation row entering an int8
+ * quantiser -- fm_hadamard_quant, fm_gate_norm_quant and the layers that
+ * call them -- held a NaN or Inf; that row's codes and scale are then
+ * undefined) or FM_ERR_CUDA (the synchronisation itself failed).  The word
+ * accumulates over every call on the device since it was last read. */
 fm_status fm_sync_status(fm_stream stream);
 /* Library ABI version (major * 100 + minor). */
 int fm_version(void);

@@ -15,11 +15,12 @@
 namespace fm {
 
 // Device error word (per device, per process): 0 = ok; bit 0 = a bounded
-// wait gave up.  Read and cleared by fm_sync_status().  The library is one
-// translation unit (fm_lib.cu includes every kernel header), so the
-// definition lives here.
+// wait gave up; bit 1 = a non-finite value reached an int8 quantiser.  Read
+// and cleared by fm_sync_status().  The library is one translation unit
+// (fm_lib.cu includes every kernel header), so the definition lives here.
 __device__ unsigned int g_error_word = 0;
 constexpr unsigned int kErrTimeout = 1u;
+constexpr unsigned int kErrNonfinite = 2u;
 
 __device__ __forceinline__ void raise_error(unsigned int bits) { atomicOr(&g_error_word, bits); }
 

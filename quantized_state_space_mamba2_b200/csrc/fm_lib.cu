@@ -85,6 +85,8 @@ extern "C" fm_status fm_sync_status(fm_stream stream) {
   if (word) {
     FM_CHECK_CUDA(cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)));
     if (word & kErrTimeout) return fail(FM_ERR_TIMEOUT, "a bounded device wait gave up");
+    if (word & kErrNonfinite)
+      return fail(FM_ERR_NONFINITE, "a non-finite value (NaN or Inf) reached an int8 quantiser");
   }
   return FM_OK;
 }
@@ -538,7 +540,6 @@ static fm_status launch_scan_v2(const ScanArgs &a, int B, const ScanWs &w, cudaS
   q.e_y = a.e_y;
   q.state = a.state;
   q.y = a.y;
-  q.k16 = 65536;
   const ScanTile t = scan_tile();
 #define FM_SEQ(N, P, C)                                      \
   if (t.npt == N && t.pc == P && t.tch == C)                 \

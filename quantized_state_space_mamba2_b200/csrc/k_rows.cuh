@@ -51,10 +51,16 @@ __device__ __forceinline__ void rotate_quant_store(float (&v)[BPW][8], int rotat
     for (int b = 0; b < BPW; ++b) fwht256_lane8(v[b], lane);
   }
   float a = 0.0f;
+  bool finite = true;  // fmaxf drops NaN, so non-finite values are flagged apart
 #pragma unroll
   for (int b = 0; b < BPW; ++b)
 #pragma unroll
-    for (int i = 0; i < 8; ++i) a = fmaxf(a, fabsf(v[b][i]));
+    for (int i = 0; i < 8; ++i) {
+      const float m = fabsf(v[b][i]);
+      finite = finite && (m <= 3.402823466e38f);
+      a = fmaxf(a, m);
+    }
+  if (!finite) raise_error(kErrNonfinite);
   const float amax = cta_max(a, s_red, s_bc);
   const float use = (mode == 0) ? amax : *static_amax;
   const float inv = use > 0.0f ? __fdiv_rn(127.0f, use) : 0.0f;

@@ -150,9 +150,6 @@ struct ScanSeqArgs {
   const int32_t *e_x, *e_C, *e_h, *e_y, *e_D;
   int32_t *state;     // [B, nh, hd, 128] or null
   int32_t *y;         // [B*T, di]
-  // 2^16, passed at run time so that the state split below stays a multiply
-  // (FMA pipe) instead of becoming shifts and a mask (ALU pipe)
-  int k16;
 };
 
 __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes,
@@ -213,9 +210,6 @@ __device__ __forceinline__ void load_bc(const int32_t (*bc)[256], int tt, int n0
 // false is used only when the chunk provably never reaches the clamp (see
 // k_scan_seq), so both instantiations give the same bits.  part[tt] holds the
 // (C hh, C hl) partial sums of step tt.
-// The splits by 2^16 are multiplies by k16 = 2^16 (a run-time value):
-// umulhi(t, 2^16) = t >> 16, mulhi(hn, 2^16) = floor(hn / 2^16) = hn >> 16,
-// hn - hh 2^16 = hn & 0xFFFF -- the same bits, issued on the FMA pipe.
 // S16: the 16-bit state spec (|h| <= 2^15 - 1, so dA h fits int32 and no
 // split is needed; the increment is rshr(u B, 7) with u carrying 7 guard
 // bits): h lives in hh, hl is unused, and the C h sum is the single .x.
@@ -225,7 +219,7 @@ constexpr int kH16Guard = 7;
 template <int NPT, bool CLAMP, bool S16 = false>
 __device__ __forceinline__ int2 scan_one_step(int (&hh)[NPT], unsigned (&hl)[NPT],
                                               const int (&Bv)[NPT], const int (&Cv)[NPT], int dA,
-                                              int u, int k16) {
+                                              int u) {
   int ahi = 0, alo = 0;
   if constexpr (S16) {
 #pragma unroll
@@ -241,10 +235,10 @@ __device__ __forceinline__ int2 scan_one_step(int (&hh)[NPT], unsigned (&hl)[NPT
 #pragma unroll
   for (int j = 0; j < NPT; ++j) {
     const unsigned t = (unsigned)dA * hl[j] + 0x8000u;
-    int hn = dA * hh[j] + (int)__umulhi(t, (unsigned)k16) + u * Bv[j];
+    int hn = dA * hh[j] + (int)(t >> 16) + u * Bv[j];
     if (CLAMP) hn = min(max(hn, -(int)kHLim), (int)kHLim);
-    hh[j] = __mulhi(hn, k16);
-    hl[j] = (unsigned)(hn - hh[j] * k16);
+    hh[j] = hn >> 16;
+    hl[j] = (unsigned)hn & 0xFFFFu;
     ahi += Cv[j] * hh[j];
     alo += Cv[j] * (int)hl[j];
   }
@@ -259,7 +253,7 @@ template <int NPT, int TCH, bool FULL, bool CLAMP, bool REDUX, bool S16 = false>
 __device__ __forceinline__ void scan_chunk_steps(int (&hh)[NPT], unsigned (&hl)[NPT],
                                                  int2 (&part)[TCH], int2 *wsum,
                                                  const int32_t (*bc)[256], const int32_t *dAv,
-                                                 const int32_t *uv, int n0, int nt, int k16) {
+                                                 const int32_t *uv, int n0, int nt) {
   // two register sets for B / C: the even step's set is refilled two steps
   // ahead while the odd step computes, and vice versa (no copies)
   int B0[NPT], C0[NPT], B1[NPT], C1[NPT];
@@ -290,11 +284,11 @@ __device__ __forceinline__ void scan_chunk_steps(int (&hh)[NPT], unsigned (&hl)[
     for (int k = 0; k < 4; k += 2) {
       const int tt = tg + k;
       if (FULL || tt + 1 < nt) load_bc<NPT>(bc, tt + 1, n0, B1, C1);
-      if (FULL || tt < nt) emit(tt, scan_one_step<NPT, CLAMP, S16>(hh, hl, B0, C0, dAs[k], us[k], k16));
+      if (FULL || tt < nt) emit(tt, scan_one_step<NPT, CLAMP, S16>(hh, hl, B0, C0, dAs[k], us[k]));
       else if constexpr (!REDUX) part[tt] = make_int2(0, 0);
       if (tt + 2 < TCH && (FULL || tt + 2 < nt)) load_bc<NPT>(bc, tt + 2, n0, B0, C0);
       if (FULL || tt + 1 < nt)
-        emit(tt + 1, scan_one_step<NPT, CLAMP, S16>(hh, hl, B1, C1, dAs[k + 1], us[k + 1], k16));
+        emit(tt + 1, scan_one_step<NPT, CLAMP, S16>(hh, hl, B1, C1, dAs[k + 1], us[k + 1]));
       else if constexpr (!REDUX) part[tt + 1] = make_int2(0, 0);
     }
   }
@@ -409,11 +403,11 @@ __global__ void __launch_bounds__(PC *(128 / NPT) + 32) k_scan_seq(ScanSeqArgs a
     int2 *wsum = reinterpret_cast<int2 *>(&part[0][0]);
     if (nt == TCH) {
       if (no_clamp)
-        scan_chunk_steps<NPT, TCH, true, false, REDUX, S16>(hh, hl, pr, wsum, s.bc, s.dA, s.u[pp], n0, nt, a.k16);
+        scan_chunk_steps<NPT, TCH, true, false, REDUX, S16>(hh, hl, pr, wsum, s.bc, s.dA, s.u[pp], n0, nt);
       else
-        scan_chunk_steps<NPT, TCH, true, true, REDUX, S16>(hh, hl, pr, wsum, s.bc, s.dA, s.u[pp], n0, nt, a.k16);
+        scan_chunk_steps<NPT, TCH, true, true, REDUX, S16>(hh, hl, pr, wsum, s.bc, s.dA, s.u[pp], n0, nt);
     } else {
-      scan_chunk_steps<NPT, TCH, false, true, REDUX, S16>(hh, hl, pr, wsum, s.bc, s.dA, s.u[pp], n0, nt, a.k16);
+      scan_chunk_steps<NPT, TCH, false, true, REDUX, S16>(hh, hl, pr, wsum, s.bc, s.dA, s.u[pp], n0, nt);
     }
     if constexpr (REDUX) {  // one channel per warp: lane tt finishes step tt
       __syncwarp();
