@@ -54,8 +54,22 @@ L2_FLUSH_BYTES = 512 << 20
 # rounding shift, dt*x*B multiply-add, clamp (2), C*h multiply-accumulate.
 SCAN_OPS_PER_CELL = 6
 SSD_CHUNK = 128  # tokens per chunk of the chunked scan mode
+# fp32 work of one state-cell update of the LQ scan: (dt x) B, the decay
+# multiply-add, the C h multiply-add
+LQ_FLOPS_PER_CELL = 5
 NOMINAL_INT8_OVER_BF16 = 2.0  # 4.5 / 2.25 PFLOP/s dense
 CPU_SAMPLE_MIN_S = 10.0
+# tokens of the all-core oracle sample (per process; one layer)
+CPU_ALLCORE_TOKENS = 512
+
+
+# DRAM bytes per launch of a roofline kernel, from the ncu summaries in
+# profiles/ (named there); None when no capture of the current kernel exists.
+DRAM_TRAFFIC = {}
+
+
+def dram_traffic(kernel: str, args):
+    return DRAM_TRAFFIC.get((kernel, args.workload))
 
 
 def parse(argv=None):
@@ -76,9 +90,44 @@ def parse(argv=None):
     ap.add_argument("--state-spec", default="31,0", choices=["31,0", "16,7"],
                     help="scan state word and increment guard bits: 31,0 the method as built, "
                          "16,7 the narrow state with the guard-bit increment")
+    ap.add_argument("--lq", action="store_true",
+                    help="the FastMamba-LQ variant of a prefill workload (fp32 conv, scan, gate)")
+    ap.add_argument("--modes", default="auto",
+                    help="comma list of sub-records measured after the headline, each a full "
+                         "timed run of the same workload in another mode: static, ssd, state16, "
+                         "lq; 'auto' = all four for the default workload, none otherwise; 'none'")
     ap.add_argument("--layers", type=int, default=None,
                     help="profiling only: run the first N layers of a stack workload")
     return ap.parse_args(argv)
+
+
+SUB_MODES = ("static", "ssd", "state16", "lq")
+
+
+def sub_modes(args) -> list:
+    if args.modes == "none" or args.impl == "reference":
+        return []
+    if args.modes == "auto":
+        return list(SUB_MODES) if args.workload == DEFAULT_WORKLOAD and not args.layers else []
+    out = [m for m in args.modes.split(",") if m]
+    bad = set(out) - set(SUB_MODES)
+    if bad:
+        raise SystemExit(f"bench: unknown --modes {sorted(bad)}")
+    return out
+
+
+def variant_args(args, mode: str):
+    """The arguments of one sub-record: the headline's, with one mode changed."""
+    v = argparse.Namespace(**vars(args))
+    if mode == "static":
+        v.mode = "static"
+    elif mode == "ssd":
+        v.scan_mode = "ssd"
+    elif mode == "state16":
+        v.state_spec = "16,7"
+    elif mode == "lq":
+        v.lq = True
+    return v
 
 
 def n_layers(args) -> int:
@@ -118,6 +167,8 @@ def config_block(args) -> dict:
                              "(GPU, stage by stage)",
                  scan_tile=args.scan_tile or "4,4,16", scan_mode=args.scan_mode,
                  state_spec=args.state_spec)
+        if getattr(args, "lq", False):
+            c.update(variant="FastMamba-LQ (W8A8 linears; fp32 conv, scan, gate)")
         if "prefill_len" in w:
             c.update(prefill_len=w["prefill_len"], step="one decode token per sequence")
     return c
@@ -179,7 +230,7 @@ class OracleSample:
     oracle's cost is linear in tokens and in layers), or a slice of the GEMM's
     rows.  value = sample tokens / (sample seconds x the workload's layers)."""
 
-    def __init__(self, workload: str, mode: str, gemm_m: int = 32768):
+    def __init__(self, workload: str, mode: str, gemm_m: int = 32768, max_tokens: int = 0):
         import oracle as O
         self.O, self.workload = O, workload
         w = S.WORKLOADS[workload]
@@ -188,7 +239,7 @@ class OracleSample:
         n_out, scale = w["n_outliers"], w["outlier_scale"]
         self.layers = w.get("layers", 1)
         if workload == "gemm2p7b_inproj":
-            rows = 128
+            rows = 128 if not max_tokens else min(128, max_tokens)
             self.x = S.activations(1, rows, shape.d_model, seed=11, n_outliers=n_out,
                                    outlier_scale=scale, outlier_seed=OUTLIER_SEED)[0]
             self.wq, self.sw = O.prepare_linear(S.layer_params(shape, 1000)["w_in"])
@@ -214,6 +265,8 @@ class OracleSample:
             return
         B, T = w["batch"], w["seqlen"]
         Ts = min(B * T, 2048 if shape.d_model <= 1024 else 256)  # ~5-10 s a run
+        if max_tokens:
+            Ts = min(Ts, max_tokens)
         self.x = S.activations(1, Ts, shape.d_model, seed=1, n_outliers=n_out,
                                outlier_scale=scale, outlier_seed=OUTLIER_SEED)
         self.tokens = Ts
@@ -251,23 +304,97 @@ class OracleSample:
                 "sample": f"{self.desc}{scaled}; {runs} run(s), {seconds:.2f} s each"}
 
 
+def _oracle_worker(workload, mode, gemm_m, max_tokens, runs, ready, go, out):
+    """One host core's share of the all-core oracle baseline (a spawned
+    process): set up the sample, wait for the common start, time `runs` runs."""
+    o = OracleSample(workload, mode, gemm_m, max_tokens)
+    o.run()
+    ready.wait()
+    go.wait()
+    secs = [o.run() for _ in range(runs)]
+    out.put((secs, o.tokens, o.layers, o.desc))
+
+
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def oracle_all_cores(workload, mode, gemm_m, max_tokens, runs, warmup=0):
+    """The oracle as it stands, one single-threaded process per host core, all
+    running the same bounded sample at once (spawned: no CUDA state is
+    inherited).  Returns (tokens/s of the whole host, per-run wall seconds,
+    cores, tokens of one process's sample, sample description)."""
+    import multiprocessing as mp
+    for v in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS"):
+        os.environ[v] = "1"
+    n = host_cores()
+    ctx = mp.get_context("spawn")
+    ready, go, out = ctx.Barrier(n + 1), ctx.Event(), ctx.Queue()
+    procs = [ctx.Process(target=_oracle_worker,
+                         args=(workload, mode, gemm_m, max_tokens, warmup + runs, ready, go, out))
+             for _ in range(n)]
+    for p in procs:
+        p.start()
+    ready.wait()
+    t0 = time.perf_counter()
+    go.set()
+    res = [out.get() for _ in range(n)]
+    wall = time.perf_counter() - t0
+    for p in procs:
+        p.join()
+    _, tokens, layers, desc = res[0]
+    # every process times its runs; the slowest process's timed runs set the
+    # host's rate (the warm-up runs share the common window but are not counted)
+    timed = max(sum(r[0][warmup:]) for r in res)
+    value = n * runs * tokens / (timed * layers)
+    return value, timed / runs, n, tokens, desc
+
+
+def cpu_baseline(args) -> dict:
+    """Rank 0, one GPU: the oracle on the host cores.  `value`/`cores` are
+    the all-core figure (one oracle process per core); the single-threaded
+    oracle's own figure is kept beside it."""
+    one = OracleSample(args.workload, args.mode, args.gemm_m).measure()
+    val, per_run, n, _, desc = oracle_all_cores(args.workload, args.mode, args.gemm_m,
+                                                CPU_ALLCORE_TOKENS, runs=1)
+    layers = S.WORKLOADS[args.workload].get("layers", 1)
+    scaled = "" if layers == 1 else f", scaled to {layers} layers"
+    return {"value": val, "unit": "tokens/s", "cores": n, "kind": "oracle",
+            "sample": f"{n} processes (one per host core) each running {desc}{scaled}, "
+                      f"concurrently; {per_run:.2f} s per run",
+            "single_thread": one}
+
+
 def run_reference(args):
-    """--impl reference: the CPU oracle on this host's cores (rank 0 only);
-    each step is the bounded sample of the chosen workload."""
+    """--impl reference: the CPU oracle as it stands on this host's cores
+    (rank 0 only).  One timed step = one bounded sample of the workload, run
+    concurrently by one oracle process per core; `value` extrapolates the
+    sample to the whole workload (the oracle's cost is linear in layers and
+    tokens: factor `extrapolation`), and `ms_per_step` is the wall time of
+    the sample that was actually timed."""
     if int(os.environ.get("RANK", "0")) != 0:
         return
-    o = OracleSample(args.workload, args.mode, args.gemm_m)
-    for _ in range(args.warmup):
-        o.run()
-    secs = [o.run() for _ in range(max(1, args.steps))]
-    mean_s = statistics.mean(secs)
-    value = o.value(mean_s)
+    steps = max(1, args.steps)
+    value, per_run, n, o_tokens, desc = oracle_all_cores(args.workload, args.mode, args.gemm_m,
+                                                         CPU_ALLCORE_TOKENS, runs=steps,
+                                                         warmup=args.warmup)
+    layers = S.WORKLOADS[args.workload].get("layers", 1)
+    factor = layers * workload_tokens(args) / (n * o_tokens)
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
-            "n_gpus": args.gpus, "steps": len(secs), "warmup": args.warmup,
-            "ms_per_step": 1000.0 * workload_tokens(args) / value, "higher_is_better": True,
+            "n_gpus": args.gpus, "steps": steps, "warmup": args.warmup,
+            "ms_per_step": 1000.0 * per_run, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "int8/int32 fixed point (CPU oracle)",
             "data": "synthetic", "config": config_block(args),
-            "cpu_baseline": o.describe(mean_s, len(secs)),
+            "step": f"one sample per host core: {desc}, {n} cores",
+            "extrapolation": {"factor": factor,
+                              "basis": "value = sample tokens x cores / (sample wall x layers); "
+                                       "one full workload step is `factor` times the timed "
+                                       "sample's work"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": n, "kind": "oracle",
+                             "sample": f"{desc}, one process per core, {steps} timed runs"},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -579,11 +706,85 @@ class GemmWorkload:
                 "algorithmic": f"2 M N K = {ops:.4g} int8 ops per launch"}
 
 
+class LqStackWorkload(StackWorkload):
+    """The FastMamba-LQ variant of a prefill workload: the same calibrated
+    layers, W8A8 linears and scales, the conv, scan and gate in fp32.  The
+    timed step calls the stage entry points in the order fm_lq_mixer_prefill
+    composes them (checked bit for bit against it), events around each
+    layer's scan."""
+
+    launches_per_layer = 6  # FWHT+quant, in_proj, conv, scan (+ gate), norm+FWHT+quant, out_proj
+
+    def __init__(self, args, torch, lib, dev, rank):
+        super().__init__(args, torch, lib, dev, rank)
+        d, M = self.shape, self.B * self.T
+        e = lambda *sh: torch.empty(sh, dtype=torch.float32, device=dev)
+        self.lbuf = dict(Y=e(M, d.n_in), xo=e(M, d.conv_ch), g=e(M, d.d_inner))
+        self.ws = self.layers[0].lq_workspace(self.B, self.T)
+        self.ssd = False
+        self.sws = None
+        _, extra = _gemm_workspace(torch, lib, d, M, dev)
+        self.launches = (self.launches_per_layer + extra) * self.n_layers
+
+    def step(self, ev=None):
+        lib, d, B, T, b, lb = self.lib, self.shape, self.B, self.T, self.buf, self.lbuf
+        di, cc = d.d_inner, d.conv_ch
+        stream = self.torch.cuda.current_stream(self.dev)
+        src = self.x0
+        for i, Ly in enumerate(self.layers):
+            lib.hadamard_quant(src, d.d_model, Ly.prenorm_w, 1, self.mode, Ly.static_amax,
+                               b["q_in"], b["sx_in"])
+            lib.w8a8_gemm(b["q_in"], b["sx_in"], Ly.w_in_q, Ly.w_in_s, lb["Y"], ws=self.gws)
+            lib.lq_conv1d(lb["Y"][:, di:di + cc], B, T, d, Ly.conv_w, Ly.conv_b, None, lb["xo"])
+            if ev is not None:
+                ev[i][0].record(stream)
+            lib.lq_scan(lb["xo"], lb["Y"][:, di + cc:], lb["Y"][:, :di], B, T, d, Ly.dt_bias,
+                        Ly.a_log, Ly.D, None, lb["g"])
+            if ev is not None:
+                ev[i][1].record(stream)
+            lib.hadamard_quant(lb["g"], di, Ly.norm_w, 1, self.mode, Ly.static_amax[1:],
+                               b["q_out"], b["sx_out"])
+            lib.w8a8_gemm(b["q_out"], b["sx_out"], Ly.w_out_q, Ly.w_out_s, self.r,
+                          residual=src if self.stack_mode else None, ws=self.gws)
+            src = self.r
+
+    def _public(self, x, out):
+        if self.stack_mode:
+            if out is not x:
+                out.copy_(x)
+            for Ly in self.layers:
+                Ly.lq_prefill(out, residual=True, out=out, ws=self.ws)
+            return out
+        return self.layers[0].lq_prefill(x, out=out, ws=self.ws)
+
+    def public_output(self):
+        return self._public(self.x0, self.torch.empty_like(self.x0))
+
+    def e2e_step(self):
+        self.xd.copy_(self.xh, non_blocking=True)
+        self._public(self.xd, self.od)
+        self.oh.copy_(self.od, non_blocking=True)
+
+    def roofline(self, dom_ms, peaks):
+        d = self.shape
+        cells = self.B * d.nheads * d.headdim * d.d_state * self.T
+        achieved = cells * LQ_FLOPS_PER_CELL / (dom_ms / 1e3) / 1e12
+        mhz = (peaks or {}).get("sm_max_mhz", 1965.0)
+        peak = 148 * 128 * 2 * mhz * 1e6 / 1e12
+        return {"bound": "alu", "kernel": "fm_lq_scan (k_lq_scan)", "achieved": achieved,
+                "peak": peak, "unit": "TFLOP/s (fp32)", "frac": achieved / peak, "traffic": None,
+                "peak_basis": f"derived: 148 SMs x 128 fp32 FMA lanes x 2 flops x {mhz:.0f} MHz",
+                "algorithmic": f"{LQ_FLOPS_PER_CELL} fp32 flops per state-cell update x {cells} "
+                               "updates per launch"}
+
+
 def make_workload(args, torch, lib, dev, rank):
     if args.workload == "gemm2p7b_inproj":
         return GemmWorkload(args, torch, lib, dev, rank)
     if args.workload == "decode2p7b_64l_b64":
         return DecodeWorkload(args, torch, lib, dev, rank)
+    if getattr(args, "lq", False):
+        return LqStackWorkload(args, torch, lib, dev, rank)
     return StackWorkload(args, torch, lib, dev, rank)
 
 
@@ -593,6 +794,89 @@ def max_over_ranks(torch, dist, world, value, dev) -> float:
     if world > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def measure(args, wl, torch, dist, lib, dev, world, flush) -> dict:
+    """W untimed warm-up steps, then K timed steps bracketed by a barrier and
+    synchronize on both sides (CUDA events on the launching stream, L2
+    flushed before each), then K end-to-end steps through the public API with
+    host copies.  Times are the max over ranks."""
+    stream = torch.cuda.current_stream(dev)
+    # the stage-by-stage step must equal the public entry points bit for bit
+    ref = wl.public_output()
+    wl.step()
+    torch.cuda.synchronize()
+    lib.sync_status()
+    if ref is not None and not torch.equal(ref, wl.output()):
+        raise SystemExit("bench: stage-by-stage step differs from the public entry points")
+    for _ in range(args.warmup):
+        wl.step()
+    torch.cuda.synchronize()
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    dev_ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(wl.n_layers)] for _ in range(args.steps)]
+    clocks = ClockSampler(dev.index or 0)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    for k in range(args.steps):
+        flush.zero_()
+        torch.cuda.nvtx.range_push("bench_step")
+        ev[k][0].record(stream)
+        wl.step(dev_ev[k])
+        ev[k][1].record(stream)
+        torch.cuda.nvtx.range_pop()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if world > 1:
+        dist.barrier()
+    lib.sync_status()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    dom_ms = [a.elapsed_time(b) for row in dev_ev for a, b in row]
+    total_ms = max_over_ranks(torch, dist, world, sum(step_ms), dev)
+    value = world * wl.tokens * args.steps / (total_ms / 1000.0)
+    roofline = wl.roofline(statistics.mean(dom_ms), measured_peaks())
+    roofline["avg_launch_us"] = 1000.0 * statistics.mean(dom_ms)
+    roofline["share_of_step"] = sum(dom_ms) / sum(step_ms)
+    roofline["traffic"] = dram_traffic(roofline["kernel"], args)
+
+    # end to end through the public API: pinned host input -> device, the
+    # computation, device -> pinned host output, every step
+    wl.e2e_setup()
+    for _ in range(2):
+        wl.e2e_step()
+    torch.cuda.synchronize()
+    e2e_ms = []
+    for _ in range(args.steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        wl.e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms.append(a.elapsed_time(b))
+    lib.sync_status()
+    if ref is not None and not wl.e2e_matches(ref):
+        raise SystemExit("bench: end-to-end output differs from the device-resident step")
+    e2e_total = max_over_ranks(torch, dist, world, sum(e2e_ms), dev)
+    e2e_value = world * wl.tokens * args.steps / (e2e_total / 1000.0)
+    return {"value": value, "ms_per_step": total_ms / args.steps, "roofline": roofline,
+            "clocks": clk,
+            "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": wl.h2d_bytes,
+                    "d2h_bytes_per_step": wl.d2h_bytes},
+            "gpu_launches": wl.launches * args.steps}
+
+
+def apply_modes(args, lib):
+    """Process-wide library settings of one run (scan tile, scan mode, state spec)."""
+    if args.scan_tile:
+        lib.set_scan_tile(*[int(v) for v in args.scan_tile.split(",")])
+    lib.set_scan_mode(args.scan_mode)
+    lib.set_state_spec(*[int(v) for v in args.state_spec.split(",")])
 
 
 def main():
@@ -618,93 +902,42 @@ def main():
     if world > 1:
         dist.barrier()
     lib.load()
-    if args.scan_tile:
-        lib.set_scan_tile(*[int(v) for v in args.scan_tile.split(",")])
-    lib.set_scan_mode(args.scan_mode)
-    lib.set_state_spec(*[int(v) for v in args.state_spec.split(",")])
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    stream = torch.cuda.current_stream(dev)
-    wl = make_workload(args, torch, lib, dev, rank)
-
-    # the stage-by-stage step must equal the public entry points bit for bit
-    ref = wl.public_output()
-    wl.step()
-    torch.cuda.synchronize()
-    lib.sync_status()
-    if ref is not None and not torch.equal(ref, wl.output()):
-        raise SystemExit("bench: stage-by-stage step differs from the public entry points")
-
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    for _ in range(args.warmup):
-        wl.step()
-    torch.cuda.synchronize()
 
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(args.steps)]
-    dev_ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(wl.n_layers)] for _ in range(args.steps)]
-    clocks = ClockSampler(local)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    clocks.start()
-    time.sleep(0.3)
-    for k in range(args.steps):
-        flush.zero_()
-        torch.cuda.nvtx.range_push("bench_step")
-        ev[k][0].record(stream)
-        wl.step(dev_ev[k])
-        ev[k][1].record(stream)
-        torch.cuda.nvtx.range_pop()
-    torch.cuda.synchronize()
-    clk = clocks.stop()
-    if world > 1:
-        dist.barrier()
-    lib.sync_status()
-    step_ms = [a.elapsed_time(b) for a, b in ev]
-    dom_ms = [a.elapsed_time(b) for row in dev_ev for a, b in row]
-    total_ms = max_over_ranks(torch, dist, world, sum(step_ms), dev)
-    value = world * wl.tokens * args.steps / (total_ms / 1000.0)
-    roofline = wl.roofline(statistics.mean(dom_ms), measured_peaks())
-    roofline["avg_launch_us"] = 1000.0 * statistics.mean(dom_ms)
-    roofline["share_of_step"] = sum(dom_ms) / sum(step_ms)
-
-    # end to end through the public API: pinned host input -> device, the
-    # computation, device -> pinned host output, every step
-    wl.e2e_setup()
-    for _ in range(2):
-        wl.e2e_step()
-    torch.cuda.synchronize()
-    e2e_ms = []
-    for _ in range(args.steps):
-        flush.zero_()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        wl.e2e_step()
-        b.record(stream)
-        torch.cuda.synchronize()
-        e2e_ms.append(a.elapsed_time(b))
-    lib.sync_status()
-    if ref is not None and not wl.e2e_matches(ref):
-        raise SystemExit("bench: end-to-end output differs from the device-resident step")
-    e2e_total = max_over_ranks(torch, dist, world, sum(e2e_ms), dev)
-    e2e_value = world * wl.tokens * args.steps / (e2e_total / 1000.0)
+    apply_modes(args, lib)
+    wl = make_workload(args, torch, lib, dev, rank)
+    head = measure(args, wl, torch, dist, lib, dev, world, flush)
+    del wl
+    subs = {}
+    for m in sub_modes(args):
+        va = variant_args(args, m)
+        apply_modes(va, lib)
+        torch.cuda.empty_cache()
+        w2 = make_workload(va, torch, lib, dev, rank)
+        r = measure(va, w2, torch, dist, lib, dev, world, flush)
+        del w2
+        r["config"] = {k: v for k, v in config_block(va).items()
+                       if config_block(args).get(k) != v}
+        subs[m] = r
+    apply_modes(args, lib)
 
     if rank == 0:
         cpu = None
         if not args.no_cpu_baseline and world == 1:
-            cpu = OracleSample(args.workload, args.mode, args.gemm_m).measure()
-        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
-                "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+            cpu = cpu_baseline(args)
+        line = {"metric": METRIC, "value": head["value"], "unit": "tokens/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-                "dtype": "int8 x int8 -> int32 GEMM + int32 fixed point",
+                "dtype": "int8 x int8 -> int32 GEMM + int32 fixed point"
+                         if not args.lq else "int8 x int8 -> int32 GEMM + fp32 conv/scan/gate",
                 "data": "synthetic (seeded outlier-injected N(0,1), random-init weights)",
-                "config": config_block(args), "roofline": roofline, "cpu_baseline": cpu,
-                "clocks": clk,
-                "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": wl.h2d_bytes,
-                        "d2h_bytes_per_step": wl.d2h_bytes},
-                "gpu_launches": wl.launches * args.steps}
+                "config": config_block(args), "roofline": head["roofline"],
+                "cpu_baseline": cpu, "clocks": head["clocks"], "e2e": head["e2e"],
+                "gpu_launches": head["gpu_launches"]}
+        if subs:
+            line["modes"] = subs
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()

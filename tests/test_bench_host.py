@@ -90,3 +90,33 @@ def test_reference_arm_line():
     assert line["impl"] == "reference" and line["cpu_baseline"]["kind"] == "oracle"
     assert line["cpu_baseline"]["value"] == line["value"] == line["e2e"]["value"]
     assert line["e2e"]["h2d_bytes_per_step"] == 0
+    # what was timed: one sample per host core, and the factor to a full step
+    cores = line["cpu_baseline"]["cores"]
+    assert cores == bench.host_cores() >= 1
+    ex = line["extrapolation"]
+    assert ex["factor"] == pytest.approx(256 / (cores * min(256, bench.CPU_ALLCORE_TOKENS)))
+    # the reported step time is the timed sample's, consistent with value
+    per_core_tokens = min(256, bench.CPU_ALLCORE_TOKENS)
+    assert line["value"] == pytest.approx(cores * per_core_tokens / (line["ms_per_step"] / 1e3),
+                                          rel=1e-6)
+
+
+def test_sub_record_modes():
+    """The headline runs alone except on the default workload, where the
+    static, chunked-scan, 16-bit-state and LQ modes follow as sub-records;
+    each sub-record differs from the headline in exactly one setting."""
+    a = bench.parse([])
+    assert bench.sub_modes(a) == ["static", "ssd", "state16", "lq"]
+    assert bench.sub_modes(bench.parse(["--modes", "none"])) == []
+    assert bench.sub_modes(bench.parse(["--workload", "stack2p7b_64l_b2_t4096"])) == []
+    assert bench.sub_modes(bench.parse(["--workload", "stack2p7b_64l_b2_t4096",
+                                        "--modes", "ssd"])) == ["ssd"]
+    with pytest.raises(SystemExit):
+        bench.sub_modes(bench.parse(["--modes", "fast"]))
+    base = bench.config_block(a)
+    for m, key in (("static", "act_quant"), ("ssd", "scan_mode"), ("state16", "state_spec"),
+                   ("lq", "variant")):
+        v = bench.variant_args(a, m)
+        diff = {k for k, x in bench.config_block(v).items() if base.get(k) != x}
+        assert diff == {key}, (m, diff)
+    assert not a.lq and a.mode == "dynamic"          # the headline's args are untouched
