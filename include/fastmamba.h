@@ -108,7 +108,11 @@ fm_exp_layout fm_exp_table_layout(const fm_shape *shape);
 /* ------------------------------------------------------------------ */
 /* a0 + a1 / a10: (pre-RMSNorm) + Hadamard rotation + int8 quantisation */
 /* ------------------------------------------------------------------ */
-/* x [M, K] fp32 -> q [M, K] int8 codes and s_x [M] fp32 scales, so that
+/* Source: Y = (XH)(H^T W^T) with H orthonormal after 1/sqrt(n) (pith.science review of FastMamba,
+ * "What carries the argument"); the scale from the max of the rotated tensor
+ * (Referee Report, major comment 1, on Algorithm 1 and Fig. 6); the stack's
+ * pre-RMSNorm is Mamba2's (the paper's reference [10], Figure 2 caption).
+ * x [M, K] fp32 -> q [M, K] int8 codes and s_x [M] fp32 scales, so that
  * dequant = q * s_x[row] approximates (RMSNorm(x) * prenorm_w) H_bd.
  *   prenorm_w  [K] or NULL: apply RMSNorm (eps 1e-5, fixed summation order)
  *              and this weight before rotating (stack layers).
@@ -121,7 +125,8 @@ fm_status fm_hadamard_quant(const float *x, int64_t M, int64_t K, const float *p
                             int rotate, int mode, const float *static_amax, int8_t *q,
                             float *s_x, float *amax_row, fm_stream stream);
 
-/* Offline: W [N, K] fp32 -> Wq [N, K] int8 and s_w [N] fp32 with
+/* Source: the pre-rotated weight H^T W^T of "What carries the argument" (pith.science review of FastMamba).
+ * Offline: W [N, K] fp32 -> Wq [N, K] int8 and s_w [N] fp32 with
  * W' = W H_bd (fp64), s_w = max|W'[n,:]| / 127, Wq = rint(W' / s_w). */
 fm_status fm_prepare_linear(const float *W, int64_t N, int64_t K, int rotate, int8_t *Wq,
                             float *s_w, fm_stream stream);
@@ -129,7 +134,10 @@ fm_status fm_prepare_linear(const float *W, int64_t N, int64_t K, int rotate, in
 /* ------------------------------------------------------------------ */
 /* a2 + a3 / a11: W8A8 GEMM on the tensor cores + dequantisation        */
 /* ------------------------------------------------------------------ */
-/* Y[m,n] = fl(fl(float(acc[m,n]) * s_x[m]) * s_w[n]) (+ residual[m,n]),
+/* Source: the 8-bit linear layers, (XH)(H^T W^T) computed as an int8 product
+ * and dequantised (pith.science review of FastMamba, "What carries the argument"; Referee
+ * major comment 1 on Algorithm 1).
+ * Y[m,n] = fl(fl(float(acc[m,n]) * s_x[m]) * s_w[n]) (+ residual[m,n]),
  * acc = sum_k A[m,k] Wq[n,k] (exact int32).
  *   A [M, K] int8, Wq [N, K] int8 (both K-major), residual [M, N] or NULL
  *   (may alias Y), acc_out [M, N] int32 or NULL (raw accumulators).
@@ -138,7 +146,10 @@ fm_status fm_w8a8_gemm(const int8_t *A, const float *s_x, int64_t M, const int8_
                        const float *s_w, int64_t N, int64_t K, const float *residual, float *Y,
                        int32_t *acc_out, fm_stream stream);
 
-/* in_proj: the same GEMM (N = n_in, K = d_model) with the split epilogue:
+/* Source: as fm_w8a8_gemm; the column split z | x | B | C | dt is Mamba2's
+ * in_proj (the paper's reference [2]; Figure 2 caption), the xBC columns
+ * quantised to the conv's power-of-two codes ("What carries the argument").
+ * in_proj: the same GEMM (N = n_in, K = d_model) with the split epilogue:
  *   z   [M, d_inner] fp32   (columns [0, di))
  *   xbc [M, conv_ch] int8   (columns [di, di+cc)): satb(rint(y * 2^-e_u[c]), 8)
  *   dt  [M, nheads] fp32    (columns [di+cc, n_in))
@@ -166,7 +177,10 @@ fm_status fm_in_proj_ws(const int8_t *A, const float *s_x, int64_t M, const int8
 /* ------------------------------------------------------------------ */
 /* a4: power-of-two causal depthwise conv1d (kernel 4) + SiLU           */
 /* ------------------------------------------------------------------ */
-/* u [B, T, cc] int8 codes at e_u -> out [B, T, cc] int8 codes at e_o:
+/* Source: fine-grained power-of-two quantisation of the convolution (pith.science review of FastMamba,
+ * "What carries the argument"; original abstract); SiLU through the shared
+ * 2^v unit (Figure 7 caption: the nonlinear approximation unit).
+ * u [B, T, cc] int8 codes at e_u -> out [B, T, cc] int8 codes at e_o:
  *   acc = bq[c] + sum_{k=0..3} wq[c,k] u[t-3+k, c]   (tap 3 = current token)
  *   x16 = satb(rshr(acc, -(e_w+e_u+16)), 32); s = SiLU_pwl(x16)
  *   out = satb(rshr(s, e_o + 16), 8)
@@ -192,7 +206,12 @@ fm_status fm_set_scan_tile(int npt, int pc, int tch);
  * dt*x factor and the skip term, B and C widened). */
 size_t fm_scan_workspace_bytes(const fm_shape *shape, int B, int T);
 
-/* xbc [B, T, cc] int8 conv output (x | B | C), dt_raw [B, T, nh] fp32.
+/* Source: power-of-two fixed point for the SSM block and the 8-segment
+ * first-order 2^v with e^x = 2^(x log2 e) and SoftPlus(x) = x + SoftPlus(-x)
+ * (pith.science review of FastMamba, "What carries the argument"; Referee minor comment 5 on
+ * Eq. (5)); the recurrence and C.h + D.x are Mamba2's SSM (Figure 2 and
+ * Figure 7 captions; the paper's reference [2]).
+ * xbc [B, T, cc] int8 conv output (x | B | C), dt_raw [B, T, nh] fp32.
  * Per token and head (Q.16): dt_q = SoftPlus_pwl(to_q16(dt_raw + dt_bias)),
  * dA_q = 2^(-rshr(dt_q * A_q, 12)).  Per (b, h, p, n), t in order:
  *   u = satb(rshr(dt_q x[p], e_h - e_B - e_x + 16), 24)
@@ -211,7 +230,10 @@ fm_status fm_ssm_scan_pot(const int8_t *xbc, const float *dt_raw, int B, int T,
 /* ------------------------------------------------------------------ */
 /* a9 + a10: gate, gated RMSNorm, rotation, int8 quantisation           */
 /* ------------------------------------------------------------------ */
-/* y [M, di] int32 (at e_y per head), z [M, di] fp32 -> q [M, di] int8, s_x [M]:
+/* Source: Mamba2's gate and gated RMSNorm before out_proj (Figure 2 caption;
+ * the paper's references [2], [10], [11]) with the SiLU through the 2^v unit,
+ * then the out_proj input's rotation and int8 codes as fm_hadamard_quant.
+ * y [M, di] int32 (at e_y per head), z [M, di] fp32 -> q [M, di] int8, s_x [M]:
  *   g = y SiLU_pwl(to_q16(z)); g_q = satb(rshr(g, e_g - e_y + 16), 16)
  *   rstd = 1/sqrt(sum g_q^2 2^(2 e_g) / di + 1e-5) (exact integer sum)
  *   o = g_q 2^e_g rstd norm_w, then as fm_hadamard_quant. */
@@ -276,7 +298,10 @@ fm_status fm_ssd_scan(const int8_t *xbc, const float *dt_raw, int B, int T,
                       const fm_shape *shape, const float *dt_bias, const int32_t *A_q,
                       const int32_t *D_q, const int32_t *exps, int32_t *state, int32_t *y,
                       void *ws, size_t ws_bytes, fm_stream stream);
-/* Process-wide state spec of every scan entry point and of the calibration:
+/* Source: the pages give the SSM block "fine-grained" power-of-two scales but
+ * neither the state's word width nor the granularity (pith.science review of
+ * FastMamba, "What carries the argument"); this selects between two readings.
+ * Process-wide state spec of every scan entry point and of the calibration:
  * (31, 0), the default, is the method as built -- an int32 state clamped at
  * +-(2^30 - 1), the increment u B with u rounded first.  (16, 7) is the narrow
  * reading: the state clamps at +-32767 and is stored as int16 -- every
@@ -290,7 +315,10 @@ fm_status fm_set_state_spec(int bits, int guard);
 /* Workspace bytes fm_mixer_prefill / fm_decode_step need for B*T tokens. */
 size_t fm_workspace_bytes(const fm_shape *shape, int B, int T);
 
-/* One mixer layer on x [B, T, d_model] fp32 -> out [B, T, d_model] fp32.
+/* Source: the Mamba2 block of Figure 2's caption (in_proj -> conv1d + SiLU
+ * -> SSM -> gate + RMSNorm -> out_proj) under the three pieces of "What
+ * carries the argument" (pith.science review of FastMamba); a0-a11 in order.
+ * One mixer layer on x [B, T, d_model] fp32 -> out [B, T, d_model] fp32.
  *   residual 1: out = x + mixer(x) (stack layer; out may alias x).
  *   conv_state [B, 3, conv_ch] int8 / ssm_state [B, nh, hd, ds] int32, or
  *   NULL: carried state in/out (prefill in chunks is bit-identical to one pass).
@@ -301,7 +329,10 @@ fm_status fm_mixer_prefill(const fm_layer *L, const float *x, int B, int T, int 
                            int8_t *conv_state, int32_t *ssm_state, float *out, void *ws,
                            size_t ws_bytes, fm_stream stream);
 
-/* Single-token decode step for B sequences: x [B, d_model] -> out [B, d_model],
+/* Source: the 2.7B decode figures of the review's Table III discussion
+ * (pith.science review of FastMamba, "What carries the argument"); Mamba2's recurrent form
+ * (the paper's reference [2]): a prefill of one token with states carried.
+ * Single-token decode step for B sequences: x [B, d_model] -> out [B, d_model],
  * updating conv_state and ssm_state (both required). */
 fm_status fm_decode_step(const fm_layer *L, const float *x, int B, int residual,
                          int8_t *conv_state, int32_t *ssm_state, float *out, void *ws,
@@ -389,7 +420,11 @@ fm_status fm_lq_mixer_prefill(const fm_layer *L, const fm_lq_params *P, const fl
                               int T, int residual, float *conv_state, float *ssm_state,
                               float *out, void *ws, size_t ws_bytes, fm_stream stream);
 
-/* Offline, per layer: quantise conv taps (e_w, wq) and the SSM parameters
+/* Source: power-of-two codes for the conv weights and the SSM parameters;
+ * A folded with log2(e) for the shift-based e^Delta (pith.science review of
+ * FastMamba, "What carries the argument"; the verdict record's supporting
+ * citation [15]).
+ * Offline, per layer: quantise conv taps (e_w, wq) and the SSM parameters
  * (A_q, D_q, e_D) from fp32 device tensors: conv_w [cc, 4], a_log [nh], D [nh].
  * Writes the e_w and e_D regions of `exps`. */
 fm_status fm_prepare_mixer_params(const fm_shape *shape, const float *conv_w, const float *a_log,
@@ -399,7 +434,11 @@ fm_status fm_prepare_mixer_params(const fm_shape *shape, const float *conv_w, co
 /* Calibration workspace bytes for B*T calibration tokens. */
 size_t fm_calib_workspace_bytes(const fm_shape *shape, int B, int T);
 
-/* Stage-by-stage calibration of one prepared layer on xcal [B, T, d_model]:
+/* Source: the static scales the hardware applies as "x s_coe >> s_shift"
+ * (pith.science review of FastMamba, Referee major comment 1 on Fig. 6); the
+ * pages do not say how they are found, so each stage's exponent is taken from
+ * that stage's maximum on the calibration tokens.
+ * Stage-by-stage calibration of one prepared layer on xcal [B, T, d_model]:
  * fills the remaining regions of exps (e_u, e_o, e_x, e_B, e_C, e_h, e_y,
  * e_g), conv_bq (from conv_b [cc] fp32 at e_w + e_u) and static_amax[2],
  * and writes the layer's output on xcal to out (next layer's calibration
