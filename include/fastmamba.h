@@ -68,12 +68,25 @@ const char *fm_status_string(fm_status s);
 const char *fm_last_error(void);
 /* Synchronises `stream`, then reads and clears the device error word of the
  * current device: FM_OK, FM_ERR_TIMEOUT (a bounded wait gave up; it takes
- * precedence), FM_ERR_NONFINITE (an activation row entering an int8
+ * precedence; the outputs and the carried states -- ssm_state, conv_state --
+ * of the calls since the last read are then undefined), FM_ERR_NONFINITE (an activation row entering an int8
  * quantiser -- fm_hadamard_quant, fm_gate_norm_quant and the layers that
  * call them -- held a NaN or Inf; that row's codes and scale are then
  * undefined) or FM_ERR_CUDA (the synchronisation itself failed).  The word
  * accumulates over every call on the device since it was last read. */
 fm_status fm_sync_status(fm_stream stream);
+/* Failure injection for tests of the bounded-wait path (the pages have no
+ * counterpart).  On the current device, for every later launch until reset:
+ *   stall_mask bit 0: the GEMM producers issue no loads; bit 1: the
+ *   sequential scan's producer issues no copies.  The consumers then wait on
+ *   a barrier that nothing completes, with no copy or MMA in flight, give up
+ *   after wait_limit_ns, set the device error word (FM_ERR_TIMEOUT at the
+ *   next fm_sync_status) and end; every kernel still frees its TMEM.
+ *   wait_limit_ns: the pipeline waits' limit; 0 = the default (4 s).  Waits
+ *   for work already issued (drains) always use the default.
+ * fm_set_fault_injection(0, 0) restores normal operation.  Synchronous
+ * (cudaMemcpyToSymbol); not for use while the device runs library kernels. */
+fm_status fm_set_fault_injection(int stall_mask, uint64_t wait_limit_ns);
 /* Library ABI version (major * 100 + minor). */
 int fm_version(void);
 

@@ -78,6 +78,18 @@ extern "C" const char *fm_status_string(fm_status s) {
 extern "C" const char *fm_last_error(void) { return tl_msg; }
 extern "C" int fm_version(void) { return 100; }
 
+extern "C" fm_status fm_set_fault_injection(int stall_mask, uint64_t wait_limit_ns) {
+  if (stall_mask & ~(kStallGemm | kStallScan))
+    return fail(FM_ERR_INVALID_ARG, "fm_set_fault_injection: unknown stall bits 0x%x", stall_mask);
+  const unsigned long long lim = wait_limit_ns ? (unsigned long long)wait_limit_ns : kWaitLimitNs;
+  if (lim > kWaitLimitNs)
+    return fail(FM_ERR_INVALID_ARG, "fm_set_fault_injection: limit above the default %llu ns",
+                kWaitLimitNs);
+  FM_CHECK_CUDA(cudaMemcpyToSymbol(g_test_stall, &stall_mask, sizeof(stall_mask)));
+  FM_CHECK_CUDA(cudaMemcpyToSymbol(g_wait_limit_ns, &lim, sizeof(lim)));
+  return FM_OK;
+}
+
 extern "C" fm_status fm_sync_status(fm_stream stream) {
   FM_CHECK_CUDA(cudaStreamSynchronize((cudaStream_t)stream));
   unsigned int word = 0, zero = 0;

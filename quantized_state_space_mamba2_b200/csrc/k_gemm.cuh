@@ -34,6 +34,17 @@ constexpr int kGemmBK = 128;  // int8 elements = bytes per row per stage (one sw
 constexpr int kGemmThreads = 192;
 constexpr unsigned long long kWaitLimitNs = 4000000000ull;  // 4 s
 
+// Failure injection for the tests of the bounded-wait path (set by
+// fm_set_fault_injection; both per device, zero-cost when unset):
+//   g_wait_limit_ns  the limit of the pipeline waits (kWaitLimitNs by default)
+//   g_test_stall     bit 0: the GEMM producers issue no loads; bit 1: the
+//                    scan producer issues no copies -- the consumers then wait
+//                    on a barrier nothing completes, with nothing in flight
+// Drains (waits for work already issued) always use the fixed kWaitLimitNs.
+__device__ unsigned long long g_wait_limit_ns = kWaitLimitNs;
+__device__ int g_test_stall = 0;
+constexpr int kStallGemm = 1, kStallScan = 2;
+
 struct GemmEpilogue {
   int mode;  // 0: plain (Y, residual), 1: in_proj split
   long long M, N;
@@ -87,17 +98,28 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// bounded wait: false (and the error word set) if the phase never completes
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
+// bounded wait: false (and the error word set) if the phase does not
+// complete within `limit` ns
+__device__ __forceinline__ bool mbar_wait_for(uint64_t *bar, uint32_t parity,
+                                              unsigned long long limit) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (globaltimer() - t0 > kWaitLimitNs) {
+    if (globaltimer() - t0 > limit) {
       raise_error(kErrTimeout);
       return false;
     }
   }
+}
+// a pipeline wait (its limit can be lowered for the failure tests)
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return mbar_wait_for(bar, parity, *(volatile unsigned long long *)&g_wait_limit_ns);
+}
+// a drain: waits for work this CTA has already issued, at the fixed limit
+__device__ __forceinline__ bool mbar_drain(uint64_t *bar, uint32_t parity) {
+  return mbar_wait_for(bar, parity, kWaitLimitNs);
 }
 __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *tm, int c0, int c1,
                                             uint64_t *bar) {
@@ -343,14 +365,21 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
 
   if (warp == 0) {
     if (lane == 0) {
-      for (int kb = 0; kb < kb_n; ++kb) {
+      const int kb_issue = (g_test_stall & kStallGemm) ? 0 : kb_n;
+      int issued = 0;
+      for (int kb = 0; kb < kb_issue; ++kb) {
         const int s = kb % STAGES;
         const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
         if (!mbar_wait(&empty_bar[s], ph ^ 1u)) break;
         mbar_arrive_expect_tx(&full_bar[s], (uint32_t)((kGemmBM + BN) * kGemmBK));
         tma_load_2d(sA + s * kGemmBM * kGemmBK, &tmA, (kb0 + kb) * kGemmBK, m0, &full_bar[s]);
         tma_load_2d(sB + s * BN * kGemmBK, &tmB, (kb0 + kb) * kGemmBK, n0, &full_bar[s]);
+        ++issued;
       }
+      // every copy issued must have landed before the CTA may exit (on the
+      // normal path the MMA lane has consumed them all and these return at once)
+      for (int j = issued > STAGES ? issued - STAGES : 0; j < issued; ++j)
+        if (!mbar_drain(&full_bar[j % STAGES], (uint32_t)(j / STAGES) & 1u)) break;
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -371,6 +400,8 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
         mma_commit(&empty_bar[s]);
       }
       mma_commit(accum_bar);
+      // every MMA issued must have completed before TMEM is released
+      mbar_drain(accum_bar, 0);
     }
   } else {
     // while the main loop runs: stage this tile's column scales and the row scale
@@ -386,13 +417,14 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
     const long long row = (long long)m0 + quarter * 32 + lane;
     const float sx = row < ep.M ? ep.s_x[row] : 0.0f;
     asm volatile("bar.sync 1, 128;" ::: "memory");  // the 4 epilogue warps only
-    const bool ok = mbar_wait(accum_bar, 0);
+    // tcgen05.ld is warp-collective: the whole warp skips it after a failed wait
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(accum_bar, 0));
     tc_fence_after();
 #pragma unroll 1
-    for (int c = 0; c < BN; c += 32) {
+    for (int c = 0; c < BN && ok; c += 32) {
       uint32_t r[32];
       tmem_ld32(tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)c, r);
-      if (!ok || n0 + c >= ep.N) continue;
+      if (n0 + c >= ep.N) continue;
       if constexpr (SPLIT) {  // add this slice's exact partial sums
         if (row < ep.M) {
           int32_t *dst = ep.split_acc + row * ep.N + n0 + c;
@@ -631,7 +663,7 @@ __global__ void __launch_bounds__(64 + 32 * EW, 1)
   if (warp == 0) {
     if (lane == 0) {
       long long it = 0;
-      bool ok = true;
+      bool ok = !(g_test_stall & kStallGemm);
       for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
         const int m0 = (t / n_tiles) * kGemmBM, n0 = (t % n_tiles) * BN;
         for (int kb = 0; kb < num_k_blocks; ++kb, ++it) {
@@ -650,7 +682,7 @@ __global__ void __launch_bounds__(64 + 32 * EW, 1)
       // normal path the MMA lane has consumed them all and these return at once)
       const long long first = it > STAGES ? it - STAGES : 0;
       for (long long j = first; j < it; ++j)
-        if (!mbar_wait(&full_bar[j % STAGES], (uint32_t)(j / STAGES) & 1u)) break;
+        if (!mbar_drain(&full_bar[j % STAGES], (uint32_t)(j / STAGES) & 1u)) break;
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -687,7 +719,7 @@ __global__ void __launch_bounds__(64 + 32 * EW, 1)
       }
       // wait for every MMA issued so far before TMEM can be released
       mma_commit(drain_bar);
-      mbar_wait(drain_bar, 0);
+      mbar_drain(drain_bar, 0);
     }
   } else {
     const int e = warp - 2;                 // 0 .. EW-1

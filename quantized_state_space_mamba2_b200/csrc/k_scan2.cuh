@@ -337,7 +337,9 @@ __global__ void __launch_bounds__(PC *(128 / NPT) + 32) k_scan_seq(ScanSeqArgs a
 
   if (warp == NW) {  // ---------------- producer
     if (lane32 == 0) {
-      for (int c = 0; c < nchunks; ++c) {
+      const int nissue = (g_test_stall & kStallScan) ? 0 : nchunks;
+      int issued = 0;
+      for (int c = 0; c < nissue; ++c) {
         const int sl = c % kScanSlots;
         if (c >= kScanSlots &&
             !mbar_wait(&sm.empty[sl], (uint32_t)((c / kScanSlots) - 1) & 1u))
@@ -358,7 +360,12 @@ __global__ void __launch_bounds__(PC *(128 / NPT) + 32) k_scan_seq(ScanSeqArgs a
           bulk_g2s(&s.u[q][0], a.u + off, TCH * 4, &sm.full[sl]);
           bulk_g2s(&s.xs[q][0], a.xs + off, TCH * 4, &sm.full[sl]);
         }
+        ++issued;
       }
+      // no copy may outlive the CTA: wait (fixed limit) for the chunks still
+      // in flight (on the normal path they have landed and these return at once)
+      for (int c = issued > kScanSlots ? issued - kScanSlots : 0; c < issued; ++c)
+        if (!mbar_drain(&sm.full[c % kScanSlots], (uint32_t)(c / kScanSlots) & 1u)) break;
     }
     return;
   }

@@ -216,7 +216,7 @@ __global__ void __launch_bounds__(kSsdThreads) k_ssd_state(SsdArgs a) {
     }
     mma_commit(bar);
   }
-  const bool ok = mbar_wait(bar, 0);
+  const bool ok = mbar_drain(bar, 0);
   tc_fence_after();
   // TMEM lane n = t holds dH^T row n: 64 columns p
   float *dst = a.dH + (bh * a.nch + c) * (kSsdHd * kSsdDs) + t;
@@ -403,7 +403,7 @@ __global__ void __launch_bounds__(kSsdThreads) k_ssd_out(SsdArgs a) {
     for (int k = 0; k < 4; ++k) mma_i8(tmem, ad + (uint64_t)(2 * k), bd + (uint64_t)(2 * k), idesc, k > 0 ? 1u : 0u);
     mma_commit(&bar[0]);
   }
-  bool ok = mbar_wait(&bar[0], 0);
+  bool ok = mbar_drain(&bar[0], 0);
   tc_fence_after();
   {  // row t of M: bf16(G[t][s] * fl32(2^(W[t]-W[s]) dt[s])) for s <= t, else 0
     const long long Wt = sW[t];
@@ -457,7 +457,7 @@ __global__ void __launch_bounds__(kSsdThreads) k_ssd_out(SsdArgs a) {
     }
     mma_commit(&bar[1]);
   }
-  ok = mbar_wait(&bar[1], 0) && ok;
+  ok = mbar_drain(&bar[1], 0) && ok;
   tc_fence_after();
   {  // y codes of token t: rint(Y 2^(e_C+e_x+e_B-e_y)) + rshr(D_q x, s_D), saturated
     const int s_y = *a.e_C + a.e_x[h] + *a.e_B - a.e_y[h];

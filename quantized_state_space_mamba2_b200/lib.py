@@ -30,7 +30,7 @@ EXPORTS = (
     "fm_calibrate_layer", "fm_decode_step_noalloc", "fm_scan_workspace_bytes",
     "fm_set_scan_tile", "fm_ssd_workspace_bytes", "fm_ssd_scan", "fm_set_scan_mode",
     "fm_set_state_spec", "fm_lq_conv1d", "fm_lq_scan", "fm_lq_workspace_bytes",
-    "fm_lq_mixer_prefill",
+    "fm_lq_mixer_prefill", "fm_set_fault_injection",
 )
 NOALLOC_SCRATCH_BYTES = 16 << 20  # FM_NOALLOC_SCRATCH_BYTES
 
@@ -113,6 +113,7 @@ def load():
         "fm_lq_conv1d": (I, [_P, I64, I, I, sp, _P, _P, _P, _P, _P]),
         "fm_lq_scan": (I, [_P, _P, I64, _P, I64, I, I, sp, _P, _P, _P, _P, _P, _P]),
         "fm_lq_workspace_bytes": (SZ, [sp, I, I]),
+        "fm_set_fault_injection": (I, [I, C.c_uint64]),
         "fm_lq_mixer_prefill": (I, [lp, C.POINTER(fm_lq_params), _P, I, I, I, _P, _P, _P, _P,
                                     SZ, _P]),
     }
@@ -155,6 +156,15 @@ def exp_table_layout(shape) -> fm_exp_layout:
 
 def sync_status(stream=None):
     _check(load().fm_sync_status(_s(stream)))
+
+
+STALL_GEMM, STALL_SCAN = 1, 2
+
+
+def set_fault_injection(stall_mask: int, wait_limit_ns: int = 0):
+    """Test hook: producers that issue nothing (STALL_GEMM, STALL_SCAN) and a
+    shorter pipeline-wait limit; (0, 0) restores normal operation."""
+    _check(load().fm_set_fault_injection(stall_mask, wait_limit_ns))
 
 
 def hadamard_quant(x, K, prenorm_w, rotate, mode, static_amax, q, s_x, amax_row=None, stream=None):
