@@ -179,6 +179,11 @@ fm_status fm_in_proj(const int8_t *A, const float *s_x, int64_t M, const int8_t 
  * points (fm_mixer_prefill, fm_decode_step) do this from their own workspace.
  * ws may be NULL (no split) when fm_gemm_workspace_bytes returns 0. */
 size_t fm_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
+/* Process-wide switch of the split-K path above: 0 (default) never splits
+ * (fm_gemm_workspace_bytes then returns 0 and the layer workspaces hold no
+ * partial sums), 1 splits small grids.  Set it before sizing workspaces and
+ * keep it while they are in use.  FM_ERR_INVALID_ARG for other values. */
+fm_status fm_set_gemm_splitk(int enable);
 fm_status fm_w8a8_gemm_ws(const int8_t *A, const float *s_x, int64_t M, const int8_t *Wq,
                           const float *s_w, int64_t N, int64_t K, const float *residual,
                           float *Y, int32_t *acc_out, void *ws, size_t ws_bytes,

@@ -256,8 +256,22 @@ static int gemm_splits(long long M, long long N, long long K, int BN, int sms, i
   *kbs = (int)((nkb + S - 1) / S);
   return (nkb + *kbs - 1) / *kbs;
 }
+// Split-K of the small-grid GEMMs, process-wide: off by default (measured
+// slower than the unsplit kernel at the 130M out_proj and the 2.7B decode
+// GEMMs: the per-element atomics and the separate dequantising pass cost more
+// than the extra CTAs gain).
+static std::atomic<int> g_gemm_splitk{0};
+
+extern "C" fm_status fm_set_gemm_splitk(int enable) {
+  if (enable != 0 && enable != 1)
+    return fail(FM_ERR_INVALID_ARG, "fm_set_gemm_splitk: enable must be 0 or 1");
+  g_gemm_splitk.store(enable, std::memory_order_relaxed);
+  return FM_OK;
+}
+
 // the small-grid path would split this GEMM (the workspace must hold M x N int32)
 static bool gemm_would_split(long long M, long long N, long long K) {
+  if (!g_gemm_splitk.load(std::memory_order_relaxed)) return false;
   const int sms = sm_count();
   const long long mt = (M + kGemmBM - 1) / kGemmBM;
   if (K % kGemmBK || mt * ((N + 127) / 128) >= sms) return false;
@@ -273,7 +287,8 @@ static fm_status launch_gemm_t(const CUtensorMap &ta, const CUtensorMap &tb, lon
   constexpr int smem = gemm_smem_bytes(BN, STAGES);
   const int nkb = (int)(K / kGemmBK);
   int kbs = nkb, splits = 1;
-  if (split_ws) splits = gemm_splits(M, N, K, BN, sm_count(), &kbs);
+  if (split_ws && g_gemm_splitk.load(std::memory_order_relaxed))
+    splits = gemm_splits(M, N, K, BN, sm_count(), &kbs);
   auto kern = splits > 1 ? k_gemm_i8_tc<BN, STAGES, true> : k_gemm_i8_tc<BN, STAGES, false>;
   FM_CHECK_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
   if (splits > 1) {

@@ -53,11 +53,21 @@ def test_exp_layout_and_workspace(so):
     # and the per-16-step growth bounds (8 bytes per channel per 16 tokens)
     per_tok = (s.d_model + 9 * s.d_inner + 2 * cc + 4 * nh + 8 + (4 * nh + 8 * s.d_inner + 1024)
                + s.d_inner // 2)
-    # + the split-K partial sums when a GEMM of the layer splits (out_proj at 2048 rows)
-    split = max(lib.gemm_workspace_bytes(2048, s.n_in, s.d_model),
-                lib.gemm_workspace_bytes(2048, s.d_model, s.d_inner))
-    assert split == 2048 * s.d_model * 4
-    assert per_tok * 2048 + split <= ws <= per_tok * 2048 + split + 256 * 17
+    # split-K is off by default: no partial sums
+    assert lib.gemm_workspace_bytes(2048, s.d_model, s.d_inner) == 0
+    assert per_tok * 2048 <= ws <= per_tok * 2048 + 256 * 17
+    # switched on, the layer holds the partial sums of a GEMM that splits
+    # (out_proj at 2048 rows)
+    lib.set_gemm_splitk(True)
+    try:
+        ws = lib.workspace_bytes(s, 1, 2048)
+        split = max(lib.gemm_workspace_bytes(2048, s.n_in, s.d_model),
+                    lib.gemm_workspace_bytes(2048, s.d_model, s.d_inner))
+        assert split == 2048 * s.d_model * 4
+        assert per_tok * 2048 + split <= ws <= per_tok * 2048 + split + 256 * 17
+    finally:
+        lib.set_gemm_splitk(False)
+    assert so.fm_set_gemm_splitk(2) == 1
     assert lib.calib_workspace_bytes(s, 16, 512) > lib.workspace_bytes(s, 16, 512)
     # a single decode step stages nothing for the scan
     assert lib.scan_workspace_bytes(s, 64, 1) == 256

@@ -142,21 +142,78 @@ def _lq_layers(s, seed, prenorm=False, mode=O.DYNAMIC):
     return P, ol, dl
 
 
+def _lq_stages(L, dl, xd):
+    """One LQ layer through the stage entry points, in the order
+    fm_lq_mixer_prefill composes them; returns every intermediate."""
+    s = dl.shape
+    B, T, _ = xd.shape
+    M, di, cc = B * T, s.d_inner, s.conv_ch
+    e = lambda *sh, dt=torch.float32: torch.empty(sh, dtype=dt, device="cuda")
+    q, sx = e(M, s.d_model, dt=torch.int8), e(M)
+    Y, xo, g = e(M, s.n_in), e(M, cc), e(M, di)
+    q2, sx2, out = e(M, di, dt=torch.int8), e(M), e(B, T, s.d_model)
+    L.hadamard_quant(xd, s.d_model, dl.prenorm_w, 1, dl.mode, dl.static_amax, q, sx)
+    L.w8a8_gemm(q, sx, dl.w_in_q, dl.w_in_s, Y)
+    L.lq_conv1d(Y[:, di:di + cc], B, T, s, dl.conv_w, dl.conv_b, None, xo)
+    L.lq_scan(xo, Y[:, di + cc:], Y[:, :di], B, T, s, dl.dt_bias, dl.a_log, dl.D, None, g)
+    L.hadamard_quant(g, di, dl.norm_w, 1, dl.mode, dl.static_amax[1:], q2, sx2)
+    L.w8a8_gemm(q2, sx2, dl.w_out_q, dl.w_out_s, out.view(M, s.d_model))
+    torch.cuda.synchronize()
+    L.sync_status()
+    return {k: v.cpu().numpy() for k, v in dict(Y=Y, xo=xo, g=g, q2=q2, sx2=sx2,
+                                                out=out).items()}
+
+
 @pytest.mark.parametrize("mode", [O.DYNAMIC, O.STATIC])
 def test_lq_layer_matches_oracle(L, mode):
-    """A calibrated 130M layer in LQ form against the oracle's lq_mixer (the
-    same calibration, computed on each side), within 1e-3 x RMS."""
+    """A calibrated 130M layer in LQ form (the same calibration, computed on
+    each side), stage by stage with the oracle fed the GPU's stage inputs:
+    the rotated W8A8 in_proj, the out_proj input's norm + rotation + int8 and
+    the out_proj are exact; the fp32 conv and scan stay within their fp32
+    bounds.  Against the oracle's own fp64 LQ mixer the fp32 gate can move
+    an out_proj code across a rounding boundary, which moves an output by up
+    to one code step times a weight column, so that whole-layer comparison is
+    held to an RMS bound (1e-3 of the output's RMS) and the stage-wise one is
+    the exact parity check."""
     s = MAMBA130
     P, ol, dl = _lq_layers(s, 1000, mode=mode)
     x = S.activations(1, 256, s.d_model, seed=3, n_outliers=8, outlier_scale=50.0,
                       outlier_seed=4242)
-    got = host(dl.lq_prefill(dev(x)))
+    xd = dev(x)
+    st = _lq_stages(L, dl, xd)
+    got = host(dl.lq_prefill(xd))
+    assert np.array_equal(got, st["out"])                     # the composition
+    di, cc, M = s.d_inner, s.conv_ch, 256
+    # in_proj: exact
+    q, sx = O.hadamard_quant(x.reshape(M, s.d_model), None, 1, mode, ol.amax_in)
+    assert np.array_equal(st["Y"], O.dequant(O.gemm_i8(q, ol.wq_in), sx, ol.sw_in))
+    # conv + SiLU on the GPU's in_proj output: fp32 bound
+    u = st["Y"][:, di:di + cc].astype(np.float64)[None]
+    acc = O.ref_conv_f64(u, P["conv_w"].astype(np.float64), P["conv_b"].astype(np.float64))
+    mag = O.ref_conv_f64(np.abs(u), np.abs(P["conv_w"].astype(np.float64)),
+                         np.abs(P["conv_b"].astype(np.float64)))
+    assert (np.abs(st["xo"] - _silu(acc)[0]) <= 1e-6 * mag[0] + 1e-30).all()
+    # scan + gate on the GPU's conv output: fp32 bound
+    dt_raw = st["Y"][:, di + cc:].reshape(1, M, s.nheads)
+    y, _ = _scan_f64(st["xo"][None], dt_raw, P["dt_bias"], P["a_log"], P["D"], di, s.d_state,
+                     s.headdim)
+    ymag, _ = _scan_f64(st["xo"][None], dt_raw, P["dt_bias"], P["a_log"], P["D"], di, s.d_state,
+                        s.headdim, absval=True)
+    sg = _silu(st["Y"][:, :di].astype(np.float64))
+    assert (np.abs(st["g"] - y[0] * sg) <= 1e-4 * ymag[0] * np.abs(sg) + 1e-30).all()
+    # gated RMSNorm + rotation + int8 on the GPU's gated values: exact
+    q2, sx2 = O.hadamard_quant(st["g"], ol.norm_w, 1, mode, ol.amax_out)
+    assert np.array_equal(st["q2"], q2) and np.array_equal(st["sx2"], sx2)
+    # out_proj: exact
+    assert np.array_equal(st["out"].reshape(M, s.d_model),
+                          O.dequant(O.gemm_i8(st["q2"], ol.wq_out), st["sx2"], ol.sw_out))
+    # against the oracle's fp64 LQ mixer
     ref = stages.lq_mixer(ol, P, x)
     rms = np.sqrt(np.mean(ref ** 2))
-    assert np.abs(got - ref).max() <= 1e-3 * rms
+    assert np.sqrt(np.mean((got - ref) ** 2)) <= 1e-3 * rms
     # the LQ variant is more accurate than the full method against fp64
     f64 = O.ref_mixer_f64(P, s, x)
-    full = host(dl.prefill(dev(x)))
+    full = host(dl.prefill(xd))
     assert O.sqnr_db(f64, got) > O.sqnr_db(f64, full) + 5.0
 
 
@@ -185,9 +242,9 @@ def test_lq_stack_layer_chunked_and_decode(L):
     # compare the mixer's contribution (output minus the residual input)
     mix = full - x
     rms = np.sqrt(np.mean(mix ** 2))
-    assert np.abs(chunked - full).max() <= 1e-3 * rms
+    assert np.sqrt(np.mean((chunked - full) ** 2)) <= 1e-4 * rms
     ref = stages.lq_mixer(ol, P, x, residual=True) - x
-    assert np.abs(mix - ref).max() <= 1e-3 * np.sqrt(np.mean(ref ** 2))
+    assert np.sqrt(np.mean((mix - ref) ** 2)) <= 1e-3 * np.sqrt(np.mean(ref ** 2))
 
 
 def test_lq_validation(L):

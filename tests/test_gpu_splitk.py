@@ -1,7 +1,8 @@
 """Split-K of the small-grid GEMM (fm_w8a8_gemm_ws, fm_in_proj_ws and the
-layer entry points): the K slices add exact int32 partial sums, so the
-results are bit for bit those of the unsplit kernel and of the oracle, at
-the decode shapes (M = 64 at 2.7B) and the 130M out_proj (M = 2048, N = 768).
+layer entry points), switched on for this module (fm_set_gemm_splitk; off by
+default): the K slices add exact int32 partial sums, so the results are bit
+for bit those of the unsplit kernel and of the oracle, at the decode shapes
+(M = 64 at 2.7B) and the 130M out_proj (M = 2048, N = 768).
 """
 import numpy as np
 import pytest
@@ -20,7 +21,9 @@ def L():
     from quantized_state_space_mamba2_b200 import build, lib
     build.build()
     lib.load()
-    return lib
+    lib.set_gemm_splitk(True)
+    yield lib
+    lib.set_gemm_splitk(False)
 
 
 def dev(a):
