@@ -325,35 +325,32 @@ __global__ void __launch_bounds__(kSsdThreads) k_ssd_out(SsdArgs a) {
   }
   if (warp == 0) tmem_alloc(slot, 256);  // G: columns 0..127 (int32), Y: 128..191 (fp32)
 
-  // this thread's token: its B and C rows (int8 operands of G) and its x codes
-  uint4 crow[8];
-  {
-    const int8_t *src = a.xbc + (row0 + t) * a.cc;
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      uint4 bv = make_uint4(0u, 0u, 0u, 0u), cv = make_uint4(0u, 0u, 0u, 0u);
-      if (t < nt) {
-        bv = *reinterpret_cast<const uint4 *>(src + a.di + k * 16);
-        cv = *reinterpret_cast<const uint4 *>(src + a.di + kSsdDs + k * 16);
-      }
-      crow[k] = cv;
-      *reinterpret_cast<uint4 *>(sB8 + sw128_off(t, k * 16, kSsdQ)) = bv;
-      *reinterpret_cast<uint4 *>(sC8 + sw128_off(t, k * 16, kSsdQ)) = cv;
-    }
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      uint4 xv = make_uint4(0u, 0u, 0u, 0u);
-      if (t < nt) xv = *reinterpret_cast<const uint4 *>(src + (long long)h * kSsdHd + k * 16);
-      *reinterpret_cast<uint4 *>(Xt + t * 64 + k * 16) = xv;
-    }
+  // the chunk's B and C rows (int8 operands of G) and x codes, zero past the
+  // end: 16 threads per token row (the B | C bytes are contiguous), so each
+  // warp load covers two whole 256-byte rows
+  for (int i = t; i < kSsdQ * 16; i += kSsdThreads) {
+    const int s = i >> 4, k = i & 15;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (s < nt) v = *reinterpret_cast<const uint4 *>(a.xbc + (row0 + s) * a.cc + a.di + k * 16);
+    uint8_t *dst = k < 8 ? sB8 + sw128_off(s, k * 16, kSsdQ) : sC8 + sw128_off(s, (k - 8) * 16, kSsdQ);
+    *reinterpret_cast<uint4 *>(dst) = v;
   }
+  for (int i = t; i < kSsdQ * 4; i += kSsdThreads) {
+    const int s = i >> 2, k = i & 3;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (s < nt)
+      v = *reinterpret_cast<const uint4 *>(a.xbc + (row0 + s) * a.cc + (long long)h * kSsdHd + k * 16);
+    *reinterpret_cast<uint4 *>(Xt + s * 64 + k * 16) = v;
+  }
+  // (its CTA barrier also makes the tiles above visible to every thread)
   const int dtq = ssd_chunk_decay(a, b, h, t0, nt, sW, wtot);
   sdt[t] = __fmul_rn(__int2float_rn(dtq), 1.0f / 65536.0f);
-  {  // row t of Ca: bf16(2^W[t] Cq[t][n])
+  {  // row t of Ca: bf16(2^W[t] Cq[t][n]), Cq read back from the int8 tile
     const float a0 = pow2_q16(sW[t]);
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
-      const uint32_t wv[4] = {crow[k].x, crow[k].y, crow[k].z, crow[k].w};
+      const uint4 cv = *reinterpret_cast<const uint4 *>(sC8 + sw128_off(t, k * 16, kSsdQ));
+      const uint32_t wv[4] = {cv.x, cv.y, cv.z, cv.w};
       uint32_t pk[8];
 #pragma unroll
       for (int q = 0; q < 4; ++q)
@@ -459,26 +456,44 @@ __global__ void __launch_bounds__(kSsdThreads) k_ssd_out(SsdArgs a) {
   }
   ok = mbar_drain(&bar[1], 0) && ok;
   tc_fence_after();
+  // the y tile is staged in shared memory (M and Ca are dead once the MMAs
+  // that read them have completed; rows padded to 68 words) and written out
+  // in whole rows
+  constexpr int kYStride = kSsdHd + 4;
+  int32_t *sY = reinterpret_cast<int32_t *>(sm + L::kC8);
+  static_assert(kSsdQ * kYStride * 4 <= L::kX - L::kC8, "the y tile fits over M and Ca");
   {  // y codes of token t: rint(Y 2^(e_C+e_x+e_B-e_y)) + rshr(D_q x, s_D), saturated
     const int s_y = *a.e_C + a.e_x[h] + *a.e_B - a.e_y[h];
     const int s_D = a.e_y[h] - a.e_D[h] - a.e_x[h];
     const long long Dq = a.D_q[h];
     const float scale = pow2f(s_y);
-    int32_t *dst = a.y + (row0 + t) * a.di + (long long)h * kSsdHd;
 #pragma unroll 1
     for (int c0 = 0; c0 < kSsdHd; c0 += 32) {
       uint32_t r[32];
       tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(128 + c0), r);
-      if (ok && t < nt) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const double yc = (double)rintf(__fmul_rn(__uint_as_float(r[j]), scale));
-          const long long skip = rshr64(Dq * (long long)Xt[t * 64 + c0 + j], s_D);
-          double v = yc + (double)skip;
-          v = fmin(fmax(v, -2147483647.0), 2147483647.0);
-          dst[c0 + j] = (int32_t)v;
+      for (int j = 0; j < 32; j += 4) {
+        int v4[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          // rint of a float is an integer; the int64 conversion is exact
+          const long long yc = __float2ll_rn(rintf(__fmul_rn(__uint_as_float(r[j + e]), scale)));
+          const long long skip = rshr64(Dq * (long long)Xt[t * 64 + c0 + j + e], s_D);
+          long long v = yc + skip;
+          v = v < -2147483647LL ? -2147483647LL : (v > 2147483647LL ? 2147483647LL : v);
+          v4[e] = (int)v;
         }
+        *reinterpret_cast<int4 *>(sY + t * kYStride + c0 + j) = make_int4(v4[0], v4[1], v4[2], v4[3]);
       }
+    }
+  }
+  __syncthreads();
+  if (ok) {  // 16 threads per token row of 64 int32
+    for (int i = t; i < kSsdQ * 16; i += kSsdThreads) {
+      const int s = i >> 4, k = i & 15;
+      if (s < nt)
+        *reinterpret_cast<int4 *>(a.y + (row0 + s) * a.di + (long long)h * kSsdHd + k * 4) =
+            *reinterpret_cast<const int4 *>(sY + s * kYStride + k * 4);
     }
   }
   tc_fence_before();
