@@ -90,6 +90,8 @@ def parse(argv=None):
     ap.add_argument("--state-spec", default="31,0", choices=["31,0", "16,7"],
                     help="scan state word and increment guard bits: 31,0 the method as built, "
                          "16,7 the narrow state with the guard-bit increment")
+    ap.add_argument("--gemm-tile", type=int, default=0, choices=[0, 128, 256],
+                    help="tile width of the persistent GEMM (0: chosen by the grid)")
     ap.add_argument("--eager", action="store_true",
                     help="launch the timed steps one by one instead of replaying them as one "
                          "captured CUDA graph")
@@ -912,6 +914,7 @@ def apply_modes(args, lib):
         lib.set_scan_tile(*[int(v) for v in args.scan_tile.split(",")])
     lib.set_scan_mode(args.scan_mode)
     lib.set_state_spec(*[int(v) for v in args.state_spec.split(",")])
+    lib.set_gemm_tile(args.gemm_tile)
 
 
 def main():

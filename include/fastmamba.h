@@ -171,6 +171,12 @@ fm_status fm_in_proj(const int8_t *A, const float *s_x, int64_t M, const int8_t 
                      const float *s_w, const fm_shape *shape, const int32_t *exps, float *z,
                      int8_t *xbc, float *dt, fm_stream stream);
 
+/* Tuning: the tile width (output columns per CTA tile) of the persistent GEMM
+ * kernel for every later call in this process: 0 (default) chooses by the
+ * grid, 128 or 256 forces it where the persistent kernel runs.  All widths
+ * compute the same bits.  FM_ERR_INVALID_ARG for other values. */
+fm_status fm_set_gemm_tile(int bn);
+
 /* Workspace variants: the same results, bit for bit.  Given a device
  * workspace of fm_gemm_workspace_bytes(M, N, K) bytes (0 when the problem
  * would not split), a grid with fewer output tiles than the GPU has SMs

@@ -345,6 +345,18 @@ static int sm_count() {
 // batch): one 128 x 64 tile per CTA (128 x 32 when even those are fewer than
 // the SMs), two CTAs per SM.
 // split_ws (nullable, M x N int32): lets the small-grid path split K.
+// Tile width of the persistent GEMM, process-wide: 0 (default) chooses by the
+// grid (256 when there are at least two 256-wide tiles per SM), 128 or 256
+// forces that width wherever the persistent kernel runs (tuning).
+static std::atomic<int> g_gemm_tile{0};
+
+extern "C" fm_status fm_set_gemm_tile(int bn) {
+  if (bn != 0 && bn != 128 && bn != 256)
+    return fail(FM_ERR_INVALID_ARG, "fm_set_gemm_tile: %d is not 0, 128 or 256", bn);
+  g_gemm_tile.store(bn, std::memory_order_relaxed);
+  return FM_OK;
+}
+
 static fm_status launch_gemm(const int8_t *A, long long M, const int8_t *W, long long N,
                              long long K, const GemmEpilogue &ep, cudaStream_t s,
                              int32_t *split_ws = nullptr) {
@@ -356,11 +368,13 @@ static fm_status launch_gemm(const int8_t *A, long long M, const int8_t *W, long
   const long long tiles256 = mt * ((N + 255) / 256), tiles128 = mt * ((N + 127) / 128);
   const int sms = sm_count();
   FM_TRY(make_tmap(&ta, A, M, K, kGemmBM));
-  if (tiles256 >= 2LL * sms) {
+  const int force = g_gemm_tile.load(std::memory_order_relaxed);
+  const bool persist = tiles256 >= 2LL * sms || tiles128 >= sms;
+  if (persist && (force == 256 || (force == 0 && tiles256 >= 2LL * sms))) {
     FM_TRY(make_tmap(&tb, W, N, K, 256));
     return launch_gemm_persist<256, 3, 8>(ta, tb, M, N, K, sms, ep, s);
   }
-  if (tiles128 >= sms) {
+  if (persist) {
     FM_TRY(make_tmap(&tb, W, N, K, 128));
     return launch_gemm_persist<128, 5, 8>(ta, tb, M, N, K, sms, ep, s);
   }

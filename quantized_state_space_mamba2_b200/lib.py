@@ -31,6 +31,7 @@ EXPORTS = (
     "fm_set_scan_tile", "fm_ssd_workspace_bytes", "fm_ssd_scan", "fm_set_scan_mode",
     "fm_set_state_spec", "fm_lq_conv1d", "fm_lq_scan", "fm_lq_workspace_bytes",
     "fm_lq_mixer_prefill", "fm_set_fault_injection", "fm_set_gemm_splitk",
+    "fm_set_gemm_tile",
 )
 NOALLOC_SCRATCH_BYTES = 16 << 20  # FM_NOALLOC_SCRATCH_BYTES
 
@@ -115,6 +116,7 @@ def load():
         "fm_lq_workspace_bytes": (SZ, [sp, I, I]),
         "fm_set_fault_injection": (I, [I, C.c_uint64]),
         "fm_set_gemm_splitk": (I, [I]),
+        "fm_set_gemm_tile": (I, [I]),
         "fm_lq_mixer_prefill": (I, [lp, C.POINTER(fm_lq_params), _P, I, I, I, _P, _P, _P, _P,
                                     SZ, _P]),
     }
@@ -177,6 +179,11 @@ def hadamard_quant(x, K, prenorm_w, rotate, mode, static_amax, q, s_x, amax_row=
 def prepare_linear(W, rotate, Wq, s_w, stream=None):
     N, K = W.shape
     _check(load().fm_prepare_linear(_p(W), N, K, rotate, _p(Wq), _p(s_w), _s(stream)))
+
+
+def set_gemm_tile(bn: int):
+    """Tile width of the persistent GEMM: 0 (by the grid), 128 or 256."""
+    _check(load().fm_set_gemm_tile(bn))
 
 
 def set_gemm_splitk(enable: bool):
