@@ -1274,19 +1274,32 @@ static fm_status launch_lq_conv(const float *u, long long ldu, int B, int T, int
   return FM_OK;
 }
 
+template <int CPW>
+static fm_status launch_lq_scan_t(const Dims &d, const float *xo, const float *dt_raw,
+                                  long long ld_dt, const float *z, long long ld_z, int B, int T,
+                                  const float *dt_bias, const float *a_log, const float *D,
+                                  float *state, float *out, cudaStream_t s) {
+  constexpr int smem = (int)sizeof(LqScanSmem<CPW>);
+  FM_CHECK_CUDA(cudaFuncSetAttribute(k_lq_scan<CPW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     smem));
+  k_lq_scan<CPW><<<dim3((unsigned)(d.hd / (4 * CPW)), (unsigned)d.nh, (unsigned)B), 128, smem,
+                   s>>>(xo, dt_raw, ld_dt, z, ld_z, T, d.nh, d.cc, d.di, dt_bias, a_log, D, state,
+                        out);
+  return launched("k_lq_scan");
+}
+
 static fm_status launch_lq_scan(const Dims &d, const float *xo, const float *dt_raw,
                                 long long ld_dt, const float *z, long long ld_z, int B, int T,
                                 const float *dt_bias, const float *a_log, const float *D,
                                 float *state, float *out, cudaStream_t s) {
-  // 4 channels per warp once there are enough CTAs to fill the GPU, else 2
-  if ((long long)B * d.nh * (d.hd / 16) >= 2LL * 148) {
-    k_lq_scan<4><<<dim3((unsigned)(d.hd / 16), (unsigned)d.nh, (unsigned)B), 128, 0, s>>>(
-        xo, dt_raw, ld_dt, z, ld_z, T, d.nh, d.cc, d.di, dt_bias, a_log, D, state, out);
-  } else {
-    k_lq_scan<2><<<dim3((unsigned)(d.hd / 8), (unsigned)d.nh, (unsigned)B), 128, 0, s>>>(
-        xo, dt_raw, ld_dt, z, ld_z, T, d.nh, d.cc, d.di, dt_bias, a_log, D, state, out);
-  }
-  return launched("k_lq_scan");
+  // one channel per warp while that leaves fewer than ~8 warps per SM to
+  // share the staged rows, else 2 (more state cells per staged row)
+  const long long warps1 = (long long)B * d.nh * d.hd;
+  if (warps1 >= 16LL * sm_count())
+    return launch_lq_scan_t<2>(d, xo, dt_raw, ld_dt, z, ld_z, B, T, dt_bias, a_log, D, state,
+                               out, s);
+  return launch_lq_scan_t<1>(d, xo, dt_raw, ld_dt, z, ld_z, B, T, dt_bias, a_log, D, state, out,
+                             s);
 }
 
 extern "C" fm_status fm_lq_conv1d(const float *u, int64_t ldu, int B, int T,

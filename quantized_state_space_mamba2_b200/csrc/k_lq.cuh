@@ -18,6 +18,7 @@
 // norm weight as its pre-norm weight.
 #pragma once
 #include "fm_common.cuh"
+#include "k_gemm.cuh"
 
 namespace fm {
 
@@ -96,17 +97,42 @@ __global__ void __launch_bounds__(256) k_lq_conv_state_update(const float *__res
 // ------------------------------------------------------------------ scan
 // Grid (hd / (4 CPW), nh, B), 4 warps; warp w owns channels p0 .. p0 + CPW - 1
 // of head h, lane l the states n = 4l .. 4l + 3 of each (CPW x 4 fp32 state
-// cells in registers for the whole sequence).  Per 32-token chunk, lane s
-// computes dt and dA of token t0 + s once; each step broadcasts them by
-// shuffle.  Each step adds its C h partial sums to a 32-entry buffer (32 / CPW
+// cells in registers for the whole sequence).  The sequence runs in 32-token
+// chunks staged in shared memory, two buffers: while the warps run chunk c,
+// chunk c + 1's B and C rows and the CTA's x values are on their way (cp.async,
+// 16 bytes a piece, whole rows per warp), and 32 threads compute its dt and
+// dA.  Each step adds its C h partial sums to a 32-entry buffer (32 / CPW
 // steps x CPW channels); a full buffer is reduced across the warp by a
-// reduce-scatter (5 xor-shuffle stages), after which lane j holds the total of
-// entry j and writes that output.
+// reduce-scatter (5 xor-shuffle stages), after which lane j holds the total
+// of entry j and writes that output.
 //   xo     [B, T, cc] conv output (x | B | C)
 //   dt_raw rows of stride ld_dt (column h), z rows of stride ld_z (nullable:
 //          no gate, y is written)
 //   state  [B, nh, hd, ds] fp32 in/out (nullable: zero initial state)
 //   out    [B, T, di]: g = y SiLU(z), or y
+constexpr int kLqChunk = 32;
+
+template <int CPW>
+struct LqScanSmem {
+  float Bm[2][kLqChunk][128];
+  float Cm[2][kLqChunk][128];
+  float X[2][kLqChunk][4 * CPW];
+  float dt[2][kLqChunk];
+  float dA[2][kLqChunk];
+};
+
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 template <int CPW>
 __global__ void __launch_bounds__(128) k_lq_scan(
     const float *__restrict__ xo, const float *__restrict__ dt_raw, long long ld_dt,
@@ -115,15 +141,48 @@ __global__ void __launch_bounds__(128) k_lq_scan(
     const float *__restrict__ Dp, float *state, float *__restrict__ out) {
   static_assert(CPW == 1 || CPW == 2 || CPW == 4, "CPW");
   constexpr int SB = 32 / CPW;  // steps per reduction
-  constexpr int hd = 64, ds = 128;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int hd = 64, ds = 128, CH = 4 * CPW;  // channels per CTA
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  LqScanSmem<CPW> &sm = *reinterpret_cast<LqScanSmem<CPW> *>(smem_raw);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int h = blockIdx.y, b = blockIdx.z;
-  const int p0 = (blockIdx.x * 4 + warp) * CPW;
+  const int pc0 = blockIdx.x * CH;            // the CTA's first channel
+  const int p0 = pc0 + warp * CPW;            // this warp's first channel
   const int n0 = lane * 4;
   const float A = -expf(a_log[h]);
   const float Dh = Dp[h];
   const float bias = dt_bias[h];
   const long long bh = (long long)b * nh + h;
+  const float *xrow = xo + (long long)b * T * cc;
+
+  // stage chunk c into buffer c & 1 (B, C rows and the CTA's x: cp.async;
+  // dt, dA of its 32 tokens: warp 0)
+  auto stage = [&](int c) {
+    const int t0 = c * kLqChunk, nt = min(kLqChunk, T - t0), buf = c & 1;
+    for (int i = tid; i < kLqChunk * 64; i += 128) {   // 64 pieces per token: 32 B, 32 C
+      const int s = i >> 6, k = i & 63;
+      if (s < nt) {
+        const float *src = xrow + (long long)(t0 + s) * cc + di + k * 4;
+        float *dst = k < 32 ? &sm.Bm[buf][s][k * 4] : &sm.Cm[buf][s][(k - 32) * 4];
+        cp_async16(dst, src);
+      }
+    }
+    for (int i = tid; i < kLqChunk * CPW; i += 128) {  // CPW pieces of 4 channels per token
+      const int s = i / CPW, k = i % CPW;
+      if (s < nt) cp_async16(&sm.X[buf][s][k * 4], xrow + (long long)(t0 + s) * cc + h * hd + pc0 + k * 4);
+    }
+    cp_async_commit();
+    if (warp == 0) {
+      float dtl = 0.0f, dAl = 0.0f;
+      if (lane < nt) {
+        const float v = __fadd_rn(dt_raw[((long long)b * T + t0 + lane) * ld_dt + h], bias);
+        dtl = softplus_f32(v);
+        dAl = expf(__fmul_rn(dtl, A));
+      }
+      sm.dt[buf][lane] = dtl;
+      sm.dA[buf][lane] = dAl;
+    }
+  };
 
   float hs[CPW][4];
   float *st = state ? state + (bh * hd + p0) * ds + n0 : nullptr;
@@ -136,41 +195,31 @@ __global__ void __launch_bounds__(128) k_lq_scan(
     hs[c][2] = v.z;
     hs[c][3] = v.w;
   }
-  const float *xrow = xo + (long long)b * T * cc;
+  const int nch = (T + kLqChunk - 1) / kLqChunk;
+  stage(0);
   float part[32];
 #pragma unroll 1
-  for (int t0 = 0; t0 < T; t0 += 32) {
-    float dtl = 0.0f, dAl = 0.0f;
-    if (t0 + lane < T) {
-      const float v = __fadd_rn(dt_raw[((long long)b * T + t0 + lane) * ld_dt + h], bias);
-      dtl = softplus_f32(v);
-      dAl = expf(__fmul_rn(dtl, A));
+  for (int ch = 0; ch < nch; ++ch) {
+    if (ch + 1 < nch) {
+      stage(ch + 1);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
     }
-    const int nt = min(32, T - t0);
+    __syncthreads();  // chunk ch staged (copies and dt / dA) for every warp
+    const int buf = ch & 1, t0 = ch * kLqChunk, nt = min(kLqChunk, T - t0);
 #pragma unroll 1
-    for (int s0 = 0; s0 < 32; s0 += SB) {
+    for (int s0 = 0; s0 < kLqChunk; s0 += SB) {
 #pragma unroll
       for (int k = 0; k < SB; ++k) {
-        const int s = s0 + k, t = t0 + s;
-        const float dts = __shfl_sync(0xffffffffu, dtl, s);
-        const float dAs = __shfl_sync(0xffffffffu, dAl, s);
+        const int s = s0 + k;
         if (s < nt) {
-          const float *row = xrow + (long long)t * cc;
-          const float4 Bv = *reinterpret_cast<const float4 *>(row + di + n0);
-          const float4 Cv = *reinterpret_cast<const float4 *>(row + di + ds + n0);
-          float xv[CPW];
-          if constexpr (CPW == 4) {
-            const float4 x4 = *reinterpret_cast<const float4 *>(row + h * hd + p0);
-            xv[0] = x4.x; xv[1] = x4.y; xv[2] = x4.z; xv[3] = x4.w;
-          } else if constexpr (CPW == 2) {
-            const float2 x2 = *reinterpret_cast<const float2 *>(row + h * hd + p0);
-            xv[0] = x2.x; xv[1] = x2.y;
-          } else {
-            xv[0] = row[h * hd + p0];
-          }
+          const float dts = sm.dt[buf][s], dAs = sm.dA[buf][s];
+          const float4 Bv = *reinterpret_cast<const float4 *>(&sm.Bm[buf][s][n0]);
+          const float4 Cv = *reinterpret_cast<const float4 *>(&sm.Cm[buf][s][n0]);
 #pragma unroll
           for (int c = 0; c < CPW; ++c) {
-            const float dtx = __fmul_rn(dts, xv[c]);
+            const float dtx = __fmul_rn(dts, sm.X[buf][s][warp * CPW + c]);
             hs[c][0] = __fmaf_rn(dAs, hs[c][0], __fmul_rn(dtx, Bv.x));
             hs[c][1] = __fmaf_rn(dAs, hs[c][1], __fmul_rn(dtx, Bv.y));
             hs[c][2] = __fmaf_rn(dAs, hs[c][2], __fmul_rn(dtx, Bv.z));
@@ -197,15 +246,15 @@ __global__ void __launch_bounds__(128) k_lq_scan(
           part[i] = __fadd_rn(keep, __shfl_xor_sync(0xffffffffu, send, m));
         }
       }
-      const int s = s0 + lane / CPW, c = lane % CPW, t = t0 + s;
+      const int s = s0 + lane / CPW, c = lane % CPW;
       if (s < nt) {
-        const long long r = (long long)b * T + t;
-        const float xv = xrow[(long long)t * cc + h * hd + p0 + c];
-        float y = __fmaf_rn(Dh, xv, part[0]);
+        const long long r = (long long)b * T + t0 + s;
+        float y = __fmaf_rn(Dh, sm.X[buf][s][warp * CPW + c], part[0]);
         if (z) y = __fmul_rn(y, silu_f32(z[r * ld_z + h * hd + p0 + c]));
         out[r * di + h * hd + p0 + c] = y;
       }
     }
+    __syncthreads();  // every warp is done with buffer buf before it is refilled
   }
   if (st) {
 #pragma unroll
