@@ -335,6 +335,20 @@ fm_status fm_ssd_scan(const int8_t *xbc, const float *dt_raw, int B, int T,
  * headroom.  Switch it before calibrating and allocating states, and keep it
  * for the layer's life.  Anything else: FM_ERR_INVALID_ARG. */
 fm_status fm_set_state_spec(int bits, int guard);
+/* Source: as fm_set_state_spec (the granularity of the "fine-grained"
+ * power-of-two scales is left open by the pages).
+ * Process-wide granularity of the conv output's exponents in the layer entry
+ * points (fm_mixer_prefill, fm_decode_step, fm_calibrate_layer): 0 (default)
+ * the static exponents as built (e_x per head, e_B, e_C); 1 per token -- each
+ * token's codes of a head's x channels, of B and of C are
+ * satb(rshr(s, e + 16), 8) with e = max(E(max |s|, 127) - 16, static - 16),
+ * s the Q.16 SiLU values, and the scan shifts u, its output and the skip
+ * term by the token's exponents (state and output exponents stay static).
+ * The layer workspace then holds the exponents ([B*T, nh + 2] int32) and the
+ * scan's per-token shifts.  Set it before calibrating and sizing workspaces;
+ * the chunked scan mode refuses it.  The standalone fm_conv1d_pot and
+ * fm_ssm_scan_pot stay static.  FM_ERR_INVALID_ARG for other values. */
+fm_status fm_set_xbc_exponents(int per_token);
 
 /* Workspace bytes fm_mixer_prefill / fm_decode_step need for B*T tokens. */
 size_t fm_workspace_bytes(const fm_shape *shape, int B, int T);

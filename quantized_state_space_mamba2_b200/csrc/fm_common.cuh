@@ -44,6 +44,11 @@ __device__ __forceinline__ long long shl_sat61(long long a, int k) {
   return a * (1LL << k);
 }
 
+// a 2^k with saturation at 2^61 for k >= 0, rshr(a, -k) for k < 0
+__device__ __forceinline__ long long pow2_sat61(long long a, int k) {
+  return k >= 0 ? shl_sat61(a, k) : rshr64(a, -k);
+}
+
 // fp32 -> nearest integer (half to even) clamped to +-lim (NaN -> -lim)
 __device__ __forceinline__ int round_clamp(float v, float lim) {
   float r = rintf(v);

@@ -405,17 +405,21 @@ static fm_status launch_hadamard_quant(const float *x, long long M, int K, const
 
 static fm_status launch_conv(const int8_t *u, int B, int T, int cc, const int8_t *wq,
                              const int32_t *bq, const int32_t *exps, int8_t *conv_state,
-                             int8_t *out, unsigned int *amax, cudaStream_t s) {
+                             int8_t *out, unsigned int *amax, cudaStream_t s,
+                             int32_t *e_tok = nullptr, const Dims *d = nullptr) {
   if ((long long)B * T == 0) return FM_OK;
   const int groups = (cc / kConvCPT + kConvQuads - 1) / kConvQuads;
   if (B > 65535) return fail(FM_ERR_SHAPE, "conv: B too large");
+  if (e_tok && (!d || amax)) return fail(FM_ERR_INVALID_ARG, "conv: per-token exponents misused");
+  const int di = d ? d->di : 0, hd = d ? d->hd : 0, ds = d ? d->ds : 0;
   if (T >= kConvTT) {
     const unsigned tiles = (unsigned)((T + kConvTokens - 1) / kConvTokens);
     k_conv1d_pot<kConvTT, kConvTG><<<dim3(tiles, groups, B), kConvQuads * kConvTG, 0, s>>>(
-        u, T, cc, wq, bq, exps, conv_state, out, amax, nullptr);
+        u, T, cc, wq, bq, exps, conv_state, out, amax, nullptr, e_tok, di, hd, ds);
   } else {  // decode steps and short chunks: one token per thread
     k_conv1d_pot<1, 1><<<dim3((unsigned)T, groups, B), kConvQuads, 0, s>>>(
-        u, T, cc, wq, bq, exps, conv_state, out, amax, T == 1 ? conv_state : nullptr);
+        u, T, cc, wq, bq, exps, conv_state, out, amax, T == 1 ? conv_state : nullptr, e_tok, di,
+        hd, ds);
   }
   FM_TRY(launched("k_conv1d_pot"));
   if (conv_state && T > 1) {  // a single step updates its state in the conv kernel
@@ -442,10 +446,23 @@ extern "C" fm_status fm_set_state_spec(int bits, int guard) {
 }
 static bool state16() { return g_state_bits.load(std::memory_order_relaxed) == 16; }
 
+// Conv-output exponent granularity, process-wide: 0 (default) the static
+// per-head / B / C exponents as built, 1 per token (the conv requantises each
+// token's groups at their own power-of-two exponent; the scans shift by them).
+static std::atomic<int> g_xbc_tok{0};
+
+extern "C" fm_status fm_set_xbc_exponents(int per_token) {
+  if (per_token != 0 && per_token != 1)
+    return fail(FM_ERR_INVALID_ARG, "fm_set_xbc_exponents: per_token must be 0 or 1");
+  g_xbc_tok.store(per_token, std::memory_order_relaxed);
+  return FM_OK;
+}
+static bool xbc_tok() { return g_xbc_tok.load(std::memory_order_relaxed) == 1; }
+
 static ScanArgs scan_args(const Dims &d, const int8_t *xbc, const float *dt_raw, int T,
                           const float *dt_bias, const int32_t *A_q, const int32_t *D_q,
                           const int32_t *exps, const fm_exp_layout &X, int32_t *state, int32_t *y,
-                          unsigned long long *stat) {
+                          unsigned long long *stat, const int32_t *e_tok = nullptr) {
   ScanArgs a;
   a.xbc = xbc;
   a.dt_raw = dt_raw;
@@ -468,6 +485,7 @@ static ScanArgs scan_args(const Dims &d, const int8_t *xbc, const float *dt_raw,
   a.stat = stat;
   a.hlim = state16() ? kH16Lim : (int)kHLim;
   a.guard = g_state_guard.load(std::memory_order_relaxed);
+  a.e_tok = e_tok;
   return a;
 }
 
@@ -527,6 +545,7 @@ struct ScanWs {
   int32_t *xs;  // [B, nh, hd, Tp]: x codes, widened
   int32_t *bc;  // [B*T, 256]
   long long *bound;  // [B, nh, Tp/16, hd]
+  int32_t *osh;      // [B, nh, Tp] per-token output shifts (per-token exponents only)
 };
 
 // prep (parallel over token tiles and heads) + the sequential kernel
@@ -561,6 +580,9 @@ static fm_status launch_scan_v2(const ScanArgs &a, int B, const ScanWs &w, cudaS
   p.bc = w.bc;
   p.bound = w.bound;
   p.guard = a.guard;
+  p.e_tok = a.e_tok;
+  p.osh = a.e_tok ? w.osh : nullptr;
+  if (a.e_tok && !w.osh) return fail(FM_ERR_WORKSPACE, "scan: per-token shifts need workspace");
   k_scan_prep<<<dim3((unsigned)(Tp / kPrepTT), a.nh, B), 256, 0, s>>>(p);
   FM_TRY(launched("k_scan_prep"));
   ScanSeqArgs q;
@@ -581,6 +603,7 @@ static fm_status launch_scan_v2(const ScanArgs &a, int B, const ScanWs &w, cudaS
   q.e_y = a.e_y;
   q.state = a.state;
   q.y = a.y;
+  q.osh = p.osh;
   const ScanTile t = scan_tile();
 #define FM_SEQ(N, P, C)                                      \
   if (t.npt == N && t.pc == P && t.tch == C)                 \
@@ -792,6 +815,7 @@ struct Carver {
 
 ScanWs carve_scan(Carver &c, const Dims &d, int B, int T) {
   ScanWs w;
+  w.osh = nullptr;
   if (T == 1) {  // single steps run k_scan_step, which stages nothing
     w.dA = nullptr;
     w.u = w.xs = w.bc = nullptr;
@@ -804,6 +828,7 @@ ScanWs carve_scan(Carver &c, const Dims &d, int B, int T) {
   w.xs = c.take<int32_t>((long long)B * d.di * Tp);
   w.bc = c.take<int32_t>(M * 256);
   w.bound = c.take<long long>((long long)B * d.di * (Tp / 16));
+  if (xbc_tok()) w.osh = c.take<int32_t>((long long)B * d.nh * Tp);
   return w;
 }
 }  // namespace
@@ -1026,6 +1051,7 @@ struct MixerWs {
   int8_t *q_out;
   float *sx_out;
   ScanWs scan;
+  int32_t *e_tok;  // [M, nh + 2] per-token conv-output exponents (per-token mode only)
   SsdWs ssd;  // chunked scan mode only (null otherwise)
   int32_t *split;  // split-K partial sums of the small-grid GEMMs (null when none split)
 };
@@ -1043,6 +1069,7 @@ MixerWs carve_mixer(Carver &c, const Dims &d, int B, int T) {
   w.q_out = c.take<int8_t>(M * d.di);
   w.sx_out = c.take<float>(M);
   w.scan = carve_scan(c, d, B, T);
+  w.e_tok = xbc_tok() ? c.take<int32_t>(M * (d.nh + 2)) : nullptr;
   if (use_ssd(T)) {
     w.ssd = carve_ssd(c, d, B, T);
   } else {
@@ -1106,15 +1133,16 @@ static fm_status mixer_impl(const fm_layer *L, const Dims &d, const float *x, in
   FM_TRY(in_proj_impl(w.q_in, w.sx_in, M, L->w_in_q, L->w_in_s, d, L->exps + X.e_u, w.z, w.xbc,
                       w.dt, s, w.split));
   FM_TRY(launch_conv(w.xbc, B, T, d.cc, L->conv_wq, L->conv_bq, L->exps, conv_state, w.xo,
-                     nullptr, s));
-  if (w.ssd.dH && state16())
-    return fail(FM_ERR_UNSUPPORTED, "chunked scan mode with the 16-bit state spec is not supported");
+                     nullptr, s, w.e_tok, &d));
+  if (w.ssd.dH && (state16() || w.e_tok))
+    return fail(FM_ERR_UNSUPPORTED, "the chunked scan mode carries the int32 state at static "
+                "exponents: the 16-bit state spec and per-token exponents are not supported");
   if (w.ssd.dH)
     FM_TRY(launch_ssd(d, w.xo, w.dt, B, T, L->dt_bias, L->A_q, L->D_q, L->exps, X, ssm_state, w.y,
                       w.ssd, s));
   else
     FM_TRY(launch_scan_v2(scan_args(d, w.xo, w.dt, T, L->dt_bias, L->A_q, L->D_q, L->exps, X,
-                                    ssm_state, w.y, nullptr),
+                                    ssm_state, w.y, nullptr, w.e_tok),
                           B, w.scan, s));
   FM_TRY(gate_impl(w.y, w.z, M, d, L->exps, X, L->norm_w, L->rotate, L->mode, amax_out, w.q_out,
                    w.sx_out, nullptr, nullptr, nullptr, s));
@@ -1647,23 +1675,24 @@ extern "C" fm_status fm_calibrate_layer(const fm_layer *L, const float *conv_b, 
   FM_TRY(launch_conv(m.xbc, B, T, d.cc, L->conv_wq, conv_bq, exps, nullptr, m.xo, w.silu_amax, s));
   k_exp_conv_out<<<1, 256, 0, s>>>(w.silu_amax, d.di, d.hd, d.ds, exps, X);
   FM_TRY(launched("k_exp_conv_out"));
-  FM_TRY(launch_conv(m.xbc, B, T, d.cc, L->conv_wq, conv_bq, exps, nullptr, m.xo, nullptr, s));
+  FM_TRY(launch_conv(m.xbc, B, T, d.cc, L->conv_wq, conv_bq, exps, nullptr, m.xo, nullptr, s,
+                     m.e_tok, &d));
   // 4. state exponent: 64-bit run at the finest exponent
   FM_CHECK_CUDA(cudaMemsetAsync(w.stat, 0, sizeof(unsigned long long) * d.nh, s));
   FM_TRY(launch_scan<2>(scan_args(d, m.xo, m.dt, T, L->dt_bias, L->A_q, L->D_q, exps, X, nullptr,
-                                  m.y, w.stat),
+                                  m.y, w.stat, m.e_tok),
                         B, s));
   k_exp_state<<<1, 128, 0, s>>>(w.stat, d.nh, exps, X, state16() ? 16384.0 : 536870912.0);
   FM_TRY(launched("k_exp_state"));
   // 5. output exponent: max |y| at the finer term exponent
   FM_CHECK_CUDA(cudaMemsetAsync(w.stat, 0, sizeof(unsigned long long) * d.nh, s));
   FM_TRY(launch_scan<1>(scan_args(d, m.xo, m.dt, T, L->dt_bias, L->A_q, L->D_q, exps, X, nullptr,
-                                  m.y, w.stat),
+                                  m.y, w.stat, m.e_tok),
                         B, s));
   k_exp_y<<<1, 128, 0, s>>>(w.stat, d.nh, exps, X);
   FM_TRY(launched("k_exp_y"));
   FM_TRY(launch_scan_v2(scan_args(d, m.xo, m.dt, T, L->dt_bias, L->A_q, L->D_q, exps, X, nullptr,
-                                  m.y, nullptr),
+                                  m.y, nullptr, m.e_tok),
                         B, m.scan, s));
   // 6. gate exponent, then the out_proj input amax
   k_exp_gate<<<1, 32, 0, s>>>(nullptr, d.nh, exps, X);

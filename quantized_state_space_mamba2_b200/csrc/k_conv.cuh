@@ -43,12 +43,19 @@ __device__ __forceinline__ void conv_transpose4(uint32_t r0, uint32_t r1, uint32
 }
 
 // amax (nullable, [cc] u32): max |SiLU output| per channel (calibration).
+// e_tok (non-null: per-token output exponents, the x of each head, B and C
+// each a group): the codes of token t and group g are
+// satb(rshr(s, e + 16), 8) with e = max(E(max_g |s|, 127) - 16, e_o - 16), E
+// the power-of-two exponent of the calibration; e_tok[t, g] (int32
+// [B*T, nh + 2]) receives e.  A head's 64 x channels are 16 consecutive
+// threads and B, C one warp each (the x | B | C boundaries are multiples of
+// 256 channels), so the group maximum is a shuffle reduction.
 template <int TT, int TG>
 __global__ void __launch_bounds__(kConvQuads *TG) k_conv1d_pot(
     const int8_t *__restrict__ u, int T, int cc, const int8_t *__restrict__ wq,
     const int32_t *__restrict__ bq, const int32_t *__restrict__ exps,
     const int8_t *conv_state, int8_t *__restrict__ out, unsigned int *amax,
-    int8_t *state_out) {
+    int8_t *state_out, int32_t *e_tok = nullptr, int di = 0, int hd = 0, int ds = 0) {
   __shared__ int tab[8];
   pwl_table_init(tab);
   __syncthreads();
@@ -106,6 +113,32 @@ __global__ void __launch_bounds__(kConvQuads *TG) k_conv1d_pot(
     }
     if (k >= nt) break;
     uint32_t packed = 0;
+    if (e_tok) {  // per-token exponents (the warp is all x, all B or all C: uniform)
+      int sv[kConvCPT];
+      int m = 0;
+#pragma unroll
+      for (int j = 0; j < kConvCPT; ++j) {
+        const long long acc = (long long)bs[j] + __dp4a((int)col[j], wr[j], 0);
+        sv[j] = silu_pwl_t((int)satb64(rshr64(acc, s_in[j]), 32), tab);
+        m = max(m, sv[j] < 0 ? -sv[j] : sv[j]);
+      }
+      const bool xgrp = c0 < di;
+#pragma unroll
+      for (int o = 1; o < 16; o <<= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+      if (!xgrp) m = max(m, __shfl_xor_sync(0xffffffffu, m, 16));
+      const int e = max(pot_exponent((double)m, 127.0) - 16, s_out[0] - 32);
+#pragma unroll
+      for (int j = 0; j < kConvCPT; ++j)
+        packed |= ((uint32_t)((int)satb64(rshr64(sv[j], e + 16), 8) & 0xFF)) << (8 * j);
+      const int lane = threadIdx.x & 31;
+      if ((lane & (xgrp ? 15 : 31)) == 0) {
+        const int nh = di / hd;
+        const int g = xgrp ? c0 / hd : (c0 < di + ds ? nh : nh + 1);
+        e_tok[((long long)b * T + t0 + k) * (nh + 2) + g] = e;
+      }
+      *reinterpret_cast<uint32_t *>(out + ((long long)b * T + t0 + k) * cc + c0) = packed;
+      continue;
+    }
 #pragma unroll
     for (int j = 0; j < kConvCPT; ++j) {
       int code;

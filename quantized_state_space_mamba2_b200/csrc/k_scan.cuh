@@ -46,6 +46,9 @@ struct ScanArgs {
   // increment is rshr(ug B, g) with ug = satb(rshr(dt_q x, s_h - g), 24));
   // the method as built is hlim = 2^30 - 1, g = 0
   int hlim, guard;
+  // per-token conv-output exponents [B*T, nh + 2] (x per head, B, C) or null
+  // (the static e_x, e_B, e_C); the state and output exponents stay static
+  const int32_t *e_tok;
 };
 
 // rshr(v, g) for g in [0, 7] (g = 0: v)
@@ -66,6 +69,9 @@ __global__ void __launch_bounds__(kScanThreads) k_ssm_scan_pot(ScanArgs a) {
   __shared__ long long su[kScanTCH][kScanPC];
   __shared__ int sx[kScanTCH][kScanPC];
   __shared__ int sy[kScanTCH][kScanPC];
+  // per-token shifts (per-token exponents): u, output, skip, and the two
+  // statistic exponents of MODE 1
+  __shared__ int tsh[kScanTCH], tsy[kScanTCH], tsD[kScanTCH], tyc[kScanTCH], tyd[kScanTCH];
 
   const int tid = threadIdx.x;
   const int pp = tid / kScanTPP;
@@ -80,9 +86,6 @@ __global__ void __launch_bounds__(kScanThreads) k_ssm_scan_pot(ScanArgs a) {
   const int e_h = MODE == 2 ? e_x + e_B - 15 : a.e_h[h];
   const int e_y = MODE == 0 ? a.e_y[h] : 0;
   const int e_D = a.e_D[h];
-  const int s_h = e_h - e_B - e_x + 16;
-  const int s_y = e_y - e_C - e_h;
-  const int s_D = e_y - e_D - e_x;
   const int ef = min(e_C + e_h, e_D + e_x);
   const long long Dq = a.D_q[h];
   const long long Aq = a.A_q[h];
@@ -112,6 +115,20 @@ __global__ void __launch_bounds__(kScanThreads) k_ssm_scan_pot(ScanArgs a) {
       const int dtq = softplus_pwl(to_q16(xf));
       sdt[tid] = dtq;
       sdA[tid] = pow2_pwl(-rshr64((long long)dtq * Aq, 12));
+      int ex = e_x, eb = e_B, ec = e_C;
+      if (a.e_tok) {
+        const int32_t *et = a.e_tok + (rowbase + t0 + tid) * (nh + 2);
+        ex = et[h];
+        eb = et[nh];
+        ec = et[nh + 1];
+      }
+      // MODE 2 keeps the state at the static finest exponent: u takes the
+      // token's own shift 1 + (e_x + e_B) - (ex + eb)
+      tsh[tid] = MODE == 2 ? 1 + e_x + e_B - ex - eb : e_h - eb - ex + 16;
+      tsy[tid] = e_y - ec - e_h;
+      tsD[tid] = e_y - e_D - ex;
+      tyc[tid] = ec + e_h - ef;
+      tyd[tid] = e_D + ex - ef;
     }
     // B and C rows (contiguous 256 bytes after x), expanded to int32
     for (int i = tid; i < nt * 16; i += kScanThreads) {
@@ -138,7 +155,9 @@ __global__ void __launch_bounds__(kScanThreads) k_ssm_scan_pot(ScanArgs a) {
     for (int i = tid; i < nt * kScanPC; i += kScanThreads) {
       const int tt = i / kScanPC, q = i % kScanPC;
       const long long prod = (long long)sdt[tt] * sx[tt][q];
-      su[tt][q] = MODE == 2 ? rshr64(prod, 1) : satb64(rshr64(prod, s_h - a.guard), 24);
+      const int sh = tsh[tt];
+      su[tt][q] = MODE == 2 ? (sh >= 0 ? rshr64(prod, sh) : shl_sat61(prod, -sh))
+                            : satb64(rshr64(prod, sh - a.guard), 24);
     }
     __syncthreads();
 
@@ -177,9 +196,9 @@ __global__ void __launch_bounds__(kScanThreads) k_ssm_scan_pot(ScanArgs a) {
       for (int o = 8; o >= 1; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
       if ((tid % kScanTPP) == 0) {
         const long long dx = Dq * sx[tt][pp];
-        sy[tt][pp] = (int)satb64(rshr64(acc, s_y) + rshr64(dx, s_D), 32);
+        sy[tt][pp] = (int)satb64(rshr64(acc, tsy[tt]) + rshr64(dx, tsD[tt]), 32);
         if (MODE == 1) {
-          long long yf = shl_sat61(acc, e_C + e_h - ef) + shl_sat61(dx, e_D + e_x - ef);
+          long long yf = pow2_sat61(acc, tyc[tt]) + pow2_sat61(dx, tyd[tt]);
           const unsigned long long ay = (unsigned long long)(yf < 0 ? -yf : yf);
           smax = ay > smax ? ay : smax;
         }

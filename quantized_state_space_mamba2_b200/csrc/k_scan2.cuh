@@ -53,7 +53,18 @@ struct ScanPrepArgs {
   int32_t *bc;   // [B*T, 256]: B then C, int32
   long long *bound;  // [B, nh, Tp/16, hd]: per 16-step chunk, bound of the increments
   int guard;         // the increment's guard bits (0: the method as built)
+  // per-token conv-output exponents ([B*T, nh + 2]: x per head, B, C) or null
+  // (static); with them the prep writes each token's output shifts, s_y in the
+  // low and s_D in the high 16 bits, to osh [B, nh, Tp]
+  const int32_t *e_tok;
+  int32_t *osh;
 };
+
+__device__ __forceinline__ int pack_osh(int s_y, int s_D) {
+  return (int)(((unsigned)s_y & 0xFFFFu) | ((unsigned)s_D << 16));
+}
+__device__ __forceinline__ int osh_sy(int v) { return (int)(int16_t)(v & 0xFFFF); }
+__device__ __forceinline__ int osh_sD(int v) { return v >> 16; }
 
 // grid = (Tp / 32, nh, B), block = 256; hd == 64
 __global__ void __launch_bounds__(256) k_scan_prep(ScanPrepArgs a) {
@@ -83,6 +94,7 @@ __global__ void __launch_bounds__(256) k_scan_prep(ScanPrepArgs a) {
     for (int o = 1; o < 8; o <<= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
     if (k == 0) s_bmax[tt] = m;
   }
+  __shared__ int s_sh[kPrepTT];  // per-token u shift (per-token exponents only)
   if (tid < kPrepTT) {
     int dtq = 0, dA = 0;
     if (tid < nt) {
@@ -92,6 +104,17 @@ __global__ void __launch_bounds__(256) k_scan_prep(ScanPrepArgs a) {
     }
     s_dtq[tid] = dtq;
     a.dA[((long long)b * nh + h) * Tp + t0 + tid] = dA;
+    if (a.e_tok) {
+      int sh = 0, o = 0;
+      if (tid < nt) {
+        const int32_t *et = a.e_tok + (rowbase + t0 + tid) * (nh + 2);
+        const int ex = et[h], eb = et[nh], ec = et[nh + 1];
+        sh = a.e_h[h] - eb - ex + 16;
+        o = pack_osh(a.e_y[h] - ec - a.e_h[h], a.e_y[h] - a.e_D[h] - ex);
+      }
+      s_sh[tid] = sh;
+      a.osh[((long long)b * nh + h) * Tp + t0 + tid] = o;
+    }
   }
   {  // x tile: 32 tokens x 64 channels, 8 bytes per thread
     const int tt = tid >> 3, k = tid & 7;
@@ -109,7 +132,8 @@ __global__ void __launch_bounds__(256) k_scan_prep(ScanPrepArgs a) {
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
       const long long x = sx[tb + k][p];
-      uv[k] = (int)satb64(rshr64((long long)s_dtq[tb + k] * x, s_h - g), 24);
+      const int sh = a.e_tok ? s_sh[tb + k] : s_h;
+      uv[k] = (int)satb64(rshr64((long long)s_dtq[tb + k] * x, sh - g), 24);
       dv[k] = (int)x;
     }
     // growth bound of |h| over this thread's 8 steps (an increment
@@ -150,6 +174,7 @@ struct ScanSeqArgs {
   const int32_t *e_x, *e_C, *e_h, *e_y, *e_D;
   int32_t *state;     // [B, nh, hd, 128] or null
   int32_t *y;         // [B*T, di]
+  const int32_t *osh; // [B, nh, Tp] per-token output shifts (pack_osh) or null
 };
 
 __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes,
@@ -177,6 +202,7 @@ struct ScanSeqSmem {
     int32_t dA[TCH];
     int32_t u[PC][TCH];
     int32_t xs[PC][TCH];
+    int32_t osh[TCH];
     long long bound[PC];
   };
   Slot slot[kScanSlots];
@@ -348,8 +374,9 @@ __global__ void __launch_bounds__(PC *(128 / NPT) + 32) k_scan_seq(ScanSeqArgs a
         const int t0 = c * TCH;
         const int nt = min(TCH, T - t0);
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        mbar_arrive_expect_tx(&sm.full[sl],
-                              (uint32_t)(nt * 1024 + TCH * 4 * (1 + 2 * PC) + PC * 8));
+        mbar_arrive_expect_tx(&sm.full[sl], (uint32_t)(nt * 1024 + TCH * 4 * (1 + 2 * PC) +
+                                                       PC * 8 + (a.osh ? TCH * 4 : 0)));
+        if (a.osh) bulk_g2s(&s.osh[0], a.osh + headrow * Tp + t0, TCH * 4, &sm.full[sl]);
         bulk_g2s(&s.bound[0], a.bound + ((headrow * (Tp / 16) + c) * hd + p0), PC * 8,
                  &sm.full[sl]);
         bulk_g2s(&s.bc[0][0], a.bc + (rowbase + t0) * 256, (uint32_t)(nt * 1024), &sm.full[sl]);
@@ -421,8 +448,10 @@ __global__ void __launch_bounds__(PC *(128 / NPT) + 32) k_scan_seq(ScanSeqArgs a
       if (lane32 < nt) {
         const int2 v = wsum[lane32];
         const long long sum = S16 ? (long long)v.x : (long long)v.x * 65536 + v.y;
+        const int sy = a.osh ? osh_sy(s.osh[lane32]) : s_y;
+        const int sD = a.osh ? osh_sD(s.osh[lane32]) : s_D;
         a.y[(rowbase + t0 + lane32) * di + (long long)h * hd + p0 + pp] =
-            (int)satb64(rshr64(sum, s_y) + rshr64(Dq * s.xs[pp][lane32], s_D), 32);
+            (int)satb64(rshr64(sum, sy) + rshr64(Dq * s.xs[pp][lane32], sD), 32);
       }
     } else {
       // partials of this warp: row (step, channel-in-warp), column = lane in channel
@@ -451,8 +480,10 @@ __global__ void __launch_bounds__(PC *(128 / NPT) + 32) k_scan_seq(ScanSeqArgs a
       const int tt = row / PPW, q = warp * PPW + row % PPW;
       if (half == 0 && tt < nt) {
         const long long sum = S16 ? (long long)shi : (long long)shi * 65536 + slo;
+        const int sy = a.osh ? osh_sy(s.osh[tt]) : s_y;
+        const int sD = a.osh ? osh_sD(s.osh[tt]) : s_D;
         a.y[(rowbase + t0 + tt) * di + (long long)h * hd + p0 + q] =
-            (int)satb64(rshr64(sum, s_y) + rshr64(Dq * s.xs[q][tt], s_D), 32);
+            (int)satb64(rshr64(sum, sy) + rshr64(Dq * s.xs[q][tt], sD), 32);
       }
     }
     __syncwarp();
@@ -509,7 +540,10 @@ __global__ void __launch_bounds__(256) k_scan_step(ScanArgs a) {
   int8_t xs[kStepPPW];
 #pragma unroll
   for (int k = 0; k < kStepPPW; ++k) xs[k] = row[h * hd + warp + 8 * k];
-  const int e_x = a.e_x[h], e_B = *a.e_B, e_C = *a.e_C, e_h = a.e_h[h], e_y = a.e_y[h];
+  // per-token exponents of this sequence's token (T == 1), else the static ones
+  const int32_t *et = a.e_tok ? a.e_tok + (long long)b * (nh + 2) : nullptr;
+  const int e_x = et ? et[h] : a.e_x[h], e_B = et ? et[nh] : *a.e_B, e_C = et ? et[nh + 1] : *a.e_C;
+  const int e_h = a.e_h[h], e_y = a.e_y[h];
   const int e_D = a.e_D[h];
   const long long Dq = a.D_q[h];
   const float xf = __fadd_rn(a.dt_raw[headrow], a.dt_bias[h]);

@@ -31,7 +31,7 @@ EXPORTS = (
     "fm_set_scan_tile", "fm_ssd_workspace_bytes", "fm_ssd_scan", "fm_set_scan_mode",
     "fm_set_state_spec", "fm_lq_conv1d", "fm_lq_scan", "fm_lq_workspace_bytes",
     "fm_lq_mixer_prefill", "fm_set_fault_injection", "fm_set_gemm_splitk",
-    "fm_set_gemm_tile",
+    "fm_set_gemm_tile", "fm_set_xbc_exponents",
 )
 NOALLOC_SCRATCH_BYTES = 16 << 20  # FM_NOALLOC_SCRATCH_BYTES
 
@@ -117,6 +117,7 @@ def load():
         "fm_set_fault_injection": (I, [I, C.c_uint64]),
         "fm_set_gemm_splitk": (I, [I]),
         "fm_set_gemm_tile": (I, [I]),
+        "fm_set_xbc_exponents": (I, [I]),
         "fm_lq_mixer_prefill": (I, [lp, C.POINTER(fm_lq_params), _P, I, I, I, _P, _P, _P, _P,
                                     SZ, _P]),
     }
@@ -245,6 +246,17 @@ def set_state_spec(bits: int, guard: int):
     global STATE_BITS
     _check(load().fm_set_state_spec(bits, guard))
     STATE_BITS = bits
+
+
+XBC_EXPONENTS = "static"  # the conv-output exponent granularity in force
+
+
+def set_xbc_exponents(kind: str):
+    """'static' (per head / B / C, as built; default) or 'token' (per token);
+    process-wide, set before calibrating and sizing workspaces."""
+    global XBC_EXPONENTS
+    _check(load().fm_set_xbc_exponents({"static": 0, "token": 1}[kind]))
+    XBC_EXPONENTS = kind
 
 
 def scan_workspace_bytes(shape, B, T) -> int:

@@ -191,6 +191,14 @@ def test_chunked_scan_validation(so):
     # scan mode switch
     assert so.fm_set_scan_mode(2) == 1
     assert so.fm_set_scan_mode(0) == 0
+def test_xbc_exponent_setting_validation(so):
+    """The conv-output exponent granularity takes 0 (static) or 1 (per token)."""
+    assert so.fm_set_xbc_exponents(2) == 1
+    assert so.fm_set_xbc_exponents(-1) == 1
+    assert so.fm_set_xbc_exponents(1) == 0
+    assert so.fm_set_xbc_exponents(0) == 0
+
+
 def test_state_spec_validation(so):
     """Only the two state specs with kernels behind them are accepted."""
     assert so.fm_set_state_spec(16, 0) == 1
