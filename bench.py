@@ -95,6 +95,8 @@ def parse(argv=None):
     ap.add_argument("--eager", action="store_true",
                     help="launch the timed steps one by one instead of replaying them as one "
                          "captured CUDA graph")
+    ap.add_argument("--xbc-exponents", default="static", choices=["static", "token"],
+                    help="conv-output exponents: static per head / B / C (as built) or per token")
     ap.add_argument("--lq", action="store_true",
                     help="the FastMamba-LQ variant of a prefill workload (fp32 conv, scan, gate)")
     ap.add_argument("--modes", default="auto",
@@ -106,7 +108,7 @@ def parse(argv=None):
     return ap.parse_args(argv)
 
 
-SUB_MODES = ("static", "ssd", "state16", "lq")
+SUB_MODES = ("static", "ssd", "state16", "candidate", "lq")
 
 
 def sub_modes(args) -> list:
@@ -130,6 +132,9 @@ def variant_args(args, mode: str):
         v.scan_mode = "ssd"
     elif mode == "state16":
         v.state_spec = "16,7"
+    elif mode == "candidate":  # per-token exponents, 16-bit state, guard-bit increment
+        v.state_spec = "16,7"
+        v.xbc_exponents = "token"
     elif mode == "lq":
         v.lq = True
     return v
@@ -171,7 +176,8 @@ def config_block(args) -> dict:
                              f"{min(w.get('prefill_len', w['seqlen']), S.CALIB_MAX_LEN)} tokens "
                              "(GPU, stage by stage)",
                  scan_tile=args.scan_tile or "4,4,16", scan_mode=args.scan_mode,
-                 state_spec=args.state_spec)
+                 state_spec=args.state_spec,
+                 xbc_exponents=getattr(args, "xbc_exponents", "static"))
         if getattr(args, "lq", False):
             c.update(variant="FastMamba-LQ (W8A8 linears; fp32 conv, scan, gate)")
         if "prefill_len" in w:
@@ -412,7 +418,7 @@ def _stage_buffers(torch, d, M, dev):
                 z=e(M, d.d_inner, dt=torch.float32), xbc=e(M, d.conv_ch, dt=torch.int8),
                 dtr=e(M, d.nheads, dt=torch.float32), xo=e(M, d.conv_ch, dt=torch.int8),
                 y=e(M, d.d_inner, dt=torch.int32), q_out=e(M, d.d_inner, dt=torch.int8),
-                sx_out=e(M, dt=torch.float32))
+                sx_out=e(M, dt=torch.float32), e_tok=e(M, d.nheads + 2, dt=torch.int32))
 
 
 def _gemm_workspace(torch, lib, d, M, dev):
@@ -460,7 +466,10 @@ class StackWorkload:
         M = self.B * self.T
         self.ws = self.layers[0].workspace(self.B, self.T)
         self.ssd = getattr(args, "scan_mode", "seq") == "ssd" and self.T > 1
-        nb = (lib.ssd_workspace_bytes if self.ssd else lib.scan_workspace_bytes)(d, self.B, self.T)
+        self.tok = getattr(args, "xbc_exponents", "static") == "token"
+        nb = (lib.ssd_workspace_bytes if self.ssd else
+              lib.scan_workspace_bytes_tok if self.tok else lib.scan_workspace_bytes)(d, self.B,
+                                                                                     self.T)
         self.sws = torch.empty(nb, dtype=torch.uint8, device=dev)
         self.buf = _stage_buffers(torch, d, M, dev)
         self.tokens = M
@@ -481,12 +490,20 @@ class StackWorkload:
                                b["q_in"], b["sx_in"])
             lib.in_proj(b["q_in"], b["sx_in"], Ly.w_in_q, Ly.w_in_s, d, Ly.exps, b["z"], b["xbc"],
                         b["dtr"], ws=self.gws)
-            lib.conv1d_pot(b["xbc"], B, T, d, Ly.conv_wq, Ly.conv_bq, Ly.exps, cs, b["xo"])
+            if self.tok:
+                lib.conv1d_pot_tok(b["xbc"], B, T, d, Ly.conv_wq, Ly.conv_bq, Ly.exps, cs, b["xo"],
+                                   b["e_tok"])
+            else:
+                lib.conv1d_pot(b["xbc"], B, T, d, Ly.conv_wq, Ly.conv_bq, Ly.exps, cs, b["xo"])
             if ev is not None:
                 ev[i][0].record(stream)
-            scan = lib.ssd_scan if self.ssd else lib.ssm_scan_pot
-            scan(b["xo"], b["dtr"], B, T, d, Ly.dt_bias, Ly.A_q, Ly.D_q, Ly.exps, ss, b["y"],
-                 self.sws)
+            if self.tok:
+                lib.ssm_scan_pot_tok(b["xo"], b["dtr"], B, T, d, Ly.dt_bias, Ly.A_q, Ly.D_q,
+                                     Ly.exps, b["e_tok"], ss, b["y"], self.sws)
+            else:
+                scan = lib.ssd_scan if self.ssd else lib.ssm_scan_pot
+                scan(b["xo"], b["dtr"], B, T, d, Ly.dt_bias, Ly.A_q, Ly.D_q, Ly.exps, ss, b["y"],
+                     self.sws)
             if ev is not None:
                 ev[i][1].record(stream)
             lib.gate_norm_quant(b["y"], b["z"], d, Ly.exps, Ly.norm_w, 1, self.mode,
@@ -566,6 +583,7 @@ class DecodeWorkload(StackWorkload):
         self.n_layers, self.B, self.T = n_layers(args), w["batch"], 1
         self.stack_mode = True
         self.ssd = False  # a single-token step always runs the sequential scan step
+        self.tok = getattr(args, "xbc_exponents", "static") == "token"
         self.mode = lib.FM_DYNAMIC if args.mode == "dynamic" else lib.FM_STATIC
         P = w["prefill_len"]
         self.stack = DeviceStack([S.layer_params(d, 1000 + l) for l in range(self.n_layers)], d,
@@ -915,6 +933,7 @@ def apply_modes(args, lib):
     lib.set_scan_mode(args.scan_mode)
     lib.set_state_spec(*[int(v) for v in args.state_spec.split(",")])
     lib.set_gemm_tile(args.gemm_tile)
+    lib.set_xbc_exponents(args.xbc_exponents)
 
 
 def main():

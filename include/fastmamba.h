@@ -215,6 +215,14 @@ fm_status fm_conv1d_pot(const int8_t *u, int B, int T, const fm_shape *shape, co
                         const int32_t *bq, const int32_t *exps, int8_t *conv_state, int8_t *out,
                         fm_stream stream);
 
+/* The same conv with per-token output exponents (see fm_set_xbc_exponents):
+ * e_tok [B*T, nheads + 2] int32 receives each token's exponents of its heads'
+ * x channels, of B and of C; the codes in `out` are at those exponents.
+ * Independent of the process-wide setting. */
+fm_status fm_conv1d_pot_tok(const int8_t *u, int B, int T, const fm_shape *shape,
+                            const int8_t *wq, const int32_t *bq, const int32_t *exps,
+                            int8_t *conv_state, int8_t *out, int32_t *e_tok, fm_stream stream);
+
 /* ------------------------------------------------------------------ */
 /* a5 - a8: selective scan in power-of-two fixed point                  */
 /* ------------------------------------------------------------------ */
@@ -250,6 +258,16 @@ fm_status fm_ssm_scan_pot(const int8_t *xbc, const float *dt_raw, int B, int T,
                           const fm_shape *shape, const float *dt_bias, const int32_t *A_q,
                           const int32_t *D_q, const int32_t *exps, int32_t *state, int32_t *y,
                           void *ws, size_t ws_bytes, fm_stream stream);
+/* The same scan on codes at per-token exponents (e_tok from fm_conv1d_pot_tok):
+ * per token, s_h = e_h - e_B,t - e_x,t + 16, the output shift
+ * e_y - e_C,t - e_h and the skip shift e_y - e_D - e_x,t.  Its workspace,
+ * fm_scan_workspace_bytes_tok, also holds the per-token shifts. */
+size_t fm_scan_workspace_bytes_tok(const fm_shape *shape, int B, int T);
+fm_status fm_ssm_scan_pot_tok(const int8_t *xbc, const float *dt_raw, int B, int T,
+                              const fm_shape *shape, const float *dt_bias, const int32_t *A_q,
+                              const int32_t *D_q, const int32_t *exps, const int32_t *e_tok,
+                              int32_t *state, int32_t *y, void *ws, size_t ws_bytes,
+                              fm_stream stream);
 
 /* ------------------------------------------------------------------ */
 /* a9 + a10: gate, gated RMSNorm, rotation, int8 quantisation           */

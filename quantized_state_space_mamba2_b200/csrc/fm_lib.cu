@@ -800,6 +800,25 @@ extern "C" fm_status fm_conv1d_pot(const int8_t *u, int B, int T, const fm_shape
   return launch_conv(u, B, T, d.cc, wq, bq, exps, conv_state, out, nullptr, (cudaStream_t)stream);
 }
 
+extern "C" fm_status fm_conv1d_pot_tok(const int8_t *u, int B, int T, const fm_shape *shape,
+                                       const int8_t *wq, const int32_t *bq, const int32_t *exps,
+                                       int8_t *conv_state, int8_t *out, int32_t *e_tok,
+                                       fm_stream stream) {
+  Dims d;
+  FM_TRY(check_shape(shape, &d, __func__));
+  if (B < 0 || T < 0) return fail(FM_ERR_SHAPE, "fm_conv1d_pot_tok: B, T must be >= 0");
+  if ((long long)B * T == 0) return FM_OK;
+  NEED(u);
+  NEED(wq);
+  NEED(bq);
+  NEED(exps);
+  NEED(out);
+  NEED(e_tok);
+  OPT(conv_state);
+  return launch_conv(u, B, T, d.cc, wq, bq, exps, conv_state, out, nullptr, (cudaStream_t)stream,
+                     e_tok, &d);
+}
+
 namespace {
 struct Carver {
   uint8_t *base;
@@ -813,7 +832,7 @@ struct Carver {
   }
 };
 
-ScanWs carve_scan(Carver &c, const Dims &d, int B, int T) {
+ScanWs carve_scan(Carver &c, const Dims &d, int B, int T, bool tok) {
   ScanWs w;
   w.osh = nullptr;
   if (T == 1) {  // single steps run k_scan_step, which stages nothing
@@ -828,17 +847,23 @@ ScanWs carve_scan(Carver &c, const Dims &d, int B, int T) {
   w.xs = c.take<int32_t>((long long)B * d.di * Tp);
   w.bc = c.take<int32_t>(M * 256);
   w.bound = c.take<long long>((long long)B * d.di * (Tp / 16));
-  if (xbc_tok()) w.osh = c.take<int32_t>((long long)B * d.nh * Tp);
+  if (tok) w.osh = c.take<int32_t>((long long)B * d.nh * Tp);
   return w;
 }
 }  // namespace
 
-extern "C" size_t fm_scan_workspace_bytes(const fm_shape *shape, int B, int T) {
+static size_t scan_ws_bytes(const fm_shape *shape, int B, int T, bool tok) {
   Dims d;
-  if (check_shape(shape, &d, __func__) != FM_OK || B < 0 || T < 0) return 0;
+  if (check_shape(shape, &d, "fm_scan_workspace_bytes") != FM_OK || B < 0 || T < 0) return 0;
   Carver c{nullptr, 0};
-  carve_scan(c, d, B, T);
+  carve_scan(c, d, B, T, tok);
   return c.off + 256;
+}
+extern "C" size_t fm_scan_workspace_bytes(const fm_shape *shape, int B, int T) {
+  return scan_ws_bytes(shape, B, T, false);
+}
+extern "C" size_t fm_scan_workspace_bytes_tok(const fm_shape *shape, int B, int T) {
+  return scan_ws_bytes(shape, B, T, true);
 }
 
 extern "C" fm_status fm_ssm_scan_pot(const int8_t *xbc, const float *dt_raw, int B, int T,
@@ -862,10 +887,40 @@ extern "C" fm_status fm_ssm_scan_pot(const int8_t *xbc, const float *dt_raw, int
   if (!ws || ws_bytes < need || !aligned16(ws))
     return fail(FM_ERR_WORKSPACE, "fm_ssm_scan_pot: workspace needs %zu bytes", need);
   Carver c{reinterpret_cast<uint8_t *>(ws), 0};
-  const ScanWs w = carve_scan(c, d, B, T);
+  const ScanWs w = carve_scan(c, d, B, T, false);
   const fm_exp_layout X = fm_exp_table_layout(shape);
   return launch_scan_v2(scan_args(d, xbc, dt_raw, T, dt_bias, A_q, D_q, exps, X, state, y, nullptr),
                         B, w, (cudaStream_t)stream);
+}
+
+extern "C" fm_status fm_ssm_scan_pot_tok(const int8_t *xbc, const float *dt_raw, int B, int T,
+                                         const fm_shape *shape, const float *dt_bias,
+                                         const int32_t *A_q, const int32_t *D_q,
+                                         const int32_t *exps, const int32_t *e_tok,
+                                         int32_t *state, int32_t *y, void *ws, size_t ws_bytes,
+                                         fm_stream stream) {
+  Dims d;
+  FM_TRY(check_shape(shape, &d, __func__));
+  if (B < 0 || T < 0) return fail(FM_ERR_SHAPE, "fm_ssm_scan_pot_tok: B, T must be >= 0");
+  if ((long long)B * T == 0) return FM_OK;
+  NEED(xbc);
+  NEED(dt_raw);
+  NEED(dt_bias);
+  NEED(A_q);
+  NEED(D_q);
+  NEED(exps);
+  NEED(e_tok);
+  NEED(y);
+  OPT(state);
+  const size_t need = fm_scan_workspace_bytes_tok(shape, B, T);
+  if (!ws || ws_bytes < need || !aligned16(ws))
+    return fail(FM_ERR_WORKSPACE, "fm_ssm_scan_pot_tok: workspace needs %zu bytes", need);
+  Carver c{reinterpret_cast<uint8_t *>(ws), 0};
+  const ScanWs w = carve_scan(c, d, B, T, true);
+  const fm_exp_layout X = fm_exp_table_layout(shape);
+  return launch_scan_v2(
+      scan_args(d, xbc, dt_raw, T, dt_bias, A_q, D_q, exps, X, state, y, nullptr, e_tok), B, w,
+      (cudaStream_t)stream);
 }
 
 // ------------------------------------------------------------------ chunked scan mode
@@ -1068,7 +1123,7 @@ MixerWs carve_mixer(Carver &c, const Dims &d, int B, int T) {
   w.y = c.take<int32_t>(M * d.di);
   w.q_out = c.take<int8_t>(M * d.di);
   w.sx_out = c.take<float>(M);
-  w.scan = carve_scan(c, d, B, T);
+  w.scan = carve_scan(c, d, B, T, xbc_tok());
   w.e_tok = xbc_tok() ? c.take<int32_t>(M * (d.nh + 2)) : nullptr;
   if (use_ssd(T)) {
     w.ssd = carve_ssd(c, d, B, T);

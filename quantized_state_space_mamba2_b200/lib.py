@@ -31,7 +31,8 @@ EXPORTS = (
     "fm_set_scan_tile", "fm_ssd_workspace_bytes", "fm_ssd_scan", "fm_set_scan_mode",
     "fm_set_state_spec", "fm_lq_conv1d", "fm_lq_scan", "fm_lq_workspace_bytes",
     "fm_lq_mixer_prefill", "fm_set_fault_injection", "fm_set_gemm_splitk",
-    "fm_set_gemm_tile", "fm_set_xbc_exponents",
+    "fm_set_gemm_tile", "fm_set_xbc_exponents", "fm_conv1d_pot_tok", "fm_ssm_scan_pot_tok",
+    "fm_scan_workspace_bytes_tok",
 )
 NOALLOC_SCRATCH_BYTES = 16 << 20  # FM_NOALLOC_SCRATCH_BYTES
 
@@ -118,6 +119,9 @@ def load():
         "fm_set_gemm_splitk": (I, [I]),
         "fm_set_gemm_tile": (I, [I]),
         "fm_set_xbc_exponents": (I, [I]),
+        "fm_conv1d_pot_tok": (I, [_P, I, I, sp, _P, _P, _P, _P, _P, _P, _P]),
+        "fm_ssm_scan_pot_tok": (I, [_P, _P, I, I, sp, _P, _P, _P, _P, _P, _P, _P, _P, SZ, _P]),
+        "fm_scan_workspace_bytes_tok": (SZ, [sp, I, I]),
         "fm_lq_mixer_prefill": (I, [lp, C.POINTER(fm_lq_params), _P, I, I, I, _P, _P, _P, _P,
                                     SZ, _P]),
     }
@@ -229,6 +233,12 @@ def conv1d_pot(u, B, T, shape, wq, bq, exps, conv_state, out, stream=None):
                                 _p(conv_state), _p(out), _s(stream)))
 
 
+def conv1d_pot_tok(u, B, T, shape, wq, bq, exps, conv_state, out, e_tok, stream=None):
+    sh = shape_struct(shape)
+    _check(load().fm_conv1d_pot_tok(_p(u), B, T, C.byref(sh), _p(wq), _p(bq), _p(exps),
+                                    _p(conv_state), _p(out), _p(e_tok), _s(stream)))
+
+
 SCAN_TILES = ((4, 4, 16), (4, 2, 16), (4, 8, 16), (8, 4, 16), (8, 2, 16), (8, 8, 16))
 
 
@@ -268,6 +278,18 @@ def ssm_scan_pot(xbc, dt_raw, B, T, shape, dt_bias, A_q, D_q, exps, state, y, ws
     _check(load().fm_ssm_scan_pot(_p(xbc), _p(dt_raw), B, T, C.byref(sh), _p(dt_bias), _p(A_q),
                                   _p(D_q), _p(exps), _p(state), _p(y), _p(ws),
                                   ws.numel() * ws.element_size(), _s(stream)))
+
+
+def scan_workspace_bytes_tok(shape, B, T) -> int:
+    return load().fm_scan_workspace_bytes_tok(C.byref(shape_struct(shape)), B, T)
+
+
+def ssm_scan_pot_tok(xbc, dt_raw, B, T, shape, dt_bias, A_q, D_q, exps, e_tok, state, y, ws,
+                     stream=None):
+    sh = shape_struct(shape)
+    _check(load().fm_ssm_scan_pot_tok(_p(xbc), _p(dt_raw), B, T, C.byref(sh), _p(dt_bias),
+                                      _p(A_q), _p(D_q), _p(exps), _p(e_tok), _p(state), _p(y),
+                                      _p(ws), ws.numel() * ws.element_size(), _s(stream)))
 
 
 SCAN_MODES = {"seq": 0, "ssd": 1}

@@ -106,7 +106,7 @@ def test_sub_record_modes():
     static, chunked-scan, 16-bit-state and LQ modes follow as sub-records;
     each sub-record differs from the headline in exactly one setting."""
     a = bench.parse([])
-    assert bench.sub_modes(a) == ["static", "ssd", "state16", "lq"]
+    assert bench.sub_modes(a) == ["static", "ssd", "state16", "candidate", "lq"]
     assert bench.sub_modes(bench.parse(["--modes", "none"])) == []
     assert bench.sub_modes(bench.parse(["--workload", "stack2p7b_64l_b2_t4096"])) == []
     assert bench.sub_modes(bench.parse(["--workload", "stack2p7b_64l_b2_t4096",
@@ -114,9 +114,10 @@ def test_sub_record_modes():
     with pytest.raises(SystemExit):
         bench.sub_modes(bench.parse(["--modes", "fast"]))
     base = bench.config_block(a)
-    for m, key in (("static", "act_quant"), ("ssd", "scan_mode"), ("state16", "state_spec"),
-                   ("lq", "variant")):
+    for m, keys in (("static", {"act_quant"}), ("ssd", {"scan_mode"}),
+                    ("state16", {"state_spec"}), ("candidate", {"state_spec", "xbc_exponents"}),
+                    ("lq", {"variant"})):
         v = bench.variant_args(a, m)
         diff = {k for k, x in bench.config_block(v).items() if base.get(k) != x}
-        assert diff == {key}, (m, diff)
+        assert diff == keys, (m, diff)
     assert not a.lq and a.mode == "dynamic"          # the headline's args are untouched

@@ -92,3 +92,42 @@ def test_per_token_refused_by_the_chunked_scan(L):
     finally:
         L.set_scan_mode("seq")
         L.set_xbc_exponents("static")
+
+
+@pytest.mark.parametrize("B,T", [(1, 1), (2, 37), (1, 300)])
+def test_standalone_per_token_conv_and_scan(L, B, T):
+    """fm_conv1d_pot_tok and fm_ssm_scan_pot_tok (independent of the
+    process-wide setting) against the oracle's per-token requantisation and
+    scan, on a calibrated layer's tables and random in_proj codes."""
+    s = MAMBA130
+    P = S.layer_params(s, 1002, conv_bias_std=0.05)
+    xcal = S.calibration_batch(s.d_model, 64, 8, 50.0, 4242, n_seqs=1)
+    ol = O.prepare_layer(P, s, xbc_exponents="token")
+    O.calibrate_layer(ol, xcal)
+    from quantized_state_space_mamba2_b200.model import DeviceLayer
+    L.set_xbc_exponents("token")
+    try:
+        dl = DeviceLayer(P, s)
+        dl.calibrate(dev(xcal))
+    finally:
+        L.set_xbc_exponents("static")
+    u = S.uniform_ints((B, T, s.conv_ch), -127, 127, seed=61 + T, dtype=np.int8)
+    dt_raw = S.normal((B, T, s.nheads), 1.0, seed=62 + T)
+    st = S.uniform_ints((B, s.nheads, s.headdim, s.d_state), -2 ** 20, 2 ** 20, seed=63)
+    xo = torch.empty((B, T, s.conv_ch), dtype=torch.int8, device="cuda")
+    e_tok = torch.empty((B * T, s.nheads + 2), dtype=torch.int32, device="cuda")
+    L.conv1d_pot_tok(dev(u), B, T, s, dl.conv_wq, dl.conv_bq, dl.exps, None, xo, e_tok)
+    xo_r, et_r = O.conv_out(ol, u)
+    assert np.array_equal(host(xo), xo_r)
+    assert np.array_equal(host(e_tok).reshape(et_r.shape), et_r)
+    y = torch.empty((B, T, s.d_inner), dtype=torch.int32, device="cuda")
+    std = dev(st)
+    ws = torch.empty(L.scan_workspace_bytes_tok(s, B, T), dtype=torch.uint8, device="cuda")
+    L.ssm_scan_pot_tok(xo, dev(dt_raw), B, T, s, dl.dt_bias, dl.A_q, dl.D_q, dl.exps, e_tok, std,
+                       y, ws)
+    L.sync_status()
+    st_r = st.copy()
+    y_r = O.ssm_scan_pot(xo_r, dt_raw, ol.dt_bias, ol.A_q, ol.D_q, ol.e_x, ol.e_B, ol.e_C, ol.e_h,
+                         ol.e_y, ol.e_D, s.headdim, s.d_state, state=st_r, e_tok=et_r)
+    assert np.array_equal(host(y), y_r)
+    assert np.array_equal(host(std), st_r)
