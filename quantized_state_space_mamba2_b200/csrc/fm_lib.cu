@@ -554,7 +554,10 @@ static fm_status launch_scan_v2(const ScanArgs &a, int B, const ScanWs &w, cudaS
   if (M == 0) return FM_OK;
   if (B > 65535 || M > 2147483647LL) return fail(FM_ERR_SHAPE, "scan: B or B*T too large");
   if (a.T == 1) {  // decode: one step per sequence, no staging
-    k_scan_step<<<dim3(a.nh, B), 256, 0, s>>>(a);
+    if (a.hlim <= kH16Lim)
+      k_scan_step<true><<<dim3(a.nh, B), 256, 0, s>>>(a);
+    else
+      k_scan_step<false><<<dim3(a.nh, B), 256, 0, s>>>(a);
     return launched("k_scan_step");
   }
   const long long Tp = scan_tpad(a.T);

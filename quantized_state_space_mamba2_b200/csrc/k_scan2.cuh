@@ -509,30 +509,36 @@ __global__ void __launch_bounds__(PC *(128 / NPT) + 32) k_scan_seq(ScanSeqArgs a
 // arithmetic as one step of k_scan_seq with the clamp.  Grid (nh, B), block 256.
 constexpr int kStepPPW = 8;  // channels per warp (hd / 8 warps)
 
+// NARROW: the 16-bit state spec, the state stored as int16 (4 columns = 8
+// bytes per load).  Either way all eight state loads are issued before any is
+// used.
+template <bool NARROW>
 __global__ void __launch_bounds__(256) k_scan_step(ScanArgs a) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int h = blockIdx.x, b = blockIdx.y;
   const int nh = a.nh, hd = a.hd, cc = a.cc, di = a.di;
   const int n0 = lane * 4;
   const long long headrow = (long long)b * nh + h;
-  // the narrow spec stores the state as int16: 4 columns = 8 bytes per load
-  const bool narrow = a.hlim <= kH16Lim;
+  constexpr bool narrow = NARROW;
   int4 *st = a.state ? reinterpret_cast<int4 *>(a.state + headrow * hd * 128) : nullptr;
   int2 *st16 = a.state ? reinterpret_cast<int2 *>(reinterpret_cast<int16_t *>(a.state) +
                                                   headrow * hd * 128)
                        : nullptr;
   int4 hv[kStepPPW];
+  if (!a.state) {
 #pragma unroll
-  for (int k = 0; k < kStepPPW; ++k) {
-    if (!a.state) {
-      hv[k] = make_int4(0, 0, 0, 0);
-    } else if (narrow) {
-      const int2 w = __ldcs(st16 + (warp + 8 * k) * 32 + lane);
-      hv[k] = make_int4((int)(int16_t)(w.x & 0xFFFF), w.x >> 16, (int)(int16_t)(w.y & 0xFFFF),
-                        w.y >> 16);
-    } else {
-      hv[k] = __ldcs(st + (warp + 8 * k) * 32 + lane);
-    }
+    for (int k = 0; k < kStepPPW; ++k) hv[k] = make_int4(0, 0, 0, 0);
+  } else if constexpr (NARROW) {
+    int2 w[kStepPPW];
+#pragma unroll
+    for (int k = 0; k < kStepPPW; ++k) w[k] = __ldcs(st16 + (warp + 8 * k) * 32 + lane);
+#pragma unroll
+    for (int k = 0; k < kStepPPW; ++k)
+      hv[k] = make_int4((int)(int16_t)(w[k].x & 0xFFFF), w[k].x >> 16,
+                        (int)(int16_t)(w[k].y & 0xFFFF), w[k].y >> 16);
+  } else {
+#pragma unroll
+    for (int k = 0; k < kStepPPW; ++k) hv[k] = __ldcs(st + (warp + 8 * k) * 32 + lane);
   }
   const int8_t *row = a.xbc + (long long)b * cc;
   const uint32_t bw = *reinterpret_cast<const uint32_t *>(row + di + n0);
@@ -566,7 +572,7 @@ __global__ void __launch_bounds__(256) k_scan_step(ScanArgs a) {
     const int hs[4] = {hv[k].x, hv[k].y, hv[k].z, hv[k].w};
     int hn[4];
     int ahi = 0, alo = 0;
-    if (narrow) {
+    if constexpr (NARROW) {
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int t = dA * hs[j] + 0x8000;
