@@ -152,12 +152,14 @@ __global__ void __launch_bounds__(kSsdThreads) k_ssd_state(SsdArgs a) {
   }
   if (warp == 0) tmem_alloc(slot, 64);
   // raw code tiles, zero past the end of the sequence
+#pragma unroll
   for (int i = t; i < kSsdQ * 8; i += kSsdThreads) {
     const int s = i >> 3, k = i & 7;
     uint4 v = make_uint4(0u, 0u, 0u, 0u);
     if (s < nt) v = *reinterpret_cast<const uint4 *>(a.xbc + (row0 + s) * a.cc + a.di + k * 16);
     *reinterpret_cast<uint4 *>(Bt + s * 128 + k * 16) = v;
   }
+#pragma unroll
   for (int i = t; i < kSsdQ * 4; i += kSsdThreads) {
     const int s = i >> 2, k = i & 3;
     uint4 v = make_uint4(0u, 0u, 0u, 0u);
@@ -328,6 +330,7 @@ __global__ void __launch_bounds__(kSsdThreads) k_ssd_out(SsdArgs a) {
   // the chunk's B and C rows (int8 operands of G) and x codes, zero past the
   // end: 16 threads per token row (the B | C bytes are contiguous), so each
   // warp load covers two whole 256-byte rows
+#pragma unroll
   for (int i = t; i < kSsdQ * 16; i += kSsdThreads) {
     const int s = i >> 4, k = i & 15;
     uint4 v = make_uint4(0u, 0u, 0u, 0u);
@@ -335,6 +338,7 @@ __global__ void __launch_bounds__(kSsdThreads) k_ssd_out(SsdArgs a) {
     uint8_t *dst = k < 8 ? sB8 + sw128_off(s, k * 16, kSsdQ) : sC8 + sw128_off(s, (k - 8) * 16, kSsdQ);
     *reinterpret_cast<uint4 *>(dst) = v;
   }
+#pragma unroll
   for (int i = t; i < kSsdQ * 4; i += kSsdThreads) {
     const int s = i >> 2, k = i & 3;
     uint4 v = make_uint4(0u, 0u, 0u, 0u);
@@ -369,6 +373,7 @@ __global__ void __launch_bounds__(kSsdThreads) k_ssd_out(SsdArgs a) {
   }
   {  // the bf16 state entering the chunk, rows p: 64 x 256 bytes
     const uint4 *src = reinterpret_cast<const uint4 *>(a.Hin + (bh * a.nch + c) * (kSsdHd * kSsdDs));
+#pragma unroll
     for (int i = t; i < kSsdHd * 16; i += kSsdThreads) {
       const int p = i >> 4, j = i & 15;  // 16-byte piece j of row p
       *reinterpret_cast<uint4 *>(sH + sw128_off(p, j * 16, kSsdHd)) = src[i];
@@ -489,6 +494,7 @@ __global__ void __launch_bounds__(kSsdThreads) k_ssd_out(SsdArgs a) {
   }
   __syncthreads();
   if (ok) {  // 16 threads per token row of 64 int32
+#pragma unroll
     for (int i = t; i < kSsdQ * 16; i += kSsdThreads) {
       const int s = i >> 4, k = i & 15;
       if (s < nt)
