@@ -87,6 +87,13 @@ fm_status fm_sync_status(fm_stream stream);
  * fm_set_fault_injection(0, 0) restores normal operation.  Synchronous
  * (cudaMemcpyToSymbol); not for use while the device runs library kernels. */
 fm_status fm_set_fault_injection(int stall_mask, uint64_t wait_limit_ns);
+/* Tuning, process-wide (the pages have no counterpart): 1 launches the hot
+ * kernels with programmatic stream serialisation, so that each may be
+ * scheduled while its predecessor in the stream drains (every such kernel
+ * waits for its predecessor before its first global memory access); 0
+ * (default) launches them plainly.  Results are the same bits either way.
+ * FM_ERR_INVALID_ARG for other values. */
+fm_status fm_set_pdl(int enable);
 /* Library ABI version (major * 100 + minor). */
 int fm_version(void);
 

@@ -24,6 +24,13 @@ constexpr unsigned int kErrNonfinite = 2u;
 
 __device__ __forceinline__ void raise_error(unsigned int bits) { atomicOr(&g_error_word, bits); }
 
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialisation may start while its predecessor in the stream drains; it
+// waits here, before its first global memory access, until the predecessor
+// has completed and its writes are visible.  Without that launch attribute
+// this returns at once.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ---------------------------------------------------------------- integers
 __device__ __forceinline__ long long rshr64(long long a, int s) {
   if (s > 0) return (a + (1LL << (s - 1))) >> s;  // >> on signed is arithmetic (floor)

@@ -60,6 +60,37 @@ static fm_status launched(const char *what) {
   return FM_OK;
 }
 
+// Programmatic dependent launch of the hot-path kernels, process-wide (off by
+// default): with it a kernel may be scheduled while its predecessor in the
+// stream drains; every kernel launched this way waits (pdl_wait) before its
+// first global memory access.
+static std::atomic<int> g_pdl{0};
+
+extern "C" fm_status fm_set_pdl(int enable) {
+  if (enable != 0 && enable != 1) return fail(FM_ERR_INVALID_ARG, "fm_set_pdl: enable must be 0 or 1");
+  g_pdl.store(enable, std::memory_order_relaxed);
+  return FM_OK;
+}
+
+template <typename... KArgs, typename... Args>
+static fm_status launch_ex(const char *name, void (*kern)(KArgs...), dim3 grid, dim3 block,
+                           size_t smem, cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = g_pdl.load(std::memory_order_relaxed) ? 1 : 0;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, args...);
+  if (e != cudaSuccess) return fail(FM_ERR_CUDA, "launch of %s: %s", name, cudaGetErrorString(e));
+  return FM_OK;
+}
+
 extern "C" const char *fm_status_string(fm_status s) {
   switch (s) {
     case FM_OK: return "FM_OK";
@@ -297,11 +328,12 @@ static fm_status launch_gemm_t(const CUtensorMap &ta, const CUtensorMap &tb, lon
   }
   dim3 grid((unsigned)((N + BN - 1) / BN), (unsigned)((M + kGemmBM - 1) / kGemmBM),
             (unsigned)splits);
-  kern<<<grid, kGemmThreads, smem, s>>>(ta, tb, nkb, kbs, ep);
+  FM_TRY(launch_ex("k_gemm_i8_tc", kern, grid, kGemmThreads, smem, s, ta, tb, nkb, kbs, ep));
   FM_TRY(launched("k_gemm_i8_tc"));
   if (splits > 1) {
     const long long n = M * ((N + 31) / 32);
-    k_gemm_splitk_epilogue<<<(unsigned)((n + 127) / 128), 128, 0, s>>>(ep);
+    FM_TRY(launch_ex("k_gemm_splitk_epilogue", k_gemm_splitk_epilogue, (unsigned)((n + 127) / 128),
+                     128, 0, s, ep));
     FM_TRY(launched("k_gemm_splitk_epilogue"));
   }
   return FM_OK;
@@ -320,8 +352,8 @@ static fm_status launch_gemm_persist(const CUtensorMap &ta, const CUtensorMap &t
   const int m_tiles = (int)((M + kGemmBM - 1) / kGemmBM), n_tiles = (int)((N + BN - 1) / BN);
   const long long tiles = (long long)m_tiles * n_tiles;
   const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);
-  kern<<<grid, 64 + 32 * EW, smem, s>>>(ta, tb, to[0], to[1], to[2], (int)(K / kGemmBK), m_tiles,
-                                        n_tiles, ep);
+  FM_TRY(launch_ex("k_gemm_i8_persist", kern, grid, 64 + 32 * EW, smem, s, ta, tb, to[0], to[1],
+                   to[2], (int)(K / kGemmBK), m_tiles, n_tiles, ep));
   return launched("k_gemm_i8_persist");
 }
 
@@ -395,11 +427,11 @@ static fm_status launch_hadamard_quant(const float *x, long long M, int K, const
   // fill the GPU; a handful of rows (a decode batch) keeps one per warp
   const int nb = K / 256;
   if (nb % 2 == 0 && M >= 2LL * sm_count())
-    k_hadamard_quant<2><<<(unsigned)M, 32 * (nb / 2), 0, s>>>(x, K, prenorm_w, rotate, mode,
-                                                              static_amax, q, s_x, amax_row);
+    FM_TRY(launch_ex("k_hadamard_quant", k_hadamard_quant<2>, (unsigned)M, 32 * (nb / 2), 0, s, x,
+                     K, prenorm_w, rotate, mode, static_amax, q, s_x, amax_row));
   else
-    k_hadamard_quant<1><<<(unsigned)M, 32 * nb, 0, s>>>(x, K, prenorm_w, rotate, mode,
-                                                        static_amax, q, s_x, amax_row);
+    FM_TRY(launch_ex("k_hadamard_quant", k_hadamard_quant<1>, (unsigned)M, 32 * nb, 0, s, x, K,
+                     prenorm_w, rotate, mode, static_amax, q, s_x, amax_row));
   return launched("k_hadamard_quant");
 }
 
@@ -414,17 +446,19 @@ static fm_status launch_conv(const int8_t *u, int B, int T, int cc, const int8_t
   const int di = d ? d->di : 0, hd = d ? d->hd : 0, ds = d ? d->ds : 0;
   if (T >= kConvTT) {
     const unsigned tiles = (unsigned)((T + kConvTokens - 1) / kConvTokens);
-    k_conv1d_pot<kConvTT, kConvTG><<<dim3(tiles, groups, B), kConvQuads * kConvTG, 0, s>>>(
-        u, T, cc, wq, bq, exps, conv_state, out, amax, nullptr, e_tok, di, hd, ds);
+    FM_TRY(launch_ex("k_conv1d_pot", k_conv1d_pot<kConvTT, kConvTG>, dim3(tiles, groups, B),
+                     kConvQuads * kConvTG, 0, s, u, T, cc, wq, bq, exps, conv_state, out, amax,
+                     nullptr, e_tok, di, hd, ds));
   } else {  // decode steps and short chunks: one token per thread
-    k_conv1d_pot<1, 1><<<dim3((unsigned)T, groups, B), kConvQuads, 0, s>>>(
-        u, T, cc, wq, bq, exps, conv_state, out, amax, T == 1 ? conv_state : nullptr, e_tok, di,
-        hd, ds);
+    FM_TRY(launch_ex("k_conv1d_pot", k_conv1d_pot<1, 1>, dim3((unsigned)T, groups, B), kConvQuads,
+                     0, s, u, T, cc, wq, bq, exps, conv_state, out, amax,
+                     T == 1 ? conv_state : nullptr, e_tok, di, hd, ds));
   }
   FM_TRY(launched("k_conv1d_pot"));
   if (conv_state && T > 1) {  // a single step updates its state in the conv kernel
     const long long n = (long long)B * cc;
-    k_conv_state_update<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(u, B, T, cc, conv_state);
+    FM_TRY(launch_ex("k_conv_state_update", k_conv_state_update, (unsigned)((n + 255) / 256), 256,
+                     0, s, u, B, T, cc, conv_state));
     FM_TRY(launched("k_conv_state_update"));
   }
   return FM_OK;
@@ -535,7 +569,7 @@ static fm_status launch_seq(const ScanSeqArgs &a, int B, cudaStream_t s) {
   auto kern = k_scan_seq<NPT, PC, TCH, S16>;
   FM_CHECK_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
   dim3 grid(a.hd / PC, a.nh, B);
-  kern<<<grid, PC * (128 / NPT) + 32, smem, s>>>(a);
+  FM_TRY(launch_ex("k_scan_seq", kern, grid, PC * (128 / NPT) + 32, smem, s, a));
   return launched("k_scan_seq");
 }
 
@@ -555,9 +589,9 @@ static fm_status launch_scan_v2(const ScanArgs &a, int B, const ScanWs &w, cudaS
   if (B > 65535 || M > 2147483647LL) return fail(FM_ERR_SHAPE, "scan: B or B*T too large");
   if (a.T == 1) {  // decode: one step per sequence, no staging
     if (a.hlim <= kH16Lim)
-      k_scan_step<true><<<dim3(a.nh, B), 256, 0, s>>>(a);
+      FM_TRY(launch_ex("k_scan_step", k_scan_step<true>, dim3(a.nh, B), 256, 0, s, a));
     else
-      k_scan_step<false><<<dim3(a.nh, B), 256, 0, s>>>(a);
+      FM_TRY(launch_ex("k_scan_step", k_scan_step<false>, dim3(a.nh, B), 256, 0, s, a));
     return launched("k_scan_step");
   }
   const long long Tp = scan_tpad(a.T);
@@ -586,7 +620,8 @@ static fm_status launch_scan_v2(const ScanArgs &a, int B, const ScanWs &w, cudaS
   p.e_tok = a.e_tok;
   p.osh = a.e_tok ? w.osh : nullptr;
   if (a.e_tok && !w.osh) return fail(FM_ERR_WORKSPACE, "scan: per-token shifts need workspace");
-  k_scan_prep<<<dim3((unsigned)(Tp / kPrepTT), a.nh, B), 256, 0, s>>>(p);
+  FM_TRY(launch_ex("k_scan_prep", k_scan_prep, dim3((unsigned)(Tp / kPrepTT), a.nh, B), 256, 0, s,
+                   p));
   FM_TRY(launched("k_scan_prep"));
   ScanSeqArgs q;
   q.dA = w.dA;
@@ -1017,11 +1052,12 @@ static fm_status launch_ssd(const Dims &d, const int8_t *xbc, const float *dt_ra
                                      SsdStateSmem::kBytes));
   FM_CHECK_CUDA(cudaFuncSetAttribute(k_ssd_out, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      SsdOutSmem::kBytes));
-  k_ssd_state<<<grid, kSsdThreads, SsdStateSmem::kBytes, s>>>(a);
+  FM_TRY(launch_ex("k_ssd_state", k_ssd_state, grid, kSsdThreads, SsdStateSmem::kBytes, s, a));
   FM_TRY(launched("k_ssd_state"));
-  k_ssd_pass<<<dim3(kSsdHd * kSsdDs / 256, (unsigned)d.nh, (unsigned)B), 256, 0, s>>>(a);
+  FM_TRY(launch_ex("k_ssd_pass", k_ssd_pass,
+                   dim3(kSsdHd * kSsdDs / 256, (unsigned)d.nh, (unsigned)B), 256, 0, s, a));
   FM_TRY(launched("k_ssd_pass"));
-  k_ssd_out<<<grid, kSsdThreads, SsdOutSmem::kBytes, s>>>(a);
+  FM_TRY(launch_ex("k_ssd_out", k_ssd_out, grid, kSsdThreads, SsdOutSmem::kBytes, s, a));
   return launched("k_ssd_out");
 }
 
@@ -1033,13 +1069,13 @@ static fm_status gate_impl(const int32_t *y, const float *z, long long M, const 
   if (M <= 0) return FM_OK;
   const int nb = d.di / 256;
   if (nb % 2 == 0 && M >= 2LL * sm_count())
-    k_gate_norm_quant<2><<<(unsigned)M, 32 * (nb / 2), 0, s>>>(
-      y, z, d.di, d.hd, exps + X.e_y, e_g_override ? e_g_override : exps + X.e_g, norm_w, rotate,
-      mode, static_amax, q, s_x, amax_row, gstat);
+    FM_TRY(launch_ex("k_gate_norm_quant", k_gate_norm_quant<2>, (unsigned)M, 32 * (nb / 2), 0, s, y,
+                     z, d.di, d.hd, exps + X.e_y, e_g_override ? e_g_override : exps + X.e_g,
+                     norm_w, rotate, mode, static_amax, q, s_x, amax_row, gstat));
   else
-    k_gate_norm_quant<1><<<(unsigned)M, 32 * nb, 0, s>>>(
-      y, z, d.di, d.hd, exps + X.e_y, e_g_override ? e_g_override : exps + X.e_g, norm_w, rotate,
-      mode, static_amax, q, s_x, amax_row, gstat);
+    FM_TRY(launch_ex("k_gate_norm_quant", k_gate_norm_quant<1>, (unsigned)M, 32 * nb, 0, s, y, z,
+                     d.di, d.hd, exps + X.e_y, e_g_override ? e_g_override : exps + X.e_g, norm_w,
+                     rotate, mode, static_amax, q, s_x, amax_row, gstat));
   return launched("k_gate_norm_quant");
 }
 
@@ -1349,12 +1385,13 @@ static fm_status launch_lq_conv(const float *u, long long ldu, int B, int T, int
                                 cudaStream_t s) {
   const dim3 grid((unsigned)((T + kLqConvTT - 1) / kLqConvTT), (unsigned)((cc + 255) / 256),
                   (unsigned)B);
-  k_lq_conv<<<grid, 256, 0, s>>>(u, ldu, T, cc, w, bias, conv_state, out);
+  FM_TRY(launch_ex("k_lq_conv", k_lq_conv, grid, 256, 0, s, u, ldu, T, cc, w, bias, conv_state,
+                   out));
   FM_TRY(launched("k_lq_conv"));
   if (conv_state) {
     const long long n = (long long)B * cc;
-    k_lq_conv_state_update<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(u, ldu, B, T, cc,
-                                                                        conv_state);
+    FM_TRY(launch_ex("k_lq_conv_state_update", k_lq_conv_state_update, (unsigned)((n + 255) / 256),
+                     256, 0, s, u, ldu, B, T, cc, conv_state));
     FM_TRY(launched("k_lq_conv_state_update"));
   }
   return FM_OK;
@@ -1368,9 +1405,9 @@ static fm_status launch_lq_scan_t(const Dims &d, const float *xo, const float *d
   constexpr int smem = (int)sizeof(LqScanSmem<CPW>);
   FM_CHECK_CUDA(cudaFuncSetAttribute(k_lq_scan<CPW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      smem));
-  k_lq_scan<CPW><<<dim3((unsigned)(d.hd / (4 * CPW)), (unsigned)d.nh, (unsigned)B), 128, smem,
-                   s>>>(xo, dt_raw, ld_dt, z, ld_z, T, d.nh, d.cc, d.di, dt_bias, a_log, D, state,
-                        out);
+  FM_TRY(launch_ex("k_lq_scan", k_lq_scan<CPW>,
+                   dim3((unsigned)(d.hd / (4 * CPW)), (unsigned)d.nh, (unsigned)B), 128, smem, s,
+                   xo, dt_raw, ld_dt, z, ld_z, T, d.nh, d.cc, d.di, dt_bias, a_log, D, state, out));
   return launched("k_lq_scan");
 }
 

@@ -362,6 +362,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();  // the prologue above touches only this CTA's shared memory and TMEM
 
   if (warp == 0) {
     if (lane == 0) {
@@ -449,6 +450,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
 // chunk) reads the exact int32 totals and runs the same gemm_store_chunk as
 // the unsplit kernels, so the outputs are bit-identical to theirs.
 __global__ void __launch_bounds__(128) k_gemm_splitk_epilogue(GemmEpilogue ep) {
+  pdl_wait();
   const long long nchunk = (ep.N + 31) / 32;
   const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= ep.M * nchunk) return;
@@ -659,6 +661,7 @@ __global__ void __launch_bounds__(64 + 32 * EW, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();  // the prologue above touches only this CTA's shared memory and TMEM
 
   if (warp == 0) {
     if (lane == 0) {

@@ -43,6 +43,7 @@ __global__ void __launch_bounds__(256) k_lq_conv(const float *__restrict__ u, lo
                                                  const float *__restrict__ bias,
                                                  const float *__restrict__ conv_state,
                                                  float *__restrict__ out) {
+  pdl_wait();
   const int c = blockIdx.y * 256 + threadIdx.x;
   const int t0 = blockIdx.x * kLqConvTT;
   const int b = blockIdx.z;
@@ -80,6 +81,7 @@ __global__ void __launch_bounds__(256) k_lq_conv(const float *__restrict__ u, lo
 __global__ void __launch_bounds__(256) k_lq_conv_state_update(const float *__restrict__ u,
                                                               long long ldu, int B, int T, int cc,
                                                               float *conv_state) {
+  pdl_wait();
   const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= (long long)B * cc) return;
   const int b = (int)(i / cc), c = (int)(i % cc);
@@ -139,6 +141,7 @@ __global__ void __launch_bounds__(128) k_lq_scan(
     const float *__restrict__ z, long long ld_z, int T, int nh, int cc, int di,
     const float *__restrict__ dt_bias, const float *__restrict__ a_log,
     const float *__restrict__ Dp, float *state, float *__restrict__ out) {
+  pdl_wait();
   static_assert(CPW == 1 || CPW == 2 || CPW == 4, "CPW");
   constexpr int SB = 32 / CPW;  // steps per reduction
   constexpr int hd = 64, ds = 128, CH = 4 * CPW;  // channels per CTA

@@ -91,6 +91,7 @@ __global__ void __launch_bounds__(1024) k_hadamard_quant(const float *__restrict
                                                          const float *static_amax,
                                                          int8_t *__restrict__ q, float *s_x,
                                                          float *amax_row) {
+  pdl_wait();
   __shared__ double s_blk[kMaxBlocks];
   __shared__ float s_red[kMaxBlocks];
   __shared__ float s_bc;
@@ -151,6 +152,7 @@ __global__ void __launch_bounds__(1024) k_gate_norm_quant(
     const int32_t *__restrict__ e_y, const int32_t *__restrict__ e_g_ptr,
     const float *__restrict__ norm_w, int rotate, int mode, const float *static_amax,
     int8_t *__restrict__ q, float *s_x, float *amax_row, unsigned long long *gstat) {
+  pdl_wait();
   __shared__ long long s_ss[kMaxBlocks];
   __shared__ float s_red[kMaxBlocks];
   __shared__ float s_bc;

@@ -32,7 +32,7 @@ EXPORTS = (
     "fm_set_state_spec", "fm_lq_conv1d", "fm_lq_scan", "fm_lq_workspace_bytes",
     "fm_lq_mixer_prefill", "fm_set_fault_injection", "fm_set_gemm_splitk",
     "fm_set_gemm_tile", "fm_set_xbc_exponents", "fm_conv1d_pot_tok", "fm_ssm_scan_pot_tok",
-    "fm_scan_workspace_bytes_tok",
+    "fm_scan_workspace_bytes_tok", "fm_set_pdl",
 )
 NOALLOC_SCRATCH_BYTES = 16 << 20  # FM_NOALLOC_SCRATCH_BYTES
 
@@ -118,6 +118,7 @@ def load():
         "fm_set_fault_injection": (I, [I, C.c_uint64]),
         "fm_set_gemm_splitk": (I, [I]),
         "fm_set_gemm_tile": (I, [I]),
+        "fm_set_pdl": (I, [I]),
         "fm_set_xbc_exponents": (I, [I]),
         "fm_conv1d_pot_tok": (I, [_P, I, I, sp, _P, _P, _P, _P, _P, _P, _P]),
         "fm_ssm_scan_pot_tok": (I, [_P, _P, I, I, sp, _P, _P, _P, _P, _P, _P, _P, _P, SZ, _P]),
@@ -184,6 +185,11 @@ def hadamard_quant(x, K, prenorm_w, rotate, mode, static_amax, q, s_x, amax_row=
 def prepare_linear(W, rotate, Wq, s_w, stream=None):
     N, K = W.shape
     _check(load().fm_prepare_linear(_p(W), N, K, rotate, _p(Wq), _p(s_w), _s(stream)))
+
+
+def set_pdl(enable: bool):
+    """Programmatic dependent launch of the hot kernels (off by default)."""
+    _check(load().fm_set_pdl(int(bool(enable))))
 
 
 def set_gemm_tile(bn: int):
