@@ -30,6 +30,13 @@ __device__ __forceinline__ void raise_error(unsigned int bits) { atomicOr(&g_err
 // has completed and its writes are visible.  Without that launch attribute
 // this returns at once.
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// ... and lets the next kernel in the stream be scheduled as soon as every
+// CTA of this one has started (all of them resident, so the dependents' CTAs
+// can only take resources this grid no longer needs); the dependents still
+// wait for this grid's completion before touching memory.
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
 
 // ---------------------------------------------------------------- integers
 __device__ __forceinline__ long long rshr64(long long a, int s) {

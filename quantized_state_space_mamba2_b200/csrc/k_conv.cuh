@@ -57,6 +57,7 @@ __global__ void __launch_bounds__(kConvQuads *TG) k_conv1d_pot(
     const int8_t *conv_state, int8_t *__restrict__ out, unsigned int *amax,
     int8_t *state_out, int32_t *e_tok = nullptr, int di = 0, int hd = 0, int ds = 0) {
   pdl_wait();
+  pdl_trigger();
   __shared__ int tab[8];
   pwl_table_init(tab);
   __syncthreads();
@@ -175,6 +176,7 @@ __global__ void __launch_bounds__(kConvQuads *TG) k_conv1d_pot(
 __global__ void k_conv_state_update(const int8_t *__restrict__ u, int B, int T, int cc,
                                     int8_t *__restrict__ conv_state) {
   pdl_wait();
+  pdl_trigger();
   const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= (long long)B * cc) return;
   const int c = (int)(i % cc);

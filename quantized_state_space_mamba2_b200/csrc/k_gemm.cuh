@@ -363,6 +363,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   pdl_wait();  // the prologue above touches only this CTA's shared memory and TMEM
+  pdl_trigger();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -451,6 +452,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
 // the unsplit kernels, so the outputs are bit-identical to theirs.
 __global__ void __launch_bounds__(128) k_gemm_splitk_epilogue(GemmEpilogue ep) {
   pdl_wait();
+  pdl_trigger();
   const long long nchunk = (ep.N + 31) / 32;
   const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= ep.M * nchunk) return;
@@ -662,6 +664,7 @@ __global__ void __launch_bounds__(64 + 32 * EW, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   pdl_wait();  // the prologue above touches only this CTA's shared memory and TMEM
+  pdl_trigger();
 
   if (warp == 0) {
     if (lane == 0) {

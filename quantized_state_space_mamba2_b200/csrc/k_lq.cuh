@@ -44,6 +44,7 @@ __global__ void __launch_bounds__(256) k_lq_conv(const float *__restrict__ u, lo
                                                  const float *__restrict__ conv_state,
                                                  float *__restrict__ out) {
   pdl_wait();
+  pdl_trigger();
   const int c = blockIdx.y * 256 + threadIdx.x;
   const int t0 = blockIdx.x * kLqConvTT;
   const int b = blockIdx.z;
@@ -82,6 +83,7 @@ __global__ void __launch_bounds__(256) k_lq_conv_state_update(const float *__res
                                                               long long ldu, int B, int T, int cc,
                                                               float *conv_state) {
   pdl_wait();
+  pdl_trigger();
   const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= (long long)B * cc) return;
   const int b = (int)(i / cc), c = (int)(i % cc);
@@ -142,6 +144,7 @@ __global__ void __launch_bounds__(128) k_lq_scan(
     const float *__restrict__ dt_bias, const float *__restrict__ a_log,
     const float *__restrict__ Dp, float *state, float *__restrict__ out) {
   pdl_wait();
+  pdl_trigger();
   static_assert(CPW == 1 || CPW == 2 || CPW == 4, "CPW");
   constexpr int SB = 32 / CPW;  // steps per reduction
   constexpr int hd = 64, ds = 128, CH = 4 * CPW;  // channels per CTA

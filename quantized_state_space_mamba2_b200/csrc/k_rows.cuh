@@ -92,6 +92,7 @@ __global__ void __launch_bounds__(1024) k_hadamard_quant(const float *__restrict
                                                          int8_t *__restrict__ q, float *s_x,
                                                          float *amax_row) {
   pdl_wait();
+  pdl_trigger();
   __shared__ double s_blk[kMaxBlocks];
   __shared__ float s_red[kMaxBlocks];
   __shared__ float s_bc;
@@ -153,6 +154,7 @@ __global__ void __launch_bounds__(1024) k_gate_norm_quant(
     const float *__restrict__ norm_w, int rotate, int mode, const float *static_amax,
     int8_t *__restrict__ q, float *s_x, float *amax_row, unsigned long long *gstat) {
   pdl_wait();
+  pdl_trigger();
   __shared__ long long s_ss[kMaxBlocks];
   __shared__ float s_red[kMaxBlocks];
   __shared__ float s_bc;

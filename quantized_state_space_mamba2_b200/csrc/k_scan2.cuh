@@ -69,6 +69,7 @@ __device__ __forceinline__ int osh_sD(int v) { return v >> 16; }
 // grid = (Tp / 32, nh, B), block = 256; hd == 64
 __global__ void __launch_bounds__(256) k_scan_prep(ScanPrepArgs a) {
   pdl_wait();
+  pdl_trigger();
   __shared__ int s_dtq[kPrepTT];
   __shared__ __align__(16) int8_t sx[kPrepTT][64];
   const int tid = threadIdx.x;
@@ -332,6 +333,7 @@ __device__ __forceinline__ void scan_chunk_steps(int (&hh)[NPT], unsigned (&hl)[
 template <int NPT, int PC, int TCH, bool S16 = false>
 __global__ void __launch_bounds__(PC *(128 / NPT) + 32) k_scan_seq(ScanSeqArgs a) {
   pdl_wait();
+  pdl_trigger();
   constexpr int LPP = 128 / NPT;
   constexpr int NW = PC * LPP / 32;
   constexpr int PPW = 32 / LPP;  // channels per warp
@@ -517,6 +519,7 @@ constexpr int kStepPPW = 8;  // channels per warp (hd / 8 warps)
 template <bool NARROW>
 __global__ void __launch_bounds__(256) k_scan_step(ScanArgs a) {
   pdl_wait();
+  pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int h = blockIdx.x, b = blockIdx.y;
   const int nh = a.nh, hd = a.hd, cc = a.cc, di = a.di;

@@ -128,6 +128,7 @@ struct SsdStateSmem {
 // grid (nch, nh, B), 128 threads
 __global__ void __launch_bounds__(kSsdThreads) k_ssd_state(SsdArgs a) {
   pdl_wait();
+  pdl_trigger();
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                             ~static_cast<uintptr_t>(1023));
@@ -246,6 +247,7 @@ __global__ void __launch_bounds__(kSsdThreads) k_ssd_state(SsdArgs a) {
 constexpr int kSsdPassGroup = 8;
 __global__ void __launch_bounds__(256) k_ssd_pass(SsdArgs a) {
   pdl_wait();
+  pdl_trigger();
   constexpr int kCells = kSsdHd * kSsdDs;
   const int e = blockIdx.x * 256 + threadIdx.x;  // cell p * 128 + n
   const int h = blockIdx.y, b = blockIdx.z;
@@ -304,6 +306,7 @@ static_assert(SsdOutSmem::kBytes <= 113 * 1024, "two k_ssd_out CTAs per SM");
 // grid (nch, nh, B), 128 threads
 __global__ void __launch_bounds__(kSsdThreads) k_ssd_out(SsdArgs a) {
   pdl_wait();
+  pdl_trigger();
   extern __shared__ uint8_t smem_raw[];
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                             ~static_cast<uintptr_t>(1023));
