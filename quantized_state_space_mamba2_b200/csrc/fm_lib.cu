@@ -446,13 +446,24 @@ static fm_status launch_conv(const int8_t *u, int B, int T, int cc, const int8_t
   const int di = d ? d->di : 0, hd = d ? d->hd : 0, ds = d ? d->ds : 0;
   if (T >= kConvTT) {
     const unsigned tiles = (unsigned)((T + kConvTokens - 1) / kConvTokens);
-    FM_TRY(launch_ex("k_conv1d_pot", k_conv1d_pot<kConvTT, kConvTG>, dim3(tiles, groups, B),
-                     kConvQuads * kConvTG, 0, s, u, T, cc, wq, bq, exps, conv_state, out, amax,
-                     nullptr, e_tok, di, hd, ds));
+    const dim3 grid(tiles, groups, B);
+    if (e_tok)
+      FM_TRY(launch_ex("k_conv1d_pot", k_conv1d_pot<kConvTT, kConvTG, true>, grid,
+                       kConvQuads * kConvTG, 0, s, u, T, cc, wq, bq, exps, conv_state, out, amax,
+                       nullptr, e_tok, di, hd, ds));
+    else
+      FM_TRY(launch_ex("k_conv1d_pot", k_conv1d_pot<kConvTT, kConvTG, false>, grid,
+                       kConvQuads * kConvTG, 0, s, u, T, cc, wq, bq, exps, conv_state, out, amax,
+                       nullptr, e_tok, di, hd, ds));
   } else {  // decode steps and short chunks: one token per thread
-    FM_TRY(launch_ex("k_conv1d_pot", k_conv1d_pot<1, 1>, dim3((unsigned)T, groups, B), kConvQuads,
-                     0, s, u, T, cc, wq, bq, exps, conv_state, out, amax,
-                     T == 1 ? conv_state : nullptr, e_tok, di, hd, ds));
+    const dim3 grid((unsigned)T, groups, B);
+    int8_t *state_out = T == 1 ? conv_state : nullptr;
+    if (e_tok)
+      FM_TRY(launch_ex("k_conv1d_pot", k_conv1d_pot<1, 1, true>, grid, kConvQuads, 0, s, u, T, cc,
+                       wq, bq, exps, conv_state, out, amax, state_out, e_tok, di, hd, ds));
+    else
+      FM_TRY(launch_ex("k_conv1d_pot", k_conv1d_pot<1, 1, false>, grid, kConvQuads, 0, s, u, T,
+                       cc, wq, bq, exps, conv_state, out, amax, state_out, e_tok, di, hd, ds));
   }
   FM_TRY(launched("k_conv1d_pot"));
   if (conv_state && T > 1) {  // a single step updates its state in the conv kernel
@@ -562,11 +573,11 @@ extern "C" fm_status fm_set_scan_tile(int npt, int pc, int tch) {
               pc, tch);
 }
 
-template <int NPT, int PC, int TCH, bool S16>
+template <int NPT, int PC, int TCH, bool S16, bool TOK>
 static fm_status launch_seq(const ScanSeqArgs &a, int B, cudaStream_t s) {
   using Sm = ScanSeqSmem<NPT, PC, TCH>;
   constexpr int smem = (int)sizeof(Sm);
-  auto kern = k_scan_seq<NPT, PC, TCH, S16>;
+  auto kern = k_scan_seq<NPT, PC, TCH, S16, TOK>;
   FM_CHECK_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
   dim3 grid(a.hd / PC, a.nh, B);
   FM_TRY(launch_ex("k_scan_seq", kern, grid, PC * (128 / NPT) + 32, smem, s, a));
@@ -620,8 +631,12 @@ static fm_status launch_scan_v2(const ScanArgs &a, int B, const ScanWs &w, cudaS
   p.e_tok = a.e_tok;
   p.osh = a.e_tok ? w.osh : nullptr;
   if (a.e_tok && !w.osh) return fail(FM_ERR_WORKSPACE, "scan: per-token shifts need workspace");
-  FM_TRY(launch_ex("k_scan_prep", k_scan_prep, dim3((unsigned)(Tp / kPrepTT), a.nh, B), 256, 0, s,
-                   p));
+  if (p.e_tok)
+    FM_TRY(launch_ex("k_scan_prep", k_scan_prep<true>, dim3((unsigned)(Tp / kPrepTT), a.nh, B),
+                     256, 0, s, p));
+  else
+    FM_TRY(launch_ex("k_scan_prep", k_scan_prep<false>, dim3((unsigned)(Tp / kPrepTT), a.nh, B),
+                     256, 0, s, p));
   FM_TRY(launched("k_scan_prep"));
   ScanSeqArgs q;
   q.dA = w.dA;
@@ -643,10 +658,14 @@ static fm_status launch_scan_v2(const ScanArgs &a, int B, const ScanWs &w, cudaS
   q.y = a.y;
   q.osh = p.osh;
   const ScanTile t = scan_tile();
-#define FM_SEQ(N, P, C)                                      \
-  if (t.npt == N && t.pc == P && t.tch == C)                 \
-    return state16() ? launch_seq<N, P, C, true>(q, B, s)    \
-                     : launch_seq<N, P, C, false>(q, B, s);
+#define FM_SEQ(N, P, C)                                                          \
+  if (t.npt == N && t.pc == P && t.tch == C) {                                   \
+    if (q.osh)                                                                   \
+      return state16() ? launch_seq<N, P, C, true, true>(q, B, s)                \
+                       : launch_seq<N, P, C, false, true>(q, B, s);              \
+    return state16() ? launch_seq<N, P, C, true, false>(q, B, s)                 \
+                     : launch_seq<N, P, C, false, false>(q, B, s);               \
+  }
   FM_SEQ(4, 4, 16)
   FM_SEQ(4, 2, 16)
   FM_SEQ(4, 8, 16)

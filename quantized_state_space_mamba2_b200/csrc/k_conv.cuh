@@ -43,14 +43,14 @@ __device__ __forceinline__ void conv_transpose4(uint32_t r0, uint32_t r1, uint32
 }
 
 // amax (nullable, [cc] u32): max |SiLU output| per channel (calibration).
-// e_tok (non-null: per-token output exponents, the x of each head, B and C
-// each a group): the codes of token t and group g are
+// TOK (per-token output exponents, the x of each head, B and C each a group;
+// e_tok non-null): the codes of token t and group g are
 // satb(rshr(s, e + 16), 8) with e = max(E(max_g |s|, 127) - 16, e_o - 16), E
 // the power-of-two exponent of the calibration; e_tok[t, g] (int32
 // [B*T, nh + 2]) receives e.  A head's 64 x channels are 16 consecutive
 // threads and B, C one warp each (the x | B | C boundaries are multiples of
 // 256 channels), so the group maximum is a shuffle reduction.
-template <int TT, int TG>
+template <int TT, int TG, bool TOK = false>
 __global__ void __launch_bounds__(kConvQuads *TG) k_conv1d_pot(
     const int8_t *__restrict__ u, int T, int cc, const int8_t *__restrict__ wq,
     const int32_t *__restrict__ bq, const int32_t *__restrict__ exps,
@@ -115,7 +115,7 @@ __global__ void __launch_bounds__(kConvQuads *TG) k_conv1d_pot(
     }
     if (k >= nt) break;
     uint32_t packed = 0;
-    if (e_tok) {  // per-token exponents (the warp is all x, all B or all C: uniform)
+    if constexpr (TOK) {  // per-token exponents (the warp is all x, all B or all C: uniform)
       int sv[kConvCPT];
       int m = 0;
 #pragma unroll

@@ -67,6 +67,7 @@ __device__ __forceinline__ int osh_sy(int v) { return (int)(int16_t)(v & 0xFFFF)
 __device__ __forceinline__ int osh_sD(int v) { return v >> 16; }
 
 // grid = (Tp / 32, nh, B), block = 256; hd == 64
+template <bool TOK>
 __global__ void __launch_bounds__(256) k_scan_prep(ScanPrepArgs a) {
   pdl_wait();
   pdl_trigger();
@@ -106,7 +107,7 @@ __global__ void __launch_bounds__(256) k_scan_prep(ScanPrepArgs a) {
     }
     s_dtq[tid] = dtq;
     a.dA[((long long)b * nh + h) * Tp + t0 + tid] = dA;
-    if (a.e_tok) {
+    if constexpr (TOK) {
       int sh = 0, o = 0;
       if (tid < nt) {
         const int32_t *et = a.e_tok + (rowbase + t0 + tid) * (nh + 2);
@@ -134,7 +135,7 @@ __global__ void __launch_bounds__(256) k_scan_prep(ScanPrepArgs a) {
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
       const long long x = sx[tb + k][p];
-      const int sh = a.e_tok ? s_sh[tb + k] : s_h;
+      const int sh = TOK ? s_sh[tb + k] : s_h;
       uv[k] = (int)satb64(rshr64((long long)s_dtq[tb + k] * x, sh - g), 24);
       dv[k] = (int)x;
     }
@@ -330,7 +331,7 @@ __device__ __forceinline__ void scan_chunk_steps(int (&hh)[NPT], unsigned (&hl)[
 // compute warp has released the chunk that used the slot before (empty
 // barrier, one arrival per compute warp), and signals it through the slot's
 // transaction-count barrier.  Compute warps never wait for each other.
-template <int NPT, int PC, int TCH, bool S16 = false>
+template <int NPT, int PC, int TCH, bool S16 = false, bool TOK = false>
 __global__ void __launch_bounds__(PC *(128 / NPT) + 32) k_scan_seq(ScanSeqArgs a) {
   pdl_wait();
   pdl_trigger();
@@ -379,8 +380,8 @@ __global__ void __launch_bounds__(PC *(128 / NPT) + 32) k_scan_seq(ScanSeqArgs a
         const int nt = min(TCH, T - t0);
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         mbar_arrive_expect_tx(&sm.full[sl], (uint32_t)(nt * 1024 + TCH * 4 * (1 + 2 * PC) +
-                                                       PC * 8 + (a.osh ? TCH * 4 : 0)));
-        if (a.osh) bulk_g2s(&s.osh[0], a.osh + headrow * Tp + t0, TCH * 4, &sm.full[sl]);
+                                                       PC * 8 + (TOK ? TCH * 4 : 0)));
+        if constexpr (TOK) bulk_g2s(&s.osh[0], a.osh + headrow * Tp + t0, TCH * 4, &sm.full[sl]);
         bulk_g2s(&s.bound[0], a.bound + ((headrow * (Tp / 16) + c) * hd + p0), PC * 8,
                  &sm.full[sl]);
         bulk_g2s(&s.bc[0][0], a.bc + (rowbase + t0) * 256, (uint32_t)(nt * 1024), &sm.full[sl]);
@@ -452,8 +453,8 @@ __global__ void __launch_bounds__(PC *(128 / NPT) + 32) k_scan_seq(ScanSeqArgs a
       if (lane32 < nt) {
         const int2 v = wsum[lane32];
         const long long sum = S16 ? (long long)v.x : (long long)v.x * 65536 + v.y;
-        const int sy = a.osh ? osh_sy(s.osh[lane32]) : s_y;
-        const int sD = a.osh ? osh_sD(s.osh[lane32]) : s_D;
+        const int sy = TOK ? osh_sy(s.osh[lane32]) : s_y;
+        const int sD = TOK ? osh_sD(s.osh[lane32]) : s_D;
         a.y[(rowbase + t0 + lane32) * di + (long long)h * hd + p0 + pp] =
             (int)satb64(rshr64(sum, sy) + rshr64(Dq * s.xs[pp][lane32], sD), 32);
       }
@@ -484,8 +485,8 @@ __global__ void __launch_bounds__(PC *(128 / NPT) + 32) k_scan_seq(ScanSeqArgs a
       const int tt = row / PPW, q = warp * PPW + row % PPW;
       if (half == 0 && tt < nt) {
         const long long sum = S16 ? (long long)shi : (long long)shi * 65536 + slo;
-        const int sy = a.osh ? osh_sy(s.osh[tt]) : s_y;
-        const int sD = a.osh ? osh_sD(s.osh[tt]) : s_D;
+        const int sy = TOK ? osh_sy(s.osh[tt]) : s_y;
+        const int sD = TOK ? osh_sD(s.osh[tt]) : s_D;
         a.y[(rowbase + t0 + tt) * di + (long long)h * hd + p0 + q] =
             (int)satb64(rshr64(sum, sy) + rshr64(Dq * s.xs[q][tt], sD), 32);
       }
