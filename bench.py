@@ -92,6 +92,8 @@ def parse(argv=None):
                          "16,7 the narrow state with the guard-bit increment")
     ap.add_argument("--gemm-tile", type=int, default=0, choices=[0, 128, 256],
                     help="tile width of the persistent GEMM (0: chosen by the grid)")
+    ap.add_argument("--lq-cpw", type=int, default=0, choices=[0, 1, 2, 4],
+                    help="channels per warp of the LQ scan (0: chosen by the grid)")
     ap.add_argument("--pdl", action="store_true",
                     help="programmatic dependent launch of the library's kernels")
     ap.add_argument("--eager", action="store_true",
@@ -936,6 +938,7 @@ def apply_modes(args, lib):
     lib.set_state_spec(*[int(v) for v in args.state_spec.split(",")])
     lib.set_gemm_tile(args.gemm_tile)
     lib.set_pdl(getattr(args, "pdl", False))
+    lib.set_lq_scan_cpw(getattr(args, "lq_cpw", 0))
     lib.set_xbc_exponents(args.xbc_exponents)
 
 

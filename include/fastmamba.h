@@ -470,6 +470,11 @@ fm_status fm_lq_scan(const float *xo, const float *dt_raw, int64_t ld_dt, const 
                      const float *a_log, const float *D, float *state, float *out,
                      fm_stream stream);
 
+/* Tuning: channels per warp of the fp32 scan (0: chosen by the grid; 1, 2 or
+ * 4).  Results differ only in the order of the warp's fp32 C.h sum.
+ * FM_ERR_INVALID_ARG for other values. */
+fm_status fm_set_lq_scan_cpw(int cpw);
+
 /* One LQ layer: fm_hadamard_quant (with L->prenorm_w) -> in_proj GEMM (fp32
  * output) -> fm_lq_conv1d -> fm_lq_scan with the gate -> gated RMSNorm
  * (eps 1e-5, L->norm_w) + rotation + int8 (fm_hadamard_quant with norm_w as

@@ -1430,14 +1430,34 @@ static fm_status launch_lq_scan_t(const Dims &d, const float *xo, const float *d
   return launched("k_lq_scan");
 }
 
+// Channels per warp of the LQ scan, process-wide: 0 (default) chooses by the
+// grid, 1, 2 or 4 forces it (tuning; the same results either way up to the
+// warp reduction's order).
+static std::atomic<int> g_lq_cpw{0};
+
+extern "C" fm_status fm_set_lq_scan_cpw(int cpw) {
+  if (cpw != 0 && cpw != 1 && cpw != 2 && cpw != 4)
+    return fail(FM_ERR_INVALID_ARG, "fm_set_lq_scan_cpw: %d is not 0, 1, 2 or 4", cpw);
+  g_lq_cpw.store(cpw, std::memory_order_relaxed);
+  return FM_OK;
+}
+
 static fm_status launch_lq_scan(const Dims &d, const float *xo, const float *dt_raw,
                                 long long ld_dt, const float *z, long long ld_z, int B, int T,
                                 const float *dt_bias, const float *a_log, const float *D,
                                 float *state, float *out, cudaStream_t s) {
-  // one channel per warp while that leaves fewer than ~8 warps per SM to
-  // share the staged rows, else 2 (more state cells per staged row)
-  const long long warps1 = (long long)B * d.nh * d.hd;
-  if (warps1 >= 16LL * sm_count())
+  // Each warp re-reads the staged B and C rows of every step for its CPW
+  // channels, so wider warps cut the shared-memory traffic per state cell:
+  // by default the widest CPW that still gives every SM a CTA.
+  int cpw = g_lq_cpw.load(std::memory_order_relaxed);
+  if (cpw == 0) {
+    const long long ctas4 = (long long)B * d.nh * (d.hd / 16), sms = sm_count();
+    cpw = ctas4 >= sms ? 4 : (2 * ctas4 >= sms ? 2 : 1);
+  }
+  if (cpw == 4)
+    return launch_lq_scan_t<4>(d, xo, dt_raw, ld_dt, z, ld_z, B, T, dt_bias, a_log, D, state,
+                               out, s);
+  if (cpw == 2)
     return launch_lq_scan_t<2>(d, xo, dt_raw, ld_dt, z, ld_z, B, T, dt_bias, a_log, D, state,
                                out, s);
   return launch_lq_scan_t<1>(d, xo, dt_raw, ld_dt, z, ld_z, B, T, dt_bias, a_log, D, state, out,

@@ -32,7 +32,7 @@ EXPORTS = (
     "fm_set_state_spec", "fm_lq_conv1d", "fm_lq_scan", "fm_lq_workspace_bytes",
     "fm_lq_mixer_prefill", "fm_set_fault_injection", "fm_set_gemm_splitk",
     "fm_set_gemm_tile", "fm_set_xbc_exponents", "fm_conv1d_pot_tok", "fm_ssm_scan_pot_tok",
-    "fm_scan_workspace_bytes_tok", "fm_set_pdl",
+    "fm_scan_workspace_bytes_tok", "fm_set_pdl", "fm_set_lq_scan_cpw",
 )
 NOALLOC_SCRATCH_BYTES = 16 << 20  # FM_NOALLOC_SCRATCH_BYTES
 
@@ -119,6 +119,7 @@ def load():
         "fm_set_gemm_splitk": (I, [I]),
         "fm_set_gemm_tile": (I, [I]),
         "fm_set_pdl": (I, [I]),
+        "fm_set_lq_scan_cpw": (I, [I]),
         "fm_set_xbc_exponents": (I, [I]),
         "fm_conv1d_pot_tok": (I, [_P, I, I, sp, _P, _P, _P, _P, _P, _P, _P]),
         "fm_ssm_scan_pot_tok": (I, [_P, _P, I, I, sp, _P, _P, _P, _P, _P, _P, _P, _P, SZ, _P]),
@@ -405,6 +406,11 @@ def lq_scan(xo, dt_raw, z, B, T, shape, dt_bias, a_log, D, state, out, stream=No
     pz, ldz = _row_view(z, shape.d_inner) if z is not None else (None, 0)
     _check(load().fm_lq_scan(_p(xo), pdt, lddt, pz, ldz, B, T, C.byref(sh), _p(dt_bias),
                              _p(a_log), _p(D), _p(state), _p(out), _s(stream)))
+
+
+def set_lq_scan_cpw(cpw: int):
+    """Channels per warp of the LQ scan: 0 (by the grid), 1, 2 or 4."""
+    _check(load().fm_set_lq_scan_cpw(cpw))
 
 
 def lq_workspace_bytes(shape, B, T) -> int:
