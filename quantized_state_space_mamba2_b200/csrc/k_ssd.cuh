@@ -88,15 +88,31 @@ __device__ __forceinline__ float pow2_q16(long long e) {
 
 // dt_q and w of token t of the chunk (0 past the end); W = inclusive prefix
 // sum of w over the chunk's 128 tokens (one per thread), into sW[t].
-__device__ __forceinline__ int ssd_chunk_decay(const SsdArgs &a, int b, int h, int t0, int nt,
-                                               long long *sW, long long *wtot) {
+// The per-thread inputs of ssd_chunk_decay, loaded at the kernel's start so
+// that their latency overlaps the tile loads: this thread's token's dt_raw
+// (0 past the end), dt_bias[h] and A_q[h].
+struct SsdDecayIn {
+  float dt_raw, bias;
+  int A_q;
+};
+__device__ __forceinline__ SsdDecayIn ssd_decay_in(const SsdArgs &a, int b, int h, int t0,
+                                                  int nt) {
+  const int t = threadIdx.x;
+  SsdDecayIn in;
+  in.dt_raw = t < nt ? a.dt_raw[((long long)b * a.T + t0 + t) * a.nh + h] : 0.0f;
+  in.bias = a.dt_bias[h];
+  in.A_q = a.A_q[h];
+  return in;
+}
+__device__ __forceinline__ int ssd_chunk_decay(const SsdDecayIn &in, int nt, long long *sW,
+                                               long long *wtot) {
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   int dtq = 0;
   long long w = 0;
   if (t < nt) {
-    const float xf = __fadd_rn(a.dt_raw[((long long)b * a.T + t0 + t) * a.nh + h], a.dt_bias[h]);
+    const float xf = __fadd_rn(in.dt_raw, in.bias);
     dtq = softplus_pwl(to_q16(xf));
-    w = -rshr64((long long)dtq * a.A_q[h], 12);
+    w = -rshr64((long long)dtq * in.A_q, 12);
   }
   long long v = w;
 #pragma unroll
@@ -148,6 +164,7 @@ __global__ void __launch_bounds__(kSsdThreads) k_ssd_state(SsdArgs a) {
   const long long row0 = (long long)b * a.T + t0;
   const long long bh = (long long)b * a.nh + h;
 
+  const SsdDecayIn din = ssd_decay_in(a, b, h, t0, nt);
   if (t == 0) {
     mbar_init(bar, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -169,7 +186,7 @@ __global__ void __launch_bounds__(kSsdThreads) k_ssd_state(SsdArgs a) {
       v = *reinterpret_cast<const uint4 *>(a.xbc + (row0 + s) * a.cc + (long long)h * kSsdHd + k * 16);
     *reinterpret_cast<uint4 *>(Xt + s * 64 + k * 16) = v;
   }
-  const int dtq = ssd_chunk_decay(a, b, h, t0, nt, sW, wtot);
+  const int dtq = ssd_chunk_decay(din, nt, sW, wtot);
   __syncthreads();
   const long long Wend = sW[kSsdQ - 1];
   const float dtf = __fmul_rn(__int2float_rn(dtq), 1.0f / 65536.0f);
@@ -326,6 +343,11 @@ __global__ void __launch_bounds__(kSsdThreads) k_ssd_out(SsdArgs a) {
   const long long row0 = (long long)b * a.T + t0;
   const long long bh = (long long)b * a.nh + h;
 
+  // every scalar input, loaded up front (their latency overlaps the tile loads)
+  const SsdDecayIn din = ssd_decay_in(a, b, h, t0, nt);
+  const int s_y = *a.e_C + a.e_x[h] + *a.e_B - a.e_y[h];
+  const int s_D = a.e_y[h] - a.e_D[h] - a.e_x[h];
+  const long long Dq = a.D_q[h];
   if (t == 0) {
     mbar_init(&bar[0], 1);
     mbar_init(&bar[1], 1);
@@ -353,7 +375,7 @@ __global__ void __launch_bounds__(kSsdThreads) k_ssd_out(SsdArgs a) {
     *reinterpret_cast<uint4 *>(Xt + s * 64 + k * 16) = v;
   }
   // (its CTA barrier also makes the tiles above visible to every thread)
-  const int dtq = ssd_chunk_decay(a, b, h, t0, nt, sW, wtot);
+  const int dtq = ssd_chunk_decay(din, nt, sW, wtot);
   sdt[t] = __fmul_rn(__int2float_rn(dtq), 1.0f / 65536.0f);
   {  // row t of Ca: bf16(2^W[t] Cq[t][n]), Cq read back from the int8 tile
     const float a0 = pow2_q16(sW[t]);
@@ -474,9 +496,6 @@ __global__ void __launch_bounds__(kSsdThreads) k_ssd_out(SsdArgs a) {
   int32_t *sY = reinterpret_cast<int32_t *>(sm + L::kC8);
   static_assert(kSsdQ * kYStride * 4 <= L::kX - L::kC8, "the y tile fits over M and Ca");
   {  // y codes of token t: rint(Y 2^(e_C+e_x+e_B-e_y)) + rshr(D_q x, s_D), saturated
-    const int s_y = *a.e_C + a.e_x[h] + *a.e_B - a.e_y[h];
-    const int s_D = a.e_y[h] - a.e_D[h] - a.e_x[h];
-    const long long Dq = a.D_q[h];
     const float scale = pow2f(s_y);
 #pragma unroll 1
     for (int c0 = 0; c0 < kSsdHd; c0 += 32) {
