@@ -63,13 +63,28 @@ CPU_SAMPLE_MIN_S = 10.0
 CPU_ALLCORE_TOKENS = 512
 
 
-# DRAM bytes per launch of a roofline kernel, from the ncu summaries in
-# profiles/ (named there); None when no capture of the current kernel exists.
-DRAM_TRAFFIC = {}
+# DRAM bytes (read + write) per launch of a roofline kernel, from one-pass ncu
+# captures of the current kernels (profiles/dram_traffic_roofline_kernels.md);
+# None where no capture of the kernel in that configuration exists.
+DRAM_TRAFFIC = {
+    # 130M stack, B 1, T 2048, static exponents, the int32 state: k_scan_prep
+    # 3,884,544 + 256 and k_scan_seq 29,099,264 + 0
+    ("fm_ssm_scan_pot (k_scan_prep + k_scan_seq)", "stack130m_24l_b1_t2048", "31,0", "static"):
+        32984064,
+    # 2.7B decode, B 64: k_scan_step 168,167,424 + 108,474,880
+    ("fm_ssm_scan_pot, T = 1 (k_scan_step)", "decode2p7b_64l_b64", "31,0", "static"): 276642304,
+    # in_proj GEMM at M = 32768: 253,903,616 + 1,340,978,944
+    ("fm_w8a8_gemm (k_gemm_i8_persist, tcgen05 kind::i8)", "gemm2p7b_inproj", 32768): 1594882560,
+}
 
 
 def dram_traffic(kernel: str, args):
-    return DRAM_TRAFFIC.get((kernel, args.workload))
+    if args.workload == "gemm2p7b_inproj":
+        return DRAM_TRAFFIC.get((kernel, args.workload, args.gemm_m))
+    if getattr(args, "lq", False) or getattr(args, "scan_mode", "seq") != "seq":
+        return None
+    return DRAM_TRAFFIC.get((kernel, args.workload, args.state_spec,
+                             getattr(args, "xbc_exponents", "static")))
 
 
 def parse(argv=None):
