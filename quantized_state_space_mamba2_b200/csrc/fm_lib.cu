@@ -314,7 +314,7 @@ static bool gemm_would_split(long long M, long long N, long long K) {
 template <int BN, int STAGES>
 static fm_status launch_gemm_t(const CUtensorMap &ta, const CUtensorMap &tb, long long M,
                                long long N, long long K, GemmEpilogue ep, int32_t *split_ws,
-                               cudaStream_t s) {
+                               cudaStream_t s, int a_rows) {
   constexpr int smem = gemm_smem_bytes(BN, STAGES);
   const int nkb = (int)(K / kGemmBK);
   int kbs = nkb, splits = 1;
@@ -328,7 +328,8 @@ static fm_status launch_gemm_t(const CUtensorMap &ta, const CUtensorMap &tb, lon
   }
   dim3 grid((unsigned)((N + BN - 1) / BN), (unsigned)((M + kGemmBM - 1) / kGemmBM),
             (unsigned)splits);
-  FM_TRY(launch_ex("k_gemm_i8_tc", kern, grid, kGemmThreads, smem, s, ta, tb, nkb, kbs, ep));
+  FM_TRY(launch_ex("k_gemm_i8_tc", kern, grid, kGemmThreads, smem, s, ta, tb, nkb, kbs, ep,
+                   a_rows));
   FM_TRY(launched("k_gemm_i8_tc"));
   if (splits > 1) {
     const long long n = M * ((N + 31) / 32);
@@ -410,12 +411,15 @@ static fm_status launch_gemm(const int8_t *A, long long M, const int8_t *W, long
     FM_TRY(make_tmap(&tb, W, N, K, 128));
     return launch_gemm_persist<128, 5, 8>(ta, tb, M, N, K, sms, ep, s);
   }
+  // a decode batch (M <= 64): load only the 64 real rows of A per stage
+  const int a_rows = M <= 64 ? 64 : kGemmBM;
+  if (a_rows != kGemmBM) FM_TRY(make_tmap(&ta, A, M, K, a_rows));
   if (mt * ((N + 63) / 64) < sms) {  // fewer 64-wide tiles than SMs: halve the tile width
     FM_TRY(make_tmap(&tb, W, N, K, 32));
-    return launch_gemm_t<32, 6>(ta, tb, M, N, K, ep, split_ws, s);
+    return launch_gemm_t<32, 6>(ta, tb, M, N, K, ep, split_ws, s, a_rows);
   }
   FM_TRY(make_tmap(&tb, W, N, K, 64));
-  return launch_gemm_t<64, 4>(ta, tb, M, N, K, ep, split_ws, s);
+  return launch_gemm_t<64, 4>(ta, tb, M, N, K, ep, split_ws, s, a_rows);
 }
 
 static fm_status launch_hadamard_quant(const float *x, long long M, int K, const float *prenorm_w,

@@ -313,10 +313,15 @@ __device__ __forceinline__ void gemm_store_chunk(const GemmEpilogue &ep, long lo
 }
 
 // ------------------------------------------------------------ the kernel
+// a_rows: rows of the A box the producer loads per stage (128, or 64 when M
+// <= 64: a decode batch).  The MMA always reads a 128-row A tile; with a
+// 64-row box the tile's rows 64..127 hold stale shared memory, which only
+// feeds accumulator rows >= M that the epilogue never stores, and the L2 ->
+// shared traffic of A halves.
 template <int BN, int STAGES, bool SPLIT = false>
 __global__ void __launch_bounds__(kGemmThreads, 2)
     k_gemm_i8_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                 int num_k_blocks, int kb_per_split, GemmEpilogue ep) {
+                 int num_k_blocks, int kb_per_split, GemmEpilogue ep, int a_rows) {
   static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN");
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -373,7 +378,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
         const int s = kb % STAGES;
         const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
         if (!mbar_wait(&empty_bar[s], ph ^ 1u)) break;
-        mbar_arrive_expect_tx(&full_bar[s], (uint32_t)((kGemmBM + BN) * kGemmBK));
+        mbar_arrive_expect_tx(&full_bar[s], (uint32_t)((a_rows + BN) * kGemmBK));
         tma_load_2d(sA + s * kGemmBM * kGemmBK, &tmA, (kb0 + kb) * kGemmBK, m0, &full_bar[s]);
         tma_load_2d(sB + s * BN * kGemmBK, &tmB, (kb0 + kb) * kGemmBK, n0, &full_bar[s]);
         ++issued;
