@@ -311,16 +311,17 @@ static bool gemm_would_split(long long M, long long N, long long K) {
   return gemm_splits(M, N, K, BN, sms, &kbs) > 1;
 }
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, int AR = kGemmBM>
 static fm_status launch_gemm_t(const CUtensorMap &ta, const CUtensorMap &tb, long long M,
                                long long N, long long K, GemmEpilogue ep, int32_t *split_ws,
-                               cudaStream_t s, int a_rows) {
-  constexpr int smem = gemm_smem_bytes(BN, STAGES);
+                               cudaStream_t s) {
+  constexpr int smem = gemm_smem_bytes(BN, STAGES, AR);
+  static_assert(smem <= 227 * 1024, "shared memory per CTA");
   const int nkb = (int)(K / kGemmBK);
   int kbs = nkb, splits = 1;
   if (split_ws && g_gemm_splitk.load(std::memory_order_relaxed))
     splits = gemm_splits(M, N, K, BN, sm_count(), &kbs);
-  auto kern = splits > 1 ? k_gemm_i8_tc<BN, STAGES, true> : k_gemm_i8_tc<BN, STAGES, false>;
+  auto kern = splits > 1 ? k_gemm_i8_tc<BN, STAGES, true, AR> : k_gemm_i8_tc<BN, STAGES, false, AR>;
   FM_CHECK_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
   if (splits > 1) {
     ep.split_acc = split_ws;
@@ -328,8 +329,7 @@ static fm_status launch_gemm_t(const CUtensorMap &ta, const CUtensorMap &tb, lon
   }
   dim3 grid((unsigned)((N + BN - 1) / BN), (unsigned)((M + kGemmBM - 1) / kGemmBM),
             (unsigned)splits);
-  FM_TRY(launch_ex("k_gemm_i8_tc", kern, grid, kGemmThreads, smem, s, ta, tb, nkb, kbs, ep,
-                   a_rows));
+  FM_TRY(launch_ex("k_gemm_i8_tc", kern, grid, kGemmThreads, smem, s, ta, tb, nkb, kbs, ep));
   FM_TRY(launched("k_gemm_i8_tc"));
   if (splits > 1) {
     const long long n = M * ((N + 31) / 32);
@@ -411,15 +411,18 @@ static fm_status launch_gemm(const int8_t *A, long long M, const int8_t *W, long
     FM_TRY(make_tmap(&tb, W, N, K, 128));
     return launch_gemm_persist<128, 5, 8>(ta, tb, M, N, K, sms, ep, s);
   }
-  // a decode batch (M <= 64): load only the 64 real rows of A per stage
-  const int a_rows = M <= 64 ? 64 : kGemmBM;
-  if (a_rows != kGemmBM) FM_TRY(make_tmap(&ta, A, M, K, a_rows));
-  if (mt * ((N + 63) / 64) < sms) {  // fewer 64-wide tiles than SMs: halve the tile width
-    FM_TRY(make_tmap(&tb, W, N, K, 32));
-    return launch_gemm_t<32, 6>(ta, tb, M, N, K, ep, split_ws, s, a_rows);
+  const bool narrow = mt * ((N + 63) / 64) < sms;  // fewer 64-wide tiles than SMs: 32 wide
+  FM_TRY(make_tmap(&tb, W, N, K, narrow ? 32 : 64));
+  if (M <= 64) {
+    // a decode batch: only the 64 real rows of A per stage, so the weight
+    // stream gets a deeper ring (64 wide: 6 x 16 KB, two CTAs per SM; 32 wide,
+    // fewer CTAs than SMs: 16 x 12 KB, one per SM)
+    FM_TRY(make_tmap(&ta, A, M, K, 64));
+    if (narrow) return launch_gemm_t<32, 16, 64>(ta, tb, M, N, K, ep, split_ws, s);
+    return launch_gemm_t<64, 6, 64>(ta, tb, M, N, K, ep, split_ws, s);
   }
-  FM_TRY(make_tmap(&tb, W, N, K, 64));
-  return launch_gemm_t<64, 4>(ta, tb, M, N, K, ep, split_ws, s, a_rows);
+  if (narrow) return launch_gemm_t<32, 6>(ta, tb, M, N, K, ep, split_ws, s);
+  return launch_gemm_t<64, 4>(ta, tb, M, N, K, ep, split_ws, s);
 }
 
 static fm_status launch_hadamard_quant(const float *x, long long M, int K, const float *prenorm_w,
@@ -1080,7 +1083,7 @@ static fm_status launch_ssd(const Dims &d, const int8_t *xbc, const float *dt_ra
   FM_TRY(launch_ex("k_ssd_pass", k_ssd_pass,
                    dim3(kSsdHd * kSsdDs / 256, (unsigned)d.nh, (unsigned)B), 256, 0, s, a));
   FM_TRY(launched("k_ssd_pass"));
-  FM_TRY(launch_ex("k_ssd_out", k_ssd_out, grid, kSsdThreads, SsdOutSmem::kBytes, s, a));
+  FM_TRY(launch_ex("k_ssd_out", k_ssd_out, grid, kSsdOutThreads, SsdOutSmem::kBytes, s, a));
   return launched("k_ssd_out");
 }
 
@@ -1451,12 +1454,15 @@ static fm_status launch_lq_scan(const Dims &d, const float *xo, const float *dt_
                                 const float *dt_bias, const float *a_log, const float *D,
                                 float *state, float *out, cudaStream_t s) {
   // Each warp re-reads the staged B and C rows of every step for its CPW
-  // channels, so wider warps cut the shared-memory traffic per state cell:
-  // by default the widest CPW that still gives every SM a CTA.
+  // channels, so wider warps cut the shared-memory traffic per state cell,
+  // but the recurrence's latency wants two CTAs on every SM: by default the
+  // widest CPW that still gives each SM two (measured on the 24-layer 130M
+  // stack, B = 1, T = 2048: 1 / 2 / 4 channels per warp = 7.64 / 8.12 /
+  // 9.42 ms per step; 64-layer 2.7B, B = 2, T = 4096: 4 beats 2 by 8 %).
   int cpw = g_lq_cpw.load(std::memory_order_relaxed);
   if (cpw == 0) {
-    const long long ctas4 = (long long)B * d.nh * (d.hd / 16), sms = sm_count();
-    cpw = ctas4 >= sms ? 4 : (2 * ctas4 >= sms ? 2 : 1);
+    const long long ctas4 = (long long)B * d.nh * (d.hd / 16), slots = 2LL * sm_count();
+    cpw = ctas4 >= slots ? 4 : (2 * ctas4 >= slots ? 2 : 1);
   }
   if (cpw == 4)
     return launch_lq_scan_t<4>(d, xo, dt_raw, ld_dt, z, ld_z, B, T, dt_bias, a_log, D, state,

@@ -210,8 +210,9 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-__host__ __device__ constexpr int gemm_smem_bytes(int BN, int stages) {
-  return stages * (kGemmBM + BN) * kGemmBK + 1024 /*align slack*/ + 256 /*barriers*/ +
+// ar: rows of A staged per stage (kGemmBM, or 64 for a decode batch)
+__host__ __device__ constexpr int gemm_smem_bytes(int BN, int stages, int ar = kGemmBM) {
+  return stages * (ar + BN) * kGemmBK + 1024 /*align slack*/ + 256 /*barriers*/ +
          2 * BN * 4 /*staged column scales*/;
 }
 
@@ -313,21 +314,25 @@ __device__ __forceinline__ void gemm_store_chunk(const GemmEpilogue &ep, long lo
 }
 
 // ------------------------------------------------------------ the kernel
-// a_rows: rows of the A box the producer loads per stage (128, or 64 when M
-// <= 64: a decode batch).  The MMA always reads a 128-row A tile; with a
-// 64-row box the tile's rows 64..127 hold stale shared memory, which only
-// feeds accumulator rows >= M that the epilogue never stores, and the L2 ->
-// shared traffic of A halves.
-template <int BN, int STAGES, bool SPLIT = false>
+// AR: rows of A staged per stage (128, or 64 when M <= 64: a decode batch,
+// whose A box then has 64 rows).  The MMA always reads a 128-row A tile; with
+// AR = 64 the tile's rows 64..127 are the next 8 KB of shared memory (the next
+// stage's A rows, or for the last stage the start of the B ring: always inside
+// the allocation), which only feed accumulator rows >= M that the epilogue
+// never stores.  The L2 -> shared traffic of A and its ring space halve, so
+// the ring can be deeper.
+template <int BN, int STAGES, bool SPLIT = false, int AR = kGemmBM>
 __global__ void __launch_bounds__(kGemmThreads, 2)
     k_gemm_i8_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                 int num_k_blocks, int kb_per_split, GemmEpilogue ep, int a_rows) {
+                 int num_k_blocks, int kb_per_split, GemmEpilogue ep) {
   static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN");
+  static_assert(AR == kGemmBM || (AR == 64 && STAGES * BN >= 64),
+                "a 64-row A stage reads 64 more rows, inside the ring");
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
   uint8_t *sA = smem;
-  uint8_t *sB = smem + STAGES * kGemmBM * kGemmBK;
+  uint8_t *sB = smem + STAGES * AR * kGemmBK;
   uint64_t *full_bar = reinterpret_cast<uint64_t *>(sB + STAGES * BN * kGemmBK);
   uint64_t *empty_bar = full_bar + STAGES;
   uint64_t *accum_bar = empty_bar + STAGES;
@@ -378,8 +383,8 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
         const int s = kb % STAGES;
         const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
         if (!mbar_wait(&empty_bar[s], ph ^ 1u)) break;
-        mbar_arrive_expect_tx(&full_bar[s], (uint32_t)((a_rows + BN) * kGemmBK));
-        tma_load_2d(sA + s * kGemmBM * kGemmBK, &tmA, (kb0 + kb) * kGemmBK, m0, &full_bar[s]);
+        mbar_arrive_expect_tx(&full_bar[s], (uint32_t)((AR + BN) * kGemmBK));
+        tma_load_2d(sA + s * AR * kGemmBK, &tmA, (kb0 + kb) * kGemmBK, m0, &full_bar[s]);
         tma_load_2d(sB + s * BN * kGemmBK, &tmB, (kb0 + kb) * kGemmBK, n0, &full_bar[s]);
         ++issued;
       }
@@ -396,7 +401,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
         const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
         if (!mbar_wait(&full_bar[s], ph)) break;
         tc_fence_after();
-        const uint64_t ad = sw128_desc(smem_u32(sA + s * kGemmBM * kGemmBK));
+        const uint64_t ad = sw128_desc(smem_u32(sA + s * AR * kGemmBK));
         const uint64_t bd = sw128_desc(smem_u32(sB + s * BN * kGemmBK));
 #pragma unroll
         for (int k = 0; k < kGemmBK / 32; ++k) {

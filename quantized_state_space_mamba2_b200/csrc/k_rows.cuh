@@ -21,6 +21,16 @@ namespace fm {
 
 constexpr int kMaxBlocks = 32;  // K <= 8192
 
+// 8 consecutive floats from a 32-byte-aligned address (two 16-byte loads;
+// the entry points require 16-byte-aligned tensors and every caller's offset
+// is a multiple of 8 elements)
+__device__ __forceinline__ void load8(const float *p, float (&v)[8]) {
+  const float4 a = *reinterpret_cast<const float4 *>(p);
+  const float4 b = *reinterpret_cast<const float4 *>(p + 4);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
 // Row max over all warps of the CTA (every thread returns the result).
 __device__ __forceinline__ float cta_max(float v, float *s_red, float *s_out) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
@@ -135,7 +145,8 @@ __global__ void __launch_bounds__(1024) k_hadamard_quant(const float *__restrict
     const float rstd = s_rstd;
 #pragma unroll
     for (int b = 0; b < BPW; ++b) {
-      const float *w = prenorm_w + (warp * BPW + b) * 256 + lane * 8;
+      float w[8];
+      load8(prenorm_w + (warp * BPW + b) * 256 + lane * 8, w);
 #pragma unroll
       for (int i = 0; i < 8; ++i) v[b][i] = __fmul_rn(__fmul_rn(v[b][i], rstd), w[i]);
     }
@@ -228,7 +239,8 @@ __global__ void __launch_bounds__(1024) k_gate_norm_quant(
   float v[BPW][8];
 #pragma unroll
   for (int b = 0; b < BPW; ++b) {
-    const float *w = norm_w + (warp * BPW + b) * 256 + lane * 8;
+    float w[8];
+    load8(norm_w + (warp * BPW + b) * 256 + lane * 8, w);
 #pragma unroll
     for (int i = 0; i < 8; ++i)
       v[b][i] = __fmul_rn(__fmul_rn(__fmul_rn(small_i2f(gq[b][i]), scale), rstd), w[i]);

@@ -431,12 +431,13 @@ __global__ void __launch_bounds__(PC *(128 / NPT) + 32) k_scan_seq(ScanSeqArgs a
     const int nt = min(TCH, T - t0);
     // |rshr(dA h, 16)| <= |h| for dA <= 2^16, so over the chunk
     // |h| <= max|h_start| + sum_t |u_t| max|B_t|: below the clamp, clamping
-    // is the identity at every step and the cheaper path is exact.
+    // is the identity at every step and the cheaper path is exact.  With the
+    // split state, |h| <= (|hh| + 1) 2^16 (hl in [0, 2^16)).
     int hmax = 0;
 #pragma unroll
-    for (int j = 0; j < NPT; ++j)
-      hmax = max(hmax, abs(S16 ? hh[j] : (int)(((unsigned)hh[j] << 16) | hl[j])));
-    const bool no_clamp = __all_sync(0xffffffffu, (long long)hmax + s.bound[pp] <=
+    for (int j = 0; j < NPT; ++j) hmax = max(hmax, abs(hh[j]));
+    const long long hbound = S16 ? (long long)hmax : ((long long)hmax + 1) << 16;
+    const bool no_clamp = __all_sync(0xffffffffu, hbound + s.bound[pp] <=
                                                       (S16 ? (long long)kH16Lim : kHLim));
     int2 pr[TCH];
     int2 *wsum = reinterpret_cast<int2 *>(&part[0][0]);

@@ -85,9 +85,23 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t base, uint32_t cols) {
 __device__ __forceinline__ float pow2_q16(long long e) {
   return exp2f(__fmul_rn(__ll2float_rn(e), 1.0f / 65536.0f));
 }
+// The same for e <= 0 with e clamped at -(2^22 - 1) (a decay below 2^-63.99,
+// far under the mode's error budget), so that the exponent converts exactly
+// without the conversion unit.
+__device__ __forceinline__ float pow2_q16_decay(long long e) {
+  const int ec = (int)(e < -4194303LL ? -4194303LL : e);
+  return exp2f(__fmul_rn(small_i2f(ec), 1.0f / 65536.0f));
+}
+// k_ssd_out's x-code tile [128 s][64 B] with its 16-byte pieces XOR-ed by
+// (s >> 1) & 3: a warp reading one piece of 32 consecutive rows, or 32 bytes
+// of one row, touches distinct banks.
+__device__ __forceinline__ int xt_off(int s, int b) {
+  return s * 64 + ((((b >> 4) ^ (s >> 1)) & 3) << 4) + (b & 15);
+}
 
 // dt_q and w of token t of the chunk (0 past the end); W = inclusive prefix
-// sum of w over the chunk's 128 tokens (one per thread), into sW[t].
+// sum of w over the chunk's 128 tokens (one per thread), into sW[t].  Threads
+// t >= kSsdQ of a wider block only pass its barrier.
 // The per-thread inputs of ssd_chunk_decay, loaded at the kernel's start so
 // that their latency overlaps the tile loads: this thread's token's dt_raw
 // (0 past the end), dt_bias[h] and A_q[h].
@@ -120,10 +134,12 @@ __device__ __forceinline__ int ssd_chunk_decay(const SsdDecayIn &in, int nt, lon
     const long long n = __shfl_up_sync(0xffffffffu, v, o);
     if (lane >= o) v += n;
   }
-  if (lane == 31) wtot[warp] = v;
+  if (lane == 31 && t < kSsdQ) wtot[warp] = v;
   __syncthreads();
-  for (int k = 0; k < warp; ++k) v += wtot[k];
-  sW[t] = v;
+  if (t < kSsdQ) {
+    for (int k = 0; k < warp; ++k) v += wtot[k];
+    sW[t] = v;
+  }
   return dtq;
 }
 
@@ -300,9 +316,11 @@ __global__ void __launch_bounds__(256) k_ssd_pass(SsdArgs a) {
 }
 
 // ------------------------------------------------------------ chunk output
-// M reuses the int8 C / B tiles: it is written only after the MMA that reads
-// them has completed (the wait on bar[0]), which keeps the CTA at 109 KB (two
-// per SM).
+// Two threads per token row (256 threads, 8 warps): warps w and w + 4 read
+// the same TMEM lanes (32 (w mod 4) ..) and split the row's columns.  M reuses
+// the int8 C / B tiles: it is written only after the MMA that reads them has
+// completed (the wait on bar[0]), which keeps the CTA at 107 KB (two per SM).
+constexpr int kSsdOutThreads = 256;
 struct SsdOutSmem {
   static constexpr int kC8 = 0;                        // [128 t x 128 B] int8 (A of G)
   static constexpr int kB8 = kC8 + kSsdQ * 128;        // [128 s x 128 B] int8 (B of G)
@@ -320,8 +338,12 @@ struct SsdOutSmem {
 };
 static_assert(SsdOutSmem::kBytes <= 113 * 1024, "two k_ssd_out CTAs per SM");
 
-// grid (nch, nh, B), 128 threads
-__global__ void __launch_bounds__(kSsdThreads) k_ssd_out(SsdArgs a) {
+// grid (nch, nh, B), 256 threads.  Order: the int8 G operands and x codes
+// are loaded; G = Cq Bq^T is issued as soon as they are in; the first half
+// builds Ca from the int8 C tile while the second half builds X'; Y = Ca Hq^T
+// is issued; once G is complete M is built (above-diagonal 32-column blocks
+// are written as zeros without reading G); Y += M X'^T; epilogue.
+__global__ void __launch_bounds__(kSsdOutThreads, 2) k_ssd_out(SsdArgs a) {
   pdl_wait();
   pdl_trigger();
   extern __shared__ uint8_t smem_raw[];
@@ -338,6 +360,9 @@ __global__ void __launch_bounds__(kSsdThreads) k_ssd_out(SsdArgs a) {
   uint32_t *slot = reinterpret_cast<uint32_t *>(sm + L::kSlot);
 
   const int t = threadIdx.x, warp = t >> 5;
+  const int r = t & (kSsdQ - 1);  // token row (and TMEM lane) of this thread
+  const int half = t >> 7;        // which half of the row's columns
+  const int q = warp & 3;         // TMEM lane quarter: rows 32 q .. 32 q + 31
   const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int t0 = c * kSsdQ, nt = min(kSsdQ, a.T - t0);
   const long long row0 = (long long)b * a.T + t0;
@@ -353,13 +378,16 @@ __global__ void __launch_bounds__(kSsdThreads) k_ssd_out(SsdArgs a) {
     mbar_init(&bar[1], 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == 0) tmem_alloc(slot, 256);  // G: columns 0..127 (int32), Y: 128..191 (fp32)
+  if (warp == 0) {
+    tmem_alloc(slot, 256);  // G: columns 0..127 (int32), Y: 128..191 (fp32)
+    tc_fence_before();
+  }
 
   // the chunk's B and C rows (int8 operands of G) and x codes, zero past the
   // end: 16 threads per token row (the B | C bytes are contiguous), so each
   // warp load covers two whole 256-byte rows
 #pragma unroll
-  for (int i = t; i < kSsdQ * 16; i += kSsdThreads) {
+  for (int i = t; i < kSsdQ * 16; i += kSsdOutThreads) {
     const int s = i >> 4, k = i & 15;
     uint4 v = make_uint4(0u, 0u, 0u, 0u);
     if (s < nt) v = *reinterpret_cast<const uint4 *>(a.xbc + (row0 + s) * a.cc + a.di + k * 16);
@@ -367,63 +395,17 @@ __global__ void __launch_bounds__(kSsdThreads) k_ssd_out(SsdArgs a) {
     *reinterpret_cast<uint4 *>(dst) = v;
   }
 #pragma unroll
-  for (int i = t; i < kSsdQ * 4; i += kSsdThreads) {
+  for (int i = t; i < kSsdQ * 4; i += kSsdOutThreads) {
     const int s = i >> 2, k = i & 3;
     uint4 v = make_uint4(0u, 0u, 0u, 0u);
     if (s < nt)
       v = *reinterpret_cast<const uint4 *>(a.xbc + (row0 + s) * a.cc + (long long)h * kSsdHd + k * 16);
-    *reinterpret_cast<uint4 *>(Xt + s * 64 + k * 16) = v;
+    *reinterpret_cast<uint4 *>(Xt + xt_off(s, k * 16)) = v;
   }
-  // (its CTA barrier also makes the tiles above visible to every thread)
+  fence_proxy_async_smem();  // the G tiles, for the tensor cores
+  // (its CTA barrier makes the tiles, the barriers and the TMEM address
+  // visible to every thread)
   const int dtq = ssd_chunk_decay(din, nt, sW, wtot);
-  sdt[t] = __fmul_rn(__int2float_rn(dtq), 1.0f / 65536.0f);
-  {  // row t of Ca: bf16(2^W[t] Cq[t][n]), Cq read back from the int8 tile
-    const float a0 = pow2_q16(sW[t]);
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const uint4 cv = *reinterpret_cast<const uint4 *>(sC8 + sw128_off(t, k * 16, kSsdQ));
-      const uint32_t wv[4] = {cv.x, cv.y, cv.z, cv.w};
-      uint32_t pk[8];
-#pragma unroll
-      for (int q = 0; q < 4; ++q)
-#pragma unroll
-        for (int j = 0; j < 4; j += 2) {
-          const float c0v = __fmul_rn(a0, (float)(int8_t)((wv[q] >> (8 * j)) & 0xFF));
-          const float c1v = __fmul_rn(a0, (float)(int8_t)((wv[q] >> (8 * (j + 1))) & 0xFF));
-          pk[q * 2 + j / 2] = bf16_bits(c0v) | (bf16_bits(c1v) << 16);
-        }
-      // 16 int8 -> 16 bf16 = 32 bytes: two 16-byte pieces at bf16 columns 16k .. 16k+15
-      *reinterpret_cast<uint4 *>(sCa + sw128_off(t, k * 32, kSsdQ)) =
-          make_uint4(pk[0], pk[1], pk[2], pk[3]);
-      *reinterpret_cast<uint4 *>(sCa + sw128_off(t, k * 32 + 16, kSsdQ)) =
-          make_uint4(pk[4], pk[5], pk[6], pk[7]);
-    }
-  }
-  {  // the bf16 state entering the chunk, rows p: 64 x 256 bytes
-    const uint4 *src = reinterpret_cast<const uint4 *>(a.Hin + (bh * a.nch + c) * (kSsdHd * kSsdDs));
-#pragma unroll
-    for (int i = t; i < kSsdHd * 16; i += kSsdThreads) {
-      const int p = i >> 4, j = i & 15;  // 16-byte piece j of row p
-      *reinterpret_cast<uint4 *>(sH + sw128_off(p, j * 16, kSsdHd)) = src[i];
-    }
-  }
-  __syncthreads();  // Xt, sdt, sW complete
-  if (t < kSsdHd) {  // row p = t of X'
-    const int p = t;
-#pragma unroll 1
-    for (int s = 0; s < kSsdQ; s += 8) {
-      uint32_t pk[4];
-#pragma unroll
-      for (int j = 0; j < 8; j += 2)
-        pk[j / 2] = bf16_bits((float)Xt[(s + j) * 64 + p]) |
-                    (bf16_bits((float)Xt[(s + j + 1) * 64 + p]) << 16);
-      *reinterpret_cast<uint4 *>(sX + sw128_off(p, s * 2, kSsdHd)) =
-          make_uint4(pk[0], pk[1], pk[2], pk[3]);
-    }
-  }
-  fence_proxy_async_smem();
-  tc_fence_before();
-  __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *slot;
   if (t == 0) {  // G = Cq Bq^T, exact int32 in TMEM columns 0..127
@@ -433,34 +415,105 @@ __global__ void __launch_bounds__(kSsdThreads) k_ssd_out(SsdArgs a) {
     for (int k = 0; k < 4; ++k) mma_i8(tmem, ad + (uint64_t)(2 * k), bd + (uint64_t)(2 * k), idesc, k > 0 ? 1u : 0u);
     mma_commit(&bar[0]);
   }
+  if (half == 0) {
+    sdt[r] = __fmul_rn(__int2float_rn(dtq), 1.0f / 65536.0f);
+    // row r of Ca: bf16(2^W[r] Cq[r][n]), Cq read back from the int8 tile
+    // (the MMA reads the same tile; neither writes it)
+    const float a0 = pow2_q16(sW[r]);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const uint4 cv = *reinterpret_cast<const uint4 *>(sC8 + sw128_off(r, k * 16, kSsdQ));
+      const uint32_t wv[4] = {cv.x, cv.y, cv.z, cv.w};
+      uint32_t pk[8];
+#pragma unroll
+      for (int qq = 0; qq < 4; ++qq)
+#pragma unroll
+        for (int j = 0; j < 4; j += 2) {
+          const float c0v = __fmul_rn(a0, (float)(int8_t)((wv[qq] >> (8 * j)) & 0xFF));
+          const float c1v = __fmul_rn(a0, (float)(int8_t)((wv[qq] >> (8 * (j + 1))) & 0xFF));
+          pk[qq * 2 + j / 2] = bf16_bits(c0v) | (bf16_bits(c1v) << 16);
+        }
+      // 16 int8 -> 16 bf16 = 32 bytes: two 16-byte pieces at bf16 columns 16k .. 16k+15
+      *reinterpret_cast<uint4 *>(sCa + sw128_off(r, k * 32, kSsdQ)) =
+          make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      *reinterpret_cast<uint4 *>(sCa + sw128_off(r, k * 32 + 16, kSsdQ)) =
+          make_uint4(pk[4], pk[5], pk[6], pk[7]);
+    }
+  } else {
+    // X': row p holds bf16 x[s][p] over s; thread r builds the 8-token
+    // pieces i = r, r + 128, ... of the 16 x 64 grid (p = i mod 64: a warp
+    // reads 32 consecutive bytes of each token row)
+#pragma unroll 2
+    for (int i = r; i < kSsdHd * (kSsdQ / 8); i += kSsdQ) {
+      const int p = i & (kSsdHd - 1), s = (i >> 6) * 8;
+      uint32_t pk[4];
+#pragma unroll
+      for (int j = 0; j < 8; j += 2)
+        pk[j / 2] = bf16_bits((float)Xt[xt_off(s + j, p)]) |
+                    (bf16_bits((float)Xt[xt_off(s + j + 1, p)]) << 16);
+      *reinterpret_cast<uint4 *>(sX + sw128_off(p, s * 2, kSsdHd)) =
+          make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    }
+  }
+  {  // the bf16 state entering the chunk, rows p: 64 x 256 bytes
+    const uint4 *src = reinterpret_cast<const uint4 *>(a.Hin + (bh * a.nch + c) * (kSsdHd * kSsdDs));
+#pragma unroll
+    for (int i = t; i < kSsdHd * 16; i += kSsdOutThreads) {
+      const int p = i >> 4, j = i & 15;  // 16-byte piece j of row p
+      *reinterpret_cast<uint4 *>(sH + sw128_off(p, j * 16, kSsdHd)) = src[i];
+    }
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();  // Ca, X', H, sdt, sW complete
+  tc_fence_after();
+  constexpr uint32_t idesc_y = bf16_idesc(128, 64);
+  const uint32_t dY = tmem + 128;
+  if (t == 0) {  // Y = Ca Hq^T, fp32 in TMEM columns 128..191
+#pragma unroll
+    for (int k = 0; k < kSsdDs / 16; ++k) {
+      const int atom = k >> 2, kk = k & 3;
+      const uint64_t ad = sw128_desc(smem_u32(sCa + atom * kSsdQ * 128)) + (uint64_t)(2 * kk);
+      const uint64_t bd = sw128_desc(smem_u32(sH + atom * kSsdHd * 128)) + (uint64_t)(2 * kk);
+      mma_bf16(dY, ad, bd, idesc_y, k > 0 ? 1u : 0u);
+    }
+  }
   bool ok = mbar_drain(&bar[0], 0);
   tc_fence_after();
-  {  // row t of M: bf16(G[t][s] * fl32(2^(W[t]-W[s]) dt[s])) for s <= t, else 0
-    const long long Wt = sW[t];
+  {  // row r of M: bf16(G[r][s] * fl32(2^(W[r]-W[s]) dt[s])) for s <= r, else 0;
+     // this thread takes the 32-column blocks half, half + 2
+    const long long Wr = sW[r];
 #pragma unroll 1
-    for (int s0 = 0; s0 < kSsdQ; s0 += 32) {
-      uint32_t r[32];
-      tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)s0, r);
+    for (int s0 = half * 32; s0 < kSsdQ; s0 += 64) {
+      if (s0 <= 32 * q + 31) {  // the warp's rows reach this block (warp-uniform)
+        uint32_t g[32];
+        tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)s0, g);
 #pragma unroll
-      for (int j = 0; j < 32; j += 8) {
-        uint32_t pk[4];
+        for (int j = 0; j < 32; j += 8) {
+          uint32_t pk[4];
 #pragma unroll
-        for (int q = 0; q < 8; q += 2) {
-          float m2[2];
+          for (int qq = 0; qq < 8; qq += 2) {
+            float m2[2];
 #pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int s = s0 + j + q + e;
-            float m = 0.0f;
-            if (s <= t) {
-              const float ad = __fmul_rn(pow2_q16(Wt - sW[s]), sdt[s]);
-              m = __fmul_rn(__int2float_rn((int)r[j + q + e]), ad);
+            for (int e = 0; e < 2; ++e) {
+              const int s = s0 + j + qq + e;
+              float m = 0.0f;
+              if (s <= r) {  // |G| <= 128 * 127^2 < 2^22: exact without the conversion unit
+                const float ad = __fmul_rn(pow2_q16_decay(Wr - sW[s]), sdt[s]);
+                m = __fmul_rn(small_i2f((int)g[j + qq + e]), ad);
+              }
+              m2[e] = m;
             }
-            m2[e] = m;
+            pk[qq / 2] = bf16_bits(m2[0]) | (bf16_bits(m2[1]) << 16);
           }
-          pk[q / 2] = bf16_bits(m2[0]) | (bf16_bits(m2[1]) << 16);
+          *reinterpret_cast<uint4 *>(sM + sw128_off(r, (s0 + j) * 2, kSsdQ)) =
+              make_uint4(pk[0], pk[1], pk[2], pk[3]);
         }
-        *reinterpret_cast<uint4 *>(sM + sw128_off(t, (s0 + j) * 2, kSsdQ)) =
-            make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; j += 8)
+          *reinterpret_cast<uint4 *>(sM + sw128_off(r, (s0 + j) * 2, kSsdQ)) =
+              make_uint4(0u, 0u, 0u, 0u);
       }
     }
   }
@@ -468,22 +521,13 @@ __global__ void __launch_bounds__(kSsdThreads) k_ssd_out(SsdArgs a) {
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (t == 0) {  // Y = M X'^T + Ca Hq^T, fp32 in TMEM columns 128..191
-    constexpr uint32_t idesc = bf16_idesc(128, 64);
-    const uint32_t dY = tmem + 128;
+  if (t == 0) {  // Y += M X'^T
 #pragma unroll
     for (int k = 0; k < kSsdQ / 16; ++k) {
       const int atom = k >> 2, kk = k & 3;
       const uint64_t ad = sw128_desc(smem_u32(sM + atom * kSsdQ * 128)) + (uint64_t)(2 * kk);
       const uint64_t bd = sw128_desc(smem_u32(sX + atom * kSsdHd * 128)) + (uint64_t)(2 * kk);
-      mma_bf16(dY, ad, bd, idesc, k > 0 ? 1u : 0u);
-    }
-#pragma unroll
-    for (int k = 0; k < kSsdDs / 16; ++k) {
-      const int atom = k >> 2, kk = k & 3;
-      const uint64_t ad = sw128_desc(smem_u32(sCa + atom * kSsdQ * 128)) + (uint64_t)(2 * kk);
-      const uint64_t bd = sw128_desc(smem_u32(sH + atom * kSsdHd * 128)) + (uint64_t)(2 * kk);
-      mma_bf16(dY, ad, bd, idesc, 1u);
+      mma_bf16(dY, ad, bd, idesc_y, 1u);
     }
     mma_commit(&bar[1]);
   }
@@ -495,32 +539,35 @@ __global__ void __launch_bounds__(kSsdThreads) k_ssd_out(SsdArgs a) {
   constexpr int kYStride = kSsdHd + 4;
   int32_t *sY = reinterpret_cast<int32_t *>(sm + L::kC8);
   static_assert(kSsdQ * kYStride * 4 <= L::kX - L::kC8, "the y tile fits over M and Ca");
-  {  // y codes of token t: rint(Y 2^(e_C+e_x+e_B-e_y)) + rshr(D_q x, s_D), saturated
+  {  // y codes of token r, columns 32 half ..: rint(Y 2^(e_C+e_x+e_B-e_y)) + rshr(D_q x, s_D), saturated
     const float scale = pow2f(s_y);
-#pragma unroll 1
-    for (int c0 = 0; c0 < kSsdHd; c0 += 32) {
-      uint32_t r[32];
-      tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(128 + c0), r);
+    const int c0 = half * 32;
+    uint32_t yv[32];
+    tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(128 + c0), yv);
+    // this row's 32 x codes (two 16-byte pieces)
+    const uint4 xa = *reinterpret_cast<const uint4 *>(Xt + xt_off(r, c0));
+    const uint4 xb = *reinterpret_cast<const uint4 *>(Xt + xt_off(r, c0 + 16));
+    const uint32_t xw[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
 #pragma unroll
-      for (int j = 0; j < 32; j += 4) {
-        int v4[4];
+    for (int j = 0; j < 32; j += 4) {
+      int v4[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          // rint of a float is an integer; the int64 conversion is exact
-          const long long yc = __float2ll_rn(rintf(__fmul_rn(__uint_as_float(r[j + e]), scale)));
-          const long long skip = rshr64(Dq * (long long)Xt[t * 64 + c0 + j + e], s_D);
-          long long v = yc + skip;
-          v = v < -2147483647LL ? -2147483647LL : (v > 2147483647LL ? 2147483647LL : v);
-          v4[e] = (int)v;
-        }
-        *reinterpret_cast<int4 *>(sY + t * kYStride + c0 + j) = make_int4(v4[0], v4[1], v4[2], v4[3]);
+      for (int e = 0; e < 4; ++e) {
+        // rint of a float is an integer; the int64 conversion is exact
+        const long long yc = __float2ll_rn(rintf(__fmul_rn(__uint_as_float(yv[j + e]), scale)));
+        const int xc = (int)(int8_t)((xw[(j + e) >> 2] >> (8 * ((j + e) & 3))) & 0xFFu);
+        const long long skip = rshr64(Dq * (long long)xc, s_D);
+        long long v = yc + skip;
+        v = v < -2147483647LL ? -2147483647LL : (v > 2147483647LL ? 2147483647LL : v);
+        v4[e] = (int)v;
       }
+      *reinterpret_cast<int4 *>(sY + r * kYStride + c0 + j) = make_int4(v4[0], v4[1], v4[2], v4[3]);
     }
   }
   __syncthreads();
   if (ok) {  // 16 threads per token row of 64 int32
 #pragma unroll
-    for (int i = t; i < kSsdQ * 16; i += kSsdThreads) {
+    for (int i = t; i < kSsdQ * 16; i += kSsdOutThreads) {
       const int s = i >> 4, k = i & 15;
       if (s < nt)
         *reinterpret_cast<int4 *>(a.y + (row0 + s) * a.di + (long long)h * kSsdHd + k * 4) =
