@@ -151,54 +151,58 @@ __device__ __forceinline__ int softplus_pwl(int v) {
 }
 
 // ---------------------------------------------------------------- fast forms
-// The same functions for element-wise kernels: the 8 (P_i, S_i) pairs are read
-// from a shared-memory table packed as P | S << 17 (per-lane indices would
-// serialise on the constant cache), and the SiLU division uses a reciprocal
-// estimate with an exact integer correction.  Bit-identical to the forms above.
-__device__ __forceinline__ void pwl_table_init(int *tab) {
-  if (threadIdx.x < 8 && threadIdx.y == 0) tab[threadIdx.x] = pwl_P(threadIdx.x) | (pwl_S(threadIdx.x) << 17);
+// The same functions for element-wise kernels: the 8 chords are read from a
+// shared-memory table (per-lane indices would serialise on the constant
+// cache) as (P_i 2^13 + 2^12, S_i), so that one multiply-add and one shift give
+// P_i + rshr(S_i r, 13) (P_i 2^13 is a multiple of 2^13; the sum stays below
+// 2^31); the SiLU division uses a reciprocal estimate with an exact integer
+// correction.  Bit-identical to the forms above.
+__device__ __forceinline__ void pwl_table_init(int2 *tab) {
+  if (threadIdx.x < 8 && threadIdx.y == 0)
+    tab[threadIdx.x] = make_int2(pwl_P(threadIdx.x) * 8192 + 4096, pwl_S(threadIdx.x));
 }
 
 // e^-|x| in Q.16 (|x| in Q.16): w = rshr(-|x| log2e_Q15, 15) as in exp_pwl,
-// then 2^(w / 2^16) from the table.  |x| is capped at 2^21 (w is then below
-// -31 * 2^16), and the rounding shift by k = -floor(w / 2^16) is capped at
-// 31, where m + 2^30 < 2^31 already rounds to 0 -- no branches.
-__device__ __forceinline__ unsigned exp_neg_abs_t(int x, const int *tab) {
+// then 2^(w / 2^16) from the table (segment (w >> 13) & 7 and offset w & 8191
+// are those of w's fraction w mod 2^16).  |x| is capped at 2^21 (w is then
+// below -31 * 2^16), and the rounding shift by k = -floor(w / 2^16) is capped
+// at 31, where m + 2^30 < 2^31 already rounds to 0 -- no branches.
+__device__ __forceinline__ unsigned exp_neg_abs_t(int x, const int2 *tab) {
   const unsigned ux = x < 0 ? 0u - (unsigned)x : (unsigned)x;
   const int ax = (int)min(ux, 1u << 21);
   const int ah = ax >> 15, al = ax & 0x7FFF;
   const int w = -ah * (int)kLog2eQ15 + ((16384 - al * (int)kLog2eQ15) >> 15);  // <= 0
   const int k = min(-(w >> 16), 31);
-  const int f = w & 0xFFFF;
-  const int e = tab[f >> 13];
-  const int m = (e & 0x1FFFF) + ((((unsigned)e >> 17) * (f & 8191) + 4096) >> 13);
-  return ((unsigned)m + ((1u << k) >> 1)) >> k;
+  const int2 e = tab[(w >> 13) & 7];
+  const unsigned m = ((unsigned)e.y * (unsigned)(w & 8191) + (unsigned)e.x) >> 13;
+  return (m + ((1u << k) >> 1)) >> k;
 }
 
 // SiLU(x / 2^16) in Q.16 for x in +-(2^31 - 1): sigma from E = e^-|x|;
 // x >= 0: floor(2^32 / (2^16 + E)), x < 0: floor(E 2^16 / (2^16 + E));
 // result rshr(x sigma, 16) = xh sigma + ((xl sigma + 2^15) >> 16) with
 // x = xh 2^16 + xl, xl in [0, 2^16) (both products fit 32 bits).
-// The floor division: d = 2^16 + E in [2^16, 2^17] and the numerator (2^32,
-// or E 2^16) are exact floats; num * rcp(d), truncated, is within 2^-5 of the
-// quotient (a few ulp of relative error on a quotient below 2^17), so one
-// correction from the exact remainder (mod 2^32) gives the floor.  The float
-// conversions avoid the conversion unit (small_i2f and a round-to-zero add of
-// 2^23).
-__device__ __forceinline__ int silu_pwl_t(int x, const int *tab) {
+// One floor division serves both signs: with d = 2^16 + E and q = floor(2^32 / d),
+// E 2^16 / d = 2^16 - 2^32 / d, so floor(E 2^16 / d) = 2^16 - ceil(2^32 / d)
+// = 2^16 - q - [d does not divide 2^32], and d in [2^16, 2^17] divides 2^32
+// only for E = 0 or E = 2^16.  The division: d and 2^32 are exact floats;
+// 2^32 rcp(d), truncated, is within 2^-5 of the quotient (a few ulp of
+// relative error on a quotient below 2^17), so one correction from the exact
+// remainder (mod 2^32) gives the floor.  The float conversions avoid the
+// conversion unit (small_i2f and a round-to-zero add of 2^23).
+__device__ __forceinline__ int silu_pwl_t(int x, const int2 *tab) {
   const unsigned E = exp_neg_abs_t(x, tab);
   const unsigned d = 65536u + E;
   float rd;
   asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(rd) : "f"(small_i2f((int)d)));
-  const float numf = x >= 0 ? 4294967296.0f : __fmul_rn(small_i2f((int)E), 65536.0f);
-  const unsigned nmod = x >= 0 ? 0u : (E << 16);  // numerator mod 2^32
-  unsigned q = __float_as_uint(__fadd_rz(__fmul_rz(numf, rd), 8388608.0f)) - 0x4B000000u;
-  const unsigned rem = nmod - q * d;
+  unsigned q = __float_as_uint(__fadd_rz(__fmul_rz(4294967296.0f, rd), 8388608.0f)) - 0x4B000000u;
+  const unsigned rem = 0u - q * d;  // 2^32 - q d (mod 2^32)
   if ((int)rem < 0) q -= 1u;
   else if (rem >= d) q += 1u;
+  const unsigned sig = x >= 0 ? q : 65536u - q - ((E - 1u) < 65535u ? 1u : 0u);
   const int xh = x >> 16;
   const unsigned xl = (unsigned)x & 0xFFFFu;
-  return xh * (int)q + (int)((xl * q + 32768u) >> 16);
+  return xh * (int)sig + (int)((xl * sig + 32768u) >> 16);
 }
 
 // rshr(v, k) for int32 v and k in [1, 31] without overflow: floor(v / 2^k) +

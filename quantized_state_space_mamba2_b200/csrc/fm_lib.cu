@@ -85,7 +85,13 @@ static fm_status launch_ex(const char *name, void (*kern)(KArgs...), dim3 grid, 
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = g_pdl.load(std::memory_order_relaxed) ? 1 : 0;
+  // never for the sequential scan, whose CTAs launched early land unevenly
+  // on SMs still busy with the prep kernel (measured 232 -> 355 us per 130M
+  // layer), nor for the gate after it, whose early CTAs would share the
+  // issue-bound scan's SMs while they wait
+  const bool placed = std::strcmp(name, "k_scan_seq") == 0 ||
+                      std::strcmp(name, "k_gate_norm_quant") == 0;
+  cfg.numAttrs = g_pdl.load(std::memory_order_relaxed) && !placed ? 1 : 0;
   const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, args...);
   if (e != cudaSuccess) return fail(FM_ERR_CUDA, "launch of %s: %s", name, cudaGetErrorString(e));
   return FM_OK;
@@ -454,23 +460,18 @@ static fm_status launch_conv(const int8_t *u, int B, int T, int cc, const int8_t
   if (T >= kConvTT) {
     const unsigned tiles = (unsigned)((T + kConvTokens - 1) / kConvTokens);
     const dim3 grid(tiles, groups, B);
-    if (e_tok)
-      FM_TRY(launch_ex("k_conv1d_pot", k_conv1d_pot<kConvTT, kConvTG, true>, grid,
-                       kConvQuads * kConvTG, 0, s, u, T, cc, wq, bq, exps, conv_state, out, amax,
-                       nullptr, e_tok, di, hd, ds));
-    else
-      FM_TRY(launch_ex("k_conv1d_pot", k_conv1d_pot<kConvTT, kConvTG, false>, grid,
-                       kConvQuads * kConvTG, 0, s, u, T, cc, wq, bq, exps, conv_state, out, amax,
-                       nullptr, e_tok, di, hd, ds));
+    auto kern = e_tok ? k_conv1d_pot<kConvTT, kConvTG, true>
+                      : (amax ? k_conv1d_pot<kConvTT, kConvTG, false, true>
+                              : k_conv1d_pot<kConvTT, kConvTG, false, false>);
+    FM_TRY(launch_ex("k_conv1d_pot", kern, grid, kConvQuads * kConvTG, 0, s, u, T, cc, wq, bq,
+                     exps, conv_state, out, amax, nullptr, e_tok, di, hd, ds));
   } else {  // decode steps and short chunks: one token per thread
     const dim3 grid((unsigned)T, groups, B);
     int8_t *state_out = T == 1 ? conv_state : nullptr;
-    if (e_tok)
-      FM_TRY(launch_ex("k_conv1d_pot", k_conv1d_pot<1, 1, true>, grid, kConvQuads, 0, s, u, T, cc,
-                       wq, bq, exps, conv_state, out, amax, state_out, e_tok, di, hd, ds));
-    else
-      FM_TRY(launch_ex("k_conv1d_pot", k_conv1d_pot<1, 1, false>, grid, kConvQuads, 0, s, u, T,
-                       cc, wq, bq, exps, conv_state, out, amax, state_out, e_tok, di, hd, ds));
+    auto kern = e_tok ? k_conv1d_pot<1, 1, true>
+                      : (amax ? k_conv1d_pot<1, 1, false, true> : k_conv1d_pot<1, 1, false, false>);
+    FM_TRY(launch_ex("k_conv1d_pot", kern, grid, kConvQuads, 0, s, u, T, cc, wq, bq, exps,
+                     conv_state, out, amax, state_out, e_tok, di, hd, ds));
   }
   FM_TRY(launched("k_conv1d_pot"));
   if (conv_state && T > 1) {  // a single step updates its state in the conv kernel
@@ -1130,7 +1131,7 @@ extern "C" fm_status fm_gate_norm_quant(const int32_t *y, const float *z, int64_
 }
 
 __global__ void k_eval_pwl(int kind, const int64_t *in, long long n, int64_t *out) {
-  __shared__ int tab[8];
+  __shared__ int2 tab[8];
   pwl_table_init(tab);
   __syncthreads();
   const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;

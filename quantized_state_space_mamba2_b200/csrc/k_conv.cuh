@@ -50,7 +50,13 @@ __device__ __forceinline__ void conv_transpose4(uint32_t r0, uint32_t r1, uint32
 // [B*T, nh + 2]) receives e.  A head's 64 x channels are 16 consecutive
 // threads and B, C one warp each (the x | B | C boundaries are multiples of
 // 256 channels), so the group maximum is a shuffle reduction.
-template <int TT, int TG, bool TOK = false>
+// CALIB: amax is non-null (calibration); otherwise it is not read.
+// The common case takes a short path: when none of the thread's 4 channels
+// can saturate x16 (|b| + 4 127^2, shifted to Q.16, stays inside int32) nor
+// overflow the output's rounding add, x16 = (dp4a(taps, w, b + rounding bias)
+// >> right) << left and the output code is a plain add-and-shift, both exact;
+// any other thread runs the general 64-bit form.
+template <int TT, int TG, bool TOK = false, bool CALIB = false>
 __global__ void __launch_bounds__(kConvQuads *TG) k_conv1d_pot(
     const int8_t *__restrict__ u, int T, int cc, const int8_t *__restrict__ wq,
     const int32_t *__restrict__ bq, const int32_t *__restrict__ exps,
@@ -58,7 +64,7 @@ __global__ void __launch_bounds__(kConvQuads *TG) k_conv1d_pot(
     int8_t *state_out, int32_t *e_tok = nullptr, int di = 0, int hd = 0, int ds = 0) {
   pdl_wait();
   pdl_trigger();
-  __shared__ int tab[8];
+  __shared__ int2 tab[8];
   pwl_table_init(tab);
   __syncthreads();
   const int quad = threadIdx.x % kConvQuads, tg = threadIdx.x / kConvQuads;
@@ -96,11 +102,26 @@ __global__ void __launch_bounds__(kConvQuads *TG) k_conv1d_pot(
   const int s_in[4] = {-(ew.x + eu.x + 16), -(ew.y + eu.y + 16), -(ew.z + eu.z + 16),
                        -(ew.w + eu.w + 16)};
   const int s_out[4] = {eo.x + 16, eo.y + 16, eo.z + 16, eo.w + 16};
-  bool fast[4];  // |acc| < 2^30 (the taps add at most 4 * 127^2) and a 32-bit shift
+  // short-path constants: dp4a accumulator (bias + the rounding bias of a
+  // right shift), right and left shifts to Q.16, the output's rounding bias
+  int cb[4], rsh[4], lsh[4], rob[4];
+  bool easy = !TOK;
 #pragma unroll
-  for (int j = 0; j < 4; ++j)
-    fast[j] = bs[j] >= -(1 << 29) && bs[j] <= (1 << 29) && s_in[j] >= -30 && s_in[j] <= 29 &&
-              s_out[j] >= 1 && s_out[j] <= 31;
+  for (int j = 0; j < 4; ++j) {
+    const int si = s_in[j], so = s_out[j];
+    const bool ok = bs[j] >= -(1 << 29) && bs[j] <= (1 << 29) && si >= -30 && si <= 29 &&
+                    so >= 1 && so <= 31;
+    rsh[j] = si > 0 ? si : 0;
+    lsh[j] = si > 0 ? 0 : -si;
+    cb[j] = ok ? bs[j] + (si > 0 ? 1 << (si - 1) : 0) : 0;
+    rob[j] = ok ? 1 << (so - 1) : 0;
+    // |x16| bound: |acc| <= |b| + 4 127^2 (+ the rounding bias), then shifted
+    const long long ab = (long long)(bs[j] < 0 ? -(long long)bs[j] : bs[j]) + 64516 +
+                         (si > 0 && si < 62 ? (1LL << (si - 1)) : 0);
+    const long long xb = ok ? (si > 0 ? (ab >> si) + 1 : ab << lsh[j]) : (1LL << 40);
+    // |SiLU(x16)| <= |x16|, so the output's rounding add cannot overflow either
+    easy = easy && ok && xb + (1LL << (so - 1)) <= 2147483647LL;
+  }
   uint32_t col[4];
   conv_transpose4(row[0], row[1], row[2], row[3], col);
   const int nt = min(TT, T - t0);
@@ -141,30 +162,25 @@ __global__ void __launch_bounds__(kConvQuads *TG) k_conv1d_pot(
       *reinterpret_cast<uint32_t *>(out + ((long long)b * T + t0 + k) * cc + c0) = packed;
       continue;
     }
+    if (easy) {
 #pragma unroll
-    for (int j = 0; j < kConvCPT; ++j) {
-      int code;
-      if (fast[j]) {
-        const int acc = __dp4a((int)col[j], wr[j], bs[j]);
-        const int si = s_in[j];
-        int x16;
-        if (si > 0) {
-          x16 = rshr32(acc, si);
-        } else {
-          const int sh = -si, lim = 0x7FFFFFFF >> sh;
-          x16 = acc > lim ? 2147483647 : (acc < -lim ? -2147483647 : acc * (1 << sh));
-        }
+      for (int j = 0; j < kConvCPT; ++j) {
+        const int x16 = (__dp4a((int)col[j], wr[j], cb[j]) >> rsh[j]) << lsh[j];
         const int sv = silu_pwl_t(x16, tab);
-        if (amax) atomicMax(amax + c0 + j, (unsigned int)(sv < 0 ? -sv : sv));
-        code = min(max(rshr32(sv, s_out[j]), -127), 127);
-      } else {
+        if constexpr (CALIB) atomicMax(amax + c0 + j, (unsigned int)(sv < 0 ? -sv : sv));
+        const int code = min(max((sv + rob[j]) >> s_out[j], -127), 127);
+        packed |= ((uint32_t)(code & 0xFF)) << (8 * j);
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < kConvCPT; ++j) {
         const long long acc = (long long)bs[j] + __dp4a((int)col[j], wr[j], 0);
         const int x16 = (int)satb64(rshr64(acc, s_in[j]), 32);
         const int sv = silu_pwl_t(x16, tab);
-        if (amax) atomicMax(amax + c0 + j, (unsigned int)(sv < 0 ? -sv : sv));
-        code = (int)satb64(rshr64(sv, s_out[j]), 8);
+        if constexpr (CALIB) atomicMax(amax + c0 + j, (unsigned int)(sv < 0 ? -sv : sv));
+        const int code = (int)satb64(rshr64(sv, s_out[j]), 8);
+        packed |= ((uint32_t)(code & 0xFF)) << (8 * j);
       }
-      packed |= ((uint32_t)(code & 0xFF)) << (8 * j);
     }
     *reinterpret_cast<uint32_t *>(out + ((long long)b * T + t0 + k) * cc + c0) = packed;
   }

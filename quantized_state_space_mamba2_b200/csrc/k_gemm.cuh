@@ -117,6 +117,22 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
   return mbar_wait_for(bar, parity, *(volatile unsigned long long *)&g_wait_limit_ns);
 }
+// a wait expected to be long (a producer waiting for its consumers, epilogue
+// warps waiting out the whole main loop): the thread sleeps between polls, so
+// it takes few issue slots from the warps doing the work
+__device__ __forceinline__ bool mbar_wait_sleepy(uint64_t *bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long limit = *(volatile unsigned long long *)&g_wait_limit_ns;
+  const unsigned long long t0 = globaltimer();
+  while (true) {
+    __nanosleep(128);
+    if (mbar_try_wait(bar, parity)) return true;
+    if (globaltimer() - t0 > limit) {
+      raise_error(kErrTimeout);
+      return false;
+    }
+  }
+}
 // a drain: waits for work this CTA has already issued, at the fixed limit
 __device__ __forceinline__ bool mbar_drain(uint64_t *bar, uint32_t parity) {
   return mbar_wait_for(bar, parity, kWaitLimitNs);
@@ -430,7 +446,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
     const float sx = row < ep.M ? ep.s_x[row] : 0.0f;
     asm volatile("bar.sync 1, 128;" ::: "memory");  // the 4 epilogue warps only
     // tcgen05.ld is warp-collective: the whole warp skips it after a failed wait
-    const bool ok = __all_sync(0xffffffffu, mbar_wait(accum_bar, 0));
+    const bool ok = __all_sync(0xffffffffu, mbar_wait_sleepy(accum_bar, 0));
     tc_fence_after();
 #pragma unroll 1
     for (int c = 0; c < BN && ok; c += 32) {

@@ -31,19 +31,15 @@ __device__ __forceinline__ void load8(const float *p, float (&v)[8]) {
   v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
 }
 
-// Row max over all warps of the CTA (every thread returns the result).
-__device__ __forceinline__ float cta_max(float v, float *s_red, float *s_out) {
+// Row max over all warps of the CTA (every thread returns the result): each
+// warp reduces the warps' maxima itself (lane i reads warp i's), so one
+// barrier suffices.  Called once per kernel (s_red is not reused).
+__device__ __forceinline__ float cta_max(float v, float *s_red) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
   v = warp_max(v);
   if (lane == 0) s_red[warp] = v;
   __syncthreads();
-  if (threadIdx.x == 0) {
-    float m = 0.0f;
-    for (int w = 0; w < nw; ++w) m = fmaxf(m, s_red[w]);
-    *s_out = m;
-  }
-  __syncthreads();
-  return *s_out;
+  return warp_max(lane < nw ? s_red[lane] : 0.0f);
 }
 
 // Rotation (optional) + per-row or static quantisation of this lane's BPW
@@ -54,7 +50,7 @@ template <int BPW>
 __device__ __forceinline__ void rotate_quant_store(float (&v)[BPW][8], int rotate, int mode,
                                                    const float *static_amax, int8_t *qrow,
                                                    float *sx_out, float *amax_out,
-                                                   float *s_red, float *s_bc) {
+                                                   float *s_red) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   if (rotate) {
 #pragma unroll
@@ -71,7 +67,7 @@ __device__ __forceinline__ void rotate_quant_store(float (&v)[BPW][8], int rotat
       a = fmaxf(a, m);
     }
   if (!finite) raise_error(kErrNonfinite);
-  const float amax = cta_max(a, s_red, s_bc);
+  const float amax = cta_max(a, s_red);
   const float use = (mode == 0) ? amax : *static_amax;
   const float inv = use > 0.0f ? __fdiv_rn(127.0f, use) : 0.0f;
 #pragma unroll
@@ -105,7 +101,6 @@ __global__ void __launch_bounds__(1024) k_hadamard_quant(const float *__restrict
   pdl_trigger();
   __shared__ double s_blk[kMaxBlocks];
   __shared__ float s_red[kMaxBlocks];
-  __shared__ float s_bc;
   __shared__ float s_rstd;
   const long long row = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -152,7 +147,7 @@ __global__ void __launch_bounds__(1024) k_hadamard_quant(const float *__restrict
     }
   }
   rotate_quant_store<BPW>(v, rotate, mode, static_amax, q + row * K, s_x + row,
-                          amax_row ? amax_row + row : nullptr, s_red, &s_bc);
+                          amax_row ? amax_row + row : nullptr, s_red);
 }
 
 // a9 + a10: gate y * SiLU(z), g_q int16 at e_g, exact-integer RMSNorm,
@@ -168,9 +163,8 @@ __global__ void __launch_bounds__(1024) k_gate_norm_quant(
   pdl_trigger();
   __shared__ long long s_ss[kMaxBlocks];
   __shared__ float s_red[kMaxBlocks];
-  __shared__ float s_bc;
   __shared__ float s_rstd;
-  __shared__ int tab[8];
+  __shared__ int2 tab[8];
   pwl_table_init(tab);
   __syncthreads();
   const long long row = blockIdx.x;
@@ -198,17 +192,33 @@ __global__ void __launch_bounds__(1024) k_gate_norm_quant(
     }
     unsigned ss0 = 0, ss1 = 0;  // g_q^2 < 2^30: four per partial fit 32 bits
     unsigned long long gmax = 0;
+    int sg[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) sg[i] = silu_pwl_t(to_q16(zv[i]), tab);
+    if (!gstat && sg_shift >= 33 && sg_shift <= 63) {
+      // the usual case (a calibrated layer's shift is 33..40): with g = hi 2^32 + lo,
+      // floor((g + 2^(s-1)) / 2^s) = floor((hi + 2^(s-33)) / 2^(s-32)) because
+      // lo / 2^32 < 1 cannot carry the integer numerator past a multiple of
+      // 2^(s-32); |hi| < 2^30, so the sum stays in int32
+      const int rb = 1 << (sg_shift - 33), sh = sg_shift - 32;
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        gq[b][i] = min(max((__mulhi(yv[i], sg[i]) + rb) >> sh, -32767), 32767);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        // g = y sg as a 64-bit value from two 32-bit multiplies
+        const long long g = (long long)(((unsigned long long)(unsigned)__mulhi(yv[i], sg[i]) << 32) |
+                                        (unsigned)(yv[i] * sg[i]));
+        if (gstat) {
+          const unsigned long long ag = (unsigned long long)(g < 0 ? -g : g);
+          gmax = ag > gmax ? ag : gmax;
+        }
+        gq[b][i] = (int)satb64(rshr64(g, sg_shift), 16);
+      }
+    }
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      const int sg = silu_pwl_t(to_q16(zv[i]), tab);
-      // g = y sg as a 64-bit value from two 32-bit multiplies
-      const long long g = (long long)(((unsigned long long)(unsigned)__mulhi(yv[i], sg) << 32) |
-                                      (unsigned)(yv[i] * sg));
-      if (gstat) {
-        const unsigned long long ag = (unsigned long long)(g < 0 ? -g : g);
-        gmax = ag > gmax ? ag : gmax;
-      }
-      gq[b][i] = (int)satb64(rshr64(g, sg_shift), 16);
       const unsigned sq = (unsigned)(gq[b][i] * gq[b][i]);
       if (i < 4) ss0 += sq;
       else ss1 += sq;
@@ -246,7 +256,7 @@ __global__ void __launch_bounds__(1024) k_gate_norm_quant(
       v[b][i] = __fmul_rn(__fmul_rn(__fmul_rn(small_i2f(gq[b][i]), scale), rstd), w[i]);
   }
   rotate_quant_store<BPW>(v, rotate, mode, static_amax, q + row * di, s_x + row,
-                          amax_row ? amax_row + row : nullptr, s_red, &s_bc);
+                          amax_row ? amax_row + row : nullptr, s_red);
 }
 
 // Offline weight preparation: W' = W H (fp64, same butterfly order),

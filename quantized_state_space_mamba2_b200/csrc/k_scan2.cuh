@@ -373,7 +373,7 @@ __global__ void __launch_bounds__(PC *(128 / NPT) + 32) k_scan_seq(ScanSeqArgs a
       for (int c = 0; c < nissue; ++c) {
         const int sl = c % kScanSlots;
         if (c >= kScanSlots &&
-            !mbar_wait(&sm.empty[sl], (uint32_t)((c / kScanSlots) - 1) & 1u))
+            !mbar_wait_sleepy(&sm.empty[sl], (uint32_t)((c / kScanSlots) - 1) & 1u))
           break;  // error word set; consumers time out on the full barrier
         typename Sm::Slot &s = sm.slot[sl];
         const int t0 = c * TCH;

@@ -240,6 +240,38 @@ def test_conv1d_pot(L, B, T, with_state):
         assert np.array_equal(host(st_d), st_r)
 
 
+@pytest.mark.parametrize("B,T", [(1, 1), (2, 37)])
+def test_conv1d_pot_extreme_exponents(L, B, T):
+    """Per-channel exponents and biases far from a calibrated layer's: large
+    left shifts that saturate the Q.16 input, right shifts past 29, biases
+    beyond 2^29, output shifts from -5 to 40.  Threads whose four channels
+    all stay clear of saturation and overflow take the kernel's short path,
+    the others its general 64-bit form; both must equal the oracle."""
+    s = MAMBA130
+    cc = s.conv_ch
+    wq = S.uniform_ints((cc, 4), -127, 127, seed=301, dtype=np.int8)
+    bq = S.uniform_ints(cc, -2 ** 12, 2 ** 12, seed=302)
+    big = S.uniform_ints(cc, 0, 29, seed=303) == 0           # ~3 % of channels
+    bq = np.where(big, S.uniform_ints(cc, -2 ** 30, 2 ** 30, seed=304), bq).astype(np.int32)
+    wild = S.uniform_ints(cc, 0, 19, seed=309) < 3          # ~15 % of channels
+    s_in = np.where(wild, S.uniform_ints(cc, -30, 35, seed=305),
+                    S.uniform_ints(cc, -10, 10, seed=310))
+    s_out = np.where(wild, S.uniform_ints(cc, -5, 40, seed=306),
+                     S.uniform_ints(cc, 10, 24, seed=311))
+    e_u = S.uniform_ints(cc, -8, 2, seed=307).astype(np.int32)
+    e_w = (-(s_in + 16) - e_u).astype(np.int32)
+    e_o = (s_out - 16).astype(np.int32)
+    exps = np.zeros(L.exp_table_layout(s).size, np.int32)
+    exps[:cc], exps[cc:2 * cc], exps[2 * cc:3 * cc] = e_u, e_w, e_o
+    u = S.uniform_ints((B, T, cc), -127, 127, seed=308 + T, dtype=np.int8)
+    out = torch.empty((B, T, cc), dtype=torch.int8, device="cuda")
+    L.conv1d_pot(dev(u), B, T, s, dev(wq), dev(bq), dev(exps), None, out)
+    ref = O.conv1d_pot(u, wq, bq, e_u, e_w, e_o)
+    assert np.array_equal(host(out), ref)
+    # both regimes occur: saturated Q.16 inputs and channels on the short path
+    assert (np.abs(ref) == 127).mean() > 0.02 and (np.abs(ref) < 127).mean() > 0.5
+
+
 def test_prepare_mixer_params(L):
     s = MAMBA130
     P = S.layer_params(s, 11, conv_bias_std=0.1)
@@ -427,14 +459,18 @@ def test_ssm_scan_clamp_regimes(L, regime):
 @pytest.mark.parametrize("M", [1, 77, 512])
 @pytest.mark.parametrize("mode", [0, 1])
 @pytest.mark.parametrize("di", [1536, 768, 5120])
-def test_gate_norm_quant(L, M, mode, di):
+@pytest.mark.parametrize("shift", ["small", "large"])
+def test_gate_norm_quant(L, M, mode, di, shift):
     """d_inner with an even number of 256-blocks (two per warp) and an odd one
-    (one per warp)."""
+    (one per warp).  The gate shift e_g - e_y + 16 per head: 14..18 ("small",
+    the 64-bit form) or 32..36 ("large": heads at 33 and above take the
+    high-word form, the head at 32 the 64-bit one, and the largest products
+    saturate the int16 gated code)."""
     s = S.MixerShape(d_model=768, d_inner=di, headdim=64, d_state=128)
     y = S.uniform_ints((M, s.d_inner), -2 ** 29, 2 ** 29, seed=M, dtype=np.int32)
     z = S.normal((M, s.d_inner), 3.0, seed=M + 1)
     e_y = S.uniform_ints(s.nheads, -22, -18, seed=M + 2)
-    e_g = int(e_y.max()) - 16 + 14
+    e_g = int(e_y.max()) - 16 + (14 if shift == "small" else 32)
     w = (1.0 + S.normal(s.d_inner, 0.2, seed=9)).astype(np.float32)
     X = L.exp_table_layout(s)
     exps = np.zeros(X.size, np.int32)
