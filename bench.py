@@ -109,8 +109,9 @@ def parse(argv=None):
                     help="tile width of the persistent GEMM (0: chosen by the grid)")
     ap.add_argument("--lq-cpw", type=int, default=0, choices=[0, 1, 2, 4],
                     help="channels per warp of the LQ scan (0: chosen by the grid)")
-    ap.add_argument("--pdl", action="store_true",
-                    help="programmatic dependent launch of the library's kernels")
+    ap.add_argument("--pdl", default="on", choices=["on", "off"],
+                    help="programmatic dependent launch of the library's kernels (on: the "
+                         "library's default)")
     ap.add_argument("--eager", action="store_true",
                     help="launch the timed steps one by one instead of replaying them as one "
                          "captured CUDA graph")
@@ -939,7 +940,8 @@ def measure(args, wl, torch, dist, lib, dev, world, flush) -> dict:
     e2e_value = world * wl.tokens * args.steps / (e2e_total / 1000.0)
     del graph
     return {"value": value, "ms_per_step": total_ms / args.steps, "roofline": roofline,
-            "clocks": clk, "launch": "eager" if args.eager else "one CUDA graph of the K steps",
+            "clocks": clk, "launch": ("eager" if args.eager else "one CUDA graph of the K steps") +
+            (", programmatic dependent launch" if getattr(args, "pdl", "on") == "on" else ""),
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": wl.h2d_bytes,
                     "d2h_bytes_per_step": wl.d2h_bytes},
             "gpu_launches": wl.launches * args.steps}
@@ -952,7 +954,7 @@ def apply_modes(args, lib):
     lib.set_scan_mode(args.scan_mode)
     lib.set_state_spec(*[int(v) for v in args.state_spec.split(",")])
     lib.set_gemm_tile(args.gemm_tile)
-    lib.set_pdl(getattr(args, "pdl", False))
+    lib.set_pdl(getattr(args, "pdl", "on") == "on")
     lib.set_lq_scan_cpw(getattr(args, "lq_cpw", 0))
     lib.set_xbc_exponents(args.xbc_exponents)
 

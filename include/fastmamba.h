@@ -87,12 +87,15 @@ fm_status fm_sync_status(fm_stream stream);
  * fm_set_fault_injection(0, 0) restores normal operation.  Synchronous
  * (cudaMemcpyToSymbol); not for use while the device runs library kernels. */
 fm_status fm_set_fault_injection(int stall_mask, uint64_t wait_limit_ns);
-/* Tuning, process-wide (the pages have no counterpart): 1 launches the hot
- * kernels with programmatic stream serialisation, so that each may be
- * scheduled while its predecessor in the stream drains (every such kernel
- * waits for its predecessor before its first global memory access); 0
- * (default) launches them plainly.  Results are the same bits either way.
- * FM_ERR_INVALID_ARG for other values. */
+/* Tuning, process-wide (the pages have no counterpart): 1 (default) launches
+ * the hot kernels with programmatic stream serialisation, so that each may be
+ * scheduled while its predecessor in the stream drains.  Every such kernel
+ * waits for its predecessor before it reads that kernel's outputs; before the
+ * wait the GEMMs fetch their first weight stages and the single decode step
+ * its state (the kernels that write a state end before any successor starts).
+ * The sequential scan and the gate after it are always launched plainly (the
+ * scan's CTA placement matters).  0 launches every kernel plainly.  Results
+ * are the same bits either way.  FM_ERR_INVALID_ARG for other values. */
 fm_status fm_set_pdl(int enable);
 /* Library ABI version (major * 100 + minor). */
 int fm_version(void);
@@ -236,7 +239,7 @@ fm_status fm_conv1d_pot_tok(const int8_t *u, int B, int T, const fm_shape *shape
 /* Tuning: selects the tile of the sequential scan kernel used by every later
  * call in this process -- npt state columns per thread, pc channels per CTA,
  * tch time steps per staged chunk.  Compiled variants: (4,4,16) (default),
- * (4,2,16), (4,8,16), (8,4,16), (8,2,16), (8,8,16);
+ * (4,2,16), (4,8,16), (8,4,16), (8,2,16), (8,8,16), (4,4,32);
  * anything else returns FM_ERR_INVALID_ARG.  All variants compute the same
  * bits. */
 fm_status fm_set_scan_tile(int npt, int pc, int tch);

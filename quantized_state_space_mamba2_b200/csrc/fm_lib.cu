@@ -64,7 +64,7 @@ static fm_status launched(const char *what) {
 // default): with it a kernel may be scheduled while its predecessor in the
 // stream drains; every kernel launched this way waits (pdl_wait) before its
 // first global memory access.
-static std::atomic<int> g_pdl{0};
+static std::atomic<int> g_pdl{1};
 
 extern "C" fm_status fm_set_pdl(int enable) {
   if (enable != 0 && enable != 1) return fail(FM_ERR_INVALID_ARG, "fm_set_pdl: enable must be 0 or 1");
@@ -557,7 +557,7 @@ struct ScanTile {
   int npt, pc, tch;
 };
 static const ScanTile kScanTiles[] = {{4, 4, 16}, {4, 2, 16}, {4, 8, 16},
-                                      {8, 4, 16}, {8, 2, 16}, {8, 8, 16}};
+                                      {8, 4, 16}, {8, 2, 16}, {8, 8, 16}, {4, 4, 32}};
 static std::atomic<int> g_scan_tile{0};
 // 0: the sequential fixed-point scan (the method); 1: the chunked scan mode for
 // prefills of more than one token (single steps stay sequential)
@@ -680,6 +680,7 @@ static fm_status launch_scan_v2(const ScanArgs &a, int B, const ScanWs &w, cudaS
   FM_SEQ(8, 4, 16)
   FM_SEQ(8, 2, 16)
   FM_SEQ(8, 8, 16)
+  FM_SEQ(4, 4, 32)
 #undef FM_SEQ
   return fail(FM_ERR_INVALID_ARG, "scan tile (%d, %d, %d) is not compiled", t.npt, t.pc, t.tch);
 }

@@ -388,14 +388,26 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  pdl_wait();  // the prologue above touches only this CTA's shared memory and TMEM
+  // The prologue above touches only this CTA's shared memory and TMEM.  Under
+  // programmatic dependent launch (fm_set_pdl) the weights -- written long
+  // before -- are fetched for the first stages while the previous kernel
+  // drains; only the producer lane (before the activations) and the epilogue
+  // warps (before the row scales and the residual) wait for it.
   pdl_trigger();
 
   if (warp == 0) {
     if (lane == 0) {
       const int kb_issue = (g_test_stall & kStallGemm) ? 0 : kb_n;
-      int issued = 0;
-      for (int kb = 0; kb < kb_issue; ++kb) {
+      const int pre = kb_issue < STAGES ? kb_issue : STAGES;
+      for (int kb = 0; kb < pre; ++kb) {  // fresh ring: no empty-slot wait
+        mbar_arrive_expect_tx(&full_bar[kb], (uint32_t)((AR + BN) * kGemmBK));
+        tma_load_2d(sB + kb * BN * kGemmBK, &tmB, (kb0 + kb) * kGemmBK, n0, &full_bar[kb]);
+      }
+      pdl_wait();
+      for (int kb = 0; kb < pre; ++kb)
+        tma_load_2d(sA + kb * AR * kGemmBK, &tmA, (kb0 + kb) * kGemmBK, m0, &full_bar[kb]);
+      int issued = pre;
+      for (int kb = pre; kb < kb_issue; ++kb) {
         const int s = kb % STAGES;
         const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
         if (!mbar_wait(&empty_bar[s], ph ^ 1u)) break;
@@ -432,6 +444,7 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
       mbar_drain(accum_bar, 0);
     }
   } else {
+    pdl_wait();
     // while the main loop runs: stage this tile's column scales and the row scale
     const int et = threadIdx.x - 64;  // 0 .. 127
     for (int j = et; j < BN; j += 128) {
@@ -689,16 +702,34 @@ __global__ void __launch_bounds__(64 + 32 * EW, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  pdl_wait();  // the prologue above touches only this CTA's shared memory and TMEM
+  // As in k_gemm_i8_tc: under programmatic dependent launch the weights of
+  // the first tile's first stages are fetched before the dependency wait;
+  // the producer lane waits before the activations, the epilogue warps before
+  // the row scales and the residual.
   pdl_trigger();
 
   if (warp == 0) {
     if (lane == 0) {
-      long long it = 0;
       bool ok = !(g_test_stall & kStallGemm);
+      const int pre = ok && (int)blockIdx.x < num_tiles
+                          ? (num_k_blocks < STAGES ? num_k_blocks : STAGES) : 0;
+      if (pre) {
+        const int n0 = ((int)blockIdx.x % n_tiles) * BN;
+        for (int kb = 0; kb < pre; ++kb) {  // fresh ring: no empty-slot wait
+          mbar_arrive_expect_tx(&full_bar[kb], (uint32_t)(Sm::kA + Sm::kB));
+          tma_load_2d(sB + kb * Sm::kB, &tmB, kb * kGemmBK, n0, &full_bar[kb]);
+        }
+      }
+      pdl_wait();
+      if (pre) {
+        const int m0 = ((int)blockIdx.x / n_tiles) * kGemmBM;
+        for (int kb = 0; kb < pre; ++kb)
+          tma_load_2d(sA + kb * Sm::kA, &tmA, kb * kGemmBK, m0, &full_bar[kb]);
+      }
+      long long it = pre;
       for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
         const int m0 = (t / n_tiles) * kGemmBM, n0 = (t % n_tiles) * BN;
-        for (int kb = 0; kb < num_k_blocks; ++kb, ++it) {
+        for (int kb = t == (int)blockIdx.x ? pre : 0; kb < num_k_blocks; ++kb, ++it) {
           const int s = (int)(it % STAGES);
           const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
           if (!mbar_wait(&empty_bar[s], ph ^ 1u)) {
@@ -754,6 +785,7 @@ __global__ void __launch_bounds__(64 + 32 * EW, 1)
       mbar_drain(drain_bar, 0);
     }
   } else {
+    pdl_wait();
     const int e = warp - 2;                 // 0 .. EW-1
     const int quarter = warp & 3;           // TMEM lanes [32 quarter, 32 quarter + 32)
     const int part = e / 4;                 // which column slice of the tile

@@ -81,12 +81,30 @@ __global__ void __launch_bounds__(256) k_scan_prep(ScanPrepArgs a) {
   const long long Tp = scan_tpad(T);
   const int nt = min(kPrepTT, T - t0);
   const long long rowbase = (long long)b * T;
+  // every global input of the tile is requested up front (B row piece, x
+  // piece, and for the first warp its token's dt_raw and the head's constants),
+  // so their latencies overlap
+  const int tt8 = tid >> 3, k8 = tid & 7;  // 8 threads per token
+  uint4 bpiece = make_uint4(0u, 0u, 0u, 0u);
+  uint2 xpiece = make_uint2(0u, 0u);
+  if (tt8 < nt) {
+    const int8_t *rowp = a.xbc + (rowbase + t0 + tt8) * a.cc;
+    bpiece = *reinterpret_cast<const uint4 *>(rowp + a.di + k8 * 16);
+    xpiece = *reinterpret_cast<const uint2 *>(rowp + (long long)h * hd + k8 * 8);
+  }
+  float dtr = 0.0f, dtb = 0.0f;
+  int aq = 0;
+  if (tid < nt) {
+    dtr = a.dt_raw[(rowbase + t0 + tid) * nh + h];
+    dtb = a.dt_bias[h];
+    aq = a.A_q[h];
+  }
   __shared__ int s_bmax[kPrepTT];
   {  // max |B[n]| of each token (0 past the end): 8 threads x 16 bytes per token
-    const int tt = tid >> 3, k = tid & 7;
+    const int tt = tt8, k = k8;
     int m = 0;
     if (tt < nt) {
-      const uint4 v = *reinterpret_cast<const uint4 *>(a.xbc + (rowbase + t0 + tt) * a.cc + a.di + k * 16);
+      const uint4 v = bpiece;
       const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
       for (int q = 0; q < 4; ++q)
@@ -101,9 +119,9 @@ __global__ void __launch_bounds__(256) k_scan_prep(ScanPrepArgs a) {
   if (tid < kPrepTT) {
     int dtq = 0, dA = 0;
     if (tid < nt) {
-      const float xf = __fadd_rn(a.dt_raw[(rowbase + t0 + tid) * nh + h], a.dt_bias[h]);
+      const float xf = __fadd_rn(dtr, dtb);
       dtq = softplus_pwl(to_q16(xf));
-      dA = pow2_pwl(-rshr64((long long)dtq * a.A_q[h], 12));
+      dA = pow2_pwl(-rshr64((long long)dtq * aq, 12));
     }
     s_dtq[tid] = dtq;
     a.dA[((long long)b * nh + h) * Tp + t0 + tid] = dA;
@@ -119,13 +137,8 @@ __global__ void __launch_bounds__(256) k_scan_prep(ScanPrepArgs a) {
       a.osh[((long long)b * nh + h) * Tp + t0 + tid] = o;
     }
   }
-  {  // x tile: 32 tokens x 64 channels, 8 bytes per thread
-    const int tt = tid >> 3, k = tid & 7;
-    uint2 v = make_uint2(0u, 0u);
-    if (tt < nt)
-      v = *reinterpret_cast<const uint2 *>(a.xbc + (rowbase + t0 + tt) * a.cc + (long long)h * hd + k * 8);
-    *reinterpret_cast<uint2 *>(&sx[tt][k * 8]) = v;
-  }
+  // x tile: 32 tokens x 64 channels, 8 bytes per thread (0 past the end)
+  *reinterpret_cast<uint2 *>(&sx[tt8][k8 * 8]) = xpiece;
   __syncthreads();
   {  // (u, x) for channel p = tid / 4, tokens 8 * (tid % 4) .. + 8
     const int p = tid >> 2, tb = (tid & 3) * 8;
@@ -206,7 +219,7 @@ struct ScanSeqSmem {
     int32_t u[PC][TCH];
     int32_t xs[PC][TCH];
     int32_t osh[TCH];
-    long long bound[PC];
+    long long bound[TCH / 16][PC];  // growth bounds of the chunk's 16-step parts
   };
   Slot slot[kScanSlots];
   int2 part[NW][TCH * (32 / LPP)][PSTRIDE];
@@ -333,14 +346,16 @@ __device__ __forceinline__ void scan_chunk_steps(int (&hh)[NPT], unsigned (&hl)[
 // transaction-count barrier.  Compute warps never wait for each other.
 template <int NPT, int PC, int TCH, bool S16 = false, bool TOK = false>
 __global__ void __launch_bounds__(PC *(128 / NPT) + 32) k_scan_seq(ScanSeqArgs a) {
+  // no early trigger: the state this kernel writes at its end may be read by
+  // a next kernel before its own dependency wait (the decode step)
   pdl_wait();
-  pdl_trigger();
   constexpr int LPP = 128 / NPT;
   constexpr int NW = PC * LPP / 32;
   constexpr int PPW = 32 / LPP;  // channels per warp
   static_assert(LPP <= 32 && 32 % LPP == 0, "a channel's threads stay inside one warp");
-  static_assert(TCH == 16, "the growth bounds are per 16-step chunk");
   constexpr bool REDUX = (LPP == 32);
+  static_assert(TCH == 16 || (TCH == 32 && REDUX),
+                "the growth bounds are per 16 steps; 32-step chunks need one channel per warp");
   using Sm = ScanSeqSmem<NPT, PC, TCH>;
   constexpr int PSTRIDE = Sm::PSTRIDE;
   extern __shared__ __align__(16) uint8_t smem_raw[];
@@ -380,10 +395,13 @@ __global__ void __launch_bounds__(PC *(128 / NPT) + 32) k_scan_seq(ScanSeqArgs a
         const int nt = min(TCH, T - t0);
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         mbar_arrive_expect_tx(&sm.full[sl], (uint32_t)(nt * 1024 + TCH * 4 * (1 + 2 * PC) +
-                                                       PC * 8 + (TOK ? TCH * 4 : 0)));
+                                                       (TCH / 16) * PC * 8 + (TOK ? TCH * 4 : 0)));
         if constexpr (TOK) bulk_g2s(&s.osh[0], a.osh + headrow * Tp + t0, TCH * 4, &sm.full[sl]);
-        bulk_g2s(&s.bound[0], a.bound + ((headrow * (Tp / 16) + c) * hd + p0), PC * 8,
-                 &sm.full[sl]);
+#pragma unroll
+        for (int j = 0; j < TCH / 16; ++j)  // Tp is a multiple of 32: every part exists
+          bulk_g2s(&s.bound[j][0],
+                   a.bound + ((headrow * (Tp / 16) + c * (TCH / 16) + j) * hd + p0), PC * 8,
+                   &sm.full[sl]);
         bulk_g2s(&s.bc[0][0], a.bc + (rowbase + t0) * 256, (uint32_t)(nt * 1024), &sm.full[sl]);
         bulk_g2s(&s.dA[0], a.dA + headrow * Tp + t0, TCH * 4, &sm.full[sl]);
 #pragma unroll
@@ -437,7 +455,10 @@ __global__ void __launch_bounds__(PC *(128 / NPT) + 32) k_scan_seq(ScanSeqArgs a
 #pragma unroll
     for (int j = 0; j < NPT; ++j) hmax = max(hmax, abs(hh[j]));
     const long long hbound = S16 ? (long long)hmax : ((long long)hmax + 1) << 16;
-    const bool no_clamp = __all_sync(0xffffffffu, hbound + s.bound[pp] <=
+    long long grow = 0;
+#pragma unroll
+    for (int j = 0; j < TCH / 16; ++j) grow += s.bound[j][pp];
+    const bool no_clamp = __all_sync(0xffffffffu, hbound + grow <=
                                                       (S16 ? (long long)kH16Lim : kHLim));
     int2 pr[TCH];
     int2 *wsum = reinterpret_cast<int2 *>(&part[0][0]);
@@ -520,8 +541,6 @@ constexpr int kStepPPW = 8;  // channels per warp (hd / 8 warps)
 // used.
 template <bool NARROW>
 __global__ void __launch_bounds__(256) k_scan_step(ScanArgs a) {
-  pdl_wait();
-  pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int h = blockIdx.x, b = blockIdx.y;
   const int nh = a.nh, hd = a.hd, cc = a.cc, di = a.di;
@@ -548,6 +567,13 @@ __global__ void __launch_bounds__(256) k_scan_step(ScanArgs a) {
 #pragma unroll
     for (int k = 0; k < kStepPPW; ++k) hv[k] = __ldcs(st + (warp + 8 * k) * 32 + lane);
   }
+  // Under programmatic dependent launch the state loads above overlap the
+  // previous kernel's drain.  They may: of the kernels that write a state,
+  // this one and k_scan_seq issue no early trigger, and k_ssd_pass is always
+  // followed by k_ssd_out, which triggers only after waiting for it -- so every
+  // kernel launched after a state's writer starts once that state is written.
+  // Everything below reads the conv's and in_proj's outputs.
+  pdl_wait();
   const int8_t *row = a.xbc + (long long)b * cc;
   const uint32_t bw = *reinterpret_cast<const uint32_t *>(row + di + n0);
   const uint32_t cw = *reinterpret_cast<const uint32_t *>(row + di + 128 + n0);

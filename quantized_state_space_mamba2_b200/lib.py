@@ -188,8 +188,11 @@ def prepare_linear(W, rotate, Wq, s_w, stream=None):
     _check(load().fm_prepare_linear(_p(W), N, K, rotate, _p(Wq), _p(s_w), _s(stream)))
 
 
+PDL_DEFAULT = True  # fm_set_pdl's default
+
+
 def set_pdl(enable: bool):
-    """Programmatic dependent launch of the hot kernels (off by default)."""
+    """Programmatic dependent launch of the hot kernels (on by default)."""
     _check(load().fm_set_pdl(int(bool(enable))))
 
 
@@ -246,7 +249,7 @@ def conv1d_pot_tok(u, B, T, shape, wq, bq, exps, conv_state, out, e_tok, stream=
                                     _p(conv_state), _p(out), _p(e_tok), _s(stream)))
 
 
-SCAN_TILES = ((4, 4, 16), (4, 2, 16), (4, 8, 16), (8, 4, 16), (8, 2, 16), (8, 8, 16))
+SCAN_TILES = ((4, 4, 16), (4, 2, 16), (4, 8, 16), (8, 4, 16), (8, 2, 16), (8, 8, 16), (4, 4, 32))
 
 
 def set_scan_tile(npt: int, pc: int, tch: int):

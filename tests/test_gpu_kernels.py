@@ -339,7 +339,8 @@ def test_ssm_scan_pot(L, B, T, with_state):
     _run_scan(L, MAMBA130, B, T, with_state, 60 + T)
 
 
-@pytest.mark.parametrize("tile", [(4, 2, 16), (4, 8, 16), (8, 4, 16), (8, 2, 16), (8, 8, 16)])
+@pytest.mark.parametrize("tile", [(4, 2, 16), (4, 8, 16), (8, 4, 16), (8, 2, 16), (8, 8, 16),
+                                  (4, 4, 32)])
 def test_ssm_scan_tiles(L, tile):
     """Every compiled tile of the sequential kernel computes the same bits
     (ragged chunk tail, carried state, two heads' worth of CTAs per SM)."""
@@ -420,11 +421,21 @@ def test_ssm_scan_skip_term_beyond_int32(L, T):
     assert (big & (np.abs(yr.astype(np.int64)) < 2 ** 31 - 1)).sum() > 0
 
 
+@pytest.mark.parametrize("tile", [(4, 4, 16), (4, 4, 32)])
 @pytest.mark.parametrize("regime", ["saturating", "small"])
-def test_ssm_scan_clamp_regimes(L, regime):
+def test_ssm_scan_clamp_regimes(L, regime, tile):
     """The sequential kernel skips the clamp for a chunk only when
     max|h| + sum |u| max|B| stays below it; both regimes must match the oracle:
-    a state driven into the +-(2^30 - 1) clamp, and one that never nears it."""
+    a state driven into the +-(2^30 - 1) clamp, and one that never nears it
+    (16- and 32-step chunks: the latter add two 16-step bounds)."""
+    L.set_scan_tile(*tile)
+    try:
+        _clamp_regime(L, regime)
+    finally:
+        L.set_scan_tile(4, 4, 16)
+
+
+def _clamp_regime(L, regime):
     s = MAMBA130
     B, T = 1, 160
     xbc, dt_raw, dt_bias, A_q, D_q, e_D, e_x, e_B, e_C, e_h, e_y = _scan_case(s, B, T, 90)
