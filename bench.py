@@ -109,6 +109,9 @@ def parse(argv=None):
                     help="tile width of the persistent GEMM (0: chosen by the grid)")
     ap.add_argument("--lq-cpw", type=int, default=0, choices=[0, 1, 2, 4],
                     help="channels per warp of the LQ scan (0: chosen by the grid)")
+    ap.add_argument("--gemm-cluster", default="on", choices=["on", "off"],
+                    help="decode-size GEMMs with fewer tiles than SMs split K over a "
+                         "thread-block cluster (on: the library's default)")
     ap.add_argument("--pdl", default="on", choices=["on", "off"],
                     help="programmatic dependent launch of the library's kernels (on: the "
                          "library's default)")
@@ -955,6 +958,7 @@ def apply_modes(args, lib):
     lib.set_state_spec(*[int(v) for v in args.state_spec.split(",")])
     lib.set_gemm_tile(args.gemm_tile)
     lib.set_pdl(getattr(args, "pdl", "on") == "on")
+    lib.set_gemm_cluster(getattr(args, "gemm_cluster", "on") == "on")
     lib.set_lq_scan_cpw(getattr(args, "lq_cpw", 0))
     lib.set_xbc_exponents(args.xbc_exponents)
 

@@ -200,6 +200,16 @@ size_t fm_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
  * partial sums), 1 splits small grids.  Set it before sizing workspaces and
  * keep it while they are in use.  FM_ERR_INVALID_ARG for other values. */
 fm_status fm_set_gemm_splitk(int enable);
+/* Process-wide: 1 (default) runs a decode-size GEMM (M <= 64) whose 32-wide
+ * output tiles are fewer than the SMs with K split over the 2..8 CTAs of a
+ * thread-block cluster -- each CTA accumulates its slice's exact int32 partial
+ * sums, rank 0 adds the others' through distributed shared memory and runs
+ * the same epilogue, so the outputs are bit-identical; no workspace.  0 runs
+ * one CTA per tile.  Not used while fm_set_gemm_splitk(1) splits through a
+ * workspace.  FM_ERR_INVALID_ARG for other values.
+ * Source: the W8A8 linear of the pith.science review of FastMamba, "What
+ * carries the argument" (the split only changes the int32 summation order). */
+fm_status fm_set_gemm_cluster(int enable);
 fm_status fm_w8a8_gemm_ws(const int8_t *A, const float *s_x, int64_t M, const int8_t *Wq,
                           const float *s_w, int64_t N, int64_t K, const float *residual,
                           float *Y, int32_t *acc_out, void *ws, size_t ws_bytes,

@@ -346,6 +346,59 @@ static fm_status launch_gemm_t(const CUtensorMap &ta, const CUtensorMap &tb, lon
   return FM_OK;
 }
 
+// Split K over a thread-block cluster (k_gemm_i8_cl), for a decode batch
+// whose 32-wide tiles are fewer than the SMs: S ranks per tile, chosen so that
+// the grid covers about two CTAs per SM and every rank gets a K block.
+// Process-wide, on by default; fm_set_gemm_cluster(0) keeps the one-CTA-per-tile
+// kernel.
+static std::atomic<int> g_gemm_cluster{1};
+
+extern "C" fm_status fm_set_gemm_cluster(int enable) {
+  if (enable != 0 && enable != 1)
+    return fail(FM_ERR_INVALID_ARG, "fm_set_gemm_cluster: %d is not 0 or 1", enable);
+  g_gemm_cluster.store(enable, std::memory_order_relaxed);
+  return FM_OK;
+}
+
+static int gemm_cluster_ranks(long long N, long long K, int sms) {
+  const long long tiles = (N + 31) / 32, nkb = K / kGemmBK;
+  int S = (int)((2LL * sms + tiles - 1) / tiles);
+  if (S > 8) S = 8;
+  while (S >= 2 && (long long)(S - 1) * ((nkb + S - 1) / S) >= nkb) --S;
+  return S;
+}
+
+template <int S>
+static fm_status launch_gemm_cl_t(const CUtensorMap &ta, const CUtensorMap &tb, long long N,
+                                  long long K, const GemmEpilogue &ep, cudaStream_t s) {
+  constexpr int BN = 32, STAGES = 4;
+  constexpr int smem = gemm_cl_smem_bytes(BN, STAGES);
+  static_assert(smem <= 75 * 1024, "three cluster CTAs per SM");
+  auto kern = k_gemm_i8_cl<BN, STAGES, S>;
+  FM_CHECK_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+  const int nkb = (int)(K / kGemmBK);
+  const int per = (nkb + S - 1) / S;
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3((unsigned)((N + BN - 1) / BN), 1, S);
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = S;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = g_pdl.load(std::memory_order_relaxed) ? 2 : 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ta, tb, nkb, per, ep);
+  if (e != cudaSuccess)
+    return fail(FM_ERR_CUDA, "launch of k_gemm_i8_cl: %s", cudaGetErrorString(e));
+  return launched("k_gemm_i8_cl");
+}
+
 template <int BN, int STAGES, int EW>
 static fm_status launch_gemm_persist(const CUtensorMap &ta, const CUtensorMap &tb, long long M,
                                      long long N, long long K, int sms, GemmEpilogue ep,
@@ -424,6 +477,19 @@ static fm_status launch_gemm(const int8_t *A, long long M, const int8_t *W, long
     // stream gets a deeper ring (64 wide: 6 x 16 KB, two CTAs per SM; 32 wide,
     // fewer CTAs than SMs: 16 x 12 KB, one per SM)
     FM_TRY(make_tmap(&ta, A, M, K, 64));
+    if (narrow && g_gemm_cluster.load(std::memory_order_relaxed) &&
+        !(split_ws && g_gemm_splitk.load(std::memory_order_relaxed))) {
+      switch (gemm_cluster_ranks(N, K, sms)) {
+        case 2: return launch_gemm_cl_t<2>(ta, tb, N, K, ep, s);
+        case 3: return launch_gemm_cl_t<3>(ta, tb, N, K, ep, s);
+        case 4: return launch_gemm_cl_t<4>(ta, tb, N, K, ep, s);
+        case 5: return launch_gemm_cl_t<5>(ta, tb, N, K, ep, s);
+        case 6: return launch_gemm_cl_t<6>(ta, tb, N, K, ep, s);
+        case 7: return launch_gemm_cl_t<7>(ta, tb, N, K, ep, s);
+        case 8: return launch_gemm_cl_t<8>(ta, tb, N, K, ep, s);
+        default: break;  // too few K blocks to split
+      }
+    }
     if (narrow) return launch_gemm_t<32, 16, 64>(ta, tb, M, N, K, ep, split_ws, s);
     return launch_gemm_t<64, 6, 64>(ta, tb, M, N, K, ep, split_ws, s);
   }

@@ -52,7 +52,7 @@ __device__ __forceinline__ void conv_transpose4(uint32_t r0, uint32_t r1, uint32
 // 256 channels), so the group maximum is a shuffle reduction.
 // CALIB: amax is non-null (calibration); otherwise it is not read.
 // The common case takes a short path: when none of the thread's 4 channels
-// can saturate x16 (|b| + 4 127^2, shifted to Q.16, stays inside int32) nor
+// can saturate x16 (|b| + 4 128^2, shifted to Q.16, stays inside int32) nor
 // overflow the output's rounding add, x16 = (dp4a(taps, w, b + rounding bias)
 // >> right) << left and the output code is a plain add-and-shift, both exact;
 // any other thread runs the general 64-bit form.
@@ -115,8 +115,9 @@ __global__ void __launch_bounds__(kConvQuads *TG) k_conv1d_pot(
     lsh[j] = si > 0 ? 0 : -si;
     cb[j] = ok ? bs[j] + (si > 0 ? 1 << (si - 1) : 0) : 0;
     rob[j] = ok ? 1 << (so - 1) : 0;
-    // |x16| bound: |acc| <= |b| + 4 127^2 (+ the rounding bias), then shifted
-    const long long ab = (long long)(bs[j] < 0 ? -(long long)bs[j] : bs[j]) + 64516 +
+    // |x16| bound: |acc| <= |b| + 4 128^2 (any int8 codes and weights, + the
+    // rounding bias), then shifted
+    const long long ab = (long long)(bs[j] < 0 ? -(long long)bs[j] : bs[j]) + 65536 +
                          (si > 0 && si < 62 ? (1LL << (si - 1)) : 0);
     const long long xb = ok ? (si > 0 ? (ab >> si) + 1 : ab << lsh[j]) : (1LL << 40);
     // |SiLU(x16)| <= |x16|, so the output's rounding add cannot overflow either

@@ -486,6 +486,212 @@ __global__ void __launch_bounds__(kGemmThreads, 2)
   }
 }
 
+// ------------------------------------------------------------ split K in a cluster
+// A decode batch (M <= 64) whose output tiles are fewer than the SMs (the
+// out_proj): each tile's K is split over the S CTAs of a thread-block cluster
+// (cluster dims (1, 1, S), rank = the K slice), so every SM streams a share of
+// the weights and of the activations.  Each CTA accumulates its slice's exact
+// int32 partial sums in TMEM; ranks 1..S-1 copy theirs to their own shared
+// memory, and after a cluster barrier rank 0 adds them (distributed shared
+// memory loads) to its own and runs the unchanged epilogue, so the outputs
+// are bit-identical to the unsplit kernel.  A second cluster barrier keeps
+// every CTA's shared memory alive until rank 0 has read it.  Every thread of
+// every CTA reaches both barriers: the kernel has no early exit and all its
+// waits are bounded.  Plain TMA loads only (no multicast).
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t dsmem_map(uint32_t local, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ uint4 dsmem_ld4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared::cluster.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+
+constexpr int kClPad = 4;  // int32 words of padding per partial-sum row
+__host__ __device__ constexpr int gemm_cl_smem_bytes(int BN, int stages) {
+  return stages * (64 + BN) * kGemmBK + kGemmBM * (BN + kClPad) * 4 + 1024 /*align slack*/ +
+         256 /*barriers*/ + 2 * BN * 4 /*staged column scales*/;
+}
+
+// grid (ceil(N / BN), 1, S), cluster (1, 1, S), kGemmThreads threads; the
+// host gives every rank at least one K block (kb_per_rank * (S - 1) < nkb)
+template <int BN, int STAGES, int S>
+__global__ void __launch_bounds__(kGemmThreads)
+    k_gemm_i8_cl(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                 int num_k_blocks, int kb_per_rank, GemmEpilogue ep) {
+  static_assert(BN % 32 == 0 && BN >= 32 && BN <= 128, "BN");
+  static_assert(STAGES * BN >= 64, "a 64-row A stage reads 64 more rows, inside the ring");
+  static_assert(S >= 2 && S <= 8, "portable cluster sizes");
+  constexpr int AR = 64;
+  constexpr int PSTR = BN + kClPad;  // partial-sum row stride (int32 words)
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~static_cast<uintptr_t>(1023));
+  uint8_t *sA = smem;
+  uint8_t *sB = smem + STAGES * AR * kGemmBK;
+  int32_t *part = reinterpret_cast<int32_t *>(sB + STAGES * BN * kGemmBK);  // [128][PSTR]
+  uint64_t *full_bar = reinterpret_cast<uint64_t *>(part + kGemmBM * PSTR);
+  uint64_t *empty_bar = full_bar + STAGES;
+  uint64_t *accum_bar = empty_bar + STAGES;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(accum_bar + 1);
+  float *col_w = reinterpret_cast<float *>((reinterpret_cast<uintptr_t>(tmem_slot + 1) + 15) &
+                                           ~static_cast<uintptr_t>(15));
+  float *col_e = col_w + BN;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int n0 = blockIdx.x * BN;
+  const uint32_t rank = cluster_rank();
+  const int kb0 = (int)rank * kb_per_rank;
+  const int kb_n = max(0, min(kb_per_rank, num_k_blocks - kb0));
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    mbar_init(accum_bar, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"((unsigned long long)&tmA) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"((unsigned long long)&tmB) : "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"((uint32_t)BN)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  pdl_trigger();
+
+  bool ok = true;  // this thread's accumulator wait (epilogue warps)
+  if (warp == 0) {
+    if (lane == 0) {
+      const int kb_issue = (g_test_stall & kStallGemm) ? 0 : kb_n;
+      const int pre = kb_issue < STAGES ? kb_issue : STAGES;
+      for (int kb = 0; kb < pre; ++kb) {  // fresh ring: no empty-slot wait
+        mbar_arrive_expect_tx(&full_bar[kb], (uint32_t)((AR + BN) * kGemmBK));
+        tma_load_2d(sB + kb * BN * kGemmBK, &tmB, (kb0 + kb) * kGemmBK, n0, &full_bar[kb]);
+      }
+      pdl_wait();
+      for (int kb = 0; kb < pre; ++kb)
+        tma_load_2d(sA + kb * AR * kGemmBK, &tmA, (kb0 + kb) * kGemmBK, 0, &full_bar[kb]);
+      int issued = pre;
+      for (int kb = pre; kb < kb_issue; ++kb) {
+        const int s = kb % STAGES;
+        const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
+        if (!mbar_wait(&empty_bar[s], ph ^ 1u)) break;
+        mbar_arrive_expect_tx(&full_bar[s], (uint32_t)((AR + BN) * kGemmBK));
+        tma_load_2d(sA + s * AR * kGemmBK, &tmA, (kb0 + kb) * kGemmBK, 0, &full_bar[s]);
+        tma_load_2d(sB + s * BN * kGemmBK, &tmB, (kb0 + kb) * kGemmBK, n0, &full_bar[s]);
+        ++issued;
+      }
+      for (int j = issued > STAGES ? issued - STAGES : 0; j < issued; ++j)
+        if (!mbar_drain(&full_bar[j % STAGES], (uint32_t)(j / STAGES) & 1u)) break;
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = i8_idesc(kGemmBM, BN);
+      for (int kb = 0; kb < kb_n; ++kb) {
+        const int s = kb % STAGES;
+        const uint32_t ph = (uint32_t)(kb / STAGES) & 1u;
+        if (!mbar_wait(&full_bar[s], ph)) break;
+        tc_fence_after();
+        const uint64_t ad = sw128_desc(smem_u32(sA + s * AR * kGemmBK));
+        const uint64_t bd = sw128_desc(smem_u32(sB + s * BN * kGemmBK));
+#pragma unroll
+        for (int k = 0; k < kGemmBK / 32; ++k)
+          mma_i8(tmem_base, ad + (uint64_t)(2 * k), bd + (uint64_t)(2 * k), idesc,
+                 (kb > 0 || k > 0) ? 1u : 0u);
+        mma_commit(&empty_bar[s]);
+      }
+      mma_commit(accum_bar);
+      mbar_drain(accum_bar, 0);
+    }
+  } else {
+    pdl_wait();
+    const int et = threadIdx.x - 64;  // 0 .. 127
+    if (rank == 0) {  // the tile's column scales (used after the first cluster barrier)
+      for (int j = et; j < BN; j += 128) {
+        const long long c = (long long)n0 + j;
+        col_w[j] = c < ep.N ? ep.s_w[c] : 0.0f;
+        float e = 0.0f;
+        if (ep.mode == 1 && c >= ep.di && c < (long long)ep.di + ep.cc) e = pow2f(-ep.e_u[c - ep.di]);
+        col_e[j] = e;
+      }
+    }
+    ok = __all_sync(0xffffffffu, mbar_wait_sleepy(accum_bar, 0));
+    tc_fence_after();
+    if (rank != 0) {  // this slice's partial sums into shared memory, row by row
+      const int quarter = warp & 3;
+      const int row = quarter * 32 + lane;
+#pragma unroll 1
+      for (int c = 0; c < BN; c += 32) {
+        uint32_t r[32];
+        if (ok) tmem_ld32(tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)c, r);
+#pragma unroll
+        for (int j = 0; j < 32; j += 4)
+          *reinterpret_cast<uint4 *>(part + row * PSTR + c + j) =
+              ok ? make_uint4(r[j], r[j + 1], r[j + 2], r[j + 3]) : make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+  }
+  tc_fence_before();
+  cluster_sync_all();  // every slice's partial sums written and visible
+  tc_fence_after();
+  if (rank == 0 && warp >= 2 && ok) {
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const float sx = row < ep.M ? ep.s_x[row] : 0.0f;
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 32) {
+      uint32_t r[32];
+      tmem_ld32(tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)c, r);
+      if (n0 + c >= ep.N) continue;
+      const uint32_t local = smem_u32(part + row * PSTR + c);
+#pragma unroll 1
+      for (int q = 1; q < S; ++q) {  // exact int32 sums, any order
+        const uint32_t remote = dsmem_map(local, (uint32_t)q);
+#pragma unroll
+        for (int j = 0; j < 32; j += 4) {
+          const uint4 v = dsmem_ld4(remote + 4u * (uint32_t)j);
+          r[j] += v.x;
+          r[j + 1] += v.y;
+          r[j + 2] += v.z;
+          r[j + 3] += v.w;
+        }
+      }
+      gemm_store_chunk(ep, row, sx, (long long)n0 + c, r, col_w + c, col_e + c);
+    }
+  }
+  cluster_sync_all();  // rank 0 has read every slice: the CTAs may leave
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"((uint32_t)BN)
+                 : "memory");
+  }
+}
+
 // The dequantising epilogue of a split-K GEMM: one thread per (row, 32-column
 // chunk) reads the exact int32 totals and runs the same gemm_store_chunk as
 // the unsplit kernels, so the outputs are bit-identical to theirs.

@@ -32,7 +32,7 @@ EXPORTS = (
     "fm_set_state_spec", "fm_lq_conv1d", "fm_lq_scan", "fm_lq_workspace_bytes",
     "fm_lq_mixer_prefill", "fm_set_fault_injection", "fm_set_gemm_splitk",
     "fm_set_gemm_tile", "fm_set_xbc_exponents", "fm_conv1d_pot_tok", "fm_ssm_scan_pot_tok",
-    "fm_scan_workspace_bytes_tok", "fm_set_pdl", "fm_set_lq_scan_cpw",
+    "fm_scan_workspace_bytes_tok", "fm_set_pdl", "fm_set_lq_scan_cpw", "fm_set_gemm_cluster",
 )
 NOALLOC_SCRATCH_BYTES = 16 << 20  # FM_NOALLOC_SCRATCH_BYTES
 
@@ -119,6 +119,7 @@ def load():
         "fm_set_gemm_splitk": (I, [I]),
         "fm_set_gemm_tile": (I, [I]),
         "fm_set_pdl": (I, [I]),
+        "fm_set_gemm_cluster": (I, [I]),
         "fm_set_lq_scan_cpw": (I, [I]),
         "fm_set_xbc_exponents": (I, [I]),
         "fm_conv1d_pot_tok": (I, [_P, I, I, sp, _P, _P, _P, _P, _P, _P, _P]),
@@ -194,6 +195,12 @@ PDL_DEFAULT = True  # fm_set_pdl's default
 def set_pdl(enable: bool):
     """Programmatic dependent launch of the hot kernels (on by default)."""
     _check(load().fm_set_pdl(int(bool(enable))))
+
+
+def set_gemm_cluster(enable: bool):
+    """Split K over a thread-block cluster for decode-size GEMMs with fewer
+    tiles than SMs (on by default; the same bits either way)."""
+    _check(load().fm_set_gemm_cluster(int(bool(enable))))
 
 
 def set_gemm_tile(bn: int):

@@ -68,6 +68,8 @@ def test_exp_layout_and_workspace(so):
     finally:
         lib.set_gemm_splitk(False)
     assert so.fm_set_gemm_splitk(2) == 1
+    assert so.fm_set_gemm_cluster(2) == 1 and so.fm_set_gemm_cluster(-1) == 1
+    assert so.fm_set_gemm_cluster(0) == 0 and so.fm_set_gemm_cluster(1) == 0
     assert lib.calib_workspace_bytes(s, 16, 512) > lib.workspace_bytes(s, 16, 512)
     # a single decode step stages nothing for the scan
     assert lib.scan_workspace_bytes(s, 64, 1) == 256

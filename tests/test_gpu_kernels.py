@@ -130,6 +130,40 @@ def test_w8a8_gemm(L, M, N, K):
     L.sync_status()
 
 
+@pytest.mark.parametrize("M,N,K", [(64, 2560, 5120), (1, 768, 1536), (37, 100, 1152),
+                                   (16, 1000, 256)])
+def test_w8a8_gemm_cluster_split(L, M, N, K):
+    """Decode-size GEMMs with fewer 32-wide tiles than SMs, K split over a
+    thread-block cluster (2..8 ranks, the last rank's slice ragged where K
+    does not divide): the int32 accumulator, the dequantised output and the
+    residual form are bit-identical to one CTA per tile and to the exact
+    product."""
+    A = S.uniform_ints((M, K), -127, 127, seed=M * 3 + K + 1, dtype=np.int8)
+    W = S.uniform_ints((N, K), -127, 127, seed=N * 5 + K + 1, dtype=np.int8)
+    sx = np.abs(S.normal(M, 0.01, seed=11)) + 1e-3
+    sw = np.abs(S.normal(N, 0.001, seed=12)) + 1e-4
+    res = S.normal((M, N), 1.0, seed=13)
+    ref = A.astype(np.int64) @ W.astype(np.int64).T
+    outs = []
+    for on in (True, False):
+        L.set_gemm_cluster(on)
+        try:
+            Y = torch.empty((M, N), dtype=torch.float32, device="cuda")
+            acc = torch.empty((M, N), dtype=torch.int32, device="cuda")
+            L.w8a8_gemm(dev(A), dev(sx), dev(W), dev(sw), Y, None, acc)
+            Yr = dev(res)
+            L.w8a8_gemm(dev(A), dev(sx), dev(W), dev(sw), Yr, Yr, None)
+            L.sync_status()
+            outs.append((host(acc), host(Y), host(Yr)))
+        finally:
+            L.set_gemm_cluster(True)
+    (a1, y1, r1), (a0, y0, r0) = outs
+    assert np.array_equal(a1, ref) and np.array_equal(a0, ref)
+    assert np.array_equal(y1, y0) and np.array_equal(r1, r0)
+    assert np.array_equal(y1, O.dequant(ref.astype(np.int32), sx, sw))
+    assert np.array_equal(r1, O.dequant(ref.astype(np.int32), sx, sw, residual=res))
+
+
 def _sample_rows(M, step=7, tail=130):
     return np.unique(np.concatenate([np.arange(0, M, step), np.arange(max(0, M - tail), M)]))
 
