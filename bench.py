@@ -67,14 +67,6 @@ CPU_ALLCORE_TOKENS = 512
 # captures of the current kernels (profiles/dram_traffic_roofline_kernels.md);
 # None where no capture of the kernel in that configuration exists.
 DRAM_TRAFFIC = {
-    # 130M stack, B 1, T 2048, static exponents, the int32 state: k_scan_prep
-    # 3,884,544 + 256 and k_scan_seq 29,099,264 + 0
-    ("fm_ssm_scan_pot (k_scan_prep + k_scan_seq)", "stack130m_24l_b1_t2048", "31,0", "static"):
-        32984064,
-    # 2.7B decode, B 64: k_scan_step 168,167,424 + 108,474,880
-    ("fm_ssm_scan_pot, T = 1 (k_scan_step)", "decode2p7b_64l_b64", "31,0", "static"): 276642304,
-    # in_proj GEMM at M = 32768: 253,903,616 + 1,340,978,944
-    ("fm_w8a8_gemm (k_gemm_i8_persist, tcgen05 kind::i8)", "gemm2p7b_inproj", 32768): 1594882560,
 }
 
 
@@ -109,9 +101,9 @@ def parse(argv=None):
                     help="tile width of the persistent GEMM (0: chosen by the grid)")
     ap.add_argument("--lq-cpw", type=int, default=0, choices=[0, 1, 2, 4],
                     help="channels per warp of the LQ scan (0: chosen by the grid)")
-    ap.add_argument("--gemm-cluster", default="on", choices=["on", "off"],
+    ap.add_argument("--gemm-cluster", default="off", choices=["on", "off"],
                     help="decode-size GEMMs with fewer tiles than SMs split K over a "
-                         "thread-block cluster (on: the library's default)")
+                         "thread-block cluster (off: the library's default)")
     ap.add_argument("--pdl", default="on", choices=["on", "off"],
                     help="programmatic dependent launch of the library's kernels (on: the "
                          "library's default)")
@@ -198,7 +190,7 @@ def config_block(args) -> dict:
                  calibration=f"{S.CALIB_SEQS} seeded sequences x "
                              f"{min(w.get('prefill_len', w['seqlen']), S.CALIB_MAX_LEN)} tokens "
                              "(GPU, stage by stage)",
-                 scan_tile=args.scan_tile or "4,4,16", scan_mode=args.scan_mode,
+                 scan_tile=args.scan_tile or "4,4,32", scan_mode=args.scan_mode,
                  state_spec=args.state_spec,
                  xbc_exponents=getattr(args, "xbc_exponents", "static"))
         if getattr(args, "lq", False):
@@ -958,7 +950,7 @@ def apply_modes(args, lib):
     lib.set_state_spec(*[int(v) for v in args.state_spec.split(",")])
     lib.set_gemm_tile(args.gemm_tile)
     lib.set_pdl(getattr(args, "pdl", "on") == "on")
-    lib.set_gemm_cluster(getattr(args, "gemm_cluster", "on") == "on")
+    lib.set_gemm_cluster(getattr(args, "gemm_cluster", "off") == "on")
     lib.set_lq_scan_cpw(getattr(args, "lq_cpw", 0))
     lib.set_xbc_exponents(args.xbc_exponents)
 

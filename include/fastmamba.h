@@ -200,13 +200,14 @@ size_t fm_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
  * partial sums), 1 splits small grids.  Set it before sizing workspaces and
  * keep it while they are in use.  FM_ERR_INVALID_ARG for other values. */
 fm_status fm_set_gemm_splitk(int enable);
-/* Process-wide: 1 (default) runs a decode-size GEMM (M <= 64) whose 32-wide
- * output tiles are fewer than the SMs with K split over the 2..8 CTAs of a
+/* Process-wide: 1 runs a decode-size GEMM (M <= 64) whose 32-wide output
+ * tiles are fewer than the SMs with K split over the 2..8 CTAs of a
  * thread-block cluster -- each CTA accumulates its slice's exact int32 partial
  * sums, rank 0 adds the others' through distributed shared memory and runs
- * the same epilogue, so the outputs are bit-identical; no workspace.  0 runs
- * one CTA per tile.  Not used while fm_set_gemm_splitk(1) splits through a
- * workspace.  FM_ERR_INVALID_ARG for other values.
+ * the same epilogue, so the outputs are bit-identical; no workspace.  0
+ * (default; measured faster) runs one CTA per tile.  Not used while
+ * fm_set_gemm_splitk(1) splits through a workspace.  FM_ERR_INVALID_ARG for
+ * other values.
  * Source: the W8A8 linear of the pith.science review of FastMamba, "What
  * carries the argument" (the split only changes the int32 summation order). */
 fm_status fm_set_gemm_cluster(int enable);
@@ -248,8 +249,8 @@ fm_status fm_conv1d_pot_tok(const int8_t *u, int B, int T, const fm_shape *shape
 /* ------------------------------------------------------------------ */
 /* Tuning: selects the tile of the sequential scan kernel used by every later
  * call in this process -- npt state columns per thread, pc channels per CTA,
- * tch time steps per staged chunk.  Compiled variants: (4,4,16) (default),
- * (4,2,16), (4,8,16), (8,4,16), (8,2,16), (8,8,16), (4,4,32);
+ * tch time steps per staged chunk.  Compiled variants: (4,4,32) (default),
+ * (4,4,16), (4,2,16), (4,8,16), (8,4,16), (8,2,16), (8,8,16);
  * anything else returns FM_ERR_INVALID_ARG.  All variants compute the same
  * bits. */
 fm_status fm_set_scan_tile(int npt, int pc, int tch);

@@ -349,9 +349,9 @@ static fm_status launch_gemm_t(const CUtensorMap &ta, const CUtensorMap &tb, lon
 // Split K over a thread-block cluster (k_gemm_i8_cl), for a decode batch
 // whose 32-wide tiles are fewer than the SMs: S ranks per tile, chosen so that
 // the grid covers about two CTAs per SM and every rank gets a K block.
-// Process-wide, on by default; fm_set_gemm_cluster(0) keeps the one-CTA-per-tile
-// kernel.
-static std::atomic<int> g_gemm_cluster{1};
+// Process-wide, off by default: measured slower on the 2.7B decode out_proj
+// (20.4 against 17.7 us per launch; the step 6.90 against 6.75 ms).
+static std::atomic<int> g_gemm_cluster{0};
 
 extern "C" fm_status fm_set_gemm_cluster(int enable) {
   if (enable != 0 && enable != 1)
@@ -622,8 +622,12 @@ static fm_status launch_scan(const ScanArgs &a, int B, cudaStream_t s) {
 struct ScanTile {
   int npt, pc, tch;
 };
-static const ScanTile kScanTiles[] = {{4, 4, 16}, {4, 2, 16}, {4, 8, 16},
-                                      {8, 4, 16}, {8, 2, 16}, {8, 8, 16}, {4, 4, 32}};
+// (4, 4, 32) first: the default (measured against (4, 4, 16): 130M stack
+// 7.10 -> 6.74 ms per step, 2.7B stack 195.4 -> 191.7 ms -- the per-chunk
+// work, the growth-bound test and the output epilogue, is spread over twice
+// the steps, and the epilogue uses all 32 lanes)
+static const ScanTile kScanTiles[] = {{4, 4, 32}, {4, 4, 16}, {4, 2, 16}, {4, 8, 16},
+                                      {8, 4, 16}, {8, 2, 16}, {8, 8, 16}};
 static std::atomic<int> g_scan_tile{0};
 // 0: the sequential fixed-point scan (the method); 1: the chunked scan mode for
 // prefills of more than one token (single steps stay sequential)

@@ -197,9 +197,12 @@ def set_pdl(enable: bool):
     _check(load().fm_set_pdl(int(bool(enable))))
 
 
+GEMM_CLUSTER_DEFAULT = False
+
+
 def set_gemm_cluster(enable: bool):
     """Split K over a thread-block cluster for decode-size GEMMs with fewer
-    tiles than SMs (on by default; the same bits either way)."""
+    tiles than SMs (off by default: measured slower; the same bits either way)."""
     _check(load().fm_set_gemm_cluster(int(bool(enable))))
 
 
@@ -256,7 +259,8 @@ def conv1d_pot_tok(u, B, T, shape, wq, bq, exps, conv_state, out, e_tok, stream=
                                     _p(conv_state), _p(out), _p(e_tok), _s(stream)))
 
 
-SCAN_TILES = ((4, 4, 16), (4, 2, 16), (4, 8, 16), (8, 4, 16), (8, 2, 16), (8, 8, 16), (4, 4, 32))
+SCAN_TILES = ((4, 4, 32), (4, 4, 16), (4, 2, 16), (4, 8, 16), (8, 4, 16), (8, 2, 16), (8, 8, 16))
+SCAN_TILE_DEFAULT = (4, 4, 32)
 
 
 def set_scan_tile(npt: int, pc: int, tch: int):
