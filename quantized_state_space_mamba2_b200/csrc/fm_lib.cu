@@ -627,7 +627,7 @@ struct ScanTile {
 // work, the growth-bound test and the output epilogue, is spread over twice
 // the steps, and the epilogue uses all 32 lanes)
 static const ScanTile kScanTiles[] = {{4, 4, 32}, {4, 4, 16}, {4, 2, 16}, {4, 8, 16},
-                                      {8, 4, 16}, {8, 2, 16}, {8, 8, 16}};
+                                      {8, 4, 16}, {8, 2, 16}, {8, 8, 16}, {4, 8, 32}};
 static std::atomic<int> g_scan_tile{0};
 // 0: the sequential fixed-point scan (the method); 1: the chunked scan mode for
 // prefills of more than one token (single steps stay sequential)
@@ -751,6 +751,7 @@ static fm_status launch_scan_v2(const ScanArgs &a, int B, const ScanWs &w, cudaS
   FM_SEQ(8, 2, 16)
   FM_SEQ(8, 8, 16)
   FM_SEQ(4, 4, 32)
+  FM_SEQ(4, 8, 32)
 #undef FM_SEQ
   return fail(FM_ERR_INVALID_ARG, "scan tile (%d, %d, %d) is not compiled", t.npt, t.pc, t.tch);
 }

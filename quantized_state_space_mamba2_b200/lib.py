@@ -259,7 +259,8 @@ def conv1d_pot_tok(u, B, T, shape, wq, bq, exps, conv_state, out, e_tok, stream=
                                     _p(conv_state), _p(out), _p(e_tok), _s(stream)))
 
 
-SCAN_TILES = ((4, 4, 32), (4, 4, 16), (4, 2, 16), (4, 8, 16), (8, 4, 16), (8, 2, 16), (8, 8, 16))
+SCAN_TILES = ((4, 4, 32), (4, 4, 16), (4, 2, 16), (4, 8, 16), (8, 4, 16), (8, 2, 16), (8, 8, 16),
+              (4, 8, 32))
 SCAN_TILE_DEFAULT = (4, 4, 32)
 
 

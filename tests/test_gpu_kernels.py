@@ -374,7 +374,7 @@ def test_ssm_scan_pot(L, B, T, with_state):
 
 
 @pytest.mark.parametrize("tile", [(4, 4, 16), (4, 2, 16), (4, 8, 16), (8, 4, 16), (8, 2, 16),
-                                  (8, 8, 16)])
+                                  (8, 8, 16), (4, 8, 32)])
 def test_ssm_scan_tiles(L, tile):
     """Every compiled tile of the sequential kernel computes the same bits
     (ragged chunk tail, carried state, two heads' worth of CTAs per SM)."""
