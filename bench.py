@@ -198,7 +198,7 @@ def config_block(args) -> dict:
                  calibration=f"{S.CALIB_SEQS} seeded sequences x "
                              f"{min(w.get('prefill_len', w['seqlen']), S.CALIB_MAX_LEN)} tokens "
                              "(GPU, stage by stage)",
-                 scan_tile=args.scan_tile or "4,4,32", scan_mode=args.scan_mode,
+                 scan_tile=args.scan_tile or "4,auto,32", scan_mode=args.scan_mode,
                  state_spec=args.state_spec,
                  xbc_exponents=getattr(args, "xbc_exponents", "static"))
         if getattr(args, "lq", False):

@@ -249,8 +249,10 @@ fm_status fm_conv1d_pot_tok(const int8_t *u, int B, int T, const fm_shape *shape
 /* ------------------------------------------------------------------ */
 /* Tuning: selects the tile of the sequential scan kernel used by every later
  * call in this process -- npt state columns per thread, pc channels per CTA,
- * tch time steps per staged chunk.  Compiled variants: (4,4,32) (default),
- * (4,4,16), (4,2,16), (4,8,16), (8,4,16), (8,2,16), (8,8,16), (4,8,32);
+ * tch time steps per staged chunk.  Compiled variants: (4,0,32) (default:
+ * pc chosen by the grid -- 8 where there are at least three 8-channel CTAs
+ * per SM, else 4), (4,4,32), (4,8,32), (4,4,16), (4,2,16), (4,8,16),
+ * (8,4,16), (8,2,16), (8,8,16);
  * anything else returns FM_ERR_INVALID_ARG.  All variants compute the same
  * bits. */
 fm_status fm_set_scan_tile(int npt, int pc, int tch);

@@ -622,12 +622,17 @@ static fm_status launch_scan(const ScanArgs &a, int B, cudaStream_t s) {
 struct ScanTile {
   int npt, pc, tch;
 };
-// (4, 4, 32) first: the default (measured against (4, 4, 16): 130M stack
-// 7.10 -> 6.74 ms per step, 2.7B stack 195.4 -> 191.7 ms -- the per-chunk
-// work, the growth-bound test and the output epilogue, is spread over twice
-// the steps, and the epilogue uses all 32 lanes)
-static const ScanTile kScanTiles[] = {{4, 4, 32}, {4, 4, 16}, {4, 2, 16}, {4, 8, 16},
-                                      {8, 4, 16}, {8, 2, 16}, {8, 8, 16}, {4, 8, 32}};
+// (4, 0, 32) first: the default, 32-step chunks with the channels per CTA
+// chosen by the grid (pc = 0): 8 where there are at least three such CTAs per
+// SM, else 4.  Measured: 32-step chunks against 16, 130M stack 7.10 -> 6.74 ms
+// per step, 2.7B stack 195.4 -> 191.7 ms (the per-chunk work -- the barrier
+// wait, the growth-bound test, the slot release, the output epilogue -- is
+// spread over twice the steps, and the epilogue uses all 32 lanes); 8 channels
+// per CTA against 4 at 2.7B 191.7 -> 185.3 ms (twice the warps per SM, B and C
+// staged once for 8 channels), at 130M B = 1 8.02 against 6.76 ms (too few CTAs).
+static const ScanTile kScanTiles[] = {{4, 0, 32}, {4, 4, 32}, {4, 8, 32}, {4, 4, 16},
+                                      {4, 2, 16}, {4, 8, 16}, {8, 4, 16}, {8, 2, 16},
+                                      {8, 8, 16}};
 static std::atomic<int> g_scan_tile{0};
 // 0: the sequential fixed-point scan (the method); 1: the chunked scan mode for
 // prefills of more than one token (single steps stay sequential)
@@ -735,7 +740,8 @@ static fm_status launch_scan_v2(const ScanArgs &a, int B, const ScanWs &w, cudaS
   q.state = a.state;
   q.y = a.y;
   q.osh = p.osh;
-  const ScanTile t = scan_tile();
+  ScanTile t = scan_tile();
+  if (t.pc == 0) t.pc = (long long)B * a.nh * a.hd / 8 >= 3LL * sm_count() ? 8 : 4;
 #define FM_SEQ(N, P, C)                                                          \
   if (t.npt == N && t.pc == P && t.tch == C) {                                   \
     if (q.osh)                                                                   \

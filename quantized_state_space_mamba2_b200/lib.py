@@ -259,9 +259,10 @@ def conv1d_pot_tok(u, B, T, shape, wq, bq, exps, conv_state, out, e_tok, stream=
                                     _p(conv_state), _p(out), _p(e_tok), _s(stream)))
 
 
-SCAN_TILES = ((4, 4, 32), (4, 4, 16), (4, 2, 16), (4, 8, 16), (8, 4, 16), (8, 2, 16), (8, 8, 16),
-              (4, 8, 32))
-SCAN_TILE_DEFAULT = (4, 4, 32)
+# (4, 0, 32): the default, channels per CTA chosen by the grid
+SCAN_TILES = ((4, 0, 32), (4, 4, 32), (4, 8, 32), (4, 4, 16), (4, 2, 16), (4, 8, 16), (8, 4, 16),
+              (8, 2, 16), (8, 8, 16))
+SCAN_TILE_DEFAULT = (4, 0, 32)
 
 
 def set_scan_tile(npt: int, pc: int, tch: int):
