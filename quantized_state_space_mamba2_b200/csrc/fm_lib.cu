@@ -670,7 +670,7 @@ static fm_status launch_seq(const ScanSeqArgs &a, int B, cudaStream_t s) {
 struct ScanWs {
   int32_t *dA;  // [B, nh, Tp]
   int32_t *u;   // [B, nh, hd, Tp]
-  int32_t *xs;  // [B, nh, hd, Tp]: x codes, widened
+  int8_t *xs;   // [B, nh, hd, Tp]: x codes
   int32_t *bc;  // [B*T, 256]
   long long *bound;  // [B, nh, Tp/16, hd]
   int32_t *osh;      // [B, nh, Tp] per-token output shifts (per-token exponents only)
@@ -980,14 +980,15 @@ ScanWs carve_scan(Carver &c, const Dims &d, int B, int T, bool tok) {
   w.osh = nullptr;
   if (T == 1) {  // single steps run k_scan_step, which stages nothing
     w.dA = nullptr;
-    w.u = w.xs = w.bc = nullptr;
+    w.u = w.bc = nullptr;
+    w.xs = nullptr;
     w.bound = nullptr;
     return w;
   }
   const long long Tp = scan_tpad(T), M = (long long)B * T;
   w.dA = c.take<int32_t>((long long)B * d.nh * Tp);
   w.u = c.take<int32_t>((long long)B * d.di * Tp);
-  w.xs = c.take<int32_t>((long long)B * d.di * Tp);
+  w.xs = c.take<int8_t>((long long)B * d.di * Tp);
   w.bc = c.take<int32_t>(M * 256);
   w.bound = c.take<long long>((long long)B * d.di * (Tp / 16));
   if (tok) w.osh = c.take<int32_t>((long long)B * d.nh * Tp);

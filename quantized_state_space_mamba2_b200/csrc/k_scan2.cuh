@@ -49,7 +49,7 @@ struct ScanPrepArgs {
   const int32_t *e_x, *e_B, *e_h, *e_y, *e_D;
   int32_t *dA;   // [B, nh, Tp]
   int32_t *u;    // [B, nh, hd, Tp]
-  int32_t *xs;   // [B, nh, hd, Tp]: the x code, widened
+  int8_t *xs;    // [B, nh, hd, Tp]: the x code
   int32_t *bc;   // [B*T, 256]: B then C, int32
   long long *bound;  // [B, nh, Tp/16, hd]: per 16-step chunk, bound of the increments
   int guard;         // the increment's guard bits (0: the method as built)
@@ -165,8 +165,11 @@ __global__ void __launch_bounds__(256) k_scan_prep(ScanPrepArgs a) {
     const long long off = (((long long)b * nh + h) * hd + p) * Tp + t0 + tb;
     *reinterpret_cast<int4 *>(a.u + off) = make_int4(uv[0], uv[1], uv[2], uv[3]);
     *reinterpret_cast<int4 *>(a.u + off + 4) = make_int4(uv[4], uv[5], uv[6], uv[7]);
-    *reinterpret_cast<int4 *>(a.xs + off) = make_int4(dv[0], dv[1], dv[2], dv[3]);
-    *reinterpret_cast<int4 *>(a.xs + off + 4) = make_int4(dv[4], dv[5], dv[6], dv[7]);
+    *reinterpret_cast<uint2 *>(a.xs + off) =
+        make_uint2((uint32_t)(dv[0] & 0xFF) | ((uint32_t)(dv[1] & 0xFF) << 8) |
+                       ((uint32_t)(dv[2] & 0xFF) << 16) | ((uint32_t)dv[3] << 24),
+                   (uint32_t)(dv[4] & 0xFF) | ((uint32_t)(dv[5] & 0xFF) << 8) |
+                       ((uint32_t)(dv[6] & 0xFF) << 16) | ((uint32_t)dv[7] << 24));
   }
   // widened B and C rows of these tokens: the CTAs of the tile share the work
   for (int i = h * 256 + tid; i < nt * 64; i += nh * 256) {
@@ -182,7 +185,7 @@ __global__ void __launch_bounds__(256) k_scan_prep(ScanPrepArgs a) {
 struct ScanSeqArgs {
   const int32_t *dA;  // [B, nh, Tp]
   const int32_t *u;   // [B, nh, hd, Tp]
-  const int32_t *xs;  // [B, nh, hd, Tp]
+  const int8_t *xs;   // [B, nh, hd, Tp]
   const int32_t *bc;  // [B*T, 256]
   const long long *bound;  // [B, nh, Tp/16, hd]
   int T, nh, hd, di;
@@ -217,7 +220,7 @@ struct ScanSeqSmem {
     int32_t bc[TCH][256];
     int32_t dA[TCH];
     int32_t u[PC][TCH];
-    int32_t xs[PC][TCH];
+    int8_t xs[PC][TCH];
     int32_t osh[TCH];
     long long bound[TCH / 16][PC];  // growth bounds of the chunk's 16-step parts
   };
@@ -394,7 +397,7 @@ __global__ void __launch_bounds__(PC *(128 / NPT) + 32) k_scan_seq(ScanSeqArgs a
         const int t0 = c * TCH;
         const int nt = min(TCH, T - t0);
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        mbar_arrive_expect_tx(&sm.full[sl], (uint32_t)(nt * 1024 + TCH * 4 * (1 + 2 * PC) +
+        mbar_arrive_expect_tx(&sm.full[sl], (uint32_t)(nt * 1024 + TCH * 4 * (1 + PC) + PC * TCH +
                                                        (TCH / 16) * PC * 8 + (TOK ? TCH * 4 : 0)));
         if constexpr (TOK) bulk_g2s(&s.osh[0], a.osh + headrow * Tp + t0, TCH * 4, &sm.full[sl]);
 #pragma unroll
@@ -408,7 +411,7 @@ __global__ void __launch_bounds__(PC *(128 / NPT) + 32) k_scan_seq(ScanSeqArgs a
         for (int q = 0; q < PC; ++q) {
           const long long off = (headrow * hd + p0 + q) * Tp + t0;
           bulk_g2s(&s.u[q][0], a.u + off, TCH * 4, &sm.full[sl]);
-          bulk_g2s(&s.xs[q][0], a.xs + off, TCH * 4, &sm.full[sl]);
+          bulk_g2s(&s.xs[q][0], a.xs + off, TCH, &sm.full[sl]);
         }
         ++issued;
       }

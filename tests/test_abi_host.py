@@ -49,9 +49,10 @@ def test_exp_layout_and_workspace(so):
     assert (L.e_u, L.e_w, L.e_o, L.e_x) == (0, cc, 2 * cc, 3 * cc)
     assert L.e_g == 3 * cc + 4 * nh + 2 and L.size == 3 * cc + 4 * nh + 3
     ws = lib.workspace_bytes(s, 1, 2048)
-    # mixer intermediates + the scan's per-token dt/dA, (u, D x) and widened B, C
+    # mixer intermediates + the scan's per-token dt/dA, u (int32), the x codes
+    # (int8) and widened B, C
     # and the per-16-step growth bounds (8 bytes per channel per 16 tokens)
-    per_tok = (s.d_model + 9 * s.d_inner + 2 * cc + 4 * nh + 8 + (4 * nh + 8 * s.d_inner + 1024)
+    per_tok = (s.d_model + 9 * s.d_inner + 2 * cc + 4 * nh + 8 + (4 * nh + 5 * s.d_inner + 1024)
                + s.d_inner // 2)
     # split-K is off by default: no partial sums
     assert lib.gemm_workspace_bytes(2048, s.d_model, s.d_inner) == 0
