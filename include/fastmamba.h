@@ -34,7 +34,8 @@
  *   - Fixed-point conventions (rshr, satb, Q.16, exponent table) are
  *     described next to fm_exp_layout below.
  *   - No exceptions cross the ABI; no global mutable state except a
- *     per-device device error word and the per-process entry-point cache.
+ *     per-device device error word, the per-process entry-point cache and
+ *     the streams and events fm_stack_prefill keeps per CUDA context.
  */
 #ifndef FASTMAMBA_H
 #define FASTMAMBA_H
@@ -94,7 +95,9 @@ fm_status fm_set_fault_injection(int stall_mask, uint64_t wait_limit_ns);
  * wait the GEMMs fetch their first weight stages and the single decode step
  * its state (the kernels that write a state end before any successor starts).
  * The sequential scan and the gate after it are always launched plainly (the
- * scan's CTA placement matters).  0 launches every kernel plainly.  Results
+ * scan's CTA placement matters), and so is the first kernel after one of
+ * fm_stack_prefill's waits on another stream.  0 launches every kernel
+ * plainly.  Results
  * are the same bits either way.  FM_ERR_INVALID_ARG for other values. */
 fm_status fm_set_pdl(int enable);
 /* Library ABI version (major * 100 + minor). */
@@ -407,6 +410,46 @@ size_t fm_workspace_bytes(const fm_shape *shape, int B, int T);
 fm_status fm_mixer_prefill(const fm_layer *L, const float *x, int B, int T, int residual,
                            int8_t *conv_state, int32_t *ssm_state, float *out, void *ws,
                            size_t ws_bytes, fm_stream stream);
+
+/* Source: as fm_mixer_prefill, for the pre-normed residual stack the
+ * review's workloads run (pith.science review of FastMamba, the 130M and
+ * 2.7B models of Table III); the recurrence's state carries only forward in
+ * time (Mamba2's recurrent form, the paper's reference [2]), which is what
+ * makes the time-pipelined schedule below exact.
+ * A stack of residual layers over one batch, in place on x [B, T, d_model]:
+ * for l = 0 .. n_layers-1, x <- x + mixer_l(x), bit for bit the loop of
+ * fm_mixer_prefill(layers[l], residual = 1, out = x) over the layers (with
+ * the sequential scan a prefill split with carried states gives the one-pass
+ * bits; in the chunked scan mode, whose state crosses a call boundary as
+ * int32, the pipelined result is that loop applied run after run with
+ * carried states).  All layers share d_model and d_inner (FM_ERR_SHAPE
+ * otherwise).
+ *   conv_states / ssm_states: NULL (every layer starts from zero states,
+ *   none written back) or arrays of n_layers per-layer state buffers as
+ *   fm_mixer_prefill takes them (read, then updated).
+ *   n_chunks 1: the plain layer loop on `stream`.  n_chunks in [2, 64]: each
+ *   sequence's tokens are cut into runs of ceil(T / n_chunks) tokens
+ *   (rounded up to a multiple of 32), and every run walks the layers on one
+ *   of up to 8 streams the library keeps per CUDA context, forked from and
+ *   joined back to `stream` (work queued on `stream` before the call runs
+ *   first; work queued after it waits for all of it).  Run k of a layer
+ *   waits only for run k-1's conv and scan of that layer (the states it
+ *   starts from), so successive runs' scans overlap each other and the other
+ *   stages; runs of different sequences do not wait for each other.  The
+ *   first pipelined call in a context creates the streams and events (make
+ *   it outside stream capture); concurrent calls from several host threads
+ *   are serialised on the host while they queue their work.
+ *   ws: device workspace of fm_stack_workspace_bytes(shape, n_layers, B, T,
+ *   n_chunks) bytes, 16-byte aligned (FM_ERR_WORKSPACE / FM_ERR_ALIGNMENT).
+ *   Launch limits as fm_mixer_prefill; n_chunks outside [1, 64] or
+ *   n_layers < 0: FM_ERR_INVALID_ARG. */
+fm_status fm_stack_prefill(const fm_layer *const *layers, int n_layers, float *x, int B, int T,
+                           int8_t *const *conv_states, int32_t *const *ssm_states, int n_chunks,
+                           void *ws, size_t ws_bytes, fm_stream stream);
+/* Workspace bytes of fm_stack_prefill (0 for an invalid shape or argument):
+ * n_chunks 1 needs fm_workspace_bytes(shape, B, T); pipelined, one run's
+ * workspace per internal stream plus zero-started states for every layer. */
+size_t fm_stack_workspace_bytes(const fm_shape *shape, int n_layers, int B, int T, int n_chunks);
 
 /* Source: the 2.7B decode figures of the review's Table III discussion
  * (pith.science review of FastMamba, "What carries the argument"); Mamba2's recurrent form

@@ -12,9 +12,11 @@
 #include <cstdlib>
 #include <cstring>
 #include <atomic>
+#include <memory>
 #include <mutex>
 #include <string>
 #include <type_traits>
+#include <vector>
 
 #include "../../include/fastmamba.h"
 
@@ -72,6 +74,13 @@ extern "C" fm_status fm_set_pdl(int enable) {
   return FM_OK;
 }
 
+// Set when this thread has just made a stream wait for an event of another
+// stream (a pipelined stack's hand-over): the next launch then carries no
+// programmatic-serialisation attribute, so that under stream capture no
+// programmatic edge can reach the other stream's kernel and every kernel
+// that reads a handed-over state waits for its writer's completion.
+static thread_local bool t_after_cross_wait = false;
+
 template <typename... KArgs, typename... Args>
 static fm_status launch_ex(const char *name, void (*kern)(KArgs...), dim3 grid, dim3 block,
                            size_t smem, cudaStream_t s, Args... args) {
@@ -91,7 +100,9 @@ static fm_status launch_ex(const char *name, void (*kern)(KArgs...), dim3 grid, 
   // issue-bound scan's SMs while they wait
   const bool placed = std::strcmp(name, "k_scan_seq") == 0 ||
                       std::strcmp(name, "k_gate_norm_quant") == 0;
-  cfg.numAttrs = g_pdl.load(std::memory_order_relaxed) && !placed ? 1 : 0;
+  const bool after_wait = t_after_cross_wait;
+  t_after_cross_wait = false;
+  cfg.numAttrs = g_pdl.load(std::memory_order_relaxed) && !placed && !after_wait ? 1 : 0;
   const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, args...);
   if (e != cudaSuccess) return fail(FM_ERR_CUDA, "launch of %s: %s", name, cudaGetErrorString(e));
   return FM_OK;
@@ -1322,9 +1333,29 @@ static fm_status check_batch(int B, int T, const char *fn) {
   return FM_OK;
 }
 
+// Hand-over points of one run of a pipelined stack prefill (fm_stack_prefill):
+// before its conv the stream waits for the previous run's conv of the layer
+// (which wrote the conv state this run reads), after it records its own; the
+// same around the scan for the SSM state.  A null event is skipped.
+struct StageSync {
+  cudaEvent_t conv_wait, conv_done, scan_wait, scan_done;
+};
+
+static fm_status sync_wait(const StageSync *sy, cudaEvent_t StageSync::*ev, cudaStream_t s) {
+  if (sy && sy->*ev) {
+    FM_CHECK_CUDA(cudaStreamWaitEvent(s, sy->*ev, 0));
+    t_after_cross_wait = true;
+  }
+  return FM_OK;
+}
+static fm_status sync_record(const StageSync *sy, cudaEvent_t StageSync::*ev, cudaStream_t s) {
+  if (sy && sy->*ev) FM_CHECK_CUDA(cudaEventRecord(sy->*ev, s));
+  return FM_OK;
+}
+
 static fm_status mixer_impl(const fm_layer *L, const Dims &d, const float *x, int B, int T,
                             int residual, int8_t *conv_state, int32_t *ssm_state, float *out,
-                            const MixerWs &w, cudaStream_t s) {
+                            const MixerWs &w, cudaStream_t s, const StageSync *sync = nullptr) {
   const long long M = (long long)B * T;
   const fm_exp_layout X = fm_exp_table_layout(&L->shape);
   const float *amax_in = L->static_amax, *amax_out = L->static_amax ? L->static_amax + 1 : nullptr;
@@ -1332,11 +1363,14 @@ static fm_status mixer_impl(const fm_layer *L, const Dims &d, const float *x, in
                                w.sx_in, nullptr, s));
   FM_TRY(in_proj_impl(w.q_in, w.sx_in, M, L->w_in_q, L->w_in_s, d, L->exps + X.e_u, w.z, w.xbc,
                       w.dt, s, w.split));
+  FM_TRY(sync_wait(sync, &StageSync::conv_wait, s));
   FM_TRY(launch_conv(w.xbc, B, T, d.cc, L->conv_wq, L->conv_bq, L->exps, conv_state, w.xo,
                      nullptr, s, w.e_tok, &d));
+  FM_TRY(sync_record(sync, &StageSync::conv_done, s));
   if (w.ssd.dH && (state16() || w.e_tok))
     return fail(FM_ERR_UNSUPPORTED, "the chunked scan mode carries the int32 state at static "
                 "exponents: the 16-bit state spec and per-token exponents are not supported");
+  FM_TRY(sync_wait(sync, &StageSync::scan_wait, s));
   if (w.ssd.dH)
     FM_TRY(launch_ssd(d, w.xo, w.dt, B, T, L->dt_bias, L->A_q, L->D_q, L->exps, X, ssm_state, w.y,
                       w.ssd, s));
@@ -1344,6 +1378,7 @@ static fm_status mixer_impl(const fm_layer *L, const Dims &d, const float *x, in
     FM_TRY(launch_scan_v2(scan_args(d, w.xo, w.dt, T, L->dt_bias, L->A_q, L->D_q, L->exps, X,
                                     ssm_state, w.y, nullptr, w.e_tok),
                           B, w.scan, s));
+  FM_TRY(sync_record(sync, &StageSync::scan_done, s));
   FM_TRY(gate_impl(w.y, w.z, M, d, L->exps, X, L->norm_w, L->rotate, L->mode, amax_out, w.q_out,
                    w.sx_out, nullptr, nullptr, nullptr, s));
   return launch_gemm(w.q_out, M, L->w_out_q, d.dm, d.di,
@@ -1473,6 +1508,215 @@ extern "C" fm_status fm_decode_step_noalloc(const fm_layer *L, const float *x, i
   void *ws = nullptr;
   FM_TRY(noalloc_scratch_ptr(&ws));
   return fm_decode_step(L, x, B, residual, conv_state, ssm_state, out, ws, need, stream);
+}
+
+// ------------------------------------------------------------------ stack prefill
+// A residual stack over one batch, x <- x + mixer_l(RMSNorm_l(x)) layer by
+// layer, optionally pipelined over time.  The recurrence and the conv carry
+// state only forward in time, and every other stage is per token, so a
+// sequence cut into runs of consecutive tokens gives the same bits when run k
+// of a layer starts from the conv and SSM states run k - 1 of that layer left.
+// Pipelined, each run walks the layers on one of the library's own streams and
+// waits only at those two hand-overs (StageSync), so the scans of successive
+// runs overlap each other and the GEMM and row stages of the neighbouring
+// runs: at B = 1 the sequential scan alone cannot fill every SM sub-partition
+// evenly.
+namespace {
+constexpr int kStackStreams = 8;     // internal streams per context
+constexpr int kStackMaxChunks = 64;  // runs per sequence
+
+struct StackPlan {
+  int runs;     // runs per sequence
+  int tc;       // tokens per run (the last run of a sequence may be shorter)
+  int chains;   // B * runs, issued in this order: run k of sequence b is b * runs + k
+  int streams;  // internal streams in use
+};
+
+// runs of ceil(T / n_chunks) tokens rounded up to the scan's 32-token tile
+StackPlan stack_plan(int B, int T, int n_chunks) {
+  StackPlan p;
+  long long tc = ((long long)T + n_chunks - 1) / n_chunks;
+  tc = (tc + kPrepTT - 1) / kPrepTT * kPrepTT;
+  if (tc > T) tc = T;
+  p.tc = (int)tc;
+  p.runs = (int)(((long long)T + tc - 1) / tc);
+  p.chains = B * p.runs;
+  p.streams = p.chains < kStackStreams ? p.chains : kStackStreams;
+  return p;
+}
+
+size_t ssm_state_bytes_per_seq(const Dims &d) {
+  return (size_t)d.nh * d.hd * d.ds * (state16() ? sizeof(int16_t) : sizeof(int32_t));
+}
+
+// Pipelined workspace: one mixer workspace (for one run) per internal stream,
+// then zero-started conv and SSM states for every layer and sequence, used
+// when the caller passes none.
+struct StackWs {
+  uint8_t *run_ws[kStackStreams];
+  size_t run_bytes;
+  int8_t *conv;
+  uint8_t *ssm;
+  size_t conv_bytes, ssm_bytes;
+};
+
+StackWs carve_stack(Carver &c, const fm_shape *shape, const Dims &d, int n_layers, int B,
+                    const StackPlan &p) {
+  StackWs w;
+  w.run_bytes = fm_workspace_bytes(shape, 1, p.tc);
+  for (int i = 0; i < kStackStreams; ++i)
+    w.run_ws[i] = i < p.streams ? c.take<uint8_t>(w.run_bytes) : nullptr;
+  w.conv_bytes = (size_t)n_layers * B * 3 * d.cc;
+  w.ssm_bytes = (size_t)n_layers * B * ssm_state_bytes_per_seq(d);
+  w.conv = c.take<int8_t>(w.conv_bytes);
+  w.ssm = c.take<uint8_t>(w.ssm_bytes);
+  return w;
+}
+
+// The internal streams and events of one CUDA context, created on first use
+// and kept for the process (keyed by the context's unique id, so a context
+// created anew gets new ones).  The mutex makes each call's host-side issue
+// atomic: the events are reused from call to call.
+struct StackPool {
+  unsigned long long ctx = 0;
+  int dev = -1;
+  cudaStream_t s[kStackStreams];
+  cudaEvent_t fork, joined[kStackStreams], conv_ev[2], scan_ev[2];
+  std::mutex mu;
+};
+
+fm_status stack_pool(StackPool **out) {
+  static std::mutex mu;
+  static std::vector<std::unique_ptr<StackPool>> pools;
+  int dev = 0;
+  FM_CHECK_CUDA(cudaGetDevice(&dev));
+  unsigned long long id = 0;
+  const bool have_id = current_context_id(&id) && id != 0;
+  std::lock_guard<std::mutex> lock(mu);
+  for (auto &p : pools)
+    if (have_id ? p->ctx == id : p->dev == dev) {
+      *out = p.get();
+      return FM_OK;
+    }
+  std::unique_ptr<StackPool> p(new StackPool);
+  p->ctx = have_id ? id : 0;
+  p->dev = dev;
+  for (int i = 0; i < kStackStreams; ++i) {
+    FM_CHECK_CUDA(cudaStreamCreateWithFlags(&p->s[i], cudaStreamNonBlocking));
+    FM_CHECK_CUDA(cudaEventCreateWithFlags(&p->joined[i], cudaEventDisableTiming));
+  }
+  FM_CHECK_CUDA(cudaEventCreateWithFlags(&p->fork, cudaEventDisableTiming));
+  for (int i = 0; i < 2; ++i) {
+    FM_CHECK_CUDA(cudaEventCreateWithFlags(&p->conv_ev[i], cudaEventDisableTiming));
+    FM_CHECK_CUDA(cudaEventCreateWithFlags(&p->scan_ev[i], cudaEventDisableTiming));
+  }
+  *out = p.get();
+  pools.push_back(std::move(p));
+  return FM_OK;
+}
+}  // namespace
+
+extern "C" size_t fm_stack_workspace_bytes(const fm_shape *shape, int n_layers, int B, int T,
+                                           int n_chunks) {
+  Dims d;
+  if (check_shape(shape, &d, __func__) != FM_OK || n_layers < 0 || B < 0 || T < 0 ||
+      n_chunks < 1 || n_chunks > kStackMaxChunks)
+    return 0;
+  if (n_chunks == 1 || (long long)B * T == 0) return fm_workspace_bytes(shape, B, T);
+  Carver c{nullptr, 0};
+  carve_stack(c, shape, d, n_layers, B, stack_plan(B, T, n_chunks));
+  return c.off + 256;
+}
+
+// The pipelined issue: layer by layer, and within a layer run by run, so that
+// each hand-over event is waited on before the next run of the same kind
+// records it again (two events of each kind alternate between neighbouring
+// runs).  Runs of different sequences share nothing and do not wait.
+static fm_status stack_issue(const fm_layer *const *layers, int n_layers, const Dims &d, float *x,
+                             int B, int T, int8_t *const *conv_states,
+                             int32_t *const *ssm_states, const StackPlan &p, const StackWs &w,
+                             StackPool &pool) {
+  const size_t conv_seq = (size_t)3 * d.cc, ssm_seq = ssm_state_bytes_per_seq(d);
+  for (int l = 0; l < n_layers; ++l)
+    for (int c = 0; c < p.chains; ++c) {
+      const int b = c / p.runs, k = c % p.runs;
+      const int t0 = k * p.tc, tn = (T - t0) < p.tc ? (T - t0) : p.tc;
+      cudaStream_t rs = pool.s[c % p.streams];
+      float *xr = x + ((long long)b * T + t0) * d.dm;
+      int8_t *cs = (conv_states ? conv_states[l] : w.conv + (size_t)l * B * conv_seq) + b * conv_seq;
+      uint8_t *sb = ssm_states ? reinterpret_cast<uint8_t *>(ssm_states[l])
+                               : w.ssm + (size_t)l * B * ssm_seq;
+      int32_t *ss = reinterpret_cast<int32_t *>(sb + (size_t)b * ssm_seq);
+      StageSync sy;
+      sy.conv_wait = k > 0 ? pool.conv_ev[(c - 1) & 1] : nullptr;
+      sy.scan_wait = k > 0 ? pool.scan_ev[(c - 1) & 1] : nullptr;
+      sy.conv_done = k + 1 < p.runs ? pool.conv_ev[c & 1] : nullptr;
+      sy.scan_done = k + 1 < p.runs ? pool.scan_ev[c & 1] : nullptr;
+      Carver rc{w.run_ws[c % p.streams], 0};
+      const MixerWs mw = carve_mixer(rc, d, 1, tn);
+      FM_TRY(mixer_impl(layers[l], d, xr, 1, tn, 1, cs, ss, xr, mw, rs, &sy));
+    }
+  return FM_OK;
+}
+
+extern "C" fm_status fm_stack_prefill(const fm_layer *const *layers, int n_layers, float *x,
+                                      int B, int T, int8_t *const *conv_states,
+                                      int32_t *const *ssm_states, int n_chunks, void *ws,
+                                      size_t ws_bytes, fm_stream stream) {
+  if (n_layers < 0) return fail(FM_ERR_INVALID_ARG, "fm_stack_prefill: n_layers < 0");
+  if (n_chunks < 1 || n_chunks > kStackMaxChunks)
+    return fail(FM_ERR_INVALID_ARG, "fm_stack_prefill: n_chunks=%d is not in [1, %d]", n_chunks,
+                kStackMaxChunks);
+  if (B < 0 || T < 0) return fail(FM_ERR_SHAPE, "fm_stack_prefill: B, T must be >= 0");
+  if (n_layers == 0 || (long long)B * T == 0) return FM_OK;
+  if (!layers) return fail(FM_ERR_INVALID_ARG, "fm_stack_prefill: layers is null");
+  Dims d;
+  FM_TRY(check_layer(layers[0], &d, __func__));
+  for (int l = 0; l < n_layers; ++l) {
+    Dims dl;
+    FM_TRY(check_layer(layers[l], &dl, __func__));
+    const fm_shape &a = layers[0]->shape, &s = layers[l]->shape;
+    if (a.d_model != s.d_model || a.d_inner != s.d_inner)
+      return fail(FM_ERR_SHAPE, "fm_stack_prefill: layer %d's shape differs from layer 0's", l);
+    if (conv_states && (!conv_states[l] || !aligned16(conv_states[l])))
+      return fail(FM_ERR_INVALID_ARG, "fm_stack_prefill: conv_states[%d] is null or misaligned",
+                  l);
+    if (ssm_states && (!ssm_states[l] || !aligned16(ssm_states[l])))
+      return fail(FM_ERR_INVALID_ARG, "fm_stack_prefill: ssm_states[%d] is null or misaligned", l);
+  }
+  NEED(x);
+  FM_TRY(check_batch(B, T, __func__));
+  const size_t need = fm_stack_workspace_bytes(&layers[0]->shape, n_layers, B, T, n_chunks);
+  if (!ws || ws_bytes < need)
+    return fail(FM_ERR_WORKSPACE, "fm_stack_prefill: workspace needs %zu bytes", need);
+  if (!aligned16(ws)) return fail(FM_ERR_ALIGNMENT, "fm_stack_prefill: ws misaligned");
+  cudaStream_t s = (cudaStream_t)stream;
+  Carver c{reinterpret_cast<uint8_t *>(ws), 0};
+  if (n_chunks == 1) {  // the plain layer loop on the caller's stream
+    const MixerWs w = carve_mixer(c, d, B, T);
+    for (int l = 0; l < n_layers; ++l)
+      FM_TRY(mixer_impl(layers[l], d, x, B, T, 1, conv_states ? conv_states[l] : nullptr,
+                        ssm_states ? ssm_states[l] : nullptr, x, w, s));
+    return FM_OK;
+  }
+  const StackPlan p = stack_plan(B, T, n_chunks);
+  const StackWs w = carve_stack(c, &layers[0]->shape, d, n_layers, B, p);
+  if (!conv_states) FM_CHECK_CUDA(cudaMemsetAsync(w.conv, 0, w.conv_bytes, s));
+  if (!ssm_states) FM_CHECK_CUDA(cudaMemsetAsync(w.ssm, 0, w.ssm_bytes, s));
+  StackPool *pool = nullptr;
+  FM_TRY(stack_pool(&pool));
+  std::lock_guard<std::mutex> lock(pool->mu);
+  FM_CHECK_CUDA(cudaEventRecord(pool->fork, s));
+  for (int i = 0; i < p.streams; ++i) FM_CHECK_CUDA(cudaStreamWaitEvent(pool->s[i], pool->fork, 0));
+  const fm_status st = stack_issue(layers, n_layers, d, x, B, T, conv_states, ssm_states, p, w,
+                                   *pool);
+  // joined back even after a failed launch, so that the caller's stream never
+  // runs ahead of work already queued on the internal streams
+  for (int i = 0; i < p.streams; ++i) {
+    FM_CHECK_CUDA(cudaEventRecord(pool->joined[i], pool->s[i]));
+    FM_CHECK_CUDA(cudaStreamWaitEvent(s, pool->joined[i], 0));
+  }
+  return st;
 }
 
 // ------------------------------------------------------------------ FastMamba-LQ

@@ -33,6 +33,7 @@ EXPORTS = (
     "fm_lq_mixer_prefill", "fm_set_fault_injection", "fm_set_gemm_splitk",
     "fm_set_gemm_tile", "fm_set_xbc_exponents", "fm_conv1d_pot_tok", "fm_ssm_scan_pot_tok",
     "fm_scan_workspace_bytes_tok", "fm_set_pdl", "fm_set_lq_scan_cpw", "fm_set_gemm_cluster",
+    "fm_stack_prefill", "fm_stack_workspace_bytes",
 )
 NOALLOC_SCRATCH_BYTES = 16 << 20  # FM_NOALLOC_SCRATCH_BYTES
 
@@ -107,6 +108,8 @@ def load():
         "fm_eval_pwl": (I, [I, _P, I64, _P, _P]),
         "fm_workspace_bytes": (SZ, [sp, I, I]),
         "fm_mixer_prefill": (I, [lp, _P, I, I, I, _P, _P, _P, _P, SZ, _P]),
+        "fm_stack_prefill": (I, [_P, I, _P, I, I, _P, _P, I, _P, SZ, _P]),
+        "fm_stack_workspace_bytes": (SZ, [sp, I, I, I, I]),
         "fm_decode_step": (I, [lp, _P, I, I, _P, _P, _P, _P, SZ, _P]),
         "fm_decode_step_noalloc": (I, [lp, _P, I, I, _P, _P, _P, _P]),
         "fm_prepare_mixer_params": (I, [sp, _P, _P, _P, _P, _P, _P, _P, _P]),
@@ -361,6 +364,26 @@ def mixer_prefill(layer: fm_layer, x, B, T, residual, conv_state, ssm_state, out
     _check(load().fm_mixer_prefill(C.byref(layer), _p(x), B, T, residual, _p(conv_state),
                                    _p(ssm_state), _p(out), _p(ws), ws.numel() * ws.element_size(),
                                    _s(stream)))
+
+
+def stack_workspace_bytes(shape, n_layers, B, T, n_chunks) -> int:
+    return load().fm_stack_workspace_bytes(C.byref(shape_struct(shape)), n_layers, B, T, n_chunks)
+
+
+def stack_prefill(layers, x, B, T, states, n_chunks, ws, stream=None):
+    """layers: fm_layer structs; states: None or a list of (conv, ssm) tensors
+    per layer.  The pointer arrays live for the call only (the library reads
+    them while it queues the work)."""
+    n = len(layers)
+    larr = (C.POINTER(fm_layer) * n)(*[C.pointer(L) for L in layers])
+    carr = sarr = None
+    if states is not None:
+        carr = (C.c_void_p * n)(*[_p(cs) for cs, _ in states])
+        sarr = (C.c_void_p * n)(*[_p(ss) for _, ss in states])
+    _check(load().fm_stack_prefill(C.cast(larr, C.c_void_p), n, _p(x), B, T,
+                                   None if carr is None else C.cast(carr, C.c_void_p),
+                                   None if sarr is None else C.cast(sarr, C.c_void_p), n_chunks,
+                                   _p(ws), ws.numel() * ws.element_size(), _s(stream)))
 
 
 def decode_step(layer: fm_layer, x, B, residual, conv_state, ssm_state, out, ws, stream=None):

@@ -160,3 +160,17 @@ class DeviceStack:
             cs, ss = states[i] if states is not None else (None, None)
             L.prefill(r, residual=True, conv_state=cs, ssm_state=ss, out=r, ws=ws, stream=stream)
         return r
+
+    def stack_workspace(self, B: int, T: int, n_chunks: int) -> torch.Tensor:
+        n = lib.stack_workspace_bytes(self.shape, len(self.layers), B, T, n_chunks)
+        return torch.empty(n, dtype=torch.uint8, device=self.layers[0].device)
+
+    def prefill_pipelined_(self, r: torch.Tensor, n_chunks: int = 2, ws=None, states=None,
+                           stream=None) -> torch.Tensor:
+        """As prefill_, in one fm_stack_prefill call: with n_chunks > 1 each
+        sequence is cut into runs that pipeline through the layers on the
+        library's own streams (bit-identical to prefill_)."""
+        B, T, _ = r.shape
+        ws = self.stack_workspace(B, T, n_chunks) if ws is None else ws
+        lib.stack_prefill([L.struct for L in self.layers], r, B, T, states, n_chunks, ws, stream)
+        return r

@@ -146,6 +146,59 @@ def test_layer_validation_before_launch(so):
                                      C.c_void_p(0x5000), x, None) in (2, 4)
 
 
+def test_stack_prefill_validation_and_workspace(so):
+    from quantized_state_space_mamba2_b200 import lib
+    from quantized_state_space_mamba2_b200 import synth as S
+    d = S.MAMBA2_130M
+    sh = lib.shape_struct(d)
+    # one chunk: the layer workspace of the whole batch
+    assert lib.stack_workspace_bytes(d, 24, 2, 512, 1) == lib.workspace_bytes(d, 2, 512)
+    # pipelined: one run's workspace per internal stream (runs of ceil(T / n)
+    # tokens rounded up to 32, at most 8 streams), then zero-started conv and
+    # SSM states for every layer and sequence, each piece 256-byte aligned
+    al = lambda n: (n + 255) // 256 * 256
+    for (nl, B, T, n) in ((24, 1, 2048, 2), (3, 2, 1000, 3), (2, 5, 64, 4)):
+        tc = min(T, ((T + n - 1) // n + 31) // 32 * 32)
+        runs = (T + tc - 1) // tc
+        streams = min(B * runs, 8)
+        off = 0
+        for _ in range(streams):
+            off = al(off) + lib.workspace_bytes(d, 1, tc)
+        off = al(off) + nl * B * 3 * d.conv_ch
+        off = al(off) + nl * B * d.nheads * d.headdim * d.d_state * 4
+        assert lib.stack_workspace_bytes(d, nl, B, T, n) == off + 256, (nl, B, T, n)
+    for bad in ((24, 1, 64, 0), (24, 1, 64, 65), (-1, 1, 64, 2), (24, -1, 64, 2)):
+        assert lib.stack_workspace_bytes(d, *bad) == 0, bad
+    # the entry point rejects before any launch
+    big = 1 << 40
+    x, ws = C.c_void_p(0x7000000), C.c_void_p(0x9000000)
+    L = _fake_layer(lib, S)
+    arr = lambda *ls: C.cast((C.POINTER(lib.fm_layer) * len(ls))(*[C.pointer(l) for l in ls]),
+                             C.c_void_p)
+    two = arr(L, L)
+    assert so.fm_stack_prefill(two, 2, x, 1, 64, None, None, 0, ws, big, None) == 1
+    assert so.fm_stack_prefill(two, 2, x, 1, 64, None, None, 65, ws, big, None) == 1
+    assert so.fm_stack_prefill(two, -1, x, 1, 64, None, None, 2, ws, big, None) == 1
+    assert so.fm_stack_prefill(None, 2, x, 1, 64, None, None, 2, ws, big, None) == 1
+    assert so.fm_stack_prefill(two, 2, x, -1, 64, None, None, 2, ws, big, None) == 2
+    # nothing to do: no layers, or no tokens
+    assert so.fm_stack_prefill(None, 0, x, 1, 64, None, None, 2, ws, big, None) == 0
+    assert so.fm_stack_prefill(two, 2, x, 0, 64, None, None, 2, ws, big, None) == 0
+    # workspace too small or misaligned
+    assert so.fm_stack_prefill(two, 2, x, 1, 64, None, None, 2, ws, 16, None) == 4
+    assert so.fm_stack_prefill(two, 2, x, 1, 64, None, None, 2, C.c_void_p(0x9000008), big,
+                               None) == 3
+    # layers of different widths
+    L27 = _fake_layer(lib, S)
+    L27.shape = lib.shape_struct(S.MAMBA2_2P7B)
+    assert so.fm_stack_prefill(arr(L, L27), 2, x, 1, 64, None, None, 2, ws, big, None) == 2
+    # a null entry in a state array
+    states = (C.c_void_p * 2)(0x3000, None)
+    assert so.fm_stack_prefill(two, 2, x, 1, 64, C.cast(states, C.c_void_p), None, 2, ws, big,
+                               None) == 1
+    assert b"conv_states[1]" in so.fm_last_error()
+
+
 def test_scan_and_tuning_validation(so):
     from quantized_state_space_mamba2_b200 import lib
     from quantized_state_space_mamba2_b200 import synth as S

@@ -104,7 +104,9 @@ def test_reference_arm_line():
 def test_sub_record_modes():
     """The headline runs alone except on the default workload, where the
     static, chunked-scan, 16-bit-state and LQ modes follow as sub-records;
-    each sub-record differs from the headline in exactly one setting."""
+    each sub-record differs from the headline in exactly its mode's settings
+    and, where that mode runs the layer loop instead of the pipelined stack
+    (the chunked scan, LQ), in the pipeline."""
     a = bench.parse([])
     assert bench.sub_modes(a) == ["static", "ssd", "state16", "candidate", "lq"]
     assert bench.sub_modes(bench.parse(["--modes", "none"])) == []
@@ -114,9 +116,9 @@ def test_sub_record_modes():
     with pytest.raises(SystemExit):
         bench.sub_modes(bench.parse(["--modes", "fast"]))
     base = bench.config_block(a)
-    for m, keys in (("static", {"act_quant"}), ("ssd", {"scan_mode"}),
+    for m, keys in (("static", {"act_quant"}), ("ssd", {"scan_mode", "pipeline"}),
                     ("state16", {"state_spec"}), ("candidate", {"state_spec", "xbc_exponents"}),
-                    ("lq", {"variant"})):
+                    ("lq", {"variant", "pipeline"})):
         v = bench.variant_args(a, m)
         diff = {k for k, x in bench.config_block(v).items() if base.get(k) != x}
         assert diff == keys, (m, diff)
