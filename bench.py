@@ -128,7 +128,7 @@ def parse(argv=None):
                          "lq; 'auto' = all four for the default workload, none otherwise; 'none'")
     ap.add_argument("--chunks", type=int, default=0,
                     help="runs per sequence of a stack prefill pipelined through the layers by "
-                         "fm_stack_prefill (0: 2 for a single-sequence stack prefill with the "
+                         "fm_stack_prefill (0: 4 for a single-sequence stack prefill with the "
                          "sequential scan, else 1; 1: the layer loop)")
     ap.add_argument("--layers", type=int, default=None,
                     help="profiling only: run the first N layers of a stack workload")
@@ -174,9 +174,11 @@ def n_layers(args) -> int:
 
 def stack_chunks(args) -> int:
     """Runs per sequence of the pipelined stack prefill (1: the layer loop).
-    By default 2 for a single sequence, whose scan alone leaves SM
-    sub-partitions idle (measured: 130M stack +11 %; at B = 2 the 2.7B scan
-    fills the GPU and pipelining gained nothing).  The FastMamba-LQ variant,
+    By default 4 for a single sequence, whose scan alone leaves SM
+    sub-partitions idle (measured, 130M stack: 302.4 k tokens/s as the layer
+    loop, 335.7 k with 2 runs, 340.3 k with 4 runs and the 16-step scan chunks
+    the library then picks; at B = 2 the 2.7B scan fills the GPU and
+    pipelining gained nothing).  The FastMamba-LQ variant,
     single-token steps and the chunked scan mode (whose state crosses a call
     boundary as int32, so a split prefill is not the one-pass result) run the
     layer loop."""
@@ -186,7 +188,7 @@ def stack_chunks(args) -> int:
         return 1
     if getattr(args, "chunks", 0) > 0:
         return args.chunks
-    return 2 if w.get("batch", 1) == 1 else 1
+    return 4 if w.get("batch", 1) == 1 else 1
 
 
 def stack_runs(T: int, n: int) -> tuple:
@@ -237,7 +239,9 @@ def config_block(args) -> dict:
             runs, tc = stack_runs(w["seqlen"], ch)
             c.update(pipeline=f"fm_stack_prefill, n_chunks {ch}: {runs} runs of up to {tc} "
                               "tokens per sequence, each on its own stream, waiting only for "
-                              "the previous run's conv and scan of the same layer")
+                              "the previous run's conv and scan of the same layer"
+                              + ("; the runs' scans stage 16-step chunks where the grid is too "
+                                 "small for 8 channels per CTA" if not args.scan_tile else ""))
         if getattr(args, "lq", False):
             c.update(variant="FastMamba-LQ (W8A8 linears; fp32 conv, scan, gate)")
         if "prefill_len" in w:

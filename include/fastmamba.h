@@ -254,7 +254,8 @@ fm_status fm_conv1d_pot_tok(const int8_t *u, int B, int T, const fm_shape *shape
  * call in this process -- npt state columns per thread, pc channels per CTA,
  * tch time steps per staged chunk.  Compiled variants: (4,0,32) (default:
  * pc chosen by the grid -- 8 where there are at least three 8-channel CTAs
- * per SM, else 4), (4,4,32), (4,8,32), (4,4,16), (4,2,16), (4,8,16),
+ * per SM, else 4, with 16-step chunks for the runs of a pipelined
+ * fm_stack_prefill), (4,4,32), (4,8,32), (4,4,16), (4,2,16), (4,8,16),
  * (8,4,16), (8,2,16), (8,8,16);
  * anything else returns FM_ERR_INVALID_ARG.  All variants compute the same
  * bits. */
@@ -441,6 +442,10 @@ fm_status fm_mixer_prefill(const fm_layer *L, const float *x, int B, int T, int 
  *   are serialised on the host while they queue their work.
  *   ws: device workspace of fm_stack_workspace_bytes(shape, n_layers, B, T,
  *   n_chunks) bytes, 16-byte aligned (FM_ERR_WORKSPACE / FM_ERR_ALIGNMENT).
+ *   With the scan tile left to the grid (fm_set_scan_tile's default), runs
+ *   whose scan grid is too small for 8 channels per CTA stage 16-step chunks
+ *   (half the shared memory), so that more of the neighbouring runs' kernels
+ *   fit beside them; the bits are the same either way.
  *   Launch limits as fm_mixer_prefill; n_chunks outside [1, 64] or
  *   n_layers < 0: FM_ERR_INVALID_ARG. */
 fm_status fm_stack_prefill(const fm_layer *const *layers, int n_layers, float *x, int B, int T,

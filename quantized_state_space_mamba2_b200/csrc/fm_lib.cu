@@ -656,6 +656,13 @@ extern "C" fm_status fm_set_scan_mode(int mode) {
 }
 static bool use_ssd(int T) { return T > 1 && g_scan_mode.load(std::memory_order_relaxed) == 1; }
 static ScanTile scan_tile() { return kScanTiles[g_scan_tile.load(std::memory_order_relaxed)]; }
+// Set while this thread queues the runs of a pipelined stack prefill
+// (fm_stack_prefill): on a grid too small for 8 channels per CTA the default
+// tile then stages 16-step chunks, half the shared memory of 32, so that more
+// CTAs of the neighbouring runs' kernels fit beside the scan.  Measured, 130M
+// stack at B = 1: 4 runs with 16-step chunks 340.3 k tokens/s, with 32-step
+// chunks 332.2 k (2 runs: 323.9 k and 335.7 k).
+static thread_local bool t_pipelined_run = false;
 
 extern "C" fm_status fm_set_scan_tile(int npt, int pc, int tch) {
   for (int i = 0; i < (int)(sizeof(kScanTiles) / sizeof(kScanTiles[0])); ++i)
@@ -752,7 +759,10 @@ static fm_status launch_scan_v2(const ScanArgs &a, int B, const ScanWs &w, cudaS
   q.y = a.y;
   q.osh = p.osh;
   ScanTile t = scan_tile();
-  if (t.pc == 0) t.pc = (long long)B * a.nh * a.hd / 8 >= 3LL * sm_count() ? 8 : 4;
+  if (t.pc == 0) {
+    t.pc = (long long)B * a.nh * a.hd / 8 >= 3LL * sm_count() ? 8 : 4;
+    if (t_pipelined_run && t.pc == 4) t.tch = 16;
+  }
 #define FM_SEQ(N, P, C)                                                          \
   if (t.npt == N && t.pc == P && t.tch == C) {                                   \
     if (q.osh)                                                                   \
@@ -1636,6 +1646,10 @@ static fm_status stack_issue(const fm_layer *const *layers, int n_layers, const 
                              int B, int T, int8_t *const *conv_states,
                              int32_t *const *ssm_states, const StackPlan &p, const StackWs &w,
                              StackPool &pool) {
+  struct RunFlag {  // the scan tile rule of pipelined runs, for this call only
+    RunFlag() { t_pipelined_run = true; }
+    ~RunFlag() { t_pipelined_run = false; }
+  } run_flag;
   const size_t conv_seq = (size_t)3 * d.cc, ssm_seq = ssm_state_bytes_per_seq(d);
   for (int l = 0; l < n_layers; ++l)
     for (int c = 0; c < p.chains; ++c) {
