@@ -501,6 +501,7 @@ class StackWorkload:
     bit for bit against it), with events around each layer's scan."""
 
     launches_per_layer = 7  # FWHT+quant, in_proj, conv, scan prep, scan, gate, out_proj
+    chunks = 1  # runs per sequence of the pipelined stack prefill (1: the layer loop)
 
     def __init__(self, args, torch, lib, dev, rank):
         from quantized_state_space_mamba2_b200.model import DeviceLayer, DeviceStack

@@ -123,3 +123,22 @@ def test_sub_record_modes():
         diff = {k for k, x in bench.config_block(v).items() if base.get(k) != x}
         assert diff == keys, (m, diff)
     assert not a.lq and a.mode == "dynamic"          # the headline's args are untouched
+
+
+def test_pipeline_defaults():
+    """Single-sequence stack prefills with the sequential scan are pipelined in
+    4 runs by default; every other workload runs the layer loop, and every
+    stack workload class (including those that build themselves without the
+    base constructor, like the decode step) reads 1 run by default."""
+    for cls in (bench.StackWorkload, bench.DecodeWorkload, bench.LqStackWorkload):
+        assert cls.chunks == 1, cls
+    assert bench.stack_chunks(bench.parse([])) == 4
+    assert bench.stack_chunks(bench.parse(["--chunks", "2"])) == 2
+    for argv in (["--workload", "stack2p7b_64l_b2_t4096"], ["--workload", "decode2p7b_64l_b64"],
+                 ["--workload", "mixer130m_b1_t256"], ["--scan-mode", "ssd"], ["--lq"],
+                 ["--workload", "decode2p7b_64l_b64", "--chunks", "4"]):
+        assert bench.stack_chunks(bench.parse(argv)) == 1, argv
+    assert bench.stack_runs(2048, 4) == (4, 512)
+    assert bench.stack_runs(200, 3) == (3, 96)
+    assert bench.stack_runs(40, 64) == (2, 32)
+    assert bench.stack_runs(1, 2) == (1, 1)
