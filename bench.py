@@ -549,8 +549,13 @@ class StackWorkload:
             self.pws = self.stack.stack_workspace(self.B, self.T, self.chunks)
             self.staged_launches = self.launches
             _, extra_run = _gemm_workspace(torch, lib, d, tc, dev)
-            self.launches = ((self.launches_per_layer + extra_run + (1 if self.ssd else 0)) *
-                             self.n_layers * self.B * runs)
+            # every run carries conv state, so a run of more than one token
+            # adds the conv-state update; a one-token run's scan is the single
+            # step (no prep) and its conv writes the state itself
+            last = self.T - (runs - 1) * tc
+            per_run = lambda tn: (self.launches_per_layer + extra_run +
+                                  ((1 if self.ssd else 0) + 1 if tn > 1 else -1))
+            self.launches = (per_run(tc) * (runs - 1) + per_run(last)) * self.n_layers * self.B
 
     def states(self, i):
         return None, None
