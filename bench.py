@@ -620,11 +620,13 @@ class StackWorkload:
         self.h2d_bytes = self.d2h_bytes = self.x_host.nbytes
 
     def e2e_step(self):
-        self.xd.copy_(self.xh, non_blocking=True)
         if self.stack_mode and self.chunks > 1:
-            self.stack.prefill_pipelined_(self.xd, n_chunks=self.chunks, ws=self.pws)
-            self.oh.copy_(self.xd, non_blocking=True)
-        elif self.stack_mode:
+            # one call with the batch in host memory: each run's input and
+            # output copies travel on the run's stream, overlapping the others
+            self.stack.prefill_host(self.xh, self.oh, self.xd, n_chunks=self.chunks, ws=self.pws)
+            return
+        self.xd.copy_(self.xh, non_blocking=True)
+        if self.stack_mode:
             self.stack.prefill_(self.xd, ws=self.ws)
             self.oh.copy_(self.xd, non_blocking=True)
         else:

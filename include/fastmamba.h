@@ -451,6 +451,21 @@ fm_status fm_mixer_prefill(const fm_layer *L, const float *x, int B, int T, int 
 fm_status fm_stack_prefill(const fm_layer *const *layers, int n_layers, float *x, int B, int T,
                            int8_t *const *conv_states, int32_t *const *ssm_states, int n_chunks,
                            void *ws, size_t ws_bytes, fm_stream stream);
+/* fm_stack_prefill with the batch in host memory: x_host [B, T, d_model] is
+ * copied to the device rows x_dev (caller-owned, [B, T, d_model], 16-byte
+ * aligned), the stack runs there, and the result is copied to out_host (may
+ * equal x_host).  Pipelined, each run's input is copied on the run's stream
+ * before its first layer and its output right after its last, so the copies
+ * of one run overlap the other runs' kernels; with n_chunks 1 the two copies
+ * bracket the layer loop on `stream`.  The call only queues the copies
+ * (cudaMemcpyAsync): they overlap only if the host buffers are pinned, and
+ * out_host holds the result once `stream` has been synchronised.  x_host and
+ * out_host are required when B * T > 0 (FM_ERR_INVALID_ARG); n_layers 0 does
+ * nothing.  Everything else as fm_stack_prefill, with the same workspace. */
+fm_status fm_stack_prefill_host(const fm_layer *const *layers, int n_layers, const float *x_host,
+                                float *out_host, float *x_dev, int B, int T,
+                                int8_t *const *conv_states, int32_t *const *ssm_states,
+                                int n_chunks, void *ws, size_t ws_bytes, fm_stream stream);
 /* Workspace bytes of fm_stack_prefill (0 for an invalid shape or argument):
  * n_chunks 1 needs fm_workspace_bytes(shape, B, T); pipelined, one run's
  * workspace per internal stream plus zero-started states for every layer. */

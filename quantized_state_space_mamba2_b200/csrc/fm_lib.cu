@@ -1643,9 +1643,9 @@ extern "C" size_t fm_stack_workspace_bytes(const fm_shape *shape, int n_layers, 
 // records it again (two events of each kind alternate between neighbouring
 // runs).  Runs of different sequences share nothing and do not wait.
 static fm_status stack_issue(const fm_layer *const *layers, int n_layers, const Dims &d, float *x,
-                             int B, int T, int8_t *const *conv_states,
-                             int32_t *const *ssm_states, const StackPlan &p, const StackWs &w,
-                             StackPool &pool) {
+                             const float *x_host, float *out_host, int B, int T,
+                             int8_t *const *conv_states, int32_t *const *ssm_states,
+                             const StackPlan &p, const StackWs &w, StackPool &pool) {
   struct RunFlag {  // the scan tile rule of pipelined runs, for this call only
     RunFlag() { t_pipelined_run = true; }
     ~RunFlag() { t_pipelined_run = false; }
@@ -1668,49 +1668,63 @@ static fm_status stack_issue(const fm_layer *const *layers, int n_layers, const 
       sy.scan_done = k + 1 < p.runs ? pool.scan_ev[c & 1] : nullptr;
       Carver rc{w.run_ws[c % p.streams], 0};
       const MixerWs mw = carve_mixer(rc, d, 1, tn);
+      const size_t run_bytes = (size_t)tn * d.dm * sizeof(float);
+      const long long row0 = (long long)b * T + t0;
+      if (l == 0 && x_host)  // this run's input, on its own stream
+        FM_CHECK_CUDA(cudaMemcpyAsync(xr, x_host + row0 * d.dm, run_bytes, cudaMemcpyHostToDevice,
+                                      rs));
       FM_TRY(mixer_impl(layers[l], d, xr, 1, tn, 1, cs, ss, xr, mw, rs, &sy));
+      if (l == n_layers - 1 && out_host)  // and its output, as soon as it is final
+        FM_CHECK_CUDA(cudaMemcpyAsync(out_host + row0 * d.dm, xr, run_bytes,
+                                      cudaMemcpyDeviceToHost, rs));
     }
   return FM_OK;
 }
 
-extern "C" fm_status fm_stack_prefill(const fm_layer *const *layers, int n_layers, float *x,
-                                      int B, int T, int8_t *const *conv_states,
-                                      int32_t *const *ssm_states, int n_chunks, void *ws,
-                                      size_t ws_bytes, fm_stream stream) {
-  if (n_layers < 0) return fail(FM_ERR_INVALID_ARG, "fm_stack_prefill: n_layers < 0");
+// The stack on device rows x; with x_host / out_host (host) the input is
+// copied in and the output out inside the same schedule (per run when
+// pipelined, so the copies of one run overlap the other runs' kernels).
+static fm_status stack_prefill(const char *fn, const fm_layer *const *layers, int n_layers,
+                               float *x, const float *x_host, float *out_host, int B, int T,
+                               int8_t *const *conv_states, int32_t *const *ssm_states,
+                               int n_chunks, void *ws, size_t ws_bytes, cudaStream_t s) {
+  if (n_layers < 0) return fail(FM_ERR_INVALID_ARG, "%s: n_layers < 0", fn);
   if (n_chunks < 1 || n_chunks > kStackMaxChunks)
-    return fail(FM_ERR_INVALID_ARG, "fm_stack_prefill: n_chunks=%d is not in [1, %d]", n_chunks,
+    return fail(FM_ERR_INVALID_ARG, "%s: n_chunks=%d is not in [1, %d]", fn, n_chunks,
                 kStackMaxChunks);
-  if (B < 0 || T < 0) return fail(FM_ERR_SHAPE, "fm_stack_prefill: B, T must be >= 0");
-  if (n_layers == 0 || (long long)B * T == 0) return FM_OK;
-  if (!layers) return fail(FM_ERR_INVALID_ARG, "fm_stack_prefill: layers is null");
+  if (B < 0 || T < 0) return fail(FM_ERR_SHAPE, "%s: B, T must be >= 0", fn);
+  if ((long long)B * T == 0) return FM_OK;
+  if (!x) return fail(FM_ERR_INVALID_ARG, "%s: the device rows x are null", fn);
+  if (!aligned16(x)) return fail(FM_ERR_ALIGNMENT, "%s: x is not 16-byte aligned", fn);
+  if (n_layers == 0) return FM_OK;  // no layer: nothing to do (no width to copy either)
+  if (!layers) return fail(FM_ERR_INVALID_ARG, "%s: layers is null", fn);
   Dims d;
-  FM_TRY(check_layer(layers[0], &d, __func__));
+  FM_TRY(check_layer(layers[0], &d, fn));
   for (int l = 0; l < n_layers; ++l) {
     Dims dl;
-    FM_TRY(check_layer(layers[l], &dl, __func__));
-    const fm_shape &a = layers[0]->shape, &s = layers[l]->shape;
-    if (a.d_model != s.d_model || a.d_inner != s.d_inner)
-      return fail(FM_ERR_SHAPE, "fm_stack_prefill: layer %d's shape differs from layer 0's", l);
+    FM_TRY(check_layer(layers[l], &dl, fn));
+    const fm_shape &a = layers[0]->shape, &sh = layers[l]->shape;
+    if (a.d_model != sh.d_model || a.d_inner != sh.d_inner)
+      return fail(FM_ERR_SHAPE, "%s: layer %d's shape differs from layer 0's", fn, l);
     if (conv_states && (!conv_states[l] || !aligned16(conv_states[l])))
-      return fail(FM_ERR_INVALID_ARG, "fm_stack_prefill: conv_states[%d] is null or misaligned",
-                  l);
+      return fail(FM_ERR_INVALID_ARG, "%s: conv_states[%d] is null or misaligned", fn, l);
     if (ssm_states && (!ssm_states[l] || !aligned16(ssm_states[l])))
-      return fail(FM_ERR_INVALID_ARG, "fm_stack_prefill: ssm_states[%d] is null or misaligned", l);
+      return fail(FM_ERR_INVALID_ARG, "%s: ssm_states[%d] is null or misaligned", fn, l);
   }
-  NEED(x);
-  FM_TRY(check_batch(B, T, __func__));
+  FM_TRY(check_batch(B, T, fn));
   const size_t need = fm_stack_workspace_bytes(&layers[0]->shape, n_layers, B, T, n_chunks);
   if (!ws || ws_bytes < need)
-    return fail(FM_ERR_WORKSPACE, "fm_stack_prefill: workspace needs %zu bytes", need);
-  if (!aligned16(ws)) return fail(FM_ERR_ALIGNMENT, "fm_stack_prefill: ws misaligned");
-  cudaStream_t s = (cudaStream_t)stream;
+    return fail(FM_ERR_WORKSPACE, "%s: workspace needs %zu bytes", fn, need);
+  if (!aligned16(ws)) return fail(FM_ERR_ALIGNMENT, "%s: ws misaligned", fn);
+  const size_t all_bytes = (size_t)B * T * d.dm * sizeof(float);
   Carver c{reinterpret_cast<uint8_t *>(ws), 0};
   if (n_chunks == 1) {  // the plain layer loop on the caller's stream
+    if (x_host) FM_CHECK_CUDA(cudaMemcpyAsync(x, x_host, all_bytes, cudaMemcpyHostToDevice, s));
     const MixerWs w = carve_mixer(c, d, B, T);
     for (int l = 0; l < n_layers; ++l)
       FM_TRY(mixer_impl(layers[l], d, x, B, T, 1, conv_states ? conv_states[l] : nullptr,
                         ssm_states ? ssm_states[l] : nullptr, x, w, s));
+    if (out_host) FM_CHECK_CUDA(cudaMemcpyAsync(out_host, x, all_bytes, cudaMemcpyDeviceToHost, s));
     return FM_OK;
   }
   const StackPlan p = stack_plan(B, T, n_chunks);
@@ -1722,8 +1736,8 @@ extern "C" fm_status fm_stack_prefill(const fm_layer *const *layers, int n_layer
   std::lock_guard<std::mutex> lock(pool->mu);
   FM_CHECK_CUDA(cudaEventRecord(pool->fork, s));
   for (int i = 0; i < p.streams; ++i) FM_CHECK_CUDA(cudaStreamWaitEvent(pool->s[i], pool->fork, 0));
-  const fm_status st = stack_issue(layers, n_layers, d, x, B, T, conv_states, ssm_states, p, w,
-                                   *pool);
+  const fm_status st = stack_issue(layers, n_layers, d, x, x_host, out_host, B, T, conv_states,
+                                   ssm_states, p, w, *pool);
   // joined back even after a failed launch, so that the caller's stream never
   // runs ahead of work already queued on the internal streams
   for (int i = 0; i < p.streams; ++i) {
@@ -1731,6 +1745,25 @@ extern "C" fm_status fm_stack_prefill(const fm_layer *const *layers, int n_layer
     FM_CHECK_CUDA(cudaStreamWaitEvent(s, pool->joined[i], 0));
   }
   return st;
+}
+
+extern "C" fm_status fm_stack_prefill(const fm_layer *const *layers, int n_layers, float *x,
+                                      int B, int T, int8_t *const *conv_states,
+                                      int32_t *const *ssm_states, int n_chunks, void *ws,
+                                      size_t ws_bytes, fm_stream stream) {
+  return stack_prefill(__func__, layers, n_layers, x, nullptr, nullptr, B, T, conv_states,
+                       ssm_states, n_chunks, ws, ws_bytes, (cudaStream_t)stream);
+}
+
+extern "C" fm_status fm_stack_prefill_host(const fm_layer *const *layers, int n_layers,
+                                           const float *x_host, float *out_host, float *x_dev,
+                                           int B, int T, int8_t *const *conv_states,
+                                           int32_t *const *ssm_states, int n_chunks, void *ws,
+                                           size_t ws_bytes, fm_stream stream) {
+  if ((long long)B * T > 0 && (!x_host || !out_host))
+    return fail(FM_ERR_INVALID_ARG, "fm_stack_prefill_host: x_host and out_host are required");
+  return stack_prefill(__func__, layers, n_layers, x_dev, x_host, out_host, B, T, conv_states,
+                       ssm_states, n_chunks, ws, ws_bytes, (cudaStream_t)stream);
 }
 
 // ------------------------------------------------------------------ FastMamba-LQ

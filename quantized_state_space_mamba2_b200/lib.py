@@ -33,7 +33,7 @@ EXPORTS = (
     "fm_lq_mixer_prefill", "fm_set_fault_injection", "fm_set_gemm_splitk",
     "fm_set_gemm_tile", "fm_set_xbc_exponents", "fm_conv1d_pot_tok", "fm_ssm_scan_pot_tok",
     "fm_scan_workspace_bytes_tok", "fm_set_pdl", "fm_set_lq_scan_cpw", "fm_set_gemm_cluster",
-    "fm_stack_prefill", "fm_stack_workspace_bytes",
+    "fm_stack_prefill", "fm_stack_workspace_bytes", "fm_stack_prefill_host",
 )
 NOALLOC_SCRATCH_BYTES = 16 << 20  # FM_NOALLOC_SCRATCH_BYTES
 
@@ -109,6 +109,7 @@ def load():
         "fm_workspace_bytes": (SZ, [sp, I, I]),
         "fm_mixer_prefill": (I, [lp, _P, I, I, I, _P, _P, _P, _P, SZ, _P]),
         "fm_stack_prefill": (I, [_P, I, _P, I, I, _P, _P, I, _P, SZ, _P]),
+        "fm_stack_prefill_host": (I, [_P, I, _P, _P, _P, I, I, _P, _P, I, _P, SZ, _P]),
         "fm_stack_workspace_bytes": (SZ, [sp, I, I, I, I]),
         "fm_decode_step": (I, [lp, _P, I, I, _P, _P, _P, _P, SZ, _P]),
         "fm_decode_step_noalloc": (I, [lp, _P, I, I, _P, _P, _P, _P]),
@@ -384,6 +385,29 @@ def stack_prefill(layers, x, B, T, states, n_chunks, ws, stream=None):
                                    None if carr is None else C.cast(carr, C.c_void_p),
                                    None if sarr is None else C.cast(sarr, C.c_void_p), n_chunks,
                                    _p(ws), ws.numel() * ws.element_size(), _s(stream)))
+
+
+def _host_ptr(t):
+    if t.is_cuda or not t.is_contiguous():
+        raise ValueError("a contiguous host tensor is required")
+    return C.c_void_p(t.data_ptr())
+
+
+def stack_prefill_host(layers, x_host, out_host, x_dev, B, T, states, n_chunks, ws, stream=None):
+    """fm_stack_prefill_host: x_host / out_host contiguous CPU tensors (pinned for
+    the copies to overlap the compute), x_dev the device rows it works in."""
+    n = len(layers)
+    larr = (C.POINTER(fm_layer) * n)(*[C.pointer(L) for L in layers])
+    carr = sarr = None
+    if states is not None:
+        carr = (C.c_void_p * n)(*[_p(cs) for cs, _ in states])
+        sarr = (C.c_void_p * n)(*[_p(ss) for _, ss in states])
+    _check(load().fm_stack_prefill_host(C.cast(larr, C.c_void_p), n, _host_ptr(x_host),
+                                        _host_ptr(out_host), _p(x_dev), B, T,
+                                        None if carr is None else C.cast(carr, C.c_void_p),
+                                        None if sarr is None else C.cast(sarr, C.c_void_p),
+                                        n_chunks, _p(ws), ws.numel() * ws.element_size(),
+                                        _s(stream)))
 
 
 def decode_step(layer: fm_layer, x, B, residual, conv_state, ssm_state, out, ws, stream=None):

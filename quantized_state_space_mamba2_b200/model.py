@@ -174,3 +174,14 @@ class DeviceStack:
         ws = self.stack_workspace(B, T, n_chunks) if ws is None else ws
         lib.stack_prefill([L.struct for L in self.layers], r, B, T, states, n_chunks, ws, stream)
         return r
+
+    def prefill_host(self, x_host: torch.Tensor, out_host: torch.Tensor, x_dev: torch.Tensor,
+                     n_chunks: int = 2, ws=None, states=None, stream=None) -> torch.Tensor:
+        """The stack on a batch in host memory (fm_stack_prefill_host): x_host in,
+        out_host out (pinned host tensors), x_dev the device rows it runs in.
+        Asynchronous on the stream: out_host is final after synchronising it."""
+        B, T, _ = x_host.shape
+        ws = self.stack_workspace(B, T, n_chunks) if ws is None else ws
+        lib.stack_prefill_host([L.struct for L in self.layers], x_host, out_host, x_dev, B, T,
+                               states, n_chunks, ws, stream)
+        return out_host

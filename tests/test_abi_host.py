@@ -197,6 +197,15 @@ def test_stack_prefill_validation_and_workspace(so):
     assert so.fm_stack_prefill(two, 2, x, 1, 64, C.cast(states, C.c_void_p), None, 2, ws, big,
                                None) == 1
     assert b"conv_states[1]" in so.fm_last_error()
+    # the host-buffer variant: both host buffers are required, the device rows aligned
+    h = C.c_void_p(0x5000000)
+    assert so.fm_stack_prefill_host(two, 2, None, h, x, 1, 64, None, None, 2, ws, big, None) == 1
+    assert so.fm_stack_prefill_host(two, 2, h, None, x, 1, 64, None, None, 2, ws, big, None) == 1
+    assert so.fm_stack_prefill_host(two, 2, h, h, C.c_void_p(0x7000004), 1, 64, None, None, 2, ws,
+                                    big, None) == 3
+    assert so.fm_stack_prefill_host(two, 2, None, None, x, 0, 64, None, None, 2, ws, big,
+                                    None) == 0
+    assert so.fm_stack_prefill_host(two, 2, h, h, x, 1, 64, None, None, 2, ws, 16, None) == 4
 
 
 def test_scan_and_tuning_validation(so):

@@ -1,7 +1,8 @@
 """GPU: the pipelined stack prefill (fm_stack_prefill) against the CPU oracle's
 stack and against the layer loop of fm_mixer_prefill, bit for bit: several
 chunk counts, ragged runs, more than one sequence, states in and out, the
-chunked scan mode, and a CUDA-graph capture of the call."""
+chunked scan mode, a CUDA-graph capture of the call, and the host-buffer
+variant (fm_stack_prefill_host)."""
 import numpy as np
 import pytest
 
@@ -145,3 +146,28 @@ def test_pipelined_stack_in_a_cuda_graph(env, stack3):
     env.sync_status()
     assert torch.equal(buf, ref)
     del g
+
+
+@pytest.mark.parametrize("B,T,n,pinned,alias", [(1, 512, 4, True, False), (2, 200, 3, True, True),
+                                                (1, 300, 1, False, False), (3, 64, 2, False, True)])
+def test_stack_prefill_host(env, stack3, B, T, n, pinned, alias):
+    """Host input and output through fm_stack_prefill_host (copies per run on
+    the runs' streams) equal the device-resident layer loop, states included."""
+    st, _ = stack3
+    x = acts(B, T, 41 + T)
+    ref = dev(x)
+    s0 = warm_states(st, B, 9)
+    s_ref = clone_states(s0)
+    st.prefill_(ref, states=s_ref)
+    xh = torch.from_numpy(x.copy())
+    if pinned:
+        xh = xh.pin_memory()
+    oh = xh if alias else (torch.empty_like(xh).pin_memory() if pinned else torch.empty_like(xh))
+    xd = torch.empty(ref.shape, dtype=torch.float32, device="cuda")
+    s_got = clone_states(s0)
+    st.prefill_host(xh, oh, xd, n_chunks=n, states=s_got)
+    torch.cuda.synchronize()
+    env.sync_status()
+    assert torch.equal(oh, ref.cpu())
+    for (c1, h1), (c2, h2) in zip(s_got, s_ref):
+        assert torch.equal(c1, c2) and torch.equal(h1, h2)
