@@ -216,6 +216,10 @@ struct ScanSeqSmem {
   // (with one channel per warp the per-step sums come from redux.sync and
   // only 16 int2 per warp are staged)
   static constexpr int PSTRIDE = LPP == 32 ? 1 : LPP + 1;
+  // rows of partial sums per warp: with one channel per warp the per-step
+  // sums of up to 32 steps (16-step chunks keep two chunks' worth, for the
+  // output epilogue that runs once per pair of chunks)
+  static constexpr int PROWS = LPP == 32 ? 32 : TCH * (32 / LPP);
   struct Slot {
     int32_t bc[TCH][256];
     int32_t dA[TCH];
@@ -225,7 +229,7 @@ struct ScanSeqSmem {
     long long bound[TCH / 16][PC];  // growth bounds of the chunk's 16-step parts
   };
   Slot slot[kScanSlots];
-  int2 part[NW][TCH * (32 / LPP)][PSTRIDE];
+  int2 part[NW][PROWS][PSTRIDE];
   uint64_t full[kScanSlots];
   uint64_t empty[kScanSlots];
 };
@@ -444,6 +448,16 @@ __global__ void __launch_bounds__(PC *(128 / NPT) + 32) k_scan_seq(ScanSeqArgs a
     hl[j] = S16 ? 0u : (unsigned)v & 0xFFFFu;
   }
   int2(*part)[PSTRIDE] = sm.part[warp];
+  // 16-step chunks with one channel per warp: the output epilogue (lane tt
+  // forms step tt's y) runs once per pair of chunks, so that all 32 lanes
+  // share it as with 32-step chunks, while each slot still holds 16 steps and
+  // is released right after them (each lane keeps its step's x code, and its
+  // output shifts, from the slot first).  Measured on the 130M stack with
+  // 16-step chunks as a layer loop: 289.2 k -> 291.4 k tokens/s (32-step
+  // chunks: 302.4 k); the pipelined stack, whose runs use 16-step chunks, was
+  // unchanged within noise.
+  constexpr bool PAIR = REDUX && TCH == 16;
+  int x_keep = 0, osh_keep = 0;
   for (int c = 0; c < nchunks; ++c) {
     const int sl = c % kScanSlots;
     if (!mbar_wait(&sm.full[sl], (uint32_t)(c / kScanSlots) & 1u)) return;  // error word set
@@ -464,7 +478,8 @@ __global__ void __launch_bounds__(PC *(128 / NPT) + 32) k_scan_seq(ScanSeqArgs a
     const bool no_clamp = __all_sync(0xffffffffu, hbound + grow <=
                                                       (S16 ? (long long)kH16Lim : kHLim));
     int2 pr[TCH];
-    int2 *wsum = reinterpret_cast<int2 *>(&part[0][0]);
+    const int half = PAIR ? (c & 1) * 16 : 0;  // PAIR: this chunk's place in its pair
+    int2 *wsum = reinterpret_cast<int2 *>(&part[0][0]) + half;
     if (nt == TCH) {
       if (no_clamp)
         scan_chunk_steps<NPT, TCH, true, false, REDUX, S16>(hh, hl, pr, wsum, s.bc, s.dA, s.u[pp], n0, nt);
@@ -473,7 +488,28 @@ __global__ void __launch_bounds__(PC *(128 / NPT) + 32) k_scan_seq(ScanSeqArgs a
     } else {
       scan_chunk_steps<NPT, TCH, false, true, REDUX, S16>(hh, hl, pr, wsum, s.bc, s.dA, s.u[pp], n0, nt);
     }
-    if constexpr (REDUX) {  // one channel per warp: lane tt finishes step tt
+    if constexpr (PAIR) {
+      if (lane32 >= half && lane32 < half + nt) {
+        x_keep = s.xs[pp][lane32 - half];
+        if constexpr (TOK) osh_keep = s.osh[lane32 - half];
+      }
+      __syncwarp();
+      if (lane32 == 0) mbar_arrive(&sm.empty[sl]);  // the slot is free again
+      if (half || c == nchunks - 1) {  // the pair is complete: lane tt finishes its step tt
+        const int np = half + nt;
+        const long long tp = t0 - half;
+        if (lane32 < np) {
+          const int2 v = reinterpret_cast<const int2 *>(&part[0][0])[lane32];
+          const long long sum = S16 ? (long long)v.x : (long long)v.x * 65536 + v.y;
+          const int sy = TOK ? osh_sy(osh_keep) : s_y;
+          const int sD = TOK ? osh_sD(osh_keep) : s_D;
+          a.y[(rowbase + tp + lane32) * di + (long long)h * hd + p0 + pp] =
+              (int)satb64(rshr64(sum, sy) + rshr64(Dq * (long long)x_keep, sD), 32);
+        }
+        __syncwarp();  // the pair's sums are read before the next pair writes them
+      }
+      continue;
+    } else if constexpr (REDUX) {  // one channel per warp: lane tt finishes step tt
       __syncwarp();
       if (lane32 < nt) {
         const int2 v = wsum[lane32];
