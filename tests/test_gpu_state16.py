@@ -65,7 +65,7 @@ def _exps(L, s, e_x, e_B, e_C, e_h, e_y, e_D):
     return e
 
 
-@pytest.mark.parametrize("B,T", [(1, 1), (64, 1), (2, 33), (1, 513)])
+@pytest.mark.parametrize("B,T", [(1, 1), (3, 1), (64, 1), (2, 33), (1, 513)])
 def test_scan_state16_matches_oracle(L, spec16, B, T):
     s = MAMBA130
     xbc, dt_raw, dt_bias, A_q, D_q, e_D, e_x, e_B, e_C, e_h, e_y = _case(s, B, T, 300 + T)
