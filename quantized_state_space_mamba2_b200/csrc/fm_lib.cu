@@ -700,7 +700,12 @@ static fm_status launch_scan_v2(const ScanArgs &a, int B, const ScanWs &w, cudaS
   if (M == 0) return FM_OK;
   if (B > 65535 || M > 2147483647LL) return fail(FM_ERR_SHAPE, "scan: B or B*T too large");
   if (a.T == 1) {  // decode: one step per sequence, no staging
-    if (a.hlim <= kH16Lim)
+    // the step kernel takes the spec's clamp and guard bits as constants
+    const bool narrow = a.hlim <= kH16Lim;
+    if (narrow ? (a.hlim != kH16Lim || a.guard != kH16Guard) : (a.hlim != kHLim || a.guard != 0))
+      return fail(FM_ERR_INVALID_ARG, "scan step: state spec (%d, %d) is not a supported one",
+                  a.hlim, a.guard);
+    if (narrow)
       FM_TRY(launch_ex("k_scan_step", k_scan_step<true>, dim3(a.nh, B), 256, 0, s, a));
     else
       FM_TRY(launch_ex("k_scan_step", k_scan_step<false>, dim3(a.nh, B), 256, 0, s, a));

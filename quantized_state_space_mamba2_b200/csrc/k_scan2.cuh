@@ -616,9 +616,10 @@ __global__ void __launch_bounds__(256) k_scan_step(ScanArgs a) {
   const int8_t *row = a.xbc + (long long)b * cc;
   const uint32_t bw = *reinterpret_cast<const uint32_t *>(row + di + n0);
   const uint32_t cw = *reinterpret_cast<const uint32_t *>(row + di + 128 + n0);
-  int8_t xs[kStepPPW];
-#pragma unroll
-  for (int k = 0; k < kStepPPW; ++k) xs[k] = row[h * hd + warp + 8 * k];
+  // lane k < 8 holds channel warp + 8k's x code (a narrow step is bound by
+  // its instruction issue, so per-channel work is done once per lane, not
+  // once per channel in every thread)
+  const int x_mine = lane < kStepPPW ? (int)row[h * hd + warp + 8 * lane] : 0;
   // per-token exponents of this sequence's token (T == 1), else the static ones
   const int32_t *et = a.e_tok ? a.e_tok + (long long)b * (nh + 2) : nullptr;
   const int e_x = et ? et[h] : a.e_x[h], e_B = et ? et[nh] : *a.e_B, e_C = et ? et[nh + 1] : *a.e_C;
@@ -635,13 +636,16 @@ __global__ void __launch_bounds__(256) k_scan_step(ScanArgs a) {
     Bv[j] = (int)(int8_t)((bw >> (8 * j)) & 0xFF);
     Cv[j] = (int)(int8_t)((cw >> (8 * j)) & 0xFF);
   }
-  // the state spec: a word of at most 16 bits needs no (hi, lo) split
-  const int g = a.guard;
+  // the state spec: a word of at most 16 bits needs no (hi, lo) split; its
+  // guard bits and clamp are fixed by the spec (the host checks the args)
+  constexpr int G = NARROW ? kH16Guard : 0;
+  constexpr int HLIM = NARROW ? kH16Lim : (int)kHLim;
+  // lane k's channel's increment factor u, one 64-bit evaluation per lane
+  const int u_mine = (int)satb64(rshr64((long long)dtq * x_mine, s_h - G), 24);
   int shi = 0, slo = 0;  // lane k (< 8) ends up holding channel warp + 8k's C.h sums
 #pragma unroll
   for (int k = 0; k < kStepPPW; ++k) {
-    const long long xq = xs[k];
-    const int u = (int)satb64(rshr64((long long)dtq * xq, s_h - g), 24);
+    const int u = __shfl_sync(0xffffffffu, u_mine, k);
     const int hs[4] = {hv[k].x, hv[k].y, hv[k].z, hv[k].w};
     int hn[4];
     int ahi = 0, alo = 0;
@@ -649,8 +653,8 @@ __global__ void __launch_bounds__(256) k_scan_step(ScanArgs a) {
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int t = dA * hs[j] + 0x8000;
-        int v = (t >> 16) + rshr_guard(u * Bv[j], g);
-        v = min(max(v, -a.hlim), a.hlim);
+        int v = (t >> 16) + rshr_guard(u * Bv[j], G);
+        v = min(max(v, -HLIM), HLIM);
         hn[j] = v;
         ahi += Cv[j] * v;
       }
@@ -660,8 +664,8 @@ __global__ void __launch_bounds__(256) k_scan_step(ScanArgs a) {
         const int hh = hs[j] >> 16;
         const unsigned hl = (unsigned)hs[j] & 0xFFFFu;
         const unsigned t = (unsigned)dA * hl + 0x8000u;
-        int v = dA * hh + (int)(t >> 16) + rshr_guard(u * Bv[j], g);
-        v = min(max(v, -a.hlim), a.hlim);
+        int v = dA * hh + (int)(t >> 16) + rshr_guard(u * Bv[j], G);
+        v = min(max(v, -HLIM), HLIM);
         hn[j] = v;
         ahi += Cv[j] * (v >> 16);
         alo += Cv[j] * (int)((unsigned)v & 0xFFFFu);
@@ -684,7 +688,7 @@ __global__ void __launch_bounds__(256) k_scan_step(ScanArgs a) {
   }
   if (lane < kStepPPW) {  // one output per lane: channel warp + 8 lane
     const int p = warp + 8 * lane;
-    const long long xq = row[h * hd + p];
+    const long long xq = x_mine;
     const long long sum = narrow ? (long long)shi : (long long)shi * 65536 + slo;
     a.y[(long long)b * di + (long long)h * hd + p] =
         (int)satb64(rshr64(sum, s_y) + rshr64(Dq * xq, s_D), 32);
