@@ -67,12 +67,14 @@ CPU_ALLCORE_TOKENS = 512
 # captures of the current kernels (profiles/dram_traffic_roofline_kernels.md);
 # None where no capture of the kernel in that configuration exists.
 DRAM_TRAFFIC = {
-    # 130M stack, B 1, T 2048, static exponents, the int32 state: k_scan_prep
-    # 3,885,312 + 256 and k_scan_seq<4, 4, 32> 29,106,176 + 0
+    # 130M stack, B 1, T 2048, static exponents, the int32 state, the layer
+    # loop the roofline is timed on: k_scan_prep 3,885,056 + 0 and
+    # k_scan_seq<4, 4, 32> 19,665,920 + 0 (the x codes staged as int8)
     ("fm_ssm_scan_pot (k_scan_prep + k_scan_seq)", "stack130m_24l_b1_t2048", "31,0", "static"):
-        32991744,
-    # 2.7B decode, B 64: k_scan_step 168,197,632 + 108,543,488
-    ("fm_ssm_scan_pot, T = 1 (k_scan_step)", "decode2p7b_64l_b64", "31,0", "static"): 276741120,
+        23550976,
+    # 2.7B decode, B 64: k_scan_step 168,172,672 + 108,671,744 (mean of the
+    # two layers' launches; u evaluated once per lane)
+    ("fm_ssm_scan_pot, T = 1 (k_scan_step)", "decode2p7b_64l_b64", "31,0", "static"): 276844416,
     # in_proj GEMM at M = 32768: 306,106,112 + 1,339,252,992
     ("fm_w8a8_gemm (k_gemm_i8_persist, tcgen05 kind::i8)", "gemm2p7b_inproj", 32768): 1645359104,
 }
