@@ -79,7 +79,8 @@ def test_pipelined_stack_matches_oracle(env, stack3):
 
 
 @pytest.mark.parametrize("B,T,n", [(1, 512, 2), (1, 300, 3), (2, 256, 4), (3, 97, 2),
-                                   (1, 64, 8), (2, 1, 2), (1, 40, 64), (2, 129, 1)])
+                                   (1, 64, 8), (2, 1, 2), (1, 40, 64), (2, 129, 1),
+                                   (3, 256, 4)])  # 12 runs share the 8 streams
 @pytest.mark.parametrize("with_states", [False, True], ids=["zero", "carried"])
 def test_pipelined_stack_equals_layer_loop(env, stack3, B, T, n, with_states):
     """Outputs and (when given) the final conv / SSM states of every layer
