@@ -212,13 +212,13 @@ struct ScanSeqSmem {
   static constexpr int LPP = 128 / NPT;          // threads per p
   static constexpr int NW = PC * LPP / 32;       // compute warps
   // int2 per partial row: LPP + 1 (rows an odd number of 8-byte words apart)
-  // keeps the per-row reads of a half-warp on distinct banks
-  // (with one channel per warp the per-step sums come from redux.sync and
-  // only 16 int2 per warp are staged)
+  // keeps the per-row reads of a half-warp on distinct banks; with one
+  // channel per warp a row is one step's (C hh, C hl) sums, already added
+  // over the warp by redux.sync
   static constexpr int PSTRIDE = LPP == 32 ? 1 : LPP + 1;
-  // rows of partial sums per warp: with one channel per warp the per-step
-  // sums of up to 32 steps (16-step chunks keep two chunks' worth, for the
-  // output epilogue that runs once per pair of chunks)
+  // rows per warp: with one channel per warp the sums of 32 steps (16-step
+  // chunks keep two chunks' worth, for the output epilogue that runs once
+  // per pair of chunks); otherwise a chunk's per-lane partials
   static constexpr int PROWS = LPP == 32 ? 32 : TCH * (32 / LPP);
   struct Slot {
     int32_t bc[TCH][256];
