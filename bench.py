@@ -549,7 +549,6 @@ class StackWorkload:
         if self.chunks > 1:
             runs, tc = stack_runs(self.T, self.chunks)
             self.pws = self.stack.stack_workspace(self.B, self.T, self.chunks)
-            self.staged_launches = self.launches
             _, extra_run = _gemm_workspace(torch, lib, d, tc, dev)
             # every run carries conv state, so a run of more than one token
             # adds the conv-state update; a one-token run's scan is the single
