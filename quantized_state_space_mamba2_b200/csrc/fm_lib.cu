@@ -84,8 +84,7 @@ static thread_local bool t_after_cross_wait = false;
 template <typename... KArgs, typename... Args>
 static fm_status launch_ex(const char *name, void (*kern)(KArgs...), dim3 grid, dim3 block,
                            size_t smem, cudaStream_t s, Args... args) {
-  cudaLaunchConfig_t cfg;
-  std::memset(&cfg, 0, sizeof(cfg));
+  cudaLaunchConfig_t cfg = {};  // no attributes unless set below
   cfg.gridDim = grid;
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
@@ -167,7 +166,7 @@ static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 
   } while (0)
 
 struct Dims {
-  int dm, di, hd, ds, nh, cc, n_in;
+  int dm = 0, di = 0, hd = 0, ds = 0, nh = 0, cc = 0, n_in = 0;  // filled by check_shape
 };
 
 static fm_status check_shape(const fm_shape *s, Dims *d, const char *fn) {
@@ -389,8 +388,7 @@ static fm_status launch_gemm_cl_t(const CUtensorMap &ta, const CUtensorMap &tb, 
   FM_CHECK_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
   const int nkb = (int)(K / kGemmBK);
   const int per = (nkb + S - 1) / S;
-  cudaLaunchConfig_t cfg;
-  std::memset(&cfg, 0, sizeof(cfg));
+  cudaLaunchConfig_t cfg = {};  // no attributes unless set below
   cfg.gridDim = dim3((unsigned)((N + BN - 1) / BN), 1, S);
   cfg.blockDim = dim3(kGemmThreads);
   cfg.dynamicSmemBytes = smem;

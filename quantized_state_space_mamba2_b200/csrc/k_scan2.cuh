@@ -280,18 +280,19 @@ __device__ __forceinline__ int2 scan_one_step(int (&hh)[NPT], unsigned (&hl)[NPT
       ahi += Cv[j] * hn;
     }
     return make_int2(ahi, 0);
-  }
+  } else {
 #pragma unroll
-  for (int j = 0; j < NPT; ++j) {
-    const unsigned t = (unsigned)dA * hl[j] + 0x8000u;
-    int hn = dA * hh[j] + (int)(t >> 16) + u * Bv[j];
-    if (CLAMP) hn = min(max(hn, -(int)kHLim), (int)kHLim);
-    hh[j] = hn >> 16;
-    hl[j] = (unsigned)hn & 0xFFFFu;
-    ahi += Cv[j] * hh[j];
-    alo += Cv[j] * (int)hl[j];
+    for (int j = 0; j < NPT; ++j) {
+      const unsigned t = (unsigned)dA * hl[j] + 0x8000u;
+      int hn = dA * hh[j] + (int)(t >> 16) + u * Bv[j];
+      if (CLAMP) hn = min(max(hn, -(int)kHLim), (int)kHLim);
+      hh[j] = hn >> 16;
+      hl[j] = (unsigned)hn & 0xFFFFu;
+      ahi += Cv[j] * hh[j];
+      alo += Cv[j] * (int)hl[j];
+    }
+    return make_int2(ahi, alo);
   }
-  return make_int2(ahi, alo);
 }
 
 // The (C hh, C hl) partial sums of step tt go to part[tt] (REDUX = false), or
