@@ -308,3 +308,23 @@ def test_lq_entry_points_validate(so):
     P = lib.fm_lq_params()
     assert so.fm_lq_mixer_prefill(C.byref(L), C.byref(P), p, 1, 5, 0, None, None, p, p, 1 << 30,
                                   None) in (1, 2)
+
+
+def test_plain_c_consumer(so, tmp_path):
+    """The header compiles as C99 (-Wall -Wextra -pedantic -Werror) and a C
+    program linked against libfastmamba.so runs its host-only checks."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    pkg = os.path.join(root, "quantized_state_space_mamba2_b200")
+    exe = str(tmp_path / "abi_consumer")
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror",
+                    "-I", os.path.join(root, "include"),
+                    os.path.join(root, "tests", "abi_consumer.c"), "-L", pkg, "-lfastmamba",
+                    f"-Wl,-rpath,{pkg}", "-o", exe], check=True)
+    r = subprocess.run([exe], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    assert "17 checks passed" in r.stdout
